@@ -1,0 +1,473 @@
+#!/usr/bin/env python
+"""Throughput of the chunked gated delta-rule scan forward (tokens/s per layer) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one prism_scan_fwd call over one batch of the GDN workload (B=4, H=8, T=4096,
+dk=dv=128, L=1, chunk 64, bf16 I/O, fp32 state).  Inputs are device resident when timing starts;
+three input batches rotate (419 MB of inputs, more than the 126 MB L2), so every step streams its
+inputs from HBM.  Steps are replayed from CUDA graphs (one per input batch) so that host overhead
+does not leave gaps between kernels.  Timing uses CUDA events on the launching stream with a
+barrier and a synchronize on both sides; the reported time is the max over ranks.
+
+With N > 1 (torchrun, one process per GPU) every rank processes its own batch (weak scaling: the
+B*H sequences are independent, so there is no collective in the data path).
+
+Besides the headline line's required keys the JSON line carries: roofline (HBM-bound; algorithmic
+bytes per launch over the measured copy bandwidth), cpu_baseline (the fp64 oracle on a bounded
+sample, rank 0 at N = 1), e2e (through the public API with pinned-host inputs copied in and the
+outputs copied back inside the timed region), clocks sampled during the timed region, and the
+decode step (B=256, H=32, d=128, L=4) as a secondary measurement.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    csrc = os.path.join(ROOT, "delta_rule_sequence_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload, kernel):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on this source."""
+    src = kernel_source_hash()
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    pat = re.compile(r"bench_traffic:\s*workload=(\S+)\s+kernel=(\S+)\s+source_sha256=(\S+)\s+"
+                     r"dram_bytes_per_launch=(\d+)")
+    for name in sorted(os.listdir(pdir)):
+        if not name.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(pdir, name)) as f:
+            for line in f:
+                m = pat.search(line)
+                if m and m.group(1) == workload and m.group(2) == kernel and m.group(3) == src:
+                    return int(m.group(4))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid):
+        self.gpu = gpu_uuid
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [c.strip() for c in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread:
+                self.thread.join(timeout=2)
+
+    def summary(self, t0, t1):
+        rows = [r for t, r in self.rows if t0 - 0.15 <= t <= t1 + 0.15] or [r for _, r in self.rows]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        smax = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[4:8]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        power = [float(r[2]) for r in rows if re.match(r"^[\d.]+$", r[2])]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic work of one scan-forward call (what must cross HBM / be computed at minimum)
+
+def scan_bytes(wl, io_bytes=2, with_S0=None):
+    B, T, H, dk, dv, L = wl.B, wl.T, wl.H, wl.dk, wl.dv, wl.L
+    tok = B * T * H
+    per_tok = (2 * dk + dv) * io_bytes + 8  # q, k, o + alpha, beta
+    if wl.write == "gdn":
+        per_tok += dv * io_bytes
+    else:
+        per_tok += L * (dk + dv) * io_bytes
+    state = B * H * dv * dk * 4
+    s0 = state if (with_S0 if with_S0 is not None else wl.s0_std > 0) else 0
+    return tok * per_tok + state + s0
+
+
+def scan_flops(wl):
+    """Algorithmic FLOPs of the chunked form (triangular products at half)."""
+    C, d, L = wl.chunk, wl.dk, wl.L
+    if wl.write == "gdn":
+        per = 5 * C * d + C * C / 3 + 6 * d * d
+    else:
+        per = C * d * (5 + 4 * L) + C * C / 3 + d * d * (6 + 2 * L)
+    return wl.B * wl.T * wl.H * per
+
+
+def decode_bytes(wl, io_bytes=2):
+    heads = wl.B * wl.H
+    per = 2 * wl.dv * wl.dk * 4 + (2 * wl.dk + wl.dv) * io_bytes + 8
+    per += wl.L * (wl.dk + wl.dv) * io_bytes
+    return heads * per
+
+
+# ------------------------------------------------------------------------------------------------
+
+def cpu_oracle_sample(wl, budget_s=12.0, n_threads=None):
+    """Time the fp64 oracle on whole (b, h) sequences of the workload.  Returns (tokens/s,
+    description, threads).  One sequence is timed alone first to size a sample of about
+    `budget_s` seconds on all threads."""
+    import oracle
+    from delta_rule_sequence_b200.workloads import make_inputs, select_heads
+
+    threads = n_threads or oracle.default_threads()
+    x = make_inputs(wl, seed=0)
+    heads_all = [(b, h) for b in range(wl.B) for h in range(wl.H)]
+    sub = select_heads(x, heads_all[:1])
+    t0 = time.perf_counter()
+    oracle.scan_ref(**sub, n_threads=1)
+    t1 = time.perf_counter() - t0
+    n = max(1, min(len(heads_all), int(budget_s * threads / max(t1, 1e-3))))
+    n = max(1, (n // threads) * threads) if n >= threads else n
+    sub = select_heads(x, heads_all[:n])
+    t0 = time.perf_counter()
+    oracle.scan_ref(**sub, n_threads=threads)
+    dt = time.perf_counter() - t0
+    tokens = n * wl.T / wl.H  # a token carries all H heads
+    desc = (f"{n} of {wl.B * wl.H} (b,h) sequences of the {wl.name} workload, full T={wl.T}, "
+            f"fp64 token recurrence on {threads} threads, {dt:.1f} s; tokens/s = sequences*T/H/s")
+    return tokens / dt, desc, threads
+
+
+def run_reference(args, rank):
+    """The base contract's reference arm: the fp64 oracle on the host cores, per step a bounded
+    sample of the same workload (a few whole (b,h) sequences, one per thread)."""
+    if rank != 0:
+        return
+    import oracle
+    from delta_rule_sequence_b200.workloads import WORKLOADS, make_inputs, select_heads
+
+    wl = WORKLOADS[args.workload]
+    threads = oracle.default_threads()
+    x = make_inputs(wl, seed=0)
+    heads_all = [(b, h) for b in range(wl.B) for h in range(wl.H)]
+    per_step = min(len(heads_all), threads)
+    subs = [select_heads(x, [heads_all[(s * per_step + i) % len(heads_all)]
+                             for i in range(per_step)]) for s in range(2)]
+    for i in range(args.warmup):
+        oracle.scan_ref(**subs[i % 2], n_threads=threads)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.scan_ref(**subs[i % 2], n_threads=threads)
+    dt = time.perf_counter() - t0
+    tokens = args.steps * per_step * wl.T / wl.H
+    value = tokens / dt
+    desc = (f"per step {per_step} whole (b,h) sequences (T={wl.T}) of the {wl.name} workload, "
+            f"fp64 oracle on {threads} threads")
+    line = {
+        "impl": "reference", "metric": "scan-fwd tokens/s per layer", "value": value,
+        "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl):
+    return {"workload": f"{wl.name}: B={wl.B} H={wl.H} T={wl.T} dk={wl.dk} dv={wl.dv} L={wl.L} "
+                        f"chunk={wl.chunk} io={wl.io} state=f32 write={wl.write}",
+            "global_batch": wl.B, "seq_len": wl.T, "heads": wl.H,
+            "l2": "3 rotating input batches (each > L2 / 3) so inputs stream from HBM"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gdn")
+    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from delta_rule_sequence_b200 import prism
+    from delta_rule_sequence_b200.workloads import (WORKLOADS, make_decode_state,
+                                                     make_decode_step, make_inputs)
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peaks_kind = load_peaks()
+    wl = WORKLOADS[args.workload]
+    stream = torch.cuda.Stream(device=dev)
+
+    # ---- inputs: three seeded batches per rank, device resident
+    host_sets = [make_inputs(wl, seed=3 * rank + i) for i in range(3)]
+    sets = [{n: (None if t is None else t.to(dev)) for n, t in s.items()} for s in host_sets]
+    o_buf = [torch.empty((wl.B, wl.T, wl.H, wl.dv), dtype=wl.torch_io, device=dev) for _ in range(3)]
+    S_buf = [torch.empty((wl.B, wl.H, wl.dv, wl.dk), dtype=torch.float32, device=dev)
+             for _ in range(3)]
+    shape = prism.make_shape(sets[0]["q"], sets[0]["v"], sets[0]["u"], wl.chunk)
+    ws = prism.workspace_for(shape, dev)
+    launches_per_step = prism.prism_scan_fwd_launch_count(shape)
+
+    def step(i, s=None):
+        x = sets[i % 3]
+        prism.prism_scan_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["u"], x["w"],
+                             x["S0"], chunk=wl.chunk, o=o_buf[i % 3], S_final=S_buf[i % 3],
+                             workspace=ws, stream=s)
+
+    # ---- capture one graph per input batch
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i, stream)
+    stream.synchronize()
+    graphs = []
+    for i in range(3):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(i, stream)
+        graphs.append(g)
+    torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % 3].replay()
+    stream.synchronize()
+    status = prism.prism_query_device_status(ws, stream)
+    if status != prism.PRISM_OK:
+        raise SystemExit(f"bench: device status after warm-up: {prism.status_string(status)}")
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    sampler.start()
+    time.sleep(0.3)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for i in range(args.steps):
+            graphs[i % 3].replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier()
+    sampler.stop()
+    ms_total = ev0.elapsed_time(ev1)
+    ms_total = max_over_ranks(ms_total)
+    ms_per_step = ms_total / args.steps
+    tokens_per_step = wl.B * wl.T
+    value = world * tokens_per_step * args.steps / (ms_total / 1e3)
+    status = prism.prism_query_device_status(ws, stream)
+    if status != prism.PRISM_OK:
+        raise SystemExit(f"bench: device status after timing: {prism.status_string(status)}")
+    clocks = sampler.summary(wall0, wall1)
+
+    # roofline of the dominant (only) kernel: algorithmic bytes per launch / launch duration
+    alg_bytes = scan_bytes(wl)
+    kernel_ms = ms_per_step / max(1, launches_per_step)
+    achieved = alg_bytes / (kernel_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"],
+                "traffic": committed_traffic(wl.name, "scan"),
+                "peak_kind": f"{peaks_kind} copy bandwidth",
+                "algorithmic_bytes_per_launch": alg_bytes,
+                "algorithmic_flops_per_launch": scan_flops(wl),
+                "tensor_frac_algorithmic": scan_flops(wl) / (kernel_ms / 1e3) / 1e12
+                / peaks["bf16_tflops"]}
+
+    # ---- end to end through the public API: pinned host inputs in, outputs back, every step
+    e2e = None
+    if args.e2e_steps > 0:
+        pinned = {n: (None if t is None else t.pin_memory()) for n, t in host_sets[0].items()}
+        o_host = torch.empty(o_buf[0].shape, dtype=o_buf[0].dtype).pin_memory()
+        S_host = torch.empty(S_buf[0].shape, dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
+        d2h = o_host.numel() * o_host.element_size() + S_host.numel() * 4
+        x = sets[0]
+        def e2e_step():
+            for n, t in pinned.items():
+                if t is not None:
+                    x[n].copy_(t, non_blocking=True)
+            step(0, stream)
+            o_host.copy_(o_buf[0], non_blocking=True)
+            S_host.copy_(S_buf[0], non_blocking=True)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.e2e_steps):
+                e2e_step()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = max_over_ranks(e0.elapsed_time(e1))
+        e2e = {"value": world * tokens_per_step * args.e2e_steps / (ems / 1e3),
+               "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": args.e2e_steps}
+
+    # ---- secondary: the decode step (B=256, H=32, d=128, L=4), state in HBM, in place
+    decode = None
+    if args.decode_steps > 0:
+        dwl = WORKLOADS["decode"]
+        st = make_decode_state(dwl, seed=rank)
+        S = st["S0"].to(dev)
+        pool = [{n: (None if t is None else t.to(dev)) for n, t in
+                 make_decode_step(dwl, st, s, seed=rank).items()} for s in range(4)]
+        o_d = torch.empty((dwl.B, 1, dwl.H, dwl.dv), dtype=torch.bfloat16, device=dev)
+        def dstep(i):
+            x = pool[i % 4]
+            prism.prism_step_decode(x["q"], x["k"], None, x["alpha"], x["beta"], x["u"], x["w"],
+                                    S, o=o_d, stream=stream)
+        with torch.cuda.stream(stream):
+            for i in range(10):
+                dstep(i)
+        torch.cuda.synchronize()
+        barrier()
+        d0 = torch.cuda.Event(enable_timing=True)
+        d1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            d0.record(stream)
+            for i in range(args.decode_steps):
+                dstep(i)
+            d1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        dms = max_over_ranks(d0.elapsed_time(d1)) / args.decode_steps
+        db = decode_bytes(dwl)
+        decode = {"workload": "decode: B=256 H=32 dk=dv=128 L=4 bf16 I/O, fp32 state in place",
+                  "ms_per_step": dms, "tokens_per_s": world * dwl.B / (dms / 1e3),
+                  "achieved_gbs": db / (dms / 1e3) / 1e9,
+                  "frac_of_measured_copy": db / (dms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                  "frac_of_8tbs": db / (dms / 1e3) / 1e9 / 8000.0,
+                  "bytes_per_step": db, "steps": args.decode_steps,
+                  "inputs": "4 seeded step batches cycled; state carried across steps"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, threads = cpu_oracle_sample(wl)
+        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    for g in graphs:
+        g.reset()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": "scan-fwd tokens/s per layer", "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(wl), parallelism=f"dp{world} over (b,h) sequences"),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps, "clocks": clocks, "decode": decode,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,143 @@
+// api.cu -- the C ABI of libprism.so (declared in include/prism.h): argument validation, plan
+// selection and kernel launches.  No allocation, no synchronisation except in
+// prism_query_device_status, no printing.
+
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace prism {
+cudaError_t launch_scan_simt(const ScanArgs &a, bool io_f32, cudaStream_t s);
+cudaError_t launch_decode(const ScanArgs &a, bool io_f32, cudaStream_t s);
+}  // namespace prism
+
+namespace {
+
+int g_debug_flags = 0;
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+bool width_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+// Shared checks of prism_scan_fwd and prism_step_decode.
+prism_status check_common(const prism_shape *s, const void *q, const void *k, const void *v,
+                          const float *alpha, const float *beta, const void *u, const void *w) {
+    if (!s) return PRISM_ERR_INVALID_ARG;
+    if (s->B < 0 || s->H < 0 || s->T < 0) return PRISM_ERR_INVALID_ARG;
+    if (s->io != PRISM_BF16 && s->io != PRISM_F32) return PRISM_ERR_INVALID_ARG;
+    if (s->L < 1) return PRISM_ERR_INVALID_ARG;  // L = 0 would have no write at all
+    if (s->dk < 1 || s->dv < 1) return PRISM_ERR_INVALID_ARG;
+    if (!width_ok(s->dk) || !width_ok(s->dv) || s->L > 8) return PRISM_ERR_UNSUPPORTED;
+    if (s->B > 65535 || s->H > 65535) return PRISM_ERR_UNSUPPORTED;
+    if ((u == nullptr) != (w == nullptr)) return PRISM_ERR_INVALID_ARG;
+    if (u == nullptr && s->L != 1) return PRISM_ERR_INVALID_ARG;
+    const bool work = (long long)s->B * s->H * s->T > 0;
+    if (work) {
+        if (!q || !k || !alpha || !beta) return PRISM_ERR_INVALID_ARG;
+        if (u == nullptr && v == nullptr) return PRISM_ERR_INVALID_ARG;
+    }
+    const void *ptrs[] = {q, k, v, alpha, beta, u, w};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return PRISM_ERR_INVALID_ARG;
+    return PRISM_OK;
+}
+
+prism::ScanArgs make_args(const prism_shape *s, const void *q, const void *k, const void *v,
+                          const float *alpha, const float *beta, const void *u, const void *w,
+                          const float *S0, void *o, float *S_final, uint32_t *status) {
+    prism::ScanArgs a;
+    a.B = s->B; a.H = s->H; a.T = s->T; a.dk = s->dk; a.dv = s->dv; a.L = s->L;
+    a.chunk = s->chunk;
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.u = u; a.w = w;
+    a.S0 = S0; a.o = o; a.S_final = S_final; a.status = status;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+prism_status prism_scan_fwd_workspace_size(const prism_shape *shape, size_t *bytes) {
+    if (!shape || !bytes) return PRISM_ERR_INVALID_ARG;
+    *bytes = prism::kStatusBytes;
+    return PRISM_OK;
+}
+
+prism_status prism_scan_fwd_launch_count(const prism_shape *shape, int *launches) {
+    if (!shape || !launches) return PRISM_ERR_INVALID_ARG;
+    int n = 1;
+    if (shape->B == 0 || shape->H == 0) n = 0;
+    *launches = n;
+    return PRISM_OK;
+}
+
+prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void *k,
+                            const void *v, const float *alpha, const float *beta,
+                            const void *u, const void *w, const float *S0, void *o,
+                            float *S_final, void *workspace, size_t ws_bytes, void *stream) {
+    prism_status st = check_common(shape, q, k, v, alpha, beta, u, w);
+    if (st != PRISM_OK) return st;
+    if (shape->chunk != 64 && shape->chunk != 128) return PRISM_ERR_INVALID_ARG;
+    size_t need = 0;
+    prism_scan_fwd_workspace_size(shape, &need);
+    if (!workspace || ws_bytes < need || ((uintptr_t)workspace & 255u)) return PRISM_ERR_INVALID_ARG;
+    if ((S0 && !aligned16(S0)) || (S_final && !aligned16(S_final))) return PRISM_ERR_INVALID_ARG;
+    const long long work = (long long)shape->B * shape->H * shape->T;
+    if (work > 0 && (!o || !aligned16(o))) return PRISM_ERR_INVALID_ARG;
+    if (o && (o == q || o == k || o == v || o == u || o == w)) return PRISM_ERR_INVALID_ARG;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t *status = (uint32_t *)workspace;
+    if (shape->B == 0 || shape->H == 0) return PRISM_OK;
+    if (shape->T == 0 && !S_final) return PRISM_OK;
+
+    prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, S0, o, S_final, status);
+    cudaError_t err = prism::launch_scan_simt(a, shape->io == PRISM_F32, s);
+    return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
+prism_status prism_step_decode(const prism_shape *shape, const void *q, const void *k,
+                               const void *v, const float *alpha, const float *beta,
+                               const void *u, const void *w, float *S, void *o, void *stream) {
+    prism_status st = check_common(shape, q, k, v, alpha, beta, u, w);
+    if (st != PRISM_OK) return st;
+    if (shape->T != 1) return PRISM_ERR_INVALID_ARG;
+    if (shape->dv > 128) return PRISM_ERR_UNSUPPORTED;
+    if (shape->B == 0 || shape->H == 0) return PRISM_OK;
+    if (!S || !aligned16(S) || !o || !aligned16(o)) return PRISM_ERR_INVALID_ARG;
+    if ((long long)shape->B * shape->H > 0x7fffffffLL) return PRISM_ERR_UNSUPPORTED;
+    prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, nullptr, o, S, nullptr);
+    cudaError_t err = prism::launch_decode(a, shape->io == PRISM_F32, (cudaStream_t)stream);
+    return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
+prism_status prism_query_device_status(void *workspace, void *stream) {
+    if (!workspace) return PRISM_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return PRISM_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return PRISM_ERR_CUDA;
+    if (word != PRISM_OK) {
+        if (cudaMemset(workspace, 0, sizeof word) != cudaSuccess) return PRISM_ERR_CUDA;
+    }
+    return word == PRISM_OK ? PRISM_OK : (prism_status)word;
+}
+
+const char *prism_status_string(prism_status status) {
+    switch (status) {
+        case PRISM_OK: return "PRISM_OK";
+        case PRISM_ERR_INVALID_ARG: return "PRISM_ERR_INVALID_ARG";
+        case PRISM_ERR_UNSUPPORTED: return "PRISM_ERR_UNSUPPORTED";
+        case PRISM_ERR_CUDA: return "PRISM_ERR_CUDA";
+        case PRISM_ERR_TIMEOUT: return "PRISM_ERR_TIMEOUT";
+    }
+    return "PRISM_ERR_UNKNOWN";
+}
+
+int prism_debug_set_flags(int flags) {
+    int old = g_debug_flags;
+    g_debug_flags = flags;
+    return old;
+}
+
+}  // extern "C"

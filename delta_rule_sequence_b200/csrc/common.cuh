@@ -1,0 +1,65 @@
+// common.cuh -- device helpers shared by the libprism kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/prism.h"
+
+namespace prism {
+
+// Arguments of one prism_scan_fwd call, as the kernels see them.
+struct ScanArgs {
+    int B, H, T, dk, dv, L, chunk;
+    const void *q, *k, *v;
+    const float *alpha, *beta;
+    const void *u, *w;
+    const float *S0;
+    void *o;
+    float *S_final;
+    uint32_t *status;  // device status word (PRISM_OK / PRISM_ERR_TIMEOUT), may be null
+};
+
+// Workspace layout: [0, 256) status block; segment data of the segmented scan after it.
+constexpr size_t kStatusBytes = 256;
+
+template <typename IO>
+__device__ __forceinline__ float ld_io(const IO *p, size_t i);
+template <>
+__device__ __forceinline__ float ld_io<float>(const float *p, size_t i) { return p[i]; }
+template <>
+__device__ __forceinline__ float ld_io<__nv_bfloat16>(const __nv_bfloat16 *p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+
+template <typename IO>
+__device__ __forceinline__ void st_io(IO *p, size_t i, float x);
+template <>
+__device__ __forceinline__ void st_io<float>(float *p, size_t i, float x) { p[i] = x; }
+template <>
+__device__ __forceinline__ void st_io<__nv_bfloat16>(__nv_bfloat16 *p, size_t i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__device__ __forceinline__ float warp_inclusive_scan(float x, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    return x;
+}
+
+// Record a device-side failure without trapping: the first failure wins.
+__device__ __forceinline__ void record_status(uint32_t *status, uint32_t code) {
+    if (status) atomicCAS(status, (uint32_t)PRISM_OK, code);
+}
+
+}  // namespace prism

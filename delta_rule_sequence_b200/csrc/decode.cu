@@ -1,0 +1,174 @@
+// decode.cu -- single-token recurrent step: an HBM-bound rank-(L+1) update of the fp32 state.
+//
+// For each (b, h) and each state row s_r (length dk), with e_r = s_r.k and p_r = s_r.q:
+//   s_r <- alpha s_r - alpha beta e_r k + sum_l u_{l,r} w_l
+//   o_r  = alpha p_r - alpha beta e_r (k.q) + sum_l u_{l,r} (w_l.q)
+// i.e. S <- alpha S (I - beta k k^T) + sum_l u_l w_l^T and o = S q with the updated S (PRISM,
+// gist.science explainer, technical summary 2.1-2.2; streaming inference of "Sequential Parallel
+// Duality in Prefix Scannable Models": one state updated per token, since the monoid is
+// associative).  The state is read once and written once; everything else is a few KB per head.
+//
+// Layout: one CTA (8 warps) per head; a warp owns rows r = warp, warp + 8, ...; a lane holds
+// dk/32 consecutive columns (a 16-byte vector at dk = 128).  Four rows are in flight per warp
+// iteration so that every SM keeps enough bytes outstanding to saturate HBM.
+
+#include "common.cuh"
+
+namespace prism {
+namespace {
+
+constexpr int NT = 256;
+constexpr int NW = NT / 32;
+constexpr int ROWS_IN_FLIGHT = 4;
+constexpr int MAXL = 8;
+
+template <int N>
+struct VecF;
+template <> struct VecF<1> { using T = float; };
+template <> struct VecF<2> { using T = float2; };
+template <> struct VecF<4> { using T = float4; };
+
+template <int N>
+__device__ __forceinline__ void vload(const float *p, float (&x)[N]) {
+    using V = typename VecF<N>::T;
+    V t = __ldcs(reinterpret_cast<const V *>(p));  // streamed: read once
+    const float *f = reinterpret_cast<const float *>(&t);
+#pragma unroll
+    for (int i = 0; i < N; ++i) x[i] = f[i];
+}
+
+template <int N>
+__device__ __forceinline__ void vstore(float *p, const float (&x)[N]) {
+    using V = typename VecF<N>::T;
+    V t;
+    float *f = reinterpret_cast<float *>(&t);
+#pragma unroll
+    for (int i = 0; i < N; ++i) f[i] = x[i];
+    __stcs(reinterpret_cast<V *>(p), t);
+}
+
+template <typename IO, int DK>
+__global__ void __launch_bounds__(NT) decode_kernel(ScanArgs p) {
+    constexpr int PER = DK / 32;  // columns per lane
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int head = blockIdx.x;  // b * H + h
+    const int dv = p.dv, L = p.L;
+    const bool gdn = (p.u == nullptr);
+    const IO *q = (const IO *)p.q, *k = (const IO *)p.k, *v = (const IO *)p.v;
+    const IO *u = (const IO *)p.u, *w = (const IO *)p.w;
+
+    __shared__ float s_u[MAXL][128];  // u_{l,r} (or beta v_r)
+    __shared__ float s_wq[MAXL];
+
+    const float a = p.alpha[head];
+    const float be = p.beta[head];
+    float kq[PER], qv[PER], wl[MAXL][PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        size_t idx = (size_t)head * DK + lane * PER + i;
+        kq[i] = ld_io(k, idx);
+        qv[i] = ld_io(q, idx);
+    }
+    const int Lw = gdn ? 1 : L;
+#pragma unroll
+    for (int l = 0; l < MAXL; ++l) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            float x = 0.f;
+            if (l < Lw) x = gdn ? kq[i] : ld_io(w, ((size_t)head * L + l) * DK + lane * PER + i);
+            wl[l][i] = x;
+        }
+    }
+    for (int e = threadIdx.x; e < Lw * dv; e += NT) {
+        int l = e / dv, r = e % dv;
+        s_u[l][r] = gdn ? be * ld_io(v, (size_t)head * dv + r)
+                        : ld_io(u, ((size_t)head * L + l) * dv + r);
+    }
+    // k.q and w_l.q (each warp computes its own copy; lane-local partials then a reduction)
+    float kdotq = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) kdotq = fmaf(kq[i], qv[i], kdotq);
+    kdotq = warp_sum(kdotq);
+    if (warp == 0) {
+#pragma unroll
+        for (int l = 0; l < MAXL; ++l) {
+            if (l < Lw) {
+                float t = 0.f;
+#pragma unroll
+                for (int i = 0; i < PER; ++i) t = fmaf(wl[l][i], qv[i], t);
+                t = warp_sum(t);
+                if (lane == 0) s_wq[l] = t;
+            }
+        }
+    }
+    __syncthreads();
+
+    float *S = p.S_final + (size_t)head * dv * DK;  // in place
+    IO *o = (IO *)p.o + (size_t)head * dv;
+    const float ab = a * be;
+
+    for (int r0 = warp * ROWS_IN_FLIGHT; r0 < dv; r0 += NW * ROWS_IN_FLIGHT) {
+        float s[ROWS_IN_FLIGHT][PER];
+#pragma unroll
+        for (int j = 0; j < ROWS_IN_FLIGHT; ++j) vload<PER>(S + (size_t)(r0 + j) * DK + lane * PER, s[j]);
+#pragma unroll
+        for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
+            const int r = r0 + j;
+            float e = 0.f, pq = 0.f;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                e = fmaf(s[j][i], kq[i], e);
+                pq = fmaf(s[j][i], qv[i], pq);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                e += __shfl_xor_sync(0xffffffffu, e, off);
+                pq += __shfl_xor_sync(0xffffffffu, pq, off);
+            }
+            float outv = a * pq - ab * e * kdotq;
+            float ns[PER];
+#pragma unroll
+            for (int i = 0; i < PER; ++i) ns[i] = fmaf(a, s[j][i], -ab * e * kq[i]);
+#pragma unroll
+            for (int l = 0; l < MAXL; ++l) {
+                if (l < Lw) {
+                    const float ur = s_u[l][r];
+                    outv = fmaf(ur, s_wq[l], outv);
+#pragma unroll
+                    for (int i = 0; i < PER; ++i) ns[i] = fmaf(ur, wl[l][i], ns[i]);
+                }
+            }
+            vstore<PER>(S + (size_t)r * DK + lane * PER, ns);
+            if (lane == 0) st_io(o, r, outv);
+        }
+    }
+}
+
+template <typename IO, int DK>
+cudaError_t launch_decode_dk(const ScanArgs &a, cudaStream_t s) {
+    decode_kernel<IO, DK><<<a.B * a.H, NT, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Entry used by the C ABI.  a.S_final is the in-place state.  Requires dv <= 128, L <= 8 and
+// dv a multiple of 32 (checked by the caller).
+cudaError_t launch_decode(const ScanArgs &a, bool io_f32, cudaStream_t s) {
+    if (io_f32) {
+        switch (a.dk) {
+            case 32: return launch_decode_dk<float, 32>(a, s);
+            case 64: return launch_decode_dk<float, 64>(a, s);
+            case 128: return launch_decode_dk<float, 128>(a, s);
+        }
+    } else {
+        switch (a.dk) {
+            case 32: return launch_decode_dk<__nv_bfloat16, 32>(a, s);
+            case 64: return launch_decode_dk<__nv_bfloat16, 64>(a, s);
+            case 128: return launch_decode_dk<__nv_bfloat16, 128>(a, s);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace prism

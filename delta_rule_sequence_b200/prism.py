@@ -1,0 +1,212 @@
+"""ctypes binding of libprism.so (C ABI in include/prism.h).
+
+Argument marshalling only: shapes are read from torch tensors, outputs and workspace are
+allocated with torch when the caller does not pass them, and every step of the computation runs
+in the library's CUDA kernels on the current torch stream.  There is no CPU fallback: if the
+library is missing or the tensors are not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libprism.so")
+
+PRISM_OK, PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED, PRISM_ERR_CUDA, PRISM_ERR_TIMEOUT = range(5)
+PRISM_BF16, PRISM_F32 = 0, 1
+
+# Every symbol that include/prism.h declares.
+EXPORTS = (
+    "prism_scan_fwd_workspace_size",
+    "prism_scan_fwd_launch_count",
+    "prism_scan_fwd",
+    "prism_step_decode",
+    "prism_query_device_status",
+    "prism_status_string",
+    "prism_debug_set_flags",
+)
+
+
+class PrismError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+class PrismShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("L", ctypes.c_int),
+                ("chunk", ctypes.c_int), ("io", ctypes.c_int)]
+
+
+_lib = None
+
+
+def load_library():
+    """Load libprism.so (built in-tree by delta_rule_sequence_b200.build); raise if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"libprism.so is not built ({LIB_PATH}); run `python -m delta_rule_sequence_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, sz, ci = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    shp = ctypes.POINTER(PrismShape)
+    lib.prism_scan_fwd_workspace_size.argtypes = [shp, ctypes.POINTER(sz)]
+    lib.prism_scan_fwd_workspace_size.restype = ci
+    lib.prism_scan_fwd_launch_count.argtypes = [shp, ctypes.POINTER(ci)]
+    lib.prism_scan_fwd_launch_count.restype = ci
+    lib.prism_scan_fwd.argtypes = [shp] + [vp] * 10 + [vp, sz, vp]
+    lib.prism_scan_fwd.restype = ci
+    lib.prism_step_decode.argtypes = [shp] + [vp] * 9 + [vp]
+    lib.prism_step_decode.restype = ci
+    lib.prism_query_device_status.argtypes = [vp, vp]
+    lib.prism_query_device_status.restype = ci
+    lib.prism_status_string.argtypes = [ci]
+    lib.prism_status_string.restype = ctypes.c_char_p
+    lib.prism_debug_set_flags.argtypes = [ci]
+    lib.prism_debug_set_flags.restype = ci
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return load_library().prism_status_string(int(status)).decode()
+    except RuntimeError:
+        return f"status {status}"
+
+
+def _ptr(x):
+    return None if x is None else ctypes.c_void_p(x.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_tensor(name, x, dtype, shape, device):
+    if x is None:
+        return
+    if not isinstance(x, torch.Tensor) or not x.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (libprism has no CPU path)")
+    if x.device != device:
+        raise ValueError(f"{name} is on {x.device}, q is on {device}")
+    if x.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {x.dtype}")
+    if tuple(x.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(x.shape)}")
+    if not x.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def make_shape(q, v=None, u=None, chunk=64, L=None) -> PrismShape:
+    B, T, H, dk = q.shape
+    if u is not None:
+        Lr, dv = u.shape[3], u.shape[4]
+    else:
+        Lr, dv = 1, v.shape[3]
+    io = PRISM_F32 if q.dtype == torch.float32 else PRISM_BF16
+    return PrismShape(B, H, T, dk, dv, L or Lr, chunk, io)
+
+
+_ws_cache = {}
+
+
+def workspace_for(shape: PrismShape, device) -> torch.Tensor:
+    """A cached device workspace of the size prism_scan_fwd needs (one per device/size)."""
+    need = ctypes.c_size_t(0)
+    rc = load_library().prism_scan_fwd_workspace_size(ctypes.byref(shape), ctypes.byref(need))
+    if rc != PRISM_OK:
+        raise PrismError(rc, "prism_scan_fwd_workspace_size")
+    key = (str(device), int(need.value))
+    ws = _ws_cache.get(key)
+    if ws is None:
+        ws = torch.zeros(max(256, int(need.value)), dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def prism_scan_fwd(q, k, v, alpha, beta, u=None, w=None, S0=None, *, chunk=64, o=None,
+                   S_final=None, want_state=True, workspace=None, stream=None):
+    """Chunked scan forward.  q, k: [B,T,H,dk]; v: [B,T,H,dv] or None; alpha, beta: [B,T,H]
+    fp32; u: [B,T,H,L,dv] / w: [B,T,H,L,dk] or None; S0: [B,H,dv,dk] fp32 or None.
+    Returns (o [B,T,H,dv], S_final [B,H,dv,dk] fp32 or None)."""
+    lib = load_library()
+    if not isinstance(q, torch.Tensor) or not q.is_cuda:
+        raise TypeError("q must be a CUDA tensor (libprism has no CPU path)")
+    dev, io = q.device, q.dtype
+    shape = make_shape(q, v, u, chunk)
+    B, T, H, dk = q.shape
+    dv, L = shape.dv, shape.L
+    _check_tensor("q", q, io, (B, T, H, dk), dev)
+    _check_tensor("k", k, io, (B, T, H, dk), dev)
+    _check_tensor("v", v, io, (B, T, H, dv), dev)
+    _check_tensor("alpha", alpha, torch.float32, (B, T, H), dev)
+    _check_tensor("beta", beta, torch.float32, (B, T, H), dev)
+    _check_tensor("u", u, io, (B, T, H, L, dv), dev)
+    _check_tensor("w", w, io, (B, T, H, L, dk), dev)
+    _check_tensor("S0", S0, torch.float32, (B, H, dv, dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=io, device=dev)
+    _check_tensor("o", o, io, (B, T, H, dv), dev)
+    if S_final is None and want_state:
+        S_final = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    _check_tensor("S_final", S_final, torch.float32, (B, H, dv, dk), dev)
+    if workspace is None:
+        workspace = workspace_for(shape, dev)
+    rc = lib.prism_scan_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                            _ptr(beta), _ptr(u), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_final),
+                            _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if rc != PRISM_OK:
+        raise PrismError(rc, "prism_scan_fwd")
+    return o, S_final
+
+
+def prism_step_decode(q, k, v, alpha, beta, u, w, S, *, o=None, stream=None):
+    """One decode step, S updated in place.  q, k: [B,1,H,dk]; v: [B,1,H,dv] or None;
+    alpha, beta: [B,1,H]; u: [B,1,H,L,dv] / w: [B,1,H,L,dk] or None; S: [B,H,dv,dk] fp32.
+    Returns o [B,1,H,dv]."""
+    lib = load_library()
+    if not isinstance(q, torch.Tensor) or not q.is_cuda:
+        raise TypeError("q must be a CUDA tensor (libprism has no CPU path)")
+    dev, io = q.device, q.dtype
+    shape = make_shape(q, v, u, 64)
+    B, T, H, dk = q.shape
+    dv, L = shape.dv, shape.L
+    _check_tensor("q", q, io, (B, T, H, dk), dev)
+    _check_tensor("k", k, io, (B, T, H, dk), dev)
+    _check_tensor("v", v, io, (B, T, H, dv), dev)
+    _check_tensor("alpha", alpha, torch.float32, (B, T, H), dev)
+    _check_tensor("beta", beta, torch.float32, (B, T, H), dev)
+    _check_tensor("u", u, io, (B, T, H, L, dv), dev)
+    _check_tensor("w", w, io, (B, T, H, L, dk), dev)
+    _check_tensor("S", S, torch.float32, (B, H, dv, dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=io, device=dev)
+    _check_tensor("o", o, io, (B, T, H, dv), dev)
+    rc = lib.prism_step_decode(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                               _ptr(beta), _ptr(u), _ptr(w), _ptr(S), _ptr(o), _stream(stream))
+    if rc != PRISM_OK:
+        raise PrismError(rc, "prism_step_decode")
+    return o
+
+
+def prism_scan_fwd_launch_count(shape: PrismShape) -> int:
+    """Kernels one prism_scan_fwd call with `shape` enqueues."""
+    n = ctypes.c_int(0)
+    rc = load_library().prism_scan_fwd_launch_count(ctypes.byref(shape), ctypes.byref(n))
+    if rc != PRISM_OK:
+        raise PrismError(rc, "prism_scan_fwd_launch_count")
+    return n.value
+
+
+def prism_query_device_status(workspace, stream=None) -> int:
+    """Synchronise and return (and clear) the status word kernels wrote into `workspace`."""
+    return load_library().prism_query_device_status(_ptr(workspace), _stream(stream))

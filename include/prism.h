@@ -1,0 +1,133 @@
+/*
+ * prism.h -- C ABI of libprism.so: the gated delta-rule chunked scan forward with a rank-L
+ * residual write, and its single-token decode step, on NVIDIA B200 (sm_100a).
+ *
+ * The operation (per batch b, head h; state S is dv x dk fp32, rows are the value index):
+ *
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + sum_{l=1..L} u_{t,l} w_{t,l}^T
+ *     o_t = S_t q_t
+ *
+ * Sources:
+ *   - "PRISM: Parallel Residual Iterative Sequence Model" (gist.science explainer), technical
+ *     summary section 2.1 (write-forget decoupling: S_t = S_{t-1} A_t + B_t, the forget A_t kept
+ *     in Gated-DeltaNet form) and section 2.2 (the rank-L write B_t = sum_l beta^(l) delta^(l)
+ *     k^(l)T; here u_{t,l} = beta^(l) delta^(l) and w_{t,l} = k^(l), produced upstream).
+ *   - banbantang.com PRISM article, section 1(4): Gated-DeltaNet's scalar decay alpha, rank-1
+ *     erase along k and rank-1 write beta v k^T (the L = 1 write used when u, w are NULL).
+ *   - "Sequential Parallel Duality in Prefix Scannable Models" (papernotes), key design 2 and the
+ *     method overview: each token is an affine element (E_t, f_t) with E_t = alpha_t(I - beta_t
+ *     k_t k_t^T), f_t = sum_l u_{t,l} w_{t,l}^T; elements compose associatively, so the sequence
+ *     is cut into chunks, each chunk is encoded, and the chunk elements are scanned.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers unless stated otherwise; every buffer is allocated by the caller.  The
+ *     library never allocates device or host memory and never synchronises the stream except in
+ *     prism_query_device_status.
+ *   - Layouts are dense row-major: activations [B,T,H,d]; u [B,T,H,L,dv]; w [B,T,H,L,dk];
+ *     alpha, beta [B,T,H]; states [B,H,dv,dk].  Every pointer must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL is the legacy default stream).  All work is
+ *     enqueued on it asynchronously.
+ *   - Arguments are validated before anything is launched; a rejected call enqueues nothing.
+ *     A launch failure returns PRISM_ERR_CUDA.  Kernels never trap: a bounded wait that runs out
+ *     records PRISM_ERR_TIMEOUT in the workspace status word (read with
+ *     prism_query_device_status).
+ *   - Outputs must not alias inputs (except the decode state, which is updated in place).
+ */
+#ifndef PRISM_H
+#define PRISM_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PRISM_OK = 0,
+    PRISM_ERR_INVALID_ARG = 1,  /* bad size, NULL pointer, misalignment, short workspace */
+    PRISM_ERR_UNSUPPORTED = 2,  /* valid but not built: d not in {32,64,128}, L > 8 ...     */
+    PRISM_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed              */
+    PRISM_ERR_TIMEOUT = 4       /* a kernel's bounded wait gave up (device status word)     */
+} prism_status;
+
+typedef enum { PRISM_BF16 = 0, PRISM_F32 = 1 } prism_dtype;
+
+typedef struct {
+    int B, H, T;      /* batch, heads, tokens (T >= 0; decode requires T == 1)              */
+    int dk, dv;       /* key and value widths, each in {32, 64, 128}                        */
+    int L;            /* write rank, 1..8; must be 1 when u and w are NULL                  */
+    int chunk;        /* chunk length of the chunked scan: 64 or 128 (ignored by decode)     */
+    prism_dtype io;   /* type of q, k, v, u, w and of o (alpha, beta, states are fp32)      */
+} prism_shape;
+
+/*
+ * prism_scan_fwd_workspace_size -- bytes of device workspace prism_scan_fwd needs for `shape`
+ * (the status word, plus the per-segment affine elements of the segmented scan when B*H is too
+ * small to fill the GPU).  Writes *bytes; never fails for a valid shape.
+ */
+prism_status prism_scan_fwd_workspace_size(const prism_shape *shape, size_t *bytes);
+
+/*
+ * prism_scan_fwd_launch_count -- number of kernels one prism_scan_fwd call with `shape` enqueues
+ * (the plan depends on B*H, T and the widths).  Host only; writes *launches.
+ */
+prism_status prism_scan_fwd_launch_count(const prism_shape *shape, int *launches);
+
+/*
+ * prism_scan_fwd -- chunked parallel-scan forward over T tokens for all B*H sequences.
+ *
+ *   q, k     [B,T,H,dk] io     queries and keys (the kernel normalises nothing)
+ *   v        [B,T,H,dv] io     values; read only when u == w == NULL (Gated-DeltaNet write
+ *                              beta_t v_t k_t^T, requires L == 1); may be NULL otherwise
+ *   alpha    [B,T,H] fp32      decay gate, in (0, 1]  (alpha = 0 is outside the domain: the
+ *                              chunk form takes log alpha)
+ *   beta     [B,T,H] fp32      erase gate
+ *   u, w     [B,T,H,L,dv], [B,T,H,L,dk] io, or both NULL: the rank-L write sum_l u w^T
+ *   S0       [B,H,dv,dk] fp32  entry state, or NULL for zeros
+ *   o        [B,T,H,dv] io     output (bf16 outputs are rounded to nearest even)
+ *   S_final  [B,H,dv,dk] fp32  exit state, or NULL to skip; S_final == S0 is allowed
+ *   workspace, ws_bytes        device scratch of at least prism_scan_fwd_workspace_size bytes,
+ *                              256-byte aligned, zero-filled by the caller before its first
+ *                              use (the status word in its first 4 bytes stays zero unless a
+ *                              kernel records a failure; prism_query_device_status reads and
+ *                              clears it); may be reused once the stream has passed this call
+ * The result equals the token recurrence above up to floating-point rounding: state and all
+ * accumulation in fp32; bf16 operands are fed to the tensor cores.  A partial last chunk is
+ * handled as if padded with identity tokens (alpha = 1, beta = 0, no write).
+ */
+prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void *k,
+                            const void *v, const float *alpha, const float *beta,
+                            const void *u, const void *w, const float *S0, void *o,
+                            float *S_final, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * prism_step_decode -- one token for each of the B*H sequences (shape->T must be 1):
+ *   S <- alpha S (I - beta k k^T) + sum_l u_l w_l^T   (in place),   o = S q.
+ * Arguments as for prism_scan_fwd with T == 1; S is read and written in place, [B,H,dv,dk]
+ * fp32; o is [B,1,H,dv] io.  A pure HBM-bound rank-(L+1) update: one read and one write of S.
+ */
+prism_status prism_step_decode(const prism_shape *shape, const void *q, const void *k,
+                               const void *v, const float *alpha, const float *beta,
+                               const void *u, const void *w, float *S, void *o, void *stream);
+
+/*
+ * prism_query_device_status -- synchronise `stream`, read the status word in `workspace`
+ * (written by kernels whose bounded waits ran out) and clear it.  Returns PRISM_OK,
+ * PRISM_ERR_TIMEOUT, or PRISM_ERR_CUDA if the stream itself reports an error.
+ */
+prism_status prism_query_device_status(void *workspace, void *stream);
+
+/* prism_status_string -- a static, human-readable name for a status code. */
+const char *prism_status_string(prism_status status);
+
+/*
+ * prism_debug_set_flags -- testing hook.  flags bit 0: the next timed-wait kernel skips one
+ * producer signal so its consumer must give up and record PRISM_ERR_TIMEOUT (checks the
+ * bounded-wait path without hanging anything).  Returns the previous flags.
+ */
+int prism_debug_set_flags(int flags);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PRISM_H */

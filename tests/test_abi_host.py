@@ -1,0 +1,122 @@
+"""Host-only checks of the C ABI: the libraries load, export every declared symbol, and reject bad
+arguments before anything is launched (so these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from delta_rule_sequence_b200 import prism as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared(header):
+    text = open(os.path.join(ROOT, "include", header)).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(prism_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from delta_rule_sequence_b200 import build
+
+    build.build()
+    return P.load_library()
+
+
+def test_prism_h_symbols_exported(lib):
+    names = _declared("prism.h")
+    assert set(names) == set(P.EXPORTS), names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_prism_ref_h_symbols_exported():
+    lib = ctypes.CDLL(oracle.build())
+    for n in _declared("prism_ref.h"):
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code, name in enumerate(["PRISM_OK", "PRISM_ERR_INVALID_ARG", "PRISM_ERR_UNSUPPORTED",
+                                 "PRISM_ERR_CUDA", "PRISM_ERR_TIMEOUT"]):
+        assert P.status_string(code) == name
+    assert P.status_string(99) == "PRISM_ERR_UNKNOWN"
+
+
+def _shape(**kw):
+    base = dict(B=1, H=2, T=256, dk=32, dv=32, L=1, chunk=64, io=P.PRISM_F32)
+    base.update(kw)
+    return P.PrismShape(**base)
+
+
+FAKE = ctypes.c_void_p(0x10000)       # 16-byte aligned, never dereferenced: calls fail before launch
+MISALIGNED = ctypes.c_void_p(0x10004)
+
+
+def _fwd(lib, shape, q=FAKE, k=FAKE, v=FAKE, a=FAKE, b=FAKE, u=None, w=None, S0=None, o=FAKE,
+         Sf=None, ws=ctypes.c_void_p(0x20000), ws_bytes=256):
+    return lib.prism_scan_fwd(ctypes.byref(shape), q, k, v, a, b, u, w, S0, o, Sf, ws,
+                              ctypes.c_size_t(ws_bytes), None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dk=48), P.PRISM_ERR_UNSUPPORTED),
+    (dict(dv=256), P.PRISM_ERR_UNSUPPORTED),
+    (dict(L=0), P.PRISM_ERR_INVALID_ARG),
+    (dict(L=9), P.PRISM_ERR_UNSUPPORTED),
+    (dict(L=2), P.PRISM_ERR_INVALID_ARG),       # u, w NULL needs L == 1
+    (dict(chunk=32), P.PRISM_ERR_INVALID_ARG),
+    (dict(T=-1), P.PRISM_ERR_INVALID_ARG),
+    (dict(io=7), P.PRISM_ERR_INVALID_ARG),
+])
+def test_scan_rejects_bad_shapes(lib, kw, expect):
+    assert _fwd(lib, _shape(**kw)) == expect
+
+
+def test_scan_rejects_bad_pointers(lib):
+    s = _shape()
+    assert _fwd(lib, s, q=None) == P.PRISM_ERR_INVALID_ARG
+    assert _fwd(lib, s, v=None) == P.PRISM_ERR_INVALID_ARG          # GDN write needs v
+    assert _fwd(lib, s, u=FAKE) == P.PRISM_ERR_INVALID_ARG          # u without w
+    assert _fwd(lib, s, k=MISALIGNED) == P.PRISM_ERR_INVALID_ARG
+    assert _fwd(lib, s, o=None) == P.PRISM_ERR_INVALID_ARG
+    assert _fwd(lib, s, o=FAKE, q=FAKE) == P.PRISM_ERR_INVALID_ARG  # o aliases q
+    assert _fwd(lib, s, ws=None) == P.PRISM_ERR_INVALID_ARG
+    assert _fwd(lib, s, ws_bytes=8) == P.PRISM_ERR_INVALID_ARG
+    assert _fwd(lib, s, ws=ctypes.c_void_p(0x20010)) == P.PRISM_ERR_INVALID_ARG  # not 256-aligned
+    assert lib.prism_scan_fwd(None, *([None] * 10), None, 0, None) == P.PRISM_ERR_INVALID_ARG
+
+
+def test_decode_rejects_bad_arguments(lib):
+    s = _shape(T=2)
+    args = [FAKE] * 5 + [None, None, FAKE, FAKE, None]
+    assert lib.prism_step_decode(ctypes.byref(s), *args) == P.PRISM_ERR_INVALID_ARG  # T != 1
+    s = _shape(T=1)
+    bad = [FAKE] * 5 + [None, None, None, FAKE, None]
+    assert lib.prism_step_decode(ctypes.byref(s), *bad) == P.PRISM_ERR_INVALID_ARG  # S NULL
+
+
+def test_workspace_size(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.prism_scan_fwd_workspace_size(ctypes.byref(_shape()), ctypes.byref(n)) == 0
+    assert n.value >= 256
+    assert lib.prism_scan_fwd_workspace_size(None, ctypes.byref(n)) == P.PRISM_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(P, "_lib", None)
+    monkeypatch.setattr(P, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        P.load_library()
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+
+    x = torch.zeros((1, 4, 1, 32))
+    with pytest.raises(TypeError, match="CUDA"):
+        P.prism_scan_fwd(x, x, x, torch.ones(1, 4, 1), torch.zeros(1, 4, 1))
