@@ -9,6 +9,8 @@
 namespace prism {
 cudaError_t launch_scan_simt(const ScanArgs &a, bool io_f32, cudaStream_t s);
 cudaError_t launch_decode(const ScanArgs &a, bool io_f32, cudaStream_t s);
+bool scan_tc_supported(const ScanArgs &a, bool io_f32);
+cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
 }  // namespace prism
 
 namespace {
@@ -28,16 +30,17 @@ prism_status check_common(const prism_shape *s, const void *q, const void *k, co
     if (s->dk < 1 || s->dv < 1) return PRISM_ERR_INVALID_ARG;
     if (!width_ok(s->dk) || !width_ok(s->dv) || s->L > 8) return PRISM_ERR_UNSUPPORTED;
     if (s->B > 65535 || s->H > 65535) return PRISM_ERR_UNSUPPORTED;
+    // With no tokens nothing below is read (an empty tensor may even have a NULL data pointer).
+    const bool work = (long long)s->B * s->H * s->T > 0;
+    if (!work) return PRISM_OK;
     if ((u == nullptr) != (w == nullptr)) return PRISM_ERR_INVALID_ARG;
     if (u == nullptr && s->L != 1) return PRISM_ERR_INVALID_ARG;
-    const bool work = (long long)s->B * s->H * s->T > 0;
-    if (work) {
-        if (!q || !k || !alpha || !beta) return PRISM_ERR_INVALID_ARG;
-        if (u == nullptr && v == nullptr) return PRISM_ERR_INVALID_ARG;
-    }
-    const void *ptrs[] = {q, k, v, alpha, beta, u, w};
+    if (!q || !k || !alpha || !beta) return PRISM_ERR_INVALID_ARG;
+    if (u == nullptr && v == nullptr) return PRISM_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, u, w};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return PRISM_ERR_INVALID_ARG;
+    if (((uintptr_t)alpha & 3u) || ((uintptr_t)beta & 3u)) return PRISM_ERR_INVALID_ARG;
     return PRISM_OK;
 }
 
@@ -91,7 +94,9 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
     if (shape->T == 0 && !S_final) return PRISM_OK;
 
     prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, S0, o, S_final, status);
-    cudaError_t err = prism::launch_scan_simt(a, shape->io == PRISM_F32, s);
+    const bool io_f32 = shape->io == PRISM_F32;
+    cudaError_t err = prism::scan_tc_supported(a, io_f32) ? prism::launch_scan_tc(a, s)
+                                                          : prism::launch_scan_simt(a, io_f32, s);
     return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 

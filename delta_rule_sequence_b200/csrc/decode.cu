@@ -8,9 +8,10 @@
 // Duality in Prefix Scannable Models": one state updated per token, since the monoid is
 // associative).  The state is read once and written once; everything else is a few KB per head.
 //
-// Layout: one CTA (8 warps) per head; a warp owns rows r = warp, warp + 8, ...; a lane holds
-// dk/32 consecutive columns (a 16-byte vector at dk = 128).  Four rows are in flight per warp
-// iteration so that every SM keeps enough bytes outstanding to saturate HBM.
+// Layout: one CTA (8 warps) per head; a warp owns blocks of 8 consecutive rows; a lane holds
+// dk/32 consecutive columns (a 16-byte vector at dk = 128).  All 8 rows of a block are loaded
+// before any is reduced so that every SM keeps enough bytes in flight to saturate HBM.  The state
+// is streamed (evict-first loads and stores): it is far larger than L2 and touched once per step.
 
 #include "common.cuh"
 
@@ -19,8 +20,7 @@ namespace {
 
 constexpr int NT = 256;
 constexpr int NW = NT / 32;
-constexpr int ROWS_IN_FLIGHT = 4;
-constexpr int MAXL = 8;
+constexpr int ROWS_IN_FLIGHT = 8;
 
 template <int N>
 struct VecF;
@@ -31,7 +31,7 @@ template <> struct VecF<4> { using T = float4; };
 template <int N>
 __device__ __forceinline__ void vload(const float *p, float (&x)[N]) {
     using V = typename VecF<N>::T;
-    V t = __ldcs(reinterpret_cast<const V *>(p));  // streamed: read once
+    V t = __ldcs(reinterpret_cast<const V *>(p));
     const float *f = reinterpret_cast<const float *>(&t);
 #pragma unroll
     for (int i = 0; i < N; ++i) x[i] = f[i];
@@ -47,8 +47,18 @@ __device__ __forceinline__ void vstore(float *p, const float (&x)[N]) {
     __stcs(reinterpret_cast<V *>(p), t);
 }
 
-template <typename IO, int DK>
-__global__ void __launch_bounds__(NT) decode_kernel(ScanArgs p) {
+template <int N>
+__device__ __forceinline__ void vload_shared(const float *p, float (&x)[N]) {
+    using V = typename VecF<N>::T;
+    V t = *reinterpret_cast<const V *>(p);
+    const float *f = reinterpret_cast<const float *>(&t);
+#pragma unroll
+    for (int i = 0; i < N; ++i) x[i] = f[i];
+}
+
+// LW = number of write terms (L, or 1 for the Gated-DeltaNet write beta v k^T).
+template <typename IO, int DK, int LW>
+__global__ void __launch_bounds__(NT, 3) decode_kernel(ScanArgs p) {
     constexpr int PER = DK / 32;  // columns per lane
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int head = blockIdx.x;  // b * H + h
@@ -57,60 +67,67 @@ __global__ void __launch_bounds__(NT) decode_kernel(ScanArgs p) {
     const IO *q = (const IO *)p.q, *k = (const IO *)p.k, *v = (const IO *)p.v;
     const IO *u = (const IO *)p.u, *w = (const IO *)p.w;
 
-    __shared__ float s_u[MAXL][128];  // u_{l,r} (or beta v_r)
-    __shared__ float s_wq[MAXL];
+    __shared__ float s_u[LW][128];                 // u_{l,r} (or beta v_r)
+    __shared__ __align__(16) float s_w[LW][DK];   // w_l (or k)
+    __shared__ float s_wq[LW];
+
+    // Issue the loads of this warp's first block of state rows before the per-head prologue,
+    // so that their latency overlaps the prologue's.
+    float *S = p.S_final + (size_t)head * dv * DK;  // in place
+    float s[ROWS_IN_FLIGHT][PER];
+    int r0 = warp * ROWS_IN_FLIGHT;
+    if (r0 < dv) {
+#pragma unroll
+        for (int j = 0; j < ROWS_IN_FLIGHT; ++j)
+            vload<PER>(S + (size_t)(r0 + j) * DK + lane * PER, s[j]);
+    }
 
     const float a = p.alpha[head];
     const float be = p.beta[head];
-    float kq[PER], qv[PER], wl[MAXL][PER];
+    float kq[PER], qv[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
         size_t idx = (size_t)head * DK + lane * PER + i;
         kq[i] = ld_io(k, idx);
         qv[i] = ld_io(q, idx);
     }
-    const int Lw = gdn ? 1 : L;
-#pragma unroll
-    for (int l = 0; l < MAXL; ++l) {
-#pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            float x = 0.f;
-            if (l < Lw) x = gdn ? kq[i] : ld_io(w, ((size_t)head * L + l) * DK + lane * PER + i);
-            wl[l][i] = x;
-        }
+    for (int e = threadIdx.x; e < LW * DK; e += NT) {
+        int l = e / DK, j = e % DK;
+        s_w[l][j] = gdn ? ld_io(k, (size_t)head * DK + j)
+                        : ld_io(w, ((size_t)head * L + l) * DK + j);
     }
-    for (int e = threadIdx.x; e < Lw * dv; e += NT) {
+    for (int e = threadIdx.x; e < LW * dv; e += NT) {
         int l = e / dv, r = e % dv;
         s_u[l][r] = gdn ? be * ld_io(v, (size_t)head * dv + r)
                         : ld_io(u, ((size_t)head * L + l) * dv + r);
     }
-    // k.q and w_l.q (each warp computes its own copy; lane-local partials then a reduction)
+    // k.q in every warp; warp 0 publishes the w_l.q
     float kdotq = 0.f;
 #pragma unroll
     for (int i = 0; i < PER; ++i) kdotq = fmaf(kq[i], qv[i], kdotq);
     kdotq = warp_sum(kdotq);
+    __syncthreads();
     if (warp == 0) {
 #pragma unroll
-        for (int l = 0; l < MAXL; ++l) {
-            if (l < Lw) {
-                float t = 0.f;
+        for (int l = 0; l < LW; ++l) {
+            float t = 0.f;
 #pragma unroll
-                for (int i = 0; i < PER; ++i) t = fmaf(wl[l][i], qv[i], t);
-                t = warp_sum(t);
-                if (lane == 0) s_wq[l] = t;
-            }
+            for (int i = 0; i < PER; ++i) t = fmaf(s_w[l][lane * PER + i], qv[i], t);
+            t = warp_sum(t);
+            if (lane == 0) s_wq[l] = t;
         }
     }
     __syncthreads();
 
-    float *S = p.S_final + (size_t)head * dv * DK;  // in place
     IO *o = (IO *)p.o + (size_t)head * dv;
     const float ab = a * be;
 
-    for (int r0 = warp * ROWS_IN_FLIGHT; r0 < dv; r0 += NW * ROWS_IN_FLIGHT) {
-        float s[ROWS_IN_FLIGHT][PER];
+    for (; r0 < dv; r0 += NW * ROWS_IN_FLIGHT) {
+        if (r0 != warp * ROWS_IN_FLIGHT) {
 #pragma unroll
-        for (int j = 0; j < ROWS_IN_FLIGHT; ++j) vload<PER>(S + (size_t)(r0 + j) * DK + lane * PER, s[j]);
+            for (int j = 0; j < ROWS_IN_FLIGHT; ++j)
+                vload<PER>(S + (size_t)(r0 + j) * DK + lane * PER, s[j]);
+        }
 #pragma unroll
         for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
             const int r = r0 + j;
@@ -129,14 +146,14 @@ __global__ void __launch_bounds__(NT) decode_kernel(ScanArgs p) {
             float ns[PER];
 #pragma unroll
             for (int i = 0; i < PER; ++i) ns[i] = fmaf(a, s[j][i], -ab * e * kq[i]);
+#pragma unroll 1
+            for (int l = 0; l < LW; ++l) {
+                const float ur = s_u[l][r];
+                outv = fmaf(ur, s_wq[l], outv);
+                float wv[PER];
+                vload_shared<PER>(&s_w[l][lane * PER], wv);
 #pragma unroll
-            for (int l = 0; l < MAXL; ++l) {
-                if (l < Lw) {
-                    const float ur = s_u[l][r];
-                    outv = fmaf(ur, s_wq[l], outv);
-#pragma unroll
-                    for (int i = 0; i < PER; ++i) ns[i] = fmaf(ur, wl[l][i], ns[i]);
-                }
+                for (int i = 0; i < PER; ++i) ns[i] = fmaf(ur, wv[i], ns[i]);
             }
             vstore<PER>(S + (size_t)r * DK + lane * PER, ns);
             if (lane == 0) st_io(o, r, outv);
@@ -144,16 +161,32 @@ __global__ void __launch_bounds__(NT) decode_kernel(ScanArgs p) {
     }
 }
 
+template <typename IO, int DK, int LW>
+cudaError_t launch_decode_l(const ScanArgs &a, cudaStream_t s) {
+    decode_kernel<IO, DK, LW><<<a.B * a.H, NT, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 template <typename IO, int DK>
 cudaError_t launch_decode_dk(const ScanArgs &a, cudaStream_t s) {
-    decode_kernel<IO, DK><<<a.B * a.H, NT, 0, s>>>(a);
-    return cudaGetLastError();
+    const int lw = (a.u == nullptr) ? 1 : a.L;
+    switch (lw) {
+        case 1: return launch_decode_l<IO, DK, 1>(a, s);
+        case 2: return launch_decode_l<IO, DK, 2>(a, s);
+        case 3: return launch_decode_l<IO, DK, 3>(a, s);
+        case 4: return launch_decode_l<IO, DK, 4>(a, s);
+        case 5: return launch_decode_l<IO, DK, 5>(a, s);
+        case 6: return launch_decode_l<IO, DK, 6>(a, s);
+        case 7: return launch_decode_l<IO, DK, 7>(a, s);
+        case 8: return launch_decode_l<IO, DK, 8>(a, s);
+    }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-// Entry used by the C ABI.  a.S_final is the in-place state.  Requires dv <= 128, L <= 8 and
-// dv a multiple of 32 (checked by the caller).
+// Entry used by the C ABI.  a.S_final is the in-place state.  Requires dv <= 128, dv a multiple
+// of 64 or dv = 32 (rows come in blocks of 8 per warp), L <= 8 (checked by the caller).
 cudaError_t launch_decode(const ScanArgs &a, bool io_f32, cudaStream_t s) {
     if (io_f32) {
         switch (a.dk) {

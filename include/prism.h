@@ -24,7 +24,8 @@
  *     library never allocates device or host memory and never synchronises the stream except in
  *     prism_query_device_status.
  *   - Layouts are dense row-major: activations [B,T,H,d]; u [B,T,H,L,dv]; w [B,T,H,L,dk];
- *     alpha, beta [B,T,H]; states [B,H,dv,dk].  Every pointer must be 16-byte aligned.
+ *     alpha, beta [B,T,H]; states [B,H,dv,dk].  alpha and beta must be 4-byte aligned, every
+ *     other pointer 16-byte aligned.
  *   - `stream` is a cudaStream_t passed as void* (NULL is the legacy default stream).  All work is
  *     enqueued on it asynchronously.
  *   - Arguments are validated before anything is launched; a rejected call enqueues nothing.

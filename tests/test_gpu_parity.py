@@ -56,6 +56,18 @@ def test_other_widths_and_ranks(dk, L, io):
     check_scan_full(make_inputs(wl, seed=dk + L), wl.chunk, io)
 
 
+@pytest.mark.parametrize("dk,T", [(64, 200), (128, 77)])
+def test_gdn_write_bf16_widths(dk, T):
+    wl = WORKLOADS["gdn"].with_(B=2, H=3, T=T, dk=dk, dv=dk)
+    check_scan_full(make_inputs(wl, seed=dk), wl.chunk, wl.io)
+
+
+@pytest.mark.parametrize("dk,L,T", [(128, 8, 130), (64, 1, 64), (128, 3, 1)])
+def test_rank_l_write_bf16(dk, L, T):
+    wl = WORKLOADS["long"].with_(H=2, T=T, dk=dk, dv=dk, L=L, chunk=64)
+    check_scan_full(make_inputs(wl, seed=L), wl.chunk, wl.io)
+
+
 def test_empty_sequence_copies_state():
     wl = WORKLOADS["long"].with_(H=2, T=1)
     x = make_inputs(wl)
