@@ -23,6 +23,7 @@ EXPORTS = (
     "prism_scan_fwd_workspace_size",
     "prism_scan_fwd_launch_count",
     "prism_scan_fwd",
+    "prism_scan_fwd_noalloc",
     "prism_step_decode",
     "prism_query_device_status",
     "prism_status_string",
@@ -62,6 +63,8 @@ def load_library():
     lib.prism_scan_fwd_launch_count.restype = ci
     lib.prism_scan_fwd.argtypes = [shp] + [vp] * 10 + [vp, sz, vp]
     lib.prism_scan_fwd.restype = ci
+    lib.prism_scan_fwd_noalloc.argtypes = [shp] + [vp] * 10 + [vp]
+    lib.prism_scan_fwd_noalloc.restype = ci
     lib.prism_step_decode.argtypes = [shp] + [vp] * 9 + [vp]
     lib.prism_step_decode.restype = ci
     lib.prism_query_device_status.argtypes = [vp, vp]
@@ -166,6 +169,34 @@ def prism_scan_fwd(q, k, v, alpha, beta, u=None, w=None, S0=None, *, chunk=64, o
                             _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
     if rc != PRISM_OK:
         raise PrismError(rc, "prism_scan_fwd")
+    return o, S_final
+
+
+def prism_scan_fwd_noalloc(q, k, v, alpha, beta, u=None, w=None, S0=None, *, chunk=64, o, S_final,
+                           stream=None):
+    """prism_scan_fwd without a workspace, for callers that cannot allocate device memory when
+    they run the scan: the library uses its own fixed device scratch instead.  The caller passes
+    every output (o, S_final or None) already allocated; this wrapper allocates nothing.  Calls
+    whose kernels overlap on the GPU share that scratch and race: keep them on one stream."""
+    lib = load_library()
+    if not isinstance(q, torch.Tensor) or not q.is_cuda:
+        raise TypeError("q must be a CUDA tensor (libprism has no CPU path)")
+    dev, io = q.device, q.dtype
+    shape = make_shape(q, v, u, chunk)
+    B, T, H, dk = q.shape
+    dv, L = shape.dv, shape.L
+    for name, x, dt, shp in (("q", q, io, (B, T, H, dk)), ("k", k, io, (B, T, H, dk)),
+                             ("v", v, io, (B, T, H, dv)), ("alpha", alpha, torch.float32, (B, T, H)),
+                             ("beta", beta, torch.float32, (B, T, H)),
+                             ("u", u, io, (B, T, H, L, dv)), ("w", w, io, (B, T, H, L, dk)),
+                             ("S0", S0, torch.float32, (B, H, dv, dk)), ("o", o, io, (B, T, H, dv)),
+                             ("S_final", S_final, torch.float32, (B, H, dv, dk))):
+        _check_tensor(name, x, dt, shp, dev)
+    rc = lib.prism_scan_fwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                    _ptr(beta), _ptr(u), _ptr(w), _ptr(S0), _ptr(o),
+                                    _ptr(S_final), _stream(stream))
+    if rc != PRISM_OK:
+        raise PrismError(rc, "prism_scan_fwd_noalloc")
     return o, S_final
 
 

@@ -112,6 +112,30 @@ prism_status prism_step_decode(const prism_shape *shape, const void *q, const vo
                                const void *u, const void *w, float *S, void *o, void *stream);
 
 /*
+ * prism_scan_fwd_noalloc -- prism_scan_fwd for callers that cannot allocate device memory when
+ * they run the scan (for example a plugin inside an engine that owns all device allocations, or
+ * a latency-critical path that cannot afford cudaMalloc's implicit synchronisation).  Same
+ * arguments and results as prism_scan_fwd, minus the workspace: the library uses its own
+ * scratch, a fixed PRISM_NOALLOC_SCRATCH_BYTES array in device global memory that every GPU which
+ * loads libprism.so holds until the process exits.  This call allocates nothing.
+ *   - Shapes whose workspace (prism_scan_fwd_workspace_size) exceeds PRISM_NOALLOC_SCRATCH_BYTES
+ *     are rejected with PRISM_ERR_UNSUPPORTED before anything is enqueued.
+ *   - The first call on each device looks up the scratch's device address (with that device
+ *     current) and caches it; make that first call before any stream capture.
+ *   - All calls on a device share the one scratch array, which keeps the last call's contents:
+ *     calls whose kernels overlap on the GPU (different streams, no ordering between them) race
+ *     on it.  Serialise them (one stream, or events).
+ *   - A kernel's bounded-wait failure is recorded in the scratch but not reported by this entry
+ *     point; callers that need that report use prism_scan_fwd with their own workspace.
+ * The method pages have no counterpart of this entry point; it exists for the callers above.
+ */
+#define PRISM_NOALLOC_SCRATCH_BYTES (16u << 20)
+prism_status prism_scan_fwd_noalloc(const prism_shape *shape, const void *q, const void *k,
+                                    const void *v, const float *alpha, const float *beta,
+                                    const void *u, const void *w, const float *S0, void *o,
+                                    float *S_final, void *stream);
+
+/*
  * prism_query_device_status -- synchronise `stream`, read the status word in `workspace`
  * (written by kernels whose bounded waits ran out) and clear it.  Returns PRISM_OK,
  * PRISM_ERR_TIMEOUT, or PRISM_ERR_CUDA if the stream itself reports an error.
