@@ -11,6 +11,8 @@ cudaError_t launch_scan_simt(const ScanArgs &a, bool io_f32, cudaStream_t s);
 cudaError_t launch_decode(const ScanArgs &a, bool io_f32, cudaStream_t s);
 bool scan_tc_supported(const ScanArgs &a, bool io_f32);
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
+size_t gdn_workspace_bytes(int B, int H, int T, int dk);
+cudaError_t launch_scan_gdn(const ScanArgs &a, void *ws, cudaStream_t s);
 }  // namespace prism
 
 namespace {
@@ -44,6 +46,15 @@ prism_status check_common(const prism_shape *s, const void *q, const void *k, co
     return PRISM_OK;
 }
 
+// Which kernels a prism_scan_fwd call with this shape runs.
+enum class Plan { Simt, TcFused, TcGdnSplit };
+
+Plan plan_for(const prism_shape *s, bool gdn_write) {
+    const bool tc = s->io == PRISM_BF16 && s->dk == s->dv && (s->dk == 64 || s->dk == 128);
+    if (!tc) return Plan::Simt;
+    return gdn_write ? Plan::TcGdnSplit : Plan::TcFused;
+}
+
 prism::ScanArgs make_args(const prism_shape *s, const void *q, const void *k, const void *v,
                           const float *alpha, const float *beta, const void *u, const void *w,
                           const float *S0, void *o, float *S_final, uint32_t *status) {
@@ -59,15 +70,22 @@ prism::ScanArgs make_args(const prism_shape *s, const void *q, const void *k, co
 
 extern "C" {
 
+// The workspace and launch count cover the larger of the two write forms (Gated-DeltaNet write
+// when u, w are NULL, rank-L otherwise), since the shape alone does not say which one is used.
 prism_status prism_scan_fwd_workspace_size(const prism_shape *shape, size_t *bytes) {
     if (!shape || !bytes) return PRISM_ERR_INVALID_ARG;
-    *bytes = prism::kStatusBytes;
+    size_t need = prism::kStatusBytes;
+    if (shape->B > 0 && shape->H > 0 && shape->T > 0 && shape->L == 1 &&
+        plan_for(shape, true) == Plan::TcGdnSplit)
+        need = prism::gdn_workspace_bytes(shape->B, shape->H, shape->T, shape->dk);
+    *bytes = need;
     return PRISM_OK;
 }
 
 prism_status prism_scan_fwd_launch_count(const prism_shape *shape, int *launches) {
     if (!shape || !launches) return PRISM_ERR_INVALID_ARG;
     int n = 1;
+    if (shape->L == 1 && plan_for(shape, true) == Plan::TcGdnSplit && shape->T > 0) n = 2;
     if (shape->B == 0 || shape->H == 0) n = 0;
     *launches = n;
     return PRISM_OK;
@@ -95,8 +113,15 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
 
     prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, S0, o, S_final, status);
     const bool io_f32 = shape->io == PRISM_F32;
-    cudaError_t err = prism::scan_tc_supported(a, io_f32) ? prism::launch_scan_tc(a, s)
-                                                          : prism::launch_scan_simt(a, io_f32, s);
+    cudaError_t err;
+    switch (plan_for(shape, u == nullptr)) {
+        case Plan::TcGdnSplit:
+            err = shape->T > 0 ? prism::launch_scan_gdn(a, workspace, s)
+                               : prism::launch_scan_tc(a, s);  // T = 0: copies S0 to S_final
+            break;
+        case Plan::TcFused: err = prism::launch_scan_tc(a, s); break;
+        default: err = prism::launch_scan_simt(a, io_f32, s); break;
+    }
     return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 

@@ -25,16 +25,12 @@
 // shared-memory operands in the canonical 128B/64B-swizzled layouts; accumulators are read back
 // with tcgen05.ld.  Waits on MMA completion are bounded and record PRISM_ERR_TIMEOUT.
 
-#include "tc.cuh"
+#include "chunk_common.cuh"
 
 namespace prism {
 namespace {
 
-using namespace tc;
-
-constexpr int C = 64;         // chunk length of the tensor-core path
 constexpr int NT = 128;       // 4 warps: TMEM lanes 0-127
-constexpr int AS = C + 1;     // padded fp32 row stride of the solve matrices
 constexpr uint32_t TMEM_COLS = 512;
 
 // Operands that are rounded intermediate results (Mqk, T, Y, S and, for the rank-L write, P, Mqw,
@@ -92,158 +88,6 @@ struct TcLayout {
     static constexpr uint32_t cDS = cQS + BV;    // F_w + K^T D Y               (BV)
     static_assert(cDS + BV <= TMEM_COLS, "TMEM budget");
 };
-
-__device__ __forceinline__ void st16(uint8_t *base, uint32_t off, uint4 v) {
-    *reinterpret_cast<uint4 *>(base + off) = v;
-}
-
-template <int BV>
-__device__ __forceinline__ uint32_t vt_off(int row, int col) {
-    // x BV tile: 64B swizzle when BV = 32, 128B when BV = 64
-    if constexpr (BV == 32) return sw64_off(row, col);
-    else return sw128_off(row, col, 0);
-}
-
-template <int BV>
-__device__ __forceinline__ uint64_t desc_vt(uint32_t base, int ks) {
-    if constexpr (BV == 32) return desc_mn_sw64(base, ks);
-    else return desc_mn_sw128(base, ks, C * 128);  // a single MN block; LBO unused
-}
-
-// hi / lo bf16 pair of 8 floats
-__device__ __forceinline__ void split8(const float *x, uint4 &hi, uint4 &lo) {
-    uint32_t h[4], l[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-        float2 hf = __bfloat1622float2(hh);
-        __nv_bfloat162 ll = __floats2bfloat162_rn(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
-        h[i] = *reinterpret_cast<uint32_t *>(&hh);
-        l[i] = *reinterpret_cast<uint32_t *>(&ll);
-    }
-    hi = make_uint4(h[0], h[1], h[2], h[3]);
-    lo = make_uint4(l[0], l[1], l[2], l[3]);
-}
-
-// A row of BV fp32 values as a hi / lo pair into two x BV tiles.
-template <int BV>
-__device__ __forceinline__ void store_row_split(uint8_t *hi, uint8_t *lo, int row, const float *x) {
-#pragma unroll
-    for (int c8 = 0; c8 < BV / 8; ++c8) {
-        uint4 h, l;
-        split8(x + c8 * 8, h, l);
-        const uint32_t off = vt_off<BV>(row, c8 * 8);
-        st16(hi, off, h);
-        st16(lo, off, l);
-    }
-}
-
-// 32 fp32 values at (row, col .. col+31) of K-major SW128 tiles, as a hi / lo pair or hi only.
-__device__ __forceinline__ void store32_split(uint8_t *hi, uint8_t *lo, int row, int col,
-                                              const float *x, uint32_t block_bytes = 0) {
-#pragma unroll
-    for (int c8 = 0; c8 < 4; ++c8) {
-        uint4 h, l;
-        split8(x + c8 * 8, h, l);
-        const uint32_t off = sw128_off(row, col + c8 * 8, block_bytes);
-        st16(hi, off, h);
-        if (lo) st16(lo, off, l);
-    }
-}
-
-// BV consecutive TMEM columns of this thread's lane (warp-collective).
-template <int BV>
-__device__ __forceinline__ void ld_row(uint32_t tbase, int warp, uint32_t col, float *x) {
-#pragma unroll
-    for (int c = 0; c < BV; c += 32) {
-        float v[32];
-        tmem_ld32(taddr(tbase, 32 * warp, col + c), v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[c + j] = v[j];
-    }
-}
-
-// Shared-memory writes become visible to the tensor core and earlier tcgen05.ld complete before
-// the issuing thread proceeds.
-__device__ __forceinline__ void sync_for_mma() {
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-}
-
-// D (+)= (A_hi + A_lo)(B_hi + B_lo) without the lo*lo term; K = 16 * nks.  Pass alo / blo = 0 to
-// skip a split.  `acc` says whether the first product accumulates onto D.
-template <class FA, class FB>
-__device__ __forceinline__ void mma_split(uint32_t d, uint32_t idesc, int nks, FA adesc, FB bdesc,
-                                          uint32_t ahi, uint32_t alo, uint32_t bhi, uint32_t blo,
-                                          bool acc) {
-    for (int ks = 0; ks < nks; ++ks) mma_bf16(d, adesc(ahi, ks), bdesc(bhi, ks), idesc, acc || ks > 0);
-    if (blo)
-        for (int ks = 0; ks < nks; ++ks) mma_bf16(d, adesc(ahi, ks), bdesc(blo, ks), idesc, 1);
-    if (alo)
-        for (int ks = 0; ks < nks; ++ks) mma_bf16(d, adesc(alo, ks), bdesc(bhi, ks), idesc, 1);
-}
-
-// T = (I + A)^{-1} for strictly lower-triangular A (C = 64), blocked: 16 x 16 diagonal blocks by
-// forward substitution, then two doubling levels T_21 = -T_22 A_21 T_11.
-__device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid) {
-    const int warp = tid >> 5, lane = tid & 31;
-    // diagonal blocks: warp w inverts block w, lane j < 16 computes column j
-    if (lane < 16) {
-        const int o = 16 * warp, j = lane;
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float s = (i == j) ? 1.f : 0.f;
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                if (k < i) s = fmaf(-A[(o + i) * AS + o + k], x[k], s);
-            x[i] = (i < j) ? 0.f : s;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) Tm[(o + i) * AS + o + j] = x[i];
-    }
-    // zero the strictly-upper blocks
-    for (int e = tid; e < C * C; e += NT) {
-        int r = e / C, c = e % C;
-        if ((c >> 4) > (r >> 4)) Tm[r * AS + c] = 0.f;
-    }
-    __syncthreads();
-    // level 1: pairs of 16-blocks (p = 0, 1): rows 32p+16.., cols 32p..
-    for (int e = tid; e < 2 * 256; e += NT) {
-        int p = e >> 8, r = (e >> 4) & 15, c = e & 15;
-        const int r0 = 32 * p + 16, c0 = 32 * p;
-        float s = 0.f;
-        for (int k = c; k < 16; ++k) s = fmaf(A[(r0 + r) * AS + c0 + k], Tm[(c0 + k) * AS + c0 + c], s);
-        tmp[p * 16 * 17 + r * 17 + c] = s;  // M1 = A_21 T_11
-    }
-    __syncthreads();
-    for (int e = tid; e < 2 * 256; e += NT) {
-        int p = e >> 8, r = (e >> 4) & 15, c = e & 15;
-        const int r0 = 32 * p + 16, c0 = 32 * p;
-        float s = 0.f;
-        for (int k = 0; k <= r; ++k) s = fmaf(Tm[(r0 + r) * AS + r0 + k], tmp[p * 16 * 17 + k * 17 + c], s);
-        Tm[(r0 + r) * AS + c0 + c] = -s;
-    }
-    __syncthreads();
-    // level 2: 32-blocks: rows 32.., cols 0..31
-    for (int e = tid; e < 32 * 32; e += NT) {
-        int r = e >> 5, c = e & 31;
-        float s = 0.f;
-        for (int k = c; k < 32; ++k) s = fmaf(A[(32 + r) * AS + k], Tm[k * AS + c], s);
-        tmp[r * 33 + c] = s;
-    }
-    __syncthreads();
-    for (int e = tid; e < 32 * 32; e += NT) {
-        int r = e >> 5, c = e & 31;
-        float s = 0.f;
-        for (int k = 0; k <= r; ++k) s = fmaf(Tm[(32 + r) * AS + 32 + k], tmp[k * 33 + c], s);
-        Tm[(32 + r) * AS + c] = -s;
-    }
-    __syncthreads();
-}
 
 template <int DK, int BV, bool GDN>
 __global__ void __launch_bounds__(NT, 1) scan_tc_kernel(ScanArgs p) {
@@ -394,7 +238,7 @@ __global__ void __launch_bounds__(NT, 1) scan_tc_kernel(ScanArgs p) {
         __syncthreads();
 
         // ---- T = (I + A)^{-1}; bf16 pairs of T diag(beta gamma) and T diag(beta) (GDN) or T
-        solve_unit_lower(sA, sT, sTmp, tid);
+        solve_unit_lower<NT>(sA, sT, sTmp, tid);
         for (int e = tid; e < C * (C / 8); e += NT) {
             const int t = e / (C / 8), c8 = e % (C / 8);
             float a1[8], a2[8];
