@@ -106,11 +106,13 @@ __device__ __forceinline__ void mma_split(uint32_t d, uint32_t idesc, int nks, F
         for (int ks = 0; ks < nks; ++ks) mma_bf16(d, adesc(alo, ks), bdesc(bhi, ks), idesc, 1);
 }
 
-// T = (I + A)^{-1} for strictly lower-triangular A (C = 64), blocked: 16 x 16 diagonal blocks by
-// forward substitution, then two doubling levels T_21 = -T_22 A_21 T_11.
-// Safe in place (A == Tm): every block is read as A before it is overwritten with T.
+// T = (I + A)^{-1} for strictly lower-triangular A (C = 64), blocked: the four 16 x 16 diagonal
+// blocks by forward substitution, then two doubling levels T_21 = -T_22 A_21 T_11 (16 -> 32 -> 64)
+// as register-blocked products with fixed trip counts.  Safe in place (A == Tm): every block is
+// read as A before it is overwritten with T.  Needs NTH == 128 threads; tmp holds 32 x 33 floats.
 template <int NTH>
 __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid) {
+    static_assert(NTH == 128, "the solve is laid out for 128 threads");
     const int warp = tid >> 5, lane = tid & 31;
     // diagonal blocks: warp w inverts block w, lane j < 16 computes column j
     if (lane < 16) {
@@ -120,50 +122,65 @@ __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid)
         for (int i = 0; i < 16; ++i) {
             float s = (i == j) ? 1.f : 0.f;
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
-                if (k < i) s = fmaf(-A[(o + i) * AS + o + k], x[k], s);
+            for (int k = 0; k < i; ++k) s = fmaf(-A[(o + i) * AS + o + k], x[k], s);
             x[i] = (i < j) ? 0.f : s;
         }
         __syncwarp(0x0000ffffu);  // every lane has read the block before any lane overwrites it
 #pragma unroll
         for (int i = 0; i < 16; ++i) Tm[(o + i) * AS + o + j] = x[i];
     }
-    // zero the strictly-upper blocks
-    for (int e = tid; e < C * C; e += NTH) {
-        int r = e / C, c = e % C;
-        if ((c >> 4) > (r >> 4)) Tm[r * AS + c] = 0.f;
+    __syncthreads();
+    // level 1, 16-blocks, pairs p = 0, 1: rows r0 = 32p + 16, cols c0 = 32p; thread: 1 row x 4 cols
+    {
+        const int pp = tid >> 6, r = (tid >> 2) & 15, cq = (tid & 3) * 4;
+        const int r0 = 32 * pp + 16, c0 = 32 * pp;
+        float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = A[(r0 + r) * AS + c0 + k];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) m[j] = fmaf(a, Tm[(c0 + k) * AS + c0 + cq + j], m[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tmp[pp * 16 * 17 + r * 17 + cq + j] = m[j];
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m[j] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float t = Tm[(r0 + r) * AS + r0 + k];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) m[j] = fmaf(t, tmp[pp * 16 * 17 + k * 17 + cq + j], m[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) Tm[(r0 + r) * AS + c0 + cq + j] = -m[j];
     }
     __syncthreads();
-    // level 1: pairs of 16-blocks (p = 0, 1): rows 32p+16.., cols 32p..
-    for (int e = tid; e < 2 * 256; e += NTH) {
-        int p = e >> 8, r = (e >> 4) & 15, c = e & 15;
-        const int r0 = 32 * p + 16, c0 = 32 * p;
-        float s = 0.f;
-        for (int k = c; k < 16; ++k) s = fmaf(A[(r0 + r) * AS + c0 + k], Tm[(c0 + k) * AS + c0 + c], s);
-        tmp[p * 16 * 17 + r * 17 + c] = s;  // M1 = A_21 T_11
-    }
-    __syncthreads();
-    for (int e = tid; e < 2 * 256; e += NTH) {
-        int p = e >> 8, r = (e >> 4) & 15, c = e & 15;
-        const int r0 = 32 * p + 16, c0 = 32 * p;
-        float s = 0.f;
-        for (int k = 0; k <= r; ++k) s = fmaf(Tm[(r0 + r) * AS + r0 + k], tmp[p * 16 * 17 + k * 17 + c], s);
-        Tm[(r0 + r) * AS + c0 + c] = -s;
-    }
-    __syncthreads();
-    // level 2: 32-blocks: rows 32.., cols 0..31
-    for (int e = tid; e < 32 * 32; e += NTH) {
-        int r = e >> 5, c = e & 31;
-        float s = 0.f;
-        for (int k = c; k < 32; ++k) s = fmaf(A[(32 + r) * AS + k], Tm[k * AS + c], s);
-        tmp[r * 33 + c] = s;
-    }
-    __syncthreads();
-    for (int e = tid; e < 32 * 32; e += NTH) {
-        int r = e >> 5, c = e & 31;
-        float s = 0.f;
-        for (int k = 0; k <= r; ++k) s = fmaf(Tm[(32 + r) * AS + 32 + k], tmp[k * 33 + c], s);
-        Tm[(32 + r) * AS + c] = -s;
+    // level 2, 32-blocks: rows 32.., cols 0..31; thread: 1 row x 8 cols
+    {
+        const int r = tid >> 2, cq = (tid & 3) * 8;
+        float m[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m[j] = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float a = A[(32 + r) * AS + k];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) m[j] = fmaf(a, Tm[k * AS + cq + j], m[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) tmp[r * 33 + cq + j] = m[j];
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m[j] = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float t = Tm[(32 + r) * AS + 32 + k];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) m[j] = fmaf(t, tmp[k * 33 + cq + j], m[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) Tm[(32 + r) * AS + cq + j] = -m[j];
     }
     __syncthreads();
 }

@@ -147,13 +147,13 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, uint8_t *ws, i
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int i = cc + j;
-                    sA[t * AS + i] = (i < t) ? bt * expf(gt - sG[i]) * gr[j] : 0.f;
+                    sA[t * AS + i] = (i < t) ? bt * __expf(gt - sG[i]) * gr[j] : 0.f;
                 }
             } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int i = cc + j;
-                    gr[j] = (i <= t) ? expf(gt - sG[i]) * gr[j] : 0.f;
+                    gr[j] = (i <= t) ? __expf(gt - sG[i]) * gr[j] : 0.f;
                 }
                 store32_split(rec + RC::MQK, rec + RC::MQKL, t, cc, gr);
             }
@@ -218,40 +218,89 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, uint8_t *ws, i
 
 // ------------------------------------------------------------------------------------------------
 // state: one CTA per (value slice, head, batch), chunks in order
+//
+// Two MMA rounds per chunk, shaped to keep the tcgen05 instruction count low:
+//   round 1:  D1  = [Q; Wk] [S_hi | S_lo]                  (M = 128, N = 2 BV: QS and X_s, hi and lo
+//                                                           halves side by side)
+//             D1[:, :BV] -= [0; T2_hi] V + [0; T2_lo] V    (U lands in the X_s rows; zero tile on top)
+//   round 2:  D3  = [Mqk_hi; 0] [Y_hi | Y_lo] ;  D3[:, :BV] += [Mqk_lo; 0] Y_hi
+//             D4  = K^T [DY_hi | DY_lo]
+// so that every operand row t of the chunk sits in TMEM lane t (QS, O) or lane 64 + t (X_s - U).
+// The per-chunk records (Wk, T2, Mqk, g) arrive by TMA bulk copies; K, Q and V by cp.async.
 
 template <int DK, int BV>
 struct StateLayout {
     static constexpr uint32_t KQW_BLK = 3 * C * 128;      // [K; Q; Wk] rows of one 64-col block
     static constexpr uint32_t ROWB = (BV == 32) ? 64 : 128;
-    static constexpr uint32_t VT = C * ROWB;
-    // one buffer of chunk inputs
+    static constexpr uint32_t VT = C * ROWB;              // C x BV tile (V slice)
+    static constexpr int N2 = 2 * BV;                     // hi | lo side by side
+    // double-buffered chunk inputs
     static constexpr uint32_t B_KQW = 0;
     static constexpr uint32_t B_V = B_KQW + KQW_BLK * (DK / 64);
-    static constexpr uint32_t B_T2 = B_V + VT;             // T diag(beta) hi, lo (contiguous)
-    static constexpr uint32_t B_T2L = B_T2 + C * 128;
-    static constexpr uint32_t B_MQK = B_T2L + C * 128;     // Mqk hi, lo
-    static constexpr uint32_t B_MQKL = B_MQK + C * 128;
-    static constexpr uint32_t B_G = B_MQKL + C * 128;      // g (64 floats)
+    static constexpr uint32_t B_G = B_V + VT;               // g (64 floats)
     static constexpr uint32_t BUF = B_G + 1024;
-    // state-only tiles
-    static constexpr uint32_t S = 2 * BUF;
-    static constexpr uint32_t SL = S + DK * ROWB;
-    static constexpr uint32_t Y = SL + DK * ROWB;
-    static constexpr uint32_t YL = Y + VT;
-    static constexpr uint32_t DY = YL + VT;
-    static constexpr uint32_t DYL = DY + VT;
-    static constexpr uint32_t GATES = DYL + VT;             // gamma, D: 2 x C floats
+    // single-buffered operands: [Mqk_hi][0][T2_hi][Mqk_lo][0][T2_lo]
+    static constexpr uint32_t MH = 2 * BUF;
+    static constexpr uint32_t Z1 = MH + C * 128;
+    static constexpr uint32_t T2H = Z1 + C * 128;
+    static constexpr uint32_t ML = T2H + C * 128;
+    static constexpr uint32_t Z2 = ML + C * 128;
+    static constexpr uint32_t T2L = Z2 + C * 128;
+    // S^T [d][hi | lo], Y [t][hi | lo], D Y [t][hi | lo]: MN-major, 64-column blocks
+    static constexpr uint32_t S_BLK = DK * 128;
+    static constexpr uint32_t S = T2L + C * 128;
+    static constexpr uint32_t Y_BLK = C * 128;
+    static constexpr uint32_t Y = S + S_BLK * (N2 / 64);
+    static constexpr uint32_t DY = Y + Y_BLK * (N2 / 64);
+    static constexpr uint32_t GATES = DY + Y_BLK * (N2 / 64);  // gamma, D: 2 x C floats
     static constexpr uint32_t BYTES = GATES + 2 * C * 4 + 1024;
     // TMEM columns
-    static constexpr uint32_t cU = 0, cXs = BV, cQS = 2 * BV, cO = 3 * BV, cDS = 4 * BV;
-    static constexpr uint32_t TCOLS = (5 * BV <= 128) ? 128 : (5 * BV <= 256 ? 256 : 512);
+    static constexpr uint32_t cD1 = 0, cD3 = N2, cD4 = 2 * N2;
+    static constexpr uint32_t TCOLS = (3 * N2 <= 128) ? 128 : (3 * N2 <= 256 ? 256 : 512);
 };
 
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// An N2-wide row of fp32 (hi | lo of one value each) stored as bf16 into an MN-major tile of
+// 64-column 128B-swizzled blocks: cols [0, BV) get bf16(x), cols [BV, 2BV) get bf16(x - hi).
+template <int BV>
+__device__ __forceinline__ void store_row_pair(uint8_t *tile, uint32_t blk_bytes, int row,
+                                               const float *x) {
+#pragma unroll
+    for (int c8 = 0; c8 < BV / 8; ++c8) {
+        uint4 h, l;
+        split8(x + c8 * 8, h, l);
+        st16(tile, sw128_off(row, c8 * 8, blk_bytes), h);
+        st16(tile, sw128_off(row, BV + c8 * 8, blk_bytes), l);
+    }
+}
+
+// out[j] = D[lane row][col + j] + D[lane row][col + BV + j]: the hi and lo halves of a pair MMA.
+template <int BV>
+__device__ __forceinline__ void ld_pair_sum(uint32_t tbase, int warp, uint32_t col, float *out) {
+#pragma unroll
+    for (int c = 0; c < BV; c += 32) {
+        float a[32], b[32];
+        tmem_ld32(taddr(tbase, 32 * warp, col + c), a);
+        tmem_ld32(taddr(tbase, 32 * warp, col + BV + c), b);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) out[c + j] = a[j] + b[j];
+    }
+}
+
 template <int DK, int BV>
-__device__ __forceinline__ void state_issue_loads(const ScanArgs &p, const uint8_t *ws, int nch,
-                                                  int c, uint8_t *buf, int tid) {
+__device__ __forceinline__ void state_issue_cp(const ScanArgs &p, int c, uint8_t *buf, int tid) {
     using LY = StateLayout<DK, BV>;
-    using RC = GdnRec<DK>;
     const int v0 = blockIdx.x * BV, h = blockIdx.y, b = blockIdx.z;
     const int H = p.H, T = p.T, dv = p.dv;
     const int c0 = c * C, n = min(C, T - c0);
@@ -270,25 +319,21 @@ __device__ __forceinline__ void state_issue_loads(const ScanArgs &p, const uint8
         const size_t g = ok ? ((((size_t)b * T + c0 + t) * H + h) * dv + v0 + ch * 8) : 0;
         cp_async16(buf + LY::B_V + vt_off<BV>(t, ch * 8), v + g, ok ? 16 : 0);
     }
-    const uint8_t *rec = ws + kRecOffset + (((size_t)b * H + h) * nch + c) * RC::BYTES;
-    // Wk image: 64-column blocks land in rows 2C..3C of the stacked tile (swizzle preserved:
-    // both bases are 1024-aligned and 2C is a multiple of 8)
-    for (int e = tid; e < (DK / 64) * (RC::WK_BLK / 16); e += NT) {
-        const int blk = e / (RC::WK_BLK / 16), off = (e % (RC::WK_BLK / 16)) * 16;
-        cp_async16(buf + LY::B_KQW + blk * LY::KQW_BLK + 2 * C * 128 + off,
-                   rec + RC::WK + blk * RC::WK_BLK + off, 16);
-    }
-    // T diag(beta) pair, Mqk pair, g: contiguous in the record and in the buffer
-    for (int e = tid; e < (4 * C * 128 + C * 4) / 16; e += NT)
-        cp_async16(buf + LY::B_T2 + e * 16, rec + RC::T2 + e * 16, 16);
+}
+
+template <int DK>
+__device__ __forceinline__ const uint8_t *record(const ScanArgs &p, const uint8_t *ws, int nch, int c) {
+    return ws + kRecOffset + (((size_t)blockIdx.z * p.H + blockIdx.y) * nch + c) * GdnRec<DK>::BYTES;
 }
 
 template <int DK, int BV>
 __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint8_t *ws, int nch) {
     using LY = StateLayout<DK, BV>;
+    using RC = GdnRec<DK>;
+    constexpr int N2 = LY::N2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t mma_bar;
+    __shared__ uint64_t mma_bar, wk_bar[2], t2_bar, mq_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int failed_sh;
 
@@ -301,34 +346,80 @@ __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint
     float *sD = sGam + C;
     const uint32_t sb = smem_u32(sm);
 
-    if (nch > 0) state_issue_loads<DK, BV>(p, ws, nch, 0, sm, tid);
-    cp_async_commit();
+    // bulk loads of a chunk record: Wk + g into the chunk buffer; T2 and Mqk into the shared tiles
+    auto load_wk = [&](int c) {
+        const uint8_t *rec = record<DK>(p, ws, nch, c);
+        uint8_t *buf = sm + (c & 1) * LY::BUF;
+        uint64_t *bar = &wk_bar[c & 1];
+        mbar_expect_tx(bar, (DK / 64) * RC::WK_BLK + C * 4);
+        for (int blk = 0; blk < DK / 64; ++blk)
+            bulk_g2s(buf + LY::B_KQW + blk * LY::KQW_BLK + 2 * C * 128, rec + RC::WK + blk * RC::WK_BLK,
+                     RC::WK_BLK, bar);
+        bulk_g2s(buf + LY::B_G, rec + RC::G, C * 4, bar);
+    };
+    auto load_t2 = [&](int c) {
+        const uint8_t *rec = record<DK>(p, ws, nch, c);
+        mbar_expect_tx(&t2_bar, 2 * C * 128);
+        bulk_g2s(sm + LY::T2H, rec + RC::T2, C * 128, &t2_bar);
+        bulk_g2s(sm + LY::T2L, rec + RC::T2L, C * 128, &t2_bar);
+    };
+    auto load_mq = [&](int c) {
+        const uint8_t *rec = record<DK>(p, ws, nch, c);
+        mbar_expect_tx(&mq_bar, 2 * C * 128);
+        bulk_g2s(sm + LY::MH, rec + RC::MQK, C * 128, &mq_bar);
+        bulk_g2s(sm + LY::ML, rec + RC::MQKL, C * 128, &mq_bar);
+    };
+
     if (warp == 0) tmem_alloc(&tmem_base_sh, LY::TCOLS);
     if (tid == 0) {
         mbar_init(&mma_bar, 1);
+        mbar_init(&wk_bar[0], 1);
+        mbar_init(&wk_bar[1], 1);
+        mbar_init(&t2_bar, 1);
+        mbar_init(&mq_bar, 1);
         mbar_fence_init();
         failed_sh = 0;
+    }
+    // zero tiles under Mqk and over T2 (never overwritten)
+    for (int e = tid; e < C * 128 / 16; e += NT) {
+        st16(sm + LY::Z1, e * 16, make_uint4(0, 0, 0, 0));
+        st16(sm + LY::Z2, e * 16, make_uint4(0, 0, 0, 0));
     }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
+    if (nch > 0) {
+        state_issue_cp<DK, BV>(p, 0, sm, tid);
+        if (tid == 0) {
+            load_wk(0);
+            load_t2(0);
+            load_mq(0);
+        }
+    }
+    cp_async_commit();
     const uint32_t tb = tmem_base_sh;
     uint32_t phase = 0;
-    auto mma_done = [&]() -> bool {
-        if (tid == 0) mma_commit(&mma_bar);
-        __syncwarp();
-        const bool ok = mbar_wait(&mma_bar, phase & 1, p.status);
-        phase++;
+    auto fail_sync = [&](bool ok) -> bool {  // make one thread's timeout everyone's
         if (!ok) failed_sh = 1;
         fence_after_sync();
         __syncthreads();
         return failed_sh == 0;
     };
-    auto dK = [](uint32_t base, int ks) { return desc_k_sw128(base, ks, 0); };
+    auto mma_done = [&]() -> bool {
+        if (tid == 0) mma_commit(&mma_bar);
+        __syncwarp();
+        const bool ok = mbar_wait(&mma_bar, phase & 1, p.status);
+        phase++;
+        return fail_sync(ok);
+    };
     auto dKQW = [](uint32_t base, int ks) { return desc_k_sw128(base, ks, LY::KQW_BLK); };
     auto dKmn = [](uint32_t base, int ks) { return desc_mn_sw128(base, ks, LY::KQW_BLK); };
+    auto dK = [](uint32_t base, int ks) { return desc_k_sw128(base, ks, 0); };
     auto dVT = [](uint32_t base, int ks) { return desc_vt<BV>(base, ks); };
+    auto dS2 = [](uint32_t base, int ks) { return desc_mn_sw128(base, ks, LY::S_BLK); };
+    auto dY2 = [](uint32_t base, int ks) { return desc_mn_sw128(base, ks, LY::Y_BLK); };
 
+    // fp32 state S^T: DK = 128 -> d = tid (M = 128); DK = 64 -> M = 64 layout (warp d/16, lane d%16)
     const bool own_d = (DK == 128) ? true : (lane < 16);
     const int d_row = (DK == 128) ? tid : (16 * warp + lane);
     float Sreg[BV];
@@ -338,72 +429,82 @@ __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint
 #pragma unroll
         for (int j = 0; j < BV; ++j) Sreg[j] = p.S0[(head * dv + v0 + j) * DK + d_row];
     }
-    if (own_d) store_row_split<BV>(sm + LY::S, sm + LY::SL, d_row, Sreg);
-    const bool own_t = lane < 16;
-    const int t_row = 16 * warp + lane;
+    if (own_d) store_row_pair<BV>(sm + LY::S, LY::S_BLK, d_row, Sreg);
 
     for (int c = 0; c < nch; ++c) {
         const int c0 = c * C, n = min(C, T - c0);
-        uint8_t *buf = sm + (c & 1) * LY::BUF;
         const uint32_t bb = sb + (c & 1) * LY::BUF;
-        if (c + 1 < nch) state_issue_loads<DK, BV>(p, ws, nch, c + 1, sm + ((c + 1) & 1) * LY::BUF, tid);
+        const uint8_t *buf = sm + (c & 1) * LY::BUF;
+        if (c + 1 < nch) {
+            state_issue_cp<DK, BV>(p, c + 1, sm + ((c + 1) & 1) * LY::BUF, tid);
+            if (tid == 0) load_wk(c + 1);
+        }
         cp_async_commit();
-        cp_async_wait<1>();  // this chunk's group has landed; the next chunk's stays in flight
+        cp_async_wait<1>();
+        bool ok = mbar_wait(&wk_bar[c & 1], (c >> 1) & 1, p.status);
+        ok = mbar_wait(&t2_bar, c & 1, p.status) && ok;
+        if (!fail_sync(ok)) break;
         const float *g = reinterpret_cast<const float *>(buf + LY::B_G);
-        __syncthreads();
         const float g_last = g[C - 1];
         if (tid < C) {
-            sGam[tid] = expf(g[tid]);
-            sD[tid] = tid < n ? expf(g_last - g[tid]) : 0.f;
+            sGam[tid] = __expf(g[tid]);
+            sD[tid] = tid < n ? __expf(g_last - g[tid]) : 0.f;
         }
         sync_for_mma();
 
-        // U = T diag(beta) V ;  X_s = Wk S^T ;  QS = Q S^T
+        // round 1
         if (tid == 0) {
-            const uint32_t id = idesc_bf16(64, BV, 0, 1);
-            mma_split(tb + LY::cU, id, C / 16, dK, dVT, bb + LY::B_T2, bb + LY::B_T2L, bb + LY::B_V, 0, false);
-            mma_split(tb + LY::cXs, id, DK / 16, dKQW, dVT, bb + LY::B_KQW + 2 * C * 128, 0,
-                      sb + LY::S, sb + LY::SL, false);
-            mma_split(tb + LY::cQS, id, DK / 16, dKQW, dVT, bb + LY::B_KQW + C * 128, 0,
-                      sb + LY::S, sb + LY::SL, false);
+            mma_split(tb + LY::cD1, idesc_bf16(128, N2, 0, 1), DK / 16, dKQW, dS2,
+                      bb + LY::B_KQW + C * 128, 0, sb + LY::S, 0, false);
+            const uint32_t idn = idesc_bf16(128, BV, 0, 1) | (1u << 13);  // negate A
+            mma_split(tb + LY::cD1, idn, C / 16, dK, dVT, sb + LY::Z1, sb + LY::Z2, bb + LY::B_V, 0,
+                      true);
         }
         if (!mma_done()) break;
+        if (tid == 0 && c + 1 < nch) load_t2(c + 1);  // the T2 tiles are free again
+        float qs[BV];  // rows 0..63 (warps 0-1): QS;  rows 64..127 (warps 2-3): X_s - U = -Y
+        ld_pair_sum<BV>(tb, warp, LY::cD1, qs);
         {
-            float xs[BV], uu[BV];
-            ld_row<BV>(tb, warp, LY::cXs, xs);
-            ld_row<BV>(tb, warp, LY::cU, uu);
-            if (own_t) {
+            if (warp >= 2) {
+                const int t = tid - 64;
                 float y[BV];
-                const float dd = sD[t_row];
 #pragma unroll
-                for (int j = 0; j < BV; ++j) y[j] = uu[j] - xs[j];
-                store_row_split<BV>(sm + LY::Y, sm + LY::YL, t_row, y);
+                for (int j = 0; j < BV; ++j) y[j] = -qs[j];
+                store_row_pair<BV>(sm + LY::Y, LY::Y_BLK, t, y);
+                const float dd = sD[t];
 #pragma unroll
                 for (int j = 0; j < BV; ++j) y[j] *= dd;
-                store_row_split<BV>(sm + LY::DY, sm + LY::DYL, t_row, y);
+                store_row_pair<BV>(sm + LY::DY, LY::Y_BLK, t, y);
             }
         }
+        ok = mbar_wait(&mq_bar, c & 1, p.status);
+        if (!fail_sync(ok)) break;
         sync_for_mma();
-        // O = Mqk Y ;  S'^T contribution K^T D Y
+
+        // round 2
         if (tid == 0) {
-            mma_split(tb + LY::cO, idesc_bf16(64, BV, 0, 1), C / 16, dK, dVT, bb + LY::B_MQK,
-                      bb + LY::B_MQKL, sb + LY::Y, sb + LY::YL, false);
-            mma_split(tb + LY::cDS, idesc_bf16(DK, BV, 1, 1), C / 16, dKmn, dVT, bb + LY::B_KQW, 0,
-                      sb + LY::DY, sb + LY::DYL, false);
+            mma_split(tb + LY::cD3, idesc_bf16(128, N2, 0, 1), C / 16, dK, dY2, sb + LY::MH, 0,
+                      sb + LY::Y, 0, false);
+            mma_split(tb + LY::cD3, idesc_bf16(128, BV, 0, 1), C / 16, dK, dY2, sb + LY::ML, 0,
+                      sb + LY::Y, 0, true);
+            mma_split(tb + LY::cD4, idesc_bf16(DK, N2, 1, 1), C / 16, dKmn, dY2, bb + LY::B_KQW, 0,
+                      sb + LY::DY, 0, false);
         }
         if (!mma_done()) break;
-        {
-            float qs[BV], op[BV];
-            ld_row<BV>(tb, warp, LY::cQS, qs);
-            ld_row<BV>(tb, warp, LY::cO, op);
-            if (own_t && t_row < n) {
-                const float gt = sGam[t_row];
-                __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t_row) * H + h) * dv + v0;
+        if (tid == 0 && c + 1 < nch) load_mq(c + 1);  // the Mqk tiles are free again
+        if (warp < 2) {
+            float x[BV];
+            ld_pair_sum<BV>(tb, warp, LY::cD3, x);
+            const int t = tid;
+            if (t < n) {
+                const float gt = sGam[t];
+                __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t) * H + h) * dv + v0;
 #pragma unroll
                 for (int c8 = 0; c8 < BV / 8; ++c8) {
                     float r[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) r[j] = fmaf(gt, qs[c8 * 8 + j], op[c8 * 8 + j]);
+                    for (int j = 0; j < 8; ++j)
+                        r[j] = fmaf(gt, qs[c8 * 8 + j], x[c8 * 8 + j]);
                     uint4 pk;
                     pk.x = pack_bf16(r[0], r[1]);
                     pk.y = pack_bf16(r[2], r[3]);
@@ -412,13 +513,15 @@ __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint
                     *reinterpret_cast<uint4 *>(dst + c8 * 8) = pk;
                 }
             }
-            float ds[BV];
-            ld_row<BV>(tb, warp, LY::cDS, ds);
-            const float gC = expf(g_last);
+        }
+        {
+            float x[BV];
+            ld_pair_sum<BV>(tb, warp, LY::cD4, x);
+            const float gC = __expf(g_last);
             if (own_d) {
 #pragma unroll
-                for (int j = 0; j < BV; ++j) Sreg[j] = fmaf(gC, Sreg[j], ds[j]);
-                store_row_split<BV>(sm + LY::S, sm + LY::SL, d_row, Sreg);
+                for (int j = 0; j < BV; ++j) Sreg[j] = fmaf(gC, Sreg[j], x[j]);
+                store_row_pair<BV>(sm + LY::S, LY::S_BLK, d_row, Sreg);
             }
         }
         sync_for_mma();

@@ -108,7 +108,6 @@ __global__ void __launch_bounds__(NT, 1) scan_tc_kernel(ScanArgs p) {
     const size_t head = (size_t)b * H + h;
 
     float *sA = (float *)(sm + LY::AF);
-    float *sT = (float *)(sm + LY::TF);
     float *sTmp = (float *)(sm + LY::TMP);
     float *sG = (float *)(sm + LY::GATES);
     float *sBeta = sG + C;
@@ -238,14 +237,14 @@ __global__ void __launch_bounds__(NT, 1) scan_tc_kernel(ScanArgs p) {
         __syncthreads();
 
         // ---- T = (I + A)^{-1}; bf16 pairs of T diag(beta gamma) and T diag(beta) (GDN) or T
-        solve_unit_lower<NT>(sA, sT, sTmp, tid);
+        solve_unit_lower<NT>(sA, sA, sTmp, tid);  // in place: sA now holds T
         for (int e = tid; e < C * (C / 8); e += NT) {
             const int t = e / (C / 8), c8 = e % (C / 8);
             float a1[8], a2[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int i = c8 * 8 + j;
-                const float tv = (i <= t) ? sT[t * AS + i] : 0.f;
+                const float tv = (i <= t) ? sA[t * AS + i] : 0.f;
                 a1[j] = tv * sBeta[i] * sGam[i];
                 a2[j] = GDN ? tv * sBeta[i] : tv;
             }
