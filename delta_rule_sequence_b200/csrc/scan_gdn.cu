@@ -8,7 +8,7 @@
 // It writes Wk (bf16), T diag(beta) and Mqk (bf16 hi/lo pairs) and g to a per-chunk record in the
 // workspace, already laid out as the 128B-swizzled shared-memory images the MMAs read.
 // `gdn_state_kernel` then walks the chunks of one (batch, head, value slice) in order with the
-// fp32 state on chip; per chunk it prefetches the next chunk's tiles (cp.async, double buffered)
+// fp32 state on chip; per chunk it prefetches the next chunk's tiles (TMA, double buffered)
 // and runs only two dependent MMA rounds:
 //   U = T diag(beta) V,  X_s = Wk S^T,  QS = Q S^T;   Y = U - X_s
 //   O = diag(e^g) QS + Mqk Y,   S'^T = e^{g_n} S^T + K^T D Y.
@@ -17,12 +17,23 @@
 // forget and rank-1 write.)  Prep runs over chunks last-first, so the records the state kernel
 // needs first are the ones most recently written and most likely still in L2.
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "chunk_common.cuh"
 
 namespace prism {
 namespace {
 
 constexpr int NT = 128;
+
+// TMA descriptors of the bf16 activations, viewed as 4-D {d, H, T, B} (innermost first) so that
+// a box {64 | BV, 1, 64, 1} is one head's chunk; rows past T read as zeros.
+struct GdnMaps {
+    CUtensorMap k, q, v;
+};
 
 // One workspace record per (b, h, chunk): swizzled shared-memory images.
 template <int DK>
@@ -37,15 +48,6 @@ struct GdnRec {
     static constexpr uint32_t BYTES = G + 1024;
 };
 constexpr size_t kRecOffset = 1024;  // records start after the status block
-
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
-                 "l"(gsrc), "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // ------------------------------------------------------------------------------------------------
 // prep: one CTA per (chunk, head, batch)
@@ -63,12 +65,13 @@ struct PrepLayout {
 };
 
 template <int DK>
-__global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, uint8_t *ws, int nch) {
+__global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_constant__ GdnMaps maps,
+                                                     uint8_t *ws, int nch) {
     using LY = PrepLayout<DK>;
     using RC = GdnRec<DK>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t mma_bar;
+    __shared__ uint64_t mma_bar, ld_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int failed_sh;
 
@@ -76,7 +79,6 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, uint8_t *ws, i
     const int c = nch - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int H = p.H, T = p.T;
     const int c0 = c * C, n = min(C, T - c0);
-    const __nv_bfloat16 *q = (const __nv_bfloat16 *)p.q, *k = (const __nv_bfloat16 *)p.k;
     uint8_t *rec = ws + kRecOffset + (((size_t)b * H + h) * nch + c) * RC::BYTES;
     float *sA = (float *)(sm + LY::AF);
     float *sTmp = (float *)(sm + LY::TMP);
@@ -85,21 +87,19 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, uint8_t *ws, i
     float *sGam = sBeta + C;
     const uint32_t sb = smem_u32(sm);
 
-    // K and Q rows (zero rows past the end of the sequence are identity tokens)
-    for (int e = tid; e < C * (DK / 8); e += NT) {
-        const int t = e / (DK / 8), ch = e % (DK / 8);
-        const bool ok = t < n;
-        const size_t g = ok ? ((((size_t)b * T + c0 + t) * H + h) * DK + ch * 8) : 0;
-        cp_async16(sm + LY::KQ + sw128_off(t, ch * 8, LY::KQ_BLK), k + g, ok ? 16 : 0);
-        cp_async16(sm + LY::KQ + sw128_off(C + t, ch * 8, LY::KQ_BLK), q + g, ok ? 16 : 0);
-    }
-    cp_async_commit();
-    if (warp == 0) tmem_alloc(&tmem_base_sh, 128);
+    // K and Q boxes by TMA (rows past the end of the sequence arrive as zeros: identity tokens)
     if (tid == 0) {
         mbar_init(&mma_bar, 1);
+        mbar_init(&ld_bar, 1);
         mbar_fence_init();
         failed_sh = 0;
+        mbar_expect_tx(&ld_bar, 2 * (DK / 64) * C * 128);
+        for (int blk = 0; blk < DK / 64; ++blk) {
+            tma_load_4d(sm + LY::KQ + blk * LY::KQ_BLK, &maps.k, blk * 64, h, c0, b, &ld_bar);
+            tma_load_4d(sm + LY::KQ + blk * LY::KQ_BLK + C * 128, &maps.q, blk * 64, h, c0, b, &ld_bar);
+        }
     }
+    if (warp == 0) tmem_alloc(&tmem_base_sh, 128);
     if (tid < C) {
         const size_t bth = ((size_t)b * T + c0 + tid) * H + h;
         sG[tid] = tid < n ? logf(p.alpha[bth]) : 0.f;
@@ -112,8 +112,7 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, uint8_t *ws, i
         sG[lane] = x0;
         sG[32 + lane] = x1;
     }
-    cp_async_wait<0>();
-    fence_async_smem();
+    if (!mbar_wait(&ld_bar, 0, p.status)) failed_sh = 1;
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -124,11 +123,13 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, uint8_t *ws, i
     }
 
     // G = [K; Q] K^T
-    if (tid == 0)
-        mma_split(tb, idesc_bf16(128, C, 0, 0), DK / 16,
-                  [](uint32_t base, int ks) { return desc_k_sw128(base, ks, LY::KQ_BLK); },
-                  [](uint32_t base, int ks) { return desc_k_sw128(base, ks, LY::KQ_BLK); },
-                  sb + LY::KQ, 0, sb + LY::KQ, 0, false);
+    auto okq = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::KQ_BLK); };
+    auto ok0 = [](int ks) { return (uint64_t)koff_k_sw128(ks, 0); };
+    auto omn = [](int ks) { return (uint64_t)koff_mn_sw128(ks); };
+    if (tid == 0 && failed_sh == 0) {
+        const uint64_t dkq = make_desc(sb + LY::KQ, 16, 1024, 2);
+        mma_steps<DK / 16>(tb, idesc_bf16(128, C, 0, 0), dkq, dkq, okq, okq, false);
+    }
     if (tid == 0) mma_commit(&mma_bar);
     __syncwarp();
     if (!mbar_wait(&mma_bar, 0, p.status)) failed_sh = 1;
@@ -189,10 +190,10 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, uint8_t *ws, i
     fence_after_sync();
     // Wk = T diag(beta gamma) K  (M = 64, N = DK; K read as an MN-major operand)
     if (ok && tid == 0) {
-        mma_split(tb, idesc_bf16(64, DK, 0, 1), C / 16,
-                  [](uint32_t base, int ks) { return desc_k_sw128(base, ks, 0); },
-                  [](uint32_t base, int ks) { return desc_mn_sw128(base, ks, LY::KQ_BLK); },
-                  sb + LY::T1, sb + LY::T1L, sb + LY::KQ, 0, false);
+        const uint32_t id = idesc_bf16(64, DK, 0, 1);
+        const uint64_t dK = make_desc(sb + LY::KQ, LY::KQ_BLK, 1024, 2);
+        mma_steps<C / 16>(tb, id, make_desc(sb + LY::T1, 16, 1024, 2), dK, ok0, omn, false);
+        mma_steps<C / 16>(tb, id, make_desc(sb + LY::T1L, 16, 1024, 2), dK, ok0, omn, true);
         mma_commit(&mma_bar);
     }
     __syncwarp();
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, uint8_t *ws, i
 //   round 2:  D3  = [Mqk_hi; 0] [Y_hi | Y_lo] ;  D3[:, :BV] += [Mqk_lo; 0] Y_hi
 //             D4  = K^T [DY_hi | DY_lo]
 // so that every operand row t of the chunk sits in TMEM lane t (QS, O) or lane 64 + t (X_s - U).
-// The per-chunk records (Wk, T2, Mqk, g) arrive by TMA bulk copies; K, Q and V by cp.async.
+// K, Q and V arrive by TMA tiled loads, the per-chunk records (Wk, T2, Mqk, g) by bulk copies.
 
 template <int DK, int BV>
 struct StateLayout {
@@ -259,17 +260,6 @@ struct StateLayout {
     static constexpr uint32_t TCOLS = (3 * N2 <= 128) ? 128 : (3 * N2 <= 256 ? 256 : 512);
 };
 
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
 // An N2-wide row of fp32 (hi | lo of one value each) stored as bf16 into an MN-major tile of
 // 64-column 128B-swizzled blocks: cols [0, BV) get bf16(x), cols [BV, 2BV) get bf16(x - hi).
 template <int BV>
@@ -298,42 +288,20 @@ __device__ __forceinline__ void ld_pair_sum(uint32_t tbase, int warp, uint32_t c
     }
 }
 
-template <int DK, int BV>
-__device__ __forceinline__ void state_issue_cp(const ScanArgs &p, int c, uint8_t *buf, int tid) {
-    using LY = StateLayout<DK, BV>;
-    const int v0 = blockIdx.x * BV, h = blockIdx.y, b = blockIdx.z;
-    const int H = p.H, T = p.T, dv = p.dv;
-    const int c0 = c * C, n = min(C, T - c0);
-    const __nv_bfloat16 *q = (const __nv_bfloat16 *)p.q, *k = (const __nv_bfloat16 *)p.k;
-    const __nv_bfloat16 *v = (const __nv_bfloat16 *)p.v;
-    for (int e = tid; e < C * (DK / 8); e += NT) {
-        const int t = e / (DK / 8), ch = e % (DK / 8);
-        const bool ok = t < n;
-        const size_t g = ok ? ((((size_t)b * T + c0 + t) * H + h) * DK + ch * 8) : 0;
-        cp_async16(buf + LY::B_KQW + sw128_off(t, ch * 8, LY::KQW_BLK), k + g, ok ? 16 : 0);
-        cp_async16(buf + LY::B_KQW + sw128_off(C + t, ch * 8, LY::KQW_BLK), q + g, ok ? 16 : 0);
-    }
-    for (int e = tid; e < C * (BV / 8); e += NT) {
-        const int t = e / (BV / 8), ch = e % (BV / 8);
-        const bool ok = t < n;
-        const size_t g = ok ? ((((size_t)b * T + c0 + t) * H + h) * dv + v0 + ch * 8) : 0;
-        cp_async16(buf + LY::B_V + vt_off<BV>(t, ch * 8), v + g, ok ? 16 : 0);
-    }
-}
-
 template <int DK>
 __device__ __forceinline__ const uint8_t *record(const ScanArgs &p, const uint8_t *ws, int nch, int c) {
     return ws + kRecOffset + (((size_t)blockIdx.z * p.H + blockIdx.y) * nch + c) * GdnRec<DK>::BYTES;
 }
 
 template <int DK, int BV>
-__global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint8_t *ws, int nch) {
+__global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const __grid_constant__ GdnMaps maps,
+                                                          const uint8_t *ws, int nch) {
     using LY = StateLayout<DK, BV>;
     using RC = GdnRec<DK>;
     constexpr int N2 = LY::N2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t mma_bar, wk_bar[2], t2_bar, mq_bar;
+    __shared__ uint64_t mma_bar, ld_bar[2], t2_bar, mq_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int failed_sh;
 
@@ -346,15 +314,20 @@ __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint
     float *sD = sGam + C;
     const uint32_t sb = smem_u32(sm);
 
-    // bulk loads of a chunk record: Wk + g into the chunk buffer; T2 and Mqk into the shared tiles
-    auto load_wk = [&](int c) {
+    // one thread fetches a chunk: K, Q, V boxes by TMA, the Wk image and g by bulk copy
+    auto load_chunk = [&](int c) {
         const uint8_t *rec = record<DK>(p, ws, nch, c);
         uint8_t *buf = sm + (c & 1) * LY::BUF;
-        uint64_t *bar = &wk_bar[c & 1];
-        mbar_expect_tx(bar, (DK / 64) * RC::WK_BLK + C * 4);
-        for (int blk = 0; blk < DK / 64; ++blk)
-            bulk_g2s(buf + LY::B_KQW + blk * LY::KQW_BLK + 2 * C * 128, rec + RC::WK + blk * RC::WK_BLK,
-                     RC::WK_BLK, bar);
+        uint64_t *bar = &ld_bar[c & 1];
+        const int c0 = c * C;
+        mbar_expect_tx(bar, 2 * (DK / 64) * C * 128 + LY::VT + (DK / 64) * RC::WK_BLK + C * 4);
+        for (int blk = 0; blk < DK / 64; ++blk) {
+            uint8_t *dst = buf + LY::B_KQW + blk * LY::KQW_BLK;
+            tma_load_4d(dst, &maps.k, blk * 64, h, c0, b, bar);
+            tma_load_4d(dst + C * 128, &maps.q, blk * 64, h, c0, b, bar);
+            bulk_g2s(dst + 2 * C * 128, rec + RC::WK + blk * RC::WK_BLK, RC::WK_BLK, bar);
+        }
+        tma_load_4d(buf + LY::B_V, &maps.v, v0, h, c0, b, bar);
         bulk_g2s(buf + LY::B_G, rec + RC::G, C * 4, bar);
     };
     auto load_t2 = [&](int c) {
@@ -373,12 +346,17 @@ __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint
     if (warp == 0) tmem_alloc(&tmem_base_sh, LY::TCOLS);
     if (tid == 0) {
         mbar_init(&mma_bar, 1);
-        mbar_init(&wk_bar[0], 1);
-        mbar_init(&wk_bar[1], 1);
+        mbar_init(&ld_bar[0], 1);
+        mbar_init(&ld_bar[1], 1);
         mbar_init(&t2_bar, 1);
         mbar_init(&mq_bar, 1);
         mbar_fence_init();
         failed_sh = 0;
+        if (nch > 0) {
+            load_chunk(0);
+            load_t2(0);
+            load_mq(0);
+        }
     }
     // zero tiles under Mqk and over T2 (never overwritten)
     for (int e = tid; e < C * 128 / 16; e += NT) {
@@ -388,18 +366,9 @@ __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
-    if (nch > 0) {
-        state_issue_cp<DK, BV>(p, 0, sm, tid);
-        if (tid == 0) {
-            load_wk(0);
-            load_t2(0);
-            load_mq(0);
-        }
-    }
-    cp_async_commit();
     const uint32_t tb = tmem_base_sh;
     uint32_t phase = 0;
-    auto fail_sync = [&](bool ok) -> bool {  // make one thread's timeout everyone's
+    auto fail_sync = [&](bool ok) -> bool {  // one thread's timeout becomes everyone's
         if (!ok) failed_sh = 1;
         fence_after_sync();
         __syncthreads();
@@ -412,12 +381,16 @@ __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint
         phase++;
         return fail_sync(ok);
     };
-    auto dKQW = [](uint32_t base, int ks) { return desc_k_sw128(base, ks, LY::KQW_BLK); };
-    auto dKmn = [](uint32_t base, int ks) { return desc_mn_sw128(base, ks, LY::KQW_BLK); };
-    auto dK = [](uint32_t base, int ks) { return desc_k_sw128(base, ks, 0); };
-    auto dVT = [](uint32_t base, int ks) { return desc_vt<BV>(base, ks); };
-    auto dS2 = [](uint32_t base, int ks) { return desc_mn_sw128(base, ks, LY::S_BLK); };
-    auto dY2 = [](uint32_t base, int ks) { return desc_mn_sw128(base, ks, LY::Y_BLK); };
+    // k-step offsets (16-byte units) of the operand kinds
+    auto oKQW = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::KQW_BLK); };
+    auto oK0 = [](int ks) { return (uint64_t)koff_k_sw128(ks, 0); };
+    auto oMN = [](int ks) { return (uint64_t)koff_mn_sw128(ks); };
+    auto oVT = [](int ks) { return (uint64_t)(BV == 32 ? koff_mn_sw64(ks) : koff_mn_sw128(ks)); };
+    const uint64_t dS2 = make_desc(sb + LY::S, LY::S_BLK, 1024, 2);
+    const uint64_t dY2 = make_desc(sb + LY::Y, LY::Y_BLK, 1024, 2);
+    const uint64_t dDY2 = make_desc(sb + LY::DY, LY::Y_BLK, 1024, 2);
+    const uint64_t dZ1 = make_desc(sb + LY::Z1, 16, 1024, 2), dZ2 = make_desc(sb + LY::Z2, 16, 1024, 2);
+    const uint64_t dMH = make_desc(sb + LY::MH, 16, 1024, 2), dML = make_desc(sb + LY::ML, 16, 1024, 2);
 
     // fp32 state S^T: DK = 128 -> d = tid (M = 128); DK = 64 -> M = 64 layout (warp d/16, lane d%16)
     const bool own_d = (DK == 128) ? true : (lane < 16);
@@ -435,13 +408,8 @@ __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint
         const int c0 = c * C, n = min(C, T - c0);
         const uint32_t bb = sb + (c & 1) * LY::BUF;
         const uint8_t *buf = sm + (c & 1) * LY::BUF;
-        if (c + 1 < nch) {
-            state_issue_cp<DK, BV>(p, c + 1, sm + ((c + 1) & 1) * LY::BUF, tid);
-            if (tid == 0) load_wk(c + 1);
-        }
-        cp_async_commit();
-        cp_async_wait<1>();
-        bool ok = mbar_wait(&wk_bar[c & 1], (c >> 1) & 1, p.status);
+        if (tid == 0 && c + 1 < nch) load_chunk(c + 1);  // buffer (c+1)&1 was released by chunk c-1
+        bool ok = mbar_wait(&ld_bar[c & 1], (c >> 1) & 1, p.status);
         ok = mbar_wait(&t2_bar, c & 1, p.status) && ok;
         if (!fail_sync(ok)) break;
         const float *g = reinterpret_cast<const float *>(buf + LY::B_G);
@@ -452,43 +420,41 @@ __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint
         }
         sync_for_mma();
 
-        // round 1
+        // round 1: D1 = [Q; Wk] [S_hi | S_lo];  D1[:, :BV] -= [0; T2_hi] V + [0; T2_lo] V
         if (tid == 0) {
-            mma_split(tb + LY::cD1, idesc_bf16(128, N2, 0, 1), DK / 16, dKQW, dS2,
-                      bb + LY::B_KQW + C * 128, 0, sb + LY::S, 0, false);
+            const uint64_t dQW = make_desc(bb + LY::B_KQW + C * 128, 16, 1024, 2);
+            const uint64_t dV = (BV == 32) ? make_desc(bb + LY::B_V, 0, 512, 4)
+                                           : make_desc(bb + LY::B_V, C * 128, 1024, 2);
+            mma_steps<DK / 16>(tb + LY::cD1, idesc_bf16(128, N2, 0, 1), dQW, dS2, oKQW, oMN, false);
             const uint32_t idn = idesc_bf16(128, BV, 0, 1) | (1u << 13);  // negate A
-            mma_split(tb + LY::cD1, idn, C / 16, dK, dVT, sb + LY::Z1, sb + LY::Z2, bb + LY::B_V, 0,
-                      true);
+            mma_steps<C / 16>(tb + LY::cD1, idn, dZ1, dV, oK0, oVT, true);
+            mma_steps<C / 16>(tb + LY::cD1, idn, dZ2, dV, oK0, oVT, true);
         }
         if (!mma_done()) break;
         if (tid == 0 && c + 1 < nch) load_t2(c + 1);  // the T2 tiles are free again
         float qs[BV];  // rows 0..63 (warps 0-1): QS;  rows 64..127 (warps 2-3): X_s - U = -Y
         ld_pair_sum<BV>(tb, warp, LY::cD1, qs);
-        {
-            if (warp >= 2) {
-                const int t = tid - 64;
-                float y[BV];
+        if (warp >= 2) {
+            const int t = tid - 64;
+            float y[BV];
 #pragma unroll
-                for (int j = 0; j < BV; ++j) y[j] = -qs[j];
-                store_row_pair<BV>(sm + LY::Y, LY::Y_BLK, t, y);
-                const float dd = sD[t];
+            for (int j = 0; j < BV; ++j) y[j] = -qs[j];
+            store_row_pair<BV>(sm + LY::Y, LY::Y_BLK, t, y);
+            const float dd = sD[t];
 #pragma unroll
-                for (int j = 0; j < BV; ++j) y[j] *= dd;
-                store_row_pair<BV>(sm + LY::DY, LY::Y_BLK, t, y);
-            }
+            for (int j = 0; j < BV; ++j) y[j] *= dd;
+            store_row_pair<BV>(sm + LY::DY, LY::Y_BLK, t, y);
         }
         ok = mbar_wait(&mq_bar, c & 1, p.status);
         if (!fail_sync(ok)) break;
         sync_for_mma();
 
-        // round 2
+        // round 2: D3 = [Mqk_hi; 0][Y_hi | Y_lo] + [Mqk_lo; 0] Y_hi ;  D4 = K^T [DY_hi | DY_lo]
         if (tid == 0) {
-            mma_split(tb + LY::cD3, idesc_bf16(128, N2, 0, 1), C / 16, dK, dY2, sb + LY::MH, 0,
-                      sb + LY::Y, 0, false);
-            mma_split(tb + LY::cD3, idesc_bf16(128, BV, 0, 1), C / 16, dK, dY2, sb + LY::ML, 0,
-                      sb + LY::Y, 0, true);
-            mma_split(tb + LY::cD4, idesc_bf16(DK, N2, 1, 1), C / 16, dKmn, dY2, bb + LY::B_KQW, 0,
-                      sb + LY::DY, 0, false);
+            mma_steps<C / 16>(tb + LY::cD3, idesc_bf16(128, N2, 0, 1), dMH, dY2, oK0, oMN, false);
+            mma_steps<C / 16>(tb + LY::cD3, idesc_bf16(128, BV, 0, 1), dML, dY2, oK0, oMN, true);
+            const uint64_t dKt = make_desc(bb + LY::B_KQW, LY::KQW_BLK, 1024, 2);
+            mma_steps<C / 16>(tb + LY::cD4, idesc_bf16(DK, N2, 1, 1), dKt, dDY2, oMN, oMN, false);
         }
         if (!mma_done()) break;
         if (tid == 0 && c + 1 < nch) load_mq(c + 1);  // the Mqk tiles are free again
@@ -503,8 +469,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint
                 for (int c8 = 0; c8 < BV / 8; ++c8) {
                     float r[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        r[j] = fmaf(gt, qs[c8 * 8 + j], x[c8 * 8 + j]);
+                    for (int j = 0; j < 8; ++j) r[j] = fmaf(gt, qs[c8 * 8 + j], x[c8 * 8 + j]);
                     uint4 pk;
                     pk.x = pack_bf16(r[0], r[1]);
                     pk.y = pack_bf16(r[2], r[3]);
@@ -526,7 +491,6 @@ __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint
         }
         sync_for_mma();
     }
-    cp_async_wait<0>();
 
     if (p.S_final && own_d && failed_sh == 0) {
 #pragma unroll
@@ -537,21 +501,52 @@ __global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const uint
     if (warp == 0) tmem_dealloc(tb, LY::TCOLS);
 }
 
+// Host: the driver's tensor-map encoder, fetched once through the runtime (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 4-D map over a bf16 activation [B, T, H, d]: dims {d, H, T, B}, box {box_d, 1, C, 1}.
+bool act_map(CUtensorMap *m, const void *base, int B, int T, int H, int d, int box_d) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)box_d, 1, (cuuint32_t)C, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapSwizzle sw = box_d * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int DK, int BV>
 cudaError_t launch_gdn(const ScanArgs &a, void *ws, cudaStream_t s) {
     const int nch = (a.T + C - 1) / C;
+    GdnMaps maps;
+    if (!act_map(&maps.k, a.k, a.B, a.T, a.H, DK, 64) || !act_map(&maps.q, a.q, a.B, a.T, a.H, DK, 64) ||
+        !act_map(&maps.v, a.v, a.B, a.T, a.H, a.dv, BV))
+        return cudaErrorInvalidValue;
     {
         using LY = PrepLayout<DK>;
         auto kern = gdn_prep_kernel<DK>;
         cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)LY::BYTES);
         if (err != cudaSuccess) return err;
-        if (nch > 0) {
-            dim3 grid(nch, a.H, a.B);
-            kern<<<grid, NT, LY::BYTES, s>>>(a, (uint8_t *)ws, nch);
-            err = cudaGetLastError();
-            if (err != cudaSuccess) return err;
-        }
+        dim3 grid(nch, a.H, a.B);
+        kern<<<grid, NT, LY::BYTES, s>>>(a, maps, (uint8_t *)ws, nch);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
     }
     {
         using LY = StateLayout<DK, BV>;
@@ -561,7 +556,7 @@ cudaError_t launch_gdn(const ScanArgs &a, void *ws, cudaStream_t s) {
                                                (int)LY::BYTES);
         if (err != cudaSuccess) return err;
         dim3 grid(a.dv / BV, a.H, a.B);
-        kern<<<grid, NT, LY::BYTES, s>>>(a, (const uint8_t *)ws, nch);
+        kern<<<grid, NT, LY::BYTES, s>>>(a, maps, (const uint8_t *)ws, nch);
         return cudaGetLastError();
     }
 }

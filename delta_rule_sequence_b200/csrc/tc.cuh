@@ -65,6 +65,52 @@ __device__ __forceinline__ uint64_t desc_mn_sw64(uint32_t base, int ks) {
     return make_desc(base + ks * 16 * 64, 0, 512, 4);
 }
 
+// k-step offsets of an operand, in the descriptor's 16-byte address units (added to a base
+// descriptor: the start-address field cannot carry because shared addresses stay below 256 KB).
+__host__ __device__ constexpr uint32_t koff_k_sw128(int ks, uint32_t block_bytes) {
+    return (((uint32_t)(ks * 16) >> 6) * block_bytes + (uint32_t)((ks * 16) & 63) * 2) >> 4;
+}
+__host__ __device__ constexpr uint32_t koff_mn_sw128(int ks) { return (uint32_t)ks * 128; }
+__host__ __device__ constexpr uint32_t koff_mn_sw64(int ks) { return (uint32_t)ks * 64; }
+
+// NKS k-steps of 16 into accumulator d: A and B base descriptors plus per-step offsets.
+template <int NKS, class OA, class OB>
+__device__ __forceinline__ void mma_steps(uint32_t d, uint32_t idesc, uint64_t a, uint64_t b, OA oa,
+                                          OB ob, bool accumulate) {
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+            :
+            : "r"(d), "l"(a + oa(ks)), "l"(b + ob(ks)), "r"(idesc),
+              "r"((accumulate || ks > 0) ? 1u : 0u));
+}
+
+// 4-D tiled TMA load of one box into shared memory, completing on `bar` (tx bytes).
+__device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int x, int y, int z, int w,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4, %5}], [%6];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(w),
+          "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Plain (untiled) bulk copy global -> shared, completing on `bar` (tx bytes); 16-byte aligned.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
 // Instruction descriptor: bf16 x bf16 -> fp32, M x N, A/B K-major (0) or MN-major (1).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
