@@ -256,8 +256,8 @@ struct StateLayout {
     static constexpr uint32_t GATES = DY + Y_BLK * (N2 / 64);  // gamma, D: 2 x C floats
     static constexpr uint32_t BYTES = GATES + 2 * C * 4 + 1024;
     // TMEM columns
-    static constexpr uint32_t cD1 = 0, cD3 = N2, cD4 = 2 * N2;
-    static constexpr uint32_t TCOLS = (3 * N2 <= 128) ? 128 : (3 * N2 <= 256 ? 256 : 512);
+    static constexpr uint32_t cD1 = 0, cD3 = N2, cD4 = 2 * N2, cU = 3 * N2;
+    static constexpr uint32_t TCOLS = (3 * N2 + BV <= 128) ? 128 : (3 * N2 + BV <= 256 ? 256 : 512);
 };
 
 // An N2-wide row of fp32 (hi | lo of one value each) stored as bf16 into an MN-major tile of
@@ -293,208 +293,246 @@ __device__ __forceinline__ const uint8_t *record(const ScanArgs &p, const uint8_
     return ws + kRecOffset + (((size_t)blockIdx.z * p.H + blockIdx.y) * nch + c) * GdnRec<DK>::BYTES;
 }
 
+// Warp roles of the state kernel: warps 0-3 epilogue (TMEM lane quarters 0-3), warp 4 issues the
+// MMAs, warp 5 issues the loads.  Every hand-off is an mbarrier; every wait is bounded.
+constexpr int ST_THREADS = 192;
+constexpr int EPI_THREADS = 128;
+
+struct StateBars {
+    uint64_t full[2];      // chunk inputs landed (tx): K, Q, V, Wk, g
+    uint64_t empty[2];     // chunk buffer released: last MMA reading it (commit) + epilogue (g read)
+    uint64_t t2_full, t2_empty, mq_full, mq_empty;
+    uint64_t s_ready, y_ready;      // epilogue -> MMA: S^T tile, Y / DY tiles written
+    uint64_t d1_full, d4_full, d3_full;  // MMA -> epilogue: accumulators complete
+};
+
 template <int DK, int BV>
-__global__ void __launch_bounds__(NT, 1) gdn_state_kernel(ScanArgs p, const __grid_constant__ GdnMaps maps,
-                                                          const uint8_t *ws, int nch) {
+__global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
+                                                                 const __grid_constant__ GdnMaps maps,
+                                                                 const uint8_t *ws, int nch) {
     using LY = StateLayout<DK, BV>;
     using RC = GdnRec<DK>;
     constexpr int N2 = LY::N2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t mma_bar, ld_bar[2], t2_bar, mq_bar;
+    __shared__ StateBars bars;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int failed_sh;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int v0 = blockIdx.x * BV, h = blockIdx.y, b = blockIdx.z;
     const int H = p.H, T = p.T, dv = p.dv;
-    __nv_bfloat16 *o = (__nv_bfloat16 *)p.o;
     const size_t head = (size_t)b * H + h;
-    float *sGam = (float *)(sm + LY::GATES);
-    float *sD = sGam + C;
     const uint32_t sb = smem_u32(sm);
-
-    // one thread fetches a chunk: K, Q, V boxes by TMA, the Wk image and g by bulk copy
-    auto load_chunk = [&](int c) {
-        const uint8_t *rec = record<DK>(p, ws, nch, c);
-        uint8_t *buf = sm + (c & 1) * LY::BUF;
-        uint64_t *bar = &ld_bar[c & 1];
-        const int c0 = c * C;
-        mbar_expect_tx(bar, 2 * (DK / 64) * C * 128 + LY::VT + (DK / 64) * RC::WK_BLK + C * 4);
-        for (int blk = 0; blk < DK / 64; ++blk) {
-            uint8_t *dst = buf + LY::B_KQW + blk * LY::KQW_BLK;
-            tma_load_4d(dst, &maps.k, blk * 64, h, c0, b, bar);
-            tma_load_4d(dst + C * 128, &maps.q, blk * 64, h, c0, b, bar);
-            bulk_g2s(dst + 2 * C * 128, rec + RC::WK + blk * RC::WK_BLK, RC::WK_BLK, bar);
-        }
-        tma_load_4d(buf + LY::B_V, &maps.v, v0, h, c0, b, bar);
-        bulk_g2s(buf + LY::B_G, rec + RC::G, C * 4, bar);
-    };
-    auto load_t2 = [&](int c) {
-        const uint8_t *rec = record<DK>(p, ws, nch, c);
-        mbar_expect_tx(&t2_bar, 2 * C * 128);
-        bulk_g2s(sm + LY::T2H, rec + RC::T2, C * 128, &t2_bar);
-        bulk_g2s(sm + LY::T2L, rec + RC::T2L, C * 128, &t2_bar);
-    };
-    auto load_mq = [&](int c) {
-        const uint8_t *rec = record<DK>(p, ws, nch, c);
-        mbar_expect_tx(&mq_bar, 2 * C * 128);
-        bulk_g2s(sm + LY::MH, rec + RC::MQK, C * 128, &mq_bar);
-        bulk_g2s(sm + LY::ML, rec + RC::MQKL, C * 128, &mq_bar);
-    };
 
     if (warp == 0) tmem_alloc(&tmem_base_sh, LY::TCOLS);
     if (tid == 0) {
-        mbar_init(&mma_bar, 1);
-        mbar_init(&ld_bar[0], 1);
-        mbar_init(&ld_bar[1], 1);
-        mbar_init(&t2_bar, 1);
-        mbar_init(&mq_bar, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars.full[i], 1);
+            mbar_init(&bars.empty[i], 2);
+        }
+        mbar_init(&bars.t2_full, 1);
+        mbar_init(&bars.t2_empty, 1);
+        mbar_init(&bars.mq_full, 1);
+        mbar_init(&bars.mq_empty, 1);
+        mbar_init(&bars.s_ready, 1);
+        mbar_init(&bars.y_ready, 1);
+        mbar_init(&bars.d1_full, 1);
+        mbar_init(&bars.d4_full, 1);
+        mbar_init(&bars.d3_full, 1);
         mbar_fence_init();
         failed_sh = 0;
-        if (nch > 0) {
-            load_chunk(0);
-            load_t2(0);
-            load_mq(0);
-        }
     }
-    // zero tiles under Mqk and over T2 (never overwritten)
-    for (int e = tid; e < C * 128 / 16; e += NT) {
+    for (int e = tid; e < C * 128 / 16; e += ST_THREADS) {  // zero tiles under Mqk and over T2
         st16(sm + LY::Z1, e * 16, make_uint4(0, 0, 0, 0));
         st16(sm + LY::Z2, e * 16, make_uint4(0, 0, 0, 0));
     }
+    fence_async_smem();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tb = tmem_base_sh;
-    uint32_t phase = 0;
-    auto fail_sync = [&](bool ok) -> bool {  // one thread's timeout becomes everyone's
-        if (!ok) failed_sh = 1;
-        fence_after_sync();
-        __syncthreads();
-        return failed_sh == 0;
-    };
-    auto mma_done = [&]() -> bool {
-        if (tid == 0) mma_commit(&mma_bar);
-        __syncwarp();
-        const bool ok = mbar_wait(&mma_bar, phase & 1, p.status);
-        phase++;
-        return fail_sync(ok);
-    };
-    // k-step offsets (16-byte units) of the operand kinds
-    auto oKQW = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::KQW_BLK); };
-    auto oK0 = [](int ks) { return (uint64_t)koff_k_sw128(ks, 0); };
-    auto oMN = [](int ks) { return (uint64_t)koff_mn_sw128(ks); };
-    auto oVT = [](int ks) { return (uint64_t)(BV == 32 ? koff_mn_sw64(ks) : koff_mn_sw128(ks)); };
-    const uint64_t dS2 = make_desc(sb + LY::S, LY::S_BLK, 1024, 2);
-    const uint64_t dY2 = make_desc(sb + LY::Y, LY::Y_BLK, 1024, 2);
-    const uint64_t dDY2 = make_desc(sb + LY::DY, LY::Y_BLK, 1024, 2);
-    const uint64_t dZ1 = make_desc(sb + LY::Z1, 16, 1024, 2), dZ2 = make_desc(sb + LY::Z2, 16, 1024, 2);
-    const uint64_t dMH = make_desc(sb + LY::MH, 16, 1024, 2), dML = make_desc(sb + LY::ML, 16, 1024, 2);
+    uint32_t *status = p.status;
+    auto fail = [&]() { failed_sh = 1; };
+    auto failed = [&]() { return *(volatile int *)&failed_sh != 0; };
 
-    // fp32 state S^T: DK = 128 -> d = tid (M = 128); DK = 64 -> M = 64 layout (warp d/16, lane d%16)
-    const bool own_d = (DK == 128) ? true : (lane < 16);
-    const int d_row = (DK == 128) ? tid : (16 * warp + lane);
-    float Sreg[BV];
-#pragma unroll
-    for (int j = 0; j < BV; ++j) Sreg[j] = 0.f;
-    if (own_d && p.S0) {
-#pragma unroll
-        for (int j = 0; j < BV; ++j) Sreg[j] = p.S0[(head * dv + v0 + j) * DK + d_row];
-    }
-    if (own_d) store_row_pair<BV>(sm + LY::S, LY::S_BLK, d_row, Sreg);
-
-    for (int c = 0; c < nch; ++c) {
-        const int c0 = c * C, n = min(C, T - c0);
-        const uint32_t bb = sb + (c & 1) * LY::BUF;
-        const uint8_t *buf = sm + (c & 1) * LY::BUF;
-        if (tid == 0 && c + 1 < nch) load_chunk(c + 1);  // buffer (c+1)&1 was released by chunk c-1
-        bool ok = mbar_wait(&ld_bar[c & 1], (c >> 1) & 1, p.status);
-        ok = mbar_wait(&t2_bar, c & 1, p.status) && ok;
-        if (!fail_sync(ok)) break;
-        const float *g = reinterpret_cast<const float *>(buf + LY::B_G);
-        const float g_last = g[C - 1];
-        if (tid < C) {
-            sGam[tid] = __expf(g[tid]);
-            sD[tid] = tid < n ? __expf(g_last - g[tid]) : 0.f;
+    if (warp == 5) {
+        // ---------------- loads ----------------
+        if (lane == 0) {
+            auto load_chunk = [&](int c) {
+                const uint8_t *rec = record<DK>(p, ws, nch, c);
+                uint8_t *buf = sm + (c & 1) * LY::BUF;
+                uint64_t *bar = &bars.full[c & 1];
+                const int c0 = c * C;
+                mbar_expect_tx(bar, 2 * (DK / 64) * C * 128 + LY::VT + (DK / 64) * RC::WK_BLK + C * 4);
+                for (int blk = 0; blk < DK / 64; ++blk) {
+                    uint8_t *dst = buf + LY::B_KQW + blk * LY::KQW_BLK;
+                    tma_load_4d(dst, &maps.k, blk * 64, h, c0, b, bar);
+                    tma_load_4d(dst + C * 128, &maps.q, blk * 64, h, c0, b, bar);
+                    bulk_g2s(dst + 2 * C * 128, rec + RC::WK + blk * RC::WK_BLK, RC::WK_BLK, bar);
+                }
+                tma_load_4d(buf + LY::B_V, &maps.v, v0, h, c0, b, bar);
+                bulk_g2s(buf + LY::B_G, rec + RC::G, C * 4, bar);
+            };
+            for (int c = 0; c < nch && !failed(); ++c) {
+                const uint8_t *rec = record<DK>(p, ws, nch, c);
+                if (c >= 2 && !mbar_wait(&bars.empty[c & 1], ((c - 2) >> 1) & 1, status)) { fail(); break; }
+                load_chunk(c);
+                if (c >= 1 && !mbar_wait(&bars.t2_empty, (c - 1) & 1, status)) { fail(); break; }
+                mbar_expect_tx(&bars.t2_full, 2 * C * 128);
+                bulk_g2s(sm + LY::T2H, rec + RC::T2, C * 128, &bars.t2_full);
+                bulk_g2s(sm + LY::T2L, rec + RC::T2L, C * 128, &bars.t2_full);
+                if (c >= 1 && !mbar_wait(&bars.mq_empty, (c - 1) & 1, status)) { fail(); break; }
+                mbar_expect_tx(&bars.mq_full, 2 * C * 128);
+                bulk_g2s(sm + LY::MH, rec + RC::MQK, C * 128, &bars.mq_full);
+                bulk_g2s(sm + LY::ML, rec + RC::MQKL, C * 128, &bars.mq_full);
+            }
         }
-        sync_for_mma();
-
-        // round 1: D1 = [Q; Wk] [S_hi | S_lo];  D1[:, :BV] -= [0; T2_hi] V + [0; T2_lo] V
-        if (tid == 0) {
-            const uint64_t dQW = make_desc(bb + LY::B_KQW + C * 128, 16, 1024, 2);
-            const uint64_t dV = (BV == 32) ? make_desc(bb + LY::B_V, 0, 512, 4)
-                                           : make_desc(bb + LY::B_V, C * 128, 1024, 2);
-            mma_steps<DK / 16>(tb + LY::cD1, idesc_bf16(128, N2, 0, 1), dQW, dS2, oKQW, oMN, false);
-            const uint32_t idn = idesc_bf16(128, BV, 0, 1) | (1u << 13);  // negate A
-            mma_steps<C / 16>(tb + LY::cD1, idn, dZ1, dV, oK0, oVT, true);
-            mma_steps<C / 16>(tb + LY::cD1, idn, dZ2, dV, oK0, oVT, true);
+    } else if (warp == 4) {
+        // ---------------- MMA issue ----------------
+        if (lane == 0) {
+            auto oKQW = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::KQW_BLK); };
+            auto oK0 = [](int ks) { return (uint64_t)koff_k_sw128(ks, 0); };
+            auto oMN = [](int ks) { return (uint64_t)koff_mn_sw128(ks); };
+            auto oVT = [](int ks) { return (uint64_t)(BV == 32 ? koff_mn_sw64(ks) : koff_mn_sw128(ks)); };
+            const uint64_t dS2 = make_desc(sb + LY::S, LY::S_BLK, 1024, 2);
+            const uint64_t dY2 = make_desc(sb + LY::Y, LY::Y_BLK, 1024, 2);
+            const uint64_t dDY2 = make_desc(sb + LY::DY, LY::Y_BLK, 1024, 2);
+            const uint64_t dZ1 = make_desc(sb + LY::Z1, 16, 1024, 2), dZ2 = make_desc(sb + LY::Z2, 16, 1024, 2);
+            const uint64_t dMH = make_desc(sb + LY::MH, 16, 1024, 2), dML = make_desc(sb + LY::ML, 16, 1024, 2);
+            const uint32_t idU = idesc_bf16(128, BV, 0, 1) | (1u << 13);  // negated A
+            const uint32_t idS = idesc_bf16(128, N2, 0, 1);
+            for (int c = 0; c < nch; ++c) {
+                const uint32_t bb = sb + (c & 1) * LY::BUF;
+                if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status)) { fail(); break; }
+                if (!mbar_wait(&bars.t2_full, c & 1, status)) { fail(); break; }
+                if (c >= 1 && !mbar_wait(&bars.y_ready, (c - 1) & 1, status)) { fail(); break; }
+                fence_after_sync();
+                // state-independent part of round 1, ahead of the state: U' = -[0; T2_hi] V - [0; T2_lo] V
+                const uint64_t dV = (BV == 32) ? make_desc(bb + LY::B_V, 0, 512, 4)
+                                               : make_desc(bb + LY::B_V, C * 128, 1024, 2);
+                mma_steps<C / 16>(tb + LY::cU, idU, dZ1, dV, oK0, oVT, false);
+                mma_steps<C / 16>(tb + LY::cU, idU, dZ2, dV, oK0, oVT, true);
+                mma_commit(&bars.t2_empty);
+                // state part: D1 = [Q; Wk] [S_hi | S_lo]
+                if (!mbar_wait(&bars.s_ready, c & 1, status)) { fail(); break; }
+                fence_after_sync();
+                const uint64_t dQW = make_desc(bb + LY::B_KQW + C * 128, 16, 1024, 2);
+                mma_steps<DK / 16>(tb + LY::cD1, idS, dQW, dS2, oKQW, oMN, false);
+                mma_commit(&bars.d1_full);
+                // round 2: the state update first (on the critical path), then the output
+                if (!mbar_wait(&bars.y_ready, c & 1, status)) { fail(); break; }
+                fence_after_sync();
+                const uint64_t dKt = make_desc(bb + LY::B_KQW, LY::KQW_BLK, 1024, 2);
+                mma_steps<C / 16>(tb + LY::cD4, idesc_bf16(DK, N2, 1, 1), dKt, dDY2, oMN, oMN, false);
+                mma_commit(&bars.d4_full);
+                if (!mbar_wait(&bars.mq_full, c & 1, status)) { fail(); break; }
+                mma_steps<C / 16>(tb + LY::cD3, idesc_bf16(128, N2, 0, 1), dMH, dY2, oK0, oMN, false);
+                mma_steps<C / 16>(tb + LY::cD3, idesc_bf16(128, BV, 0, 1), dML, dY2, oK0, oMN, true);
+                mma_commit(&bars.d3_full);
+                mma_commit(&bars.mq_empty);
+                mma_commit(&bars.empty[c & 1]);
+            }
         }
-        if (!mma_done()) break;
-        if (tid == 0 && c + 1 < nch) load_t2(c + 1);  // the T2 tiles are free again
-        float qs[BV];  // rows 0..63 (warps 0-1): QS;  rows 64..127 (warps 2-3): X_s - U = -Y
-        ld_pair_sum<BV>(tb, warp, LY::cD1, qs);
-        if (warp >= 2) {
-            const int t = tid - 64;
-            float y[BV];
+    } else {
+        // ---------------- epilogue: warps 0-3 ----------------
+        __nv_bfloat16 *o = (__nv_bfloat16 *)p.o;
+        float *sGam = (float *)(sm + LY::GATES);
+        float *sD = sGam + C;
+        const bool own_d = (DK == 128) ? true : (lane < 16);
+        const int d_row = (DK == 128) ? tid : (16 * warp + lane);
+        float Sreg[BV];
 #pragma unroll
-            for (int j = 0; j < BV; ++j) y[j] = -qs[j];
-            store_row_pair<BV>(sm + LY::Y, LY::Y_BLK, t, y);
-            const float dd = sD[t];
+        for (int j = 0; j < BV; ++j) Sreg[j] = 0.f;
+        if (own_d && p.S0) {
 #pragma unroll
-            for (int j = 0; j < BV; ++j) y[j] *= dd;
-            store_row_pair<BV>(sm + LY::DY, LY::Y_BLK, t, y);
+            for (int j = 0; j < BV; ++j) Sreg[j] = p.S0[(head * dv + v0 + j) * DK + d_row];
         }
-        ok = mbar_wait(&mq_bar, c & 1, p.status);
-        if (!fail_sync(ok)) break;
-        sync_for_mma();
-
-        // round 2: D3 = [Mqk_hi; 0][Y_hi | Y_lo] + [Mqk_lo; 0] Y_hi ;  D4 = K^T [DY_hi | DY_lo]
-        if (tid == 0) {
-            mma_steps<C / 16>(tb + LY::cD3, idesc_bf16(128, N2, 0, 1), dMH, dY2, oK0, oMN, false);
-            mma_steps<C / 16>(tb + LY::cD3, idesc_bf16(128, BV, 0, 1), dML, dY2, oK0, oMN, true);
-            const uint64_t dKt = make_desc(bb + LY::B_KQW, LY::KQW_BLK, 1024, 2);
-            mma_steps<C / 16>(tb + LY::cD4, idesc_bf16(DK, N2, 1, 1), dKt, dDY2, oMN, oMN, false);
-        }
-        if (!mma_done()) break;
-        if (tid == 0 && c + 1 < nch) load_mq(c + 1);  // the Mqk tiles are free again
-        if (warp < 2) {
-            float x[BV];
-            ld_pair_sum<BV>(tb, warp, LY::cD3, x);
-            const int t = tid;
-            if (t < n) {
-                const float gt = sGam[t];
-                __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t) * H + h) * dv + v0;
+        if (own_d) store_row_pair<BV>(sm + LY::S, LY::S_BLK, d_row, Sreg);
+        fence_async_smem();
+        named_sync(1, EPI_THREADS);
+        if (tid == 0) mbar_arrive(&bars.s_ready);
+        for (int c = 0; c < nch; ++c) {
+            const int c0 = c * C, n = min(C, T - c0);
+            const uint8_t *buf = sm + (c & 1) * LY::BUF;
+            if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status)) { fail(); break; }
+            const float *g = reinterpret_cast<const float *>(buf + LY::B_G);
+            const float g_last = g[C - 1];
+            if (tid < C) {
+                sGam[tid] = __expf(g[tid]);
+                sD[tid] = tid < n ? __expf(g_last - g[tid]) : 0.f;
+            }
+            named_sync(1, EPI_THREADS);
+            if (tid == 0) mbar_arrive(&bars.empty[c & 1]);  // g has been read
+            // Y = U - X_s (rows 64..127 of D1), QS (rows 0..63)
+            if (!mbar_wait(&bars.d1_full, c & 1, status)) { fail(); break; }
+            fence_after_sync();
+            float qs[BV];
+            ld_pair_sum<BV>(tb, warp, LY::cD1, qs);
+            if (warp >= 2) {
+                const int t = tid - 64;
+                float y[BV];
+                ld_row<BV>(tb, warp, LY::cU, y);  // -U
 #pragma unroll
-                for (int c8 = 0; c8 < BV / 8; ++c8) {
-                    float r[8];
+                for (int j = 0; j < BV; ++j) y[j] = -(qs[j] + y[j]);
+                store_row_pair<BV>(sm + LY::Y, LY::Y_BLK, t, y);
+                const float dd = sD[t];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) r[j] = fmaf(gt, qs[c8 * 8 + j], x[c8 * 8 + j]);
-                    uint4 pk;
-                    pk.x = pack_bf16(r[0], r[1]);
-                    pk.y = pack_bf16(r[2], r[3]);
-                    pk.z = pack_bf16(r[4], r[5]);
-                    pk.w = pack_bf16(r[6], r[7]);
-                    *reinterpret_cast<uint4 *>(dst + c8 * 8) = pk;
+                for (int j = 0; j < BV; ++j) y[j] *= dd;
+                store_row_pair<BV>(sm + LY::DY, LY::Y_BLK, t, y);
+            }
+            fence_async_smem();
+            fence_before_sync();
+            named_sync(1, EPI_THREADS);
+            if (tid == 0) mbar_arrive(&bars.y_ready);
+            // state update S^T <- e^{g_n} S^T + K^T D Y
+            if (!mbar_wait(&bars.d4_full, c & 1, status)) { fail(); break; }
+            fence_after_sync();
+            {
+                float x[BV];
+                ld_pair_sum<BV>(tb, warp, LY::cD4, x);
+                const float gC = __expf(g_last);
+                if (own_d) {
+#pragma unroll
+                    for (int j = 0; j < BV; ++j) Sreg[j] = fmaf(gC, Sreg[j], x[j]);
+                    store_row_pair<BV>(sm + LY::S, LY::S_BLK, d_row, Sreg);
                 }
             }
-        }
-        {
-            float x[BV];
-            ld_pair_sum<BV>(tb, warp, LY::cD4, x);
-            const float gC = __expf(g_last);
-            if (own_d) {
+            fence_async_smem();
+            fence_before_sync();
+            named_sync(1, EPI_THREADS);
+            if (tid == 0) mbar_arrive(&bars.s_ready);
+            // output O = diag(e^g) QS + Mqk Y (overlaps the next chunk's first MMAs)
+            if (!mbar_wait(&bars.d3_full, c & 1, status)) { fail(); break; }
+            fence_after_sync();
+            if (warp < 2) {
+                float x[BV];
+                ld_pair_sum<BV>(tb, warp, LY::cD3, x);
+                const int t = tid;
+                if (t < n) {
+                    const float gt = sGam[t];
+                    __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t) * H + h) * dv + v0;
 #pragma unroll
-                for (int j = 0; j < BV; ++j) Sreg[j] = fmaf(gC, Sreg[j], x[j]);
-                store_row_pair<BV>(sm + LY::S, LY::S_BLK, d_row, Sreg);
+                    for (int c8 = 0; c8 < BV / 8; ++c8) {
+                        float r[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) r[j] = fmaf(gt, qs[c8 * 8 + j], x[c8 * 8 + j]);
+                        uint4 pk;
+                        pk.x = pack_bf16(r[0], r[1]);
+                        pk.y = pack_bf16(r[2], r[3]);
+                        pk.z = pack_bf16(r[4], r[5]);
+                        pk.w = pack_bf16(r[6], r[7]);
+                        *reinterpret_cast<uint4 *>(dst + c8 * 8) = pk;
+                    }
+                }
             }
+            fence_before_sync();
+            named_sync(1, EPI_THREADS);  // D3 read before the next chunk's round 2 overwrites it
         }
-        sync_for_mma();
-    }
-
-    if (p.S_final && own_d && failed_sh == 0) {
+        if (p.S_final && own_d && !failed()) {
 #pragma unroll
-        for (int j = 0; j < BV; ++j) p.S_final[(head * dv + v0 + j) * DK + d_row] = Sreg[j];
+            for (int j = 0; j < BV; ++j) p.S_final[(head * dv + v0 + j) * DK + d_row] = Sreg[j];
+        }
     }
     fence_before_sync();
     __syncthreads();
@@ -556,7 +594,7 @@ cudaError_t launch_gdn(const ScanArgs &a, void *ws, cudaStream_t s) {
                                                (int)LY::BYTES);
         if (err != cudaSuccess) return err;
         dim3 grid(a.dv / BV, a.H, a.B);
-        kern<<<grid, NT, LY::BYTES, s>>>(a, maps, (const uint8_t *)ws, nch);
+        kern<<<grid, ST_THREADS, LY::BYTES, s>>>(a, maps, (const uint8_t *)ws, nch);
         return cudaGetLastError();
     }
 }
