@@ -9,6 +9,7 @@
 namespace prism {
 cudaError_t launch_scan_simt(const ScanArgs &a, bool io_f32, cudaStream_t s);
 cudaError_t launch_decode(const ScanArgs &a, bool io_f32, cudaStream_t s);
+cudaError_t decode_status(uint32_t *out);
 bool scan_tc_supported(const ScanArgs &a, bool io_f32);
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
 size_t gdn_workspace_bytes(int B, int H, int T, int dk);
@@ -141,16 +142,19 @@ prism_status prism_step_decode(const prism_shape *shape, const void *q, const vo
 }
 
 prism_status prism_query_device_status(void *workspace, void *stream) {
-    if (!workspace) return PRISM_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     if (cudaStreamSynchronize(s) != cudaSuccess) return PRISM_ERR_CUDA;
     uint32_t word = 0;
-    if (cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
-        return PRISM_ERR_CUDA;
-    if (word != PRISM_OK) {
-        if (cudaMemset(workspace, 0, sizeof word) != cudaSuccess) return PRISM_ERR_CUDA;
+    if (workspace) {
+        if (cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return PRISM_ERR_CUDA;
+        if (word != PRISM_OK && cudaMemset(workspace, 0, sizeof word) != cudaSuccess)
+            return PRISM_ERR_CUDA;
     }
-    return word == PRISM_OK ? PRISM_OK : (prism_status)word;
+    uint32_t dword = 0;
+    if (prism::decode_status(&dword) != cudaSuccess) return PRISM_ERR_CUDA;
+    if (word == PRISM_OK) word = dword;
+    return (prism_status)word;
 }
 
 const char *prism_status_string(prism_status status) {

@@ -136,9 +136,10 @@ prism_status prism_scan_fwd_noalloc(const prism_shape *shape, const void *q, con
                                     float *S_final, void *stream);
 
 /*
- * prism_query_device_status -- synchronise `stream`, read the status word in `workspace`
- * (written by kernels whose bounded waits ran out) and clear it.  Returns PRISM_OK,
- * PRISM_ERR_TIMEOUT, or PRISM_ERR_CUDA if the stream itself reports an error.
+ * prism_query_device_status -- synchronise `stream`, read the status word in `workspace` (written
+ * by scan kernels whose bounded waits ran out; workspace may be NULL) and the library's decode
+ * status word, and clear them.  Returns PRISM_OK, PRISM_ERR_TIMEOUT, or PRISM_ERR_CUDA if the
+ * stream itself reports an error.
  */
 prism_status prism_query_device_status(void *workspace, void *stream);
 
