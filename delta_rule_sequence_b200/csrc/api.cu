@@ -14,6 +14,10 @@ bool scan_tc_supported(const ScanArgs &a, bool io_f32);
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
 size_t gdn_workspace_bytes(int B, int H, int T, int dk);
 cudaError_t launch_scan_gdn(const ScanArgs &a, void *ws, cudaStream_t s);
+int segmented_combine_launches(int G, bool with_state);
+size_t segmented_extra_bytes(int B, int H, int G, int dk, int dv);
+cudaError_t launch_segmented(const ScanArgs &a, int route, bool io_f32, int G, void *ws,
+                             size_t rec_bytes, cudaStream_t s);
 }  // namespace prism
 
 namespace {
@@ -56,6 +60,49 @@ Plan plan_for(const prism_shape *s, bool gdn_write) {
     return gdn_write ? Plan::TcGdnSplit : Plan::TcFused;
 }
 
+// Debug flag bits (prism_debug_set_flags): 2 = take the segmented scan whenever the shape allows
+// it, 4 = never take it.
+constexpr int kForceSegments = 2, kNoSegments = 4;
+
+// Number of segments G of the segmented inter-chunk scan (1 = one in-order pass per sequence).
+// It needs dk == dv (the identity pass) and T divisible by G with at least one chunk per segment.
+int sm_count() {
+    static int sms[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        sms[dev] = n;
+    }
+    return sms[dev];
+}
+
+// Measured on B200: on the Gated-DeltaNet route (whose in-order pass is latency-bound per chunk),
+// cutting 16 sequence slices of 65536 tokens into 16 segments halves the time; on the fused rank-L
+// route (one CTA per SM) the tripled work of the segmented scan does not pay.  So segments are
+// taken on the Gated-DeltaNet route when the in-order passes fill at most a quarter of the SMs.
+int segments_for(const prism_shape *s, bool gdn_write) {
+    if ((g_debug_flags & kNoSegments) || s->dk != s->dv || s->T < 128) return 1;
+    auto largest_G = [&](int max_g, int min_len) {
+        for (int G = 16; G >= 2; G /= 2)
+            if (G <= max_g && s->T % G == 0 && s->T / G >= min_len) return G;
+        return 1;
+    };
+    if (g_debug_flags & kForceSegments) return largest_G(16, 64);
+    if (plan_for(s, gdn_write) != Plan::TcGdnSplit) return 1;
+    const long long chains = (long long)s->B * s->H * (s->dv == 128 ? 4 : 1);
+    const int sms = sm_count();
+    if (chains * 4 > sms || s->T < 4096) return 1;
+    return largest_G((int)(sms / chains), 256);
+}
+
+size_t records_bytes(const prism_shape *s, Plan plan, int G) {
+    if (plan != Plan::TcGdnSplit || s->T <= 0 || s->B == 0 || s->H == 0) return prism::kStatusBytes;
+    return prism::gdn_workspace_bytes(s->B * G, s->H, s->T / G, s->dk);
+}
+
 prism::ScanArgs make_args(const prism_shape *s, const void *q, const void *k, const void *v,
                           const float *alpha, const float *beta, const void *u, const void *w,
                           const float *S0, void *o, float *S_final, uint32_t *status) {
@@ -64,6 +111,7 @@ prism::ScanArgs make_args(const prism_shape *s, const void *q, const void *k, co
     a.chunk = s->chunk;
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.u = u; a.w = w;
     a.S0 = S0; a.o = o; a.S_final = S_final; a.status = status;
+    a.flags = 0;
     return a;
 }
 
@@ -75,18 +123,21 @@ extern "C" {
 // when u, w are NULL, rank-L otherwise), since the shape alone does not say which one is used.
 prism_status prism_scan_fwd_workspace_size(const prism_shape *shape, size_t *bytes) {
     if (!shape || !bytes) return PRISM_ERR_INVALID_ARG;
-    size_t need = prism::kStatusBytes;
-    if (shape->B > 0 && shape->H > 0 && shape->T > 0 && shape->L == 1 &&
-        plan_for(shape, true) == Plan::TcGdnSplit)
-        need = prism::gdn_workspace_bytes(shape->B, shape->H, shape->T, shape->dk);
+    const Plan plan = plan_for(shape, shape->L == 1);
+    const int G = segments_for(shape, shape->L == 1);
+    size_t need = records_bytes(shape, plan, G);
+    if (G > 1) need += prism::segmented_extra_bytes(shape->B, shape->H, G, shape->dk, shape->dv);
     *bytes = need;
     return PRISM_OK;
 }
 
 prism_status prism_scan_fwd_launch_count(const prism_shape *shape, int *launches) {
     if (!shape || !launches) return PRISM_ERR_INVALID_ARG;
-    int n = 1;
-    if (shape->L == 1 && plan_for(shape, true) == Plan::TcGdnSplit && shape->T > 0) n = 2;
+    const Plan plan = plan_for(shape, shape->L == 1);
+    const int G = segments_for(shape, shape->L == 1);
+    const bool split = plan == Plan::TcGdnSplit && shape->T > 0;
+    int n = split ? 2 : 1;
+    if (G > 1) n = (split ? 1 : 0) + 3 + prism::segmented_combine_launches(G, true);
     if (shape->B == 0 || shape->H == 0) n = 0;
     *launches = n;
     return PRISM_OK;
@@ -115,7 +166,14 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
     prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, S0, o, S_final, status);
     const bool io_f32 = shape->io == PRISM_F32;
     cudaError_t err;
-    switch (plan_for(shape, u == nullptr)) {
+    const Plan plan = plan_for(shape, u == nullptr);
+    const int G = segments_for(shape, u == nullptr);
+    if (G > 1) {
+        const int route = plan == Plan::TcGdnSplit ? 2 : plan == Plan::TcFused ? 1 : 0;
+        err = prism::launch_segmented(a, route, io_f32, G, workspace, records_bytes(shape, plan, G), s);
+        return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+    }
+    switch (plan) {
         case Plan::TcGdnSplit:
             err = shape->T > 0 ? prism::launch_scan_gdn(a, workspace, s)
                                : prism::launch_scan_tc(a, s);  // T = 0: copies S0 to S_final

@@ -19,7 +19,13 @@ struct ScanArgs {
     void *o;
     float *S_final;
     uint32_t *status;  // device status word (PRISM_OK / PRISM_ERR_TIMEOUT), may be null
+    int flags;         // kNoWrite | kS0Identity | kNoOutput (segment passes of the segmented scan)
 };
+
+// Flags of a scan pass.  kNoWrite: the write term is zero (u = 0 / v = 0);  kS0Identity: the entry
+// state's row r is the unit vector e_r (requires dk == dv), so S_final returns the pass's affine
+// map E;  kNoOutput: o is not written.
+enum : int { kNoWrite = 1, kS0Identity = 2, kNoOutput = 4 };
 
 // Workspace layout: [0, 256) status block; segment data of the segmented scan after it.
 constexpr size_t kStatusBytes = 256;

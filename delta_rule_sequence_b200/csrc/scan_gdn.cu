@@ -444,7 +444,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
         float Sreg[BV];
 #pragma unroll
         for (int j = 0; j < BV; ++j) Sreg[j] = 0.f;
-        if (own_d && p.S0) {
+        if (own_d && (p.flags & kS0Identity)) {
+#pragma unroll
+            for (int j = 0; j < BV; ++j) Sreg[j] = (v0 + j == d_row) ? 1.f : 0.f;
+        } else if (own_d && p.S0) {
 #pragma unroll
             for (int j = 0; j < BV; ++j) Sreg[j] = p.S0[(head * dv + v0 + j) * DK + d_row];
         }
@@ -473,8 +476,9 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 const int t = tid - 64;
                 float y[BV];
                 ld_row<BV>(tb, warp, LY::cU, y);  // -U
+                const bool wr = !(p.flags & kNoWrite);
 #pragma unroll
-                for (int j = 0; j < BV; ++j) y[j] = -(qs[j] + y[j]);
+                for (int j = 0; j < BV; ++j) y[j] = -(qs[j] + (wr ? y[j] : 0.f));
                 store_row_pair<BV>(sm + LY::Y, LY::Y_BLK, t, y);
                 const float dd = sD[t];
 #pragma unroll
@@ -509,7 +513,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 float x[BV];
                 ld_pair_sum<BV>(tb, warp, LY::cD3, x);
                 const int t = tid;
-                if (t < n) {
+                if (t < n && !(p.flags & kNoOutput)) {
                     const float gt = sGam[t];
                     __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t) * H + h) * dv + v0;
 #pragma unroll
@@ -569,34 +573,38 @@ bool act_map(CUtensorMap *m, const void *base, int B, int T, int H, int d, int b
 }
 
 template <int DK, int BV>
-cudaError_t launch_gdn(const ScanArgs &a, void *ws, cudaStream_t s) {
+bool gdn_maps(const ScanArgs &a, GdnMaps *maps) {
+    return act_map(&maps->k, a.k, a.B, a.T, a.H, DK, 64) && act_map(&maps->q, a.q, a.B, a.T, a.H, DK, 64) &&
+           act_map(&maps->v, a.v, a.B, a.T, a.H, a.dv, BV);
+}
+
+template <int DK, int BV>
+cudaError_t launch_gdn_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
     const int nch = (a.T + C - 1) / C;
     GdnMaps maps;
-    if (!act_map(&maps.k, a.k, a.B, a.T, a.H, DK, 64) || !act_map(&maps.q, a.q, a.B, a.T, a.H, DK, 64) ||
-        !act_map(&maps.v, a.v, a.B, a.T, a.H, a.dv, BV))
-        return cudaErrorInvalidValue;
-    {
-        using LY = PrepLayout<DK>;
-        auto kern = gdn_prep_kernel<DK>;
-        cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)LY::BYTES);
-        if (err != cudaSuccess) return err;
-        dim3 grid(nch, a.H, a.B);
-        kern<<<grid, NT, LY::BYTES, s>>>(a, maps, (uint8_t *)ws, nch);
-        err = cudaGetLastError();
-        if (err != cudaSuccess) return err;
-    }
-    {
-        using LY = StateLayout<DK, BV>;
-        static_assert(LY::BYTES <= 227 * 1024, "shared memory budget");
-        auto kern = gdn_state_kernel<DK, BV>;
-        cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)LY::BYTES);
-        if (err != cudaSuccess) return err;
-        dim3 grid(a.dv / BV, a.H, a.B);
-        kern<<<grid, ST_THREADS, LY::BYTES, s>>>(a, maps, (const uint8_t *)ws, nch);
-        return cudaGetLastError();
-    }
+    if (!gdn_maps<DK, BV>(a, &maps)) return cudaErrorInvalidValue;
+    using LY = PrepLayout<DK>;
+    auto kern = gdn_prep_kernel<DK>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
+    if (err != cudaSuccess) return err;
+    dim3 grid(nch, a.H, a.B);
+    kern<<<grid, NT, LY::BYTES, s>>>(a, maps, (uint8_t *)ws, nch);
+    return cudaGetLastError();
+}
+
+template <int DK, int BV>
+cudaError_t launch_gdn_state_t(const ScanArgs &a, const void *ws, cudaStream_t s) {
+    const int nch = (a.T + C - 1) / C;
+    GdnMaps maps;
+    if (!gdn_maps<DK, BV>(a, &maps)) return cudaErrorInvalidValue;
+    using LY = StateLayout<DK, BV>;
+    static_assert(LY::BYTES <= 227 * 1024, "shared memory budget");
+    auto kern = gdn_state_kernel<DK, BV>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
+    if (err != cudaSuccess) return err;
+    dim3 grid(a.dv / BV, a.H, a.B);
+    kern<<<grid, ST_THREADS, LY::BYTES, s>>>(a, maps, (const uint8_t *)ws, nch);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -608,9 +616,21 @@ size_t gdn_workspace_bytes(int B, int H, int T, int dk) {
     return kRecOffset + (size_t)B * H * nch * rec;
 }
 
+// The per-chunk records (prep) and the in-order pass over them (state); records depend only on
+// q, k, alpha, beta, so several state passes over the same tokens can share one prep.
+cudaError_t launch_gdn_prep(const ScanArgs &a, void *ws, cudaStream_t s) {
+    if (a.T <= 0) return cudaSuccess;
+    return a.dk == 128 ? launch_gdn_prep_t<128, 32>(a, ws, s) : launch_gdn_prep_t<64, 64>(a, ws, s);
+}
+
+cudaError_t launch_gdn_state(const ScanArgs &a, const void *ws, cudaStream_t s) {
+    return a.dk == 128 ? launch_gdn_state_t<128, 32>(a, ws, s) : launch_gdn_state_t<64, 64>(a, ws, s);
+}
+
 cudaError_t launch_scan_gdn(const ScanArgs &a, void *ws, cudaStream_t s) {
-    if (a.dk == 128) return launch_gdn<128, 32>(a, ws, s);
-    return launch_gdn<64, 64>(a, ws, s);
+    cudaError_t err = launch_gdn_prep(a, ws, s);
+    if (err != cudaSuccess) return err;
+    return launch_gdn_state(a, ws, s);
 }
 
 }  // namespace prism

@@ -67,7 +67,8 @@ __global__ void __launch_bounds__(NT) scan_simt_kernel(ScanArgs p) {
     for (int e = tid; e < BV * DK; e += NT) {
         int r = e / DK, j = e % DK;
         float s = 0.f;
-        if (p.S0 && r < nrows) s = p.S0[(head * dv + v0 + r) * DK + j];
+        if (p.flags & kS0Identity) s = (v0 + r == j) ? 1.f : 0.f;
+        else if (p.S0 && r < nrows) s = p.S0[(head * dv + v0 + r) * DK + j];
         sS[r * KS + j] = s;
     }
 
@@ -134,7 +135,8 @@ __global__ void __launch_bounds__(NT) scan_simt_kernel(ScanArgs p) {
         }
 
         // rank-L write terms (the Gated-DeltaNet write is u = beta v, w = k, L = 1)
-        for (int l = 0; l < L; ++l) {
+        const int Lw = (p.flags & kNoWrite) ? 0 : L;
+        for (int l = 0; l < Lw; ++l) {
             const float *Wl = gdn ? sK : sW;
             for (int e = tid; e < CS * XS; e += NT) {
                 int i = e / XS, r = e % XS;
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(NT) scan_simt_kernel(ScanArgs p) {
         // O -= Mqk X ; store o
         for (int e = tid; e < CS * BV; e += NT) {
             int t = e / BV, r = e % BV;
-            if (t < n) {
+            if (t < n && !(p.flags & kNoOutput)) {
                 float acc = sO[t * XS + r];
                 for (int i = 0; i <= t; ++i) acc = fmaf(-sM[t * GS + i], sR[i * XS + r], acc);
                 size_t bth = ((size_t)b * T + c0 + t) * H + h;

@@ -101,6 +101,8 @@ __global__ void __launch_bounds__(NT, 1) scan_tc_kernel(ScanArgs p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int v0 = blockIdx.x * BV, h = blockIdx.y, b = blockIdx.z;
     const int H = p.H, T = p.T, dv = p.dv, L = GDN ? 1 : p.L;
+    const bool wr = !(p.flags & kNoWrite);  // the write term is present
+    const bool rank_l = !GDN && wr;         // the rank-L terms X_u, O_w, F_w are present
     const __nv_bfloat16 *q = (const __nv_bfloat16 *)p.q, *k = (const __nv_bfloat16 *)p.k;
     const __nv_bfloat16 *v = (const __nv_bfloat16 *)p.v, *u = (const __nv_bfloat16 *)p.u;
     const __nv_bfloat16 *w = (const __nv_bfloat16 *)p.w;
@@ -150,7 +152,10 @@ __global__ void __launch_bounds__(NT, 1) scan_tc_kernel(ScanArgs p) {
     float Sreg[BV];
 #pragma unroll
     for (int j = 0; j < BV; ++j) Sreg[j] = 0.f;
-    if (own_d && p.S0) {
+    if (own_d && (p.flags & kS0Identity)) {
+#pragma unroll
+        for (int j = 0; j < BV; ++j) Sreg[j] = (v0 + j == d_row) ? 1.f : 0.f;
+    } else if (own_d && p.S0) {
 #pragma unroll
         for (int j = 0; j < BV; ++j) Sreg[j] = p.S0[(head * dv + v0 + j) * DK + d_row];
     }
@@ -277,7 +282,7 @@ __global__ void __launch_bounds__(NT, 1) scan_tc_kernel(ScanArgs p) {
         }
 
         // ---- rank-L write terms: sum_l P_l U_l, O_w = sum_l Mqw_l U_l, F_w = sum_l W_l^T D U_l
-        if constexpr (!GDN) {
+        if (rank_l) {
             bool ok = true;
             for (int l = 0; l < L; ++l) {
                 sync_for_mma();  // the previous MMAs have finished reading the l-tiles
@@ -375,7 +380,8 @@ __global__ void __launch_bounds__(NT, 1) scan_tc_kernel(ScanArgs p) {
                 float y[BV];
                 const float dd = sD[t_row];
 #pragma unroll
-                for (int j = 0; j < BV; ++j) y[j] = GDN ? (uu[j] - xs[j]) : -(uu[j] + xs[j]);
+                for (int j = 0; j < BV; ++j)
+                    y[j] = !wr ? -xs[j] : (GDN ? (uu[j] - xs[j]) : -(uu[j] + xs[j]));
                 store_row_split<BV>(sm + LY::Y, sm + LY::YL, t_row, y);
 #pragma unroll
                 for (int j = 0; j < BV; ++j) y[j] *= dd;
@@ -386,16 +392,16 @@ __global__ void __launch_bounds__(NT, 1) scan_tc_kernel(ScanArgs p) {
         // ---- O (+)= Mqk Y ; S'^T (+)= K^T D Y
         if (tid == 0) {
             mma_split(tb + LY::cO, idesc_bf16(64, BV, 0, 1), C / 16, dK, dVT, sb + LY::MQK,
-                      sb + LY::MQKL, sb + LY::Y, sb + LY::YL, !GDN);
+                      sb + LY::MQKL, sb + LY::Y, sb + LY::YL, rank_l);
             mma_split(tb + LY::cDS, idesc_bf16(DK, BV, 1, 1), C / 16, dKmn, dVT, sb + LY::KQW, 0,
-                      sb + LY::DY, sb + LY::DYL, !GDN);
+                      sb + LY::DY, sb + LY::DYL, rank_l);
         }
         if (!mma_done()) break;
         {
             float qs[BV], op[BV];
             ld_row<BV>(tb, warp, LY::cQS, qs);
             ld_row<BV>(tb, warp, LY::cO, op);
-            if (own_t && t_row < n) {
+            if (own_t && t_row < n && !(p.flags & kNoOutput)) {
                 const float gt = sGam[t_row];
                 __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t_row) * H + h) * dv + v0;
 #pragma unroll

@@ -147,9 +147,11 @@ prism_status prism_query_device_status(void *workspace, void *stream);
 const char *prism_status_string(prism_status status);
 
 /*
- * prism_debug_set_flags -- testing hook.  flags bit 0: the next timed-wait kernel skips one
- * producer signal so its consumer must give up and record PRISM_ERR_TIMEOUT (checks the
- * bounded-wait path without hanging anything).  Returns the previous flags.
+ * prism_debug_set_flags -- testing and measurement hook (process-wide; set it before
+ * prism_scan_fwd_workspace_size, which depends on it).  flags bit 1: prism_scan_fwd takes the
+ * segmented inter-chunk scan (segment elements, a Blelloch scan over them, a re-run of every
+ * segment) whenever the shape allows it (dk == dv, T divisible into segments of >= 64 tokens);
+ * bit 2: it never does.  Returns the previous flags.
  */
 int prism_debug_set_flags(int flags);
 
