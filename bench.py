@@ -14,7 +14,8 @@ With N > 1 (torchrun, one process per GPU) every rank processes its own batch (w
 B*H sequences are independent, so there is no collective in the data path).
 
 Besides the headline line's required keys the JSON line carries: roofline (HBM-bound; algorithmic
-bytes per launch over the measured copy bandwidth), cpu_baseline (the fp64 oracle on a bounded
+bytes per step over the summed device time of the step's launches, each launch timed by CUDA events
+the library records around it, against the measured copy bandwidth), cpu_baseline (the fp64 oracle on a bounded
 sample, rank 0 at N = 1), e2e (through the public API with pinned-host inputs copied in and the
 outputs copied back inside the timed region), clocks sampled during the timed region, and the
 decode step (B=256, H=32, d=128, L=4) as a secondary measurement.
@@ -51,19 +52,34 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
-    csrc = os.path.join(ROOT, "delta_rule_sequence_b200", "csrc")
+# The kernels a step of each bench workload launches, in launch order, and the source files each
+# is compiled from (the hash of those files keys the committed ncu traffic figures).
+STEP_KERNELS = {
+    "gdn": ["gdn_prep_kernel", "gdn_state_kernel"],
+}
+_GDN_SOURCES = ["csrc/scan_gdn.cu", "csrc/tc.cuh", "csrc/chunk_common.cuh", "csrc/common.cuh",
+                "../include/prism.h"]
+KERNEL_SOURCES = {
+    "gdn_prep_kernel": _GDN_SOURCES,
+    "gdn_state_kernel": _GDN_SOURCES,
+    "decode_kernel": ["csrc/decode.cu", "csrc/common.cuh", "../include/prism.h"],
+}
+
+
+def kernel_source_hash(kernel):
+    pkg = os.path.join(ROOT, "delta_rule_sequence_b200")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for rel in KERNEL_SOURCES[kernel]:
+        with open(os.path.normpath(os.path.join(pkg, rel)), "rb") as f:
+            h.update(os.path.basename(rel).encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
 def committed_traffic(workload, kernel):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on this source."""
-    src = kernel_source_hash()
+    if kernel not in KERNEL_SOURCES:
+        return None
+    src = kernel_source_hash(kernel)
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
         return None
@@ -366,18 +382,62 @@ def main():
         raise SystemExit(f"bench: device status after timing: {prism.status_string(status)}")
     clocks = sampler.summary(wall0, wall1)
 
-    # roofline of the dominant (only) kernel: algorithmic bytes per launch / launch duration
+    # ---- per-kernel durations: a second timed region of the same steps, launched without graphs,
+    # with the library recording CUDA events on the launching stream around every launch
+    names = STEP_KERNELS.get(wl.name, [f"launch{j}" for j in range(launches_per_step)])
+    if len(names) != launches_per_step:
+        names = [f"launch{j}" for j in range(launches_per_step)]
+    probe_steps = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(launches_per_step + 1)]
+           for _ in range(probe_steps)]
+    with torch.cuda.stream(stream):
+        for row in evs:  # record once so that every event handle exists
+            for e in row:
+                e.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    p0 = torch.cuda.Event(enable_timing=True)
+    p1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        p0.record(stream)
+        for i in range(probe_steps):
+            prism.record_launch_events(evs[i])
+            step(i, stream)
+        p1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    probe_ms_per_step = max_over_ranks(p0.elapsed_time(p1)) / probe_steps
+    launch_ms = [max_over_ranks(sum(row[j].elapsed_time(row[j + 1]) for row in evs) / probe_steps)
+                 for j in range(launches_per_step)]
+    del evs
+    kernels = []
+    for j, n in enumerate(names):
+        kernels.append({"name": n, "ms_per_launch": launch_ms[j],
+                        "share": launch_ms[j] / max(1e-12, sum(launch_ms)),
+                        "dram_bytes_per_launch": committed_traffic(wl.name, n)})
+    dominant = max(range(launches_per_step), key=lambda j: launch_ms[j])
+
+    # Roofline.  The algorithmic bytes are defined for the whole path (inputs read once, outputs
+    # and the state written once), which the step's launches share, so the roofline unit is the
+    # step: algorithmic bytes per step over the summed device time of its launches.
     alg_bytes = scan_bytes(wl)
-    kernel_ms = ms_per_step / max(1, launches_per_step)
-    achieved = alg_bytes / (kernel_ms / 1e3) / 1e9
+    step_kernel_ms = sum(launch_ms)
+    achieved = alg_bytes / (step_kernel_ms / 1e3) / 1e9
+    traffic = [k["dram_bytes_per_launch"] for k in kernels]
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"],
-                "traffic": committed_traffic(wl.name, "scan"),
-                "peak_kind": f"{peaks_kind} copy bandwidth",
-                "algorithmic_bytes_per_launch": alg_bytes,
-                "algorithmic_flops_per_launch": scan_flops(wl),
-                "tensor_frac_algorithmic": scan_flops(wl) / (kernel_ms / 1e3) / 1e12
-                / peaks["bf16_tflops"]}
+                "traffic": sum(traffic) if all(t is not None for t in traffic) else None,
+                "peak_kind": f"{peaks_kind} copy bandwidth (burst)",
+                "unit_of_work": "one step: " + " + ".join(names),
+                "dominant_kernel": names[dominant],
+                "kernels": kernels,
+                "algorithmic_bytes_per_step": alg_bytes,
+                "algorithmic_flops_per_step": scan_flops(wl),
+                "tensor_frac_algorithmic": scan_flops(wl) / (step_kernel_ms / 1e3) / 1e12
+                / peaks["bf16_tflops"],
+                "timing": f"CUDA events recorded by the library on the launching stream around "
+                          f"each launch, {probe_steps} steps without graphs "
+                          f"({probe_ms_per_step:.4f} ms/step there)"}
 
     # ---- end to end through the public API: pinned host inputs in, outputs back, every step
     e2e = None

@@ -24,6 +24,21 @@ namespace {
 
 int g_debug_flags = 0;
 
+// Armed launch probe of this host thread: the events to record before each launch of the next
+// prism_scan_fwd / prism_step_decode call, and after its last launch.
+constexpr int kMaxProbeEvents = 64;
+struct LaunchProbe {
+    void *events[kMaxProbeEvents] = {};  // copied from the caller: its array need not outlive the arming call
+    int n = 0, next = 0;
+};
+thread_local LaunchProbe t_probe;
+
+// Records the probe's last event after a probed call's final launch and disarms the probe.
+void probe_finish(cudaStream_t s) {
+    prism::launch_probe_mark(s);
+    t_probe = LaunchProbe{};
+}
+
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 bool width_ok(int d) { return d == 32 || d == 64 || d == 128; }
 
@@ -117,6 +132,13 @@ prism::ScanArgs make_args(const prism_shape *s, const void *q, const void *k, co
 
 }  // namespace
 
+namespace prism {
+void launch_probe_mark(cudaStream_t s) {
+    LaunchProbe &p = t_probe;
+    if (p.next < p.n) cudaEventRecord((cudaEvent_t)p.events[p.next++], s);
+}
+}  // namespace prism
+
 extern "C" {
 
 // The workspace and launch count cover the larger of the two write forms (Gated-DeltaNet write
@@ -171,16 +193,17 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
     if (G > 1) {
         const int route = plan == Plan::TcGdnSplit ? 2 : plan == Plan::TcFused ? 1 : 0;
         err = prism::launch_segmented(a, route, io_f32, G, workspace, records_bytes(shape, plan, G), s);
-        return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+    } else {
+        switch (plan) {
+            case Plan::TcGdnSplit:
+                err = shape->T > 0 ? prism::launch_scan_gdn(a, workspace, s)
+                                   : prism::launch_scan_tc(a, s);  // T = 0: copies S0 to S_final
+                break;
+            case Plan::TcFused: err = prism::launch_scan_tc(a, s); break;
+            default: err = prism::launch_scan_simt(a, io_f32, s); break;
+        }
     }
-    switch (plan) {
-        case Plan::TcGdnSplit:
-            err = shape->T > 0 ? prism::launch_scan_gdn(a, workspace, s)
-                               : prism::launch_scan_tc(a, s);  // T = 0: copies S0 to S_final
-            break;
-        case Plan::TcFused: err = prism::launch_scan_tc(a, s); break;
-        default: err = prism::launch_scan_simt(a, io_f32, s); break;
-    }
+    probe_finish(s);
     return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 
@@ -196,6 +219,7 @@ prism_status prism_step_decode(const prism_shape *shape, const void *q, const vo
     if ((long long)shape->B * shape->H > 0x7fffffffLL) return PRISM_ERR_UNSUPPORTED;
     prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, nullptr, o, S, nullptr);
     cudaError_t err = prism::launch_decode(a, shape->io == PRISM_F32, (cudaStream_t)stream);
+    probe_finish((cudaStream_t)stream);
     return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 
@@ -230,6 +254,17 @@ int prism_debug_set_flags(int flags) {
     int old = g_debug_flags;
     g_debug_flags = flags;
     return old;
+}
+
+prism_status prism_debug_record_launch_events(void *const *events, int n_events) {
+    if (n_events < 0 || (n_events > 0 && !events)) return PRISM_ERR_INVALID_ARG;
+    if (n_events > kMaxProbeEvents) return PRISM_ERR_UNSUPPORTED;
+    for (int i = 0; i < n_events; ++i)
+        if (!events[i]) return PRISM_ERR_INVALID_ARG;
+    t_probe = LaunchProbe{};
+    for (int i = 0; i < n_events; ++i) t_probe.events[i] = events[i];
+    t_probe.n = n_events;
+    return PRISM_OK;
 }
 
 }  // extern "C"

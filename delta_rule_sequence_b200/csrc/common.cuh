@@ -63,6 +63,10 @@ __device__ __forceinline__ float warp_inclusive_scan(float x, int lane) {
     return x;
 }
 
+// Launch probe (prism_debug_record_launch_events): records the caller's next event on the stream
+// right before a kernel launch of an armed call.  Every launcher calls it before each launch.
+void launch_probe_mark(cudaStream_t s);
+
 // Record a device-side failure without trapping: the first failure wins.
 __device__ __forceinline__ void record_status(uint32_t *status, uint32_t code) {
     if (status) atomicCAS(status, (uint32_t)PRISM_OK, code);

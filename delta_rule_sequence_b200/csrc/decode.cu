@@ -163,6 +163,7 @@ __global__ void __launch_bounds__(NT, 3) decode_kernel(ScanArgs p) {
 
 template <typename IO, int DK, int LW>
 cudaError_t launch_decode_l(const ScanArgs &a, cudaStream_t s) {
+    launch_probe_mark(s);
     decode_kernel<IO, DK, LW><<<a.B * a.H, NT, 0, s>>>(a);
     return cudaGetLastError();
 }

@@ -588,6 +588,7 @@ cudaError_t launch_gdn_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
     if (err != cudaSuccess) return err;
     dim3 grid(nch, a.H, a.B);
+    launch_probe_mark(s);
     kern<<<grid, NT, LY::BYTES, s>>>(a, maps, (uint8_t *)ws, nch);
     return cudaGetLastError();
 }
@@ -603,6 +604,7 @@ cudaError_t launch_gdn_state_t(const ScanArgs &a, const void *ws, cudaStream_t s
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
     if (err != cudaSuccess) return err;
     dim3 grid(a.dv / BV, a.H, a.B);
+    launch_probe_mark(s);
     kern<<<grid, ST_THREADS, LY::BYTES, s>>>(a, maps, (const uint8_t *)ws, nch);
     return cudaGetLastError();
 }

@@ -243,6 +243,7 @@ cudaError_t launch_simt_dk(const ScanArgs &a, cudaStream_t s) {
                                            (int)bytes);
     if (err != cudaSuccess) return err;
     dim3 grid(a.dv / BV, a.H, a.B);
+    launch_probe_mark(s);
     kern<<<grid, NT, bytes, s>>>(a);
     return cudaGetLastError();
 }

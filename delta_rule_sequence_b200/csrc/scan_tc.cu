@@ -445,6 +445,7 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t s) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (err != cudaSuccess) return err;
     dim3 grid(a.dv / BV, a.H, a.B);
+    launch_probe_mark(s);
     kern<<<grid, NT, bytes, s>>>(a);
     return cudaGetLastError();
 }

@@ -165,12 +165,20 @@ cudaError_t combine(const SegTree &t, const float *S0, float *S_final, cudaStrea
     int levels = 0;
     while ((1 << levels) < t.G) ++levels;
     const int iblocks = (int)(((size_t)t.dv * t.dk + 1023) / 1024);
+    launch_probe_mark(s);
     seg_init_kernel<<<dim3(iblocks, 1, BH), NTH, 0, s>>>(t, S0);
-    for (int lv = 1; lv < levels; ++lv)  // up-sweep (the root's element is not needed)
+    for (int lv = 1; lv < levels; ++lv) {  // up-sweep (the root's element is not needed)
+        launch_probe_mark(s);
         seg_compose_kernel<D><<<dim3(eblocks + vblocks, t.G >> lv, BH), NTH, smem, s>>>(t, lv);
-    for (int lv = levels; lv >= 1; --lv)  // down-sweep, root to leaves
+    }
+    for (int lv = levels; lv >= 1; --lv) {  // down-sweep, root to leaves
+        launch_probe_mark(s);
         seg_apply_kernel<D><<<dim3(vblocks, t.G >> lv, BH), NTH, smem, s>>>(t, lv);
-    if (S_final) seg_exit_kernel<D><<<dim3(vblocks, 1, BH), NTH, smem, s>>>(t, S_final);
+    }
+    if (S_final) {
+        launch_probe_mark(s);
+        seg_exit_kernel<D><<<dim3(vblocks, 1, BH), NTH, smem, s>>>(t, S_final);
+    }
     return cudaGetLastError();
 }
 

@@ -28,6 +28,7 @@ EXPORTS = (
     "prism_query_device_status",
     "prism_status_string",
     "prism_debug_set_flags",
+    "prism_debug_record_launch_events",
 )
 
 
@@ -73,6 +74,8 @@ def load_library():
     lib.prism_status_string.restype = ctypes.c_char_p
     lib.prism_debug_set_flags.argtypes = [ci]
     lib.prism_debug_set_flags.restype = ci
+    lib.prism_debug_record_launch_events.argtypes = [ctypes.POINTER(vp), ci]
+    lib.prism_debug_record_launch_events.restype = ci
     _lib = lib
     return lib
 
@@ -241,3 +244,13 @@ def prism_scan_fwd_launch_count(shape: PrismShape) -> int:
 def prism_query_device_status(workspace, stream=None) -> int:
     """Synchronise and return (and clear) the status word kernels wrote into `workspace`."""
     return load_library().prism_query_device_status(_ptr(workspace), _stream(stream))
+
+
+def record_launch_events(events) -> None:
+    """Arm this thread's next prism_scan_fwd / prism_step_decode call to record events[j] (torch
+    CUDA events, already recorded once so that their handles exist) before its launch j and the
+    last one after its final launch."""
+    handles = (ctypes.c_void_p * max(1, len(events)))(*[e.cuda_event for e in events])
+    rc = load_library().prism_debug_record_launch_events(handles, len(events))
+    if rc != PRISM_OK:
+        raise PrismError(rc, "prism_debug_record_launch_events")

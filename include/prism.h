@@ -155,6 +155,19 @@ const char *prism_status_string(prism_status status);
  */
 int prism_debug_set_flags(int flags);
 
+/*
+ * prism_debug_record_launch_events -- measurement hook.  Arms the calling host thread's next
+ * prism_scan_fwd or prism_step_decode call to record events[j] (cudaEvent_t handles owned by the
+ * caller, created on the stream's device) on its stream right before its kernel launch j, and one
+ * more event after its last launch, for as many events as n_events allows (a call makes
+ * prism_scan_fwd_launch_count() launches, so n_events = launches + 1 brackets every one).  The
+ * probe is disarmed by that call, whatever it returns; n_events = 0 disarms it.  The handles are
+ * copied: the array need not outlive this call, the events must outlive the probed call.  Event
+ * record errors are not reported.  Returns PRISM_ERR_INVALID_ARG if n_events < 0 or a handle is
+ * NULL, PRISM_ERR_UNSUPPORTED if n_events > 64.
+ */
+prism_status prism_debug_record_launch_events(void *const *events, int n_events);
+
 #ifdef __cplusplus
 }
 #endif

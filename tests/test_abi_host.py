@@ -100,6 +100,16 @@ def test_decode_rejects_bad_arguments(lib):
     assert lib.prism_step_decode(ctypes.byref(s), *bad) == P.PRISM_ERR_INVALID_ARG  # S NULL
 
 
+def test_launch_probe_arguments(lib):
+    assert lib.prism_debug_record_launch_events(None, -1) == P.PRISM_ERR_INVALID_ARG
+    assert lib.prism_debug_record_launch_events(None, 2) == P.PRISM_ERR_INVALID_ARG
+    null_handles = (ctypes.c_void_p * 2)(None, None)
+    assert lib.prism_debug_record_launch_events(null_handles, 2) == P.PRISM_ERR_INVALID_ARG
+    many = (ctypes.c_void_p * 65)(*([1] * 65))
+    assert lib.prism_debug_record_launch_events(many, 65) == P.PRISM_ERR_UNSUPPORTED
+    assert lib.prism_debug_record_launch_events(None, 0) == P.PRISM_OK  # disarm
+
+
 def test_workspace_size(lib):
     n = ctypes.c_size_t(0)
     assert lib.prism_scan_fwd_workspace_size(ctypes.byref(_shape()), ctypes.byref(n)) == 0

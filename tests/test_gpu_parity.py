@@ -125,6 +125,31 @@ def test_resume_from_state_matches_one_pass():
         compare("S", S2.cpu().numpy(), S.cpu().numpy(), TOL["bf16"])
 
 
+def test_launch_probe_brackets_every_launch():
+    """The events that prism_debug_record_launch_events arms are recorded around each launch of
+    the next call only (the bench times its kernels with them)."""
+    from delta_rule_sequence_b200 import prism
+
+    wl = WORKLOADS["gdn"].with_(B=1, H=2, T=512)
+    d = to_device(make_inputs(wl))
+    shape = prism.make_shape(d["q"], d["v"], None, wl.chunk)
+    n = prism.prism_scan_fwd_launch_count(shape)
+    assert n == 2
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    for e in evs:
+        e.record()
+    torch.cuda.synchronize()
+    marker = torch.cuda.Event(enable_timing=True)
+    marker.record()
+    prism.record_launch_events(evs)
+    prism.prism_scan_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], chunk=wl.chunk)
+    prism.prism_scan_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], chunk=wl.chunk)
+    torch.cuda.synchronize()
+    assert marker.elapsed_time(evs[0]) >= 0.0  # recorded after the marker, i.e. re-recorded
+    for j in range(n):
+        assert evs[j].elapsed_time(evs[j + 1]) > 0.0
+
+
 # ---------------------------------------------------------------------------------------------
 # full sizes, in the launch configuration the bench uses; sampled sequences
 
