@@ -33,6 +33,15 @@ struct LaunchProbe {
 };
 thread_local LaunchProbe t_probe;
 
+// The CUDA error behind this thread's last PRISM_ERR_CUDA (cudaSuccess if none yet).
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+prism_status cuda_status(cudaError_t err) {
+    if (err == cudaSuccess) return PRISM_OK;
+    t_last_cuda_error = err;
+    return PRISM_ERR_CUDA;
+}
+
 // Records the probe's last event after a probed call's final launch and disarms the probe.
 void probe_finish(cudaStream_t s) {
     prism::launch_probe_mark(s);
@@ -204,7 +213,7 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
         }
     }
     probe_finish(s);
-    return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+    return cuda_status(err);
 }
 
 prism_status prism_step_decode(const prism_shape *shape, const void *q, const void *k,
@@ -220,21 +229,22 @@ prism_status prism_step_decode(const prism_shape *shape, const void *q, const vo
     prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, nullptr, o, S, nullptr);
     cudaError_t err = prism::launch_decode(a, shape->io == PRISM_F32, (cudaStream_t)stream);
     probe_finish((cudaStream_t)stream);
-    return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+    return cuda_status(err);
 }
 
 prism_status prism_query_device_status(void *workspace, void *stream) {
     cudaStream_t s = (cudaStream_t)stream;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return PRISM_ERR_CUDA;
+    cudaError_t err = cudaStreamSynchronize(s);
+    if (err != cudaSuccess) return cuda_status(err);
     uint32_t word = 0;
     if (workspace) {
-        if (cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
-            return PRISM_ERR_CUDA;
-        if (word != PRISM_OK && cudaMemset(workspace, 0, sizeof word) != cudaSuccess)
-            return PRISM_ERR_CUDA;
+        if ((err = cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost)) != cudaSuccess)
+            return cuda_status(err);
+        if (word != PRISM_OK && (err = cudaMemset(workspace, 0, sizeof word)) != cudaSuccess)
+            return cuda_status(err);
     }
     uint32_t dword = 0;
-    if (prism::decode_status(&dword) != cudaSuccess) return PRISM_ERR_CUDA;
+    if ((err = prism::decode_status(&dword)) != cudaSuccess) return cuda_status(err);
     if (word == PRISM_OK) word = dword;
     return (prism_status)word;
 }
@@ -248,6 +258,10 @@ const char *prism_status_string(prism_status status) {
         case PRISM_ERR_TIMEOUT: return "PRISM_ERR_TIMEOUT";
     }
     return "PRISM_ERR_UNKNOWN";
+}
+
+const char *prism_last_cuda_error(void) {
+    return t_last_cuda_error == cudaSuccess ? "" : cudaGetErrorString(t_last_cuda_error);
 }
 
 int prism_debug_set_flags(int flags) {

@@ -4,18 +4,21 @@
 // state-dependent part.  The first depends only on the chunk's own tokens, so it runs for every
 // (batch, head, chunk) at once in `gdn_prep_kernel`, once per head (not once per value slice):
 //   G = [K; Q] K^T,   A = strict(diag(beta) Gamma o K K^T),   Mqk = incl(Gamma o Q K^T),
-//   T = (I + A)^{-1},  Wk = T diag(beta e^g) K,  and the operand T diag(beta) of U = T diag(beta) V.
-// It writes Wk (bf16), T diag(beta) and Mqk (bf16 hi/lo pairs) and g to a per-chunk record in the
-// workspace, already laid out as the 128B-swizzled shared-memory images the MMAs read.
+//   T = (I + A)^{-1},  Wk = T diag(beta e^g) K,  U = T diag(beta) V.
+// It writes Wk (bf16), Mqk (a bf16 hi/lo pair), U (fp32) and g to a per-chunk record in the
+// workspace, laid out as the shared-memory images the state kernel reads.
 // `gdn_state_kernel` then walks the chunks of one (batch, head, value slice) in order with the
 // fp32 state on chip; per chunk it prefetches the next chunk's tiles (TMA, double buffered)
-// and runs only two dependent MMA rounds:
-//   U = T diag(beta) V,  X_s = Wk S^T,  QS = Q S^T;   Y = U - X_s
-//   O = diag(e^g) QS + Mqk Y,   S'^T = e^{g_n} S^T + K^T D Y.
+// and runs two dependent MMA rounds, the second shared by the state update and the output:
+//   X_s = Wk S^T,  QS = Q S^T;   Y = U - X_s;   S'^T = e^{g_n} S^T + K^T D Y,   O = diag(e^g) QS + Mqk Y.
 // ("Sequential Parallel Duality in Prefix Scannable Models", method overview: encode all chunks
 // in parallel, then combine them in order; banbantang.com PRISM article, section 1(4): the GDN
 // forget and rank-1 write.)  Prep runs over chunks last-first, so the records the state kernel
 // needs first are the ones most recently written and most likely still in L2.
+//
+// A tcgen05.mma issued by one thread costs about 53 cycles whatever its N up to 128 (measured on
+// B200), so both kernels are shaped to issue few, wide MMAs: hi and lo halves of an operand sit
+// side by side along N, and two 64-row operands are stacked into one M = 128 instruction.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -27,34 +30,48 @@
 namespace prism {
 namespace {
 
-constexpr int NT = 128;
+constexpr int NT = 128;  // prep threads
+
+// Value-slice width of the state kernel for a key width: 4 slices of 32 at d = 128, one of 64 at
+// d = 64 (the Gated-DeltaNet route has dv = dk).
+template <int DK>
+constexpr int kBV = DK == 128 ? 32 : 64;
 
 // TMA descriptors of the bf16 activations, viewed as 4-D {d, H, T, B} (innermost first) so that
-// a box {64 | BV, 1, 64, 1} is one head's chunk; rows past T read as zeros.
+// a box {64, 1, 64, 1} is one head's chunk of 64 columns; rows past T read as zeros.
 struct GdnMaps {
     CUtensorMap k, q, v;
 };
 
-// One workspace record per (b, h, chunk): swizzled shared-memory images.
+// One workspace record per (b, h, chunk).
 template <int DK>
 struct GdnRec {
+    static constexpr int DV = DK, BV = kBV<DK>;
     static constexpr uint32_t WK_BLK = C * 128;                  // 64 rows x 128 B per 64 columns
-    static constexpr uint32_t WK = 0;                             // Wk, bf16
-    static constexpr uint32_t T2 = WK + WK_BLK * (DK / 64);       // T diag(beta), hi then lo
-    static constexpr uint32_t T2L = T2 + C * 128;
-    static constexpr uint32_t MQK = T2L + C * 128;                // Mqk, hi then lo
-    static constexpr uint32_t MQKL = MQK + C * 128;
-    static constexpr uint32_t G = MQKL + C * 128;                 // g_t, 64 floats
+    static constexpr uint32_t WK = 0;                             // Wk, bf16, K-major SW128
+    static constexpr uint32_t MQK = WK + WK_BLK * (DK / 64);      // Mqk hi (rows 0..63), lo (64..127)
+    static constexpr uint32_t U_SLICE = C * BV * 4;               // U, fp32, one value slice
+    static constexpr uint32_t U = MQK + 2 * C * 128;
+    static constexpr uint32_t G = U + U_SLICE * (DV / BV);        // g_t, 64 floats
     static constexpr uint32_t BYTES = G + 1024;
 };
 constexpr size_t kRecOffset = 1024;  // records start after the status block
+
+// Byte offset of U[t][j] in one value slice of BV fp32 columns: 16-byte chunks XORed with t % 8,
+// so that eight consecutive rows read at one column hit eight different bank groups.
+template <int BV>
+__device__ __forceinline__ uint32_t u_off(int t, int j) {
+    return (uint32_t)t * BV * 4 + ((((uint32_t)j >> 2) ^ ((uint32_t)t & 7)) << 4) + ((uint32_t)j & 3) * 4;
+}
 
 // ------------------------------------------------------------------------------------------------
 // prep: one CTA per (chunk, head, batch)
 
 template <int DK>
 struct PrepLayout {
-    static constexpr uint32_t KQ_BLK = 2 * C * 128;     // [K; Q] rows of one 64-column block
+    static constexpr uint32_t KQ_BLK = 2 * C * 128;     // [K; Q] rows of one 64-column block; V
+                                                        // replaces Q once G is done, U is staged
+                                                        // over K and V at the end
     static constexpr uint32_t KQ = 0;
     static constexpr uint32_t T1 = KQ + KQ_BLK * (DK / 64);
     static constexpr uint32_t T1L = T1 + C * 128;
@@ -62,6 +79,7 @@ struct PrepLayout {
     static constexpr uint32_t TMP = AF + C * AS * 4;
     static constexpr uint32_t GATES = TMP + 32 * 33 * 4;
     static constexpr uint32_t BYTES = GATES + 3 * C * 4 + 1024;
+    static_assert(KQ_BLK * (DK / 64) >= (uint32_t)C * DK * 4, "U staging fits over K and V");
 };
 
 template <int DK>
@@ -69,6 +87,7 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
                                                      uint8_t *ws, int nch) {
     using LY = PrepLayout<DK>;
     using RC = GdnRec<DK>;
+    constexpr int DV = RC::DV, BV = RC::BV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     __shared__ uint64_t mma_bar, ld_bar;
@@ -136,6 +155,13 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
     fence_after_sync();
     __syncthreads();
     bool ok = failed_sh == 0;  // uniform across the CTA
+    // V into the Q rows, which G no longer needs; it lands while the solve runs
+    const bool v_issued = ok;
+    if (ok && tid == 0) {
+        mbar_expect_tx(&ld_bar, (DV / 64) * C * 128);
+        for (int blk = 0; blk < DV / 64; ++blk)
+            tma_load_4d(sm + LY::KQ + blk * LY::KQ_BLK + C * 128, &maps.v, blk * 64, h, c0, b, &ld_bar);
+    }
     if (ok) {
         const int t = (warp & 1) * 32 + lane;
         const float gt = sG[t], bt = sBeta[t];
@@ -156,38 +182,35 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
                     const int i = cc + j;
                     gr[j] = (i <= t) ? __expf(gt - sG[i]) * gr[j] : 0.f;
                 }
-                store32_split(rec + RC::MQK, rec + RC::MQKL, t, cc, gr);
+                store32_split(rec + RC::MQK, rec + RC::MQK + C * 128, t, cc, gr);
             }
         }
     }
     fence_before_sync();
     __syncthreads();
-    if (ok) {
-        solve_unit_lower<NT>(sA, sA, sTmp, tid);
+    // T diag(beta scale) as a bf16 hi / lo pair into the T1 tiles (scale = e^g for Wk, 1 for U)
+    auto store_t_pair = [&](bool with_gamma) {
         for (int e = tid; e < C * (C / 8); e += NT) {
             const int t = e / (C / 8), c8 = e % (C / 8);
-            float a1[8], a2[8];
+            float a[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int i = c8 * 8 + j;
                 const float tv = (i <= t) ? sA[t * AS + i] : 0.f;
-                a1[j] = tv * sBeta[i] * sGam[i];
-                a2[j] = tv * sBeta[i];
+                a[j] = tv * sBeta[i] * (with_gamma ? sGam[i] : 1.f);
             }
-            uint4 h1, l1, h2, l2;
-            split8(a1, h1, l1);
-            split8(a2, h2, l2);
+            uint4 hv, lv;
+            split8(a, hv, lv);
             const uint32_t off = sw128_off(t, c8 * 8, 0);
-            st16(sm + LY::T1, off, h1);
-            st16(sm + LY::T1L, off, l1);
-            st16(rec + RC::T2, off, h2);
-            st16(rec + RC::T2L, off, l2);
+            st16(sm + LY::T1, off, hv);
+            st16(sm + LY::T1L, off, lv);
         }
+    };
+    if (ok) {
+        solve_unit_lower<NT>(sA, sA, sTmp, tid);
+        store_t_pair(true);
     }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
+    sync_for_mma();
     // Wk = T diag(beta gamma) K  (M = 64, N = DK; K read as an MN-major operand)
     if (ok && tid == 0) {
         const uint32_t id = idesc_bf16(64, DK, 0, 1);
@@ -201,9 +224,10 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
     fence_after_sync();
     __syncthreads();
     ok = failed_sh == 0;
+    // M = 64 accumulators: row r sits in lane 32 (r / 16) + r % 16
+    const bool own_t = lane < 16;
+    const int t_row = 16 * warp + lane;
     if (ok) {
-        const bool own_t = lane < 16;
-        const int t_row = 16 * warp + lane;
 #pragma unroll
         for (int cc = 0; cc < DK; cc += 32) {
             float x[32];
@@ -214,77 +238,126 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
     }
     fence_before_sync();
     __syncthreads();
+    // U = T diag(beta) V  (M = 64, N = DV; V read as an MN-major operand from the Q rows)
+    if (ok) store_t_pair(false);  // the Wk MMA has completed: the T1 tiles are free
+    if (ok && !mbar_wait(&ld_bar, 1, p.status)) failed_sh = 1;
+    sync_for_mma();
+    ok = failed_sh == 0;
+    if (ok && tid == 0) {
+        const uint32_t id = idesc_bf16(64, DV, 0, 1);
+        const uint64_t dV = make_desc(sb + LY::KQ + C * 128, LY::KQ_BLK, 1024, 2);
+        mma_steps<C / 16>(tb, id, make_desc(sb + LY::T1, 16, 1024, 2), dV, ok0, omn, false);
+        mma_steps<C / 16>(tb, id, make_desc(sb + LY::T1L, 16, 1024, 2), dV, ok0, omn, true);
+        mma_commit(&mma_bar);
+    }
+    __syncwarp();
+    if (ok && !mbar_wait(&mma_bar, 0, p.status)) failed_sh = 1;
+    fence_after_sync();
+    __syncthreads();
+    ok = failed_sh == 0;
+    // U: TMEM -> the record's slice layout, staged over K and V (both read by completed MMAs),
+    // then one bulk store
+    if (ok) {
+        uint8_t *stage = sm + LY::KQ;
+#pragma unroll
+        for (int cc = 0; cc < DV; cc += 32) {
+            float x[32];
+            tmem_ld32(taddr(tb, 32 * warp, cc), x);
+            tmem_wait_ld();
+            if (own_t) {
+#pragma unroll
+                for (int j4 = 0; j4 < 32; j4 += 4) {
+                    const int j = cc + j4;
+                    *reinterpret_cast<float4 *>(stage + (j / BV) * RC::U_SLICE + u_off<BV>(t_row, j % BV)) =
+                        make_float4(x[j4], x[j4 + 1], x[j4 + 2], x[j4 + 3]);
+                }
+            }
+        }
+    }
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    if (ok && tid == 0) {
+        bulk_s2g(rec + RC::U, sm + LY::KQ, (uint32_t)(C * DV * 4));
+        bulk_commit();
+        bulk_wait_all();
+    }
+    // after a failure, let the tile loads still in flight land before the CTA exits
+    if (!ok && tid == 0) mbar_wait(&ld_bar, v_issued ? 1 : 0, nullptr);
+    __syncthreads();
     if (warp == 0) tmem_dealloc(tb, 128);
 }
 
 // ------------------------------------------------------------------------------------------------
 // state: one CTA per (value slice, head, batch), chunks in order
 //
-// Two MMA rounds per chunk, shaped to keep the tcgen05 instruction count low:
-//   round 1:  D1  = [Q; Wk] [S_hi | S_lo]                  (M = 128, N = 2 BV: QS and X_s, hi and lo
-//                                                           halves side by side)
-//             D1[:, :BV] -= [0; T2_hi] V + [0; T2_lo] V    (U lands in the X_s rows; zero tile on top)
-//   round 2:  D3  = [Mqk_hi; 0] [Y_hi | Y_lo] ;  D3[:, :BV] += [Mqk_lo; 0] Y_hi
-//             D4  = K^T [DY_hi | DY_lo]
-// so that every operand row t of the chunk sits in TMEM lane t (QS, O) or lane 64 + t (X_s - U).
-// K, Q and V arrive by TMA tiled loads, the per-chunk records (Wk, T2, Mqk, g) by bulk copies.
+// Two MMA rounds per chunk (7 instructions at d = 128 for the first, 4 + 4 for the second):
+//   round 1:  D1 = [Q; Wk] [S_hi | S_lo]                    (M = 128, N = 2 BV: QS and X_s)
+//   round 2:  D4 = K^T [DY_hi | DY_lo]                      (the state update, on the chain)
+//             D3 = [Mqk_hi; Mqk_lo] [Y_hi | Y_lo]           (the output's intra-chunk term)
+// D1 is double-buffered in TMEM so that the output epilogue of chunk c overlaps round 1 of
+// chunk c + 1.  K, Q arrive by TMA tiled loads, the per-chunk record (Wk, Mqk, the U slice, g)
+// by bulk copies, one chunk ahead.
 
-template <int DK, int BV>
+template <int DK>
 struct StateLayout {
-    static constexpr uint32_t KQW_BLK = 3 * C * 128;      // [K; Q; Wk] rows of one 64-col block
-    static constexpr uint32_t ROWB = (BV == 32) ? 64 : 128;
-    static constexpr uint32_t VT = C * ROWB;              // C x BV tile (V slice)
+    static constexpr int BV = kBV<DK>;
     static constexpr int N2 = 2 * BV;                     // hi | lo side by side
+    static constexpr int CH = BV / 2;                     // columns of one epilogue warp
+    static constexpr uint32_t KQW_BLK = 3 * C * 128;      // [K; Q; Wk] rows of one 64-col block
+    static constexpr uint32_t U_BYTES = C * BV * 4;
     // double-buffered chunk inputs
     static constexpr uint32_t B_KQW = 0;
-    static constexpr uint32_t B_V = B_KQW + KQW_BLK * (DK / 64);
-    static constexpr uint32_t B_G = B_V + VT;               // g (64 floats)
+    static constexpr uint32_t B_MQ = B_KQW + KQW_BLK * (DK / 64);   // [Mqk_hi; Mqk_lo]
+    static constexpr uint32_t B_U = B_MQ + 2 * C * 128;
+    static constexpr uint32_t B_G = B_U + U_BYTES;                   // g (64 floats)
     static constexpr uint32_t BUF = B_G + 1024;
-    // single-buffered operands: [Mqk_hi][0][T2_hi][Mqk_lo][0][T2_lo]
-    static constexpr uint32_t MH = 2 * BUF;
-    static constexpr uint32_t Z1 = MH + C * 128;
-    static constexpr uint32_t T2H = Z1 + C * 128;
-    static constexpr uint32_t ML = T2H + C * 128;
-    static constexpr uint32_t Z2 = ML + C * 128;
-    static constexpr uint32_t T2L = Z2 + C * 128;
     // S^T [d][hi | lo], Y [t][hi | lo], D Y [t][hi | lo]: MN-major, 64-column blocks
     static constexpr uint32_t S_BLK = DK * 128;
-    static constexpr uint32_t S = T2L + C * 128;
+    static constexpr uint32_t S = 2 * BUF;
     static constexpr uint32_t Y_BLK = C * 128;
     static constexpr uint32_t Y = S + S_BLK * (N2 / 64);
     static constexpr uint32_t DY = Y + Y_BLK * (N2 / 64);
-    static constexpr uint32_t GATES = DY + Y_BLK * (N2 / 64);  // gamma, D: 2 x C floats
-    static constexpr uint32_t BYTES = GATES + 2 * C * 4 + 1024;
-    // TMEM columns
-    static constexpr uint32_t cD1 = 0, cD3 = N2, cD4 = 2 * N2, cU = 3 * N2;
-    static constexpr uint32_t TCOLS = (3 * N2 + BV <= 128) ? 128 : (3 * N2 + BV <= 256 ? 256 : 512);
+    static constexpr int OXS = BV + 4;                      // fp32 row stride of the output exchange
+    static constexpr uint32_t OX = DY + Y_BLK * (N2 / 64);
+    static constexpr uint32_t BYTES = OX + C * OXS * 4 + 1024;
+    // TMEM columns: D1 (two buffers), D3, D4
+    static constexpr uint32_t cD1 = 0, cD3 = 2 * N2, cD4 = 3 * N2;
+    static constexpr uint32_t TCOLS = 4 * N2 <= 256 ? 256 : 512;
 };
 
-// An N2-wide row of fp32 (hi | lo of one value each) stored as bf16 into an MN-major tile of
-// 64-column 128B-swizzled blocks: cols [0, BV) get bf16(x), cols [BV, 2BV) get bf16(x - hi).
-template <int BV>
-__device__ __forceinline__ void store_row_pair(uint8_t *tile, uint32_t blk_bytes, int row,
-                                               const float *x) {
-#pragma unroll
-    for (int c8 = 0; c8 < BV / 8; ++c8) {
-        uint4 h, l;
-        split8(x + c8 * 8, h, l);
-        st16(tile, sw128_off(row, c8 * 8, blk_bytes), h);
-        st16(tile, sw128_off(row, BV + c8 * 8, blk_bytes), l);
-    }
+// Warp roles of the state kernel: warps 0-7 epilogue (warp w reads TMEM lane quarter w % 4 and
+// the column half w / 4 of every BV-wide group), warp 8 issues the MMAs, warp 9 the loads.  Every
+// hand-off is an mbarrier; every wait is bounded.
+constexpr int ST_THREADS = 320;
+constexpr int EPI_THREADS = 256;
+constexpr int EPI_WARPS = EPI_THREADS / 32;
+
+struct StateBars {
+    uint64_t full[2];      // chunk inputs landed (tx)
+    uint64_t empty[2];     // chunk buffer released: the MMAs reading it (commit) + every epilogue warp
+    uint64_t s_ready, y_ready;           // epilogue -> MMA: S^T tile, Y / DY tiles written
+    uint64_t d1_full, d4_full, d3_full;  // MMA -> epilogue: accumulators complete
+    uint64_t drain;                      // the MMA thread's last operations
+};
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t a, float (&v)[N]) {
+    if constexpr (N == 16) tmem_ld16(a, v);
+    else tmem_ld32(a, v);
 }
 
-// out[j] = D[lane row][col + j] + D[lane row][col + BV + j]: the hi and lo halves of a pair MMA.
-template <int BV>
-__device__ __forceinline__ void ld_pair_sum(uint32_t tbase, int warp, uint32_t col, float *out) {
+// CH fp32 values at (row, j0 .. j0+CH) as a hi / lo pair into an MN-major tile of 64-column
+// 128B-swizzled blocks: hi at columns j0.., lo at BV + j0...
+template <int BV, int CH>
+__device__ __forceinline__ void store_half_pair(uint8_t *tile, uint32_t blk_bytes, int row, int j0,
+                                                const float *x) {
 #pragma unroll
-    for (int c = 0; c < BV; c += 32) {
-        float a[32], b[32];
-        tmem_ld32(taddr(tbase, 32 * warp, col + c), a);
-        tmem_ld32(taddr(tbase, 32 * warp, col + BV + c), b);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) out[c + j] = a[j] + b[j];
+    for (int c8 = 0; c8 < CH / 8; ++c8) {
+        uint4 hv, lv;
+        split8(x + c8 * 8, hv, lv);
+        st16(tile, sw128_off(row, j0 + c8 * 8, blk_bytes), hv);
+        st16(tile, sw128_off(row, BV + j0 + c8 * 8, blk_bytes), lv);
     }
 }
 
@@ -293,26 +366,14 @@ __device__ __forceinline__ const uint8_t *record(const ScanArgs &p, const uint8_
     return ws + kRecOffset + (((size_t)blockIdx.z * p.H + blockIdx.y) * nch + c) * GdnRec<DK>::BYTES;
 }
 
-// Warp roles of the state kernel: warps 0-3 epilogue (TMEM lane quarters 0-3), warp 4 issues the
-// MMAs, warp 5 issues the loads.  Every hand-off is an mbarrier; every wait is bounded.
-constexpr int ST_THREADS = 192;
-constexpr int EPI_THREADS = 128;
-
-struct StateBars {
-    uint64_t full[2];      // chunk inputs landed (tx): K, Q, V, Wk, g
-    uint64_t empty[2];     // chunk buffer released: last MMA reading it (commit) + epilogue (g read)
-    uint64_t t2_full, t2_empty, mq_full, mq_empty;
-    uint64_t s_ready, y_ready;      // epilogue -> MMA: S^T tile, Y / DY tiles written
-    uint64_t d1_full, d4_full, d3_full;  // MMA -> epilogue: accumulators complete
-};
-
-template <int DK, int BV>
+// 10 warps: the sub-partition holding three of them caps a thread at 168 registers.
+template <int DK>
 __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                                                                  const __grid_constant__ GdnMaps maps,
                                                                  const uint8_t *ws, int nch) {
-    using LY = StateLayout<DK, BV>;
+    using LY = StateLayout<DK>;
     using RC = GdnRec<DK>;
-    constexpr int N2 = LY::N2;
+    constexpr int BV = LY::BV, N2 = LY::N2, CH = LY::CH;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     __shared__ StateBars bars;
@@ -329,25 +390,17 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars.full[i], 1);
-            mbar_init(&bars.empty[i], 2);
+            mbar_init(&bars.empty[i], 1 + EPI_WARPS);
         }
-        mbar_init(&bars.t2_full, 1);
-        mbar_init(&bars.t2_empty, 1);
-        mbar_init(&bars.mq_full, 1);
-        mbar_init(&bars.mq_empty, 1);
         mbar_init(&bars.s_ready, 1);
         mbar_init(&bars.y_ready, 1);
         mbar_init(&bars.d1_full, 1);
         mbar_init(&bars.d4_full, 1);
         mbar_init(&bars.d3_full, 1);
+        mbar_init(&bars.drain, 1);
         mbar_fence_init();
         failed_sh = 0;
     }
-    for (int e = tid; e < C * 128 / 16; e += ST_THREADS) {  // zero tiles under Mqk and over T2
-        st16(sm + LY::Z1, e * 16, make_uint4(0, 0, 0, 0));
-        st16(sm + LY::Z2, e * 16, make_uint4(0, 0, 0, 0));
-    }
-    fence_async_smem();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -356,171 +409,200 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
     auto fail = [&]() { failed_sh = 1; };
     auto failed = [&]() { return *(volatile int *)&failed_sh != 0; };
 
-    if (warp == 5) {
+    if (warp == EPI_WARPS + 1) {
         // ---------------- loads ----------------
         if (lane == 0) {
-            auto load_chunk = [&](int c) {
+            constexpr uint32_t bytes = 3 * (DK / 64) * C * 128 + 2 * C * 128 + LY::U_BYTES + C * 4;
+            int issued = -1;
+            for (int c = 0; c < nch && !failed(); ++c) {
+                if (c >= 2 && !mbar_wait(&bars.empty[c & 1], ((c - 2) >> 1) & 1, status)) { fail(); break; }
                 const uint8_t *rec = record<DK>(p, ws, nch, c);
                 uint8_t *buf = sm + (c & 1) * LY::BUF;
                 uint64_t *bar = &bars.full[c & 1];
                 const int c0 = c * C;
-                mbar_expect_tx(bar, 2 * (DK / 64) * C * 128 + LY::VT + (DK / 64) * RC::WK_BLK + C * 4);
+                mbar_expect_tx(bar, bytes);
                 for (int blk = 0; blk < DK / 64; ++blk) {
                     uint8_t *dst = buf + LY::B_KQW + blk * LY::KQW_BLK;
                     tma_load_4d(dst, &maps.k, blk * 64, h, c0, b, bar);
                     tma_load_4d(dst + C * 128, &maps.q, blk * 64, h, c0, b, bar);
                     bulk_g2s(dst + 2 * C * 128, rec + RC::WK + blk * RC::WK_BLK, RC::WK_BLK, bar);
                 }
-                tma_load_4d(buf + LY::B_V, &maps.v, v0, h, c0, b, bar);
+                bulk_g2s(buf + LY::B_MQ, rec + RC::MQK, 2 * C * 128, bar);
+                bulk_g2s(buf + LY::B_U, rec + RC::U + blockIdx.x * RC::U_SLICE, LY::U_BYTES, bar);
                 bulk_g2s(buf + LY::B_G, rec + RC::G, C * 4, bar);
-            };
-            for (int c = 0; c < nch && !failed(); ++c) {
-                const uint8_t *rec = record<DK>(p, ws, nch, c);
-                if (c >= 2 && !mbar_wait(&bars.empty[c & 1], ((c - 2) >> 1) & 1, status)) { fail(); break; }
-                load_chunk(c);
-                if (c >= 1 && !mbar_wait(&bars.t2_empty, (c - 1) & 1, status)) { fail(); break; }
-                mbar_expect_tx(&bars.t2_full, 2 * C * 128);
-                bulk_g2s(sm + LY::T2H, rec + RC::T2, C * 128, &bars.t2_full);
-                bulk_g2s(sm + LY::T2L, rec + RC::T2L, C * 128, &bars.t2_full);
-                if (c >= 1 && !mbar_wait(&bars.mq_empty, (c - 1) & 1, status)) { fail(); break; }
-                mbar_expect_tx(&bars.mq_full, 2 * C * 128);
-                bulk_g2s(sm + LY::MH, rec + RC::MQK, C * 128, &bars.mq_full);
-                bulk_g2s(sm + LY::ML, rec + RC::MQKL, C * 128, &bars.mq_full);
+                issued = c;
             }
+            // let the copies still in flight land before the CTA can exit
+            for (int c = issued > 0 ? issued - 1 : 0; c <= issued; ++c)
+                mbar_wait(&bars.full[c & 1], (c >> 1) & 1, nullptr);
         }
-    } else if (warp == 4) {
+    } else if (warp == EPI_WARPS) {
         // ---------------- MMA issue ----------------
         if (lane == 0) {
             auto oKQW = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::KQW_BLK); };
             auto oK0 = [](int ks) { return (uint64_t)koff_k_sw128(ks, 0); };
             auto oMN = [](int ks) { return (uint64_t)koff_mn_sw128(ks); };
-            auto oVT = [](int ks) { return (uint64_t)(BV == 32 ? koff_mn_sw64(ks) : koff_mn_sw128(ks)); };
             const uint64_t dS2 = make_desc(sb + LY::S, LY::S_BLK, 1024, 2);
             const uint64_t dY2 = make_desc(sb + LY::Y, LY::Y_BLK, 1024, 2);
             const uint64_t dDY2 = make_desc(sb + LY::DY, LY::Y_BLK, 1024, 2);
-            const uint64_t dZ1 = make_desc(sb + LY::Z1, 16, 1024, 2), dZ2 = make_desc(sb + LY::Z2, 16, 1024, 2);
-            const uint64_t dMH = make_desc(sb + LY::MH, 16, 1024, 2), dML = make_desc(sb + LY::ML, 16, 1024, 2);
-            const uint32_t idU = idesc_bf16(128, BV, 0, 1) | (1u << 13);  // negated A
             const uint32_t idS = idesc_bf16(128, N2, 0, 1);
+            const uint32_t id4 = idesc_bf16(DK, N2, 1, 1);
             for (int c = 0; c < nch; ++c) {
                 const uint32_t bb = sb + (c & 1) * LY::BUF;
                 if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status)) { fail(); break; }
-                if (!mbar_wait(&bars.t2_full, c & 1, status)) { fail(); break; }
-                if (c >= 1 && !mbar_wait(&bars.y_ready, (c - 1) & 1, status)) { fail(); break; }
-                fence_after_sync();
-                // state-independent part of round 1, ahead of the state: U' = -[0; T2_hi] V - [0; T2_lo] V
-                const uint64_t dV = (BV == 32) ? make_desc(bb + LY::B_V, 0, 512, 4)
-                                               : make_desc(bb + LY::B_V, C * 128, 1024, 2);
-                mma_steps<C / 16>(tb + LY::cU, idU, dZ1, dV, oK0, oVT, false);
-                mma_steps<C / 16>(tb + LY::cU, idU, dZ2, dV, oK0, oVT, true);
-                mma_commit(&bars.t2_empty);
-                // state part: D1 = [Q; Wk] [S_hi | S_lo]
+                // S_c written (which also means the output epilogue of chunk c - 2 is done with
+                // this D1 buffer: the epilogue warps work through the chunks in order)
                 if (!mbar_wait(&bars.s_ready, c & 1, status)) { fail(); break; }
                 fence_after_sync();
                 const uint64_t dQW = make_desc(bb + LY::B_KQW + C * 128, 16, 1024, 2);
-                mma_steps<DK / 16>(tb + LY::cD1, idS, dQW, dS2, oKQW, oMN, false);
+                mma_steps<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dQW, dS2, oKQW, oMN, false);
                 mma_commit(&bars.d1_full);
-                // round 2: the state update first (on the critical path), then the output
+                // Y_c written (and the output epilogue of chunk c - 1 is done with D3)
                 if (!mbar_wait(&bars.y_ready, c & 1, status)) { fail(); break; }
                 fence_after_sync();
                 const uint64_t dKt = make_desc(bb + LY::B_KQW, LY::KQW_BLK, 1024, 2);
-                mma_steps<C / 16>(tb + LY::cD4, idesc_bf16(DK, N2, 1, 1), dKt, dDY2, oMN, oMN, false);
+                mma_steps<C / 16>(tb + LY::cD4, id4, dKt, dDY2, oMN, oMN, false);
                 mma_commit(&bars.d4_full);
-                if (!mbar_wait(&bars.mq_full, c & 1, status)) { fail(); break; }
-                mma_steps<C / 16>(tb + LY::cD3, idesc_bf16(128, N2, 0, 1), dMH, dY2, oK0, oMN, false);
-                mma_steps<C / 16>(tb + LY::cD3, idesc_bf16(128, BV, 0, 1), dML, dY2, oK0, oMN, true);
+                const uint64_t dMQ = make_desc(bb + LY::B_MQ, 16, 1024, 2);
+                mma_steps<C / 16>(tb + LY::cD3, idS, dMQ, dY2, oK0, oMN, false);
                 mma_commit(&bars.d3_full);
-                mma_commit(&bars.mq_empty);
                 mma_commit(&bars.empty[c & 1]);
             }
+            mma_commit(&bars.drain);
+            mbar_wait(&bars.drain, 0, nullptr);
         }
     } else {
-        // ---------------- epilogue: warps 0-3 ----------------
+        // ---------------- epilogue: warps 0-7 ----------------
         __nv_bfloat16 *o = (__nv_bfloat16 *)p.o;
-        float *sGam = (float *)(sm + LY::GATES);
-        float *sD = sGam + C;
+        const int q = warp & 3;            // TMEM lane quarter
+        const int j0 = (warp >> 2) * CH;   // first column of this warp in each BV-wide group
+        const int lrow = 32 * q + lane;    // TMEM lane of this thread
+        // state rows: lane = row for M = 128 (d = 128); lanes 32q + r, r < 16, for M = 64
         const bool own_d = (DK == 128) ? true : (lane < 16);
-        const int d_row = (DK == 128) ? tid : (16 * warp + lane);
-        float Sreg[BV];
+        const int d_row = (DK == 128) ? lrow : (16 * q + lane);
+        const bool wr = !(p.flags & kNoWrite), out = !(p.flags & kNoOutput);
+        float *ox = (float *)(sm + LY::OX);
+        float Sreg[CH];
 #pragma unroll
-        for (int j = 0; j < BV; ++j) Sreg[j] = 0.f;
+        for (int j = 0; j < CH; ++j) Sreg[j] = 0.f;
         if (own_d && (p.flags & kS0Identity)) {
 #pragma unroll
-            for (int j = 0; j < BV; ++j) Sreg[j] = (v0 + j == d_row) ? 1.f : 0.f;
+            for (int j = 0; j < CH; ++j) Sreg[j] = (v0 + j0 + j == d_row) ? 1.f : 0.f;
         } else if (own_d && p.S0) {
 #pragma unroll
-            for (int j = 0; j < BV; ++j) Sreg[j] = p.S0[(head * dv + v0 + j) * DK + d_row];
+            for (int j = 0; j < CH; ++j) Sreg[j] = p.S0[(head * dv + v0 + j0 + j) * DK + d_row];
         }
-        if (own_d) store_row_pair<BV>(sm + LY::S, LY::S_BLK, d_row, Sreg);
+        if (own_d) store_half_pair<BV, CH>(sm + LY::S, LY::S_BLK, d_row, j0, Sreg);
         fence_async_smem();
         named_sync(1, EPI_THREADS);
         if (tid == 0) mbar_arrive(&bars.s_ready);
         for (int c = 0; c < nch; ++c) {
             const int c0 = c * C, n = min(C, T - c0);
             const uint8_t *buf = sm + (c & 1) * LY::BUF;
-            if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status)) { fail(); break; }
+            bool bad = !mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status);
+            bad = bad || !mbar_wait(&bars.d1_full, c & 1, status);
+            if (named_sync_or(1, EPI_THREADS, bad)) { fail(); break; }
+            fence_after_sync();
             const float *g = reinterpret_cast<const float *>(buf + LY::B_G);
             const float g_last = g[C - 1];
-            if (tid < C) {
-                sGam[tid] = __expf(g[tid]);
-                sD[tid] = tid < n ? __expf(g_last - g[tid]) : 0.f;
-            }
-            named_sync(1, EPI_THREADS);
-            if (tid == 0) mbar_arrive(&bars.empty[c & 1]);  // g has been read
-            // Y = U - X_s (rows 64..127 of D1), QS (rows 0..63)
-            if (!mbar_wait(&bars.d1_full, c & 1, status)) { fail(); break; }
-            fence_after_sync();
-            float qs[BV];
-            ld_pair_sum<BV>(tb, warp, LY::cD1, qs);
-            if (warp >= 2) {
-                const int t = tid - 64;
-                float y[BV];
-                ld_row<BV>(tb, warp, LY::cU, y);  // -U
-                const bool wr = !(p.flags & kNoWrite);
+            const uint32_t d1 = LY::cD1 + (c & 1) * N2;
+            // Y = U - X_s (rows 64..127 of D1), and D Y
+            if (q >= 2) {
+                const int t = lrow - 64;
+                float xh[CH], xl[CH], y[CH];
+                tmem_ld_n<CH>(taddr(tb, 32 * q, d1 + j0), xh);
+                tmem_ld_n<CH>(taddr(tb, 32 * q, d1 + BV + j0), xl);
+                tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < BV; ++j) y[j] = -(qs[j] + (wr ? y[j] : 0.f));
-                store_row_pair<BV>(sm + LY::Y, LY::Y_BLK, t, y);
-                const float dd = sD[t];
+                for (int j = 0; j < CH; ++j) y[j] = -(xh[j] + xl[j]);
+                if (wr) {
 #pragma unroll
-                for (int j = 0; j < BV; ++j) y[j] *= dd;
-                store_row_pair<BV>(sm + LY::DY, LY::Y_BLK, t, y);
+                    for (int j4 = 0; j4 < CH; j4 += 4) {
+                        const float4 u = *reinterpret_cast<const float4 *>(buf + LY::B_U + u_off<BV>(t, j0 + j4));
+                        y[j4] += u.x;
+                        y[j4 + 1] += u.y;
+                        y[j4 + 2] += u.z;
+                        y[j4 + 3] += u.w;
+                    }
+                }
+                store_half_pair<BV, CH>(sm + LY::Y, LY::Y_BLK, t, j0, y);
+                const float dd = t < n ? __expf(g_last - g[t]) : 0.f;
+#pragma unroll
+                for (int j = 0; j < CH; ++j) y[j] *= dd;
+                store_half_pair<BV, CH>(sm + LY::DY, LY::Y_BLK, t, j0, y);
             }
             fence_async_smem();
             fence_before_sync();
             named_sync(1, EPI_THREADS);
             if (tid == 0) mbar_arrive(&bars.y_ready);
             // state update S^T <- e^{g_n} S^T + K^T D Y
-            if (!mbar_wait(&bars.d4_full, c & 1, status)) { fail(); break; }
+            bad = !mbar_wait(&bars.d4_full, c & 1, status);
+            if (named_sync_or(1, EPI_THREADS, bad)) { fail(); break; }
             fence_after_sync();
             {
-                float x[BV];
-                ld_pair_sum<BV>(tb, warp, LY::cD4, x);
+                float xh[CH], xl[CH];
+                tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD4 + j0), xh);
+                tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD4 + BV + j0), xl);
+                tmem_wait_ld();
                 const float gC = __expf(g_last);
                 if (own_d) {
 #pragma unroll
-                    for (int j = 0; j < BV; ++j) Sreg[j] = fmaf(gC, Sreg[j], x[j]);
-                    store_row_pair<BV>(sm + LY::S, LY::S_BLK, d_row, Sreg);
+                    for (int j = 0; j < CH; ++j) Sreg[j] = fmaf(gC, Sreg[j], xh[j] + xl[j]);
+                    store_half_pair<BV, CH>(sm + LY::S, LY::S_BLK, d_row, j0, Sreg);
                 }
             }
             fence_async_smem();
             fence_before_sync();
             named_sync(1, EPI_THREADS);
             if (tid == 0) mbar_arrive(&bars.s_ready);
-            // output O = diag(e^g) QS + Mqk Y (overlaps the next chunk's first MMAs)
-            if (!mbar_wait(&bars.d3_full, c & 1, status)) { fail(); break; }
+            // output O = diag(e^g) QS + Mqk Y: the Mqk_lo rows (lanes 64..127) pass their
+            // partial sums through shared memory to the threads that own the output rows
+            bad = !mbar_wait(&bars.d3_full, c & 1, status);
+            if (named_sync_or(1, EPI_THREADS, bad)) { fail(); break; }
             fence_after_sync();
-            if (warp < 2) {
-                float x[BV];
-                ld_pair_sum<BV>(tb, warp, LY::cD3, x);
-                const int t = tid;
-                if (t < n && !(p.flags & kNoOutput)) {
-                    const float gt = sGam[t];
-                    __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t) * H + h) * dv + v0;
+            if (q >= 2) {
+                const int t = lrow - 64;
+                float a[CH], bb[CH];
+                tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD3 + j0), a);
+                tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD3 + BV + j0), bb);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int c8 = 0; c8 < BV / 8; ++c8) {
+                for (int j4 = 0; j4 < CH; j4 += 4)
+                    *reinterpret_cast<float4 *>(ox + t * LY::OXS + j0 + j4) =
+                        make_float4(a[j4] + bb[j4], a[j4 + 1] + bb[j4 + 1], a[j4 + 2] + bb[j4 + 2],
+                                    a[j4 + 3] + bb[j4 + 3]);
+            }
+            named_sync(1, EPI_THREADS);
+            if (q < 2) {
+                const int t = lrow;
+                float up[CH], qs[CH];
+                {
+                    float a[CH], bb[CH];
+                    tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD3 + j0), a);
+                    tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD3 + BV + j0), bb);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < CH; ++j) up[j] = a[j] + bb[j];
+                    tmem_ld_n<CH>(taddr(tb, 32 * q, d1 + j0), a);
+                    tmem_ld_n<CH>(taddr(tb, 32 * q, d1 + BV + j0), bb);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < CH; ++j) qs[j] = a[j] + bb[j];
+                }
+                if (t < n && out) {
+                    const float gt = __expf(g[t]);
+                    __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t) * H + h) * dv + v0 + j0;
+#pragma unroll
+                    for (int c8 = 0; c8 < CH / 8; ++c8) {
+                        const float4 p0 = *reinterpret_cast<const float4 *>(ox + t * LY::OXS + j0 + c8 * 8);
+                        const float4 p1 = *reinterpret_cast<const float4 *>(ox + t * LY::OXS + j0 + c8 * 8 + 4);
+                        const float pp[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
                         float r[8];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) r[j] = fmaf(gt, qs[c8 * 8 + j], x[c8 * 8 + j]);
+                        for (int j = 0; j < 8; ++j) {
+                            const int jj = c8 * 8 + j;
+                            r[j] = fmaf(gt, qs[jj], up[jj] + pp[j]);
+                        }
                         uint4 pk;
                         pk.x = pack_bf16(r[0], r[1]);
                         pk.y = pack_bf16(r[2], r[3]);
@@ -530,12 +612,15 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                     }
                 }
             }
+            // D1 / D3 reads done before the MMA thread reuses them (it learns so from later
+            // hand-offs of these warps); the chunk buffer (g, U) is released
             fence_before_sync();
-            named_sync(1, EPI_THREADS);  // D3 read before the next chunk's round 2 overwrites it
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.empty[c & 1]);
         }
         if (p.S_final && own_d && !failed()) {
 #pragma unroll
-            for (int j = 0; j < BV; ++j) p.S_final[(head * dv + v0 + j) * DK + d_row] = Sreg[j];
+            for (int j = 0; j < CH; ++j) p.S_final[(head * dv + v0 + j0 + j) * DK + d_row] = Sreg[j];
         }
     }
     fence_before_sync();
@@ -572,17 +657,17 @@ bool act_map(CUtensorMap *m, const void *base, int B, int T, int H, int d, int b
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DK, int BV>
+template <int DK>
 bool gdn_maps(const ScanArgs &a, GdnMaps *maps) {
     return act_map(&maps->k, a.k, a.B, a.T, a.H, DK, 64) && act_map(&maps->q, a.q, a.B, a.T, a.H, DK, 64) &&
-           act_map(&maps->v, a.v, a.B, a.T, a.H, a.dv, BV);
+           act_map(&maps->v, a.v, a.B, a.T, a.H, a.dv, 64);
 }
 
-template <int DK, int BV>
+template <int DK>
 cudaError_t launch_gdn_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
     const int nch = (a.T + C - 1) / C;
     GdnMaps maps;
-    if (!gdn_maps<DK, BV>(a, &maps)) return cudaErrorInvalidValue;
+    if (!gdn_maps<DK>(a, &maps)) return cudaErrorInvalidValue;
     using LY = PrepLayout<DK>;
     auto kern = gdn_prep_kernel<DK>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
@@ -593,17 +678,17 @@ cudaError_t launch_gdn_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-template <int DK, int BV>
+template <int DK>
 cudaError_t launch_gdn_state_t(const ScanArgs &a, const void *ws, cudaStream_t s) {
     const int nch = (a.T + C - 1) / C;
     GdnMaps maps;
-    if (!gdn_maps<DK, BV>(a, &maps)) return cudaErrorInvalidValue;
-    using LY = StateLayout<DK, BV>;
+    if (!gdn_maps<DK>(a, &maps)) return cudaErrorInvalidValue;
+    using LY = StateLayout<DK>;
     static_assert(LY::BYTES <= 227 * 1024, "shared memory budget");
-    auto kern = gdn_state_kernel<DK, BV>;
+    auto kern = gdn_state_kernel<DK>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
     if (err != cudaSuccess) return err;
-    dim3 grid(a.dv / BV, a.H, a.B);
+    dim3 grid(a.dv / LY::BV, a.H, a.B);
     launch_probe_mark(s);
     kern<<<grid, ST_THREADS, LY::BYTES, s>>>(a, maps, (const uint8_t *)ws, nch);
     return cudaGetLastError();
@@ -619,14 +704,15 @@ size_t gdn_workspace_bytes(int B, int H, int T, int dk) {
 }
 
 // The per-chunk records (prep) and the in-order pass over them (state); records depend only on
-// q, k, alpha, beta, so several state passes over the same tokens can share one prep.
+// the tokens (q, k, v, alpha, beta), so several state passes over the same tokens can share one
+// prep (a pass with kNoWrite ignores the records' U).
 cudaError_t launch_gdn_prep(const ScanArgs &a, void *ws, cudaStream_t s) {
     if (a.T <= 0) return cudaSuccess;
-    return a.dk == 128 ? launch_gdn_prep_t<128, 32>(a, ws, s) : launch_gdn_prep_t<64, 64>(a, ws, s);
+    return a.dk == 128 ? launch_gdn_prep_t<128>(a, ws, s) : launch_gdn_prep_t<64>(a, ws, s);
 }
 
 cudaError_t launch_gdn_state(const ScanArgs &a, const void *ws, cudaStream_t s) {
-    return a.dk == 128 ? launch_gdn_state_t<128, 32>(a, ws, s) : launch_gdn_state_t<64, 64>(a, ws, s);
+    return a.dk == 128 ? launch_gdn_state_t<128>(a, ws, s) : launch_gdn_state_t<64>(a, ws, s);
 }
 
 cudaError_t launch_scan_gdn(const ScanArgs &a, void *ws, cudaStream_t s) {

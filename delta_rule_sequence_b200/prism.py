@@ -27,6 +27,7 @@ EXPORTS = (
     "prism_step_decode",
     "prism_query_device_status",
     "prism_status_string",
+    "prism_last_cuda_error",
     "prism_debug_set_flags",
     "prism_debug_record_launch_events",
 )
@@ -35,7 +36,13 @@ EXPORTS = (
 class PrismError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} ({status})")
+        detail = ""
+        if status == PRISM_ERR_CUDA:
+            try:
+                detail = load_library().prism_last_cuda_error().decode()
+            except RuntimeError:
+                pass
+        super().__init__(f"{where}: {status_string(status)} ({status})" + (f": {detail}" if detail else ""))
 
 
 class PrismShape(ctypes.Structure):
@@ -72,6 +79,8 @@ def load_library():
     lib.prism_query_device_status.restype = ci
     lib.prism_status_string.argtypes = [ci]
     lib.prism_status_string.restype = ctypes.c_char_p
+    lib.prism_last_cuda_error.argtypes = []
+    lib.prism_last_cuda_error.restype = ctypes.c_char_p
     lib.prism_debug_set_flags.argtypes = [ci]
     lib.prism_debug_set_flags.restype = ci
     lib.prism_debug_record_launch_events.argtypes = [ctypes.POINTER(vp), ci]

@@ -147,6 +147,12 @@ prism_status prism_query_device_status(void *workspace, void *stream);
 const char *prism_status_string(prism_status status);
 
 /*
+ * prism_last_cuda_error -- the CUDA runtime's description of the error behind the calling host
+ * thread's most recent PRISM_ERR_CUDA ("" if there was none).  Static storage; never NULL.
+ */
+const char *prism_last_cuda_error(void);
+
+/*
  * prism_debug_set_flags -- testing and measurement hook (process-wide; set it before
  * prism_scan_fwd_workspace_size, which depends on it).  flags bit 1: prism_scan_fwd takes the
  * segmented inter-chunk scan (segment elements, a Blelloch scan over them, a re-run of every
