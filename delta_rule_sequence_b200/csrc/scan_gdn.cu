@@ -67,15 +67,15 @@ __device__ __forceinline__ uint32_t u_off(int t, int j) {
 // ------------------------------------------------------------------------------------------------
 // prep: one CTA per (chunk, head, batch)
 
+// 55 KB at either width, so four CTAs share an SM.  At d = 128 the T pair tiles live in the Q
+// rows (free once G is done); V replaces K once Wk is done; U is staged over all of it at the end.
 template <int DK>
 struct PrepLayout {
-    static constexpr uint32_t KQ_BLK = 2 * C * 128;     // [K; Q] rows of one 64-column block; V
-                                                        // replaces Q once G is done, U is staged
-                                                        // over K and V at the end
+    static constexpr uint32_t KQ_BLK = 2 * C * 128;     // [K; Q] rows of one 64-column block
     static constexpr uint32_t KQ = 0;
-    static constexpr uint32_t T1 = KQ + KQ_BLK * (DK / 64);
-    static constexpr uint32_t T1L = T1 + C * 128;
-    static constexpr uint32_t AF = T1L + C * 128;       // fp32 A, solved in place into T
+    static constexpr uint32_t T1 = DK == 128 ? KQ + C * 128 : KQ + KQ_BLK;
+    static constexpr uint32_t T1L = DK == 128 ? KQ + KQ_BLK + C * 128 : T1 + C * 128;
+    static constexpr uint32_t AF = DK == 128 ? KQ + 2 * KQ_BLK : T1L + C * 128;  // fp32 A, solved in place into T
     static constexpr uint32_t TMP = AF + C * AS * 4;
     static constexpr uint32_t GATES = TMP + 32 * 33 * 4;
     static constexpr uint32_t BYTES = GATES + 3 * C * 4 + 1024;
@@ -155,13 +155,6 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
     fence_after_sync();
     __syncthreads();
     bool ok = failed_sh == 0;  // uniform across the CTA
-    // V into the Q rows, which G no longer needs; it lands while the solve runs
-    const bool v_issued = ok;
-    if (ok && tid == 0) {
-        mbar_expect_tx(&ld_bar, (DV / 64) * C * 128);
-        for (int blk = 0; blk < DV / 64; ++blk)
-            tma_load_4d(sm + LY::KQ + blk * LY::KQ_BLK + C * 128, &maps.v, blk * 64, h, c0, b, &ld_bar);
-    }
     if (ok) {
         const int t = (warp & 1) * 32 + lane;
         const float gt = sG[t], bt = sBeta[t];
@@ -224,6 +217,13 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
     fence_after_sync();
     __syncthreads();
     ok = failed_sh == 0;
+    // V into the K rows, which no MMA reads any more; it lands during the Wk epilogue
+    const bool v_issued = ok;
+    if (ok && tid == 0) {
+        mbar_expect_tx(&ld_bar, (DV / 64) * C * 128);
+        for (int blk = 0; blk < DV / 64; ++blk)
+            tma_load_4d(sm + LY::KQ + blk * LY::KQ_BLK, &maps.v, blk * 64, h, c0, b, &ld_bar);
+    }
     // M = 64 accumulators: row r sits in lane 32 (r / 16) + r % 16
     const bool own_t = lane < 16;
     const int t_row = 16 * warp + lane;
@@ -238,14 +238,14 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
     }
     fence_before_sync();
     __syncthreads();
-    // U = T diag(beta) V  (M = 64, N = DV; V read as an MN-major operand from the Q rows)
+    // U = T diag(beta) V  (M = 64, N = DV; V read as an MN-major operand from the K rows)
     if (ok) store_t_pair(false);  // the Wk MMA has completed: the T1 tiles are free
     if (ok && !mbar_wait(&ld_bar, 1, p.status)) failed_sh = 1;
     sync_for_mma();
     ok = failed_sh == 0;
     if (ok && tid == 0) {
         const uint32_t id = idesc_bf16(64, DV, 0, 1);
-        const uint64_t dV = make_desc(sb + LY::KQ + C * 128, LY::KQ_BLK, 1024, 2);
+        const uint64_t dV = make_desc(sb + LY::KQ, LY::KQ_BLK, 1024, 2);
         mma_steps<C / 16>(tb, id, make_desc(sb + LY::T1, 16, 1024, 2), dV, ok0, omn, false);
         mma_steps<C / 16>(tb, id, make_desc(sb + LY::T1L, 16, 1024, 2), dV, ok0, omn, true);
         mma_commit(&mma_bar);
@@ -255,8 +255,8 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
     fence_after_sync();
     __syncthreads();
     ok = failed_sh == 0;
-    // U: TMEM -> the record's slice layout, staged over K and V (both read by completed MMAs),
-    // then one bulk store
+    // U: TMEM -> the record's slice layout, staged over the K / Q rows (everything there was read
+    // by completed MMAs), then one bulk store
     if (ok) {
         uint8_t *stage = sm + LY::KQ;
 #pragma unroll
@@ -291,24 +291,26 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
 // ------------------------------------------------------------------------------------------------
 // state: one CTA per (value slice, head, batch), chunks in order
 //
-// Two MMA rounds per chunk (7 instructions at d = 128 for the first, 4 + 4 for the second):
-//   round 1:  D1 = [Q; Wk] [S_hi | S_lo]                    (M = 128, N = 2 BV: QS and X_s)
+// Two MMA rounds per chunk (8 instructions at d = 128 for the first, 4 + 4 for the second):
+//   round 1:  D1 = [Wk; Q] [S_hi | S_lo]                    (M = 128, N = 2 BV: X_s and QS)
 //   round 2:  D4 = K^T [DY_hi | DY_lo]                      (the state update, on the chain)
-//             D3 = [Mqk_hi; Mqk_lo] [Y_hi | Y_lo]           (the output's intra-chunk term)
-// D1 is double-buffered in TMEM so that the output epilogue of chunk c overlaps round 1 of
-// chunk c + 1.  K, Q arrive by TMA tiled loads, the per-chunk record (Wk, Mqk, the U slice, g)
-// by bulk copies, one chunk ahead.
+//             D3 = [Mqk_lo; Mqk_hi] [Y_hi | Y_lo]           (the output's intra-chunk term)
+// X_s and the Mqk_lo product sit in TMEM lanes 0..63, QS and the Mqk_hi product in lanes 64..127,
+// so the Y epilogue runs on sub-partitions 0-1 and the output epilogue on 2-3, where it does not
+// slow the MMA warp (sub-partition 0) issuing the next chunk's round 1.  D1 is double-buffered in
+// TMEM.  K, Q arrive by TMA tiled loads, the per-chunk record (Wk, Mqk, the U slice, g) by bulk
+// copies, one chunk ahead.
 
 template <int DK>
 struct StateLayout {
     static constexpr int BV = kBV<DK>;
     static constexpr int N2 = 2 * BV;                     // hi | lo side by side
-    static constexpr int CH = BV / 2;                     // columns of one epilogue warp
-    static constexpr uint32_t KQW_BLK = 3 * C * 128;      // [K; Q; Wk] rows of one 64-col block
+    static constexpr int CH = BV / 4;                     // columns of one epilogue warp
+    static constexpr uint32_t KWQ_BLK = 3 * C * 128;      // [K; Wk; Q] rows of one 64-col block
     static constexpr uint32_t U_BYTES = C * BV * 4;
     // double-buffered chunk inputs
-    static constexpr uint32_t B_KQW = 0;
-    static constexpr uint32_t B_MQ = B_KQW + KQW_BLK * (DK / 64);   // [Mqk_hi; Mqk_lo]
+    static constexpr uint32_t B_KWQ = 0;
+    static constexpr uint32_t B_MQ = B_KWQ + KWQ_BLK * (DK / 64);   // [Mqk_lo; Mqk_hi]
     static constexpr uint32_t B_U = B_MQ + 2 * C * 128;
     static constexpr uint32_t B_G = B_U + U_BYTES;                   // g (64 floats)
     static constexpr uint32_t BUF = B_G + 1024;
@@ -326,24 +328,27 @@ struct StateLayout {
     static constexpr uint32_t TCOLS = 4 * N2 <= 256 ? 256 : 512;
 };
 
-// Warp roles of the state kernel: warps 0-7 epilogue (warp w reads TMEM lane quarter w % 4 and
-// the column half w / 4 of every BV-wide group), warp 8 issues the MMAs, warp 9 the loads.  Every
-// hand-off is an mbarrier; every wait is bounded.
-constexpr int ST_THREADS = 320;
-constexpr int EPI_THREADS = 256;
-constexpr int EPI_WARPS = EPI_THREADS / 32;
+// Warp roles of the state kernel: warps 0-15 epilogue (warp w reads TMEM lane quarter w % 4 and
+// the column quarter w / 4 of every BV-wide group), warp 16 issues the MMAs, warp 17 the loads.
+// Every hand-off is an mbarrier (no CTA-wide barrier inside the chunk loop); every wait is bounded.
+constexpr int EPI_WARPS = 16;
+constexpr int EPI_THREADS = 32 * EPI_WARPS;
+constexpr int ST_THREADS = EPI_THREADS + 64;
 
 struct StateBars {
     uint64_t full[2];      // chunk inputs landed (tx)
     uint64_t empty[2];     // chunk buffer released: the MMAs reading it (commit) + every epilogue warp
-    uint64_t s_ready, y_ready;           // epilogue -> MMA: S^T tile, Y / DY tiles written
+    uint64_t s_ready;      // S^T tile written (every epilogue warp)
+    uint64_t y_ready;      // Y / DY tiles written (lane quarters 0-1), earlier chunk's output done (2-3)
+    uint64_t ox_full;      // output partial sums of the Mqk_lo rows written (lane quarters 0-1)
     uint64_t d1_full, d4_full, d3_full;  // MMA -> epilogue: accumulators complete
     uint64_t drain;                      // the MMA thread's last operations
 };
 
 template <int N>
 __device__ __forceinline__ void tmem_ld_n(uint32_t a, float (&v)[N]) {
-    if constexpr (N == 16) tmem_ld16(a, v);
+    if constexpr (N == 8) tmem_ld8(a, v);
+    else if constexpr (N == 16) tmem_ld16(a, v);
     else tmem_ld32(a, v);
 }
 
@@ -366,7 +371,15 @@ __device__ __forceinline__ const uint8_t *record(const ScanArgs &p, const uint8_
     return ws + kRecOffset + (((size_t)blockIdx.z * p.H + blockIdx.y) * nch + c) * GdnRec<DK>::BYTES;
 }
 
-// 10 warps: the sub-partition holding three of them caps a thread at 168 registers.
+// One arrival per warp on `bar` once every lane's earlier writes (shared memory, for the tensor
+// core) and TMEM reads are complete.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
+    fence_async_smem();
+    fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+}
+
 template <int DK>
 __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                                                                  const __grid_constant__ GdnMaps maps,
@@ -392,8 +405,9 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             mbar_init(&bars.full[i], 1);
             mbar_init(&bars.empty[i], 1 + EPI_WARPS);
         }
-        mbar_init(&bars.s_ready, 1);
-        mbar_init(&bars.y_ready, 1);
+        mbar_init(&bars.s_ready, EPI_WARPS);
+        mbar_init(&bars.y_ready, EPI_WARPS);
+        mbar_init(&bars.ox_full, EPI_WARPS / 2);
         mbar_init(&bars.d1_full, 1);
         mbar_init(&bars.d4_full, 1);
         mbar_init(&bars.d3_full, 1);
@@ -422,12 +436,13 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 const int c0 = c * C;
                 mbar_expect_tx(bar, bytes);
                 for (int blk = 0; blk < DK / 64; ++blk) {
-                    uint8_t *dst = buf + LY::B_KQW + blk * LY::KQW_BLK;
+                    uint8_t *dst = buf + LY::B_KWQ + blk * LY::KWQ_BLK;
                     tma_load_4d(dst, &maps.k, blk * 64, h, c0, b, bar);
-                    tma_load_4d(dst + C * 128, &maps.q, blk * 64, h, c0, b, bar);
-                    bulk_g2s(dst + 2 * C * 128, rec + RC::WK + blk * RC::WK_BLK, RC::WK_BLK, bar);
+                    bulk_g2s(dst + C * 128, rec + RC::WK + blk * RC::WK_BLK, RC::WK_BLK, bar);
+                    tma_load_4d(dst + 2 * C * 128, &maps.q, blk * 64, h, c0, b, bar);
                 }
-                bulk_g2s(buf + LY::B_MQ, rec + RC::MQK, 2 * C * 128, bar);
+                bulk_g2s(buf + LY::B_MQ, rec + RC::MQK + C * 128, C * 128, bar);   // Mqk_lo
+                bulk_g2s(buf + LY::B_MQ + C * 128, rec + RC::MQK, C * 128, bar);   // Mqk_hi
                 bulk_g2s(buf + LY::B_U, rec + RC::U + blockIdx.x * RC::U_SLICE, LY::U_BYTES, bar);
                 bulk_g2s(buf + LY::B_G, rec + RC::G, C * 4, bar);
                 issued = c;
@@ -439,7 +454,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
     } else if (warp == EPI_WARPS) {
         // ---------------- MMA issue ----------------
         if (lane == 0) {
-            auto oKQW = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::KQW_BLK); };
+            auto oKWQ = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::KWQ_BLK); };
             auto oK0 = [](int ks) { return (uint64_t)koff_k_sw128(ks, 0); };
             auto oMN = [](int ks) { return (uint64_t)koff_mn_sw128(ks); };
             const uint64_t dS2 = make_desc(sb + LY::S, LY::S_BLK, 1024, 2);
@@ -447,36 +462,43 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             const uint64_t dDY2 = make_desc(sb + LY::DY, LY::Y_BLK, 1024, 2);
             const uint32_t idS = idesc_bf16(128, N2, 0, 1);
             const uint32_t id4 = idesc_bf16(DK, N2, 1, 1);
-            for (int c = 0; c < nch; ++c) {
+            bool ok = nch == 0 || mbar_wait(&bars.full[0], 0, status);
+            for (int c = 0; c < nch && ok; ++c) {
                 const uint32_t bb = sb + (c & 1) * LY::BUF;
-                if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status)) { fail(); break; }
-                // S_c written (which also means the output epilogue of chunk c - 2 is done with
-                // this D1 buffer: the epilogue warps work through the chunks in order)
-                if (!mbar_wait(&bars.s_ready, c & 1, status)) { fail(); break; }
+                // S_c written (which also means every epilogue read of this D1 buffer, two chunks
+                // back, is done: the epilogue warps work through the chunks in order)
+                if (!mbar_wait(&bars.s_ready, c & 1, status)) { ok = false; break; }
                 fence_after_sync();
-                const uint64_t dQW = make_desc(bb + LY::B_KQW + C * 128, 16, 1024, 2);
-                mma_steps<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dQW, dS2, oKQW, oMN, false);
+                const uint64_t dWQ = make_desc(bb + LY::B_KWQ + C * 128, 16, 1024, 2);
+                mma_steps<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dWQ, dS2, oKWQ, oMN, false);
                 mma_commit(&bars.d1_full);
-                // Y_c written (and the output epilogue of chunk c - 1 is done with D3)
-                if (!mbar_wait(&bars.y_ready, c & 1, status)) { fail(); break; }
+                // Y_c written, and the output epilogue of chunk c - 1 is done with D3
+                if (!mbar_wait(&bars.y_ready, c & 1, status)) { ok = false; break; }
                 fence_after_sync();
-                const uint64_t dKt = make_desc(bb + LY::B_KQW, LY::KQW_BLK, 1024, 2);
+                const uint64_t dKt = make_desc(bb + LY::B_KWQ, LY::KWQ_BLK, 1024, 2);
                 mma_steps<C / 16>(tb + LY::cD4, id4, dKt, dDY2, oMN, oMN, false);
                 mma_commit(&bars.d4_full);
                 const uint64_t dMQ = make_desc(bb + LY::B_MQ, 16, 1024, 2);
                 mma_steps<C / 16>(tb + LY::cD3, idS, dMQ, dY2, oK0, oMN, false);
                 mma_commit(&bars.d3_full);
                 mma_commit(&bars.empty[c & 1]);
+                // the next chunk's inputs, off the chain while the state epilogue runs
+                if (c + 1 < nch && !mbar_wait(&bars.full[(c + 1) & 1], ((c + 1) >> 1) & 1, status)) {
+                    ok = false;
+                    break;
+                }
             }
+            if (!ok) fail();
             mma_commit(&bars.drain);
             mbar_wait(&bars.drain, 0, nullptr);
         }
     } else {
-        // ---------------- epilogue: warps 0-7 ----------------
+        // ---------------- epilogue: warps 0-15 ----------------
         __nv_bfloat16 *o = (__nv_bfloat16 *)p.o;
         const int q = warp & 3;            // TMEM lane quarter
         const int j0 = (warp >> 2) * CH;   // first column of this warp in each BV-wide group
         const int lrow = 32 * q + lane;    // TMEM lane of this thread
+        const bool lowq = q < 2;           // lanes 0..63: X_s -> Y, and the Mqk_lo output partial
         // state rows: lane = row for M = 128 (d = 128); lanes 32q + r, r < 16, for M = 64
         const bool own_d = (DK == 128) ? true : (lane < 16);
         const int d_row = (DK == 128) ? lrow : (16 * q + lane);
@@ -493,22 +515,21 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             for (int j = 0; j < CH; ++j) Sreg[j] = p.S0[(head * dv + v0 + j0 + j) * DK + d_row];
         }
         if (own_d) store_half_pair<BV, CH>(sm + LY::S, LY::S_BLK, d_row, j0, Sreg);
-        fence_async_smem();
-        named_sync(1, EPI_THREADS);
-        if (tid == 0) mbar_arrive(&bars.s_ready);
-        for (int c = 0; c < nch; ++c) {
+        warp_arrive(&bars.s_ready, lane);
+        bool ok = true;
+        for (int c = 0; c < nch && ok; ++c) {
             const int c0 = c * C, n = min(C, T - c0);
             const uint8_t *buf = sm + (c & 1) * LY::BUF;
-            bool bad = !mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status);
-            bad = bad || !mbar_wait(&bars.d1_full, c & 1, status);
-            if (named_sync_or(1, EPI_THREADS, bad)) { fail(); break; }
-            fence_after_sync();
+            if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status)) { ok = false; break; }
             const float *g = reinterpret_cast<const float *>(buf + LY::B_G);
             const float g_last = g[C - 1];
             const uint32_t d1 = LY::cD1 + (c & 1) * N2;
-            // Y = U - X_s (rows 64..127 of D1), and D Y
-            if (q >= 2) {
-                const int t = lrow - 64;
+            // Y = U - X_s (lanes 0..63 of D1), and D Y
+            if (lowq) {
+                const int t = lrow;
+                const float dd = t < n ? __expf(g_last - g[t]) : 0.f;
+                if (!mbar_wait(&bars.d1_full, c & 1, status)) { ok = false; break; }
+                fence_after_sync();
                 float xh[CH], xl[CH], y[CH];
                 tmem_ld_n<CH>(taddr(tb, 32 * q, d1 + j0), xh);
                 tmem_ld_n<CH>(taddr(tb, 32 * q, d1 + BV + j0), xl);
@@ -526,42 +547,33 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                     }
                 }
                 store_half_pair<BV, CH>(sm + LY::Y, LY::Y_BLK, t, j0, y);
-                const float dd = t < n ? __expf(g_last - g[t]) : 0.f;
 #pragma unroll
                 for (int j = 0; j < CH; ++j) y[j] *= dd;
                 store_half_pair<BV, CH>(sm + LY::DY, LY::Y_BLK, t, j0, y);
             }
-            fence_async_smem();
-            fence_before_sync();
-            named_sync(1, EPI_THREADS);
-            if (tid == 0) mbar_arrive(&bars.y_ready);
+            warp_arrive(&bars.y_ready, lane);
             // state update S^T <- e^{g_n} S^T + K^T D Y
-            bad = !mbar_wait(&bars.d4_full, c & 1, status);
-            if (named_sync_or(1, EPI_THREADS, bad)) { fail(); break; }
-            fence_after_sync();
             {
+                const float gC = __expf(g_last);
+                if (!mbar_wait(&bars.d4_full, c & 1, status)) { ok = false; break; }
+                fence_after_sync();
                 float xh[CH], xl[CH];
                 tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD4 + j0), xh);
                 tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD4 + BV + j0), xl);
                 tmem_wait_ld();
-                const float gC = __expf(g_last);
                 if (own_d) {
 #pragma unroll
                     for (int j = 0; j < CH; ++j) Sreg[j] = fmaf(gC, Sreg[j], xh[j] + xl[j]);
                     store_half_pair<BV, CH>(sm + LY::S, LY::S_BLK, d_row, j0, Sreg);
                 }
             }
-            fence_async_smem();
-            fence_before_sync();
-            named_sync(1, EPI_THREADS);
-            if (tid == 0) mbar_arrive(&bars.s_ready);
-            // output O = diag(e^g) QS + Mqk Y: the Mqk_lo rows (lanes 64..127) pass their
-            // partial sums through shared memory to the threads that own the output rows
-            bad = !mbar_wait(&bars.d3_full, c & 1, status);
-            if (named_sync_or(1, EPI_THREADS, bad)) { fail(); break; }
+            warp_arrive(&bars.s_ready, lane);
+            // output O = diag(e^g) QS + Mqk Y: the Mqk_lo rows (lanes 0..63) pass their partial
+            // sums through shared memory to the threads of the output rows (lanes 64..127)
+            if (!mbar_wait(&bars.d3_full, c & 1, status)) { ok = false; break; }
             fence_after_sync();
-            if (q >= 2) {
-                const int t = lrow - 64;
+            if (lowq) {
+                const int t = lrow;
                 float a[CH], bb[CH];
                 tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD3 + j0), a);
                 tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD3 + BV + j0), bb);
@@ -571,10 +583,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                     *reinterpret_cast<float4 *>(ox + t * LY::OXS + j0 + j4) =
                         make_float4(a[j4] + bb[j4], a[j4 + 1] + bb[j4 + 1], a[j4 + 2] + bb[j4 + 2],
                                     a[j4 + 3] + bb[j4 + 3]);
-            }
-            named_sync(1, EPI_THREADS);
-            if (q < 2) {
-                const int t = lrow;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars.ox_full);
+            } else {
+                const int t = lrow - 64;
                 float up[CH], qs[CH];
                 {
                     float a[CH], bb[CH];
@@ -589,6 +601,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
 #pragma unroll
                     for (int j = 0; j < CH; ++j) qs[j] = a[j] + bb[j];
                 }
+                if (!mbar_wait(&bars.ox_full, c & 1, status)) { ok = false; break; }
                 if (t < n && out) {
                     const float gt = __expf(g[t]);
                     __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t) * H + h) * dv + v0 + j0;
@@ -612,12 +625,11 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                     }
                 }
             }
-            // D1 / D3 reads done before the MMA thread reuses them (it learns so from later
-            // hand-offs of these warps); the chunk buffer (g, U) is released
-            fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.empty[c & 1]);
+            // D1 / D3 reads done (the MMA thread learns so from this warp's later arrivals); the
+            // chunk buffer (g, U) is released
+            warp_arrive(&bars.empty[c & 1], lane);
         }
+        if (!ok) fail();
         if (p.S_final && own_d && !failed()) {
 #pragma unroll
             for (int j = 0; j < CH; ++j) p.S_final[(head * dv + v0 + j0 + j) * DK + d_row] = Sreg[j];
