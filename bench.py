@@ -14,11 +14,12 @@ With N > 1 (torchrun, one process per GPU) every rank processes its own batch (w
 B*H sequences are independent, so there is no collective in the data path).
 
 Besides the headline line's required keys the JSON line carries: roofline (HBM-bound; algorithmic
-bytes per step over the summed device time of the step's launches, each launch timed by CUDA events
-the library records around it, against the measured copy bandwidth), cpu_baseline (the fp64 oracle on a bounded
-sample, rank 0 at N = 1), e2e (through the public API with pinned-host inputs copied in and the
-outputs copied back inside the timed region), clocks sampled during the timed region, and the
-decode step (B=256, H=32, d=128, L=4) as a secondary measurement.
+bytes per step over the summed device time of the step's launches, each launch timed by CUDA
+events the library records around it, against the measured copy bandwidth), cpu_baseline (the
+fp64 oracle on a bounded sample, rank 0 at N = 1), e2e (through the public API with pinned-host
+inputs copied in and the outputs copied back inside the timed region), clocks sampled during the
+timed region, and, as secondary measurements, the decode step (B=256, H=32, d=128, L=4) and the
+two rank-L scan workloads (recsys, long).
 """
 from __future__ import annotations
 
@@ -57,12 +58,12 @@ def load_peaks():
 STEP_KERNELS = {
     "gdn": ["gdn_prep_kernel", "gdn_state_kernel"],
 }
-_GDN_SOURCES = ["csrc/scan_gdn.cu", "csrc/tc.cuh", "csrc/chunk_common.cuh", "csrc/common.cuh",
-                "../include/prism.h"]
+_GDN_SOURCES = ["csrc/scan_gdn.cu", "csrc/tc.cuh", "csrc/chunk_common.cuh", "csrc/common.cuh"]
 KERNEL_SOURCES = {
     "gdn_prep_kernel": _GDN_SOURCES,
     "gdn_state_kernel": _GDN_SOURCES,
-    "decode_kernel": ["csrc/decode.cu", "csrc/common.cuh", "../include/prism.h"],
+    "decode_kernel": ["csrc/decode.cu", "csrc/common.cuh"],
+    "scan_tc_kernel": ["csrc/scan_tc.cu", "csrc/tc.cuh", "csrc/chunk_common.cuh", "csrc/common.cuh"],
 }
 
 
@@ -261,6 +262,65 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def time_workload(wl, dev, stream, peaks, rank, max_over_ranks, barrier, world, steps=5):
+    """One scan workload timed on its own: device-resident seeded inputs (larger than L2), one
+    warm-up call, `steps` timed calls with CUDA events around each launch (library probe)."""
+    import torch
+
+    from delta_rule_sequence_b200 import prism
+    from delta_rule_sequence_b200.workloads import make_inputs
+
+    x = {n: (None if t is None else t.to(dev)) for n, t in make_inputs(wl, seed=7 + rank).items()}
+    o = torch.empty((wl.B, wl.T, wl.H, wl.dv), dtype=wl.torch_io, device=dev)
+    S = torch.empty((wl.B, wl.H, wl.dv, wl.dk), dtype=torch.float32, device=dev)
+    shape = prism.make_shape(x["q"], x["v"], x["u"], wl.chunk)
+    ws = prism.workspace_for(shape, dev)
+    n_launch = prism.prism_scan_fwd_launch_count(shape)
+
+    def call():
+        prism.prism_scan_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["u"], x["w"], x["S0"],
+                             chunk=wl.chunk, o=o, S_final=S, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        call()
+    stream.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)] for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for row in evs:
+            for e in row:
+                e.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(steps):
+            prism.record_launch_events(evs[i])
+            call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    status = prism.prism_query_device_status(ws, stream)
+    if status != prism.PRISM_OK:
+        raise SystemExit(f"bench: device status after {wl.name}: {prism.status_string(status)}")
+    ms = max_over_ranks(e0.elapsed_time(e1)) / steps
+    launch_ms = [sum(r[j].elapsed_time(r[j + 1]) for r in evs) / steps for j in range(n_launch)]
+    kern_ms = sum(launch_ms)
+    alg = scan_bytes(wl)
+    achieved = alg / (kern_ms / 1e3) / 1e9
+    del x, o, S
+    return {"workload": workload_config(wl)["workload"], "ms_per_call": ms,
+            "tokens_per_s": world * wl.B * wl.T / (ms / 1e3), "launches": n_launch,
+            "ms_per_launch": launch_ms,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "algorithmic_bytes": alg, "algorithmic_flops": scan_flops(wl),
+                         "tensor_frac_algorithmic": scan_flops(wl) / (kern_ms / 1e3) / 1e12
+                         / peaks["bf16_tflops"]},
+            "steps": steps}
+
+
 def workload_config(wl):
     return {"workload": f"{wl.name}: B={wl.B} H={wl.H} T={wl.T} dk={wl.dk} dv={wl.dv} L={wl.L} "
                         f"chunk={wl.chunk} io={wl.io} state=f32 write={wl.write}",
@@ -278,6 +338,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the secondary timing of the recsys and long workloads")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -511,6 +573,13 @@ def main():
                   "bytes_per_step": db, "steps": args.decode_steps,
                   "inputs": "4 seeded step batches cycled; state carried across steps"}
 
+    # ---- secondary: the other scan workloads (rank-L writes), each timed alone on its own inputs
+    others = {}
+    if not args.no_configs:
+        for name in ("recsys", "long"):
+            others[name] = time_workload(WORKLOADS[name], dev, stream, peaks, rank, max_over_ranks,
+                                         barrier, world)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, threads = cpu_oracle_sample(wl)
@@ -531,6 +600,7 @@ def main():
         "config": dict(workload_config(wl), parallelism=f"dp{world} over (b,h) sequences"),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps, "clocks": clocks, "decode": decode,
+        "other_workloads": others or None,
     }
     print(json.dumps(line), flush=True)
 

@@ -18,6 +18,10 @@ int segmented_combine_launches(int G, bool with_state);
 size_t segmented_extra_bytes(int B, int H, int G, int dk, int dv);
 cudaError_t launch_segmented(const ScanArgs &a, int route, bool io_f32, int G, void *ws,
                              size_t rec_bytes, cudaStream_t s);
+cudaError_t launch_segment_element(const ScanArgs &a, int route, bool io_f32, void *ws, float *e_out,
+                                   float *f_out, cudaStream_t s);
+cudaError_t launch_state_fold(int BH, int dk, int dv, const float *S_in, const float *E, const float *f,
+                              float *S_out, cudaStream_t s);
 }  // namespace prism
 
 namespace {
@@ -212,6 +216,44 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
             default: err = prism::launch_scan_simt(a, io_f32, s); break;
         }
     }
+    probe_finish(s);
+    return cuda_status(err);
+}
+
+prism_status prism_scan_segment_element(const prism_shape *shape, const void *q, const void *k,
+                                        const void *v, const float *alpha, const float *beta,
+                                        const void *u, const void *w, float *E, float *f,
+                                        void *workspace, size_t ws_bytes, void *stream) {
+    prism_status st = check_common(shape, q, k, v, alpha, beta, u, w);
+    if (st != PRISM_OK) return st;
+    if (shape->chunk != 64 && shape->chunk != 128) return PRISM_ERR_INVALID_ARG;
+    if (shape->dk != shape->dv) return PRISM_ERR_UNSUPPORTED;
+    size_t need = 0;
+    prism_scan_fwd_workspace_size(shape, &need);
+    if (!workspace || ws_bytes < need || ((uintptr_t)workspace & 255u)) return PRISM_ERR_INVALID_ARG;
+    if (shape->B == 0 || shape->H == 0) return PRISM_OK;
+    if (!E || !f || !aligned16(E) || !aligned16(f) || E == f) return PRISM_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, nullptr, nullptr, nullptr,
+                                  (uint32_t *)workspace);
+    const Plan plan = plan_for(shape, u == nullptr);
+    const int route = plan == Plan::TcGdnSplit ? 2 : plan == Plan::TcFused ? 1 : 0;
+    cudaError_t err = prism::launch_segment_element(a, route, shape->io == PRISM_F32, workspace, E, f, s);
+    probe_finish(s);
+    return cuda_status(err);
+}
+
+prism_status prism_state_fold(int BH, int dk, int dv, const float *S_in, const float *E,
+                              const float *f, float *S_out, void *stream) {
+    if (BH < 0 || dk < 1 || dv < 1) return PRISM_ERR_INVALID_ARG;
+    if (!width_ok(dk) || !width_ok(dv)) return PRISM_ERR_UNSUPPORTED;
+    if (BH == 0) return PRISM_OK;
+    if (!E || !f || !S_out || !aligned16(E) || !aligned16(f) || !aligned16(S_out) ||
+        (S_in && !aligned16(S_in)))
+        return PRISM_ERR_INVALID_ARG;
+    if (S_out == E || S_out == f) return PRISM_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t err = prism::launch_state_fold(BH, dk, dv, S_in, E, f, S_out, s);
     probe_finish(s);
     return cuda_status(err);
 }

@@ -182,7 +182,72 @@ cudaError_t combine(const SegTree &t, const float *S0, float *S_final, cudaStrea
     return cudaGetLastError();
 }
 
+// S_out = S_in E + f for every (b, h): S_in, f, S_out [BH, dv, D], E [BH, D, D].  S_out may be
+// S_in (each CTA stages its own rows before writing them).  grid: x = b * H + h, y = row blocks.
+template <int D>
+__global__ void __launch_bounds__(NTH) state_fold_kernel(const float *S_in, const float *E, const float *f,
+                                                         float *S_out, int dv) {
+    extern __shared__ float smem[];
+    float *sE = smem, *sx = smem + D * D;
+    const size_t bh = blockIdx.x, fe = (size_t)dv * D;
+    rows_times<D>(S_in + bh * fe, E + bh * D * D, f + bh * fe, S_out + bh * fe, dv, blockIdx.y, sE, sx);
+}
+
+template <int D>
+cudaError_t fold_t(int BH, int dv, const float *S_in, const float *E, const float *f, float *S_out,
+                   cudaStream_t s) {
+    const size_t smem = ((size_t)D * D + (size_t)RB * (D + 1)) * sizeof(float);
+    cudaError_t err = cudaFuncSetAttribute(state_fold_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    launch_probe_mark(s);
+    state_fold_kernel<D><<<dim3(BH, (dv + RB - 1) / RB), NTH, smem, s>>>(S_in, E, f, S_out, dv);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+// S_out = S_in E + f per (b, h) (S_in NULL: S_out = f).  dk in {32, 64, 128}.
+cudaError_t launch_state_fold(int BH, int dk, int dv, const float *S_in, const float *E, const float *f,
+                              float *S_out, cudaStream_t s) {
+    if (BH == 0) return cudaSuccess;
+    if (!S_in) {
+        launch_probe_mark(s);
+        return cudaMemcpyAsync(S_out, f, (size_t)BH * dv * dk * sizeof(float), cudaMemcpyDeviceToDevice, s);
+    }
+    switch (dk) {
+        case 128: return fold_t<128>(BH, dv, S_in, E, f, S_out, s);
+        case 64: return fold_t<64>(BH, dv, S_in, E, f, S_out, s);
+        case 32: return fold_t<32>(BH, dv, S_in, E, f, S_out, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+// The affine map of each (b, h) sequence of `a` (dk == dv): E into e_out ([B, H, dk, dk]) from
+// S0 = I with the write off, f into f_out ([B, H, dv, dk]) from S0 = 0 with the write; no outputs.
+cudaError_t launch_segment_element(const ScanArgs &a, int route, bool io_f32, void *ws, float *e_out,
+                                   float *f_out, cudaStream_t s) {
+    auto pass = [&](const ScanArgs &x) -> cudaError_t {
+        switch (route) {
+            case 2: return launch_gdn_state(x, ws, s);
+            case 1: return launch_scan_tc(x, s);
+            default: return launch_scan_simt(x, io_f32, s);
+        }
+    };
+    cudaError_t err = cudaSuccess;
+    if (route == 2 && a.T > 0 && (err = launch_gdn_prep(a, ws, s)) != cudaSuccess) return err;
+    ScanArgs e = a;
+    e.S0 = nullptr;
+    e.o = nullptr;
+    e.flags = kNoWrite | kS0Identity | kNoOutput;
+    e.S_final = e_out;
+    if ((err = (route == 2 && a.T == 0) ? launch_scan_tc(e, s) : pass(e)) != cudaSuccess) return err;
+    ScanArgs f = a;
+    f.S0 = nullptr;
+    f.o = nullptr;
+    f.flags = kNoOutput;
+    f.S_final = f_out;
+    return (route == 2 && a.T == 0) ? launch_scan_tc(f, s) : pass(f);
+}
 
 // Kernels one segmented scan launches besides the passes: slot-0 init, the up- and down-sweep
 // levels, and the exit state.

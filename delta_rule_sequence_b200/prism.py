@@ -24,6 +24,8 @@ EXPORTS = (
     "prism_scan_fwd_launch_count",
     "prism_scan_fwd",
     "prism_scan_fwd_noalloc",
+    "prism_scan_segment_element",
+    "prism_state_fold",
     "prism_step_decode",
     "prism_query_device_status",
     "prism_status_string",
@@ -73,6 +75,10 @@ def load_library():
     lib.prism_scan_fwd.restype = ci
     lib.prism_scan_fwd_noalloc.argtypes = [shp] + [vp] * 10 + [vp]
     lib.prism_scan_fwd_noalloc.restype = ci
+    lib.prism_scan_segment_element.argtypes = [shp] + [vp] * 9 + [vp, sz, vp]
+    lib.prism_scan_segment_element.restype = ci
+    lib.prism_state_fold.argtypes = [ci, ci, ci, vp, vp, vp, vp, vp]
+    lib.prism_state_fold.restype = ci
     lib.prism_step_decode.argtypes = [shp] + [vp] * 9 + [vp]
     lib.prism_step_decode.restype = ci
     lib.prism_query_device_status.argtypes = [vp, vp]
@@ -263,3 +269,58 @@ def record_launch_events(events) -> None:
     rc = load_library().prism_debug_record_launch_events(handles, len(events))
     if rc != PRISM_OK:
         raise PrismError(rc, "prism_debug_record_launch_events")
+
+
+def prism_scan_segment_element(q, k, v, alpha, beta, u=None, w=None, *, chunk=64, E=None, f=None,
+                               workspace=None, stream=None):
+    """Affine map (E, f) of each (b, h) sequence over these T tokens: S -> S E + f.
+    E: [B,H,dk,dk] fp32, f: [B,H,dv,dk] fp32 (allocated when not given).  Requires dk == dv."""
+    lib = load_library()
+    dev = q.device
+    io = q.dtype
+    B, T, H, dk = q.shape
+    shape = make_shape(q, v, u, chunk)
+    dv, L = shape.dv, shape.L
+    _check_tensor("q", q, io, (B, T, H, dk), dev)
+    _check_tensor("k", k, io, (B, T, H, dk), dev)
+    _check_tensor("v", v, io, (B, T, H, dv), dev)
+    _check_tensor("alpha", alpha, torch.float32, (B, T, H), dev)
+    _check_tensor("beta", beta, torch.float32, (B, T, H), dev)
+    _check_tensor("u", u, io, (B, T, H, L, dv), dev)
+    _check_tensor("w", w, io, (B, T, H, L, dk), dev)
+    if E is None:
+        E = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev)
+    if f is None:
+        f = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    _check_tensor("E", E, torch.float32, (B, H, dk, dk), dev)
+    _check_tensor("f", f, torch.float32, (B, H, dv, dk), dev)
+    if workspace is None:
+        workspace = workspace_for(shape, dev)
+    rc = lib.prism_scan_segment_element(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                        _ptr(beta), _ptr(u), _ptr(w), _ptr(E), _ptr(f), _ptr(workspace),
+                                        ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if rc != PRISM_OK:
+        raise PrismError(rc, "prism_scan_segment_element")
+    return E, f
+
+
+def prism_state_fold(S_in, E, f, S_out=None, stream=None):
+    """S_out = S_in E + f per state; S_in None means zero.  S_in, f, S_out: [..., dv, dk] fp32,
+    E: [..., dk, dk] fp32 with the same leading dims."""
+    lib = load_library()
+    dv, dk = f.shape[-2], f.shape[-1]
+    lead = tuple(f.shape[:-2])
+    BH = 1
+    for n in lead:
+        BH *= n
+    dev = f.device
+    _check_tensor("E", E, torch.float32, lead + (dk, dk), dev)
+    _check_tensor("f", f, torch.float32, lead + (dv, dk), dev)
+    _check_tensor("S_in", S_in, torch.float32, lead + (dv, dk), dev)
+    if S_out is None:
+        S_out = torch.empty_like(f)
+    _check_tensor("S_out", S_out, torch.float32, lead + (dv, dk), dev)
+    rc = lib.prism_state_fold(BH, dk, dv, _ptr(S_in), _ptr(E), _ptr(f), _ptr(S_out), _stream(stream))
+    if rc != PRISM_OK:
+        raise PrismError(rc, "prism_state_fold")
+    return S_out

@@ -102,6 +102,30 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
                             float *S_final, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * prism_scan_segment_element -- the affine map of a token segment, the building block of a scan
+ * split across devices along T ("Sequential Parallel Duality in Prefix Scannable Models", method
+ * overview: every chunk is an element of an associative operator and elements compose in order).
+ * For every (b, h), the recurrence over the segment sends any entry state S to  S E + f  with
+ *   E        [B,H,dk,dk] fp32  the product of the per-token transitions alpha_t (I - beta_t k_t k_t^T)
+ *   f        [B,H,dv,dk] fp32  the exit state from S = 0 (the writes carried to the segment end)
+ * Requires dk == dv.  Other arguments, the workspace and the rounding are as for prism_scan_fwd
+ * (no S0, no outputs).  E and f must not overlap.
+ */
+prism_status prism_scan_segment_element(const prism_shape *shape, const void *q, const void *k,
+                                        const void *v, const float *alpha, const float *beta,
+                                        const void *u, const void *w, float *E, float *f,
+                                        void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * prism_state_fold -- S_out = S_in E + f for each of BH states (the element composition of
+ * prism_scan_segment_element applied to a state): S_in, f, S_out [BH,dv,dk] fp32, E [BH,dk,dk]
+ * fp32; S_in NULL means zero (S_out = f); S_out may be S_in but not E or f.  fp32 on CUDA cores.
+ * dk, dv in {32, 64, 128}.
+ */
+prism_status prism_state_fold(int BH, int dk, int dv, const float *S_in, const float *E,
+                              const float *f, float *S_out, void *stream);
+
+/*
  * prism_step_decode -- one token for each of the B*H sequences (shape->T must be 1):
  *   S <- alpha S (I - beta k k^T) + sum_l u_l w_l^T   (in place),   o = S q.
  * Arguments as for prism_scan_fwd with T == 1; S is read and written in place, [B,H,dv,dk]
