@@ -89,8 +89,8 @@ Plan plan_for(const prism_shape *s, bool gdn_write) {
 }
 
 // Debug flag bits (prism_debug_set_flags): 2 = take the segmented scan whenever the shape allows
-// it, 4 = never take it.
-constexpr int kForceSegments = 2, kNoSegments = 4;
+// it, 4 = never take it, 8 = the stall test of the Gated-DeltaNet state kernel (its waits give up).
+constexpr int kForceSegments = 2, kNoSegments = 4, kDebugStall = 8;
 
 // Number of segments G of the segmented inter-chunk scan (1 = one in-order pass per sequence).
 // It needs dk == dv (the identity pass) and T divisible by G with at least one chunk per segment.
@@ -199,6 +199,7 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
     if (shape->T == 0 && !S_final) return PRISM_OK;
 
     prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, S0, o, S_final, status);
+    if (g_debug_flags & kDebugStall) a.flags |= prism::kStallTest;
     const bool io_f32 = shape->io == PRISM_F32;
     cudaError_t err;
     const Plan plan = plan_for(shape, u == nullptr);

@@ -24,8 +24,13 @@ struct ScanArgs {
 
 // Flags of a scan pass.  kNoWrite: the write term is zero (u = 0 / v = 0);  kS0Identity: the entry
 // state's row r is the unit vector e_r (requires dk == dv), so S_final returns the pass's affine
-// map E;  kNoOutput: o is not written.
-enum : int { kNoWrite = 1, kS0Identity = 2, kNoOutput = 4 };
+// map E;  kNoOutput: o is not written;  kStallTest: the Gated-DeltaNet state kernel's load warp
+// issues nothing and every wait gives up after a short limit (a test of the give-up path).
+enum : int { kNoWrite = 1, kS0Identity = 2, kNoOutput = 4, kStallTest = 8 };
+
+// Poll limits of the bounded mbarrier waits: normal operation, and the stall test.
+constexpr uint32_t kWaitPolls = 1u << 24;
+constexpr uint32_t kStallTestPolls = 1u << 12;
 
 // Workspace layout: [0, 256) status block; segment data of the segmented scan after it.
 constexpr size_t kStatusBytes = 256;

@@ -420,6 +420,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
     fence_after_sync();
     const uint32_t tb = tmem_base_sh;
     uint32_t *status = p.status;
+    const uint32_t lim = (p.flags & kStallTest) ? kStallTestPolls : kWaitPolls;
     auto fail = [&]() { failed_sh = 1; };
     auto failed = [&]() { return *(volatile int *)&failed_sh != 0; };
 
@@ -428,8 +429,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
         if (lane == 0) {
             constexpr uint32_t bytes = 3 * (DK / 64) * C * 128 + 2 * C * 128 + LY::U_BYTES + C * 4;
             int issued = -1;
-            for (int c = 0; c < nch && !failed(); ++c) {
-                if (c >= 2 && !mbar_wait(&bars.empty[c & 1], ((c - 2) >> 1) & 1, status)) { fail(); break; }
+            for (int c = 0; c < nch && !failed() && !(p.flags & kStallTest); ++c) {
+                if (c >= 2 && !mbar_wait(&bars.empty[c & 1], ((c - 2) >> 1) & 1, status, lim)) { fail(); break; }
                 const uint8_t *rec = record<DK>(p, ws, nch, c);
                 uint8_t *buf = sm + (c & 1) * LY::BUF;
                 uint64_t *bar = &bars.full[c & 1];
@@ -449,7 +450,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             }
             // let the copies still in flight land before the CTA can exit
             for (int c = issued > 0 ? issued - 1 : 0; c <= issued; ++c)
-                mbar_wait(&bars.full[c & 1], (c >> 1) & 1, nullptr);
+                mbar_wait(&bars.full[c & 1], (c >> 1) & 1, nullptr, lim);
         }
     } else if (warp == EPI_WARPS) {
         // ---------------- MMA issue ----------------
@@ -462,18 +463,18 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             const uint64_t dDY2 = make_desc(sb + LY::DY, LY::Y_BLK, 1024, 2);
             const uint32_t idS = idesc_bf16(128, N2, 0, 1);
             const uint32_t id4 = idesc_bf16(DK, N2, 1, 1);
-            bool ok = nch == 0 || mbar_wait(&bars.full[0], 0, status);
+            bool ok = nch == 0 || mbar_wait(&bars.full[0], 0, status, lim);
             for (int c = 0; c < nch && ok; ++c) {
                 const uint32_t bb = sb + (c & 1) * LY::BUF;
                 // S_c written (which also means every epilogue read of this D1 buffer, two chunks
                 // back, is done: the epilogue warps work through the chunks in order)
-                if (!mbar_wait(&bars.s_ready, c & 1, status)) { ok = false; break; }
+                if (!mbar_wait(&bars.s_ready, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 const uint64_t dWQ = make_desc(bb + LY::B_KWQ + C * 128, 16, 1024, 2);
                 mma_steps<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dWQ, dS2, oKWQ, oMN, false);
                 mma_commit(&bars.d1_full);
                 // Y_c written, and the output epilogue of chunk c - 1 is done with D3
-                if (!mbar_wait(&bars.y_ready, c & 1, status)) { ok = false; break; }
+                if (!mbar_wait(&bars.y_ready, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 const uint64_t dKt = make_desc(bb + LY::B_KWQ, LY::KWQ_BLK, 1024, 2);
                 mma_steps<C / 16>(tb + LY::cD4, id4, dKt, dDY2, oMN, oMN, false);
@@ -483,14 +484,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 mma_commit(&bars.d3_full);
                 mma_commit(&bars.empty[c & 1]);
                 // the next chunk's inputs, off the chain while the state epilogue runs
-                if (c + 1 < nch && !mbar_wait(&bars.full[(c + 1) & 1], ((c + 1) >> 1) & 1, status)) {
+                if (c + 1 < nch && !mbar_wait(&bars.full[(c + 1) & 1], ((c + 1) >> 1) & 1, status, lim)) {
                     ok = false;
                     break;
                 }
             }
             if (!ok) fail();
             mma_commit(&bars.drain);
-            mbar_wait(&bars.drain, 0, nullptr);
+            mbar_wait(&bars.drain, 0, nullptr, lim);
         }
     } else {
         // ---------------- epilogue: warps 0-15 ----------------
@@ -520,7 +521,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
         for (int c = 0; c < nch && ok; ++c) {
             const int c0 = c * C, n = min(C, T - c0);
             const uint8_t *buf = sm + (c & 1) * LY::BUF;
-            if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status)) { ok = false; break; }
+            if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status, lim)) { ok = false; break; }
             const float *g = reinterpret_cast<const float *>(buf + LY::B_G);
             const float g_last = g[C - 1];
             const uint32_t d1 = LY::cD1 + (c & 1) * N2;
@@ -528,7 +529,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             if (lowq) {
                 const int t = lrow;
                 const float dd = t < n ? __expf(g_last - g[t]) : 0.f;
-                if (!mbar_wait(&bars.d1_full, c & 1, status)) { ok = false; break; }
+                if (!mbar_wait(&bars.d1_full, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 float xh[CH], xl[CH], y[CH];
                 tmem_ld_n<CH>(taddr(tb, 32 * q, d1 + j0), xh);
@@ -555,7 +556,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             // state update S^T <- e^{g_n} S^T + K^T D Y
             {
                 const float gC = __expf(g_last);
-                if (!mbar_wait(&bars.d4_full, c & 1, status)) { ok = false; break; }
+                if (!mbar_wait(&bars.d4_full, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 float xh[CH], xl[CH];
                 tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD4 + j0), xh);
@@ -570,7 +571,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             warp_arrive(&bars.s_ready, lane);
             // output O = diag(e^g) QS + Mqk Y: the Mqk_lo rows (lanes 0..63) pass their partial
             // sums through shared memory to the threads of the output rows (lanes 64..127)
-            if (!mbar_wait(&bars.d3_full, c & 1, status)) { ok = false; break; }
+            if (!mbar_wait(&bars.d3_full, c & 1, status, lim)) { ok = false; break; }
             fence_after_sync();
             if (lowq) {
                 const int t = lrow;
@@ -601,7 +602,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
 #pragma unroll
                     for (int j = 0; j < CH; ++j) qs[j] = a[j] + bb[j];
                 }
-                if (!mbar_wait(&bars.ox_full, c & 1, status)) { ok = false; break; }
+                if (!mbar_wait(&bars.ox_full, c & 1, status, lim)) { ok = false; break; }
                 if (t < n && out) {
                     const float gt = __expf(g[t]);
                     __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t) * H + h) * dv + v0 + j0;

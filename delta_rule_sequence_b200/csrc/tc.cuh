@@ -273,7 +273,7 @@ __device__ __forceinline__ bool named_sync_or(uint32_t id, uint32_t nthreads, bo
 // Wait for phase `parity` of `bar` to complete.  Gives up after `limit` polls (each poll blocks
 // for a bounded, implementation-defined time), records PRISM_ERR_TIMEOUT and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status,
-                                          uint32_t limit = (1u << 24)) {
+                                          uint32_t limit = kWaitPolls) {
     for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
     }

@@ -181,7 +181,10 @@ const char *prism_last_cuda_error(void);
  * prism_scan_fwd_workspace_size, which depends on it).  flags bit 1: prism_scan_fwd takes the
  * segmented inter-chunk scan (segment elements, a Blelloch scan over them, a re-run of every
  * segment) whenever the shape allows it (dk == dv, T divisible into segments of >= 64 tokens);
- * bit 2: it never does.  Returns the previous flags.
+ * bit 2: it never does; bit 3: the stall test -- the Gated-DeltaNet state kernel's load warp
+ * issues nothing, every wait gives up after a short limit, the kernel records PRISM_ERR_TIMEOUT
+ * in the workspace status word and returns (outputs are then undefined).  Returns the previous
+ * flags.
  */
 int prism_debug_set_flags(int flags);
 
