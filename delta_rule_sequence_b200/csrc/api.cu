@@ -14,6 +14,8 @@ bool scan_tc_supported(const ScanArgs &a, bool io_f32);
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
 size_t gdn_workspace_bytes(int B, int H, int T, int dk);
 cudaError_t launch_scan_gdn(const ScanArgs &a, void *ws, cudaStream_t s);
+size_t lrank_workspace_bytes(int B, int H, int T, int dk);
+cudaError_t launch_scan_lrank(const ScanArgs &a, void *ws, cudaStream_t s);
 int segmented_combine_launches(int G, bool with_state);
 size_t segmented_extra_bytes(int B, int H, int G, int dk, int dv);
 cudaError_t launch_segmented(const ScanArgs &a, int route, bool io_f32, int G, void *ws,
@@ -79,13 +81,29 @@ prism_status check_common(const prism_shape *s, const void *q, const void *k, co
     return PRISM_OK;
 }
 
-// Which kernels a prism_scan_fwd call with this shape runs.
-enum class Plan { Simt, TcFused, TcGdnSplit };
+// Which kernels a prism_scan_fwd call with this shape runs: the fp32 CUDA-core kernel; the
+// two-kernel tensor-core schedule (per-chunk prep, then the in-order state kernel) for the
+// Gated-DeltaNet or the rank-L write; the fused tensor-core kernel only copies S0 when T = 0.
+enum class Plan { Simt, TcFused, TcGdnSplit, TcRankLSplit };
 
 Plan plan_for(const prism_shape *s, bool gdn_write) {
     const bool tc = s->io == PRISM_BF16 && s->dk == s->dv && (s->dk == 64 || s->dk == 128);
     if (!tc) return Plan::Simt;
-    return gdn_write ? Plan::TcGdnSplit : Plan::TcFused;
+    if (s->T <= 0) return Plan::TcFused;
+    return gdn_write ? Plan::TcGdnSplit : Plan::TcRankLSplit;
+}
+
+bool split_plan(Plan p) { return p == Plan::TcGdnSplit || p == Plan::TcRankLSplit; }
+
+// Route number of the segmented scan and the segment element: 0 fp32, 1 fused, 2 GDN split,
+// 3 rank-L split.
+int route_of(Plan p) {
+    switch (p) {
+        case Plan::TcGdnSplit: return 2;
+        case Plan::TcRankLSplit: return 3;
+        case Plan::TcFused: return 1;
+        default: return 0;
+    }
 }
 
 // Debug flag bits (prism_debug_set_flags): 2 = take the segmented scan whenever the shape allows
@@ -119,7 +137,7 @@ int segments_for(const prism_shape *s, bool gdn_write) {
         return 1;
     };
     if (g_debug_flags & kForceSegments) return largest_G(16, 64);
-    if (plan_for(s, gdn_write) != Plan::TcGdnSplit) return 1;
+    if (!split_plan(plan_for(s, gdn_write))) return 1;
     const long long chains = (long long)s->B * s->H * (s->dv == 128 ? 4 : 1);
     const int sms = sm_count();
     if (chains * 4 > sms || s->T < 4096) return 1;
@@ -127,8 +145,9 @@ int segments_for(const prism_shape *s, bool gdn_write) {
 }
 
 size_t records_bytes(const prism_shape *s, Plan plan, int G) {
-    if (plan != Plan::TcGdnSplit || s->T <= 0 || s->B == 0 || s->H == 0) return prism::kStatusBytes;
-    return prism::gdn_workspace_bytes(s->B * G, s->H, s->T / G, s->dk);
+    if (!split_plan(plan) || s->T <= 0 || s->B == 0 || s->H == 0) return prism::kStatusBytes;
+    return plan == Plan::TcGdnSplit ? prism::gdn_workspace_bytes(s->B * G, s->H, s->T / G, s->dk)
+                                    : prism::lrank_workspace_bytes(s->B * G, s->H, s->T / G, s->dk);
 }
 
 prism::ScanArgs make_args(const prism_shape *s, const void *q, const void *k, const void *v,
@@ -158,23 +177,33 @@ extern "C" {
 // when u, w are NULL, rank-L otherwise), since the shape alone does not say which one is used.
 prism_status prism_scan_fwd_workspace_size(const prism_shape *shape, size_t *bytes) {
     if (!shape || !bytes) return PRISM_ERR_INVALID_ARG;
-    const Plan plan = plan_for(shape, shape->L == 1);
-    const int G = segments_for(shape, shape->L == 1);
-    size_t need = records_bytes(shape, plan, G);
-    if (G > 1) need += prism::segmented_extra_bytes(shape->B, shape->H, G, shape->dk, shape->dv);
+    size_t need = 0;
+    for (int gdn = 0; gdn < 2; ++gdn) {
+        if (gdn && shape->L != 1) continue;  // the Gated-DeltaNet write exists only for L = 1
+        const Plan plan = plan_for(shape, gdn);
+        const int G = segments_for(shape, gdn);
+        size_t n = records_bytes(shape, plan, G);
+        if (G > 1) n += prism::segmented_extra_bytes(shape->B, shape->H, G, shape->dk, shape->dv);
+        if (n > need) need = n;
+    }
     *bytes = need;
     return PRISM_OK;
 }
 
 prism_status prism_scan_fwd_launch_count(const prism_shape *shape, int *launches) {
     if (!shape || !launches) return PRISM_ERR_INVALID_ARG;
-    const Plan plan = plan_for(shape, shape->L == 1);
-    const int G = segments_for(shape, shape->L == 1);
-    const bool split = plan == Plan::TcGdnSplit && shape->T > 0;
-    int n = split ? 2 : 1;
-    if (G > 1) n = (split ? 1 : 0) + 3 + prism::segmented_combine_launches(G, true);
-    if (shape->B == 0 || shape->H == 0) n = 0;
-    *launches = n;
+    int most = 0;
+    for (int gdn = 0; gdn < 2; ++gdn) {
+        if (gdn && shape->L != 1) continue;
+        const Plan plan = plan_for(shape, gdn);
+        const int G = segments_for(shape, gdn);
+        const bool split = split_plan(plan);
+        int n = split ? 2 : 1;
+        if (G > 1) n = (split ? 1 : 0) + 3 + prism::segmented_combine_launches(G, true);
+        if (n > most) most = n;
+    }
+    if (shape->B == 0 || shape->H == 0) most = 0;
+    *launches = most;
     return PRISM_OK;
 }
 
@@ -205,15 +234,12 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
     const Plan plan = plan_for(shape, u == nullptr);
     const int G = segments_for(shape, u == nullptr);
     if (G > 1) {
-        const int route = plan == Plan::TcGdnSplit ? 2 : plan == Plan::TcFused ? 1 : 0;
-        err = prism::launch_segmented(a, route, io_f32, G, workspace, records_bytes(shape, plan, G), s);
+        err = prism::launch_segmented(a, route_of(plan), io_f32, G, workspace, records_bytes(shape, plan, G), s);
     } else {
         switch (plan) {
-            case Plan::TcGdnSplit:
-                err = shape->T > 0 ? prism::launch_scan_gdn(a, workspace, s)
-                                   : prism::launch_scan_tc(a, s);  // T = 0: copies S0 to S_final
-                break;
-            case Plan::TcFused: err = prism::launch_scan_tc(a, s); break;
+            case Plan::TcGdnSplit: err = prism::launch_scan_gdn(a, workspace, s); break;
+            case Plan::TcRankLSplit: err = prism::launch_scan_lrank(a, workspace, s); break;
+            case Plan::TcFused: err = prism::launch_scan_tc(a, s); break;  // T = 0: copies S0 to S_final
             default: err = prism::launch_scan_simt(a, io_f32, s); break;
         }
     }
@@ -238,8 +264,7 @@ prism_status prism_scan_segment_element(const prism_shape *shape, const void *q,
     prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, nullptr, nullptr, nullptr,
                                   (uint32_t *)workspace);
     const Plan plan = plan_for(shape, u == nullptr);
-    const int route = plan == Plan::TcGdnSplit ? 2 : plan == Plan::TcFused ? 1 : 0;
-    cudaError_t err = prism::launch_segment_element(a, route, shape->io == PRISM_F32, workspace, E, f, s);
+    cudaError_t err = prism::launch_segment_element(a, route_of(plan), shape->io == PRISM_F32, workspace, E, f, s);
     probe_finish(s);
     return cuda_status(err);
 }

@@ -43,8 +43,9 @@ struct GdnMaps {
     CUtensorMap k, q, v;
 };
 
-// One workspace record per (b, h, chunk).
-template <int DK>
+// One workspace record per (b, h, chunk).  The rank-L record (RL) adds the write's own terms:
+// O_w = sum_l Mqw_l U_l and F_w = sum_l W_l^T D U_l; its U slot holds -X_u = -T sum_l P_l U_l.
+template <int DK, bool RL = false>
 struct GdnRec {
     static constexpr int DV = DK, BV = kBV<DK>;
     static constexpr uint32_t WK_BLK = C * 128;                  // 64 rows x 128 B per 64 columns
@@ -53,7 +54,10 @@ struct GdnRec {
     static constexpr uint32_t U_SLICE = C * BV * 4;               // U, fp32, one value slice
     static constexpr uint32_t U = MQK + 2 * C * 128;
     static constexpr uint32_t G = U + U_SLICE * (DV / BV);        // g_t, 64 floats
-    static constexpr uint32_t BYTES = G + 1024;
+    static constexpr uint32_t OW = G + 1024;                      // O_w, fp32 [C][DV] (rank L)
+    static constexpr uint32_t FW_SLICE = DK * BV * 4;             // F_w, fp32, one value slice
+    static constexpr uint32_t FW = OW + (RL ? C * DV * 4 : 0);    // F_w slices [d][BV], XOR-swizzled
+    static constexpr uint32_t BYTES = FW + (RL ? FW_SLICE * (DV / BV) : 0);
 };
 constexpr size_t kRecOffset = 1024;  // records start after the status block
 
@@ -289,6 +293,359 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
 }
 
 // ------------------------------------------------------------------------------------------------
+// rank-L prep: one CTA per (chunk, head, batch), all value columns at once
+//
+// The state-independent part of a chunk with the write sum_l u_l w_l^T:
+//   G = [K; Q] K^T -> A, Mqk;  T = (I + A)^{-1};  Wk = T diag(beta e^g) K;
+//   per l:  G_l = [K; Q] W_l^T -> P_l = strict(diag(beta) Gamma o K W_l^T), Mqw_l = incl(Gamma o Q W_l^T),
+//           sum P_l U_l,  O_w += Mqw_l U_l,  F_w += W_l^T D U_l;
+//   X_u = T sum_l P_l U_l.
+// The record gets Wk, Mqk, -X_u (in the U slot, so that the state kernel's Y = U - Wk S^T holds for
+// both writes), O_w, F_w and g.
+
+struct LMaps {
+    CUtensorMap k, q, w, u;  // w, u viewed as {d, H*L, T, B}: box row (h, l) = h L + l
+};
+
+template <int DK>
+struct LPrepLayout {
+    static constexpr uint32_t KQ_BLK = 2 * C * 128;     // [K; Q] rows of one 64-column block
+    static constexpr uint32_t BLK = C * 128;            // one 64-column block of a C-row tile
+    static constexpr uint32_t KQ = 0;
+    static constexpr uint32_t W = KQ + KQ_BLK * (DK / 64);   // W_l, K-major (rows t)
+    static constexpr uint32_t U = W + BLK * (DK / 64);       // U_l, [t][dv] (MN-major B operand)
+    static constexpr uint32_t DU = U + BLK * (DK / 64);      // D U_l hi, lo; later sum P U hi, lo
+    static constexpr uint32_t DUL = DU + BLK * (DK / 64);
+    static constexpr uint32_t T1 = DUL + BLK * (DK / 64);    // T diag(beta gamma), then T: hi, lo
+    static constexpr uint32_t T1L = T1 + BLK;
+    static constexpr uint32_t MQW = T1L + BLK;               // Mqw_l hi, lo
+    static constexpr uint32_t MQWL = MQW + BLK;
+    static constexpr uint32_t AF = MQWL + BLK;               // fp32 A, solved in place into T
+    static constexpr uint32_t P = AF;                        // P_l hi, lo over the solve buffers,
+    static constexpr uint32_t PL = P + BLK;                  // free once both T tiles are built
+    static constexpr uint32_t TMP = AF + C * AS * 4;
+    static constexpr uint32_t GATES = TMP + 32 * 33 * 4;     // g, beta, gamma, D
+    static constexpr uint32_t BYTES = GATES + 4 * C * 4 + 1024;
+    static_assert(KQ_BLK * (DK / 64) >= (uint32_t)C * DK * 4, "-X_u staging fits over K and Q");
+    static_assert(PL + BLK <= GATES, "the P tiles fit over the solve buffers");
+    // TMEM: G (64 columns, M = 128), then Wk / sum P U / X_u, O_w, F_w (DK columns each)
+    static constexpr uint32_t cG = 0, cA = 64, cO = cA + DK, cF = cO + DK;
+    static constexpr uint32_t TCOLS = cF + DK <= 256 ? 256 : 512;
+};
+
+template <int DK>
+__global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid_constant__ LMaps maps,
+                                                       uint8_t *ws, int nch) {
+    using LY = LPrepLayout<DK>;
+    using RC = GdnRec<DK, true>;
+    constexpr int DV = RC::DV, BV = RC::BV;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    __shared__ uint64_t mma_bar, ld_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int failed_sh;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = nch - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int H = p.H, T = p.T, L = p.L;
+    const int c0 = c * C, n = min(C, T - c0);
+    uint8_t *rec = ws + kRecOffset + (((size_t)b * H + h) * nch + c) * RC::BYTES;
+    float *sA = (float *)(sm + LY::AF);
+    float *sTmp = (float *)(sm + LY::TMP);
+    float *sG = (float *)(sm + LY::GATES);
+    float *sBeta = sG + C;
+    float *sGam = sBeta + C;
+    float *sD = sGam + C;
+    const uint32_t sb = smem_u32(sm);
+    uint32_t mph = 0, lph = 0;  // phases of mma_bar and ld_bar
+
+    if (tid == 0) {
+        mbar_init(&mma_bar, 1);
+        mbar_init(&ld_bar, 1);
+        mbar_fence_init();
+        failed_sh = 0;
+        mbar_expect_tx(&ld_bar, 2 * (DK / 64) * C * 128);
+        for (int blk = 0; blk < DK / 64; ++blk) {
+            tma_load_4d(sm + LY::KQ + blk * LY::KQ_BLK, &maps.k, blk * 64, h, c0, b, &ld_bar);
+            tma_load_4d(sm + LY::KQ + blk * LY::KQ_BLK + C * 128, &maps.q, blk * 64, h, c0, b, &ld_bar);
+        }
+    }
+    if (warp == 0) tmem_alloc(&tmem_base_sh, LY::TCOLS);
+    if (tid < C) {
+        const size_t bth = ((size_t)b * T + c0 + tid) * H + h;
+        sG[tid] = tid < n ? logf(p.alpha[bth]) : 0.f;
+        sBeta[tid] = tid < n ? p.beta[bth] : 0.f;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const float x0 = warp_inclusive_scan(sG[lane], lane);
+        const float x1 = warp_inclusive_scan(sG[32 + lane], lane) + __shfl_sync(0xffffffffu, x0, 31);
+        sG[lane] = x0;
+        sG[32 + lane] = x1;
+    }
+    if (!mbar_wait(&ld_bar, lph++ & 1, p.status)) failed_sh = 1;
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tb = tmem_base_sh;
+    if (tid < C) {
+        sGam[tid] = expf(sG[tid]);
+        sD[tid] = tid < n ? expf(sG[C - 1] - sG[tid]) : 0.f;
+        reinterpret_cast<float *>(rec + RC::G)[tid] = sG[tid];
+    }
+    // thread 0 issued MMAs: commit, and every thread waits (bounded) for their completion
+    auto mma_done = [&](bool issued) -> bool {
+        if (tid == 0 && issued) mma_commit(&mma_bar);
+        __syncwarp();
+        if (issued && !mbar_wait(&mma_bar, mph & 1, p.status)) failed_sh = 1;
+        if (issued) mph++;
+        fence_after_sync();
+        __syncthreads();
+        return failed_sh == 0;
+    };
+    auto okq = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::KQ_BLK); };
+    auto okb = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::BLK); };
+    auto ok0 = [](int ks) { return (uint64_t)koff_k_sw128(ks, 0); };
+    auto omn = [](int ks) { return (uint64_t)koff_mn_sw128(ks); };
+    const uint64_t dKQ = make_desc(sb + LY::KQ, 16, 1024, 2);
+
+    // G = [K; Q] K^T  ->  A (fp32, shared) and Mqk (hi / lo, straight to the record)
+    bool ok = failed_sh == 0;
+    if (ok && tid == 0) mma_steps<DK / 16>(tb + LY::cG, idesc_bf16(128, C, 0, 0), dKQ, dKQ, okq, okq, false);
+    ok = mma_done(ok);
+    if (ok) {
+        const int t = (warp & 1) * 32 + lane;
+        const float gt = sG[t], bt = sBeta[t];
+#pragma unroll
+        for (int cc = 0; cc < C; cc += 32) {
+            float gr[32];
+            tmem_ld32(taddr(tb, 32 * warp, LY::cG + cc), gr);
+            tmem_wait_ld();
+            if (warp < 2) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int i = cc + j;
+                    sA[t * AS + i] = (i < t) ? bt * __expf(gt - sG[i]) * gr[j] : 0.f;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int i = cc + j;
+                    gr[j] = (i <= t) ? __expf(gt - sG[i]) * gr[j] : 0.f;
+                }
+                store32_split(rec + RC::MQK, rec + RC::MQK + C * 128, t, cc, gr);
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    // T pair tiles: T diag(beta gamma) for Wk, then T itself for X_u
+    auto store_t_pair = [&](bool scaled) {
+        for (int e = tid; e < C * (C / 8); e += NT) {
+            const int t = e / (C / 8), c8 = e % (C / 8);
+            float a[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = c8 * 8 + j;
+                const float tv = (i <= t) ? sA[t * AS + i] : 0.f;
+                a[j] = scaled ? tv * sBeta[i] * sGam[i] : tv;
+            }
+            uint4 hv, lv;
+            split8(a, hv, lv);
+            const uint32_t off = sw128_off(t, c8 * 8, 0);
+            st16(sm + LY::T1, off, hv);
+            st16(sm + LY::T1L, off, lv);
+        }
+    };
+    if (ok) {
+        solve_unit_lower<NT>(sA, sA, sTmp, tid);
+        store_t_pair(true);
+    }
+    sync_for_mma();
+    // Wk = T diag(beta gamma) K  (M = 64; row r of an M = 64 accumulator sits in lane 32 (r / 16) + r % 16)
+    const uint64_t dKmn = make_desc(sb + LY::KQ, LY::KQ_BLK, 1024, 2);
+    if (ok && tid == 0) {
+        const uint32_t id = idesc_bf16(64, DK, 0, 1);
+        mma_steps<C / 16>(tb + LY::cA, id, make_desc(sb + LY::T1, 16, 1024, 2), dKmn, ok0, omn, false);
+        mma_steps<C / 16>(tb + LY::cA, id, make_desc(sb + LY::T1L, 16, 1024, 2), dKmn, ok0, omn, true);
+    }
+    ok = mma_done(ok);
+    const bool own_t = lane < 16;
+    const int t_row = 16 * warp + lane;
+    if (ok) {
+#pragma unroll
+        for (int cc = 0; cc < DK; cc += 32) {
+            float x[32];
+            tmem_ld32(taddr(tb, 32 * warp, LY::cA + cc), x);
+            tmem_wait_ld();
+            if (own_t) store32_split(rec + RC::WK, nullptr, t_row, cc, x, RC::WK_BLK);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (ok) store_t_pair(false);  // the Wk MMA has completed: the T tiles are free
+
+    // the write terms, one rank at a time
+    const uint64_t dW = make_desc(sb + LY::W, 16, 1024, 2);
+    const uint64_t dWmn = make_desc(sb + LY::W, LY::BLK, 1024, 2);
+    const uint64_t dU = make_desc(sb + LY::U, LY::BLK, 1024, 2);
+    const uint32_t idV = idesc_bf16(64, DV, 0, 1);
+    for (int l = 0; l < L && ok; ++l) {
+        if (tid == 0) {
+            mbar_expect_tx(&ld_bar, 2 * (DK / 64) * C * 128);
+            for (int blk = 0; blk < DK / 64; ++blk) {
+                tma_load_4d(sm + LY::W + blk * LY::BLK, &maps.w, blk * 64, h * L + l, c0, b, &ld_bar);
+                tma_load_4d(sm + LY::U + blk * LY::BLK, &maps.u, blk * 64, h * L + l, c0, b, &ld_bar);
+            }
+        }
+        if (!mbar_wait(&ld_bar, lph++ & 1, p.status)) failed_sh = 1;
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        ok = failed_sh == 0;
+        // G_l = [K; Q] W_l^T
+        if (ok && tid == 0) mma_steps<DK / 16>(tb + LY::cG, idesc_bf16(128, C, 0, 0), dKQ, dW, okq, okb, false);
+        ok = mma_done(ok);
+        if (!ok) break;
+        {   // P_l (rows of K W^T, warps 0-1) and Mqw_l (rows of Q W^T, warps 2-3) as hi / lo pairs
+            const int t = (warp & 1) * 32 + lane;
+            const float gt = sG[t], bt = sBeta[t];
+            uint8_t *dh = sm + (warp < 2 ? LY::P : LY::MQW);
+            uint8_t *dl = sm + (warp < 2 ? LY::PL : LY::MQWL);
+#pragma unroll
+            for (int cc = 0; cc < C; cc += 32) {
+                float gr[32];
+                tmem_ld32(taddr(tb, 32 * warp, LY::cG + cc), gr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int i = cc + j;
+                    const bool keep = (warp < 2) ? (i < t) : (i <= t);
+                    gr[j] = keep ? (warp < 2 ? bt : 1.f) * __expf(gt - sG[i]) * gr[j] : 0.f;
+                }
+                store32_split(dh, dl, t, cc, gr);
+            }
+        }
+        for (int e = tid; e < C * (DV / 8); e += NT) {  // D U_l as a hi / lo pair
+            const int t = e / (DV / 8), c8 = e % (DV / 8);
+            const uint32_t off = sw128_off(t, c8 * 8, LY::BLK);
+            const uint4 uv = *reinterpret_cast<const uint4 *>(sm + LY::U + off);
+            const __nv_bfloat16 *hv = reinterpret_cast<const __nv_bfloat16 *>(&uv);
+            float du[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) du[j] = sD[t] * __bfloat162float(hv[j]);
+            uint4 dh, dl;
+            split8(du, dh, dl);
+            st16(sm + LY::DU, off, dh);
+            st16(sm + LY::DUL, off, dl);
+        }
+        sync_for_mma();
+        if (tid == 0) {
+            const bool acc = l > 0;
+            // sum P U (accumulated over l in the Wk columns) and O_w
+            mma_steps<C / 16>(tb + LY::cA, idV, make_desc(sb + LY::P, 16, 1024, 2), dU, ok0, omn, acc);
+            mma_steps<C / 16>(tb + LY::cA, idV, make_desc(sb + LY::PL, 16, 1024, 2), dU, ok0, omn, true);
+            mma_steps<C / 16>(tb + LY::cO, idV, make_desc(sb + LY::MQW, 16, 1024, 2), dU, ok0, omn, acc);
+            mma_steps<C / 16>(tb + LY::cO, idV, make_desc(sb + LY::MQWL, 16, 1024, 2), dU, ok0, omn, true);
+            // F_w = sum W_l^T (D U_l)  (M = DK: W_l read as an MN-major A operand)
+            const uint32_t idF = idesc_bf16(DK, DV, 1, 1);
+            mma_steps<C / 16>(tb + LY::cF, idF, dWmn, make_desc(sb + LY::DU, LY::BLK, 1024, 2), omn, omn, acc);
+            mma_steps<C / 16>(tb + LY::cF, idF, dWmn, make_desc(sb + LY::DUL, LY::BLK, 1024, 2), omn, omn, true);
+        }
+        ok = mma_done(ok);
+    }
+    // sum P U -> hi / lo pair (over the D U tiles), then X_u = T (sum P U)
+    if (ok) {
+#pragma unroll
+        for (int cc = 0; cc < DV; cc += 32) {
+            float x[32];
+            tmem_ld32(taddr(tb, 32 * warp, LY::cA + cc), x);
+            tmem_wait_ld();
+            if (own_t) {
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    uint4 hv, lv;
+                    split8(x + 8 * c8, hv, lv);
+                    const uint32_t off = sw128_off(t_row, cc + 8 * c8, LY::BLK);
+                    st16(sm + LY::DU, off, hv);
+                    st16(sm + LY::DUL, off, lv);
+                }
+            }
+        }
+    }
+    sync_for_mma();
+    if (ok && tid == 0) {
+        const uint64_t dPU = make_desc(sb + LY::DU, LY::BLK, 1024, 2);
+        const uint64_t dPUL = make_desc(sb + LY::DUL, LY::BLK, 1024, 2);
+        const uint64_t dT = make_desc(sb + LY::T1, 16, 1024, 2), dTL = make_desc(sb + LY::T1L, 16, 1024, 2);
+        mma_steps<C / 16>(tb + LY::cA, idV, dT, dPU, ok0, omn, false);
+        mma_steps<C / 16>(tb + LY::cA, idV, dT, dPUL, ok0, omn, true);
+        mma_steps<C / 16>(tb + LY::cA, idV, dTL, dPU, ok0, omn, true);
+    }
+    ok = mma_done(ok);
+    // -X_u -> the U slot (staged over K and Q in the record's slice layout, one bulk store);
+    // O_w and F_w straight to the record
+    if (ok) {
+        uint8_t *stage = sm + LY::KQ;
+#pragma unroll
+        for (int cc = 0; cc < DV; cc += 32) {
+            float x[32];
+            tmem_ld32(taddr(tb, 32 * warp, LY::cA + cc), x);
+            tmem_wait_ld();
+            if (own_t) {
+#pragma unroll
+                for (int j4 = 0; j4 < 32; j4 += 4) {
+                    const int j = cc + j4;
+                    *reinterpret_cast<float4 *>(stage + (j / BV) * RC::U_SLICE + u_off<BV>(t_row, j % BV)) =
+                        make_float4(-x[j4], -x[j4 + 1], -x[j4 + 2], -x[j4 + 3]);
+                }
+            }
+        }
+#pragma unroll
+        for (int cc = 0; cc < DV; cc += 32) {
+            float x[32];
+            tmem_ld32(taddr(tb, 32 * warp, LY::cO + cc), x);
+            tmem_wait_ld();
+            if (own_t) {
+                float *dst = reinterpret_cast<float *>(rec + RC::OW) + (size_t)t_row * DV + cc;
+#pragma unroll
+                for (int j4 = 0; j4 < 32; j4 += 4)
+                    *reinterpret_cast<float4 *>(dst + j4) = make_float4(x[j4], x[j4 + 1], x[j4 + 2], x[j4 + 3]);
+            }
+        }
+        // F_w rows d: lane = d for M = 128 (DK = 128); lanes 32q + r, r < 16, for M = 64
+        const bool own_d = (DK == 128) ? true : (lane < 16);
+        const int d_row = (DK == 128) ? tid : (16 * warp + lane);
+#pragma unroll
+        for (int cc = 0; cc < DV; cc += 32) {
+            float x[32];
+            tmem_ld32(taddr(tb, 32 * warp, LY::cF + cc), x);
+            tmem_wait_ld();
+            if (own_d) {
+#pragma unroll
+                for (int j4 = 0; j4 < 32; j4 += 4) {
+                    const int j = cc + j4;
+                    *reinterpret_cast<float4 *>(rec + RC::FW + (j / BV) * RC::FW_SLICE + u_off<BV>(d_row, j % BV)) =
+                        make_float4(x[j4], x[j4 + 1], x[j4 + 2], x[j4 + 3]);
+                }
+            }
+        }
+    }
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    if (ok && tid == 0) {
+        bulk_s2g(rec + RC::U, sm + LY::KQ, (uint32_t)(C * DV * 4));
+        bulk_commit();
+        bulk_wait_all();
+    }
+    // after a failure, let a tile load still in flight land before the CTA exits
+    if (!ok && tid == 0 && lph > 0) mbar_wait(&ld_bar, (lph - 1) & 1, nullptr, kStallTestPolls);
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tb, LY::TCOLS);
+}
+
+// ------------------------------------------------------------------------------------------------
 // state: one CTA per (value slice, head, batch), chunks in order
 //
 // Two MMA rounds per chunk (8 instructions at d = 128 for the first, 4 + 4 for the second):
@@ -301,7 +658,7 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
 // TMEM.  K, Q arrive by TMA tiled loads, the per-chunk record (Wk, Mqk, the U slice, g) by bulk
 // copies, one chunk ahead.
 
-template <int DK>
+template <int DK, bool RL = false>
 struct StateLayout {
     static constexpr int BV = kBV<DK>;
     static constexpr int N2 = 2 * BV;                     // hi | lo side by side
@@ -313,7 +670,9 @@ struct StateLayout {
     static constexpr uint32_t B_MQ = B_KWQ + KWQ_BLK * (DK / 64);   // [Mqk_lo; Mqk_hi]
     static constexpr uint32_t B_U = B_MQ + 2 * C * 128;
     static constexpr uint32_t B_G = B_U + U_BYTES;                   // g (64 floats)
-    static constexpr uint32_t BUF = B_G + 1024;
+    static constexpr uint32_t FW_BYTES = RL ? DK * BV * 4 : 0;       // F_w slice (rank L)
+    static constexpr uint32_t B_FW = B_G + 1024;
+    static constexpr uint32_t BUF = B_FW + FW_BYTES;
     // S^T [d][hi | lo], Y [t][hi | lo], D Y [t][hi | lo]: MN-major, 64-column blocks
     static constexpr uint32_t S_BLK = DK * 128;
     static constexpr uint32_t S = 2 * BUF;
@@ -366,9 +725,9 @@ __device__ __forceinline__ void store_half_pair(uint8_t *tile, uint32_t blk_byte
     }
 }
 
-template <int DK>
+template <int DK, bool RL>
 __device__ __forceinline__ const uint8_t *record(const ScanArgs &p, const uint8_t *ws, int nch, int c) {
-    return ws + kRecOffset + (((size_t)blockIdx.z * p.H + blockIdx.y) * nch + c) * GdnRec<DK>::BYTES;
+    return ws + kRecOffset + (((size_t)blockIdx.z * p.H + blockIdx.y) * nch + c) * GdnRec<DK, RL>::BYTES;
 }
 
 // One arrival per warp on `bar` once every lane's earlier writes (shared memory, for the tensor
@@ -380,12 +739,12 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
     if (lane == 0) mbar_arrive(bar);
 }
 
-template <int DK>
+template <int DK, bool RL>
 __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                                                                  const __grid_constant__ GdnMaps maps,
                                                                  const uint8_t *ws, int nch) {
-    using LY = StateLayout<DK>;
-    using RC = GdnRec<DK>;
+    using LY = StateLayout<DK, RL>;
+    using RC = GdnRec<DK, RL>;
     constexpr int BV = LY::BV, N2 = LY::N2, CH = LY::CH;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -427,11 +786,11 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
     if (warp == EPI_WARPS + 1) {
         // ---------------- loads ----------------
         if (lane == 0) {
-            constexpr uint32_t bytes = 3 * (DK / 64) * C * 128 + 2 * C * 128 + LY::U_BYTES + C * 4;
+            constexpr uint32_t bytes = 3 * (DK / 64) * C * 128 + 2 * C * 128 + LY::U_BYTES + C * 4 + LY::FW_BYTES;
             int issued = -1;
             for (int c = 0; c < nch && !failed() && !(p.flags & kStallTest); ++c) {
                 if (c >= 2 && !mbar_wait(&bars.empty[c & 1], ((c - 2) >> 1) & 1, status, lim)) { fail(); break; }
-                const uint8_t *rec = record<DK>(p, ws, nch, c);
+                const uint8_t *rec = record<DK, RL>(p, ws, nch, c);
                 uint8_t *buf = sm + (c & 1) * LY::BUF;
                 uint64_t *bar = &bars.full[c & 1];
                 const int c0 = c * C;
@@ -446,6 +805,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 bulk_g2s(buf + LY::B_MQ + C * 128, rec + RC::MQK, C * 128, bar);   // Mqk_hi
                 bulk_g2s(buf + LY::B_U, rec + RC::U + blockIdx.x * RC::U_SLICE, LY::U_BYTES, bar);
                 bulk_g2s(buf + LY::B_G, rec + RC::G, C * 4, bar);
+                if constexpr (RL)
+                    bulk_g2s(buf + LY::B_FW, rec + RC::FW + blockIdx.x * RC::FW_SLICE, LY::FW_BYTES, bar);
                 issued = c;
             }
             // let the copies still in flight land before the CTA can exit
@@ -525,6 +886,21 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             const float *g = reinterpret_cast<const float *>(buf + LY::B_G);
             const float g_last = g[C - 1];
             const uint32_t d1 = LY::cD1 + (c & 1) * N2;
+            float ow[CH];  // rank L: O_w of this thread's output row, fetched early
+#pragma unroll
+            for (int j = 0; j < CH; ++j) ow[j] = 0.f;
+            if (RL && wr && out && !lowq && lrow - 64 < n) {
+                const float *src = reinterpret_cast<const float *>(record<DK, RL>(p, ws, nch, c) + RC::OW) +
+                                   (size_t)(lrow - 64) * dv + v0 + j0;
+#pragma unroll
+                for (int j4 = 0; j4 < CH; j4 += 4) {
+                    const float4 f4 = __ldg(reinterpret_cast<const float4 *>(src + j4));
+                    ow[j4] = f4.x;
+                    ow[j4 + 1] = f4.y;
+                    ow[j4 + 2] = f4.z;
+                    ow[j4 + 3] = f4.w;
+                }
+            }
             // Y = U - X_s (lanes 0..63 of D1), and D Y
             if (lowq) {
                 const int t = lrow;
@@ -563,6 +939,16 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD4 + BV + j0), xl);
                 tmem_wait_ld();
                 if (own_d) {
+                    if (RL && wr) {  // + F_w = sum_l W_l^T D U_l
+#pragma unroll
+                        for (int j4 = 0; j4 < CH; j4 += 4) {
+                            const float4 f4 = *reinterpret_cast<const float4 *>(buf + LY::B_FW + u_off<BV>(d_row, j0 + j4));
+                            xh[j4] += f4.x;
+                            xh[j4 + 1] += f4.y;
+                            xh[j4 + 2] += f4.z;
+                            xh[j4 + 3] += f4.w;
+                        }
+                    }
 #pragma unroll
                     for (int j = 0; j < CH; ++j) Sreg[j] = fmaf(gC, Sreg[j], xh[j] + xl[j]);
                     store_half_pair<BV, CH>(sm + LY::S, LY::S_BLK, d_row, j0, Sreg);
@@ -615,7 +1001,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
                             const int jj = c8 * 8 + j;
-                            r[j] = fmaf(gt, qs[jj], up[jj] + pp[j]);
+                            r[j] = fmaf(gt, qs[jj], up[jj] + pp[j] + ow[jj]);
                         }
                         uint4 pk;
                         pk.x = pack_bf16(r[0], r[1]);
@@ -691,14 +1077,16 @@ cudaError_t launch_gdn_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-template <int DK>
+// The state kernel reads only K and Q through tensor maps (v may be absent on the rank-L route).
+template <int DK, bool RL>
 cudaError_t launch_gdn_state_t(const ScanArgs &a, const void *ws, cudaStream_t s) {
     const int nch = (a.T + C - 1) / C;
-    GdnMaps maps;
-    if (!gdn_maps<DK>(a, &maps)) return cudaErrorInvalidValue;
-    using LY = StateLayout<DK>;
+    GdnMaps maps = {};
+    if (!act_map(&maps.k, a.k, a.B, a.T, a.H, DK, 64) || !act_map(&maps.q, a.q, a.B, a.T, a.H, DK, 64))
+        return cudaErrorInvalidValue;
+    using LY = StateLayout<DK, RL>;
     static_assert(LY::BYTES <= 227 * 1024, "shared memory budget");
-    auto kern = gdn_state_kernel<DK>;
+    auto kern = gdn_state_kernel<DK, RL>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
     if (err != cudaSuccess) return err;
     dim3 grid(a.dv / LY::BV, a.H, a.B);
@@ -707,12 +1095,36 @@ cudaError_t launch_gdn_state_t(const ScanArgs &a, const void *ws, cudaStream_t s
     return cudaGetLastError();
 }
 
+template <int DK>
+cudaError_t launch_lrank_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
+    const int nch = (a.T + C - 1) / C;
+    LMaps maps;
+    if (!act_map(&maps.k, a.k, a.B, a.T, a.H, DK, 64) || !act_map(&maps.q, a.q, a.B, a.T, a.H, DK, 64) ||
+        !act_map(&maps.w, a.w, a.B, a.T, a.H * a.L, DK, 64) ||
+        !act_map(&maps.u, a.u, a.B, a.T, a.H * a.L, a.dv, 64))
+        return cudaErrorInvalidValue;
+    using LY = LPrepLayout<DK>;
+    static_assert(LY::BYTES <= 227 * 1024, "shared memory budget");
+    auto kern = lrank_prep_kernel<DK>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
+    if (err != cudaSuccess) return err;
+    dim3 grid(nch, a.H, a.B);
+    launch_probe_mark(s);
+    kern<<<grid, NT, LY::BYTES, s>>>(a, maps, (uint8_t *)ws, nch);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
-// Workspace bytes of the two-kernel GDN path: the status block plus one record per chunk.
+// Workspace bytes of the two-kernel path: the status block plus one record per chunk.
 size_t gdn_workspace_bytes(int B, int H, int T, int dk) {
     const size_t nch = (size_t)((T + C - 1) / C);
     const size_t rec = dk == 128 ? GdnRec<128>::BYTES : GdnRec<64>::BYTES;
+    return kRecOffset + (size_t)B * H * nch * rec;
+}
+size_t lrank_workspace_bytes(int B, int H, int T, int dk) {
+    const size_t nch = (size_t)((T + C - 1) / C);
+    const size_t rec = dk == 128 ? GdnRec<128, true>::BYTES : GdnRec<64, true>::BYTES;
     return kRecOffset + (size_t)B * H * nch * rec;
 }
 
@@ -725,13 +1137,30 @@ cudaError_t launch_gdn_prep(const ScanArgs &a, void *ws, cudaStream_t s) {
 }
 
 cudaError_t launch_gdn_state(const ScanArgs &a, const void *ws, cudaStream_t s) {
-    return a.dk == 128 ? launch_gdn_state_t<128>(a, ws, s) : launch_gdn_state_t<64>(a, ws, s);
+    return a.dk == 128 ? launch_gdn_state_t<128, false>(a, ws, s) : launch_gdn_state_t<64, false>(a, ws, s);
 }
 
 cudaError_t launch_scan_gdn(const ScanArgs &a, void *ws, cudaStream_t s) {
     cudaError_t err = launch_gdn_prep(a, ws, s);
     if (err != cudaSuccess) return err;
     return launch_gdn_state(a, ws, s);
+}
+
+// The rank-L write on the same two-kernel schedule: the records add O_w and F_w, and their U slot
+// holds -X_u.  Requires bf16 I/O, dk == dv in {64, 128}, 1 <= L <= 8.
+cudaError_t launch_lrank_prep(const ScanArgs &a, void *ws, cudaStream_t s) {
+    if (a.T <= 0) return cudaSuccess;
+    return a.dk == 128 ? launch_lrank_prep_t<128>(a, ws, s) : launch_lrank_prep_t<64>(a, ws, s);
+}
+
+cudaError_t launch_lrank_state(const ScanArgs &a, const void *ws, cudaStream_t s) {
+    return a.dk == 128 ? launch_gdn_state_t<128, true>(a, ws, s) : launch_gdn_state_t<64, true>(a, ws, s);
+}
+
+cudaError_t launch_scan_lrank(const ScanArgs &a, void *ws, cudaStream_t s) {
+    cudaError_t err = launch_lrank_prep(a, ws, s);
+    if (err != cudaSuccess) return err;
+    return launch_lrank_state(a, ws, s);
 }
 
 }  // namespace prism

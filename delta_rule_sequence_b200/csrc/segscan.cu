@@ -27,7 +27,8 @@ cudaError_t launch_scan_simt(const ScanArgs &a, bool io_f32, cudaStream_t s);
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
 cudaError_t launch_gdn_prep(const ScanArgs &a, void *ws, cudaStream_t s);
 cudaError_t launch_gdn_state(const ScanArgs &a, const void *ws, cudaStream_t s);
-size_t gdn_workspace_bytes(int B, int H, int T, int dk);
+cudaError_t launch_lrank_prep(const ScanArgs &a, void *ws, cudaStream_t s);
+cudaError_t launch_lrank_state(const ScanArgs &a, const void *ws, cudaStream_t s);
 
 namespace {
 
@@ -228,6 +229,7 @@ cudaError_t launch_segment_element(const ScanArgs &a, int route, bool io_f32, vo
                                    float *f_out, cudaStream_t s) {
     auto pass = [&](const ScanArgs &x) -> cudaError_t {
         switch (route) {
+            case 3: return launch_lrank_state(x, ws, s);
             case 2: return launch_gdn_state(x, ws, s);
             case 1: return launch_scan_tc(x, s);
             default: return launch_scan_simt(x, io_f32, s);
@@ -235,18 +237,19 @@ cudaError_t launch_segment_element(const ScanArgs &a, int route, bool io_f32, vo
     };
     cudaError_t err = cudaSuccess;
     if (route == 2 && a.T > 0 && (err = launch_gdn_prep(a, ws, s)) != cudaSuccess) return err;
+    if (route == 3 && a.T > 0 && (err = launch_lrank_prep(a, ws, s)) != cudaSuccess) return err;
     ScanArgs e = a;
     e.S0 = nullptr;
     e.o = nullptr;
     e.flags = kNoWrite | kS0Identity | kNoOutput;
     e.S_final = e_out;
-    if ((err = (route == 2 && a.T == 0) ? launch_scan_tc(e, s) : pass(e)) != cudaSuccess) return err;
+    if ((err = (route >= 2 && a.T == 0) ? launch_scan_tc(e, s) : pass(e)) != cudaSuccess) return err;
     ScanArgs f = a;
     f.S0 = nullptr;
     f.o = nullptr;
     f.flags = kNoOutput;
     f.S_final = f_out;
-    return (route == 2 && a.T == 0) ? launch_scan_tc(f, s) : pass(f);
+    return (route >= 2 && a.T == 0) ? launch_scan_tc(f, s) : pass(f);
 }
 
 // Kernels one segmented scan launches besides the passes: slot-0 init, the up- and down-sweep
@@ -264,7 +267,8 @@ size_t segmented_extra_bytes(int B, int H, int G, int dk, int dv) {
     return (size_t)B * G * H * (ee + fe) + (size_t)B * H * (G - 1) * (ee + fe) + (size_t)B * G * H * fe;
 }
 
-// route: 0 fp32 CUDA cores, 1 fused tensor-core kernel, 2 Gated-DeltaNet prep + state kernels.
+// route: 0 fp32 CUDA cores, 1 fused tensor-core kernel, 2 Gated-DeltaNet prep + state kernels,
+// 3 rank-L prep + state kernels.
 // ws: the caller's workspace (status word first); `rec_bytes` bytes of records follow the status
 // block on route 2, and the segment arrays follow those.
 cudaError_t launch_segmented(const ScanArgs &a, int route, bool io_f32, int G, void *ws,
@@ -287,6 +291,7 @@ cudaError_t launch_segmented(const ScanArgs &a, int route, bool io_f32, int G, v
 
     auto pass = [&](const ScanArgs &x) -> cudaError_t {
         switch (route) {
+            case 3: return launch_lrank_state(x, ws, s);
             case 2: return launch_gdn_state(x, ws, s);
             case 1: return launch_scan_tc(x, s);
             default: return launch_scan_simt(x, io_f32, s);
@@ -294,6 +299,7 @@ cudaError_t launch_segmented(const ScanArgs &a, int route, bool io_f32, int G, v
     };
     cudaError_t err = cudaSuccess;
     if (route == 2 && (err = launch_gdn_prep(v, ws, s)) != cudaSuccess) return err;
+    if (route == 3 && (err = launch_lrank_prep(v, ws, s)) != cudaSuccess) return err;
     // 1. encode: E_g (identity rows, no write) and f_g (zero state, with the write)
     ScanArgs e = v;
     e.flags = kNoWrite | kS0Identity | kNoOutput;
