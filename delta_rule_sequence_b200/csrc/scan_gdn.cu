@@ -311,10 +311,14 @@ template <int DK>
 struct LPrepLayout {
     static constexpr uint32_t KQ_BLK = 2 * C * 128;     // [K; Q] rows of one 64-column block
     static constexpr uint32_t BLK = C * 128;            // one 64-column block of a C-row tile
+    // W_l / U_l buffers: two at d = 128 (the next rank loads while this one is used); one at
+    // d = 64, where shared memory is kept small enough for two CTAs per SM
+    static constexpr int NBUF = DK == 128 ? 2 : 1;
+    static constexpr uint32_t TILE = BLK * (DK / 64);   // one C x DK bf16 tile
     static constexpr uint32_t KQ = 0;
     static constexpr uint32_t W = KQ + KQ_BLK * (DK / 64);   // W_l, K-major (rows t)
-    static constexpr uint32_t U = W + BLK * (DK / 64);       // U_l, [t][dv] (MN-major B operand)
-    static constexpr uint32_t DU = U + BLK * (DK / 64);      // D U_l hi, lo; later sum P U hi, lo
+    static constexpr uint32_t U = W + NBUF * TILE;           // U_l, [t][dv] (MN-major B operand)
+    static constexpr uint32_t DU = U + NBUF * TILE;          // D U_l hi, lo; later sum P U hi, lo
     static constexpr uint32_t DUL = DU + BLK * (DK / 64);
     static constexpr uint32_t T1 = DUL + BLK * (DK / 64);    // T diag(beta gamma), then T: hi, lo
     static constexpr uint32_t T1L = T1 + BLK;
@@ -341,13 +345,14 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
     constexpr int DV = RC::DV, BV = RC::BV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t mma_bar, ld_bar;
+    __shared__ uint64_t mma_bar, ld_bar, wu_bar[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int failed_sh;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = nch - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int H = p.H, T = p.T, L = p.L;
+    constexpr int NBUF = LY::NBUF;
     const int c0 = c * C, n = min(C, T - c0);
     uint8_t *rec = ws + kRecOffset + (((size_t)b * H + h) * nch + c) * RC::BYTES;
     float *sA = (float *)(sm + LY::AF);
@@ -358,10 +363,22 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
     float *sD = sGam + C;
     const uint32_t sb = smem_u32(sm);
     uint32_t mph = 0, lph = 0;  // phases of mma_bar and ld_bar
+    // W_l and U_l of rank l into buffer l % NBUF, completing on wu_bar[l % NBUF]
+    auto load_wu = [&](int l) {
+        const int bi = l % NBUF;
+        mbar_expect_tx(&wu_bar[bi], 2 * LY::TILE);
+        for (int blk = 0; blk < DK / 64; ++blk) {
+            tma_load_4d(sm + LY::W + bi * LY::TILE + blk * LY::BLK, &maps.w, blk * 64, h * L + l, c0, b, &wu_bar[bi]);
+            tma_load_4d(sm + LY::U + bi * LY::TILE + blk * LY::BLK, &maps.u, blk * 64, h * L + l, c0, b, &wu_bar[bi]);
+        }
+    };
+    int wu_issued = 0;  // ranks whose loads were issued (thread 0)
 
     if (tid == 0) {
         mbar_init(&mma_bar, 1);
         mbar_init(&ld_bar, 1);
+        mbar_init(&wu_bar[0], 1);
+        mbar_init(&wu_bar[1], 1);
         mbar_fence_init();
         failed_sh = 0;
         mbar_expect_tx(&ld_bar, 2 * (DK / 64) * C * 128);
@@ -369,6 +386,8 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
             tma_load_4d(sm + LY::KQ + blk * LY::KQ_BLK, &maps.k, blk * 64, h, c0, b, &ld_bar);
             tma_load_4d(sm + LY::KQ + blk * LY::KQ_BLK + C * 128, &maps.q, blk * 64, h, c0, b, &ld_bar);
         }
+        // the first ranks' W_l, U_l load while A, T and Wk are computed
+        for (; wu_issued < L && wu_issued < NBUF; ++wu_issued) load_wu(wu_issued);
     }
     if (warp == 0) tmem_alloc(&tmem_base_sh, LY::TCOLS);
     if (tid < C) {
@@ -486,19 +505,20 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
     if (ok) store_t_pair(false);  // the Wk MMA has completed: the T tiles are free
 
     // the write terms, one rank at a time
-    const uint64_t dW = make_desc(sb + LY::W, 16, 1024, 2);
-    const uint64_t dWmn = make_desc(sb + LY::W, LY::BLK, 1024, 2);
-    const uint64_t dU = make_desc(sb + LY::U, LY::BLK, 1024, 2);
     const uint32_t idV = idesc_bf16(64, DV, 0, 1);
     for (int l = 0; l < L && ok; ++l) {
-        if (tid == 0) {
-            mbar_expect_tx(&ld_bar, 2 * (DK / 64) * C * 128);
+        const int bi = l % NBUF;
+        const uint32_t wb = LY::W + bi * LY::TILE, ub = LY::U + bi * LY::TILE;
+        const uint64_t dW = make_desc(sb + wb, 16, 1024, 2);
+        const uint64_t dWmn = make_desc(sb + wb, LY::BLK, 1024, 2);
+        const uint64_t dU = make_desc(sb + ub, LY::BLK, 1024, 2);
+        if (tid == 0 && l + NBUF < L) {  // the rank after the ones in flight: start it toward L2
             for (int blk = 0; blk < DK / 64; ++blk) {
-                tma_load_4d(sm + LY::W + blk * LY::BLK, &maps.w, blk * 64, h * L + l, c0, b, &ld_bar);
-                tma_load_4d(sm + LY::U + blk * LY::BLK, &maps.u, blk * 64, h * L + l, c0, b, &ld_bar);
+                tma_prefetch_4d(&maps.w, blk * 64, h * L + l + NBUF, c0, b);
+                tma_prefetch_4d(&maps.u, blk * 64, h * L + l + NBUF, c0, b);
             }
         }
-        if (!mbar_wait(&ld_bar, lph++ & 1, p.status)) failed_sh = 1;
+        if (!mbar_wait(&wu_bar[bi], (l / NBUF) & 1, p.status)) failed_sh = 1;
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
@@ -529,7 +549,7 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
         for (int e = tid; e < C * (DV / 8); e += NT) {  // D U_l as a hi / lo pair
             const int t = e / (DV / 8), c8 = e % (DV / 8);
             const uint32_t off = sw128_off(t, c8 * 8, LY::BLK);
-            const uint4 uv = *reinterpret_cast<const uint4 *>(sm + LY::U + off);
+            const uint4 uv = *reinterpret_cast<const uint4 *>(sm + ub + off);
             const __nv_bfloat16 *hv = reinterpret_cast<const __nv_bfloat16 *>(&uv);
             float du[8];
 #pragma unroll
@@ -553,6 +573,8 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
             mma_steps<C / 16>(tb + LY::cF, idF, dWmn, make_desc(sb + LY::DUL, LY::BLK, 1024, 2), omn, omn, true);
         }
         ok = mma_done(ok);
+        // this buffer's MMAs are done: the rank NBUF ahead can load into it
+        if (ok && tid == 0 && wu_issued < L) load_wu(wu_issued++);
     }
     // sum P U -> hi / lo pair (over the D U tiles), then X_u = T (sum P U)
     if (ok) {
@@ -639,8 +661,12 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
         bulk_commit();
         bulk_wait_all();
     }
-    // after a failure, let a tile load still in flight land before the CTA exits
-    if (!ok && tid == 0 && lph > 0) mbar_wait(&ld_bar, (lph - 1) & 1, nullptr, kStallTestPolls);
+    // after a failure, let the tile loads still in flight land before the CTA exits
+    if (!ok && tid == 0) {
+        mbar_wait(&ld_bar, 0, nullptr, kStallTestPolls);
+        for (int l = wu_issued > NBUF ? wu_issued - NBUF : 0; l < wu_issued; ++l)
+            mbar_wait(&wu_bar[l % NBUF], (l / NBUF) & 1, nullptr, kStallTestPolls);
+    }
     __syncthreads();
     if (warp == 0) tmem_dealloc(tb, LY::TCOLS);
 }

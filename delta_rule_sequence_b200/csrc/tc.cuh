@@ -99,6 +99,13 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int x, 
         : "memory");
 }
 
+// Prefetch of one 4-D tiled box into L2 (no shared memory, no completion signal).
+__device__ __forceinline__ void tma_prefetch_4d(const void *tmap, int x, int y, int z, int w) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];"
+                 ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
+}
+
 // Plain (untiled) bulk copy global -> shared, completing on `bar` (tx bytes); 16-byte aligned.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile(
