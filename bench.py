@@ -57,10 +57,13 @@ def load_peaks():
 # is compiled from (the hash of those files keys the committed ncu traffic figures).
 STEP_KERNELS = {
     "gdn": ["gdn_prep_kernel", "gdn_state_kernel"],
+    "recsys": ["lrank_prep_kernel", "gdn_state_kernel"],
+    "long": ["lrank_prep_kernel", "gdn_state_kernel"],
 }
 _GDN_SOURCES = ["csrc/scan_gdn.cu", "csrc/tc.cuh", "csrc/chunk_common.cuh", "csrc/common.cuh"]
 KERNEL_SOURCES = {
     "gdn_prep_kernel": _GDN_SOURCES,
+    "lrank_prep_kernel": _GDN_SOURCES,
     "gdn_state_kernel": _GDN_SOURCES,
     "decode_kernel": ["csrc/decode.cu", "csrc/common.cuh"],
     "scan_tc_kernel": ["csrc/scan_tc.cu", "csrc/tc.cuh", "csrc/chunk_common.cuh", "csrc/common.cuh"],
@@ -310,9 +313,13 @@ def time_workload(wl, dev, stream, peaks, rank, max_over_ranks, barrier, world, 
     alg = scan_bytes(wl)
     achieved = alg / (kern_ms / 1e3) / 1e9
     del x, o, S
+    names = STEP_KERNELS.get(wl.name, [])
+    if len(names) != n_launch:
+        names = [f"launch{j}" for j in range(n_launch)]
     return {"workload": workload_config(wl)["workload"], "ms_per_call": ms,
             "tokens_per_s": world * wl.B * wl.T / (ms / 1e3), "launches": n_launch,
-            "ms_per_launch": launch_ms,
+            "ms_per_launch": dict(zip(names, launch_ms)),
+            "dram_bytes_per_launch": {n: committed_traffic(wl.name, n) for n in names},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                          "algorithmic_bytes": alg, "algorithmic_flops": scan_flops(wl),
