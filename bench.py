@@ -66,7 +66,6 @@ KERNEL_SOURCES = {
     "lrank_prep_kernel": _GDN_SOURCES,
     "gdn_state_kernel": _GDN_SOURCES,
     "decode_kernel": ["csrc/decode.cu", "csrc/common.cuh"],
-    "scan_tc_kernel": ["csrc/scan_tc.cu", "csrc/tc.cuh", "csrc/chunk_common.cuh", "csrc/common.cuh"],
 }
 
 

@@ -10,8 +10,7 @@ namespace prism {
 cudaError_t launch_scan_simt(const ScanArgs &a, bool io_f32, cudaStream_t s);
 cudaError_t launch_decode(const ScanArgs &a, bool io_f32, cudaStream_t s);
 cudaError_t decode_status(uint32_t *out);
-bool scan_tc_supported(const ScanArgs &a, bool io_f32);
-cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
+cudaError_t launch_state_init(const ScanArgs &a, cudaStream_t s);
 size_t gdn_workspace_bytes(int B, int H, int T, int dk);
 cudaError_t launch_scan_gdn(const ScanArgs &a, void *ws, cudaStream_t s);
 size_t lrank_workspace_bytes(int B, int H, int T, int dk);
@@ -81,27 +80,25 @@ prism_status check_common(const prism_shape *s, const void *q, const void *k, co
     return PRISM_OK;
 }
 
-// Which kernels a prism_scan_fwd call with this shape runs: the fp32 CUDA-core kernel; the
-// two-kernel tensor-core schedule (per-chunk prep, then the in-order state kernel) for the
-// Gated-DeltaNet or the rank-L write; the fused tensor-core kernel only copies S0 when T = 0.
-enum class Plan { Simt, TcFused, TcGdnSplit, TcRankLSplit };
+// Which kernels a prism_scan_fwd call with this shape runs: nothing but the exit state when there
+// are no tokens; the two-kernel tensor-core schedule (per-chunk prep, then the in-order state
+// kernel) for the Gated-DeltaNet or the rank-L write; the fp32 CUDA-core kernel otherwise.
+enum class Plan { Empty, Simt, TcGdnSplit, TcRankLSplit };
 
 Plan plan_for(const prism_shape *s, bool gdn_write) {
+    if (s->T <= 0) return Plan::Empty;
     const bool tc = s->io == PRISM_BF16 && s->dk == s->dv && (s->dk == 64 || s->dk == 128);
     if (!tc) return Plan::Simt;
-    if (s->T <= 0) return Plan::TcFused;
     return gdn_write ? Plan::TcGdnSplit : Plan::TcRankLSplit;
 }
 
 bool split_plan(Plan p) { return p == Plan::TcGdnSplit || p == Plan::TcRankLSplit; }
 
-// Route number of the segmented scan and the segment element: 0 fp32, 1 fused, 2 GDN split,
-// 3 rank-L split.
+// Route number of the segmented scan and the segment element: 0 fp32, 2 GDN split, 3 rank-L split.
 int route_of(Plan p) {
     switch (p) {
         case Plan::TcGdnSplit: return 2;
         case Plan::TcRankLSplit: return 3;
-        case Plan::TcFused: return 1;
         default: return 0;
     }
 }
@@ -239,7 +236,7 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
         switch (plan) {
             case Plan::TcGdnSplit: err = prism::launch_scan_gdn(a, workspace, s); break;
             case Plan::TcRankLSplit: err = prism::launch_scan_lrank(a, workspace, s); break;
-            case Plan::TcFused: err = prism::launch_scan_tc(a, s); break;  // T = 0: copies S0 to S_final
+            case Plan::Empty: err = prism::launch_state_init(a, s); break;  // S_final = S0
             default: err = prism::launch_scan_simt(a, io_f32, s); break;
         }
     }

@@ -1,24 +1,34 @@
-// scan_gdn.cu -- the Gated-DeltaNet write (u = beta v, w = k) as two tensor-core kernels.
+// scan_gdn.cu -- the chunked scan forward on the tcgen05 tensor cores as two kernels: a per-chunk
+// prep that runs for every (batch, head, chunk) at once, and an in-order state kernel.
 //
-// The chunk form (see scan_tc.cu) splits each chunk's work into a state-independent part and a
-// state-dependent part.  The first depends only on the chunk's own tokens, so it runs for every
-// (batch, head, chunk) at once in `gdn_prep_kernel`, once per head (not once per value slice):
-//   G = [K; Q] K^T,   A = strict(diag(beta) Gamma o K K^T),   Mqk = incl(Gamma o Q K^T),
-//   T = (I + A)^{-1},  Wk = T diag(beta e^g) K,  U = T diag(beta) V.
-// It writes Wk (bf16), Mqk (a bf16 hi/lo pair), U (fp32) and g to a per-chunk record in the
-// workspace, laid out as the shared-memory images the state kernel reads.
+// The chunk form ("Sequential Parallel Duality in Prefix Scannable Models", method overview:
+// chunk, encode, scan; exact because the per-token affine elements E_t = alpha_t (I - beta_t k_t
+// k_t^T), f_t = sum_l u w^T compose associatively).  Per chunk of C = 64 tokens with entry state S,
+// g_t = sum_{r<=t} log alpha_r, Gamma_{t,i} = e^{g_t - g_i}, D_i = e^{g_n - g_i}:
+//   A = strict(diag(beta) Gamma o K K^T),  Mqk = incl(Gamma o Q K^T),  T = (I + A)^{-1},
+//   Wk = T diag(beta e^g) K;
+//   Gated-DeltaNet write (u = beta v, w = k):  U = T diag(beta) V;
+//   rank-L write:  P_l = strict(diag(beta) Gamma o K W_l^T),  Mqw_l = incl(Gamma o Q W_l^T),
+//     U = -X_u = -T sum_l P_l U_l,  O_w = sum_l Mqw_l U_l,  F_w = sum_l W_l^T D U_l;
+//   Y = U - Wk S^T,   O = diag(e^g) Q S^T + Mqk Y (+ O_w),   S'^T = e^{g_n} S^T + K^T D Y (+ F_w),
+// which is the token recurrence S_t = alpha_t S_{t-1}(I - beta_t k_t k_t^T) + sum_l u_{t,l}
+// w_{t,l}^T, o_t = S_t q_t (PRISM, gist.science explainer, technical summary 2.1 and 2.2;
+// banbantang.com PRISM article, section 1(4): the GDN forget and rank-1 write) unrolled over the
+// chunk.  Everything but the last line depends only on the chunk's own tokens: the prep kernels
+// (`gdn_prep_kernel`, `lrank_prep_kernel`) compute it for all chunks in parallel and write a
+// per-chunk record to the workspace, laid out as the shared-memory images the state kernel reads;
 // `gdn_state_kernel` then walks the chunks of one (batch, head, value slice) in order with the
-// fp32 state on chip; per chunk it prefetches the next chunk's tiles (TMA, double buffered)
-// and runs two dependent MMA rounds, the second shared by the state update and the output:
-//   X_s = Wk S^T,  QS = Q S^T;   Y = U - X_s;   S'^T = e^{g_n} S^T + K^T D Y,   O = diag(e^g) QS + Mqk Y.
-// ("Sequential Parallel Duality in Prefix Scannable Models", method overview: encode all chunks
-// in parallel, then combine them in order; banbantang.com PRISM article, section 1(4): the GDN
-// forget and rank-1 write.)  Prep runs over chunks last-first, so the records the state kernel
-// needs first are the ones most recently written and most likely still in L2.
+// fp32 state on chip, prefetching the next chunk's tiles (TMA, double buffered).  Prep runs over
+// chunks last-first, so the records the state kernel needs first are the ones most recently
+// written and most likely still in L2.
 //
-// A tcgen05.mma issued by one thread costs about 53 cycles whatever its N up to 128 (measured on
-// B200), so both kernels are shaped to issue few, wide MMAs: hi and lo halves of an operand sit
-// side by side along N, and two 64-row operands are stacked into one M = 128 instruction.
+// Operands that are rounded intermediate results (Mqk, T, Y, S and on the rank-L route P, Mqw,
+// D U, sum P U) are kept as an unevaluated bf16 pair x = hi + lo (lo = bf16(x - hi)); a product is
+// then a_hi b_hi + a_hi b_lo + a_lo b_hi, about 16 significant bits.  The inputs q, k, v, u, w are
+// exact bf16.  A tcgen05.mma issued by one thread costs about 53 cycles whatever its N up to 128
+// (measured on B200), so the kernels issue few, wide MMAs: hi and lo halves of an operand sit side
+// by side along N, and two 64-row operands are stacked into one M = 128 instruction.  Every wait is
+// a bounded mbarrier poll that records PRISM_ERR_TIMEOUT when it runs out.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>

@@ -24,7 +24,6 @@
 namespace prism {
 
 cudaError_t launch_scan_simt(const ScanArgs &a, bool io_f32, cudaStream_t s);
-cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
 cudaError_t launch_gdn_prep(const ScanArgs &a, void *ws, cudaStream_t s);
 cudaError_t launch_gdn_state(const ScanArgs &a, const void *ws, cudaStream_t s);
 cudaError_t launch_lrank_prep(const ScanArgs &a, void *ws, cudaStream_t s);
@@ -183,6 +182,14 @@ cudaError_t combine(const SegTree &t, const float *S0, float *S_final, cudaStrea
     return cudaGetLastError();
 }
 
+// S_final of a pass over no tokens: the entry state (S0, zero, or the identity under kS0Identity).
+__global__ void __launch_bounds__(NTH) state_init_kernel(ScanArgs a, size_t n) {
+    const size_t i = (size_t)blockIdx.x * NTH + threadIdx.x;
+    if (i >= n) return;
+    const int c = (int)(i % a.dk), r = (int)((i / a.dk) % a.dv);
+    a.S_final[i] = (a.flags & kS0Identity) ? (r == c ? 1.f : 0.f) : (a.S0 ? a.S0[i] : 0.f);
+}
+
 // S_out = S_in E + f for every (b, h): S_in, f, S_out [BH, dv, D], E [BH, D, D].  S_out may be
 // S_in (each CTA stages its own rows before writing them).  grid: x = b * H + h, y = row blocks.
 template <int D>
@@ -206,6 +213,15 @@ cudaError_t fold_t(int BH, int dv, const float *S_in, const float *E, const floa
 }
 
 }  // namespace
+
+// A scan pass over T = 0 tokens: S_final receives the entry state (nothing if S_final is NULL).
+cudaError_t launch_state_init(const ScanArgs &a, cudaStream_t s) {
+    const size_t n = (size_t)a.B * a.H * a.dv * a.dk;
+    if (!a.S_final || n == 0) return cudaSuccess;
+    launch_probe_mark(s);
+    state_init_kernel<<<(unsigned)((n + NTH - 1) / NTH), NTH, 0, s>>>(a, n);
+    return cudaGetLastError();
+}
 
 // S_out = S_in E + f per (b, h) (S_in NULL: S_out = f).  dk in {32, 64, 128}.
 cudaError_t launch_state_fold(int BH, int dk, int dv, const float *S_in, const float *E, const float *f,
@@ -231,7 +247,6 @@ cudaError_t launch_segment_element(const ScanArgs &a, int route, bool io_f32, vo
         switch (route) {
             case 3: return launch_lrank_state(x, ws, s);
             case 2: return launch_gdn_state(x, ws, s);
-            case 1: return launch_scan_tc(x, s);
             default: return launch_scan_simt(x, io_f32, s);
         }
     };
@@ -243,13 +258,13 @@ cudaError_t launch_segment_element(const ScanArgs &a, int route, bool io_f32, vo
     e.o = nullptr;
     e.flags = kNoWrite | kS0Identity | kNoOutput;
     e.S_final = e_out;
-    if ((err = (route >= 2 && a.T == 0) ? launch_scan_tc(e, s) : pass(e)) != cudaSuccess) return err;
+    if ((err = a.T == 0 ? launch_state_init(e, s) : pass(e)) != cudaSuccess) return err;
     ScanArgs f = a;
     f.S0 = nullptr;
     f.o = nullptr;
     f.flags = kNoOutput;
     f.S_final = f_out;
-    return (route >= 2 && a.T == 0) ? launch_scan_tc(f, s) : pass(f);
+    return a.T == 0 ? launch_state_init(f, s) : pass(f);
 }
 
 // Kernels one segmented scan launches besides the passes: slot-0 init, the up- and down-sweep
@@ -267,8 +282,7 @@ size_t segmented_extra_bytes(int B, int H, int G, int dk, int dv) {
     return (size_t)B * G * H * (ee + fe) + (size_t)B * H * (G - 1) * (ee + fe) + (size_t)B * G * H * fe;
 }
 
-// route: 0 fp32 CUDA cores, 1 fused tensor-core kernel, 2 Gated-DeltaNet prep + state kernels,
-// 3 rank-L prep + state kernels.
+// route: 0 fp32 CUDA cores, 2 Gated-DeltaNet prep + state kernels, 3 rank-L prep + state kernels.
 // ws: the caller's workspace (status word first); `rec_bytes` bytes of records follow the status
 // block on route 2, and the segment arrays follow those.
 cudaError_t launch_segmented(const ScanArgs &a, int route, bool io_f32, int G, void *ws,
@@ -293,7 +307,6 @@ cudaError_t launch_segmented(const ScanArgs &a, int route, bool io_f32, int G, v
         switch (route) {
             case 3: return launch_lrank_state(x, ws, s);
             case 2: return launch_gdn_state(x, ws, s);
-            case 1: return launch_scan_tc(x, s);
             default: return launch_scan_simt(x, io_f32, s);
         }
     };
