@@ -56,6 +56,28 @@ __device__ __forceinline__ void vload_shared(const float *p, float (&x)[N]) {
     for (int i = 0; i < N; ++i) x[i] = f[i];
 }
 
+// Reduce-scatter of 8 per-lane partial sums (rows j = 0..7 of a block) over the warp: afterwards
+// every lane holds the full sum of row lane / 4.  Three exchange steps halve the rows a lane keeps
+// (offsets 16, 8, 4: 4 + 2 + 1 shuffles), two more finish the sum over the lanes sharing a row.
+__device__ __forceinline__ float rows8_reduce_scatter(const float (&x)[ROWS_IN_FLIGHT], int lane) {
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    float y[4], z[2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float send = b4 ? x[j] : x[j + 4], keep = b4 ? x[j + 4] : x[j];
+        y[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const float send = b3 ? y[j] : y[j + 2], keep = b3 ? y[j + 2] : y[j];
+        z[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float r = (b2 ? z[1] : z[0]) + __shfl_xor_sync(0xffffffffu, b2 ? z[0] : z[1], 4);
+    r += __shfl_xor_sync(0xffffffffu, r, 2);
+    r += __shfl_xor_sync(0xffffffffu, r, 1);
+    return r;
+}
+
 // LW = number of write terms (L, or 1 for the Gated-DeltaNet write beta v k^T).
 template <typename IO, int DK, int LW>
 __global__ void __launch_bounds__(NT, 3) decode_kernel(ScanArgs p) {
@@ -67,7 +89,7 @@ __global__ void __launch_bounds__(NT, 3) decode_kernel(ScanArgs p) {
     const IO *q = (const IO *)p.q, *k = (const IO *)p.k, *v = (const IO *)p.v;
     const IO *u = (const IO *)p.u, *w = (const IO *)p.w;
 
-    __shared__ float s_u[LW][128];                 // u_{l,r} (or beta v_r)
+    __shared__ __align__(16) float s_u[LW][128];  // u_{l,r} (or beta v_r)
     __shared__ __align__(16) float s_w[LW][DK];   // w_l (or k)
     __shared__ float s_wq[LW];
 
@@ -121,6 +143,7 @@ __global__ void __launch_bounds__(NT, 3) decode_kernel(ScanArgs p) {
 
     IO *o = (IO *)p.o + (size_t)head * dv;
     const float ab = a * be;
+    const int my_row = lane >> 2;  // the row of the block whose sums this lane ends up holding
 
     for (; r0 < dv; r0 += NW * ROWS_IN_FLIGHT) {
         if (r0 != warp * ROWS_IN_FLIGHT) {
@@ -128,36 +151,51 @@ __global__ void __launch_bounds__(NT, 3) decode_kernel(ScanArgs p) {
             for (int j = 0; j < ROWS_IN_FLIGHT; ++j)
                 vload<PER>(S + (size_t)(r0 + j) * DK + lane * PER, s[j]);
         }
+        // e_r = s_r . k and p_r = s_r . q for the 8 rows: per-lane partials, then one butterfly
+        float ep[ROWS_IN_FLIGHT], pp[ROWS_IN_FLIGHT];
 #pragma unroll
         for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
-            const int r = r0 + j;
             float e = 0.f, pq = 0.f;
 #pragma unroll
             for (int i = 0; i < PER; ++i) {
                 e = fmaf(s[j][i], kq[i], e);
                 pq = fmaf(s[j][i], qv[i], pq);
             }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                e += __shfl_xor_sync(0xffffffffu, e, off);
-                pq += __shfl_xor_sync(0xffffffffu, pq, off);
-            }
-            float outv = a * pq - ab * e * kdotq;
-            float ns[PER];
-#pragma unroll
-            for (int i = 0; i < PER; ++i) ns[i] = fmaf(a, s[j][i], -ab * e * kq[i]);
-#pragma unroll 1
-            for (int l = 0; l < LW; ++l) {
-                const float ur = s_u[l][r];
-                outv = fmaf(ur, s_wq[l], outv);
-                float wv[PER];
-                vload_shared<PER>(&s_w[l][lane * PER], wv);
-#pragma unroll
-                for (int i = 0; i < PER; ++i) ns[i] = fmaf(ur, wv[i], ns[i]);
-            }
-            vstore<PER>(S + (size_t)r * DK + lane * PER, ns);
-            if (lane == 0) st_io(o, r, outv);
+            ep[j] = e;
+            pp[j] = pq;
         }
+        const float e_mine = rows8_reduce_scatter(ep, lane);
+        const float p_mine = rows8_reduce_scatter(pp, lane);
+        // o_r = alpha p_r - alpha beta e_r (k.q) + sum_l u_{l,r} (w_l.q), by lane 4 r
+        if ((lane & 3) == 0) {
+            const int r = r0 + my_row;
+            float outv = a * p_mine - ab * e_mine * kdotq;
+#pragma unroll
+            for (int l = 0; l < LW; ++l) outv = fmaf(s_u[l][r], s_wq[l], outv);
+            st_io(o, r, outv);
+        }
+        // s_r <- alpha s_r - alpha beta e_r k + sum_l u_{l,r} w_l
+#pragma unroll
+        for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
+            const float ej = __shfl_sync(0xffffffffu, e_mine, 4 * j);
+#pragma unroll
+            for (int i = 0; i < PER; ++i) s[j][i] = fmaf(a, s[j][i], -ab * ej * kq[i]);
+        }
+#pragma unroll
+        for (int l = 0; l < LW; ++l) {
+            float wv[PER];
+            vload_shared<PER>(&s_w[l][lane * PER], wv);
+            const float4 u0 = *reinterpret_cast<const float4 *>(&s_u[l][r0]);
+            const float4 u1 = *reinterpret_cast<const float4 *>(&s_u[l][r0 + 4]);
+            const float uu[ROWS_IN_FLIGHT] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+            for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
+#pragma unroll
+                for (int i = 0; i < PER; ++i) s[j][i] = fmaf(uu[j], wv[i], s[j][i]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < ROWS_IN_FLIGHT; ++j) vstore<PER>(S + (size_t)(r0 + j) * DK + lane * PER, s[j]);
     }
 }
 

@@ -941,33 +941,47 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             if (lowq) {
                 const int t = lrow;
                 const float dd = t < n ? __expf(g_last - g[t]) : 0.f;
+                float y[CH];  // U first: it does not depend on D1
+#pragma unroll
+                for (int j4 = 0; j4 < CH; j4 += 4) {
+                    const float4 u = wr ? *reinterpret_cast<const float4 *>(buf + LY::B_U + u_off<BV>(t, j0 + j4))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    y[j4] = u.x;
+                    y[j4 + 1] = u.y;
+                    y[j4 + 2] = u.z;
+                    y[j4 + 3] = u.w;
+                }
                 if (!mbar_wait(&bars.d1_full, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
-                float xh[CH], xl[CH], y[CH];
+                float xh[CH], xl[CH];
                 tmem_ld_n<CH>(taddr(tb, 32 * q, d1 + j0), xh);
                 tmem_ld_n<CH>(taddr(tb, 32 * q, d1 + BV + j0), xl);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < CH; ++j) y[j] = -(xh[j] + xl[j]);
-                if (wr) {
-#pragma unroll
-                    for (int j4 = 0; j4 < CH; j4 += 4) {
-                        const float4 u = *reinterpret_cast<const float4 *>(buf + LY::B_U + u_off<BV>(t, j0 + j4));
-                        y[j4] += u.x;
-                        y[j4 + 1] += u.y;
-                        y[j4 + 2] += u.z;
-                        y[j4 + 3] += u.w;
-                    }
-                }
+                for (int j = 0; j < CH; ++j) y[j] -= xh[j] + xl[j];
                 store_half_pair<BV, CH>(sm + LY::Y, LY::Y_BLK, t, j0, y);
 #pragma unroll
                 for (int j = 0; j < CH; ++j) y[j] *= dd;
                 store_half_pair<BV, CH>(sm + LY::DY, LY::Y_BLK, t, j0, y);
             }
             warp_arrive(&bars.y_ready, lane);
-            // state update S^T <- e^{g_n} S^T + K^T D Y
+            // state update S^T <- e^{g_n} S^T + K^T D Y (+ F_w)
             {
                 const float gC = __expf(g_last);
+                if (own_d) {  // e^{g_n} S^T (+ F_w) first: it does not depend on D4
+#pragma unroll
+                    for (int j = 0; j < CH; ++j) Sreg[j] *= gC;
+                    if (RL && wr) {
+#pragma unroll
+                        for (int j4 = 0; j4 < CH; j4 += 4) {
+                            const float4 f4 = *reinterpret_cast<const float4 *>(buf + LY::B_FW + u_off<BV>(d_row, j0 + j4));
+                            Sreg[j4] += f4.x;
+                            Sreg[j4 + 1] += f4.y;
+                            Sreg[j4 + 2] += f4.z;
+                            Sreg[j4 + 3] += f4.w;
+                        }
+                    }
+                }
                 if (!mbar_wait(&bars.d4_full, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 float xh[CH], xl[CH];
@@ -975,18 +989,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD4 + BV + j0), xl);
                 tmem_wait_ld();
                 if (own_d) {
-                    if (RL && wr) {  // + F_w = sum_l W_l^T D U_l
 #pragma unroll
-                        for (int j4 = 0; j4 < CH; j4 += 4) {
-                            const float4 f4 = *reinterpret_cast<const float4 *>(buf + LY::B_FW + u_off<BV>(d_row, j0 + j4));
-                            xh[j4] += f4.x;
-                            xh[j4 + 1] += f4.y;
-                            xh[j4 + 2] += f4.z;
-                            xh[j4 + 3] += f4.w;
-                        }
-                    }
-#pragma unroll
-                    for (int j = 0; j < CH; ++j) Sreg[j] = fmaf(gC, Sreg[j], xh[j] + xl[j]);
+                    for (int j = 0; j < CH; ++j) Sreg[j] += xh[j] + xl[j];
                     store_half_pair<BV, CH>(sm + LY::S, LY::S_BLK, d_row, j0, Sreg);
                 }
             }
