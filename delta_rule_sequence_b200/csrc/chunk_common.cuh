@@ -109,9 +109,14 @@ __device__ __forceinline__ void mma_split(uint32_t d, uint32_t idesc, int nks, F
 // T = (I + A)^{-1} for strictly lower-triangular A (C = 64), blocked: the four 16 x 16 diagonal
 // blocks by forward substitution, then two doubling levels T_21 = -T_22 A_21 T_11 (16 -> 32 -> 64)
 // as register-blocked products with fixed trip counts.  Safe in place (A == Tm): every block is
-// read as A before it is overwritten with T.  Needs NTH == 128 threads; tmp holds 32 x 33 floats.
-template <int NTH>
-__device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid) {
+// read as A before it is overwritten with T.  Run by 128 threads (tid < 128); SYNC(), a barrier
+// among exactly those threads, separates its phases.  tmp holds 32 x 33 floats.
+struct CtaSync {
+    __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+
+template <int NTH, class SYNC = CtaSync>
+__device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid, SYNC sync = SYNC()) {
     static_assert(NTH == 128, "the solve is laid out for 128 threads");
     const int warp = tid >> 5, lane = tid & 31;
     // diagonal blocks: warp w inverts block w, lane j < 16 computes column j
@@ -129,7 +134,7 @@ __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid)
 #pragma unroll
         for (int i = 0; i < 16; ++i) Tm[(o + i) * AS + o + j] = x[i];
     }
-    __syncthreads();
+    sync();
     // level 1, 16-blocks, pairs p = 0, 1: rows r0 = 32p + 16, cols c0 = 32p; thread: 1 row x 4 cols
     {
         const int pp = tid >> 6, r = (tid >> 2) & 15, cq = (tid & 3) * 4;
@@ -143,7 +148,7 @@ __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid)
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) tmp[pp * 16 * 17 + r * 17 + cq + j] = m[j];
-        __syncthreads();
+        sync();
 #pragma unroll
         for (int j = 0; j < 4; ++j) m[j] = 0.f;
 #pragma unroll
@@ -155,7 +160,7 @@ __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid)
 #pragma unroll
         for (int j = 0; j < 4; ++j) Tm[(r0 + r) * AS + c0 + cq + j] = -m[j];
     }
-    __syncthreads();
+    sync();
     // level 2, 32-blocks: rows 32.., cols 0..31; thread: 1 row x 8 cols
     {
         const int r = tid >> 2, cq = (tid & 3) * 8;
@@ -170,7 +175,7 @@ __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid)
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) tmp[r * 33 + cq + j] = m[j];
-        __syncthreads();
+        sync();
 #pragma unroll
         for (int j = 0; j < 8; ++j) m[j] = 0.f;
 #pragma unroll 8
@@ -182,7 +187,7 @@ __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid)
 #pragma unroll
         for (int j = 0; j < 8; ++j) Tm[(32 + r) * AS + cq + j] = -m[j];
     }
-    __syncthreads();
+    sync();
 }
 
 }  // namespace

@@ -347,10 +347,18 @@ struct LPrepLayout {
     static constexpr uint32_t TCOLS = cF + DK <= 256 ? 256 : 512;
 };
 
+// 8 warps at d = 128 (one CTA per SM: its TMEM accumulators take 448 columns), 4 at d = 64 (two
+// CTAs per SM).  Warp w reads TMEM lane quarter w % 4; with 8 warps, warps w and w + 4 split the
+// columns of every epilogue.
 template <int DK>
-__global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid_constant__ LMaps maps,
-                                                       uint8_t *ws, int nch) {
+constexpr int kLPrepThreads = DK == 128 ? 256 : 128;
+
+template <int DK>
+__global__ void __launch_bounds__(kLPrepThreads<DK>) lrank_prep_kernel(ScanArgs p, const __grid_constant__ LMaps maps,
+                                                                      uint8_t *ws, int nch) {
     using LY = LPrepLayout<DK>;
+    constexpr int NTH = kLPrepThreads<DK>;
+    constexpr int NH = NTH / 128;  // column splits of an epilogue
     using RC = GdnRec<DK, true>;
     constexpr int DV = RC::DV, BV = RC::BV;
     extern __shared__ uint8_t smem_raw[];
@@ -360,6 +368,7 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
     __shared__ int failed_sh;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, hs = warp >> 2;  // TMEM lane quarter, column split
     const int c = nch - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int H = p.H, T = p.T, L = p.L;
     constexpr int NBUF = LY::NBUF;
@@ -443,14 +452,14 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
     if (ok && tid == 0) mma_steps<DK / 16>(tb + LY::cG, idesc_bf16(128, C, 0, 0), dKQ, dKQ, okq, okq, false);
     ok = mma_done(ok);
     if (ok) {
-        const int t = (warp & 1) * 32 + lane;
+        const int t = (q & 1) * 32 + lane;
         const float gt = sG[t], bt = sBeta[t];
 #pragma unroll
-        for (int cc = 0; cc < C; cc += 32) {
+        for (int cc = hs * (C / NH); cc < (hs + 1) * (C / NH); cc += 32) {
             float gr[32];
-            tmem_ld32(taddr(tb, 32 * warp, LY::cG + cc), gr);
+            tmem_ld32(taddr(tb, 32 * q, LY::cG + cc), gr);
             tmem_wait_ld();
-            if (warp < 2) {
+            if (q < 2) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int i = cc + j;
@@ -470,7 +479,7 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
     __syncthreads();
     // T pair tiles: T diag(beta gamma) for Wk, then T itself for X_u
     auto store_t_pair = [&](bool scaled) {
-        for (int e = tid; e < C * (C / 8); e += NT) {
+        for (int e = tid; e < C * (C / 8); e += NTH) {
             const int t = e / (C / 8), c8 = e % (C / 8);
             float a[8];
 #pragma unroll
@@ -487,7 +496,11 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
         }
     };
     if (ok) {
-        solve_unit_lower<NT>(sA, sA, sTmp, tid);
+        if (tid < 128) {
+            if constexpr (NTH == 128) solve_unit_lower<128>(sA, sA, sTmp, tid);
+            else solve_unit_lower<128>(sA, sA, sTmp, tid, [] { named_sync(2, 128); });
+        }
+        __syncthreads();
         store_t_pair(true);
     }
     sync_for_mma();
@@ -500,12 +513,12 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
     }
     ok = mma_done(ok);
     const bool own_t = lane < 16;
-    const int t_row = 16 * warp + lane;
+    const int t_row = 16 * q + lane;
     if (ok) {
 #pragma unroll
-        for (int cc = 0; cc < DK; cc += 32) {
+        for (int cc = hs * (DK / NH); cc < (hs + 1) * (DK / NH); cc += 32) {
             float x[32];
-            tmem_ld32(taddr(tb, 32 * warp, LY::cA + cc), x);
+            tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
             tmem_wait_ld();
             if (own_t) store32_split(rec + RC::WK, nullptr, t_row, cc, x, RC::WK_BLK);
         }
@@ -537,26 +550,26 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
         if (ok && tid == 0) mma_steps<DK / 16>(tb + LY::cG, idesc_bf16(128, C, 0, 0), dKQ, dW, okq, okb, false);
         ok = mma_done(ok);
         if (!ok) break;
-        {   // P_l (rows of K W^T, warps 0-1) and Mqw_l (rows of Q W^T, warps 2-3) as hi / lo pairs
-            const int t = (warp & 1) * 32 + lane;
+        {   // P_l (rows of K W^T, quarters 0-1) and Mqw_l (rows of Q W^T, quarters 2-3) as pairs
+            const int t = (q & 1) * 32 + lane;
             const float gt = sG[t], bt = sBeta[t];
-            uint8_t *dh = sm + (warp < 2 ? LY::P : LY::MQW);
-            uint8_t *dl = sm + (warp < 2 ? LY::PL : LY::MQWL);
+            uint8_t *dh = sm + (q < 2 ? LY::P : LY::MQW);
+            uint8_t *dl = sm + (q < 2 ? LY::PL : LY::MQWL);
 #pragma unroll
-            for (int cc = 0; cc < C; cc += 32) {
+            for (int cc = hs * (C / NH); cc < (hs + 1) * (C / NH); cc += 32) {
                 float gr[32];
-                tmem_ld32(taddr(tb, 32 * warp, LY::cG + cc), gr);
+                tmem_ld32(taddr(tb, 32 * q, LY::cG + cc), gr);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int i = cc + j;
-                    const bool keep = (warp < 2) ? (i < t) : (i <= t);
-                    gr[j] = keep ? (warp < 2 ? bt : 1.f) * __expf(gt - sG[i]) * gr[j] : 0.f;
+                    const bool keep = (q < 2) ? (i < t) : (i <= t);
+                    gr[j] = keep ? (q < 2 ? bt : 1.f) * __expf(gt - sG[i]) * gr[j] : 0.f;
                 }
                 store32_split(dh, dl, t, cc, gr);
             }
         }
-        for (int e = tid; e < C * (DV / 8); e += NT) {  // D U_l as a hi / lo pair
+        for (int e = tid; e < C * (DV / 8); e += NTH) {  // D U_l as a hi / lo pair
             const int t = e / (DV / 8), c8 = e % (DV / 8);
             const uint32_t off = sw128_off(t, c8 * 8, LY::BLK);
             const uint4 uv = *reinterpret_cast<const uint4 *>(sm + ub + off);
@@ -589,9 +602,9 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
     // sum P U -> hi / lo pair (over the D U tiles), then X_u = T (sum P U)
     if (ok) {
 #pragma unroll
-        for (int cc = 0; cc < DV; cc += 32) {
+        for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
             float x[32];
-            tmem_ld32(taddr(tb, 32 * warp, LY::cA + cc), x);
+            tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
             tmem_wait_ld();
             if (own_t) {
 #pragma unroll
@@ -620,9 +633,9 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
     if (ok) {
         uint8_t *stage = sm + LY::KQ;
 #pragma unroll
-        for (int cc = 0; cc < DV; cc += 32) {
+        for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
             float x[32];
-            tmem_ld32(taddr(tb, 32 * warp, LY::cA + cc), x);
+            tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
             tmem_wait_ld();
             if (own_t) {
 #pragma unroll
@@ -634,9 +647,9 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
             }
         }
 #pragma unroll
-        for (int cc = 0; cc < DV; cc += 32) {
+        for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
             float x[32];
-            tmem_ld32(taddr(tb, 32 * warp, LY::cO + cc), x);
+            tmem_ld32(taddr(tb, 32 * q, LY::cO + cc), x);
             tmem_wait_ld();
             if (own_t) {
                 float *dst = reinterpret_cast<float *>(rec + RC::OW) + (size_t)t_row * DV + cc;
@@ -647,11 +660,11 @@ __global__ void __launch_bounds__(NT) lrank_prep_kernel(ScanArgs p, const __grid
         }
         // F_w rows d: lane = d for M = 128 (DK = 128); lanes 32q + r, r < 16, for M = 64
         const bool own_d = (DK == 128) ? true : (lane < 16);
-        const int d_row = (DK == 128) ? tid : (16 * warp + lane);
+        const int d_row = (DK == 128) ? 32 * q + lane : (16 * q + lane);
 #pragma unroll
-        for (int cc = 0; cc < DV; cc += 32) {
+        for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
             float x[32];
-            tmem_ld32(taddr(tb, 32 * warp, LY::cF + cc), x);
+            tmem_ld32(taddr(tb, 32 * q, LY::cF + cc), x);
             tmem_wait_ld();
             if (own_d) {
 #pragma unroll
@@ -1150,7 +1163,7 @@ cudaError_t launch_lrank_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     dim3 grid(nch, a.H, a.B);
     launch_probe_mark(s);
-    kern<<<grid, NT, LY::BYTES, s>>>(a, maps, (uint8_t *)ws, nch);
+    kern<<<grid, kLPrepThreads<DK>, LY::BYTES, s>>>(a, maps, (uint8_t *)ws, nch);
     return cudaGetLastError();
 }
 
