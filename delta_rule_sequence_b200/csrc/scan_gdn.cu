@@ -96,12 +96,17 @@ struct PrepLayout {
     static_assert(KQ_BLK * (DK / 64) >= (uint32_t)C * DK * 4, "U staging fits over K and V");
 };
 
+// 8 warps, 4 CTAs per SM (64 registers a thread): warp w reads TMEM lane quarter w % 4, and warps
+// w and w + 4 split the columns of every epilogue; the solve runs on warps 0-3.
+constexpr int PREP_THREADS = 256;
+
 template <int DK>
-__global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_constant__ GdnMaps maps,
-                                                     uint8_t *ws, int nch) {
+__global__ void __launch_bounds__(PREP_THREADS, 4) gdn_prep_kernel(ScanArgs p, const __grid_constant__ GdnMaps maps,
+                                                                  uint8_t *ws, int nch) {
     using LY = PrepLayout<DK>;
     using RC = GdnRec<DK>;
     constexpr int DV = RC::DV, BV = RC::BV;
+    constexpr int NTH = PREP_THREADS, NH = NTH / 128;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     __shared__ uint64_t mma_bar, ld_bar;
@@ -109,6 +114,7 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
     __shared__ int failed_sh;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, hs = warp >> 2;  // TMEM lane quarter, column split
     const int c = nch - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int H = p.H, T = p.T;
     const int c0 = c * C, n = min(C, T - c0);
@@ -170,14 +176,14 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
     __syncthreads();
     bool ok = failed_sh == 0;  // uniform across the CTA
     if (ok) {
-        const int t = (warp & 1) * 32 + lane;
+        const int t = (q & 1) * 32 + lane;
         const float gt = sG[t], bt = sBeta[t];
-#pragma unroll
-        for (int cc = 0; cc < C; cc += 32) {
+        {
+            const int cc = hs * 32;
             float gr[32];
-            tmem_ld32(taddr(tb, 32 * warp, cc), gr);
+            tmem_ld32(taddr(tb, 32 * q, cc), gr);
             tmem_wait_ld();
-            if (warp < 2) {
+            if (q < 2) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int i = cc + j;
@@ -197,7 +203,7 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
     __syncthreads();
     // T diag(beta scale) as a bf16 hi / lo pair into the T1 tiles (scale = e^g for Wk, 1 for U)
     auto store_t_pair = [&](bool with_gamma) {
-        for (int e = tid; e < C * (C / 8); e += NT) {
+        for (int e = tid; e < C * (C / 8); e += NTH) {
             const int t = e / (C / 8), c8 = e % (C / 8);
             float a[8];
 #pragma unroll
@@ -214,7 +220,8 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
         }
     };
     if (ok) {
-        solve_unit_lower<NT>(sA, sA, sTmp, tid);
+        if (tid < 128) solve_unit_lower<128>(sA, sA, sTmp, tid, [] { named_sync(2, 128); });
+        __syncthreads();
         store_t_pair(true);
     }
     sync_for_mma();
@@ -240,12 +247,12 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
     }
     // M = 64 accumulators: row r sits in lane 32 (r / 16) + r % 16
     const bool own_t = lane < 16;
-    const int t_row = 16 * warp + lane;
+    const int t_row = 16 * q + lane;
     if (ok) {
 #pragma unroll
-        for (int cc = 0; cc < DK; cc += 32) {
+        for (int cc = hs * (DK / NH); cc < (hs + 1) * (DK / NH); cc += 32) {
             float x[32];
-            tmem_ld32(taddr(tb, 32 * warp, cc), x);
+            tmem_ld32(taddr(tb, 32 * q, cc), x);
             tmem_wait_ld();
             if (own_t) store32_split(rec + RC::WK, nullptr, t_row, cc, x, RC::WK_BLK);
         }
@@ -274,9 +281,9 @@ __global__ void __launch_bounds__(NT) gdn_prep_kernel(ScanArgs p, const __grid_c
     if (ok) {
         uint8_t *stage = sm + LY::KQ;
 #pragma unroll
-        for (int cc = 0; cc < DV; cc += 32) {
+        for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
             float x[32];
-            tmem_ld32(taddr(tb, 32 * warp, cc), x);
+            tmem_ld32(taddr(tb, 32 * q, cc), x);
             tmem_wait_ld();
             if (own_t) {
 #pragma unroll
@@ -1126,7 +1133,7 @@ cudaError_t launch_gdn_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     dim3 grid(nch, a.H, a.B);
     launch_probe_mark(s);
-    kern<<<grid, NT, LY::BYTES, s>>>(a, maps, (uint8_t *)ws, nch);
+    kern<<<grid, PREP_THREADS, LY::BYTES, s>>>(a, maps, (uint8_t *)ws, nch);
     return cudaGetLastError();
 }
 
