@@ -11,7 +11,40 @@ namespace {
 using namespace tc;
 
 constexpr int C = 64;         // chunk length of the tensor-core path
-constexpr int AS = C + 1;     // padded fp32 row stride of the solve matrix
+// fp32 row stride of the solve matrix: rows stay 16-byte aligned for vector loads, and the 4-word
+// pad spreads eight consecutive rows over the eight 16-byte bank groups
+constexpr int AS = C + 4;
+constexpr int kTmp1 = 20, kTmp2 = 36;         // row strides of the solve's two product buffers
+constexpr int kSolveTmpFloats = 32 * kTmp2;   // its scratch (the 16-block pair buffer fits inside)
+
+// N consecutive fp32 in shared memory (16-byte aligned; 8-byte for N = 2) to / from registers
+template <int N>
+__device__ __forceinline__ void vld(const float *p, float *v) {
+    if constexpr (N == 2) {
+        const float2 a = *reinterpret_cast<const float2 *>(p);
+        v[0] = a.x;
+        v[1] = a.y;
+    } else {
+#pragma unroll
+        for (int m = 0; m < N / 4; ++m) {
+            const float4 a = reinterpret_cast<const float4 *>(p)[m];
+            v[4 * m] = a.x;
+            v[4 * m + 1] = a.y;
+            v[4 * m + 2] = a.z;
+            v[4 * m + 3] = a.w;
+        }
+    }
+}
+template <int N>
+__device__ __forceinline__ void vst(float *p, const float *v) {
+    if constexpr (N == 2) {
+        *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+    } else {
+#pragma unroll
+        for (int m = 0; m < N / 4; ++m)
+            reinterpret_cast<float4 *>(p)[m] = make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
+    }
+}
 
 __device__ __forceinline__ void st16(uint8_t *base, uint32_t off, uint4 v) {
     *reinterpret_cast<uint4 *>(base + off) = v;
@@ -108,26 +141,32 @@ __device__ __forceinline__ void mma_split(uint32_t d, uint32_t idesc, int nks, F
 
 // T = (I + A)^{-1} for strictly lower-triangular A (C = 64), blocked: the four 16 x 16 diagonal
 // blocks by forward substitution, then two doubling levels T_21 = -T_22 A_21 T_11 (16 -> 32 -> 64)
-// as register-blocked products with fixed trip counts.  Safe in place (A == Tm): every block is
-// read as A before it is overwritten with T.  Run by 128 threads (tid < 128); SYNC(), a barrier
-// among exactly those threads, separates its phases.  tmp holds 32 x 33 floats.
+// as register-blocked products with fixed trip counts and vector shared-memory accesses.  Safe in
+// place (A == Tm): every block is read as A before it is overwritten with T.  Run by NTH = 128 or
+// 256 threads (tid < NTH); SYNC(), a barrier among exactly those threads, separates its phases.
+// The diagonal blocks take warps 0-3; each doubling product spreads over all NTH threads (one
+// row, 512 / NTH or 1024 / NTH columns a thread).  A, Tm and tmp are 16-byte aligned; tmp holds
+// kSolveTmpFloats floats.
 struct CtaSync {
     __device__ __forceinline__ void operator()() const { __syncthreads(); }
 };
 
 template <int NTH, class SYNC = CtaSync>
 __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid, SYNC sync = SYNC()) {
-    static_assert(NTH == 128, "the solve is laid out for 128 threads");
+    static_assert(NTH == 128 || NTH == 256, "the solve is laid out for 128 or 256 threads");
     const int warp = tid >> 5, lane = tid & 31;
-    // diagonal blocks: warp w inverts block w, lane j < 16 computes column j
-    if (lane < 16) {
+    // diagonal blocks: warp w < 4 inverts block w, lane j < 16 computes column j
+    if (warp < 4 && lane < 16) {
         const int o = 16 * warp, j = lane;
         float x[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
+            float a[16];
+#pragma unroll
+            for (int m = 0; m < (i + 3) / 4; ++m) vld<4>(A + (o + i) * AS + o + 4 * m, a + 4 * m);
             float s = (i == j) ? 1.f : 0.f;
 #pragma unroll
-            for (int k = 0; k < i; ++k) s = fmaf(-A[(o + i) * AS + o + k], x[k], s);
+            for (int k = 0; k < i; ++k) s = fmaf(-a[k], x[k], s);
             x[i] = (i < j) ? 0.f : s;
         }
         __syncwarp(0x0000ffffu);  // every lane has read the block before any lane overwrites it
@@ -135,57 +174,79 @@ __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid,
         for (int i = 0; i < 16; ++i) Tm[(o + i) * AS + o + j] = x[i];
     }
     sync();
-    // level 1, 16-blocks, pairs p = 0, 1: rows r0 = 32p + 16, cols c0 = 32p; thread: 1 row x 4 cols
+    constexpr int TPR = NTH / 32;  // threads per row of a doubling product
+    // level 1, 16-blocks, pairs p = 0, 1: rows r0 = 32p + 16, cols c0 = 32p
     {
-        const int pp = tid >> 6, r = (tid >> 2) & 15, cq = (tid & 3) * 4;
+        constexpr int NC = 16 / TPR;
+        const int pp = tid / (NTH / 2), r = (tid / TPR) & 15, cq = (tid % TPR) * NC;
         const int r0 = 32 * pp + 16, c0 = 32 * pp;
-        float m[4] = {0.f, 0.f, 0.f, 0.f};
+        float *tp = tmp + pp * 16 * kTmp1;
+        float a[16], m[NC];
+        vld<16>(A + (r0 + r) * AS + c0, a);  // row r of A_21
+#pragma unroll
+        for (int j = 0; j < NC; ++j) m[j] = 0.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            const float a = A[(r0 + r) * AS + c0 + k];
+            float tv[NC];
+            vld<NC>(Tm + (c0 + k) * AS + c0 + cq, tv);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) m[j] = fmaf(a, Tm[(c0 + k) * AS + c0 + cq + j], m[j]);
+            for (int j = 0; j < NC; ++j) m[j] = fmaf(a[k], tv[j], m[j]);
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) tmp[pp * 16 * 17 + r * 17 + cq + j] = m[j];
+        vst<NC>(tp + r * kTmp1 + cq, m);
         sync();
+        vld<16>(Tm + (r0 + r) * AS + r0, a);  // row r of T_22
 #pragma unroll
-        for (int j = 0; j < 4; ++j) m[j] = 0.f;
+        for (int j = 0; j < NC; ++j) m[j] = 0.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            const float t = Tm[(r0 + r) * AS + r0 + k];
+            float tv[NC];
+            vld<NC>(tp + k * kTmp1 + cq, tv);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) m[j] = fmaf(t, tmp[pp * 16 * 17 + k * 17 + cq + j], m[j]);
+            for (int j = 0; j < NC; ++j) m[j] = fmaf(a[k], tv[j], m[j]);
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) Tm[(r0 + r) * AS + c0 + cq + j] = -m[j];
+        for (int j = 0; j < NC; ++j) m[j] = -m[j];
+        vst<NC>(Tm + (r0 + r) * AS + c0 + cq, m);
     }
     sync();
-    // level 2, 32-blocks: rows 32.., cols 0..31; thread: 1 row x 8 cols
+    // level 2, 32-blocks: rows 32.., cols 0..31; the 32-long rows are taken in two halves
     {
-        const int r = tid >> 2, cq = (tid & 3) * 8;
-        float m[8];
+        constexpr int NC = 32 / TPR;
+        const int r = tid / TPR, cq = (tid % TPR) * NC;
+        float m[NC];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) m[j] = 0.f;
-#pragma unroll 8
-        for (int k = 0; k < 32; ++k) {
-            const float a = A[(32 + r) * AS + k];
+        for (int j = 0; j < NC; ++j) m[j] = 0.f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) m[j] = fmaf(a, Tm[k * AS + cq + j], m[j]);
+        for (int kh = 0; kh < 2; ++kh) {
+            float a[16];
+            vld<16>(A + (32 + r) * AS + 16 * kh, a);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                float tv[NC];
+                vld<NC>(Tm + (16 * kh + k) * AS + cq, tv);
+#pragma unroll
+                for (int j = 0; j < NC; ++j) m[j] = fmaf(a[k], tv[j], m[j]);
+            }
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) tmp[r * 33 + cq + j] = m[j];
+        vst<NC>(tmp + r * kTmp2 + cq, m);
         sync();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) m[j] = 0.f;
-#pragma unroll 8
-        for (int k = 0; k < 32; ++k) {
-            const float t = Tm[(32 + r) * AS + 32 + k];
+        for (int j = 0; j < NC; ++j) m[j] = 0.f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) m[j] = fmaf(t, tmp[k * 33 + cq + j], m[j]);
+        for (int kh = 0; kh < 2; ++kh) {
+            float a[16];
+            vld<16>(Tm + (32 + r) * AS + 32 + 16 * kh, a);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                float tv[NC];
+                vld<NC>(tmp + (16 * kh + k) * kTmp2 + cq, tv);
+#pragma unroll
+                for (int j = 0; j < NC; ++j) m[j] = fmaf(a[k], tv[j], m[j]);
+            }
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) Tm[(32 + r) * AS + cq + j] = -m[j];
+        for (int j = 0; j < NC; ++j) m[j] = -m[j];
+        vst<NC>(Tm + (32 + r) * AS + cq, m);
     }
     sync();
 }

@@ -91,9 +91,10 @@ struct PrepLayout {
     static constexpr uint32_t T1L = DK == 128 ? KQ + KQ_BLK + C * 128 : T1 + C * 128;
     static constexpr uint32_t AF = DK == 128 ? KQ + 2 * KQ_BLK : T1L + C * 128;  // fp32 A, solved in place into T
     static constexpr uint32_t TMP = AF + C * AS * 4;
-    static constexpr uint32_t GATES = TMP + 32 * 33 * 4;
+    static constexpr uint32_t GATES = TMP + kSolveTmpFloats * 4;
     static constexpr uint32_t BYTES = GATES + 3 * C * 4 + 1024;
     static_assert(KQ_BLK * (DK / 64) >= (uint32_t)C * DK * 4, "U staging fits over K and V");
+    static_assert(4 * (BYTES + 1024 + 64) <= 228 * 1024, "four CTAs share an SM");
 };
 
 // 8 warps, 4 CTAs per SM (64 registers a thread): warp w reads TMEM lane quarter w % 4, and warps
@@ -187,8 +188,9 @@ __global__ void __launch_bounds__(PREP_THREADS, 4) gdn_prep_kernel(ScanArgs p, c
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int i = cc + j;
-                    sA[t * AS + i] = (i < t) ? bt * __expf(gt - sG[i]) * gr[j] : 0.f;
+                    gr[j] = (i < t) ? bt * __expf(gt - sG[i]) * gr[j] : 0.f;
                 }
+                vst<32>(sA + t * AS + cc, gr);
             } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
@@ -206,11 +208,11 @@ __global__ void __launch_bounds__(PREP_THREADS, 4) gdn_prep_kernel(ScanArgs p, c
         for (int e = tid; e < C * (C / 8); e += NTH) {
             const int t = e / (C / 8), c8 = e % (C / 8);
             float a[8];
+            vld<8>(sA + t * AS + c8 * 8, a);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int i = c8 * 8 + j;
-                const float tv = (i <= t) ? sA[t * AS + i] : 0.f;
-                a[j] = tv * sBeta[i] * (with_gamma ? sGam[i] : 1.f);
+                a[j] = (i <= t) ? a[j] * sBeta[i] * (with_gamma ? sGam[i] : 1.f) : 0.f;
             }
             uint4 hv, lv;
             split8(a, hv, lv);
@@ -220,6 +222,7 @@ __global__ void __launch_bounds__(PREP_THREADS, 4) gdn_prep_kernel(ScanArgs p, c
         }
     };
     if (ok) {
+        // on warps 0-3 (measured faster here than spreading it over all 8 warps)
         if (tid < 128) solve_unit_lower<128>(sA, sA, sTmp, tid, [] { named_sync(2, 128); });
         __syncthreads();
         store_t_pair(true);
@@ -345,7 +348,7 @@ struct LPrepLayout {
     static constexpr uint32_t P = AF;                        // P_l hi, lo over the solve buffers,
     static constexpr uint32_t PL = P + BLK;                  // free once both T tiles are built
     static constexpr uint32_t TMP = AF + C * AS * 4;
-    static constexpr uint32_t GATES = TMP + 32 * 33 * 4;     // g, beta, gamma, D
+    static constexpr uint32_t GATES = TMP + kSolveTmpFloats * 4;   // g, beta, gamma, D
     static constexpr uint32_t BYTES = GATES + 4 * C * 4 + 1024;
     static_assert(KQ_BLK * (DK / 64) >= (uint32_t)C * DK * 4, "-X_u staging fits over K and Q");
     static_assert(PL + BLK <= GATES, "the P tiles fit over the solve buffers");
@@ -354,14 +357,14 @@ struct LPrepLayout {
     static constexpr uint32_t TCOLS = cF + DK <= 256 ? 256 : 512;
 };
 
-// 8 warps at d = 128 (one CTA per SM: its TMEM accumulators take 448 columns), 4 at d = 64 (two
-// CTAs per SM).  Warp w reads TMEM lane quarter w % 4; with 8 warps, warps w and w + 4 split the
-// columns of every epilogue.
+// 8 warps: one CTA per SM at d = 128 (its TMEM accumulators take 448 columns), two at d = 64
+// (256 columns and 103 KB of shared memory each).  Warp w reads TMEM lane quarter w % 4; warps w
+// and w + 4 split the columns of every epilogue.
 template <int DK>
-constexpr int kLPrepThreads = DK == 128 ? 256 : 128;
+constexpr int kLPrepThreads = 256;
 
 template <int DK>
-__global__ void __launch_bounds__(kLPrepThreads<DK>) lrank_prep_kernel(ScanArgs p, const __grid_constant__ LMaps maps,
+__global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_prep_kernel(ScanArgs p, const __grid_constant__ LMaps maps,
                                                                       uint8_t *ws, int nch) {
     using LY = LPrepLayout<DK>;
     constexpr int NTH = kLPrepThreads<DK>;
@@ -470,8 +473,9 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>) lrank_prep_kernel(ScanArgs 
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int i = cc + j;
-                    sA[t * AS + i] = (i < t) ? bt * __expf(gt - sG[i]) * gr[j] : 0.f;
+                    gr[j] = (i < t) ? bt * __expf(gt - sG[i]) * gr[j] : 0.f;
                 }
+                vst<32>(sA + t * AS + cc, gr);
             } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
@@ -489,11 +493,11 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>) lrank_prep_kernel(ScanArgs 
         for (int e = tid; e < C * (C / 8); e += NTH) {
             const int t = e / (C / 8), c8 = e % (C / 8);
             float a[8];
+            vld<8>(sA + t * AS + c8 * 8, a);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int i = c8 * 8 + j;
-                const float tv = (i <= t) ? sA[t * AS + i] : 0.f;
-                a[j] = scaled ? tv * sBeta[i] * sGam[i] : tv;
+                a[j] = (i <= t) ? (scaled ? a[j] * sBeta[i] * sGam[i] : a[j]) : 0.f;
             }
             uint4 hv, lv;
             split8(a, hv, lv);
@@ -503,11 +507,7 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>) lrank_prep_kernel(ScanArgs 
         }
     };
     if (ok) {
-        if (tid < 128) {
-            if constexpr (NTH == 128) solve_unit_lower<128>(sA, sA, sTmp, tid);
-            else solve_unit_lower<128>(sA, sA, sTmp, tid, [] { named_sync(2, 128); });
-        }
-        __syncthreads();
+        solve_unit_lower<NTH>(sA, sA, sTmp, tid);  // ends with a CTA barrier
         store_t_pair(true);
     }
     sync_for_mma();
@@ -941,6 +941,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status, lim)) { ok = false; break; }
             const float *g = reinterpret_cast<const float *>(buf + LY::B_G);
             const float g_last = g[C - 1];
+            const float g_row = g[lowq ? lrow : lrow - 64];  // g of this thread's Y / output row
             const uint32_t d1 = LY::cD1 + (c & 1) * N2;
             float ow[CH];  // rank L: O_w of this thread's output row, fetched early
 #pragma unroll
@@ -960,7 +961,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             // Y = U - X_s (lanes 0..63 of D1), and D Y
             if (lowq) {
                 const int t = lrow;
-                const float dd = t < n ? __expf(g_last - g[t]) : 0.f;
+                const float dd = t < n ? __expf(g_last - g_row) : 0.f;
                 float y[CH];  // U first: it does not depend on D1
 #pragma unroll
                 for (int j4 = 0; j4 < CH; j4 += 4) {
@@ -1002,6 +1003,9 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                         }
                     }
                 }
+                // the last read of the chunk buffer (g is held in registers): release it, so that
+                // the chunk two ahead loads while this one's state and output epilogues run
+                warp_arrive(&bars.empty[c & 1], lane);
                 if (!mbar_wait(&bars.d4_full, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 float xh[CH], xl[CH];
@@ -1050,7 +1054,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 }
                 if (!mbar_wait(&bars.ox_full, c & 1, status, lim)) { ok = false; break; }
                 if (t < n && out) {
-                    const float gt = __expf(g[t]);
+                    const float gt = __expf(g_row);
                     __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t) * H + h) * dv + v0 + j0;
 #pragma unroll
                     for (int c8 = 0; c8 < CH / 8; ++c8) {
@@ -1072,9 +1076,6 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                     }
                 }
             }
-            // D1 / D3 reads done (the MMA thread learns so from this warp's later arrivals); the
-            // chunk buffer (g, U) is released
-            warp_arrive(&bars.empty[c & 1], lane);
         }
         if (!ok) fail();
         if (p.S_final && own_d && !failed()) {
