@@ -331,14 +331,14 @@ template <int DK>
 struct LPrepLayout {
     static constexpr uint32_t KQ_BLK = 2 * C * 128;     // [K; Q] rows of one 64-column block
     static constexpr uint32_t BLK = C * 128;            // one 64-column block of a C-row tile
-    // W_l / U_l buffers: two at d = 128 (the next rank loads while this one is used); one at
-    // d = 64, where shared memory is kept small enough for two CTAs per SM
-    static constexpr int NBUF = DK == 128 ? 2 : 1;
+    // W_l buffers: two (the next rank's W loads while this one's is read); U_l buffers: two at
+    // d = 128, one at d = 64, where shared memory is kept small enough for two CTAs per SM
+    static constexpr int NBU = DK == 128 ? 2 : 1;
     static constexpr uint32_t TILE = BLK * (DK / 64);   // one C x DK bf16 tile
     static constexpr uint32_t KQ = 0;
     static constexpr uint32_t W = KQ + KQ_BLK * (DK / 64);   // W_l, K-major (rows t)
-    static constexpr uint32_t U = W + NBUF * TILE;           // U_l, [t][dv] (MN-major B operand)
-    static constexpr uint32_t DU = U + NBUF * TILE;          // D U_l hi, lo; later sum P U hi, lo
+    static constexpr uint32_t U = W + 2 * TILE;              // U_l, [t][dv] (MN-major B operand)
+    static constexpr uint32_t DU = U + NBU * TILE;           // D U_l hi, lo; later sum P U hi, lo
     static constexpr uint32_t DUL = DU + BLK * (DK / 64);
     static constexpr uint32_t T1 = DUL + BLK * (DK / 64);    // T diag(beta gamma), then T: hi, lo
     static constexpr uint32_t T1L = T1 + BLK;
@@ -352,6 +352,7 @@ struct LPrepLayout {
     static constexpr uint32_t BYTES = GATES + 4 * C * 4 + 1024;
     static_assert(KQ_BLK * (DK / 64) >= (uint32_t)C * DK * 4, "-X_u staging fits over K and Q");
     static_assert(PL + BLK <= GATES, "the P tiles fit over the solve buffers");
+    static_assert(DK == 128 || 2 * (BYTES + 1024 + 64) <= 228 * 1024, "two CTAs share an SM at d = 64");
     // TMEM: G (64 columns, M = 128), then Wk / sum P U / X_u, O_w, F_w (DK columns each)
     static constexpr uint32_t cG = 0, cA = 64, cO = cA + DK, cF = cO + DK;
     static constexpr uint32_t TCOLS = cF + DK <= 256 ? 256 : 512;
@@ -369,11 +370,13 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     using LY = LPrepLayout<DK>;
     constexpr int NTH = kLPrepThreads<DK>;
     constexpr int NH = NTH / 128;  // column splits of an epilogue
+    constexpr int CW = C / NH;     // columns of G a thread owns
+    static_assert(CW == 32, "the G epilogues move 32 columns a thread");
     using RC = GdnRec<DK, true>;
     constexpr int DV = RC::DV, BV = RC::BV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t mma_bar, ld_bar, wu_bar[2];
+    __shared__ uint64_t mma_bar, ld_bar, w_bar[2], u_bar[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int failed_sh;
 
@@ -381,7 +384,7 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     const int q = warp & 3, hs = warp >> 2;  // TMEM lane quarter, column split
     const int c = nch - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int H = p.H, T = p.T, L = p.L;
-    constexpr int NBUF = LY::NBUF;
+    constexpr int NBU = LY::NBU;
     const int c0 = c * C, n = min(C, T - c0);
     uint8_t *rec = ws + kRecOffset + (((size_t)b * H + h) * nch + c) * RC::BYTES;
     float *sA = (float *)(sm + LY::AF);
@@ -392,22 +395,28 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     float *sD = sGam + C;
     const uint32_t sb = smem_u32(sm);
     uint32_t mph = 0, lph = 0;  // phases of mma_bar and ld_bar
-    // W_l and U_l of rank l into buffer l % NBUF, completing on wu_bar[l % NBUF]
-    auto load_wu = [&](int l) {
-        const int bi = l % NBUF;
-        mbar_expect_tx(&wu_bar[bi], 2 * LY::TILE);
-        for (int blk = 0; blk < DK / 64; ++blk) {
-            tma_load_4d(sm + LY::W + bi * LY::TILE + blk * LY::BLK, &maps.w, blk * 64, h * L + l, c0, b, &wu_bar[bi]);
-            tma_load_4d(sm + LY::U + bi * LY::TILE + blk * LY::BLK, &maps.u, blk * 64, h * L + l, c0, b, &wu_bar[bi]);
-        }
+    // W_l into W buffer l % 2 (completing on w_bar[l % 2]), U_l into U buffer l % NBU (u_bar)
+    auto load_w = [&](int l) {
+        const int bi = l & 1;
+        mbar_expect_tx(&w_bar[bi], LY::TILE);
+        for (int blk = 0; blk < DK / 64; ++blk)
+            tma_load_4d(sm + LY::W + bi * LY::TILE + blk * LY::BLK, &maps.w, blk * 64, h * L + l, c0, b, &w_bar[bi]);
     };
-    int wu_issued = 0;  // ranks whose loads were issued (thread 0)
+    auto load_u = [&](int l) {
+        const int bi = l % NBU;
+        mbar_expect_tx(&u_bar[bi], LY::TILE);
+        for (int blk = 0; blk < DK / 64; ++blk)
+            tma_load_4d(sm + LY::U + bi * LY::TILE + blk * LY::BLK, &maps.u, blk * 64, h * L + l, c0, b, &u_bar[bi]);
+    };
+    int w_issued = 0, u_issued = 0;  // ranks whose W / U loads were issued (thread 0)
 
     if (tid == 0) {
         mbar_init(&mma_bar, 1);
         mbar_init(&ld_bar, 1);
-        mbar_init(&wu_bar[0], 1);
-        mbar_init(&wu_bar[1], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&w_bar[i], 1);
+            mbar_init(&u_bar[i], 1);
+        }
         mbar_fence_init();
         failed_sh = 0;
         mbar_expect_tx(&ld_bar, 2 * (DK / 64) * C * 128);
@@ -416,7 +425,8 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
             tma_load_4d(sm + LY::KQ + blk * LY::KQ_BLK + C * 128, &maps.q, blk * 64, h, c0, b, &ld_bar);
         }
         // the first ranks' W_l, U_l load while A, T and Wk are computed
-        for (; wu_issued < L && wu_issued < NBUF; ++wu_issued) load_wu(wu_issued);
+        for (; w_issued < L && w_issued < 2; ++w_issued) load_w(w_issued);
+        for (; u_issued < L && u_issued < NBU; ++u_issued) load_u(u_issued);
     }
     if (warp == 0) tmem_alloc(&tmem_base_sh, LY::TCOLS);
     if (tid < C) {
@@ -451,6 +461,15 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
         __syncthreads();
         return failed_sh == 0;
     };
+    // the same wait, for MMAs whose commit thread 0 already issued
+    auto mma_done_committed = [&](bool issued) -> bool {
+        __syncwarp();
+        if (issued && !mbar_wait(&mma_bar, mph & 1, p.status)) failed_sh = 1;
+        if (issued) mph++;
+        fence_after_sync();
+        __syncthreads();
+        return failed_sh == 0;
+    };
     auto okq = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::KQ_BLK); };
     auto okb = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::BLK); };
     auto ok0 = [](int ks) { return (uint64_t)koff_k_sw128(ks, 0); };
@@ -459,32 +478,33 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
 
     // G = [K; Q] K^T  ->  A (fp32, shared) and Mqk (hi / lo, straight to the record)
     bool ok = failed_sh == 0;
-    if (ok && tid == 0) mma_steps<DK / 16>(tb + LY::cG, idesc_bf16(128, C, 0, 0), dKQ, dKQ, okq, okq, false);
-    ok = mma_done(ok);
-    if (ok) {
-        const int t = (q & 1) * 32 + lane;
-        const float gt = sG[t], bt = sBeta[t];
+    if (ok && tid == 0) {
+        mma_steps<DK / 16>(tb + LY::cG, idesc_bf16(128, C, 0, 0), dKQ, dKQ, okq, okq, false);
+        mma_commit(&mma_bar);
+    }
+    // Every G epilogue (this one and one per rank) gives this thread row t_g, columns cg ..
+    // cg + 31, and scales them by the same factors, computed once while the MMA runs:
+    // beta_t e^{g_t - g_i} for i < t on the K rows (lane quarters 0-1: A and P_l), e^{g_t - g_i}
+    // for i <= t on the Q rows (quarters 2-3: Mqk and Mqw_l).
+    const int t_g = (q & 1) * 32 + lane, cg = hs * CW;
+    float dec[CW];
+    {
+        const float gt = sG[t_g], sc = q < 2 ? sBeta[t_g] : 1.f;
 #pragma unroll
-        for (int cc = hs * (C / NH); cc < (hs + 1) * (C / NH); cc += 32) {
-            float gr[32];
-            tmem_ld32(taddr(tb, 32 * q, LY::cG + cc), gr);
-            tmem_wait_ld();
-            if (q < 2) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int i = cc + j;
-                    gr[j] = (i < t) ? bt * __expf(gt - sG[i]) * gr[j] : 0.f;
-                }
-                vst<32>(sA + t * AS + cc, gr);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int i = cc + j;
-                    gr[j] = (i <= t) ? __expf(gt - sG[i]) * gr[j] : 0.f;
-                }
-                store32_split(rec + RC::MQK, rec + RC::MQK + C * 128, t, cc, gr);
-            }
+        for (int j = 0; j < CW; ++j) {
+            const int i = cg + j;
+            dec[j] = (q < 2 ? i < t_g : i <= t_g) ? sc * __expf(gt - sG[i]) : 0.f;
         }
+    }
+    ok = mma_done_committed(ok);
+    if (ok) {
+        float gr[CW];
+        tmem_ld32(taddr(tb, 32 * q, LY::cG + cg), gr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < CW; ++j) gr[j] *= dec[j];
+        if (q < 2) vst<CW>(sA + t_g * AS + cg, gr);
+        else store32_split(rec + RC::MQK, rec + RC::MQK + C * 128, t_g, cg, gr);
     }
     fence_before_sync();
     __syncthreads();
@@ -534,48 +554,37 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     __syncthreads();
     if (ok) store_t_pair(false);  // the Wk MMA has completed: the T tiles are free
 
-    // the write terms, one rank at a time
+    // the write terms, one rank at a time.  G_l = [K; Q] W_l^T is issued together with the
+    // previous rank's MMAs (W is double-buffered), so each rank waits for one MMA batch.
     const uint32_t idV = idesc_bf16(64, DV, 0, 1);
+    auto issue_g = [&](int l) {  // thread 0, once W_l has landed
+        const uint64_t dW = make_desc(sb + LY::W + (l & 1) * LY::TILE, 16, 1024, 2);
+        mma_steps<DK / 16>(tb + LY::cG, idesc_bf16(128, C, 0, 0), dKQ, dW, okq, okb, false);
+    };
+    if (ok && tid == 0) {
+        if (mbar_wait(&w_bar[0], 0, p.status)) issue_g(0);
+        else failed_sh = 1;
+    }
+    ok = mma_done(ok);
     for (int l = 0; l < L && ok; ++l) {
-        const int bi = l % NBUF;
-        const uint32_t wb = LY::W + bi * LY::TILE, ub = LY::U + bi * LY::TILE;
-        const uint64_t dW = make_desc(sb + wb, 16, 1024, 2);
+        const uint32_t wb = LY::W + (l & 1) * LY::TILE, ub = LY::U + (l % NBU) * LY::TILE;
         const uint64_t dWmn = make_desc(sb + wb, LY::BLK, 1024, 2);
         const uint64_t dU = make_desc(sb + ub, LY::BLK, 1024, 2);
-        if (tid == 0 && l + NBUF < L) {  // the rank after the ones in flight: start it toward L2
+        if (tid == 0 && l + 2 < L) {  // the rank after the ones in flight: start it toward L2
             for (int blk = 0; blk < DK / 64; ++blk) {
-                tma_prefetch_4d(&maps.w, blk * 64, h * L + l + NBUF, c0, b);
-                tma_prefetch_4d(&maps.u, blk * 64, h * L + l + NBUF, c0, b);
+                tma_prefetch_4d(&maps.w, blk * 64, h * L + l + 2, c0, b);
+                tma_prefetch_4d(&maps.u, blk * 64, h * L + l + 2, c0, b);
             }
         }
-        if (!mbar_wait(&wu_bar[bi], (l / NBUF) & 1, p.status)) failed_sh = 1;
-        fence_before_sync();
-        __syncthreads();
-        fence_after_sync();
-        ok = failed_sh == 0;
-        // G_l = [K; Q] W_l^T
-        if (ok && tid == 0) mma_steps<DK / 16>(tb + LY::cG, idesc_bf16(128, C, 0, 0), dKQ, dW, okq, okb, false);
-        ok = mma_done(ok);
-        if (!ok) break;
         {   // P_l (rows of K W^T, quarters 0-1) and Mqw_l (rows of Q W^T, quarters 2-3) as pairs
-            const int t = (q & 1) * 32 + lane;
-            const float gt = sG[t], bt = sBeta[t];
-            uint8_t *dh = sm + (q < 2 ? LY::P : LY::MQW);
-            uint8_t *dl = sm + (q < 2 ? LY::PL : LY::MQWL);
+            float gr[CW];
+            tmem_ld32(taddr(tb, 32 * q, LY::cG + cg), gr);
+            tmem_wait_ld();
 #pragma unroll
-            for (int cc = hs * (C / NH); cc < (hs + 1) * (C / NH); cc += 32) {
-                float gr[32];
-                tmem_ld32(taddr(tb, 32 * q, LY::cG + cc), gr);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int i = cc + j;
-                    const bool keep = (q < 2) ? (i < t) : (i <= t);
-                    gr[j] = keep ? (q < 2 ? bt : 1.f) * __expf(gt - sG[i]) * gr[j] : 0.f;
-                }
-                store32_split(dh, dl, t, cc, gr);
-            }
+            for (int j = 0; j < CW; ++j) gr[j] *= dec[j];
+            store32_split(sm + (q < 2 ? LY::P : LY::MQW), sm + (q < 2 ? LY::PL : LY::MQWL), t_g, cg, gr);
         }
+        if (!mbar_wait(&u_bar[l % NBU], (l / NBU) & 1, p.status)) failed_sh = 1;
         for (int e = tid; e < C * (DV / 8); e += NTH) {  // D U_l as a hi / lo pair
             const int t = e / (DV / 8), c8 = e % (DV / 8);
             const uint32_t off = sw128_off(t, c8 * 8, LY::BLK);
@@ -590,7 +599,8 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
             st16(sm + LY::DUL, off, dl);
         }
         sync_for_mma();
-        if (tid == 0) {
+        ok = failed_sh == 0;
+        if (ok && tid == 0) {
             const bool acc = l > 0;
             // sum P U (accumulated over l in the Wk columns) and O_w
             mma_steps<C / 16>(tb + LY::cA, idV, make_desc(sb + LY::P, 16, 1024, 2), dU, ok0, omn, acc);
@@ -601,10 +611,18 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
             const uint32_t idF = idesc_bf16(DK, DV, 1, 1);
             mma_steps<C / 16>(tb + LY::cF, idF, dWmn, make_desc(sb + LY::DU, LY::BLK, 1024, 2), omn, omn, acc);
             mma_steps<C / 16>(tb + LY::cF, idF, dWmn, make_desc(sb + LY::DUL, LY::BLK, 1024, 2), omn, omn, true);
+            // the next rank's G (its epilogue read of the G columns above is complete)
+            if (l + 1 < L) {
+                if (mbar_wait(&w_bar[(l + 1) & 1], ((l + 1) >> 1) & 1, p.status)) issue_g(l + 1);
+                else failed_sh = 1;
+            }
         }
         ok = mma_done(ok);
-        // this buffer's MMAs are done: the rank NBUF ahead can load into it
-        if (ok && tid == 0 && wu_issued < L) load_wu(wu_issued++);
+        // rank l's W and U buffers are free: W_{l+2} and U_{l+NBU} load into them
+        if (ok && tid == 0) {
+            if (w_issued < L) load_w(w_issued++);
+            if (u_issued < L) load_u(u_issued++);
+        }
     }
     // sum P U -> hi / lo pair (over the D U tiles), then X_u = T (sum P U)
     if (ok) {
@@ -694,8 +712,10 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     // after a failure, let the tile loads still in flight land before the CTA exits
     if (!ok && tid == 0) {
         mbar_wait(&ld_bar, 0, nullptr, kStallTestPolls);
-        for (int l = wu_issued > NBUF ? wu_issued - NBUF : 0; l < wu_issued; ++l)
-            mbar_wait(&wu_bar[l % NBUF], (l / NBUF) & 1, nullptr, kStallTestPolls);
+        for (int l = w_issued > 2 ? w_issued - 2 : 0; l < w_issued; ++l)
+            mbar_wait(&w_bar[l & 1], (l >> 1) & 1, nullptr, kStallTestPolls);
+        for (int l = u_issued > NBU ? u_issued - NBU : 0; l < u_issued; ++l)
+            mbar_wait(&u_bar[l % NBU], (l / NBU) & 1, nullptr, kStallTestPolls);
     }
     __syncthreads();
     if (warp == 0) tmem_dealloc(tb, LY::TCOLS);
