@@ -155,19 +155,18 @@ template <int NTH, class SYNC = CtaSync>
 __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid, SYNC sync = SYNC()) {
     static_assert(NTH == 128 || NTH == 256, "the solve is laid out for 128 or 256 threads");
     const int warp = tid >> 5, lane = tid & 31;
-    // diagonal blocks: warp w < 4 inverts block w, lane j < 16 computes column j
+    // diagonal blocks: warp w < 4 inverts block w, lane j < 16 computes column j by forward
+    // substitution in column order (once x_k is final it is eliminated from every later row, so
+    // the dependent chain is 15 steps long, each step a set of independent FMAs)
     if (warp < 4 && lane < 16) {
         const int o = 16 * warp, j = lane;
         float x[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float a[16];
+        for (int i = 0; i < 16; ++i) x[i] = (i == j) ? 1.f : 0.f;
 #pragma unroll
-            for (int m = 0; m < (i + 3) / 4; ++m) vld<4>(A + (o + i) * AS + o + 4 * m, a + 4 * m);
-            float s = (i == j) ? 1.f : 0.f;
+        for (int k = 0; k < 15; ++k) {
 #pragma unroll
-            for (int k = 0; k < i; ++k) s = fmaf(-a[k], x[k], s);
-            x[i] = (i < j) ? 0.f : s;
+            for (int i = k + 1; i < 16; ++i) x[i] = fmaf(-A[(o + i) * AS + o + k], x[k], x[i]);
         }
         __syncwarp(0x0000ffffu);  // every lane has read the block before any lane overwrites it
 #pragma unroll

@@ -342,24 +342,27 @@ struct LPrepLayout {
     static constexpr uint32_t DUL = DU + BLK * (DK / 64);
     static constexpr uint32_t T1 = DUL + BLK * (DK / 64);    // T diag(beta gamma), then T: hi, lo
     static constexpr uint32_t T1L = T1 + BLK;
-    static constexpr uint32_t MQW = T1L + BLK;               // Mqw_l hi, lo
-    static constexpr uint32_t MQWL = MQW + BLK;
+    // [P_l; Mqw_l] as two M = 128 operands: the lo rows after the T tiles, the hi rows over the
+    // solve buffer (free once both T tiles are built)
+    static constexpr uint32_t PL = T1L + BLK;
+    static constexpr uint32_t MQWL = PL + BLK;
     static constexpr uint32_t AF = MQWL + BLK;               // fp32 A, solved in place into T
-    static constexpr uint32_t P = AF;                        // P_l hi, lo over the solve buffers,
-    static constexpr uint32_t PL = P + BLK;                  // free once both T tiles are built
+    static constexpr uint32_t P = AF;
+    static constexpr uint32_t MQW = P + BLK;
     static constexpr uint32_t TMP = AF + C * AS * 4;
     static constexpr uint32_t GATES = TMP + kSolveTmpFloats * 4;   // g, beta, gamma, D
     static constexpr uint32_t BYTES = GATES + 4 * C * 4 + 1024;
     static_assert(KQ_BLK * (DK / 64) >= (uint32_t)C * DK * 4, "-X_u staging fits over K and Q");
-    static_assert(PL + BLK <= GATES, "the P tiles fit over the solve buffers");
+    static_assert(MQW + BLK <= TMP, "the hi P / Mqw rows fit over the solve matrix");
     static_assert(DK == 128 || 2 * (BYTES + 1024 + 64) <= 228 * 1024, "two CTAs share an SM at d = 64");
-    // TMEM: G (64 columns, M = 128), then Wk / sum P U / X_u, O_w, F_w (DK columns each)
-    static constexpr uint32_t cG = 0, cA = 64, cO = cA + DK, cF = cO + DK;
-    static constexpr uint32_t TCOLS = cF + DK <= 256 ? 256 : 512;
+    // TMEM: G (64 columns, M = 128); Wk, then [sum P U; O_w] (M = 128), then X_u (DK columns);
+    // F_w as its D U_hi and D U_lo halves (2 DK columns)
+    static constexpr uint32_t cG = 0, cA = 64, cF = cA + DK;
+    static constexpr uint32_t TCOLS = cF + 2 * DK <= 256 ? 256 : 512;
 };
 
 // 8 warps: one CTA per SM at d = 128 (its TMEM accumulators take 448 columns), two at d = 64
-// (256 columns and 103 KB of shared memory each).  Warp w reads TMEM lane quarter w % 4; warps w
+// (256 columns and 112 KB of shared memory each).  Warp w reads TMEM lane quarter w % 4; warps w
 // and w + 4 split the columns of every epilogue.
 template <int DK>
 constexpr int kLPrepThreads = 256;
@@ -602,15 +605,14 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
         ok = failed_sh == 0;
         if (ok && tid == 0) {
             const bool acc = l > 0;
-            // sum P U (accumulated over l in the Wk columns) and O_w
-            mma_steps<C / 16>(tb + LY::cA, idV, make_desc(sb + LY::P, 16, 1024, 2), dU, ok0, omn, acc);
-            mma_steps<C / 16>(tb + LY::cA, idV, make_desc(sb + LY::PL, 16, 1024, 2), dU, ok0, omn, true);
-            mma_steps<C / 16>(tb + LY::cO, idV, make_desc(sb + LY::MQW, 16, 1024, 2), dU, ok0, omn, acc);
-            mma_steps<C / 16>(tb + LY::cO, idV, make_desc(sb + LY::MQWL, 16, 1024, 2), dU, ok0, omn, true);
-            // F_w = sum W_l^T (D U_l)  (M = DK: W_l read as an MN-major A operand)
-            const uint32_t idF = idesc_bf16(DK, DV, 1, 1);
+            // [sum P U; O_w] += [P_l; Mqw_l] U_l  (M = 128, accumulated over l in the Wk columns)
+            const uint32_t idPU = idesc_bf16(128, DV, 0, 1);
+            mma_steps<C / 16>(tb + LY::cA, idPU, make_desc(sb + LY::P, 16, 1024, 2), dU, ok0, omn, acc);
+            mma_steps<C / 16>(tb + LY::cA, idPU, make_desc(sb + LY::PL, 16, 1024, 2), dU, ok0, omn, true);
+            // F_w += W_l^T [D U_l hi | D U_l lo]  (M = DK: W_l read as an MN-major A operand;
+            // N = 2 DV: the D U tiles sit side by side as one operand)
+            const uint32_t idF = idesc_bf16(DK, 2 * DV, 1, 1);
             mma_steps<C / 16>(tb + LY::cF, idF, dWmn, make_desc(sb + LY::DU, LY::BLK, 1024, 2), omn, omn, acc);
-            mma_steps<C / 16>(tb + LY::cF, idF, dWmn, make_desc(sb + LY::DUL, LY::BLK, 1024, 2), omn, omn, true);
             // the next rank's G (its epilogue read of the G columns above is complete)
             if (l + 1 < L) {
                 if (mbar_wait(&w_bar[(l + 1) & 1], ((l + 1) >> 1) & 1, p.status)) issue_g(l + 1);
@@ -624,26 +626,34 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
             if (u_issued < L) load_u(u_issued++);
         }
     }
-    // sum P U -> hi / lo pair (over the D U tiles), then X_u = T (sum P U)
+    // [sum P U; O_w]: the sum P U rows (lane quarters 0-1) become a hi / lo pair over the D U
+    // tiles, the O_w rows (quarters 2-3) go straight to the record
     if (ok) {
+        const int t = 32 * (q & 1) + lane;
 #pragma unroll
         for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
             float x[32];
             tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
             tmem_wait_ld();
-            if (own_t) {
+            if (q < 2) {
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
                     uint4 hv, lv;
                     split8(x + 8 * c8, hv, lv);
-                    const uint32_t off = sw128_off(t_row, cc + 8 * c8, LY::BLK);
+                    const uint32_t off = sw128_off(t, cc + 8 * c8, LY::BLK);
                     st16(sm + LY::DU, off, hv);
                     st16(sm + LY::DUL, off, lv);
                 }
+            } else {
+                float *dst = reinterpret_cast<float *>(rec + RC::OW) + (size_t)t * DV + cc;
+#pragma unroll
+                for (int j4 = 0; j4 < 32; j4 += 4)
+                    *reinterpret_cast<float4 *>(dst + j4) = make_float4(x[j4], x[j4 + 1], x[j4 + 2], x[j4 + 3]);
             }
         }
     }
     sync_for_mma();
+    // X_u = T (sum P U)  (M = 64, into the same columns)
     if (ok && tid == 0) {
         const uint64_t dPU = make_desc(sb + LY::DU, LY::BLK, 1024, 2);
         const uint64_t dPUL = make_desc(sb + LY::DUL, LY::BLK, 1024, 2);
@@ -651,10 +661,32 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
         mma_steps<C / 16>(tb + LY::cA, idV, dT, dPU, ok0, omn, false);
         mma_steps<C / 16>(tb + LY::cA, idV, dT, dPUL, ok0, omn, true);
         mma_steps<C / 16>(tb + LY::cA, idV, dTL, dPU, ok0, omn, true);
+        mma_commit(&mma_bar);
     }
-    ok = mma_done(ok);
-    // -X_u -> the U slot (staged over K and Q in the record's slice layout, one bulk store);
-    // O_w and F_w straight to the record
+    // F_w (its MMAs are complete) while X_u runs: the D U_hi and D U_lo halves summed; rows d:
+    // lane = d for M = 128 (DK = 128), lanes 32q + r, r < 16, for M = 64
+    if (ok) {
+        const bool own_d = (DK == 128) ? true : (lane < 16);
+        const int d_row = (DK == 128) ? 32 * q + lane : (16 * q + lane);
+#pragma unroll
+        for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 16) {
+            float xh[16], xl[16];
+            tmem_ld16(taddr(tb, 32 * q, LY::cF + cc), xh);
+            tmem_ld16(taddr(tb, 32 * q, LY::cF + DV + cc), xl);
+            tmem_wait_ld();
+            if (own_d) {
+#pragma unroll
+                for (int j4 = 0; j4 < 16; j4 += 4) {
+                    const int j = cc + j4;
+                    *reinterpret_cast<float4 *>(rec + RC::FW + (j / BV) * RC::FW_SLICE + u_off<BV>(d_row, j % BV)) =
+                        make_float4(xh[j4] + xl[j4], xh[j4 + 1] + xl[j4 + 1], xh[j4 + 2] + xl[j4 + 2],
+                                    xh[j4 + 3] + xl[j4 + 3]);
+                }
+            }
+        }
+    }
+    ok = mma_done_committed(ok);
+    // -X_u -> the U slot (staged over K and Q in the record's slice layout, one bulk store)
     if (ok) {
         uint8_t *stage = sm + LY::KQ;
 #pragma unroll
@@ -668,35 +700,6 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
                     const int j = cc + j4;
                     *reinterpret_cast<float4 *>(stage + (j / BV) * RC::U_SLICE + u_off<BV>(t_row, j % BV)) =
                         make_float4(-x[j4], -x[j4 + 1], -x[j4 + 2], -x[j4 + 3]);
-                }
-            }
-        }
-#pragma unroll
-        for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
-            float x[32];
-            tmem_ld32(taddr(tb, 32 * q, LY::cO + cc), x);
-            tmem_wait_ld();
-            if (own_t) {
-                float *dst = reinterpret_cast<float *>(rec + RC::OW) + (size_t)t_row * DV + cc;
-#pragma unroll
-                for (int j4 = 0; j4 < 32; j4 += 4)
-                    *reinterpret_cast<float4 *>(dst + j4) = make_float4(x[j4], x[j4 + 1], x[j4 + 2], x[j4 + 3]);
-            }
-        }
-        // F_w rows d: lane = d for M = 128 (DK = 128); lanes 32q + r, r < 16, for M = 64
-        const bool own_d = (DK == 128) ? true : (lane < 16);
-        const int d_row = (DK == 128) ? 32 * q + lane : (16 * q + lane);
-#pragma unroll
-        for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
-            float x[32];
-            tmem_ld32(taddr(tb, 32 * q, LY::cF + cc), x);
-            tmem_wait_ld();
-            if (own_d) {
-#pragma unroll
-                for (int j4 = 0; j4 < 32; j4 += 4) {
-                    const int j = cc + j4;
-                    *reinterpret_cast<float4 *>(rec + RC::FW + (j / BV) * RC::FW_SLICE + u_off<BV>(d_row, j % BV)) =
-                        make_float4(x[j4], x[j4 + 1], x[j4 + 2], x[j4 + 3]);
                 }
             }
         }
