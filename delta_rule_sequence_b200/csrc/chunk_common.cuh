@@ -139,6 +139,31 @@ __device__ __forceinline__ void mma_split(uint32_t d, uint32_t idesc, int nks, F
         for (int ks = 0; ks < nks; ++ks) mma_bf16(d, adesc(alo, ks), bdesc(bhi, ks), idesc, 1);
 }
 
+// Two fp32 lanes per instruction (the packed f32x2 arithmetic of sm_100): d = a * b + c, each
+// lane rounded as fmaf rounds it
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long ra, rb, rc, rd;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(rc) : "f"(c.x), "f"(c.y));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+    float2 d;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+    return d;
+}
+
+// m[0..N) += a * v[0..N) for even N, two lanes an instruction
+template <int N>
+__device__ __forceinline__ void axpy2(float a, const float *v, float *m) {
+    static_assert(N % 2 == 0, "pairs");
+#pragma unroll
+    for (int p = 0; p < N / 2; ++p) {
+        const float2 r = ffma2(make_float2(a, a), make_float2(v[2 * p], v[2 * p + 1]), make_float2(m[2 * p], m[2 * p + 1]));
+        m[2 * p] = r.x;
+        m[2 * p + 1] = r.y;
+    }
+}
+
 // T = (I + A)^{-1} for strictly lower-triangular A (C = 64), blocked: the four 16 x 16 diagonal
 // blocks by forward substitution, then two doubling levels T_21 = -T_22 A_21 T_11 (16 -> 32 -> 64)
 // as register-blocked products with fixed trip counts and vector shared-memory accesses.  Safe in
@@ -188,8 +213,7 @@ __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid,
         for (int k = 0; k < 16; ++k) {
             float tv[NC];
             vld<NC>(Tm + (c0 + k) * AS + c0 + cq, tv);
-#pragma unroll
-            for (int j = 0; j < NC; ++j) m[j] = fmaf(a[k], tv[j], m[j]);
+            axpy2<NC>(a[k], tv, m);
         }
         vst<NC>(tp + r * kTmp1 + cq, m);
         sync();
@@ -200,8 +224,7 @@ __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid,
         for (int k = 0; k < 16; ++k) {
             float tv[NC];
             vld<NC>(tp + k * kTmp1 + cq, tv);
-#pragma unroll
-            for (int j = 0; j < NC; ++j) m[j] = fmaf(a[k], tv[j], m[j]);
+            axpy2<NC>(a[k], tv, m);
         }
 #pragma unroll
         for (int j = 0; j < NC; ++j) m[j] = -m[j];
@@ -223,8 +246,7 @@ __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid,
             for (int k = 0; k < 16; ++k) {
                 float tv[NC];
                 vld<NC>(Tm + (16 * kh + k) * AS + cq, tv);
-#pragma unroll
-                for (int j = 0; j < NC; ++j) m[j] = fmaf(a[k], tv[j], m[j]);
+                axpy2<NC>(a[k], tv, m);
             }
         }
         vst<NC>(tmp + r * kTmp2 + cq, m);
@@ -239,8 +261,7 @@ __device__ void solve_unit_lower(const float *A, float *Tm, float *tmp, int tid,
             for (int k = 0; k < 16; ++k) {
                 float tv[NC];
                 vld<NC>(tmp + (16 * kh + k) * kTmp2 + cq, tv);
-#pragma unroll
-                for (int j = 0; j < NC; ++j) m[j] = fmaf(a[k], tv[j], m[j]);
+                axpy2<NC>(a[k], tv, m);
             }
         }
 #pragma unroll

@@ -304,7 +304,8 @@ __global__ void __launch_bounds__(PREP_THREADS, 4) gdn_prep_kernel(ScanArgs p, c
     if (ok && tid == 0) {
         bulk_s2g(rec + RC::U, sm + LY::KQ, (uint32_t)(C * DV * 4));
         bulk_commit();
-        bulk_wait_all();
+        bulk_wait_read();  // the staging buffer is read out before the CTA frees it; the kernel's
+                           // end makes the writes visible to the next launch
     }
     // after a failure, let the tile loads still in flight land before the CTA exits
     if (!ok && tid == 0) mbar_wait(&ld_bar, v_issued ? 1 : 0, nullptr);
@@ -710,7 +711,8 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     if (ok && tid == 0) {
         bulk_s2g(rec + RC::U, sm + LY::KQ, (uint32_t)(C * DV * 4));
         bulk_commit();
-        bulk_wait_all();
+        bulk_wait_read();  // the staging buffer is read out before the CTA frees it; the kernel's
+                           // end makes the writes visible to the next launch
     }
     // after a failure, let the tile loads still in flight land before the CTA exits
     if (!ok && tid == 0) {
