@@ -54,7 +54,7 @@ def load_peaks():
 
 
 # The kernels a step of each bench workload launches, in launch order, and the source files each
-# is compiled from (the hash of those files keys the committed ncu traffic figures).
+# is compiled from (the hash of those files' code keys the committed ncu traffic figures).
 STEP_KERNELS = {
     "gdn": ["gdn_prep_kernel", "gdn_state_kernel"],
     "recsys": ["lrank_prep_kernel", "gdn_state_kernel"],
@@ -69,12 +69,20 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text):
+    """C++ source without its comments and with runs of blank space folded, so that editing a
+    comment does not invalidate a traffic figure measured on the same code."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash(kernel):
     pkg = os.path.join(ROOT, "delta_rule_sequence_b200")
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES[kernel]:
-        with open(os.path.normpath(os.path.join(pkg, rel)), "rb") as f:
-            h.update(os.path.basename(rel).encode() + b"\0" + f.read())
+        with open(os.path.normpath(os.path.join(pkg, rel)), encoding="utf-8") as f:
+            h.update(os.path.basename(rel).encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -737,7 +737,8 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
 // so the Y epilogue runs on sub-partitions 0-1 and the output epilogue on 2-3, where it does not
 // slow the MMA warp (sub-partition 0) issuing the next chunk's round 1.  D1 is double-buffered in
 // TMEM.  K, Q arrive by TMA tiled loads, the per-chunk record (Wk, Mqk, the U slice, g) by bulk
-// copies, one chunk ahead.
+// copies, into two chunk buffers: chunk c + 2 loads into chunk c's buffer as soon as its last
+// readers (the round 2 MMAs and the state epilogue's F_w read) are done.
 
 template <int DK, bool RL = false>
 struct StateLayout {

@@ -62,7 +62,8 @@ def test_gdn_write_bf16_widths(dk, T):
     check_scan_full(make_inputs(wl, seed=dk), wl.chunk, wl.io)
 
 
-@pytest.mark.parametrize("dk,L,T", [(128, 8, 130), (64, 1, 64), (128, 3, 1)])
+@pytest.mark.parametrize("dk,L,T", [(128, 8, 130), (64, 1, 64), (128, 3, 1), (64, 3, 200),
+                                    (64, 5, 129), (128, 2, 257)])
 def test_rank_l_write_bf16(dk, L, T):
     wl = WORKLOADS["long"].with_(H=2, T=T, dk=dk, dv=dk, L=L, chunk=64)
     check_scan_full(make_inputs(wl, seed=L), wl.chunk, wl.io)
