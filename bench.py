@@ -66,6 +66,8 @@ KERNEL_SOURCES = {
     "lrank_prep_kernel": _GDN_SOURCES,
     "gdn_state_kernel": _GDN_SOURCES,
     "decode_kernel": ["csrc/decode.cu", "csrc/common.cuh"],
+    "write_producer_kernel": ["csrc/producer.cu", "csrc/producer.cuh", "csrc/chunk_common.cuh",
+                              "csrc/tc.cuh", "csrc/common.cuh"],
 }
 
 
@@ -190,6 +192,19 @@ def scan_flops(wl):
     else:
         per = C * d * (5 + 4 * L) + C * C / 3 + d * d * (6 + 2 * L)
     return wl.B * wl.T * wl.H * per
+
+
+def producer_bytes(wl):
+    """Algorithmic bytes of one write-producer call: per token x, v in and the L pairs (u, w) out
+    at bf16, beta in fp32; per head the weights [W_k; W_p] (bf16) and the ShortConv taps (fp32)."""
+    d, L = wl.dk, wl.L
+    tok = wl.B * wl.T * wl.H
+    return tok * (2 * d * 2 + 4 * L + 2 * L * d * 2) + wl.H * (L * 2 * d * d * 2 + 4 * d * 4)
+
+
+def producer_flops(wl):
+    """The 2L projections of every token's anchor (W_k a, W_p a: 2 FLOPs a multiply-add)."""
+    return wl.B * wl.T * wl.H * 2 * (2 * wl.L * wl.dk * wl.dk)
 
 
 def decode_bytes(wl, io_bytes=2):
@@ -332,6 +347,61 @@ def time_workload(wl, dev, stream, peaks, rank, max_over_ranks, barrier, world, 
                          "algorithmic_bytes": alg, "algorithmic_flops": scan_flops(wl),
                          "tensor_frac_algorithmic": scan_flops(wl) / (kern_ms / 1e3) / 1e12
                          / peaks["bf16_tflops"]},
+            "steps": steps}
+
+
+def time_producer(wl, dev, stream, peaks, rank, max_over_ranks, barrier, world, steps=20):
+    """The write-term producer on a scan workload's shape (random weights), timed alone."""
+    from delta_rule_sequence_b200 import prism
+    from delta_rule_sequence_b200.workloads import make_producer_inputs
+
+    p = {n: t.to(dev) for n, t in make_producer_inputs(wl, seed=7 + rank).items()}
+    u = torch.empty((wl.B, wl.T, wl.H, wl.L, wl.dk), dtype=torch.bfloat16, device=dev)
+    w = torch.empty_like(u)
+
+    def call():
+        prism.prism_write_producer(p["x"], p["v"], p["conv"], p["Wk"], p["Wp"], p["beta"], u=u, w=w,
+                                   stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+    stream.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for row in evs:
+            for e in row:
+                e.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(steps):
+            prism.record_launch_events(evs[i])
+            call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    status = prism.prism_query_device_status(None, stream)
+    if status != prism.PRISM_OK:
+        raise SystemExit(f"bench: device status after the producer: {prism.status_string(status)}")
+    ms = max_over_ranks(e0.elapsed_time(e1)) / steps
+    kern_ms = sum(r[0].elapsed_time(r[1]) for r in evs) / steps
+    alg, fl = producer_bytes(wl), producer_flops(wl)
+    achieved = alg / (kern_ms / 1e3) / 1e9
+    del p, u, w
+    return {"workload": f"write producer on {wl.name}: B={wl.B} H={wl.H} T={wl.T} d={wl.dk} L={wl.L} "
+                        f"bf16 I/O, random weights",
+            "ms_per_call": ms, "tokens_per_s": world * wl.B * wl.T / (ms / 1e3), "launches": 1,
+            "ms_per_launch": {"write_producer_kernel": kern_ms},
+            "dram_bytes_per_launch": {"write_producer_kernel":
+                                      committed_traffic("producer_" + wl.name, "write_producer_kernel")},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "algorithmic_bytes": alg, "algorithmic_flops": fl,
+                         "tensor_frac_algorithmic": fl / (kern_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
             "steps": steps}
 
 
@@ -621,6 +691,9 @@ def main():
         for name in ("recsys", "long"):
             others[name] = time_workload(WORKLOADS[name], dev, stream, peaks, rank, max_over_ranks,
                                          barrier, world)
+        for name in ("recsys", "long"):  # the write-term producer on the same shapes
+            others["producer_" + name] = time_producer(WORKLOADS[name], dev, stream, peaks, rank,
+                                                       max_over_ranks, barrier, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "producer.cuh"
 
 namespace prism {
 cudaError_t launch_scan_simt(const ScanArgs &a, bool io_f32, cudaStream_t s);
@@ -297,6 +298,29 @@ prism_status prism_step_decode(const prism_shape *shape, const void *q, const vo
     return cuda_status(err);
 }
 
+prism_status prism_write_producer(const prism_shape *shape, const void *x, const void *v,
+                                  const float *conv, const void *Wk, const void *Wp,
+                                  const float *beta, void *u, void *w, void *stream) {
+    if (!shape) return PRISM_ERR_INVALID_ARG;
+    const prism_shape &s = *shape;
+    if (s.B < 0 || s.H < 0 || s.T < 0 || s.L < 1 || s.dk < 1 || s.dv < 1) return PRISM_ERR_INVALID_ARG;
+    if (s.io != PRISM_BF16 && s.io != PRISM_F32) return PRISM_ERR_INVALID_ARG;
+    if (s.io != PRISM_BF16 || s.dk != s.dv || (s.dk != 64 && s.dk != 128) || s.L > 64)
+        return PRISM_ERR_UNSUPPORTED;
+    if (s.B > 65535 || s.H > 65535) return PRISM_ERR_UNSUPPORTED;
+    if ((long long)s.B * s.H * s.T == 0) return PRISM_OK;
+    for (const void *ptr : {x, v, (const void *)conv, Wk, Wp, (const void *)u, (const void *)w})
+        if (!ptr || !aligned16(ptr)) return PRISM_ERR_INVALID_ARG;
+    if (!beta || ((uintptr_t)beta & 3u)) return PRISM_ERR_INVALID_ARG;
+    for (const void *in : {x, v, (const void *)conv, Wk, Wp, (const void *)beta})
+        if (in == u || in == w) return PRISM_ERR_INVALID_ARG;  // outputs alias an input
+    if (u == w) return PRISM_ERR_INVALID_ARG;
+    prism::ProducerArgs a{s.B, s.H, s.T, s.dk, s.L, x, v, conv, Wk, Wp, beta, u, w};
+    cudaError_t err = prism::launch_write_producer(a, (cudaStream_t)stream);
+    probe_finish((cudaStream_t)stream);
+    return cuda_status(err);
+}
+
 prism_status prism_query_device_status(void *workspace, void *stream) {
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t err = cudaStreamSynchronize(s);
@@ -308,9 +332,11 @@ prism_status prism_query_device_status(void *workspace, void *stream) {
         if (word != PRISM_OK && (err = cudaMemset(workspace, 0, sizeof word)) != cudaSuccess)
             return cuda_status(err);
     }
-    uint32_t dword = 0;
+    uint32_t dword = 0, pword = 0;
     if ((err = prism::decode_status(&dword)) != cudaSuccess) return cuda_status(err);
+    if ((err = prism::producer_status(&pword)) != cudaSuccess) return cuda_status(err);
     if (word == PRISM_OK) word = dword;
+    if (word == PRISM_OK) word = pword;
     return (prism_status)word;
 }
 

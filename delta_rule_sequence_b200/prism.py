@@ -27,6 +27,7 @@ EXPORTS = (
     "prism_scan_segment_element",
     "prism_state_fold",
     "prism_step_decode",
+    "prism_write_producer",
     "prism_query_device_status",
     "prism_status_string",
     "prism_last_cuda_error",
@@ -81,6 +82,8 @@ def load_library():
     lib.prism_state_fold.restype = ci
     lib.prism_step_decode.argtypes = [shp] + [vp] * 9 + [vp]
     lib.prism_step_decode.restype = ci
+    lib.prism_write_producer.argtypes = [shp] + [vp] * 8 + [vp]
+    lib.prism_write_producer.restype = ci
     lib.prism_query_device_status.argtypes = [vp, vp]
     lib.prism_query_device_status.restype = ci
     lib.prism_status_string.argtypes = [ci]
@@ -245,6 +248,37 @@ def prism_step_decode(q, k, v, alpha, beta, u, w, S, *, o=None, stream=None):
     if rc != PRISM_OK:
         raise PrismError(rc, "prism_step_decode")
     return o
+
+
+def prism_write_producer(x, v, conv, Wk, Wp, beta, *, u=None, w=None, stream=None):
+    """The input-anchored write terms (include/prism.h, prism_write_producer).  x, v: [B,T,H,d]
+    bf16; conv: [H,4,d] fp32; Wk, Wp: [H,L,d,d] bf16; beta: [B,T,H,L] fp32.  Returns (u, w), each
+    [B,T,H,L,d] bf16, ready for prism_scan_fwd."""
+    lib = load_library()
+    if not isinstance(x, torch.Tensor) or not x.is_cuda:
+        raise TypeError("x must be a CUDA tensor (libprism has no CPU path)")
+    dev = x.device
+    B, T, H, d = x.shape
+    L = Wk.shape[1]
+    bf = torch.bfloat16
+    _check_tensor("x", x, bf, (B, T, H, d), dev)
+    _check_tensor("v", v, bf, (B, T, H, d), dev)
+    _check_tensor("conv", conv, torch.float32, (H, 4, d), dev)
+    _check_tensor("Wk", Wk, bf, (H, L, d, d), dev)
+    _check_tensor("Wp", Wp, bf, (H, L, d, d), dev)
+    _check_tensor("beta", beta, torch.float32, (B, T, H, L), dev)
+    if u is None:
+        u = torch.empty((B, T, H, L, d), dtype=bf, device=dev)
+    if w is None:
+        w = torch.empty((B, T, H, L, d), dtype=bf, device=dev)
+    _check_tensor("u", u, bf, (B, T, H, L, d), dev)
+    _check_tensor("w", w, bf, (B, T, H, L, d), dev)
+    shape = PrismShape(B, H, T, d, d, L, 64, PRISM_BF16)
+    rc = lib.prism_write_producer(ctypes.byref(shape), _ptr(x), _ptr(v), _ptr(conv), _ptr(Wk),
+                                  _ptr(Wp), _ptr(beta), _ptr(u), _ptr(w), _stream(stream))
+    if rc != PRISM_OK:
+        raise PrismError(rc, "prism_write_producer")
+    return u, w
 
 
 def prism_scan_fwd_launch_count(shape: PrismShape) -> int:

@@ -123,6 +123,21 @@ def make_inputs(wl: Workload, seed: int = 0) -> dict:
     return {"q": q, "k": k, "v": v, "alpha": alpha, "beta": beta, "u": u, "w": w, "S0": S0}
 
 
+def make_producer_inputs(wl: Workload, seed: int = 0) -> dict:
+    """Inputs of the write-term producer for a workload's shape (d = dk = dv, L ranks), random
+    weights: x, v [B,T,H,d] ~ N(0, 1) bf16; conv [H,4,d] ~ N(0, 1/4) fp32; Wk, Wp [H,L,d,d] ~
+    N(0, 1/d) bf16; beta [B,T,H,L] = sigmoid(N(0, 1)) fp32."""
+    g = _gen(seed * 7919 + 17)
+    B, T, H, d, L = wl.B, wl.T, wl.H, wl.dk, wl.L
+    x = torch.randn((B, T, H, d), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, T, H, d), generator=g).to(torch.bfloat16)
+    conv = (torch.randn((H, 4, d), generator=g) * 0.5).float().contiguous()
+    Wk = (torch.randn((H, L, d, d), generator=g) / d ** 0.5).to(torch.bfloat16)
+    Wp = (torch.randn((H, L, d, d), generator=g) / d ** 0.5).to(torch.bfloat16)
+    beta = torch.sigmoid(torch.randn((B, T, H, L), generator=g)).float().contiguous()
+    return {"x": x, "v": v, "conv": conv, "Wk": Wk, "Wp": Wp, "beta": beta}
+
+
 def make_decode_state(wl: Workload, seed: int = 0) -> dict:
     """Entry state and the fixed write projections of a decode run."""
     g = _gen(seed * 1_000_003 + 7)

@@ -160,10 +160,33 @@ prism_status prism_scan_fwd_noalloc(const prism_shape *shape, const void *q, con
                                     float *S_final, void *stream);
 
 /*
+ * prism_write_producer -- the input-anchored write terms in front of the scan ("PRISM: Parallel
+ * Residual Iterative Sequence Model", gist.science explainer, technical summary 2.2; the anchor
+ * width of the banbantang.com PRISM article, section 5(1), the first residual of its section
+ * 3(4)).  For every (b, t, h), with d = dk = dv:
+ *   a_t     = sum_{j=0..3} conv[h][j] * x_{t-j}            depthwise causal ShortConv, x_{<0} = 0
+ *   k^(l)   = Wk[h][l] a_t,   p^(l) = Wp[h][l] a_t          l = 1..L (row = output index)
+ *   r^(1)   = v_t,   delta^(l) = GELU(p^(l) * r^(l)),   r^(l+1) = r^(l) - delta^(l)   (exact GELU)
+ *   u_{t,l} = beta_t^(l) delta^(l),   w_{t,l} = k^(l)
+ * so that prism_scan_fwd with these u, w writes B_t = sum_l beta delta k^T.
+ *   x, v     [B,T,H,d]   bf16          conv  [H,4,d]  fp32 (conv[h][0] multiplies x_t)
+ *   Wk, Wp   [H,L,d,d]   bf16          beta  [B,T,H,L] fp32 (4-byte aligned)
+ *   u, w     [B,T,H,L,d] bf16 outputs  (must not overlap each other or any input)
+ * Uses shape->B, H, T, dk, dv, L, io; requires io == PRISM_BF16 and dk == dv in {64, 128}
+ * (PRISM_ERR_UNSUPPORTED otherwise), 1 <= L <= 64.  The two projections run on the tensor cores
+ * from a bf16 anchor with fp32 accumulation; the residual chain and GELU in fp32; u, w are rounded
+ * to bf16 (nearest even).  A bounded wait that gives up records PRISM_ERR_TIMEOUT in the library's
+ * producer status word (prism_query_device_status).
+ */
+prism_status prism_write_producer(const prism_shape *shape, const void *x, const void *v,
+                                  const float *conv, const void *Wk, const void *Wp,
+                                  const float *beta, void *u, void *w, void *stream);
+
+/*
  * prism_query_device_status -- synchronise `stream`, read the status word in `workspace` (written
  * by scan kernels whose bounded waits ran out; workspace may be NULL) and the library's decode
- * status word, and clear them.  Returns PRISM_OK, PRISM_ERR_TIMEOUT, or PRISM_ERR_CUDA if the
- * stream itself reports an error.
+ * and producer status words, and clear them.  Returns PRISM_OK, PRISM_ERR_TIMEOUT, or
+ * PRISM_ERR_CUDA if the stream itself reports an error.
  */
 prism_status prism_query_device_status(void *workspace, void *stream);
 

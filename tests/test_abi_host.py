@@ -100,6 +100,26 @@ def test_decode_rejects_bad_arguments(lib):
     assert lib.prism_step_decode(ctypes.byref(s), *bad) == P.PRISM_ERR_INVALID_ARG  # S NULL
 
 
+def test_producer_rejects_bad_arguments(lib):
+    def call(shape, x=FAKE, v=FAKE, conv=FAKE, Wk=FAKE, Wp=FAKE, beta=FAKE,
+             u=ctypes.c_void_p(0x30000), w=ctypes.c_void_p(0x40000)):
+        return lib.prism_write_producer(ctypes.byref(shape), x, v, conv, Wk, Wp, beta, u, w, None)
+
+    ok = dict(dk=64, dv=64, L=3, io=P.PRISM_BF16)
+    assert call(_shape(**dict(ok, T=0))) == P.PRISM_OK                       # nothing to do
+    assert call(_shape(**dict(ok, dk=32, dv=32))) == P.PRISM_ERR_UNSUPPORTED
+    assert call(_shape(**dict(ok, dv=128))) == P.PRISM_ERR_UNSUPPORTED      # dk != dv
+    assert call(_shape(**dict(ok, io=P.PRISM_F32))) == P.PRISM_ERR_UNSUPPORTED
+    assert call(_shape(**dict(ok, L=0))) == P.PRISM_ERR_INVALID_ARG
+    assert call(_shape(**dict(ok, L=65))) == P.PRISM_ERR_UNSUPPORTED
+    assert call(_shape(**ok), x=None) == P.PRISM_ERR_INVALID_ARG
+    assert call(_shape(**ok), Wp=MISALIGNED) == P.PRISM_ERR_INVALID_ARG
+    assert call(_shape(**ok), beta=ctypes.c_void_p(0x10002)) == P.PRISM_ERR_INVALID_ARG
+    assert call(_shape(**ok), u=FAKE) == P.PRISM_ERR_INVALID_ARG             # u aliases the inputs
+    assert call(_shape(**ok), w=ctypes.c_void_p(0x30000)) == P.PRISM_ERR_INVALID_ARG  # u == w
+    assert lib.prism_write_producer(None, *([None] * 8), None) == P.PRISM_ERR_INVALID_ARG
+
+
 def test_launch_probe_arguments(lib):
     assert lib.prism_debug_record_launch_events(None, -1) == P.PRISM_ERR_INVALID_ARG
     assert lib.prism_debug_record_launch_events(None, 2) == P.PRISM_ERR_INVALID_ARG

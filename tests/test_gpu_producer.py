@@ -1,0 +1,106 @@
+"""GPU parity of the write-term producer (prism_write_producer) against its fp64 oracle
+(oracle/write_producer.py), element by element on the same seeded bf16 bytes: ragged token
+counts around the 128-token tile, L = 1 and odd L, both widths; the full-size recsys and
+long-context shapes on sampled token windows; and the producer feeding the scan, against the
+oracle producer feeding the oracle scan.  Tolerance: bf16 outputs, |x - r| <= 2e-2 (1 + |r|)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.write_producer import CONV_WIDTH, write_producer_ref
+from delta_rule_sequence_b200.workloads import WORKLOADS, make_inputs, make_producer_inputs
+from tests.parity import TOL, compare, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from delta_rule_sequence_b200 import build
+
+    build.build()
+
+
+def _run_device(p):
+    from delta_rule_sequence_b200.prism import prism_query_device_status, prism_write_producer
+
+    d = to_device(p)
+    u, w = prism_write_producer(d["x"], d["v"], d["conv"], d["Wk"], d["Wp"], d["beta"])
+    assert prism_query_device_status(None) == 0  # synchronises; no bounded wait gave up
+    return u, w
+
+
+def _run(p):
+    u, w = _run_device(p)
+    return u.float().cpu().numpy(), w.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("d,L,B,H,T", [(64, 3, 1, 2, 200), (128, 2, 2, 1, 130), (64, 1, 1, 1, 64),
+                                       (128, 5, 1, 2, 1), (64, 4, 2, 2, 257), (128, 1, 1, 1, 128)])
+def test_producer_matches_oracle(d, L, B, H, T):
+    wl = WORKLOADS["recsys"].with_(B=B, H=H, T=T, dk=d, dv=d, L=L)
+    p = make_producer_inputs(wl, seed=d + L + T)
+    u, w = _run(p)
+    u_ref, w_ref, _ = write_producer_ref(**p)
+    compare("u", u, u_ref, TOL["bf16"])
+    compare("w", w, w_ref, TOL["bf16"])
+
+
+@pytest.mark.parametrize("name", ["recsys", "long"])
+def test_producer_full_size_sampled(name):
+    """The full-size shape in one launch; sampled (b, h) sequences on token windows that cross
+    a tile boundary, against the oracle run on the window and the 3 tokens before it."""
+    wl = WORKLOADS[name]
+    p = make_producer_inputs(wl, seed=5)
+    u, w = _run_device(p)
+    g = np.random.default_rng(11)
+    for _ in range(3):
+        b, h = int(g.integers(wl.B)), int(g.integers(wl.H))
+        t0 = int(g.integers(1, wl.T // 128)) * 128 - 5  # straddles a 128-token tile boundary
+        lo = t0 - (CONV_WIDTH - 1)
+        sl = {k: (t[b:b + 1, lo:t0 + 16, h:h + 1] if t.dim() >= 4 and k in ("x", "v", "beta")
+                  else t[h:h + 1]) for k, t in p.items()}
+        u_ref, w_ref, _ = write_producer_ref(**sl)
+        got_u = u[b:b + 1, t0:t0 + 16, h:h + 1].float().cpu().numpy()
+        got_w = w[b:b + 1, t0:t0 + 16, h:h + 1].float().cpu().numpy()
+        compare(f"u[{b},{t0}:,{h}]", got_u, u_ref[:, CONV_WIDTH - 1:], TOL["bf16"])
+        compare(f"w[{b},{t0}:,{h}]", got_w, w_ref[:, CONV_WIDTH - 1:], TOL["bf16"])
+
+
+def test_producer_feeds_the_scan():
+    """producer -> scan on the GPU against oracle producer -> oracle scan (same bf16 inputs; the
+    oracle scan reads the GPU's bf16 u, w only through the bf16 rounding of its own u, w)."""
+    from delta_rule_sequence_b200.prism import prism_scan_fwd
+
+    wl = WORKLOADS["recsys"].with_(B=1, H=2, T=300, L=3)
+    p = make_producer_inputs(wl, seed=3)
+    x = make_inputs(wl, seed=3)
+    d = to_device(p)
+    from delta_rule_sequence_b200.prism import prism_write_producer
+
+    u, w = prism_write_producer(d["x"], d["v"], d["conv"], d["Wk"], d["Wp"], d["beta"])
+    dx = to_device(x)
+    o, S = prism_scan_fwd(dx["q"], dx["k"], None, dx["alpha"], dx["beta"], u, w, None, chunk=64)
+    torch.cuda.synchronize()
+    u_ref, w_ref, _ = write_producer_ref(**p)
+    u_bf = torch.from_numpy(u_ref).to(torch.bfloat16)
+    w_bf = torch.from_numpy(w_ref).to(torch.bfloat16)
+    o_ref, S_ref = oracle.scan_ref(x["q"], x["k"], None, x["alpha"], x["beta"], u_bf, w_bf, None)
+    compare("o", o.float().cpu().numpy(), o_ref, TOL["bf16"])
+    compare("S_final", S.cpu().numpy(), S_ref, TOL["bf16"])
+
+
+def test_producer_leaves_no_tokens_untouched_and_no_status():
+    """T not a multiple of the tile: every output element is written (the buffers start as NaN)."""
+    from delta_rule_sequence_b200.prism import prism_write_producer
+
+    wl = WORKLOADS["long"].with_(H=3, T=333, L=2)
+    p = to_device(make_producer_inputs(wl, seed=9))
+    u = torch.full((1, 333, 3, 2, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    w = torch.full_like(u, float("nan"))
+    prism_write_producer(p["x"], p["v"], p["conv"], p["Wk"], p["Wp"], p["beta"], u=u, w=w)
+    torch.cuda.synchronize()
+    assert torch.isfinite(u.float()).all() and torch.isfinite(w.float()).all()
