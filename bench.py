@@ -352,6 +352,8 @@ def time_workload(wl, dev, stream, peaks, rank, max_over_ranks, barrier, world, 
 
 def time_producer(wl, dev, stream, peaks, rank, max_over_ranks, barrier, world, steps=20):
     """The write-term producer on a scan workload's shape (random weights), timed alone."""
+    import torch
+
     from delta_rule_sequence_b200 import prism
     from delta_rule_sequence_b200.workloads import make_producer_inputs
 
