@@ -12,7 +12,7 @@
 // The anchor depends only on the input window, so every token's chain runs at once; the 2L
 // projections of a token are one GEMM row against the stacked weights [W_k^(l); W_p^(l)].
 //
-// One CTA per 128 tokens of one (batch, head): eight epilogue warps build the anchor tile (the A
+// One CTA per 128 tokens of one (batch, head), two CTAs per SM at d = 64: eight epilogue warps build the anchor tile (the A
 // operand, as a bf16 hi / lo pair: a single bf16 anchor lets the residual chain amplify its
 // rounding past the bf16 output tolerance by the fourth rank) and hold the residual in registers (a token row and half its columns a thread);
 // one warp loads the weights by TMA (double-buffered per l) and issues, for each l, one
@@ -67,7 +67,7 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(P_THREADS, 1) write_producer_kernel(ProducerArgs p,
+__global__ void __launch_bounds__(P_THREADS, D == 64 ? 2 : 1) write_producer_kernel(ProducerArgs p,
                                                                      const __grid_constant__ CUtensorMap mk,
                                                                      const __grid_constant__ CUtensorMap mp) {
     using LY = ProdLayout<D>;
@@ -199,26 +199,30 @@ __global__ void __launch_bounds__(P_THREADS, 1) write_producer_kernel(ProducerAr
             fence_after_sync();
             const float bl = live ? p.beta[tok * L + l] : 0.f;
             const size_t orow = (tok * L + l) * D;
+            // 16 columns at a time (directions, then gains), few registers beyond the residual
 #pragma unroll
-            for (int ci = 0; ci < HALF / 32; ++ci) {
-                const int col = c_base + 32 * ci;
-                float kk[32], pp[32];
-                tmem_ld32(taddr(tb, 32 * q, bi * 2 * D + col), kk);
-                tmem_ld32(taddr(tb, 32 * q, bi * 2 * D + D + col), pp);
+            for (int ci = 0; ci < HALF / 16; ++ci) {
+                const int col = c_base + 16 * ci;
+                float kk[16];
+                tmem_ld16(taddr(tb, 32 * q, bi * 2 * D + col), kk);
+                tmem_wait_ld();
+                if (live) {
+                    *reinterpret_cast<uint4 *>(wo + orow + col) = pack8(kk);
+                    *reinterpret_cast<uint4 *>(wo + orow + col + 8) = pack8(kk + 8);
+                }
+                float pp[16];
+                tmem_ld16(taddr(tb, 32 * q, bi * 2 * D + D + col), pp);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float z = pp[j] * r[32 * ci + j];
+                for (int j = 0; j < 16; ++j) {
+                    const float z = pp[j] * r[16 * ci + j];
                     const float dl = 0.5f * z * (1.f + erff(z * kRsqrt2));
-                    r[32 * ci + j] -= dl;
+                    r[16 * ci + j] -= dl;
                     pp[j] = bl * dl;
                 }
                 if (live) {
-#pragma unroll
-                    for (int c8 = 0; c8 < 32; c8 += 8) {
-                        *reinterpret_cast<uint4 *>(wo + orow + col + c8) = pack8(kk + c8);
-                        *reinterpret_cast<uint4 *>(uo + orow + col + c8) = pack8(pp + c8);
-                    }
+                    *reinterpret_cast<uint4 *>(uo + orow + col) = pack8(pp);
+                    *reinterpret_cast<uint4 *>(uo + orow + col + 8) = pack8(pp + 8);
                 }
             }
             fence_before_sync();
