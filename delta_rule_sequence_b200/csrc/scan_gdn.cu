@@ -729,16 +729,16 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
 // ------------------------------------------------------------------------------------------------
 // state: one CTA per (value slice, head, batch), chunks in order
 //
-// Two MMA rounds per chunk (8 instructions at d = 128 for the first, 4 + 4 for the second):
-//   round 1:  D1 = [Wk; Q] [S_hi | S_lo]                    (M = 128, N = 2 BV: X_s and QS)
-//   round 2:  D4 = K^T [DY_hi | DY_lo]                      (the state update, on the chain)
+// Two MMA stages per chunk (8 instructions at d = 128 for the first, 4 + 4 for the second):
+//   stage 1:  D1 = [Wk; Q] [S_hi | S_lo]                    (M = 128, N = 2 BV: X_s and QS)
+//   stage 2:  D4 = K^T [DY_hi | DY_lo]                      (the state update, on the chain)
 //             D3 = [Mqk_lo; Mqk_hi] [Y_hi | Y_lo]           (the output's intra-chunk term)
 // X_s and the Mqk_lo product sit in TMEM lanes 0..63, QS and the Mqk_hi product in lanes 64..127,
 // so the Y epilogue runs on sub-partitions 0-1 and the output epilogue on 2-3, where it does not
-// slow the MMA warp (sub-partition 0) issuing the next chunk's round 1.  D1 is double-buffered in
+// slow the MMA warp (sub-partition 0) issuing the next chunk's stage 1.  D1 is double-buffered in
 // TMEM.  K, Q arrive by TMA tiled loads, the per-chunk record (Wk, Mqk, the U slice, g) by bulk
 // copies, into two chunk buffers: chunk c + 2 loads into chunk c's buffer as soon as its last
-// readers (the round 2 MMAs and the state epilogue's F_w read) are done.
+// readers (the stage 2 MMAs and the state epilogue's F_w read) are done.
 
 template <int DK, bool RL = false>
 struct StateLayout {
