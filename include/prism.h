@@ -93,8 +93,12 @@ prism_status prism_scan_fwd_launch_count(const prism_shape *shape, int *launches
  *                              kernel records a failure; prism_query_device_status reads and
  *                              clears it); may be reused once the stream has passed this call
  * The result equals the token recurrence above up to floating-point rounding: state and all
- * accumulation in fp32; bf16 operands are fed to the tensor cores.  A partial last chunk is
- * handled as if padded with identity tokens (alpha = 1, beta = 0, no write).
+ * accumulation in fp32; bf16 operands are fed to the tensor cores (intermediate results as bf16
+ * hi / lo pairs, except the chunk's Wk, a single bf16).  The bf16 tolerance |x - r| <= 2e-2
+ * (1 + |r|) is met for unit-norm keys and write directions; with write directions of norm ~8
+ * the state grows into the hundreds and one output element in ~4e4 was seen at 1.4x that
+ * bound.  A partial last chunk is handled as if padded with identity tokens (alpha = 1,
+ * beta = 0, no write).
  */
 prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void *k,
                             const void *v, const float *alpha, const float *beta,
