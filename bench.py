@@ -216,6 +216,18 @@ def decode_bytes(wl, io_bytes=2):
 
 # ------------------------------------------------------------------------------------------------
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_oracle_sample(wl, budget_s=12.0, n_threads=None):
     """Time the fp64 oracle on whole (b, h) sequences of the workload.  Returns (tokens/s,
     description, threads).  One sequence is timed alone first to size a sample of about
@@ -280,7 +292,7 @@ def run_reference(args, rank):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(wl),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -700,7 +712,8 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, threads = cpu_oracle_sample(wl)
-        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
+        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "cpu_model": cpu_model()}
 
     for g in graphs:
         g.reset()

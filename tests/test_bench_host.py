@@ -61,3 +61,8 @@ def test_peaks_come_from_the_measured_file_when_present():
     if os.path.exists(os.path.join(bench.ROOT, "MEASURED_PEAKS.json")):
         assert kind == "measured"
     assert peaks["hbm_gbs"] > 0
+
+
+def test_cpu_model_is_a_string():
+    m = bench.cpu_model()
+    assert isinstance(m, str) and m
