@@ -3,7 +3,6 @@
 Reduced sizes compare every element and span several chunks plus a ragged tail; full sizes run
 the launch configuration the bench times and compare sampled (b, h) sequences.  Tolerances:
 2e-2 for bf16 I/O, 1e-4 for fp32 I/O, element-wise |x - r| <= tol (1 + |r|)."""
-import numpy as np
 import pytest
 import torch
 
