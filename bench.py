@@ -1,25 +1,28 @@
 #!/usr/bin/env python
 """Throughput of the chunked gated delta-rule scan forward (tokens/s per layer) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
-A step is one prism_scan_fwd call over one batch of the GDN workload (B=4, H=8, T=4096,
-dk=dv=128, L=1, chunk 64, bf16 I/O, fp32 state).  Inputs are device resident when timing starts;
-three input batches rotate (419 MB of inputs, more than the 126 MB L2), so every step streams its
-inputs from HBM.  Steps are replayed from CUDA graphs (one per input batch) so that host overhead
-does not leave gaps between kernels.  Timing uses CUDA events on the launching stream with a
-barrier and a synchronize on both sides; the reported time is the max over ranks.
+A step is one prism_scan_fwd call over one batch of the headline workload, by default the
+long-context one (B=1, H=16, T=65536, dk=dv=128, L=2 projected rank-L write, chunk 128, bf16 I/O,
+fp32 state, nonzero S0): the largest of the scan workloads that fit one GPU.  Inputs are device
+resident when timing starts; three input batches rotate (each larger than the 126 MB L2), so every
+step streams its inputs from HBM.  Steps are replayed from CUDA graphs (one per input batch) so
+that host overhead does not leave gaps between kernels.  Timing uses CUDA events on the launching
+stream with a barrier and a synchronize on both sides; the reported time is the max over ranks.
 
 With N > 1 (torchrun, one process per GPU) every rank processes its own batch (weak scaling: the
 B*H sequences are independent, so there is no collective in the data path).
 
 Besides the headline line's required keys the JSON line carries: roofline (HBM-bound; algorithmic
-bytes per step over the summed device time of the step's launches, each launch timed by CUDA
+bytes per call over the summed device time of the call's launches, each launch timed by CUDA
 events the library records around it, against the measured copy bandwidth), cpu_baseline (the
 fp64 oracle on a bounded sample, rank 0 at N = 1), e2e (through the public API with pinned-host
 inputs copied in and the outputs copied back inside the timed region), clocks sampled during the
-timed region, and, as secondary measurements, the decode step (B=256, H=32, d=128, L=4) and the
-two rank-L scan workloads (recsys, long).
+timed region, and, as secondary measurements: the other two chunked-scan workloads (gdn: B=4,
+H=8, T=4096, d=128, Gated-DeltaNet write; recsys: B=32, H=4, T=8192, d=64, L=4), each measured the
+same way with its own roofline and oracle baseline; the decode step (B=256, H=32, d=128, L=4); and
+the write-term producer on the two rank-L shapes.
 """
 from __future__ import annotations
 
@@ -228,15 +231,20 @@ def cpu_model():
     return "unknown"
 
 
+ORACLE_WINDOW = 4096  # tokens of each sequence the oracle baselines run over (throughput of the
+                      # token recurrence does not depend on where in the sequence a window sits)
+
+
 def cpu_oracle_sample(wl, budget_s=12.0, n_threads=None):
-    """Time the fp64 oracle on whole (b, h) sequences of the workload.  Returns (tokens/s,
-    description, threads).  One sequence is timed alone first to size a sample of about
-    `budget_s` seconds on all threads."""
+    """Time the fp64 oracle on (b, h) sequences of the workload, each over its first
+    min(T, ORACLE_WINDOW) tokens.  Returns (tokens/s, description, threads).  One sequence is
+    timed alone first to size a sample of about `budget_s` seconds on all threads."""
     import oracle
     from delta_rule_sequence_b200.workloads import make_inputs, select_heads
 
     threads = n_threads or oracle.default_threads()
-    x = make_inputs(wl, seed=0)
+    Ts = min(wl.T, ORACLE_WINDOW)
+    x = make_inputs(wl.with_(T=Ts), seed=0)
     heads_all = [(b, h) for b in range(wl.B) for h in range(wl.H)]
     sub = select_heads(x, heads_all[:1])
     t0 = time.perf_counter()
@@ -253,16 +261,17 @@ def cpu_oracle_sample(wl, budget_s=12.0, n_threads=None):
         dt = time.perf_counter() - t0
         if dt >= budget_s or passes >= 1000:
             break
-    tokens = passes * n * wl.T / wl.H  # a token carries all H heads
+    tokens = passes * n * Ts / wl.H  # a token carries all H heads
     desc = (f"{passes} pass(es) over {n} of {wl.B * wl.H} (b,h) sequences of the {wl.name} "
-            f"workload, full T={wl.T}, fp64 token recurrence on {threads} threads, {dt:.1f} s; "
-            f"tokens/s = passes*sequences*T/H/s")
+            f"workload, first {Ts} of T={wl.T} tokens each, fp64 token recurrence on {threads} "
+            f"threads, {dt:.1f} s; tokens/s = passes*sequences*tokens/H/s")
     return tokens / dt, desc, threads
 
 
 def run_reference(args, rank):
     """The base contract's reference arm: the fp64 oracle on the host cores, per step a bounded
-    sample of the same workload (a few whole (b,h) sequences, one per thread)."""
+    sample of the same workload (one (b,h) sequence per thread, over its first
+    min(T, ORACLE_WINDOW) tokens)."""
     if rank != 0:
         return
     import oracle
@@ -270,7 +279,8 @@ def run_reference(args, rank):
 
     wl = WORKLOADS[args.workload]
     threads = oracle.default_threads()
-    x = make_inputs(wl, seed=0)
+    Ts = min(wl.T, ORACLE_WINDOW)
+    x = make_inputs(wl.with_(T=Ts), seed=0)
     heads_all = [(b, h) for b in range(wl.B) for h in range(wl.H)]
     per_step = min(len(heads_all), threads)
     subs = [select_heads(x, [heads_all[(s * per_step + i) % len(heads_all)]
@@ -281,10 +291,10 @@ def run_reference(args, rank):
     for i in range(args.steps):
         oracle.scan_ref(**subs[i % 2], n_threads=threads)
     dt = time.perf_counter() - t0
-    tokens = args.steps * per_step * wl.T / wl.H
+    tokens = args.steps * per_step * Ts / wl.H
     value = tokens / dt
-    desc = (f"per step {per_step} whole (b,h) sequences (T={wl.T}) of the {wl.name} workload, "
-            f"fp64 oracle on {threads} threads")
+    desc = (f"per step {per_step} (b,h) sequences of the {wl.name} workload, first {Ts} of "
+            f"T={wl.T} tokens each, fp64 oracle on {threads} threads")
     line = {
         "impl": "reference", "metric": "scan-fwd tokens/s per layer", "value": value,
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -299,67 +309,177 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
-def time_workload(wl, dev, stream, peaks, rank, max_over_ranks, barrier, world, steps=5):
-    """One scan workload timed on its own: device-resident seeded inputs (larger than L2), one
-    warm-up call, `steps` timed calls with CUDA events around each launch (library probe)."""
-    import torch
+class ScanBench:
+    """One chunked-scan workload on one rank: three seeded input batches resident on the device
+    (rotated, so that steps stream their inputs from HBM rather than L2), one CUDA graph per batch
+    for the throughput, and the library's per-launch events for the kernel durations."""
 
-    from delta_rule_sequence_b200 import prism
-    from delta_rule_sequence_b200.workloads import make_inputs
+    def __init__(self, wl, dev, stream, rank):
+        import torch
 
-    x = {n: (None if t is None else t.to(dev)) for n, t in make_inputs(wl, seed=7 + rank).items()}
-    o = torch.empty((wl.B, wl.T, wl.H, wl.dv), dtype=wl.torch_io, device=dev)
-    S = torch.empty((wl.B, wl.H, wl.dv, wl.dk), dtype=torch.float32, device=dev)
-    shape = prism.make_shape(x["q"], x["v"], x["u"], wl.chunk)
-    ws = prism.workspace_for(shape, dev)
-    n_launch = prism.prism_scan_fwd_launch_count(shape)
+        from delta_rule_sequence_b200 import prism
+        from delta_rule_sequence_b200.workloads import make_inputs
 
-    def call():
-        prism.prism_scan_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["u"], x["w"], x["S0"],
-                             chunk=wl.chunk, o=o, S_final=S, workspace=ws, stream=stream)
+        self.wl, self.dev, self.stream = wl, dev, stream
+        self.host_sets = [make_inputs(wl, seed=3 * rank + i) for i in range(3)]
+        self.sets = [{n: (None if t is None else t.to(dev)) for n, t in s.items()}
+                     for s in self.host_sets]
+        self.o = [torch.empty((wl.B, wl.T, wl.H, wl.dv), dtype=wl.torch_io, device=dev)
+                  for _ in range(3)]
+        self.S = [torch.empty((wl.B, wl.H, wl.dv, wl.dk), dtype=torch.float32, device=dev)
+                  for _ in range(3)]
+        self.shape = prism.make_shape(self.sets[0]["q"], self.sets[0]["v"], self.sets[0]["u"],
+                                      wl.chunk)
+        self.ws = prism.workspace_for(self.shape, dev)
+        self.launches = prism.prism_scan_fwd_launch_count(self.shape)
+        self.graphs = []
 
-    with torch.cuda.stream(stream):
-        call()
-    stream.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)] for _ in range(steps)]
-    with torch.cuda.stream(stream):
-        for row in evs:
-            for e in row:
-                e.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for i in range(steps):
-            prism.record_launch_events(evs[i])
-            call()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    status = prism.prism_query_device_status(ws, stream)
-    if status != prism.PRISM_OK:
-        raise SystemExit(f"bench: device status after {wl.name}: {prism.status_string(status)}")
-    ms = max_over_ranks(e0.elapsed_time(e1)) / steps
-    launch_ms = [sum(r[j].elapsed_time(r[j + 1]) for r in evs) / steps for j in range(n_launch)]
-    kern_ms = sum(launch_ms)
-    alg = scan_bytes(wl)
-    achieved = alg / (kern_ms / 1e3) / 1e9
-    del x, o, S
+    def step(self, i, workspace=None, o=None, S=None, x=None):
+        from delta_rule_sequence_b200 import prism
+
+        x = x if x is not None else self.sets[i % 3]
+        prism.prism_scan_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["u"], x["w"],
+                             x["S0"], chunk=self.wl.chunk, o=o if o is not None else self.o[i % 3],
+                             S_final=S if S is not None else self.S[i % 3],
+                             workspace=workspace if workspace is not None else self.ws,
+                             stream=self.stream)
+
+    def capture(self):
+        import torch
+
+        with torch.cuda.stream(self.stream):
+            for i in range(3):
+                self.step(i)
+        self.stream.synchronize()
+        for i in range(3):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                self.step(i)
+            self.graphs.append(g)
+        torch.cuda.synchronize()
+
+    def check_status(self, where):
+        from delta_rule_sequence_b200 import prism
+
+        status = prism.prism_query_device_status(self.ws, self.stream)
+        if status != prism.PRISM_OK:
+            raise SystemExit(f"bench: device status {where} ({self.wl.name}): "
+                             f"{prism.status_string(status)}")
+
+    def run_graphs(self, n, start=0):
+        import torch
+
+        with torch.cuda.stream(self.stream):
+            for i in range(start, start + n):
+                self.graphs[i % 3].replay()
+
+    def timed_graphs(self, steps, barrier, max_over_ranks):
+        """Device time of `steps` graph-replayed steps: ms in total (max over ranks)."""
+        import torch
+
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(self.stream):
+            e0.record(self.stream)
+            for i in range(steps):
+                self.graphs[i % 3].replay()
+            e1.record(self.stream)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1))
+
+    def launch_times(self, steps, barrier, max_over_ranks):
+        """Average device time of each launch of a step (CUDA events the library records on the
+        launching stream around each launch), over `steps` steps launched without graphs.
+        Returns (ms per launch, ms per step of that region)."""
+        import torch
+
+        from delta_rule_sequence_b200 import prism
+
+        n = self.launches
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+        with torch.cuda.stream(self.stream):
+            for row in evs:  # record once so that every event handle exists
+                for e in row:
+                    e.record(self.stream)
+        torch.cuda.synchronize()
+        barrier()
+        p0 = torch.cuda.Event(enable_timing=True)
+        p1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.stream):
+            p0.record(self.stream)
+            for i in range(steps):
+                prism.record_launch_events(evs[i])
+                self.step(i)
+            p1.record(self.stream)
+        torch.cuda.synchronize()
+        barrier()
+        per_step = max_over_ranks(p0.elapsed_time(p1)) / steps
+        launch_ms = [max_over_ranks(sum(r[j].elapsed_time(r[j + 1]) for r in evs) / steps)
+                     for j in range(n)]
+        return launch_ms, per_step
+
+    def release(self):
+        for g in self.graphs:
+            g.reset()
+        self.graphs = []
+
+
+def scan_roofline(wl, launch_ms, peaks, peaks_kind, timing):
+    """Roofline of one scan call.  The algorithmic bytes are defined for the whole path (inputs read
+    once, outputs and the state written once), which the call's launches share, so the unit is the
+    call: algorithmic bytes per call over the summed device time of its launches."""
     names = STEP_KERNELS.get(wl.name, [])
-    if len(names) != n_launch:
-        names = [f"launch{j}" for j in range(n_launch)]
-    return {"workload": workload_config(wl)["workload"], "ms_per_call": ms,
-            "tokens_per_s": world * wl.B * wl.T / (ms / 1e3), "launches": n_launch,
-            "ms_per_launch": dict(zip(names, launch_ms)),
-            "dram_bytes_per_launch": {n: committed_traffic(wl.name, n) for n in names},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                         "algorithmic_bytes": alg, "algorithmic_flops": scan_flops(wl),
-                         "tensor_frac_algorithmic": scan_flops(wl) / (kern_ms / 1e3) / 1e12
-                         / peaks["bf16_tflops"]},
-            "steps": steps}
+    if len(names) != len(launch_ms):
+        names = [f"launch{j}" for j in range(len(launch_ms))]
+    kernels = [{"name": n, "ms_per_launch": launch_ms[j],
+                "share": launch_ms[j] / max(1e-12, sum(launch_ms)),
+                "dram_bytes_per_launch": committed_traffic(wl.name, n)}
+               for j, n in enumerate(names)]
+    dominant = max(range(len(launch_ms)), key=lambda j: launch_ms[j])
+    alg = scan_bytes(wl)
+    kern_ms = sum(launch_ms)
+    achieved = alg / (kern_ms / 1e3) / 1e9
+    traffic = [k["dram_bytes_per_launch"] for k in kernels]
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"],
+            "traffic": sum(traffic) if all(t is not None for t in traffic) else None,
+            "peak_kind": f"{peaks_kind} copy bandwidth (burst)",
+            "unit_of_work": "one call: " + " + ".join(names),
+            "dominant_kernel": names[dominant], "kernels": kernels,
+            "algorithmic_bytes_per_step": alg, "algorithmic_flops_per_step": scan_flops(wl),
+            "tensor_frac_algorithmic": scan_flops(wl) / (kern_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "timing": timing}
+
+
+def secondary_scan(wl, dev, stream, peaks, peaks_kind, rank, max_over_ranks, barrier, world,
+                   steps, warmup, cpu_budget):
+    """A scan workload measured like the headline (rotated inputs, graph-replayed steps, per-launch
+    events), with its own roofline and, on rank 0 at N = 1, its own oracle baseline."""
+    sb = ScanBench(wl, dev, stream, rank)
+    sb.capture()
+    sb.run_graphs(warmup)
+    stream.synchronize()
+    sb.check_status("after warm-up")
+    ms = sb.timed_graphs(steps, barrier, max_over_ranks) / steps
+    launch_ms, probe_ms = sb.launch_times(steps, barrier, max_over_ranks)
+    sb.check_status("after timing")
+    sb.release()
+    out = {"workload": workload_config(wl)["workload"], "ms_per_call": ms,
+           "tokens_per_s": world * wl.B * wl.T / (ms / 1e3), "launches": sb.launches,
+           "steps": steps, "warmup": warmup,
+           "roofline": scan_roofline(wl, launch_ms, peaks, peaks_kind,
+                                     f"CUDA events recorded by the library around each launch, "
+                                     f"{steps} calls without graphs ({probe_ms:.4f} ms/call there)"),
+           "cpu_baseline": None}
+    del sb
+    if rank == 0 and world == 1 and cpu_budget > 0:
+        v, desc, threads = cpu_oracle_sample(wl, budget_s=cpu_budget)
+        out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                               "sample": desc, "cpu_model": cpu_model()}
+    return out
 
 
 def time_producer(wl, dev, stream, peaks, rank, max_over_ranks, barrier, world, steps=20):
@@ -429,15 +549,17 @@ def workload_config(wl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="gdn")
+    ap.add_argument("--workload", default="long")
     ap.add_argument("--decode-steps", type=int, default=200)
-    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
-                    help="skip the secondary timing of the recsys and long workloads")
+                    help="skip the secondary scan workloads and the write producer")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override the headline workload's T (small cases for profiler captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -453,8 +575,7 @@ def main():
     import torch.distributed as dist
 
     from delta_rule_sequence_b200 import prism
-    from delta_rule_sequence_b200.workloads import (WORKLOADS, make_decode_state,
-                                                     make_decode_step, make_inputs)
+    from delta_rule_sequence_b200.workloads import WORKLOADS, make_decode_state, make_decode_step
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -475,129 +596,41 @@ def main():
 
     peaks, peaks_kind = load_peaks()
     wl = WORKLOADS[args.workload]
+    if args.seq_len > 0:
+        wl = wl.with_(T=args.seq_len)
     stream = torch.cuda.Stream(device=dev)
 
-    # ---- inputs: three seeded batches per rank, device resident
-    host_sets = [make_inputs(wl, seed=3 * rank + i) for i in range(3)]
-    sets = [{n: (None if t is None else t.to(dev)) for n, t in s.items()} for s in host_sets]
-    o_buf = [torch.empty((wl.B, wl.T, wl.H, wl.dv), dtype=wl.torch_io, device=dev) for _ in range(3)]
-    S_buf = [torch.empty((wl.B, wl.H, wl.dv, wl.dk), dtype=torch.float32, device=dev)
-             for _ in range(3)]
-    shape = prism.make_shape(sets[0]["q"], sets[0]["v"], sets[0]["u"], wl.chunk)
-    ws = prism.workspace_for(shape, dev)
-    launches_per_step = prism.prism_scan_fwd_launch_count(shape)
-
-    def step(i, s=None):
-        x = sets[i % 3]
-        prism.prism_scan_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["u"], x["w"],
-                             x["S0"], chunk=wl.chunk, o=o_buf[i % 3], S_final=S_buf[i % 3],
-                             workspace=ws, stream=s)
-
-    # ---- capture one graph per input batch
-    with torch.cuda.stream(stream):
-        for i in range(3):
-            step(i, stream)
+    # ---- the headline workload: three seeded batches per rank, device resident, one CUDA graph
+    # per batch, steps rotating over them
+    sb = ScanBench(wl, dev, stream, rank)
+    sb_launches = sb.launches
+    sb.capture()
+    sb.run_graphs(args.warmup)
     stream.synchronize()
-    graphs = []
-    for i in range(3):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            step(i, stream)
-        graphs.append(g)
-    torch.cuda.synchronize()
-
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            graphs[i % 3].replay()
-    stream.synchronize()
-    status = prism.prism_query_device_status(ws, stream)
-    if status != prism.PRISM_OK:
-        raise SystemExit(f"bench: device status after warm-up: {prism.status_string(status)}")
+    sb.check_status("after warm-up")
 
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
     sampler.start()
     time.sleep(0.3)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
     wall0 = time.time()
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        for i in range(args.steps):
-            graphs[i % 3].replay()
-        ev1.record(stream)
-    torch.cuda.synchronize()
+    ms_total = sb.timed_graphs(args.steps, barrier, max_over_ranks)
     wall1 = time.time()
-    barrier()
     sampler.stop()
-    ms_total = ev0.elapsed_time(ev1)
-    ms_total = max_over_ranks(ms_total)
     ms_per_step = ms_total / args.steps
     tokens_per_step = wl.B * wl.T
     value = world * tokens_per_step * args.steps / (ms_total / 1e3)
-    status = prism.prism_query_device_status(ws, stream)
-    if status != prism.PRISM_OK:
-        raise SystemExit(f"bench: device status after timing: {prism.status_string(status)}")
+    sb.check_status("after timing")
     clocks = sampler.summary(wall0, wall1)
 
     # ---- per-kernel durations: a second timed region of the same steps, launched without graphs,
     # with the library recording CUDA events on the launching stream around every launch
-    names = STEP_KERNELS.get(wl.name, [f"launch{j}" for j in range(launches_per_step)])
-    if len(names) != launches_per_step:
-        names = [f"launch{j}" for j in range(launches_per_step)]
-    probe_steps = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(launches_per_step + 1)]
-           for _ in range(probe_steps)]
-    with torch.cuda.stream(stream):
-        for row in evs:  # record once so that every event handle exists
-            for e in row:
-                e.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    p0 = torch.cuda.Event(enable_timing=True)
-    p1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        p0.record(stream)
-        for i in range(probe_steps):
-            prism.record_launch_events(evs[i])
-            step(i, stream)
-        p1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    probe_ms_per_step = max_over_ranks(p0.elapsed_time(p1)) / probe_steps
-    launch_ms = [max_over_ranks(sum(row[j].elapsed_time(row[j + 1]) for row in evs) / probe_steps)
-                 for j in range(launches_per_step)]
-    del evs
-    kernels = []
-    for j, n in enumerate(names):
-        kernels.append({"name": n, "ms_per_launch": launch_ms[j],
-                        "share": launch_ms[j] / max(1e-12, sum(launch_ms)),
-                        "dram_bytes_per_launch": committed_traffic(wl.name, n)})
-    dominant = max(range(launches_per_step), key=lambda j: launch_ms[j])
-
-    # Roofline.  The algorithmic bytes are defined for the whole path (inputs read once, outputs
-    # and the state written once), which the step's launches share, so the roofline unit is the
-    # step: algorithmic bytes per step over the summed device time of its launches.
-    alg_bytes = scan_bytes(wl)
-    step_kernel_ms = sum(launch_ms)
-    achieved = alg_bytes / (step_kernel_ms / 1e3) / 1e9
-    traffic = [k["dram_bytes_per_launch"] for k in kernels]
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"],
-                "traffic": sum(traffic) if all(t is not None for t in traffic) else None,
-                "peak_kind": f"{peaks_kind} copy bandwidth (burst)",
-                "unit_of_work": "one step: " + " + ".join(names),
-                "dominant_kernel": names[dominant],
-                "kernels": kernels,
-                "algorithmic_bytes_per_step": alg_bytes,
-                "algorithmic_flops_per_step": scan_flops(wl),
-                "tensor_frac_algorithmic": scan_flops(wl) / (step_kernel_ms / 1e3) / 1e12
-                / peaks["bf16_tflops"],
-                "timing": f"CUDA events recorded by the library on the launching stream around "
-                          f"each launch, {probe_steps} steps without graphs "
-                          f"({probe_ms_per_step:.4f} ms/step there)"}
+    launch_ms, probe_ms = sb.launch_times(args.steps, barrier, max_over_ranks)
+    roofline = scan_roofline(wl, launch_ms, peaks, peaks_kind,
+                             f"CUDA events recorded by the library on the launching stream around "
+                             f"each launch, {args.steps} steps without graphs "
+                             f"({probe_ms:.4f} ms/step there)")
+    sb.release()
 
     # ---- end to end through the public API: pinned host inputs in, outputs back, every step.
     # Copies in, scans and copies out run on three streams with two device buffers each (a caller
@@ -605,14 +638,14 @@ def main():
     # and step i-2's copy back; every step still moves its own inputs and results.
     e2e = None
     if args.e2e_steps > 0:
-        pinned = {n: (None if t is None else t.pin_memory()) for n, t in host_sets[0].items()}
-        o_host = torch.empty(o_buf[0].shape, dtype=o_buf[0].dtype).pin_memory()
-        S_host = torch.empty(S_buf[0].shape, dtype=torch.float32).pin_memory()
+        pinned = {n: (None if t is None else t.pin_memory()) for n, t in sb.host_sets[0].items()}
+        o_host = torch.empty(sb.o[0].shape, dtype=sb.o[0].dtype).pin_memory()
+        S_host = torch.empty(sb.S[0].shape, dtype=torch.float32).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
         d2h = o_host.numel() * o_host.element_size() + S_host.numel() * 4
         s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-        dbuf = [sets[0], sets[1]]
-        ws2 = [ws, torch.zeros_like(ws)]
+        dbuf = [sb.sets[0], sb.sets[1]]
+        ws2 = [sb.ws, torch.zeros_like(sb.ws)]
         n_e2e = args.e2e_steps
 
         def run_e2e(nsteps):
@@ -632,14 +665,12 @@ def main():
                     stream.wait_event(ev_in[i])
                     if i >= 2:
                         stream.wait_event(ev_out[i - 2])  # the copy back of this output is done
-                    prism.prism_scan_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["u"],
-                                         x["w"], x["S0"], chunk=wl.chunk, o=o_buf[bi],
-                                         S_final=S_buf[bi], workspace=ws2[bi], stream=stream)
+                    sb.step(bi, workspace=ws2[bi], o=sb.o[bi], S=sb.S[bi], x=x)
                     ev_cmp[i].record(stream)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(ev_cmp[i])
-                    o_host.copy_(o_buf[bi], non_blocking=True)
-                    S_host.copy_(S_buf[bi], non_blocking=True)
+                    o_host.copy_(sb.o[bi], non_blocking=True)
+                    S_host.copy_(sb.S[bi], non_blocking=True)
                     ev_out[i].record(s_out)
             return ev_out[-1]
 
@@ -657,10 +688,24 @@ def main():
         torch.cuda.synchronize()
         barrier()
         ems = max_over_ranks(e0.elapsed_time(e1))
+        sb.check_status("after the end-to-end run")
         e2e = {"value": world * tokens_per_step * n_e2e / (ems / 1e3),
                "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": n_e2e, "ms_per_step": ems / n_e2e,
                "schedule": "copy in / scan / copy out on three streams, two buffers each"}
+        del pinned, o_host, S_host, ws2, dbuf
+    del sb
+
+    # ---- secondary: the other chunked-scan workloads, measured the same way
+    others = {}
+    if not args.no_configs:
+        for name in ("gdn", "recsys", "long"):
+            if name == args.workload:
+                continue
+            others[name] = secondary_scan(
+                WORKLOADS[name], dev, stream, peaks, peaks_kind, rank, max_over_ranks, barrier,
+                world, steps=max(20, min(args.steps, 200)), warmup=args.warmup,
+                cpu_budget=0.0 if args.no_cpu_baseline else 6.0)
 
     # ---- secondary: the decode step (B=256, H=32, d=128, L=4), state in HBM, in place
     decode = None
@@ -671,6 +716,7 @@ def main():
         pool = [{n: (None if t is None else t.to(dev)) for n, t in
                  make_decode_step(dwl, st, s, seed=rank).items()} for s in range(4)]
         o_d = torch.empty((dwl.B, 1, dwl.H, dwl.dv), dtype=torch.bfloat16, device=dev)
+
         def dstep(i):
             x = pool[i % 4]
             prism.prism_step_decode(x["q"], x["k"], None, x["alpha"], x["beta"], x["u"], x["w"],
@@ -689,6 +735,8 @@ def main():
             d1.record(stream)
         torch.cuda.synchronize()
         barrier()
+        if prism.prism_query_device_status(None, stream) != prism.PRISM_OK:
+            raise SystemExit("bench: device status after the decode steps")
         dms = max_over_ranks(d0.elapsed_time(d1)) / args.decode_steps
         db = decode_bytes(dwl)
         decode = {"workload": "decode: B=256 H=32 dk=dv=128 L=4 bf16 I/O, fp32 state in place",
@@ -698,14 +746,11 @@ def main():
                   "frac_of_8tbs": db / (dms / 1e3) / 1e9 / 8000.0,
                   "bytes_per_step": db, "steps": args.decode_steps,
                   "inputs": "4 seeded step batches cycled; state carried across steps"}
+        del S, pool, o_d
 
-    # ---- secondary: the other scan workloads (rank-L writes), each timed alone on its own inputs
-    others = {}
+    # ---- secondary: the write-term producer on the two rank-L shapes
     if not args.no_configs:
         for name in ("recsys", "long"):
-            others[name] = time_workload(WORKLOADS[name], dev, stream, peaks, rank, max_over_ranks,
-                                         barrier, world)
-        for name in ("recsys", "long"):  # the write-term producer on the same shapes
             others["producer_" + name] = time_producer(WORKLOADS[name], dev, stream, peaks, rank,
                                                        max_over_ranks, barrier, world)
 
@@ -715,8 +760,6 @@ def main():
         cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc,
                "cpu_model": cpu_model()}
 
-    for g in graphs:
-        g.reset()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -729,7 +772,7 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_config(wl), parallelism=f"dp{world} over (b,h) sequences"),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps, "clocks": clocks, "decode": decode,
+        "gpu_launches": sb_launches * args.steps, "clocks": clocks, "decode": decode,
         "other_workloads": others or None,
     }
     print(json.dumps(line), flush=True)

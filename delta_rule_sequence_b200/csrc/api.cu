@@ -24,6 +24,11 @@ cudaError_t launch_segment_element(const ScanArgs &a, int route, bool io_f32, vo
                                    float *f_out, cudaStream_t s);
 cudaError_t launch_state_fold(int BH, int dk, int dv, const float *S_in, const float *E, const float *f,
                               float *S_out, cudaStream_t s);
+cudaError_t noalloc_status(uint32_t *out);
+size_t bwd_workspace_bytes(int B, int H, int T, int dk, int dv);
+cudaError_t launch_scan_bwd(const ScanArgs &f, const void *dO, const float *dS_final, float *dq,
+                            float *dk, float *dv, float *dalpha, float *dbeta, float *du, float *dw,
+                            float *dS0, void *ws, bool io_f32, cudaStream_t s);
 }  // namespace prism
 
 namespace {
@@ -105,8 +110,12 @@ int route_of(Plan p) {
 }
 
 // Debug flag bits (prism_debug_set_flags): 2 = take the segmented scan whenever the shape allows
-// it, 4 = never take it, 8 = the stall test of the Gated-DeltaNet state kernel (its waits give up).
-constexpr int kForceSegments = 2, kNoSegments = 4, kDebugStall = 8;
+// it, 4 = never take it, 8 = the stall test of the Gated-DeltaNet state kernel (its waits give up),
+// 16 = the state kernel's Wk_lo term from the first chunk on, whatever the size of the state,
+// 32 = the stall test of the per-chunk prep kernels, 64 = of the write producer, 128 = of the
+// bulk-copy decode kernel.
+constexpr int kForceSegments = 2, kNoSegments = 4, kDebugStall = 8, kDebugForceWkLo = 16,
+              kDebugStallPrep = 32, kDebugStallProducer = 64, kDebugStallDecode = 128;
 
 // Number of segments G of the segmented inter-chunk scan (1 = one in-order pass per sequence).
 // It needs dk == dv (the identity pass) and T divisible by G with at least one chunk per segment.
@@ -163,6 +172,21 @@ prism::ScanArgs make_args(const prism_shape *s, const void *q, const void *k, co
 }  // namespace
 
 namespace prism {
+// Every check of a prism_scan_fwd call that does not involve the workspace (prism_scan_fwd_noalloc
+// runs these before it sizes anything).
+prism_status check_scan_call(const prism_shape *shape, const void *q, const void *k, const void *v,
+                             const float *alpha, const float *beta, const void *u, const void *w,
+                             const float *S0, const void *o, const float *S_final) {
+    prism_status st = check_common(shape, q, k, v, alpha, beta, u, w);
+    if (st != PRISM_OK) return st;
+    if (shape->chunk != 64 && shape->chunk != 128) return PRISM_ERR_INVALID_ARG;
+    if ((S0 && !aligned16(S0)) || (S_final && !aligned16(S_final))) return PRISM_ERR_INVALID_ARG;
+    const long long work = (long long)shape->B * shape->H * shape->T;
+    if (work > 0 && (!o || !aligned16(o))) return PRISM_ERR_INVALID_ARG;
+    if (o && (o == q || o == k || o == v || o == u || o == w)) return PRISM_ERR_INVALID_ARG;
+    return PRISM_OK;
+}
+
 void launch_probe_mark(cudaStream_t s) {
     LaunchProbe &p = t_probe;
     if (p.next < p.n) cudaEventRecord((cudaEvent_t)p.events[p.next++], s);
@@ -209,16 +233,11 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
                             const void *v, const float *alpha, const float *beta,
                             const void *u, const void *w, const float *S0, void *o,
                             float *S_final, void *workspace, size_t ws_bytes, void *stream) {
-    prism_status st = check_common(shape, q, k, v, alpha, beta, u, w);
+    prism_status st = prism::check_scan_call(shape, q, k, v, alpha, beta, u, w, S0, o, S_final);
     if (st != PRISM_OK) return st;
-    if (shape->chunk != 64 && shape->chunk != 128) return PRISM_ERR_INVALID_ARG;
     size_t need = 0;
     prism_scan_fwd_workspace_size(shape, &need);
     if (!workspace || ws_bytes < need || ((uintptr_t)workspace & 255u)) return PRISM_ERR_INVALID_ARG;
-    if ((S0 && !aligned16(S0)) || (S_final && !aligned16(S_final))) return PRISM_ERR_INVALID_ARG;
-    const long long work = (long long)shape->B * shape->H * shape->T;
-    if (work > 0 && (!o || !aligned16(o))) return PRISM_ERR_INVALID_ARG;
-    if (o && (o == q || o == k || o == v || o == u || o == w)) return PRISM_ERR_INVALID_ARG;
 
     cudaStream_t s = (cudaStream_t)stream;
     uint32_t *status = (uint32_t *)workspace;
@@ -227,6 +246,8 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
 
     prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, S0, o, S_final, status);
     if (g_debug_flags & kDebugStall) a.flags |= prism::kStallTest;
+    if (g_debug_flags & kDebugForceWkLo) a.flags |= prism::kForceWkLo;
+    if (g_debug_flags & kDebugStallPrep) a.flags |= prism::kStallPrep;
     const bool io_f32 = shape->io == PRISM_F32;
     cudaError_t err;
     const Plan plan = plan_for(shape, u == nullptr);
@@ -261,6 +282,7 @@ prism_status prism_scan_segment_element(const prism_shape *shape, const void *q,
     cudaStream_t s = (cudaStream_t)stream;
     prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, nullptr, nullptr, nullptr,
                                   (uint32_t *)workspace);
+    if (g_debug_flags & kDebugForceWkLo) a.flags |= prism::kForceWkLo;
     const Plan plan = plan_for(shape, u == nullptr);
     cudaError_t err = prism::launch_segment_element(a, route_of(plan), shape->io == PRISM_F32, workspace, E, f, s);
     probe_finish(s);
@@ -282,6 +304,56 @@ prism_status prism_state_fold(int BH, int dk, int dv, const float *S_in, const f
     return cuda_status(err);
 }
 
+prism_status prism_scan_bwd_workspace_size(const prism_shape *shape, size_t *bytes) {
+    if (!shape || !bytes) return PRISM_ERR_INVALID_ARG;
+    const prism_shape &s = *shape;
+    if (s.B < 0 || s.H < 0 || s.T < 0 || !width_ok(s.dk) || !width_ok(s.dv)) return PRISM_ERR_INVALID_ARG;
+    *bytes = prism::bwd_workspace_bytes(s.B, s.H, s.T, s.dk, s.dv);
+    return PRISM_OK;
+}
+
+prism_status prism_scan_bwd(const prism_shape *shape, const void *q, const void *k, const void *v,
+                            const float *alpha, const float *beta, const void *u, const void *w,
+                            const float *S0, const void *dO, const float *dS_final, float *dq,
+                            float *dk, float *dv, float *dalpha, float *dbeta, float *du, float *dw,
+                            float *dS0, void *workspace, size_t ws_bytes, void *stream) {
+    prism_status st = check_common(shape, q, k, v, alpha, beta, u, w);
+    if (st != PRISM_OK) return st;
+    if (shape->B == 0 || shape->H == 0) return PRISM_OK;
+    size_t need = 0;
+    prism_scan_bwd_workspace_size(shape, &need);
+    if (!workspace || ws_bytes < need || ((uintptr_t)workspace & 255u)) return PRISM_ERR_INVALID_ARG;
+    if ((S0 && !aligned16(S0)) || (dS_final && !aligned16(dS_final)) || (dS0 && !aligned16(dS0)))
+        return PRISM_ERR_INVALID_ARG;
+    const bool gdn = u == nullptr;
+    if (shape->T > 0) {
+        if (!dO || !aligned16(dO)) return PRISM_ERR_INVALID_ARG;
+        for (const float *g : {dq, dk, dalpha, dbeta})
+            if (!g || ((uintptr_t)g & 15u)) return PRISM_ERR_INVALID_ARG;
+        if (gdn && (!dv || !aligned16(dv))) return PRISM_ERR_INVALID_ARG;
+        if (!gdn && (!du || !dw || !aligned16(du) || !aligned16(dw))) return PRISM_ERR_INVALID_ARG;
+        // no gradient may overlap another one or an input
+        const void *outs[] = {dq, dk, gdn ? dv : nullptr, dalpha, dbeta, gdn ? nullptr : du,
+                              gdn ? nullptr : dw, dS0};
+        const void *ins[] = {q, k, v, alpha, beta, u, w, S0, dO, dS_final};
+        for (int i = 0; i < 8; ++i) {
+            if (!outs[i]) continue;
+            for (int j = i + 1; j < 8; ++j)
+                if (outs[i] == outs[j]) return PRISM_ERR_INVALID_ARG;
+            for (const void *in : ins)
+                if (in && in == outs[i]) return PRISM_ERR_INVALID_ARG;
+        }
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, S0, nullptr, nullptr,
+                                  (uint32_t *)workspace);
+    cudaError_t err = prism::launch_scan_bwd(a, dO, dS_final, dq, dk, gdn ? dv : nullptr, dalpha, dbeta,
+                                             gdn ? nullptr : du, gdn ? nullptr : dw, dS0, workspace,
+                                             shape->io == PRISM_F32, s);
+    probe_finish(s);
+    return cuda_status(err);
+}
+
 prism_status prism_step_decode(const prism_shape *shape, const void *q, const void *k,
                                const void *v, const float *alpha, const float *beta,
                                const void *u, const void *w, float *S, void *o, void *stream) {
@@ -293,6 +365,7 @@ prism_status prism_step_decode(const prism_shape *shape, const void *q, const vo
     if (!S || !aligned16(S) || !o || !aligned16(o)) return PRISM_ERR_INVALID_ARG;
     if ((long long)shape->B * shape->H > 0x7fffffffLL) return PRISM_ERR_UNSUPPORTED;
     prism::ScanArgs a = make_args(shape, q, k, v, alpha, beta, u, w, nullptr, o, S, nullptr);
+    if (g_debug_flags & kDebugStallDecode) a.flags |= prism::kStallDecode;
     cudaError_t err = prism::launch_decode(a, shape->io == PRISM_F32, (cudaStream_t)stream);
     probe_finish((cudaStream_t)stream);
     return cuda_status(err);
@@ -315,7 +388,8 @@ prism_status prism_write_producer(const prism_shape *shape, const void *x, const
     for (const void *in : {x, v, (const void *)conv, Wk, Wp, (const void *)beta})
         if (in == u || in == w) return PRISM_ERR_INVALID_ARG;  // outputs alias an input
     if (u == w) return PRISM_ERR_INVALID_ARG;
-    prism::ProducerArgs a{s.B, s.H, s.T, s.dk, s.L, x, v, conv, Wk, Wp, beta, u, w};
+    prism::ProducerArgs a{s.B, s.H, s.T, s.dk, s.L, x, v, conv, Wk, Wp, beta, u, w,
+                          (g_debug_flags & kDebugStallProducer) ? 1 : 0};
     cudaError_t err = prism::launch_write_producer(a, (cudaStream_t)stream);
     probe_finish((cudaStream_t)stream);
     return cuda_status(err);
@@ -332,11 +406,13 @@ prism_status prism_query_device_status(void *workspace, void *stream) {
         if (word != PRISM_OK && (err = cudaMemset(workspace, 0, sizeof word)) != cudaSuccess)
             return cuda_status(err);
     }
-    uint32_t dword = 0, pword = 0;
+    uint32_t dword = 0, pword = 0, nword = 0;
     if ((err = prism::decode_status(&dword)) != cudaSuccess) return cuda_status(err);
     if ((err = prism::producer_status(&pword)) != cudaSuccess) return cuda_status(err);
+    if ((err = prism::noalloc_status(&nword)) != cudaSuccess) return cuda_status(err);
     if (word == PRISM_OK) word = dword;
     if (word == PRISM_OK) word = pword;
+    if (word == PRISM_OK) word = nword;
     return (prism_status)word;
 }
 

@@ -25,8 +25,12 @@ struct ScanArgs {
 // Flags of a scan pass.  kNoWrite: the write term is zero (u = 0 / v = 0);  kS0Identity: the entry
 // state's row r is the unit vector e_r (requires dk == dv), so S_final returns the pass's affine
 // map E;  kNoOutput: o is not written;  kStallTest: the Gated-DeltaNet state kernel's load warp
-// issues nothing and every wait gives up after a short limit (a test of the give-up path).
-enum : int { kNoWrite = 1, kS0Identity = 2, kNoOutput = 4, kStallTest = 8 };
+// issues nothing and every wait gives up after a short limit (a test of the give-up path);
+// kForceWkLo: the state kernel adds the Wk_lo term from the first chunk, whatever the state's size;
+// kStallPrep, kStallDecode: the same give-up test for the per-chunk prep kernels (their tile loads
+// are not issued) and for the bulk-copy decode kernel (its state copies are not issued).
+enum : int { kNoWrite = 1, kS0Identity = 2, kNoOutput = 4, kStallTest = 8, kForceWkLo = 16,
+             kStallPrep = 32, kStallDecode = 64 };
 
 // Poll limits of the bounded mbarrier waits: normal operation, and the stall test.
 constexpr uint32_t kWaitPolls = 1u << 24;

@@ -9,11 +9,17 @@
 // associative).  The state is read once and written once; everything else is a few KB per head.
 //
 // Layout: one CTA (8 warps) per head; a warp owns blocks of 8 consecutive rows; a lane holds
-// dk/32 consecutive columns (a 16-byte vector at dk = 128).  All 8 rows of a block are loaded
-// before any is reduced so that every SM keeps enough bytes in flight to saturate HBM.  The state
-// is streamed (evict-first loads and stores): it is far larger than L2 and touched once per step.
+// dk/32 consecutive columns (a 16-byte vector at dk = 128).  The state is streamed: it is far
+// larger than L2 and touched once per step.
+//
+// Two variants.  `decode_bulk_kernel` (dk = 128, dv = 64 or 128) copies the head's whole state
+// into shared memory with four bulk copies (cp.async.bulk, one mbarrier each) issued before
+// anything else, so that the bytes in flight per SM are set by shared memory (three CTAs, up to
+// 192 KB) rather than by registers; each warp starts on its rows as soon as their quarter has
+// landed and stores the new rows with evict-first stores.  `decode_kernel` (every other shape)
+// loads 8 rows per warp into registers (evict-first) before reducing any of them.
 
-#include "common.cuh"
+#include "tc.cuh"
 
 namespace prism {
 namespace {
@@ -78,24 +84,193 @@ __device__ __forceinline__ float rows8_reduce_scatter(const float (&x)[ROWS_IN_F
     return r;
 }
 
+// Library status word of the decode kernels (a bounded wait that gave up), read and cleared by
+// prism_query_device_status.
+__device__ uint32_t g_decode_status;
+
+// The per-head prologue shared by both variants: k, q in registers; w_l (or k) and u_{l,r} (or
+// beta v_r) in shared memory; k.q; the w_l.q in shared memory.
+template <typename IO, int DK, int LW>
+struct DecodeHead {
+    float kq[DK / 32], qv[DK / 32];
+    float kdotq;
+};
+
+template <typename IO, int DK, int LW>
+__device__ __forceinline__ void decode_prologue(const ScanArgs &p, int head, float (&s_u)[LW][128],
+                                                float (&s_w)[LW][DK], float (&s_wq)[LW],
+                                                DecodeHead<IO, DK, LW> &hd) {
+    constexpr int PER = DK / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int dv = p.dv, L = p.L;
+    const bool gdn = (p.u == nullptr);
+    const IO *q = (const IO *)p.q, *k = (const IO *)p.k, *v = (const IO *)p.v;
+    const IO *u = (const IO *)p.u, *w = (const IO *)p.w;
+    const float be = p.beta[head];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        size_t idx = (size_t)head * DK + lane * PER + i;
+        hd.kq[i] = ld_io(k, idx);
+        hd.qv[i] = ld_io(q, idx);
+    }
+    for (int e = threadIdx.x; e < LW * DK; e += NT) {
+        int l = e / DK, j = e % DK;
+        s_w[l][j] = gdn ? ld_io(k, (size_t)head * DK + j) : ld_io(w, ((size_t)head * L + l) * DK + j);
+    }
+    for (int e = threadIdx.x; e < LW * dv; e += NT) {
+        int l = e / dv, r = e % dv;
+        s_u[l][r] = gdn ? be * ld_io(v, (size_t)head * dv + r) : ld_io(u, ((size_t)head * L + l) * dv + r);
+    }
+    float kdotq = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) kdotq = fmaf(hd.kq[i], hd.qv[i], kdotq);
+    hd.kdotq = warp_sum(kdotq);
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+        for (int l = 0; l < LW; ++l) {
+            float t = 0.f;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) t = fmaf(s_w[l][lane * PER + i], hd.qv[i], t);
+            t = warp_sum(t);
+            if (lane == 0) s_wq[l] = t;
+        }
+    }
+    __syncthreads();
+}
+
+// One block of 8 rows r0 .. r0 + 7 held in registers (s[j] = row r0 + j, this lane's columns):
+// the output o_r and the new rows, stored with evict-first stores.
+template <typename IO, int DK, int LW>
+__device__ __forceinline__ void decode_rows8(const ScanArgs &p, int head, int r0,
+                                             float (&s)[ROWS_IN_FLIGHT][DK / 32],
+                                             const float (&s_u)[LW][128], const float (&s_w)[LW][DK],
+                                             const float (&s_wq)[LW], const DecodeHead<IO, DK, LW> &hd) {
+    constexpr int PER = DK / 32;
+    const int lane = threadIdx.x & 31;
+    const float a = p.alpha[head];
+    const float ab = a * p.beta[head];
+    IO *o = (IO *)p.o + (size_t)head * p.dv;
+    float *S = p.S_final + (size_t)head * p.dv * DK;
+    const int my_row = lane >> 2;  // the row of the block whose sums this lane ends up holding
+    // e_r = s_r . k and p_r = s_r . q for the 8 rows: per-lane partials, then one butterfly
+    float ep[ROWS_IN_FLIGHT], pp[ROWS_IN_FLIGHT];
+#pragma unroll
+    for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
+        float e = 0.f, pq = 0.f;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            e = fmaf(s[j][i], hd.kq[i], e);
+            pq = fmaf(s[j][i], hd.qv[i], pq);
+        }
+        ep[j] = e;
+        pp[j] = pq;
+    }
+    const float e_mine = rows8_reduce_scatter(ep, lane);
+    const float p_mine = rows8_reduce_scatter(pp, lane);
+    // o_r = alpha p_r - alpha beta e_r (k.q) + sum_l u_{l,r} (w_l.q), by lane 4 r
+    if ((lane & 3) == 0) {
+        const int r = r0 + my_row;
+        float outv = a * p_mine - ab * e_mine * hd.kdotq;
+#pragma unroll
+        for (int l = 0; l < LW; ++l) outv = fmaf(s_u[l][r], s_wq[l], outv);
+        st_io(o, r, outv);
+    }
+    // s_r <- alpha s_r - alpha beta e_r k + sum_l u_{l,r} w_l
+#pragma unroll
+    for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
+        const float ej = __shfl_sync(0xffffffffu, e_mine, 4 * j);
+#pragma unroll
+        for (int i = 0; i < PER; ++i) s[j][i] = fmaf(a, s[j][i], -ab * ej * hd.kq[i]);
+    }
+#pragma unroll
+    for (int l = 0; l < LW; ++l) {
+        float wv[PER];
+        vload_shared<PER>(&s_w[l][lane * PER], wv);
+        const float4 u0 = *reinterpret_cast<const float4 *>(&s_u[l][r0]);
+        const float4 u1 = *reinterpret_cast<const float4 *>(&s_u[l][r0 + 4]);
+        const float uu[ROWS_IN_FLIGHT] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
+#pragma unroll
+            for (int i = 0; i < PER; ++i) s[j][i] = fmaf(uu[j], wv[i], s[j][i]);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < ROWS_IN_FLIGHT; ++j) vstore<PER>(S + (size_t)(r0 + j) * DK + lane * PER, s[j]);
+}
+
+// dk = 128, dv = DV in {64, 128}: the head's state arrives in shared memory by four bulk copies;
+// warps 2c and 2c + 1 take quarter c (DV / 8 rows each, in blocks of 8).
+constexpr int kDecodePieces = 4;
+
+template <typename IO, int DV, int LW>
+__global__ void __launch_bounds__(NT, 3) decode_bulk_kernel(ScanArgs p) {
+    constexpr int DK = 128, PER = DK / 32;
+    constexpr int RP = DV / kDecodePieces;       // rows per piece
+    constexpr int RW = RP / 2;                   // rows per warp
+    static_assert(RW % ROWS_IN_FLIGHT == 0, "a warp's rows come in blocks of 8");
+    constexpr uint32_t PIECE_BYTES = RP * DK * 4;
+    extern __shared__ __align__(128) float sS[];  // [DV][DK]
+    __shared__ uint64_t bar[kDecodePieces];
+    __shared__ __align__(16) float s_u[LW][128];
+    __shared__ __align__(16) float s_w[LW][DK];
+    __shared__ float s_wq[LW];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int head = blockIdx.x;
+    const float *S = p.S_final + (size_t)head * DV * DK;
+    // the give-up test: the copies are not issued and the waits run out after a short limit
+    const bool stall = (p.flags & kStallDecode) != 0;
+    const uint32_t lim = stall ? kStallTestPolls : kWaitPolls;
+
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int c = 0; c < kDecodePieces; ++c) tc::mbar_init(&bar[c], 1);
+        tc::mbar_fence_init();
+        if (!stall) {
+#pragma unroll
+            for (int c = 0; c < kDecodePieces; ++c) {
+                tc::mbar_expect_tx(&bar[c], PIECE_BYTES);
+                tc::bulk_g2s(sS + (size_t)c * RP * DK, S + (size_t)c * RP * DK, PIECE_BYTES, &bar[c]);
+            }
+        }
+    }
+    DecodeHead<IO, DK, LW> hd;
+    decode_prologue<IO, DK, LW>(p, head, s_u, s_w, s_wq, hd);  // ends with a CTA barrier
+
+    const int piece = warp >> 1;
+    const bool landed = tc::mbar_wait(&bar[piece], 0, &g_decode_status, lim);
+    if (landed) {
+        for (int rb = 0; rb < RW; rb += ROWS_IN_FLIGHT) {
+            const int r0 = piece * RP + (warp & 1) * RW + rb;
+            float s[ROWS_IN_FLIGHT][PER];
+#pragma unroll
+            for (int j = 0; j < ROWS_IN_FLIGHT; ++j)
+                vload_shared<PER>(sS + (size_t)(r0 + j) * DK + lane * PER, s[j]);
+            decode_rows8<IO, DK, LW>(p, head, r0, s, s_u, s_w, s_wq, hd);
+        }
+    }
+    // every copy has landed before the CTA's shared memory is released (bounded)
+    if (threadIdx.x == 0 && !stall) {
+#pragma unroll
+        for (int c = 0; c < kDecodePieces; ++c) tc::mbar_wait(&bar[c], 0, nullptr);
+    }
+}
+
 // LW = number of write terms (L, or 1 for the Gated-DeltaNet write beta v k^T).
 template <typename IO, int DK, int LW>
 __global__ void __launch_bounds__(NT, 3) decode_kernel(ScanArgs p) {
     constexpr int PER = DK / 32;  // columns per lane
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int head = blockIdx.x;  // b * H + h
-    const int dv = p.dv, L = p.L;
-    const bool gdn = (p.u == nullptr);
-    const IO *q = (const IO *)p.q, *k = (const IO *)p.k, *v = (const IO *)p.v;
-    const IO *u = (const IO *)p.u, *w = (const IO *)p.w;
-
+    const int dv = p.dv;
     __shared__ __align__(16) float s_u[LW][128];  // u_{l,r} (or beta v_r)
     __shared__ __align__(16) float s_w[LW][DK];   // w_l (or k)
     __shared__ float s_wq[LW];
 
     // Issue the loads of this warp's first block of state rows before the per-head prologue,
     // so that their latency overlaps the prologue's.
-    float *S = p.S_final + (size_t)head * dv * DK;  // in place
+    const float *S = p.S_final + (size_t)head * dv * DK;  // in place
     float s[ROWS_IN_FLIGHT][PER];
     int r0 = warp * ROWS_IN_FLIGHT;
     if (r0 < dv) {
@@ -103,104 +278,31 @@ __global__ void __launch_bounds__(NT, 3) decode_kernel(ScanArgs p) {
         for (int j = 0; j < ROWS_IN_FLIGHT; ++j)
             vload<PER>(S + (size_t)(r0 + j) * DK + lane * PER, s[j]);
     }
-
-    const float a = p.alpha[head];
-    const float be = p.beta[head];
-    float kq[PER], qv[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        size_t idx = (size_t)head * DK + lane * PER + i;
-        kq[i] = ld_io(k, idx);
-        qv[i] = ld_io(q, idx);
-    }
-    for (int e = threadIdx.x; e < LW * DK; e += NT) {
-        int l = e / DK, j = e % DK;
-        s_w[l][j] = gdn ? ld_io(k, (size_t)head * DK + j)
-                        : ld_io(w, ((size_t)head * L + l) * DK + j);
-    }
-    for (int e = threadIdx.x; e < LW * dv; e += NT) {
-        int l = e / dv, r = e % dv;
-        s_u[l][r] = gdn ? be * ld_io(v, (size_t)head * dv + r)
-                        : ld_io(u, ((size_t)head * L + l) * dv + r);
-    }
-    // k.q in every warp; warp 0 publishes the w_l.q
-    float kdotq = 0.f;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) kdotq = fmaf(kq[i], qv[i], kdotq);
-    kdotq = warp_sum(kdotq);
-    __syncthreads();
-    if (warp == 0) {
-#pragma unroll
-        for (int l = 0; l < LW; ++l) {
-            float t = 0.f;
-#pragma unroll
-            for (int i = 0; i < PER; ++i) t = fmaf(s_w[l][lane * PER + i], qv[i], t);
-            t = warp_sum(t);
-            if (lane == 0) s_wq[l] = t;
-        }
-    }
-    __syncthreads();
-
-    IO *o = (IO *)p.o + (size_t)head * dv;
-    const float ab = a * be;
-    const int my_row = lane >> 2;  // the row of the block whose sums this lane ends up holding
-
+    DecodeHead<IO, DK, LW> hd;
+    decode_prologue<IO, DK, LW>(p, head, s_u, s_w, s_wq, hd);
     for (; r0 < dv; r0 += NW * ROWS_IN_FLIGHT) {
         if (r0 != warp * ROWS_IN_FLIGHT) {
 #pragma unroll
             for (int j = 0; j < ROWS_IN_FLIGHT; ++j)
                 vload<PER>(S + (size_t)(r0 + j) * DK + lane * PER, s[j]);
         }
-        // e_r = s_r . k and p_r = s_r . q for the 8 rows: per-lane partials, then one butterfly
-        float ep[ROWS_IN_FLIGHT], pp[ROWS_IN_FLIGHT];
-#pragma unroll
-        for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
-            float e = 0.f, pq = 0.f;
-#pragma unroll
-            for (int i = 0; i < PER; ++i) {
-                e = fmaf(s[j][i], kq[i], e);
-                pq = fmaf(s[j][i], qv[i], pq);
-            }
-            ep[j] = e;
-            pp[j] = pq;
-        }
-        const float e_mine = rows8_reduce_scatter(ep, lane);
-        const float p_mine = rows8_reduce_scatter(pp, lane);
-        // o_r = alpha p_r - alpha beta e_r (k.q) + sum_l u_{l,r} (w_l.q), by lane 4 r
-        if ((lane & 3) == 0) {
-            const int r = r0 + my_row;
-            float outv = a * p_mine - ab * e_mine * kdotq;
-#pragma unroll
-            for (int l = 0; l < LW; ++l) outv = fmaf(s_u[l][r], s_wq[l], outv);
-            st_io(o, r, outv);
-        }
-        // s_r <- alpha s_r - alpha beta e_r k + sum_l u_{l,r} w_l
-#pragma unroll
-        for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
-            const float ej = __shfl_sync(0xffffffffu, e_mine, 4 * j);
-#pragma unroll
-            for (int i = 0; i < PER; ++i) s[j][i] = fmaf(a, s[j][i], -ab * ej * kq[i]);
-        }
-#pragma unroll
-        for (int l = 0; l < LW; ++l) {
-            float wv[PER];
-            vload_shared<PER>(&s_w[l][lane * PER], wv);
-            const float4 u0 = *reinterpret_cast<const float4 *>(&s_u[l][r0]);
-            const float4 u1 = *reinterpret_cast<const float4 *>(&s_u[l][r0 + 4]);
-            const float uu[ROWS_IN_FLIGHT] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-            for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
-#pragma unroll
-                for (int i = 0; i < PER; ++i) s[j][i] = fmaf(uu[j], wv[i], s[j][i]);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < ROWS_IN_FLIGHT; ++j) vstore<PER>(S + (size_t)(r0 + j) * DK + lane * PER, s[j]);
+        decode_rows8<IO, DK, LW>(p, head, r0, s, s_u, s_w, s_wq, hd);
     }
 }
 
 template <typename IO, int DK, int LW>
 cudaError_t launch_decode_l(const ScanArgs &a, cudaStream_t s) {
+    if constexpr (DK == 128) {
+        if (a.dv == 128 || a.dv == 64) {
+            auto kern = a.dv == 128 ? decode_bulk_kernel<IO, 128, LW> : decode_bulk_kernel<IO, 64, LW>;
+            const int bytes = a.dv * DK * 4;
+            cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+            if (err != cudaSuccess) return err;
+            launch_probe_mark(s);
+            kern<<<a.B * a.H, NT, bytes, s>>>(a);
+            return cudaGetLastError();
+        }
+    }
     launch_probe_mark(s);
     decode_kernel<IO, DK, LW><<<a.B * a.H, NT, 0, s>>>(a);
     return cudaGetLastError();
@@ -243,9 +345,16 @@ cudaError_t launch_decode(const ScanArgs &a, bool io_f32, cudaStream_t s) {
     return cudaErrorInvalidValue;
 }
 
-// The decode kernel has no waits: its status is always PRISM_OK.
+// Read and clear the decode kernels' status word (PRISM_ERR_TIMEOUT if a bulk copy's wait gave up).
 cudaError_t decode_status(uint32_t *out) {
-    *out = PRISM_OK;
+    uint32_t word = 0;
+    cudaError_t err = cudaMemcpyFromSymbol(&word, g_decode_status, sizeof word);
+    if (err != cudaSuccess) return err;
+    if (word != 0) {
+        const uint32_t zero = 0;
+        if ((err = cudaMemcpyToSymbol(g_decode_status, &zero, sizeof zero)) != cudaSuccess) return err;
+    }
+    *out = word;
     return cudaSuccess;
 }
 

@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(P_THREADS, D == 64 ? 2 : 1) write_producer_ker
     const int T = p.T, H = p.H, L = p.L;
     const uint32_t sb = smem_u32(sm);
     uint32_t *status = &g_producer_status;
+    const uint32_t lim = p.stall ? kStallTestPolls : kWaitPolls;
 
     if (warp == P_EPI) tmem_alloc(&tmem_base_sh, LY::TCOLS);
     if (tid == 0) {
@@ -114,8 +115,9 @@ __global__ void __launch_bounds__(P_THREADS, D == 64 ? 2 : 1) write_producer_ker
                 }
             };
             int issued = 0;
-            for (; issued < L && issued < 2; ++issued) load_w(issued);
-            bool ok = mbar_wait(&a_ready, 0, status);
+            if (!p.stall)
+                for (; issued < L && issued < 2; ++issued) load_w(issued);
+            bool ok = mbar_wait(&a_ready, 0, status, lim);
             const uint32_t id = idesc_bf16(128, 2 * D, 0, 0);
             auto oa = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::A_BLK); };
             auto ow = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::W_BLK); };
@@ -123,9 +125,9 @@ __global__ void __launch_bounds__(P_THREADS, D == 64 ? 2 : 1) write_producer_ker
             const uint64_t dAl = make_desc(sb + LY::A_LO, 16, 1024, 2);
             for (int l = 0; l < L && ok; ++l) {
                 const int bi = l & 1;
-                if (!mbar_wait(&wbar[bi], (l >> 1) & 1, status)) { ok = false; break; }
+                if (!mbar_wait(&wbar[bi], (l >> 1) & 1, status, lim)) { ok = false; break; }
                 // the epilogue of rank l - 2 has read this accumulator
-                if (l >= 2 && !mbar_wait(&tfree[bi], ((l - 2) >> 1) & 1, status)) { ok = false; break; }
+                if (l >= 2 && !mbar_wait(&tfree[bi], ((l - 2) >> 1) & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 const uint64_t dW = make_desc(sb + LY::W + bi * LY::WBUF, 16, 1024, 2);
                 // the anchor as a bf16 hi / lo pair: (a_hi + a_lo) W^T, the weights exact bf16
@@ -133,13 +135,13 @@ __global__ void __launch_bounds__(P_THREADS, D == 64 ? 2 : 1) write_producer_ker
                 mma_steps<D / 16>(tb + bi * 2 * D, id, dAl, dW, oa, ow, true);
                 mma_commit(&full[bi]);
                 if (issued < L) {  // W of rank l + 2 into this buffer once the MMA has read it
-                    if (!mbar_wait(&full[bi], (l >> 1) & 1, status)) { ok = false; break; }
+                    if (!mbar_wait(&full[bi], (l >> 1) & 1, status, lim)) { ok = false; break; }
                     load_w(issued++);
                 }
             }
             if (!ok) failed_sh = 1;
             mma_commit(&drain);
-            mbar_wait(&drain, 0, nullptr);
+            mbar_wait(&drain, 0, nullptr, lim);
             // after a failure, weight loads still in flight land before the CTA exits
             if (!ok)
                 for (int l = issued > 2 ? issued - 2 : 0; l < issued; ++l)
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(P_THREADS, D == 64 ? 2 : 1) write_producer_ker
         bool ok = true;
         for (int l = 0; l < L && ok; ++l) {
             const int bi = l & 1;
-            if (!mbar_wait(&full[bi], (l >> 1) & 1, status)) { ok = false; break; }
+            if (!mbar_wait(&full[bi], (l >> 1) & 1, status, lim)) { ok = false; break; }
             fence_after_sync();
             const float bl = live ? p.beta[tok * L + l] : 0.f;
             const size_t orow = (tok * L + l) * D;

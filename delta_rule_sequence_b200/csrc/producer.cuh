@@ -16,6 +16,7 @@ struct ProducerArgs {
     const void *Wk, *Wp;
     const float *beta;
     void *u, *w;
+    int stall;  // the give-up test: no weight load is issued, every wait runs out after a short limit
 };
 
 cudaError_t launch_write_producer(const ProducerArgs &a, cudaStream_t s);

@@ -36,9 +36,10 @@ constexpr int NTH = 256;
 
 // Row block `rb` of out = x E (+ add): rows rb*RB .. rb*RB+RB-1 of x (nrows x D), E (D x D)
 // staged in shared memory.
+// x and out may be the same array (prism_state_fold in place), so neither is restrict-qualified.
 template <int D>
-__device__ __forceinline__ void rows_times(const float *__restrict__ x, const float *__restrict__ E,
-                                           const float *__restrict__ add, float *__restrict__ out,
+__device__ __forceinline__ void rows_times(const float *x, const float *__restrict__ E,
+                                           const float *__restrict__ add, float *out,
                                            int nrows, int rb, float *sE, float *sx) {
     for (int e = threadIdx.x; e < D * D / 4; e += NTH)
         reinterpret_cast<float4 *>(sE)[e] = reinterpret_cast<const float4 *>(E)[e];
@@ -256,13 +257,13 @@ cudaError_t launch_segment_element(const ScanArgs &a, int route, bool io_f32, vo
     ScanArgs e = a;
     e.S0 = nullptr;
     e.o = nullptr;
-    e.flags = kNoWrite | kS0Identity | kNoOutput;
+    e.flags = (a.flags & (kForceWkLo | kStallTest | kStallPrep)) | kNoWrite | kS0Identity | kNoOutput;
     e.S_final = e_out;
     if ((err = a.T == 0 ? launch_state_init(e, s) : pass(e)) != cudaSuccess) return err;
     ScanArgs f = a;
     f.S0 = nullptr;
     f.o = nullptr;
-    f.flags = kNoOutput;
+    f.flags = (a.flags & (kForceWkLo | kStallTest | kStallPrep)) | kNoOutput;
     f.S_final = f_out;
     return a.T == 0 ? launch_state_init(f, s) : pass(f);
 }
@@ -315,11 +316,11 @@ cudaError_t launch_segmented(const ScanArgs &a, int route, bool io_f32, int G, v
     if (route == 3 && (err = launch_lrank_prep(v, ws, s)) != cudaSuccess) return err;
     // 1. encode: E_g (identity rows, no write) and f_g (zero state, with the write)
     ScanArgs e = v;
-    e.flags = kNoWrite | kS0Identity | kNoOutput;
+    e.flags = (a.flags & (kForceWkLo | kStallTest | kStallPrep)) | kNoWrite | kS0Identity | kNoOutput;
     e.S_final = Eleaf;
     if ((err = pass(e)) != cudaSuccess) return err;
     ScanArgs f = v;
-    f.flags = kNoOutput;
+    f.flags = (a.flags & (kForceWkLo | kStallTest | kStallPrep)) | kNoOutput;
     f.S_final = Fleaf;
     if ((err = pass(f)) != cudaSuccess) return err;
     // 2. Blelloch over the segment elements -> entry states; exit state

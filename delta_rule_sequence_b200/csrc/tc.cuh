@@ -88,6 +88,23 @@ __device__ __forceinline__ void mma_steps(uint32_t d, uint32_t idesc, uint64_t a
               "r"((accumulate || ks > 0) ? 1u : 0u));
 }
 
+// mma_steps with an output-lane mask: TMEM lanes whose bit is set in `off` (lane i <-> bit i % 32
+// of off[i / 32]) keep their contents; the other lanes receive the product as usual.
+template <int NKS, class OA, class OB>
+__device__ __forceinline__ void mma_steps_lanes(uint32_t d, uint32_t idesc, uint64_t a, uint64_t b, OA oa,
+                                                OB ob, bool accumulate, const uint32_t (&off)[4]) {
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+            :
+            : "r"(d), "l"(a + oa(ks)), "l"(b + ob(ks)), "r"(idesc),
+              "r"((accumulate || ks > 0) ? 1u : 0u), "r"(off[0]), "r"(off[1]), "r"(off[2]),
+              "r"(off[3]));
+}
+
 // 4-D tiled TMA load of one box into shared memory, completing on `bar` (tx bytes).
 __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int x, int y, int z, int w,
                                             uint64_t *bar) {

@@ -24,6 +24,8 @@ EXPORTS = (
     "prism_scan_fwd_launch_count",
     "prism_scan_fwd",
     "prism_scan_fwd_noalloc",
+    "prism_scan_bwd_workspace_size",
+    "prism_scan_bwd",
     "prism_scan_segment_element",
     "prism_state_fold",
     "prism_step_decode",
@@ -76,6 +78,10 @@ def load_library():
     lib.prism_scan_fwd.restype = ci
     lib.prism_scan_fwd_noalloc.argtypes = [shp] + [vp] * 10 + [vp]
     lib.prism_scan_fwd_noalloc.restype = ci
+    lib.prism_scan_bwd_workspace_size.argtypes = [shp, ctypes.POINTER(sz)]
+    lib.prism_scan_bwd_workspace_size.restype = ci
+    lib.prism_scan_bwd.argtypes = [shp] + [vp] * 18 + [vp, sz, vp]
+    lib.prism_scan_bwd.restype = ci
     lib.prism_scan_segment_element.argtypes = [shp] + [vp] * 9 + [vp, sz, vp]
     lib.prism_scan_segment_element.restype = ci
     lib.prism_state_fold.argtypes = [ci, ci, ci, vp, vp, vp, vp, vp]
@@ -109,10 +115,21 @@ def _ptr(x):
     return None if x is None else ctypes.c_void_p(x.data_ptr())
 
 
-def _stream(stream):
+def _stream(stream, device):
+    """The stream to launch on: the caller's (which must belong to `device`), else the current
+    stream of `device` (not of whichever device happens to be current)."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors are on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _call(device, fn, *args):
+    """Run a library entry point with `device` current (the library launches on the current
+    device and looks up per-device state there)."""
+    with torch.cuda.device(device):
+        return fn(*args)
 
 
 def _check_tensor(name, x, dtype, shape, device):
@@ -185,9 +202,10 @@ def prism_scan_fwd(q, k, v, alpha, beta, u=None, w=None, S0=None, *, chunk=64, o
     _check_tensor("S_final", S_final, torch.float32, (B, H, dv, dk), dev)
     if workspace is None:
         workspace = workspace_for(shape, dev)
-    rc = lib.prism_scan_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
-                            _ptr(beta), _ptr(u), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_final),
-                            _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check_tensor("workspace", workspace, torch.uint8, (workspace.numel(),), dev)
+    rc = _call(dev, lib.prism_scan_fwd, ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+               _ptr(beta), _ptr(u), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_final),
+               _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream, dev))
     if rc != PRISM_OK:
         raise PrismError(rc, "prism_scan_fwd")
     return o, S_final
@@ -213,12 +231,72 @@ def prism_scan_fwd_noalloc(q, k, v, alpha, beta, u=None, w=None, S0=None, *, chu
                              ("S0", S0, torch.float32, (B, H, dv, dk)), ("o", o, io, (B, T, H, dv)),
                              ("S_final", S_final, torch.float32, (B, H, dv, dk))):
         _check_tensor(name, x, dt, shp, dev)
-    rc = lib.prism_scan_fwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
-                                    _ptr(beta), _ptr(u), _ptr(w), _ptr(S0), _ptr(o),
-                                    _ptr(S_final), _stream(stream))
+    rc = _call(dev, lib.prism_scan_fwd_noalloc, ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+               _ptr(alpha), _ptr(beta), _ptr(u), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_final),
+               _stream(stream, dev))
     if rc != PRISM_OK:
         raise PrismError(rc, "prism_scan_fwd_noalloc")
     return o, S_final
+
+
+def bwd_workspace_for(shape: PrismShape, device) -> torch.Tensor:
+    """A cached device workspace of the size prism_scan_bwd needs (one per device/size)."""
+    need = ctypes.c_size_t(0)
+    rc = load_library().prism_scan_bwd_workspace_size(ctypes.byref(shape), ctypes.byref(need))
+    if rc != PRISM_OK:
+        raise PrismError(rc, "prism_scan_bwd_workspace_size")
+    key = ("bwd", str(device), int(need.value))
+    ws = _ws_cache.get(key)
+    if ws is None:
+        ws = torch.zeros(max(256, int(need.value)), dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def prism_scan_bwd(q, k, v, alpha, beta, u=None, w=None, S0=None, *, dO, dS_final=None,
+                   want_dS0=True, workspace=None, stream=None):
+    """Backward of prism_scan_fwd: gradients of every input, fp32.  Inputs as for prism_scan_fwd;
+    dO: [B,T,H,dv] (io dtype); dS_final: [B,H,dv,dk] fp32 or None.  Returns a dict with dq, dk
+    [B,T,H,dk], dalpha, dbeta [B,T,H], dv [B,T,H,dv] (GDN write) or du [B,T,H,L,dv] and dw
+    [B,T,H,L,dk] (rank-L write), and dS0 [B,H,dv,dk] (or None)."""
+    lib = load_library()
+    if not isinstance(q, torch.Tensor) or not q.is_cuda:
+        raise TypeError("q must be a CUDA tensor (libprism has no CPU path)")
+    dev, io = q.device, q.dtype
+    shape = make_shape(q, v, u)
+    B, T, H, dk = q.shape
+    dv, L = shape.dv, shape.L
+    f32 = torch.float32
+    _check_tensor("q", q, io, (B, T, H, dk), dev)
+    _check_tensor("k", k, io, (B, T, H, dk), dev)
+    _check_tensor("v", v, io, (B, T, H, dv), dev)
+    _check_tensor("alpha", alpha, f32, (B, T, H), dev)
+    _check_tensor("beta", beta, f32, (B, T, H), dev)
+    _check_tensor("u", u, io, (B, T, H, L, dv), dev)
+    _check_tensor("w", w, io, (B, T, H, L, dk), dev)
+    _check_tensor("S0", S0, f32, (B, H, dv, dk), dev)
+    _check_tensor("dO", dO, io, (B, T, H, dv), dev)
+    _check_tensor("dS_final", dS_final, f32, (B, H, dv, dk), dev)
+    gdn = u is None
+    out = {"dq": torch.empty((B, T, H, dk), dtype=f32, device=dev),
+           "dk": torch.empty((B, T, H, dk), dtype=f32, device=dev),
+           "dv": torch.empty((B, T, H, dv), dtype=f32, device=dev) if gdn else None,
+           "dalpha": torch.empty((B, T, H), dtype=f32, device=dev),
+           "dbeta": torch.empty((B, T, H), dtype=f32, device=dev),
+           "du": None if gdn else torch.empty((B, T, H, L, dv), dtype=f32, device=dev),
+           "dw": None if gdn else torch.empty((B, T, H, L, dk), dtype=f32, device=dev),
+           "dS0": torch.empty((B, H, dv, dk), dtype=f32, device=dev) if want_dS0 else None}
+    if workspace is None:
+        workspace = bwd_workspace_for(shape, dev)
+    _check_tensor("workspace", workspace, torch.uint8, (workspace.numel(),), dev)
+    rc = _call(dev, lib.prism_scan_bwd, ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+               _ptr(beta), _ptr(u), _ptr(w), _ptr(S0), _ptr(dO), _ptr(dS_final), _ptr(out["dq"]),
+               _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dalpha"]), _ptr(out["dbeta"]),
+               _ptr(out["du"]), _ptr(out["dw"]), _ptr(out["dS0"]), _ptr(workspace),
+               ctypes.c_size_t(workspace.numel()), _stream(stream, dev))
+    if rc != PRISM_OK:
+        raise PrismError(rc, "prism_scan_bwd")
+    return out
 
 
 def prism_step_decode(q, k, v, alpha, beta, u, w, S, *, o=None, stream=None):
@@ -243,8 +321,8 @@ def prism_step_decode(q, k, v, alpha, beta, u, w, S, *, o=None, stream=None):
     if o is None:
         o = torch.empty((B, T, H, dv), dtype=io, device=dev)
     _check_tensor("o", o, io, (B, T, H, dv), dev)
-    rc = lib.prism_step_decode(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
-                               _ptr(beta), _ptr(u), _ptr(w), _ptr(S), _ptr(o), _stream(stream))
+    rc = _call(dev, lib.prism_step_decode, ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+               _ptr(alpha), _ptr(beta), _ptr(u), _ptr(w), _ptr(S), _ptr(o), _stream(stream, dev))
     if rc != PRISM_OK:
         raise PrismError(rc, "prism_step_decode")
     return o
@@ -274,8 +352,8 @@ def prism_write_producer(x, v, conv, Wk, Wp, beta, *, u=None, w=None, stream=Non
     _check_tensor("u", u, bf, (B, T, H, L, d), dev)
     _check_tensor("w", w, bf, (B, T, H, L, d), dev)
     shape = PrismShape(B, H, T, d, d, L, 64, PRISM_BF16)
-    rc = lib.prism_write_producer(ctypes.byref(shape), _ptr(x), _ptr(v), _ptr(conv), _ptr(Wk),
-                                  _ptr(Wp), _ptr(beta), _ptr(u), _ptr(w), _stream(stream))
+    rc = _call(dev, lib.prism_write_producer, ctypes.byref(shape), _ptr(x), _ptr(v), _ptr(conv),
+               _ptr(Wk), _ptr(Wp), _ptr(beta), _ptr(u), _ptr(w), _stream(stream, dev))
     if rc != PRISM_OK:
         raise PrismError(rc, "prism_write_producer")
     return u, w
@@ -290,9 +368,17 @@ def prism_scan_fwd_launch_count(shape: PrismShape) -> int:
     return n.value
 
 
-def prism_query_device_status(workspace, stream=None) -> int:
-    """Synchronise and return (and clear) the status word kernels wrote into `workspace`."""
-    return load_library().prism_query_device_status(_ptr(workspace), _stream(stream))
+def prism_query_device_status(workspace, stream=None, device=None) -> int:
+    """Synchronise and return (and clear) the status words: the one kernels wrote into
+    `workspace` (or None), and the library's own (decode, producer, no-alloc scratch) on the
+    workspace's device (else `device`, else the current device)."""
+    if workspace is not None:
+        device = workspace.device
+    elif device is None:
+        device = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
+    device = torch.device(device)
+    return _call(device, load_library().prism_query_device_status, _ptr(workspace),
+                 _stream(stream, device))
 
 
 def record_launch_events(events) -> None:
@@ -330,9 +416,10 @@ def prism_scan_segment_element(q, k, v, alpha, beta, u=None, w=None, *, chunk=64
     _check_tensor("f", f, torch.float32, (B, H, dv, dk), dev)
     if workspace is None:
         workspace = workspace_for(shape, dev)
-    rc = lib.prism_scan_segment_element(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
-                                        _ptr(beta), _ptr(u), _ptr(w), _ptr(E), _ptr(f), _ptr(workspace),
-                                        ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check_tensor("workspace", workspace, torch.uint8, (workspace.numel(),), dev)
+    rc = _call(dev, lib.prism_scan_segment_element, ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+               _ptr(alpha), _ptr(beta), _ptr(u), _ptr(w), _ptr(E), _ptr(f), _ptr(workspace),
+               ctypes.c_size_t(workspace.numel()), _stream(stream, dev))
     if rc != PRISM_OK:
         raise PrismError(rc, "prism_scan_segment_element")
     return E, f
@@ -354,7 +441,8 @@ def prism_state_fold(S_in, E, f, S_out=None, stream=None):
     if S_out is None:
         S_out = torch.empty_like(f)
     _check_tensor("S_out", S_out, torch.float32, lead + (dv, dk), dev)
-    rc = lib.prism_state_fold(BH, dk, dv, _ptr(S_in), _ptr(E), _ptr(f), _ptr(S_out), _stream(stream))
+    rc = _call(dev, lib.prism_state_fold, BH, dk, dv, _ptr(S_in), _ptr(E), _ptr(f), _ptr(S_out),
+               _stream(stream, dev))
     if rc != PRISM_OK:
         raise PrismError(rc, "prism_state_fold")
     return S_out

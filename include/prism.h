@@ -93,17 +93,58 @@ prism_status prism_scan_fwd_launch_count(const prism_shape *shape, int *launches
  *                              kernel records a failure; prism_query_device_status reads and
  *                              clears it); may be reused once the stream has passed this call
  * The result equals the token recurrence above up to floating-point rounding: state and all
- * accumulation in fp32; bf16 operands are fed to the tensor cores (intermediate results as bf16
- * hi / lo pairs, except the chunk's Wk, a single bf16).  The bf16 tolerance |x - r| <= 2e-2
- * (1 + |r|) is met for unit-norm keys and write directions; with write directions of norm ~8
- * the state grows into the hundreds and one output element in ~4e4 was seen at 1.4x that
- * bound.  A partial last chunk is handled as if padded with identity tokens (alpha = 1,
- * beta = 0, no write).
+ * accumulation in fp32; bf16 operands are fed to the tensor cores, intermediate results as bf16
+ * hi / lo pairs (the chunk's Wk as one bf16 while every state element stays below 4 in
+ * magnitude, as a pair once one exceeds it).  Tested against |x - r| <= 2e-2 (1 + |r|) for bf16
+ * I/O and 1e-4 (1 + |r|) for fp32 I/O, including write directions of norm ~8 whose state grows
+ * into the hundreds.  A partial last chunk is handled as if padded with identity tokens
+ * (alpha = 1, beta = 0, no write).
  */
 prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void *k,
                             const void *v, const float *alpha, const float *beta,
                             const void *u, const void *w, const float *S0, void *o,
                             float *S_final, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * prism_scan_bwd_workspace_size -- bytes of device workspace prism_scan_bwd needs for `shape`:
+ * the status block, the state of every (b, h) at each 64-token chunk start, and one chunk of
+ * states per CTA.  Writes *bytes.
+ */
+prism_status prism_scan_bwd_workspace_size(const prism_shape *shape, size_t *bytes);
+
+/*
+ * prism_scan_bwd -- the backward pass of prism_scan_fwd: given the forward's inputs and the
+ * upstream gradients dO of o and dS_final of S_final, the gradients of every input, for training
+ * ("PRISM: Parallel Residual Iterative Sequence Model", gist.science explainer, section 4: the
+ * method's throughput is training throughput; the recurrence of technical summary 2.1-2.2).  With
+ * G_t the gradient of S_t (G_T = dS_final), running from the last token to the first:
+ *   G_t += dO_t q_t^T;   dq_t = S_t^T dO_t;
+ *   dalpha_t = <G_t, S_{t-1}(I - beta_t k_t k_t^T)>;
+ *   dbeta_t = -alpha_t (S_{t-1}k_t).(G_t k_t)  (+ v_t.(G_t k_t) for the GDN write);
+ *   dk_t = -alpha_t beta_t (G_t^T S_{t-1}k_t + S_{t-1}^T G_t k_t)  (+ beta_t G_t^T v_t);
+ *   dv_t = beta_t G_t k_t  (GDN write)  |  du_{t,l} = G_t w_{t,l},  dw_{t,l} = G_t^T u_{t,l};
+ *   G_{t-1} = alpha_t G_t (I - beta_t k_t k_t^T);   dS0 = G_0.
+ *   q, k, v, alpha, beta, u, w, S0   exactly as passed to prism_scan_fwd (same shape rules)
+ *   dO        [B,T,H,dv] io       upstream gradient of o
+ *   dS_final  [B,H,dv,dk] fp32    upstream gradient of S_final, or NULL for zero
+ *   dq, dk    [B,T,H,dk] fp32     outputs (gradients are fp32 whatever the I/O type)
+ *   dv        [B,T,H,dv] fp32     output, GDN write only (ignored on the rank-L write)
+ *   dalpha, dbeta [B,T,H] fp32    outputs
+ *   du, dw    [B,T,H,L,dv], [B,T,H,L,dk] fp32   outputs, rank-L write only (ignored otherwise)
+ *   dS0       [B,H,dv,dk] fp32    output, or NULL to skip
+ *   workspace, ws_bytes           at least prism_scan_bwd_workspace_size bytes, 256-byte aligned
+ * Every pointer 16-byte aligned; no gradient may overlap another or an input.  All arithmetic is
+ * fp32 on CUDA cores from the exact input values: each CTA re-runs the forward recurrence for its
+ * value rows (checkpointing every 64 tokens), then walks the tokens backwards chunk by chunk.
+ * dq, dk, dw, dalpha and dbeta are sums over value rows accumulated with atomic adds (cleared on
+ * the stream first), so their last bits depend on the order of those adds.  Tested against
+ * |x - r| <= tol (1 + |r|) with tol = 2e-2 (bf16 I/O) and 1e-4 (fp32 I/O).
+ */
+prism_status prism_scan_bwd(const prism_shape *shape, const void *q, const void *k, const void *v,
+                            const float *alpha, const float *beta, const void *u, const void *w,
+                            const float *S0, const void *dO, const float *dS_final, float *dq,
+                            float *dk, float *dv, float *dalpha, float *dbeta, float *du, float *dw,
+                            float *dS0, void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * prism_scan_segment_element -- the affine map of a token segment, the building block of a scan
@@ -148,13 +189,18 @@ prism_status prism_step_decode(const prism_shape *shape, const void *q, const vo
  * loads libprism.so holds until the process exits.  This call allocates nothing.
  *   - Shapes whose workspace (prism_scan_fwd_workspace_size) exceeds PRISM_NOALLOC_SCRATCH_BYTES
  *     are rejected with PRISM_ERR_UNSUPPORTED before anything is enqueued.
+ *   - Arguments are checked as prism_scan_fwd checks them, with the same status codes, before
+ *     anything is sized or enqueued.
  *   - The first call on each device looks up the scratch's device address (with that device
- *     current) and caches it; make that first call before any stream capture.
+ *     current) and caches it, and looks it up again if the device's context has changed (after
+ *     a cudaDeviceReset); make that first call before any stream capture.
  *   - All calls on a device share the one scratch array, which keeps the last call's contents:
  *     calls whose kernels overlap on the GPU (different streams, no ordering between them) race
  *     on it.  Serialise them (one stream, or events).
- *   - A kernel's bounded-wait failure is recorded in the scratch but not reported by this entry
- *     point; callers that need that report use prism_scan_fwd with their own workspace.
+ *   - The scratch's first 4 bytes are the scan's status word (zero when the library loads): a
+ *     kernel whose bounded wait gave up records PRISM_ERR_TIMEOUT there, and
+ *     prism_query_device_status(NULL, stream), called with the same device current, reports
+ *     and clears it.
  * The method pages have no counterpart of this entry point; it exists for the callers above.
  */
 #define PRISM_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -188,8 +234,9 @@ prism_status prism_write_producer(const prism_shape *shape, const void *x, const
 
 /*
  * prism_query_device_status -- synchronise `stream`, read the status word in `workspace` (written
- * by scan kernels whose bounded waits ran out; workspace may be NULL) and the library's decode
- * and producer status words, and clear them.  Returns PRISM_OK, PRISM_ERR_TIMEOUT, or
+ * by scan kernels whose bounded waits ran out; workspace may be NULL) and the library's own
+ * status words on the current device (decode, producer, and the scratch of
+ * prism_scan_fwd_noalloc), and clear them.  Returns PRISM_OK, PRISM_ERR_TIMEOUT, or
  * PRISM_ERR_CUDA if the stream itself reports an error.
  */
 prism_status prism_query_device_status(void *workspace, void *stream);
@@ -210,8 +257,13 @@ const char *prism_last_cuda_error(void);
  * segment) whenever the shape allows it (dk == dv, T divisible into segments of >= 64 tokens);
  * bit 2: it never does; bit 3: the stall test -- the Gated-DeltaNet state kernel's load warp
  * issues nothing, every wait gives up after a short limit, the kernel records PRISM_ERR_TIMEOUT
- * in the workspace status word and returns (outputs are then undefined).  Returns the previous
- * flags.
+ * in the workspace status word and returns (outputs are then undefined); bit 4: the tensor-core
+ * state kernel applies its Wk_lo precision term from the first chunk instead of only once the
+ * state has grown large (results stay within the same tolerance); bits 5, 6, 7: the same stall
+ * test for the per-chunk prep kernels of the tensor-core scan (their tile loads are not issued;
+ * PRISM_ERR_TIMEOUT in the workspace status word), for prism_write_producer (its weight loads;
+ * the producer status word) and for the bulk-copy decode kernel (its state copies; the decode
+ * status word).  Returns the previous flags.
  */
 int prism_debug_set_flags(int flags);
 

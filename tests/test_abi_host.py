@@ -150,3 +150,45 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros((1, 4, 1, 32))
     with pytest.raises(TypeError, match="CUDA"):
         P.prism_scan_fwd(x, x, x, torch.ones(1, 4, 1), torch.zeros(1, 4, 1))
+
+
+def _bwd(lib, shape, q=FAKE, k=FAKE, v=FAKE, a=FAKE, b=FAKE, u=None, w=None, S0=None,
+         dO=ctypes.c_void_p(0x50000), dSf=None, dq=ctypes.c_void_p(0x60000),
+         dk=ctypes.c_void_p(0x70000), dv=ctypes.c_void_p(0x80000), da=ctypes.c_void_p(0x90000),
+         db=ctypes.c_void_p(0xA0000), du=None, dw=None, dS0=None, ws=ctypes.c_void_p(0x100000),
+         ws_bytes=1 << 30):
+    return lib.prism_scan_bwd(ctypes.byref(shape), q, k, v, a, b, u, w, S0, dO, dSf, dq, dk, dv,
+                              da, db, du, dw, dS0, ws, ctypes.c_size_t(ws_bytes), None)
+
+
+def test_backward_rejects_bad_arguments(lib):
+    s = _shape()
+    assert _bwd(lib, _shape(dk=48)) == P.PRISM_ERR_UNSUPPORTED
+    assert _bwd(lib, _shape(L=0)) == P.PRISM_ERR_INVALID_ARG
+    assert _bwd(lib, s, dO=None) == P.PRISM_ERR_INVALID_ARG
+    assert _bwd(lib, s, dq=None) == P.PRISM_ERR_INVALID_ARG
+    assert _bwd(lib, s, dv=None) == P.PRISM_ERR_INVALID_ARG                 # GDN write needs dv
+    assert _bwd(lib, s, dk=ctypes.c_void_p(0x60000)) == P.PRISM_ERR_INVALID_ARG  # dk overlaps dq
+    assert _bwd(lib, s, dq=FAKE) == P.PRISM_ERR_INVALID_ARG                 # dq overlaps q
+    assert _bwd(lib, s, da=MISALIGNED) == P.PRISM_ERR_INVALID_ARG
+    assert _bwd(lib, s, ws_bytes=8) == P.PRISM_ERR_INVALID_ARG
+    rank = _shape(L=2)
+    u, w = ctypes.c_void_p(0xB0000), ctypes.c_void_p(0xC0000)
+    assert _bwd(lib, rank, u=u, w=w) == P.PRISM_ERR_INVALID_ARG              # rank L needs du, dw
+    assert _bwd(lib, rank, u=u, w=w, du=ctypes.c_void_p(0xD0000)) == P.PRISM_ERR_INVALID_ARG
+    assert lib.prism_scan_bwd(None, *([None] * 18), None, 0, None) == P.PRISM_ERR_INVALID_ARG
+    n = ctypes.c_size_t(0)
+    assert lib.prism_scan_bwd_workspace_size(ctypes.byref(s), ctypes.byref(n)) == P.PRISM_OK
+    assert n.value >= 4 * 2 * 4 * 32 * 32  # at least the chunk-start states
+    assert lib.prism_scan_bwd_workspace_size(None, ctypes.byref(n)) == P.PRISM_ERR_INVALID_ARG
+
+
+def test_noalloc_rejects_like_the_workspace_entry(lib):
+    """Checked before any sizing: the same status codes as prism_scan_fwd for malformed shapes."""
+    for kw in (dict(B=-1, dk=64, dv=64, io=P.PRISM_BF16), dict(dk=48), dict(chunk=32), dict(L=0),
+               dict(L=9), dict(io=7)):
+        s = _shape(**kw)
+        rc = lib.prism_scan_fwd_noalloc(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
+                                        None, ctypes.c_void_p(0x20000), None, None)
+        assert rc == _fwd(lib, s, o=ctypes.c_void_p(0x20000)), kw
+        assert rc != P.PRISM_OK

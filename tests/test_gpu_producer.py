@@ -69,37 +69,62 @@ def test_producer_full_size_sampled(name):
         compare(f"w[{b},{t0}:,{h}]", got_w, w_ref[:, CONV_WIDTH - 1:], TOL["bf16"])
 
 
-def test_producer_feeds_the_scan():
-    """The producer's write terms through the scan.  Element by element: the GPU scan on the
-    oracle producer's u, w (rounded to bf16) against the oracle scan on the same bytes.  End to
-    end (GPU producer -> GPU scan against oracle producer -> oracle scan): the two u, w differ by
-    bf16 rounding flips (one ulp where the fp32 value sits on a rounding boundary), which the
-    scan's unnormalised write directions carry into o, so that comparison is norm-wise."""
+def _bf16_neighbours(x):
+    """For each fp64 value: its bf16 rounding (nearest even) and the bf16 neighbour on the other
+    side of it (equal to the rounding where x is representable)."""
+    t = torch.from_numpy(np.asarray(x, dtype=np.float64))
+    nb = t.to(torch.bfloat16)
+    near = nb.double()
+    bits = nb.view(torch.int16).to(torch.int32)
+    away = (t.abs() > near.abs()).to(torch.int32) - (t.abs() < near.abs()).to(torch.int32)
+    other = (bits + away).to(torch.int16).view(torch.bfloat16).double()  # magnitude one ulp away
+    return near.numpy(), other.numpy()
+
+
+def _oracle_write_terms(p, u_gpu, w_gpu):
+    """The oracle producer's u, w rounded to bf16 (nearest even), as the scan receives them.
+    Where the GPU rounded an element to the other bf16 neighbour of the exact value (its fp32
+    arithmetic landed on the far side of a rounding midpoint), that element is checked to be that
+    neighbour, with the exact value within a quarter ulp of the midpoint, and its value is taken
+    from the GPU: both are the correct bf16 result up to the producer's own fp32 rounding.
+    Returns the terms and the fraction of such elements."""
+    u_ref, w_ref, _ = write_producer_ref(**p)
+    out, flips = [], 0
+    for ref, got in ((u_ref, u_gpu), (w_ref, w_gpu)):
+        near, other = _bf16_neighbours(ref)
+        flip = got != near
+        assert np.all(got[flip] == other[flip]), "a GPU write term is not a bf16 neighbour of the exact value"
+        ulp = np.abs(other - near)
+        assert np.all((np.abs(ref - (near + other) / 2) <= ulp / 4)[flip]), \
+            "a flipped element is not near a rounding midpoint"
+        flips += int(flip.sum())
+        out.append(torch.from_numpy(np.where(flip, got, near)).to(torch.bfloat16))
+    return out[0], out[1], flips / (u_ref.size + w_ref.size)
+
+
+@pytest.mark.parametrize("d,L,T", [(64, 3, 300), (128, 2, 200)])
+def test_producer_feeds_the_scan(d, L, T):
+    """The producer's write terms through the scan, element by element, with the producer's raw
+    (unnormalised) directions: |W_k a| is about 8 with these random weights, so the state grows
+    well beyond the unit-norm workloads.  GPU producer -> GPU scan against oracle producer ->
+    bf16 rounding -> oracle scan, at the bf16 tolerance 2e-2 (1 + |r|)."""
     from delta_rule_sequence_b200.prism import prism_scan_fwd, prism_write_producer
 
-    wl = WORKLOADS["recsys"].with_(B=1, H=2, T=300, L=3)
+    wl = WORKLOADS["recsys"].with_(B=1, H=2, T=T, dk=d, dv=d, L=L)
     p = make_producer_inputs(wl, seed=3)
-    # W_k scaled by 1/8 so that the write directions have about unit norm, as the scan's keys do
-    # (|W_k a| is about 8 with these random weights); the scan's bf16 operand design is validated
-    # for that range (with directions of norm ~8 one element in 38400 of o exceeded the tolerance)
-    p["Wk"] = (p["Wk"].float() / 8).to(torch.bfloat16)
     x = make_inputs(wl, seed=3)
-    u_ref, w_ref, _ = write_producer_ref(**p)
-    u_bf = torch.from_numpy(u_ref).to(torch.bfloat16)
-    w_bf = torch.from_numpy(w_ref).to(torch.bfloat16)
-    o_ref, S_ref = oracle.scan_ref(x["q"], x["k"], None, x["alpha"], x["beta"], u_bf, w_bf, None)
+    d_p = to_device(p)
+    u, w = prism_write_producer(d_p["x"], d_p["v"], d_p["conv"], d_p["Wk"], d_p["Wp"], d_p["beta"])
     dx = to_device(x)
-    o1, S1 = prism_scan_fwd(dx["q"], dx["k"], None, dx["alpha"], dx["beta"], u_bf.cuda(),
-                            w_bf.cuda(), None, chunk=64)
-    d = to_device(p)
-    u, w = prism_write_producer(d["x"], d["v"], d["conv"], d["Wk"], d["Wp"], d["beta"])
-    o2, S2 = prism_scan_fwd(dx["q"], dx["k"], None, dx["alpha"], dx["beta"], u, w, None, chunk=64)
+    o, S = prism_scan_fwd(dx["q"], dx["k"], None, dx["alpha"], dx["beta"], u, w, None, chunk=64)
     torch.cuda.synchronize()
-    compare("o (scan on the oracle's write terms)", o1.float().cpu().numpy(), o_ref, TOL["bf16"])
-    compare("S_final (same)", S1.cpu().numpy(), S_ref, TOL["bf16"])
-    rel = lambda a, r: float(np.linalg.norm(a - r) / np.linalg.norm(r))
-    assert rel(o2.float().cpu().numpy(), o_ref) < 1e-2
-    assert rel(S2.cpu().numpy(), S_ref) < 1e-2
+    u_or, w_or, flip_frac = _oracle_write_terms(p, u.float().cpu().numpy(), w.float().cpu().numpy())
+    assert flip_frac < 1e-2
+    wnorm = float(w_or.float().norm(dim=-1).mean())
+    assert wnorm > 4.0, wnorm  # the directions really are far from unit norm
+    o_ref, S_ref = oracle.scan_ref(x["q"], x["k"], None, x["alpha"], x["beta"], u_or, w_or, None)
+    compare("o (producer -> scan)", o.float().cpu().numpy(), o_ref, TOL["bf16"])
+    compare("S_final (producer -> scan)", S.cpu().numpy(), S_ref, TOL["bf16"])
 
 
 def test_producer_leaves_no_tokens_untouched_and_no_status():
