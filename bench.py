@@ -539,6 +539,76 @@ def time_producer(wl, dev, stream, peaks, rank, max_over_ranks, barrier, world, 
             "steps": steps}
 
 
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # 148 SMs x 128 fp32 FMA lanes x 2 x 1965 MHz
+
+
+def backward_bytes(wl, io_bytes=2):
+    """Algorithmic bytes of one backward call: the forward's inputs and dO read once, every
+    gradient written once in fp32, S0 and dS_final read and dS0 written."""
+    B, T, H, dk, dv, L = wl.B, wl.T, wl.H, wl.dk, wl.dv, wl.L
+    tok = B * T * H
+    rd = (2 * dk + dv) * io_bytes + 8                     # q, k, dO, alpha, beta
+    wr = (2 * dk) * 4 + 8                                 # dq, dk, dalpha, dbeta
+    if wl.write == "gdn":
+        rd += dv * io_bytes
+        wr += dv * 4
+    else:
+        rd += L * (dk + dv) * io_bytes
+        wr += L * (dk + dv) * 4
+    return tok * (rd + wr) + 3 * B * H * dv * dk * 4
+
+
+def backward_flops(wl):
+    """FLOPs of the reverse recurrence itself (one forward step and one backward step per token
+    and value row; the kernel's recomputation of the forward is not counted)."""
+    L = 1 if wl.write == "gdn" else wl.L
+    return wl.B * wl.T * wl.H * wl.dv * wl.dk * (18 + 5 * L)
+
+
+def time_backward(wl, dev, stream, peaks, rank, max_over_ranks, barrier, world, steps=5):
+    """prism_scan_bwd on a scan workload, timed alone (device-resident inputs and dO)."""
+    import torch
+
+    from delta_rule_sequence_b200 import prism
+    from delta_rule_sequence_b200.workloads import make_inputs
+
+    x = {n: (None if t is None else t.to(dev)) for n, t in make_inputs(wl, seed=7 + rank).items()}
+    g = torch.Generator().manual_seed(11 + rank)
+    dO = torch.randn((wl.B, wl.T, wl.H, wl.dv), generator=g).to(wl.torch_io).to(dev)
+    dS = (torch.randn((wl.B, wl.H, wl.dv, wl.dk), generator=g) * 0.1).float().to(dev)
+
+    def call():
+        return prism.prism_scan_bwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["u"], x["w"],
+                                    x["S0"], dO=dO, dS_final=dS, stream=stream)
+
+    with torch.cuda.stream(stream):
+        call()
+    stream.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1)) / steps
+    alg, fl = backward_bytes(wl), backward_flops(wl)
+    del x, dO, dS
+    return {"workload": f"backward on {workload_config(wl)['workload']}",
+            "ms_per_call": ms, "tokens_per_s": world * wl.B * wl.T / (ms / 1e3), "launches": 1,
+            "roofline": {"bound": "alu", "achieved": fl / (ms / 1e3) / 1e12,
+                         "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                         "frac": fl / (ms / 1e3) / 1e12 / FP32_ALU_TFLOPS,
+                         "peak_kind": "fp32 CUDA-core FMA peak from unit counts and the 1965 MHz clock",
+                         "algorithmic_flops": fl, "algorithmic_bytes": alg,
+                         "hbm_frac": alg / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
+            "steps": steps,
+            "timing": "CUDA events around the calls (each call clears the summed gradients first)"}
+
+
 def workload_config(wl):
     return {"workload": f"{wl.name}: B={wl.B} H={wl.H} T={wl.T} dk={wl.dk} dv={wl.dv} L={wl.L} "
                         f"chunk={wl.chunk} io={wl.io} state=f32 write={wl.write}",
@@ -748,11 +818,14 @@ def main():
                   "inputs": "4 seeded step batches cycled; state carried across steps"}
         del S, pool, o_d
 
-    # ---- secondary: the write-term producer on the two rank-L shapes
+    # ---- secondary: the write-term producer on the two rank-L shapes, and the backward pass
     if not args.no_configs:
         for name in ("recsys", "long"):
             others["producer_" + name] = time_producer(WORKLOADS[name], dev, stream, peaks, rank,
                                                        max_over_ranks, barrier, world)
+        for name, steps in (("gdn", 5), ("long", 2)):
+            others["backward_" + name] = time_backward(WORKLOADS[name], dev, stream, peaks, rank,
+                                                       max_over_ranks, barrier, world, steps=steps)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

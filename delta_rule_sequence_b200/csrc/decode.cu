@@ -12,12 +12,12 @@
 // dk/32 consecutive columns (a 16-byte vector at dk = 128).  The state is streamed: it is far
 // larger than L2 and touched once per step.
 //
-// Two variants.  `decode_bulk_kernel` (dk = 128, dv = 64 or 128) copies the head's whole state
-// into shared memory with four bulk copies (cp.async.bulk, one mbarrier each) issued before
-// anything else, so that the bytes in flight per SM are set by shared memory (three CTAs, up to
-// 192 KB) rather than by registers; each warp starts on its rows as soon as their quarter has
-// landed and stores the new rows with evict-first stores.  `decode_kernel` (every other shape)
-// loads 8 rows per warp into registers (evict-first) before reducing any of them.
+// Two variants.  `decode_ring_kernel` (dk = 128, dv = 64 or 128) is persistent, one CTA per SM:
+// each head's state and token vectors arrive in one of three shared-memory stages by bulk copies
+// (cp.async.bulk) issued three heads ahead, so that the bytes in flight per SM are set by shared
+// memory rather than by registers and stay in flight while the current head is updated.
+// `decode_kernel` (every other shape) loads 8 rows per warp into registers (evict-first) before
+// reducing any of them.
 
 #include "tc.cuh"
 
@@ -200,60 +200,162 @@ __device__ __forceinline__ void decode_rows8(const ScanArgs &p, int head, int r0
     for (int j = 0; j < ROWS_IN_FLIGHT; ++j) vstore<PER>(S + (size_t)(r0 + j) * DK + lane * PER, s[j]);
 }
 
-// dk = 128, dv = DV in {64, 128}: the head's state arrives in shared memory by four bulk copies;
-// warps 2c and 2c + 1 take quarter c (DV / 8 rows each, in blocks of 8).
-constexpr int kDecodePieces = 4;
+// dk = 128, dv = DV in {64, 128}: a persistent CTA per SM walks the heads blockIdx.x,
+// blockIdx.x + gridDim.x, ...  Each head's state and token vectors (k, q, and u, w or v) arrive in
+// one of NSTAGE shared-memory stages by bulk copies issued NSTAGE heads ahead, so that while one
+// head is updated the next ones are already in flight; warp w updates rows [w DV/8, (w+1) DV/8)
+// in blocks of 8 and stores them with evict-first stores.
+constexpr int kDecodeStages = 3;
 
 template <typename IO, int DV, int LW>
-__global__ void __launch_bounds__(NT, 3) decode_bulk_kernel(ScanArgs p) {
+struct RingLayout {
+    static constexpr int DK = 128;
+    static constexpr uint32_t S = 0;                                 // fp32 [DV][DK]
+    static constexpr uint32_t K = S + DV * DK * 4;                   // io [DK]
+    static constexpr uint32_t Q = K + DK * sizeof(IO);               // io [DK]
+    static constexpr uint32_t U = Q + DK * sizeof(IO);               // io [LW][DV] (or v [DV])
+    static constexpr uint32_t W = U + LW * DV * sizeof(IO);          // io [LW][DK] (rank L)
+    static constexpr uint32_t STAGE = W + LW * DK * sizeof(IO);
+    static constexpr uint32_t BYTES = kDecodeStages * STAGE;
+    static_assert(STAGE % 16 == 0 && (DK * sizeof(IO)) % 16 == 0, "bulk copies move 16-byte units");
+};
+
+template <typename IO, int DV, int LW>
+__global__ void __launch_bounds__(NT, 1) decode_ring_kernel(ScanArgs p, int nheads) {
+    using LY = RingLayout<IO, DV, LW>;
     constexpr int DK = 128, PER = DK / 32;
-    constexpr int RP = DV / kDecodePieces;       // rows per piece
-    constexpr int RW = RP / 2;                   // rows per warp
+    constexpr int RW = DV / NW;  // rows per warp
     static_assert(RW % ROWS_IN_FLIGHT == 0, "a warp's rows come in blocks of 8");
-    constexpr uint32_t PIECE_BYTES = RP * DK * 4;
-    extern __shared__ __align__(128) float sS[];  // [DV][DK]
-    __shared__ uint64_t bar[kDecodePieces];
-    __shared__ __align__(16) float s_u[LW][128];
-    __shared__ __align__(16) float s_w[LW][DK];
-    __shared__ float s_wq[LW];
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t full[kDecodeStages];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int head = blockIdx.x;
-    const float *S = p.S_final + (size_t)head * DV * DK;
+    const bool gdn = (p.u == nullptr);
+    const int L = p.L;
+    const IO *qg = (const IO *)p.q, *kg = (const IO *)p.k, *vg = (const IO *)p.v;
+    const IO *ug = (const IO *)p.u, *wg = (const IO *)p.w;
     // the give-up test: the copies are not issued and the waits run out after a short limit
     const bool stall = (p.flags & kStallDecode) != 0;
     const uint32_t lim = stall ? kStallTestPolls : kWaitPolls;
 
-    if (threadIdx.x == 0) {
-#pragma unroll
-        for (int c = 0; c < kDecodePieces; ++c) tc::mbar_init(&bar[c], 1);
-        tc::mbar_fence_init();
-        if (!stall) {
-#pragma unroll
-            for (int c = 0; c < kDecodePieces; ++c) {
-                tc::mbar_expect_tx(&bar[c], PIECE_BYTES);
-                tc::bulk_g2s(sS + (size_t)c * RP * DK, S + (size_t)c * RP * DK, PIECE_BYTES, &bar[c]);
-            }
+    auto issue = [&](int st, int head) {  // thread 0: one head into stage st
+        uint8_t *dst = smem + st * LY::STAGE;
+        const uint32_t vec = gdn ? DV * sizeof(IO) : LW * (DV + DK) * sizeof(IO);
+        tc::mbar_expect_tx(&full[st], DV * DK * 4 + 2 * DK * sizeof(IO) + vec);
+        tc::bulk_g2s(dst + LY::S, p.S_final + (size_t)head * DV * DK, DV * DK * 4, &full[st]);
+        tc::bulk_g2s(dst + LY::K, kg + (size_t)head * DK, DK * sizeof(IO), &full[st]);
+        tc::bulk_g2s(dst + LY::Q, qg + (size_t)head * DK, DK * sizeof(IO), &full[st]);
+        if (gdn) {
+            tc::bulk_g2s(dst + LY::U, vg + (size_t)head * DV, DV * sizeof(IO), &full[st]);
+        } else {
+            tc::bulk_g2s(dst + LY::U, ug + (size_t)head * LW * DV, LW * DV * sizeof(IO), &full[st]);
+            tc::bulk_g2s(dst + LY::W, wg + (size_t)head * LW * DK, LW * DK * sizeof(IO), &full[st]);
         }
+    };
+    const int first = blockIdx.x, step = gridDim.x;
+    const int mine = first < nheads ? (nheads - 1 - first) / step + 1 : 0;  // heads of this CTA
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kDecodeStages; ++i) tc::mbar_init(&full[i], 1);
+        tc::mbar_fence_init();
+        if (!stall)
+            for (int i = 0; i < kDecodeStages && i < mine; ++i) issue(i, first + i * step);
     }
-    DecodeHead<IO, DK, LW> hd;
-    decode_prologue<IO, DK, LW>(p, head, s_u, s_w, s_wq, hd);  // ends with a CTA barrier
-
-    const int piece = warp >> 1;
-    const bool landed = tc::mbar_wait(&bar[piece], 0, &g_decode_status, lim);
-    if (landed) {
+    __syncthreads();
+    int done = 0;  // heads consumed
+    for (int i = 0; i < mine; ++i) {
+        const int st = i % kDecodeStages, head = first + i * step;
+        const bool landed = tc::mbar_wait(&full[st], (i / kDecodeStages) & 1, &g_decode_status, lim);
+        if (__syncthreads_or(!landed)) break;
+        const uint8_t *stg = smem + st * LY::STAGE;
+        const float *sS = reinterpret_cast<const float *>(stg + LY::S);
+        const IO *sk = reinterpret_cast<const IO *>(stg + LY::K);
+        const IO *sq = reinterpret_cast<const IO *>(stg + LY::Q);
+        const IO *su = reinterpret_cast<const IO *>(stg + LY::U);
+        const IO *sw = gdn ? sk : reinterpret_cast<const IO *>(stg + LY::W);
+        const float a = p.alpha[head], be = p.beta[head], ab = a * be;
+        float kq[PER], qv[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            kq[e] = ld_io(sk, lane * PER + e);
+            qv[e] = ld_io(sq, lane * PER + e);
+        }
+        float kdotq = 0.f;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) kdotq = fmaf(kq[e], qv[e], kdotq);
+        kdotq = warp_sum(kdotq);
+        float wq[LW];  // w_l . q (every warp computes its own copy)
+#pragma unroll
+        for (int l = 0; l < LW; ++l) {
+            float t = 0.f;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) t = fmaf(ld_io(sw, (gdn ? 0 : l * DK) + lane * PER + e), qv[e], t);
+            wq[l] = warp_sum(t);
+        }
+        IO *o = (IO *)p.o + (size_t)head * DV;
+        float *S = p.S_final + (size_t)head * DV * DK;
+        const int my_row = lane >> 2;
         for (int rb = 0; rb < RW; rb += ROWS_IN_FLIGHT) {
-            const int r0 = piece * RP + (warp & 1) * RW + rb;
+            const int r0 = warp * RW + rb;
             float s[ROWS_IN_FLIGHT][PER];
 #pragma unroll
             for (int j = 0; j < ROWS_IN_FLIGHT; ++j)
                 vload_shared<PER>(sS + (size_t)(r0 + j) * DK + lane * PER, s[j]);
-            decode_rows8<IO, DK, LW>(p, head, r0, s, s_u, s_w, s_wq, hd);
-        }
-    }
-    // every copy has landed before the CTA's shared memory is released (bounded)
-    if (threadIdx.x == 0 && !stall) {
+            float ep[ROWS_IN_FLIGHT], pp[ROWS_IN_FLIGHT];
 #pragma unroll
-        for (int c = 0; c < kDecodePieces; ++c) tc::mbar_wait(&bar[c], 0, nullptr);
+            for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
+                float e = 0.f, pq = 0.f;
+#pragma unroll
+                for (int c = 0; c < PER; ++c) {
+                    e = fmaf(s[j][c], kq[c], e);
+                    pq = fmaf(s[j][c], qv[c], pq);
+                }
+                ep[j] = e;
+                pp[j] = pq;
+            }
+            const float e_mine = rows8_reduce_scatter(ep, lane);
+            const float p_mine = rows8_reduce_scatter(pp, lane);
+            // u_{l,r} of the 8 rows (beta v_r on the Gated-DeltaNet write)
+            float uu[LW][ROWS_IN_FLIGHT];
+#pragma unroll
+            for (int l = 0; l < LW; ++l)
+#pragma unroll
+                for (int j = 0; j < ROWS_IN_FLIGHT; ++j)
+                    uu[l][j] = gdn ? be * ld_io(su, r0 + j) : ld_io(su, l * DV + r0 + j);
+            if ((lane & 3) == 0) {
+                const int r = r0 + my_row;
+                float outv = a * p_mine - ab * e_mine * kdotq;
+#pragma unroll
+                for (int l = 0; l < LW; ++l)
+                    outv = fmaf(gdn ? be * ld_io(su, r) : ld_io(su, l * DV + r), wq[l], outv);
+                st_io(o, r, outv);
+            }
+#pragma unroll
+            for (int j = 0; j < ROWS_IN_FLIGHT; ++j) {
+                const float ej = __shfl_sync(0xffffffffu, e_mine, 4 * j);
+#pragma unroll
+                for (int c = 0; c < PER; ++c) s[j][c] = fmaf(a, s[j][c], -ab * ej * kq[c]);
+            }
+#pragma unroll
+            for (int l = 0; l < LW; ++l) {
+                float wv[PER];
+#pragma unroll
+                for (int c = 0; c < PER; ++c) wv[c] = ld_io(sw, (gdn ? 0 : l * DK) + lane * PER + c);
+#pragma unroll
+                for (int j = 0; j < ROWS_IN_FLIGHT; ++j)
+#pragma unroll
+                    for (int c = 0; c < PER; ++c) s[j][c] = fmaf(uu[l][j], wv[c], s[j][c]);
+            }
+#pragma unroll
+            for (int j = 0; j < ROWS_IN_FLIGHT; ++j) vstore<PER>(S + (size_t)(r0 + j) * DK + lane * PER, s[j]);
+        }
+        ++done;
+        __syncthreads();  // every warp is done with this stage: it takes the head NSTAGE ahead
+        if (threadIdx.x == 0 && !stall && i + kDecodeStages < mine)
+            issue(st, first + (i + kDecodeStages) * step);
+    }
+    // after a wait that gave up, the copies still in flight land before the CTA exits (bounded)
+    if (threadIdx.x == 0 && !stall) {
+        for (int i = done; i < mine && i < done + kDecodeStages; ++i)
+            tc::mbar_wait(&full[i % kDecodeStages], (i / kDecodeStages) & 1, nullptr);
     }
 }
 
@@ -294,12 +396,16 @@ template <typename IO, int DK, int LW>
 cudaError_t launch_decode_l(const ScanArgs &a, cudaStream_t s) {
     if constexpr (DK == 128) {
         if (a.dv == 128 || a.dv == 64) {
-            auto kern = a.dv == 128 ? decode_bulk_kernel<IO, 128, LW> : decode_bulk_kernel<IO, 64, LW>;
-            const int bytes = a.dv * DK * 4;
+            auto kern = a.dv == 128 ? decode_ring_kernel<IO, 128, LW> : decode_ring_kernel<IO, 64, LW>;
+            const int bytes = a.dv == 128 ? (int)RingLayout<IO, 128, LW>::BYTES : (int)RingLayout<IO, 64, LW>::BYTES;
             cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
             if (err != cudaSuccess) return err;
+            int dev = 0, sms = 148;
+            if (cudaGetDevice(&dev) == cudaSuccess)
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            const int heads = a.B * a.H;
             launch_probe_mark(s);
-            kern<<<a.B * a.H, NT, bytes, s>>>(a);
+            kern<<<heads < sms ? heads : sms, NT, bytes, s>>>(a, heads);
             return cudaGetLastError();
         }
     }

@@ -42,6 +42,31 @@ namespace {
 
 constexpr int NT = 128;  // prep threads
 
+// N consecutive TMEM columns of this thread's lane (N = 8, 16 or 32; warp-collective).
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t a, float (&v)[N]) {
+    if constexpr (N == 8) tmem_ld8(a, v);
+    else if constexpr (N == 16) tmem_ld16(a, v);
+    else tmem_ld32(a, v);
+}
+
+// N fp32 values at (row, col .. col+N-1) of K-major SW128 tiles as a bf16 hi / lo pair (N = 16, 32).
+template <int N>
+__device__ __forceinline__ void store_split_n(uint8_t *hi, uint8_t *lo, int row, int col, const float *x) {
+    if constexpr (N == 32) {
+        store32_split(hi, lo, row, col, x);
+    } else {
+#pragma unroll
+        for (int c8 = 0; c8 < N / 8; ++c8) {
+            uint4 h, l;
+            split8(x + c8 * 8, h, l);
+            const uint32_t off = sw128_off(row, col + c8 * 8, 0);
+            st16(hi, off, h);
+            st16(lo, off, l);
+        }
+    }
+}
+
 // Value-slice width of the state kernel for a key width: 4 slices of 32 at d = 128, one of 64 at
 // d = 64 (the Gated-DeltaNet route has dv = dk).
 template <int DK>
@@ -368,11 +393,11 @@ struct LPrepLayout {
     static constexpr uint32_t TCOLS = cF + 2 * DK <= 256 ? 256 : 512;
 };
 
-// 8 warps: one CTA per SM at d = 128 (its TMEM accumulators take 448 columns), two at d = 64
-// (256 columns and 112 KB of shared memory each).  Warp w reads TMEM lane quarter w % 4; warps w
-// and w + 4 split the columns of every epilogue.
+// One CTA per SM at d = 128 (its TMEM accumulators take 448 columns), with 16 warps; two CTAs per
+// SM at d = 64 (256 columns and 112 KB of shared memory each), with 8 warps.  Warp w reads TMEM lane
+// quarter w % 4; the warps sharing a quarter split the columns of every epilogue.
 template <int DK>
-constexpr int kLPrepThreads = 256;
+constexpr int kLPrepThreads = DK == 128 ? 512 : 256;
 
 template <int DK>
 __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_prep_kernel(ScanArgs p, const __grid_constant__ LMaps maps,
@@ -381,7 +406,7 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     constexpr int NTH = kLPrepThreads<DK>;
     constexpr int NH = NTH / 128;  // column splits of an epilogue
     constexpr int CW = C / NH;     // columns of G a thread owns
-    static_assert(CW == 32, "the G epilogues move 32 columns a thread");
+    static_assert(CW == 32 || CW == 16, "the G epilogues move 16 or 32 columns a thread");
     using RC = GdnRec<DK, true>;
     constexpr int DV = RC::DV, BV = RC::BV;
     extern __shared__ uint8_t smem_raw[];
@@ -514,12 +539,12 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     ok = mma_done_committed(ok);
     if (ok) {
         float gr[CW];
-        tmem_ld32(taddr(tb, 32 * q, LY::cG + cg), gr);
+        tmem_ld_n<CW>(taddr(tb, 32 * q, LY::cG + cg), gr);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < CW; ++j) gr[j] *= dec[j];
         if (q < 2) vst<CW>(sA + t_g * AS + cg, gr);
-        else store32_split(rec + RC::MQK, rec + RC::MQK + C * 128, t_g, cg, gr);
+        else store_split_n<CW>(rec + RC::MQK, rec + RC::MQK + C * 128, t_g, cg, gr);
     }
     fence_before_sync();
     __syncthreads();
@@ -542,7 +567,12 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
         }
     };
     if (ok) {
-        solve_unit_lower<NTH>(sA, sA, sTmp, tid);  // ends with a CTA barrier
+        if constexpr (NTH == 512) {  // the solve on warps 0-7
+            if (tid < 256) solve_unit_lower<256>(sA, sA, sTmp, tid, [] { named_sync(3, 256); });
+            __syncthreads();
+        } else {
+            solve_unit_lower<NTH>(sA, sA, sTmp, tid);  // ends with a CTA barrier
+        }
         store_t_pair(true);
     }
     sync_for_mma();
@@ -593,11 +623,11 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
         }
         {   // P_l (rows of K W^T, quarters 0-1) and Mqw_l (rows of Q W^T, quarters 2-3) as pairs
             float gr[CW];
-            tmem_ld32(taddr(tb, 32 * q, LY::cG + cg), gr);
+            tmem_ld_n<CW>(taddr(tb, 32 * q, LY::cG + cg), gr);
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < CW; ++j) gr[j] *= dec[j];
-            store32_split(sm + (q < 2 ? LY::P : LY::MQW), sm + (q < 2 ? LY::PL : LY::MQWL), t_g, cg, gr);
+            store_split_n<CW>(sm + (q < 2 ? LY::P : LY::MQW), sm + (q < 2 ? LY::PL : LY::MQWL), t_g, cg, gr);
         }
         if (!mbar_wait(&u_bar[l % NBU], (l / NBU) & 1, p.status, lim)) failed_sh = 1;
         for (int e = tid; e < C * (DV / 8); e += NTH) {  // D U_l as a hi / lo pair
@@ -816,12 +846,6 @@ struct StateBars {
     uint64_t drain;                      // the MMA thread's last operations
 };
 
-template <int N>
-__device__ __forceinline__ void tmem_ld_n(uint32_t a, float (&v)[N]) {
-    if constexpr (N == 8) tmem_ld8(a, v);
-    else if constexpr (N == 16) tmem_ld16(a, v);
-    else tmem_ld32(a, v);
-}
 
 // CH fp32 values at (row, j0 .. j0+CH) as a hi / lo pair into an MN-major tile of 64-column
 // 128B-swizzled blocks: hi at columns j0.., lo at BV + j0...
@@ -864,6 +888,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
     __shared__ uint32_t tmem_base_sh;
     __shared__ int failed_sh;
     __shared__ int big_sh;  // set once some |S| element of this slice exceeds kBigState
+    __shared__ int lo_sh[2];  // chunk buffer b holds Wk_lo (the load warp loads it once big_sh is set)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int v0 = blockIdx.x * BV, h = blockIdx.y, b = blockIdx.z;
@@ -887,6 +912,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
         mbar_fence_init();
         failed_sh = 0;
         big_sh = (p.flags & kForceWkLo) ? 1 : 0;
+        lo_sh[0] = lo_sh[1] = 0;
     }
     fence_before_sync();
     __syncthreads();
@@ -900,7 +926,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
     if (warp == EPI_WARPS + 1) {
         // ---------------- loads ----------------
         if (lane == 0) {
-            constexpr uint32_t bytes = 4 * (DK / 64) * C * 128 + 2 * C * 128 + LY::U_BYTES + C * 4;
+            constexpr uint32_t bytes = 3 * (DK / 64) * C * 128 + 2 * C * 128 + LY::U_BYTES + C * 4;
+            constexpr uint32_t lo_bytes = (DK / 64) * C * 128;
             int issued = -1;
             for (int c = 0; c < nch && !failed() && !(p.flags & kStallTest); ++c) {
                 if (c >= 2 && !mbar_wait(&bars.empty[c & 1], ((c - 2) >> 1) & 1, status, lim)) { fail(); break; }
@@ -908,11 +935,15 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 uint8_t *buf = sm + (c & 1) * LY::BUF;
                 uint64_t *bar = &bars.full[c & 1];
                 const int c0 = c * C;
-                mbar_expect_tx(bar, bytes);
+                // Wk_lo only once the state has grown large (the MMA warp reads lo_sh after this
+                // buffer's full barrier, which orders it after this store)
+                const bool lo = *(volatile int *)&big_sh != 0;
+                lo_sh[c & 1] = lo ? 1 : 0;
+                mbar_expect_tx(bar, bytes + (lo ? lo_bytes : 0u));
                 for (int blk = 0; blk < DK / 64; ++blk) {
                     uint8_t *dst = buf + LY::B_KWQ + blk * LY::KWQ_BLK;
                     tma_load_4d(dst, &maps.k, blk * 64, h, c0, b, bar);
-                    bulk_g2s(dst + C * 128, rec + RC::WKL + blk * RC::WK_BLK, RC::WK_BLK, bar);
+                    if (lo) bulk_g2s(dst + C * 128, rec + RC::WKL + blk * RC::WK_BLK, RC::WK_BLK, bar);
                     bulk_g2s(dst + 2 * C * 128, rec + RC::WK + blk * RC::WK_BLK, RC::WK_BLK, bar);
                     tma_load_4d(dst + 3 * C * 128, &maps.q, blk * 64, h, c0, b, bar);
                 }
@@ -920,6 +951,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 bulk_g2s(buf + LY::B_MQ + C * 128, rec + RC::MQK, C * 128, bar);   // Mqk_hi
                 bulk_g2s(buf + LY::B_U, rec + RC::U + blockIdx.x * RC::U_SLICE, LY::U_BYTES, bar);
                 bulk_g2s(buf + LY::B_G, rec + RC::G, C * 4, bar);
+                if constexpr (RL)  // the F_w slice the epilogue warps fetch a chunk ahead: into L2 now
+                    bulk_prefetch_l2(rec + RC::FW + blockIdx.x * RC::FW_SLICE, RC::FW_SLICE);
                 issued = c;
             }
             // let the copies still in flight land before the CTA can exit
@@ -948,7 +981,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 fence_after_sync();
                 const uint64_t dWQ = make_desc(bb + LY::B_KWQ + 2 * C * 128, 16, 1024, 2);
                 mma_steps<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dWQ, dS2, oKWQ, oMN, false);
-                if (*(volatile int *)&big_sh) {  // X_s += Wk_lo S (rows 64..127 hold Q S: masked)
+                if (*(volatile int *)&lo_sh[c & 1]) {  // X_s += Wk_lo S (rows 64..127 hold Q S: masked)
                     const uint64_t dLW = make_desc(bb + LY::B_KWQ + C * 128, 16, 1024, 2);
                     mma_steps_lanes<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dLW, dS2, oKWQ, oMN, true, xmask);
                 }
@@ -1007,31 +1040,36 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             watch_state();
         }
         warp_arrive(&bars.s_ready, lane);
+        // rank L: this thread's F_w elements of a chunk, fetched from the record (which the load warp
+        // prefetches into L2 two chunks ahead): a chunk ahead into registers when a thread holds 8
+        // of them, after the chunk's own Y epilogue when it holds 16 (keeping the registers of the
+        // two phases apart)
+        constexpr bool kEarlyFw = CH <= 8;
+        auto fetch_fw = [&](int cc, float (&dst)[CH]) {
+#pragma unroll
+            for (int j = 0; j < CH; ++j) dst[j] = 0.f;
+            if (RL && wr && own_d) {
+                const uint8_t *src = record<DK, RL>(p, ws, nch, cc) + RC::FW + blockIdx.x * RC::FW_SLICE;
+#pragma unroll
+                for (int j4 = 0; j4 < CH; j4 += 4) {
+                    const float4 f4 = __ldg(reinterpret_cast<const float4 *>(src + u_off<BV>(d_row, j0 + j4)));
+                    dst[j4] = f4.x;
+                    dst[j4 + 1] = f4.y;
+                    dst[j4 + 2] = f4.z;
+                    dst[j4 + 3] = f4.w;
+                }
+            }
+        };
+        float fw_next[CH];
+        if (kEarlyFw && nch > 0) fetch_fw(0, fw_next);
         bool ok = true;
         for (int c = 0; c < nch && ok; ++c) {
             const int c0 = c * C, n = min(C, T - c0);
             const uint8_t *buf = sm + (c & 1) * LY::BUF;
-            // rank L: this thread's F_w elements of the chunk, fetched from the record early (at the
-            // chunk's start when a thread holds 8 of them; after its Y epilogue when it holds 16,
-            // which keeps the registers of the two phases apart)
             float fw[CH];
 #pragma unroll
-            for (int j = 0; j < CH; ++j) fw[j] = 0.f;
-            auto fetch_fw = [&]() {
-                if (RL && wr && own_d) {
-                    const uint8_t *src = record<DK, RL>(p, ws, nch, c) + RC::FW + blockIdx.x * RC::FW_SLICE;
-#pragma unroll
-                    for (int j4 = 0; j4 < CH; j4 += 4) {
-                        const float4 f4 = __ldg(reinterpret_cast<const float4 *>(src + u_off<BV>(d_row, j0 + j4)));
-                        fw[j4] = f4.x;
-                        fw[j4 + 1] = f4.y;
-                        fw[j4 + 2] = f4.z;
-                        fw[j4 + 3] = f4.w;
-                    }
-                }
-            };
-            constexpr bool kEarlyFw = CH <= 8;
-            if (kEarlyFw) fetch_fw();
+            for (int j = 0; j < CH; ++j) fw[j] = kEarlyFw ? fw_next[j] : 0.f;
+            if (kEarlyFw && c + 1 < nch) fetch_fw(c + 1, fw_next);
             if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status, lim)) { ok = false; break; }
             const float *g = reinterpret_cast<const float *>(buf + LY::B_G);
             const float g_last = g[C - 1];
@@ -1080,7 +1118,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 store_half_pair<BV, CH>(sm + LY::DY, LY::Y_BLK, t, j0, y);
             }
             warp_arrive(&bars.y_ready, lane);
-            if (!kEarlyFw) fetch_fw();
+            if (!kEarlyFw) fetch_fw(c, fw);
             // state update S^T <- e^{g_n} S^T + K^T D Y (+ F_w)
             {
                 const float gC = __expf(g_last);
@@ -1102,10 +1140,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
 #pragma unroll
                     for (int j = 0; j < CH; ++j) Sreg[j] += xh[j] + xl[j];
                     store_half_pair<BV, CH>(sm + LY::S, LY::S_BLK, d_row, j0, Sreg);
-                    watch_state();
                 }
             }
             warp_arrive(&bars.s_ready, lane);
+            if (own_d) watch_state();  // after the hand-off, off the chain
             // output O = diag(e^g) QS + Mqk Y: the Mqk_lo rows (lanes 0..63) pass their partial
             // sums through shared memory to the threads of the output rows (lanes 64..127)
             if (!mbar_wait(&bars.d3_full, c & 1, status, lim)) { ok = false; break; }

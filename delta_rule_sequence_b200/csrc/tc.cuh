@@ -123,6 +123,11 @@ __device__ __forceinline__ void tma_prefetch_4d(const void *tmap, int x, int y, 
                  : "memory");
 }
 
+// Prefetch of `bytes` contiguous bytes into L2 (16-byte aligned, a multiple of 16; no completion).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Plain (untiled) bulk copy global -> shared, completing on `bar` (tx bytes); 16-byte aligned.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile(
