@@ -23,7 +23,7 @@
 // checkpoint into a per-CTA workspace buffer (and S_{t-1} k_t into shared memory) and walks the
 // chunk's tokens backwards.  All arithmetic is fp32 from the exact input values.
 
-#include "common.cuh"
+#include "tc.cuh"
 
 namespace prism {
 namespace {
@@ -31,7 +31,8 @@ namespace {
 constexpr int BW_NW = 16;              // value rows (warps) per CTA
 constexpr int BW_THREADS = 32 * BW_NW;
 constexpr int BW_C = 64;               // tokens between checkpoints
-constexpr int BW_TS = 8;               // tokens per flush of the cross-row sums
+constexpr int BW_TB = 8;               // tokens per staged block (and per flush of the row sums)
+constexpr int BW_SPC = BW_C / BW_TB;   // staged blocks per checkpoint interval
 
 struct BwdArgs {
     int B, H, T, dk, dv, L, nch;
@@ -42,71 +43,157 @@ struct BwdArgs {
     float *scratch;  // per CTA: [BW_C + 1][BW_NW][dk] states of the current chunk
 };
 
-template <int DK>
+// One staged block of BW_TB tokens (io type unless noted): k, q [TB][DK]; w [TB][L][DK];
+// u [TB][L][NW] (or v [TB][NW]) and dO [TB][NW] for this CTA's NW rows; alpha, beta [TB] fp32.
+template <typename IO, int DK>
+struct BwdStage {
+    static constexpr uint32_t K = 0;
+    static constexpr uint32_t Q = K + BW_TB * DK * sizeof(IO);
+    static constexpr uint32_t W = Q + BW_TB * DK * sizeof(IO);
+    // u (or v: one "rank") slot, then dO, then alpha / beta; L = 0 on the Gated-DeltaNet write
+    __host__ __device__ static uint32_t U(int L) { return W + BW_TB * L * DK * sizeof(IO); }
+    __host__ __device__ static uint32_t DO(int L) { return U(L) + BW_TB * (L > 0 ? L : 1) * BW_NW * sizeof(IO); }
+    __host__ __device__ static uint32_t AB(int L) { return DO(L) + BW_TB * BW_NW * sizeof(IO); }
+    __host__ __device__ static uint32_t bytes(int L) { return (AB(L) + 2 * BW_TB * 4 + 15) & ~15u; }
+};
+
+template <typename IO, int DK>
 struct BwdSmem {
-    // cross-row sums of BW_TS tokens: dq, dk, dw (L ranks), dalpha, dbeta; S_{t-1} k_t per warp
+    // two staged blocks; cross-row sums of a block: dq, dk, dw (L ranks), dalpha, dbeta; S_{t-1} k_t
     static size_t bytes(int L) {
-        return sizeof(float) * ((size_t)(2 + L) * BW_TS * DK + 2 * BW_TS + (size_t)BW_NW * BW_C);
+        return 2 * (size_t)BwdStage<IO, DK>::bytes(L) +
+               sizeof(float) * ((size_t)(2 + L) * BW_TB * DK + 2 * BW_TB + (size_t)BW_NW * BW_C);
     }
 };
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc::smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <typename IO, int DK>
 __global__ void __launch_bounds__(BW_THREADS) scan_bwd_kernel(BwdArgs p) {
     constexpr int E = DK / 32;  // columns per lane
-    extern __shared__ float smem[];
+    using SG = BwdStage<IO, DK>;
+    extern __shared__ __align__(16) uint8_t smem[];
     const int L = p.L;
-    float *acc_dq = smem;                      // [BW_TS][DK]
-    float *acc_dk = acc_dq + BW_TS * DK;       // [BW_TS][DK]
-    float *acc_dw = acc_dk + BW_TS * DK;       // [BW_TS][L][DK]
-    float *acc_da = acc_dw + (size_t)BW_TS * L * DK;  // [BW_TS]
-    float *acc_db = acc_da + BW_TS;            // [BW_TS]
-    float *pk_all = acc_db + BW_TS;            // [BW_NW][BW_C]
+    const bool gdn = p.u == nullptr;
+    const int Lw = gdn ? 0 : L;                       // staged write ranks
+    const uint32_t SB = SG::bytes(Lw);
+    float *acc_dq = reinterpret_cast<float *>(smem + 2 * SB);   // [TB][DK]
+    float *acc_dk = acc_dq + BW_TB * DK;                        // [TB][DK]
+    float *acc_dw = acc_dk + BW_TB * DK;                        // [TB][L][DK]
+    float *acc_da = acc_dw + (size_t)BW_TB * Lw * DK;           // [TB]
+    float *acc_db = acc_da + BW_TB;                             // [TB]
+    float *pk_all = acc_db + BW_TB;                             // [NW][C]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int r = blockIdx.x * BW_NW + warp;   // value row of this warp
+    const int r0 = blockIdx.x * BW_NW, r = r0 + warp;  // this warp's value row
     const int h = blockIdx.y, b = blockIdx.z;
     const int H = p.H, T = p.T, dv = p.dv, nch = p.nch;
-    const bool gdn = p.u == nullptr;
     const size_t head = (size_t)b * H + h;
     const IO *q = (const IO *)p.q, *k = (const IO *)p.k, *v = (const IO *)p.v;
     const IO *u = (const IO *)p.u, *w = (const IO *)p.w, *dO = (const IO *)p.dO;
     float *pk = pk_all + warp * BW_C;
     const size_t cta = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
     float *scr = p.scratch + cta * (size_t)(BW_C + 1) * BW_NW * DK + warp * DK;  // + i * NW * DK
-
     auto tok = [&](int t) { return ((size_t)b * T + t) * H + h; };  // index of (b, t, h)
-    auto load_row = [&](const IO *base, size_t off, float (&x)[E]) {
-#pragma unroll
-        for (int i = 0; i < E; ++i) x[i] = ld_io<IO>(base, off + lane + 32 * i);
+    auto ckpt_row = [&](int c) { return p.ckpt + (((head * nch + c) * dv) + r) * DK; };
+
+    // ---- staging of token blocks (cp.async, all threads)
+    const int nsb = (T + BW_TB - 1) / BW_TB;
+    auto stage = [&](int buf, int sb) {
+        uint8_t *st = smem + buf * SB;
+        const int t0 = sb * BW_TB, m = min(BW_TB, T - t0);
+        constexpr int RC = DK * sizeof(IO) / 16;          // 16-byte pieces of a k / q / w row
+        constexpr int NC = BW_NW * sizeof(IO) / 16;       // pieces of a 16-row slice
+        const int nk = m * RC, nw = m * Lw * RC, nu = m * Lw * NC, nd = m * NC;
+        const int nv = gdn ? m * NC : 0;
+        const int total = 2 * nk + nw + nu + nd + nv + 2 * m;
+        for (int e = tid; e < total; e += BW_THREADS) {
+            int x = e;
+            if (x < 2 * nk) {  // k, q rows
+                const int which = x / nk, y = x % nk, i = y / RC, pc = y % RC;
+                const IO *src = (which ? q : k) + tok(t0 + i) * DK;
+                cp_async16(st + (which ? SG::Q : SG::K) + (i * DK) * sizeof(IO) + pc * 16,
+                           reinterpret_cast<const uint8_t *>(src) + pc * 16);
+                continue;
+            }
+            x -= 2 * nk;
+            if (x < nw) {  // w rows
+                const int i = x / (Lw * RC), l = (x / RC) % Lw, pc = x % RC;
+                cp_async16(st + SG::W + ((i * Lw + l) * DK) * sizeof(IO) + pc * 16,
+                           reinterpret_cast<const uint8_t *>(w + (tok(t0 + i) * L + l) * DK) + pc * 16);
+                continue;
+            }
+            x -= nw;
+            if (x < nu) {  // u slices of this CTA's rows
+                const int i = x / (Lw * NC), l = (x / NC) % Lw, pc = x % NC;
+                cp_async16(st + SG::U(Lw) + ((i * Lw + l) * BW_NW) * sizeof(IO) + pc * 16,
+                           reinterpret_cast<const uint8_t *>(u + (tok(t0 + i) * L + l) * dv + r0) + pc * 16);
+                continue;
+            }
+            x -= nu;
+            if (x < nd + nv) {  // dO slices, then v slices (into the u slot on the GDN write)
+                const bool isv = x >= nd;
+                const int y = isv ? x - nd : x, i = y / NC, pc = y % NC;
+                const IO *src = (isv ? v : dO) + tok(t0 + i) * dv + r0;
+                cp_async16(st + (isv ? SG::U(Lw) : SG::DO(Lw)) + (i * BW_NW) * sizeof(IO) + pc * 16,
+                           reinterpret_cast<const uint8_t *>(src) + pc * 16);
+                continue;
+            }
+            x -= nd + nv;
+            {  // alpha, beta
+                const int which = x / m, i = x % m;
+                cp_async4(st + SG::AB(Lw) + (which * BW_TB + i) * 4, (which ? p.beta : p.alpha) + tok(t0 + i));
+            }
+        }
     };
+    // staged values of token i of the block in buffer `buf`
+    auto sk = [&](int buf, int i, int c) { return ld_io<IO>((const IO *)(smem + buf * SB + SG::K), i * DK + c); };
+    auto sq = [&](int buf, int i, int c) { return ld_io<IO>((const IO *)(smem + buf * SB + SG::Q), i * DK + c); };
+    auto sw = [&](int buf, int i, int l, int c) {
+        return ld_io<IO>((const IO *)(smem + buf * SB + SG::W), (i * Lw + l) * DK + c);
+    };
+    auto su = [&](int buf, int i, int l) {  // u_{t,l} of this warp's row (v_t on the GDN write)
+        return ld_io<IO>((const IO *)(smem + buf * SB + SG::U(Lw)), (i * (gdn ? 1 : Lw) + l) * BW_NW + warp);
+    };
+    auto sdo = [&](int buf, int i) { return ld_io<IO>((const IO *)(smem + buf * SB + SG::DO(Lw)), i * BW_NW + warp); };
+    auto sa = [&](int buf, int i) { return reinterpret_cast<const float *>(smem + buf * SB + SG::AB(Lw))[i]; };
+    auto sbeta = [&](int buf, int i) { return reinterpret_cast<const float *>(smem + buf * SB + SG::AB(Lw))[BW_TB + i]; };
+
     auto dot = [&](const float (&a)[E], const float (&c)[E]) {
         float s = 0.f;
 #pragma unroll
         for (int i = 0; i < E; ++i) s = fmaf(a[i], c[i], s);
         return warp_sum(s);
     };
-    // one forward step of row r at token t; returns S_{t-1} k_t (of this row)
-    auto step = [&](float (&s)[E], int t) -> float {
+    // one forward step of this warp's row at staged token i; returns S_{t-1} k_t of the row
+    auto step = [&](float (&s)[E], int buf, int i) -> float {
         float kk[E];
-        load_row(k, tok(t) * DK, kk);
-        const float sk = dot(s, kk);
-        const float a = p.alpha[tok(t)], be = p.beta[tok(t)];
 #pragma unroll
-        for (int i = 0; i < E; ++i) s[i] = a * fmaf(-be * sk, kk[i], s[i]);
+        for (int e = 0; e < E; ++e) kk[e] = sk(buf, i, lane + 32 * e);
+        const float sk_ = dot(s, kk);
+        const float a = sa(buf, i), be = sbeta(buf, i);
+#pragma unroll
+        for (int e = 0; e < E; ++e) s[e] = a * fmaf(-be * sk_, kk[e], s[e]);
         if (gdn) {
-            const float bv = be * ld_io<IO>(v, tok(t) * dv + r);
+            const float bv = be * su(buf, i, 0);
 #pragma unroll
-            for (int i = 0; i < E; ++i) s[i] = fmaf(bv, kk[i], s[i]);
+            for (int e = 0; e < E; ++e) s[e] = fmaf(bv, kk[e], s[e]);
         } else {
             for (int l = 0; l < L; ++l) {
-                float ww[E];
-                load_row(w, (tok(t) * L + l) * DK, ww);
-                const float ur = ld_io<IO>(u, (tok(t) * L + l) * dv + r);
+                const float ur = su(buf, i, l);
 #pragma unroll
-                for (int i = 0; i < E; ++i) s[i] = fmaf(ur, ww[i], s[i]);
+                for (int e = 0; e < E; ++e) s[e] = fmaf(ur, sw(buf, i, l, lane + 32 * e), s[e]);
             }
         }
-        return sk;
+        return sk_;
     };
     auto store_state = [&](float *dst, const float (&s)[E]) {
 #pragma unroll
@@ -116,125 +203,162 @@ __global__ void __launch_bounds__(BW_THREADS) scan_bwd_kernel(BwdArgs p) {
 #pragma unroll
         for (int i = 0; i < E; ++i) s[i] = src[lane + 32 * i];
     };
-    auto ckpt_row = [&](int c) { return p.ckpt + (((head * nch + c) * dv) + r) * DK; };
 
-    // 1. forward over the whole sequence, checkpointing this row at every chunk start
-    float s[E];
+    // ---- the schedule: the forward sweep over every block, then for each checkpoint interval from
+    // the last: its blocks forwards (recomputing the states), then backwards
+    enum { kFwd, kRecomp, kRev };
+    const int last_sb = (nch - 1) * BW_SPC, m_last = nsb - last_sb;  // blocks of the last interval
+    auto schedule = [&](int j, int &sb, int &mode) {
+        if (j < nsb) { sb = j; mode = kFwd; return; }
+        int j2 = j - nsb, c, kk, m;
+        if (j2 < 2 * m_last) {
+            c = nch - 1; kk = j2; m = m_last;
+        } else {
+            const int jj = j2 - 2 * m_last;
+            c = nch - 2 - jj / (2 * BW_SPC); kk = jj % (2 * BW_SPC); m = BW_SPC;
+        }
+        mode = kk < m ? kRecomp : kRev;
+        sb = c * BW_SPC + (kk < m ? kk : 2 * m - 1 - kk);
+    };
+    const int steps = 3 * nsb;
+
+    float s[E], g[E];
     if (p.S0) load_state(p.S0 + (head * dv + r) * DK, s);
     else {
 #pragma unroll
         for (int i = 0; i < E; ++i) s[i] = 0.f;
     }
-    for (int c = 0; c < nch; ++c) {
-        store_state(ckpt_row(c), s);
-        const int c0 = c * BW_C, n = min(BW_C, T - c0);
-        for (int i = 0; i < n; ++i) step(s, c0 + i);
-    }
-
-    // 2. backward, chunk by chunk from the last
-    float g[E];
     if (p.dS_final) load_state(p.dS_final + (head * dv + r) * DK, g);
     else {
 #pragma unroll
         for (int i = 0; i < E; ++i) g[i] = 0.f;
     }
-    const int acc_n = (2 + L) * BW_TS * DK + 2 * BW_TS;
-    for (int e = tid; e < acc_n; e += BW_THREADS) smem[e] = 0.f;
-    __syncthreads();
-    for (int c = nch - 1; c >= 0; --c) {
-        const int c0 = c * BW_C, n = min(BW_C, T - c0);
-        // the chunk's states S_{c0-1+i} (i = 0..n) and S_{t-1} k_t, recomputed from the checkpoint
-        load_state(ckpt_row(c), s);
-        store_state(scr, s);
-        for (int i = 0; i < n; ++i) {
-            const float sk = step(s, c0 + i);
-            if (lane == 0) pk[i] = sk;
-            store_state(scr + (size_t)(i + 1) * BW_NW * DK, s);
+    const int acc_n = (2 + Lw) * BW_TB * DK + 2 * BW_TB;
+    for (int e = tid; e < acc_n; e += BW_THREADS) acc_dq[e] = 0.f;
+
+    if (steps > 0) {
+        int sb0, md0;
+        schedule(0, sb0, md0);
+        stage(0, sb0);
+    }
+    cp_async_commit();
+    for (int j = 0; j < steps; ++j) {
+        const int buf = j & 1;
+        if (j + 1 < steps) {
+            int sbn, mdn;
+            schedule(j + 1, sbn, mdn);
+            stage(buf ^ 1, sbn);
         }
-        __syncwarp();
-        for (int i = n - 1; i >= 0; --i) {
-            const int t = c0 + i, slot = i % BW_TS;
-            float sp[E], sc[E], kk[E], qq[E];
-            load_state(scr + (size_t)i * BW_NW * DK, sp);
-            load_state(scr + (size_t)(i + 1) * BW_NW * DK, sc);
-            load_row(k, tok(t) * DK, kk);
-            load_row(q, tok(t) * DK, qq);
-            const float dd = ld_io<IO>(dO, tok(t) * dv + r);
-            const float a = p.alpha[tok(t)], be = p.beta[tok(t)];
-            const float Pk = pk[i];
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                g[e] = fmaf(dd, qq[e], g[e]);
-                atomicAdd(&acc_dq[slot * DK + lane + 32 * e], dd * sc[e]);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        int sb, mode;
+        schedule(j, sb, mode);
+        const int t0 = sb * BW_TB, m = min(BW_TB, T - t0);
+        const int c = sb / BW_SPC, ci0 = (sb % BW_SPC) * BW_TB;  // interval, first index in it
+        if (mode == kFwd) {
+            if (ci0 == 0) store_state(ckpt_row(c), s);
+            for (int i = 0; i < m; ++i) step(s, buf, i);
+        } else if (mode == kRecomp) {
+            if (ci0 == 0) {
+                load_state(ckpt_row(c), s);
+                store_state(scr, s);
             }
-            const float Gk = dot(g, kk), gs = dot(g, sp);
-            float da = gs - be * Pk * Gk, db = -a * Pk * Gk;
-            const float ab = a * be;
-            float dk_[E];
+            for (int i = 0; i < m; ++i) {
+                const float pki = step(s, buf, i);
+                if (lane == 0) pk[ci0 + i] = pki;
+                store_state(scr + (size_t)(ci0 + i + 1) * BW_NW * DK, s);
+            }
+        } else {
+            __syncwarp();
+            // the block's states S_{t0-1} .. S_{t0+m-1} of this row, all loads issued at once
+            float st[BW_TB + 1][E];
 #pragma unroll
-            for (int e = 0; e < E; ++e) dk_[e] = -ab * fmaf(g[e], Pk, sp[e] * Gk);
-            if (gdn) {
-                const float vr = ld_io<IO>(v, tok(t) * dv + r);
-                db = fmaf(vr, Gk, db);
+            for (int i = 0; i <= BW_TB; ++i)
+                if (i <= m) load_state(scr + (size_t)(ci0 + i) * BW_NW * DK, st[i]);
 #pragma unroll
-                for (int e = 0; e < E; ++e) dk_[e] = fmaf(be * vr, g[e], dk_[e]);
-                if (lane == 0) p.dv_out[tok(t) * dv + r] = be * Gk;
-            } else {
-                for (int l = 0; l < L; ++l) {
-                    float ww[E];
-                    load_row(w, (tok(t) * L + l) * DK, ww);
-                    const float ur = ld_io<IO>(u, (tok(t) * L + l) * dv + r);
-                    const float dul = dot(g, ww);
-                    if (lane == 0) p.du[(tok(t) * L + l) * dv + r] = dul;
+            for (int i = BW_TB - 1; i >= 0; --i) {
+                if (i >= m) continue;
+                const int t = t0 + i;
+                float kk[E], qq[E];
 #pragma unroll
-                    for (int e = 0; e < E; ++e)
-                        atomicAdd(&acc_dw[((size_t)slot * L + l) * DK + lane + 32 * e], ur * g[e]);
+                for (int e = 0; e < E; ++e) {
+                    kk[e] = sk(buf, i, lane + 32 * e);
+                    qq[e] = sq(buf, i, lane + 32 * e);
                 }
-            }
+                const float dd = sdo(buf, i);
+                const float a = sa(buf, i), be = sbeta(buf, i);
+                const float Pk = pk[ci0 + i];
 #pragma unroll
-            for (int e = 0; e < E; ++e) atomicAdd(&acc_dk[slot * DK + lane + 32 * e], dk_[e]);
-            if (lane == 0) {
-                atomicAdd(&acc_da[slot], da);
-                atomicAdd(&acc_db[slot], db);
-            }
-#pragma unroll
-            for (int e = 0; e < E; ++e) g[e] = a * fmaf(-be * Gk, kk[e], g[e]);
-            if (slot == 0) {
-                // tokens i .. i + m - 1 of the chunk are complete: add this CTA's row sums to the
-                // global gradients, then clear the slots
-                __syncthreads();
-                const int m = min(BW_TS, n - i);
-                for (int e = tid; e < m * DK; e += BW_THREADS) {
-                    const int sl = e / DK, j = e % DK;
-                    const size_t o = tok(t + sl) * DK + j;
-                    atomicAdd(&p.dq[o], acc_dq[sl * DK + j]);
-                    atomicAdd(&p.dk_out[o], acc_dk[sl * DK + j]);
-                    acc_dq[sl * DK + j] = 0.f;
-                    acc_dk[sl * DK + j] = 0.f;
+                for (int e = 0; e < E; ++e) {
+                    g[e] = fmaf(dd, qq[e], g[e]);
+                    atomicAdd(&acc_dq[i * DK + lane + 32 * e], dd * st[i + 1][e]);
                 }
-                if (!gdn) {
-                    for (int e = tid; e < m * L * DK; e += BW_THREADS) {
-                        const int sl = e / (L * DK), l = (e / DK) % L, j = e % DK;
-                        atomicAdd(&p.dw[(tok(t + sl) * L + l) * DK + j], acc_dw[e]);
-                        acc_dw[e] = 0.f;
+                const float Gk = dot(g, kk), gs = dot(g, st[i]);
+                float da = gs - be * Pk * Gk, db = -a * Pk * Gk;
+                const float ab = a * be;
+                float dk_[E];
+#pragma unroll
+                for (int e = 0; e < E; ++e) dk_[e] = -ab * fmaf(g[e], Pk, st[i][e] * Gk);
+                if (gdn) {
+                    const float vr = su(buf, i, 0);
+                    db = fmaf(vr, Gk, db);
+#pragma unroll
+                    for (int e = 0; e < E; ++e) dk_[e] = fmaf(be * vr, g[e], dk_[e]);
+                    if (lane == 0) p.dv_out[tok(t) * dv + r] = be * Gk;
+                } else {
+                    for (int l = 0; l < L; ++l) {
+                        float ww[E];
+#pragma unroll
+                        for (int e = 0; e < E; ++e) ww[e] = sw(buf, i, l, lane + 32 * e);
+                        const float ur = su(buf, i, l);
+                        const float dul = dot(g, ww);
+                        if (lane == 0) p.du[(tok(t) * L + l) * dv + r] = dul;
+#pragma unroll
+                        for (int e = 0; e < E; ++e)
+                            atomicAdd(&acc_dw[((size_t)i * Lw + l) * DK + lane + 32 * e], ur * g[e]);
                     }
                 }
-                if (tid < m) {
-                    atomicAdd(&p.dalpha[tok(t + tid)], acc_da[tid]);
-                    atomicAdd(&p.dbeta[tok(t + tid)], acc_db[tid]);
-                    acc_da[tid] = 0.f;
-                    acc_db[tid] = 0.f;
+#pragma unroll
+                for (int e = 0; e < E; ++e) atomicAdd(&acc_dk[i * DK + lane + 32 * e], dk_[e]);
+                if (lane == 0) {
+                    atomicAdd(&acc_da[i], da);
+                    atomicAdd(&acc_db[i], db);
                 }
-                __syncthreads();
+#pragma unroll
+                for (int e = 0; e < E; ++e) g[e] = a * fmaf(-be * Gk, kk[e], g[e]);
+            }
+            // the block's row sums from this CTA into the global gradients, then clear them
+            __syncthreads();
+            for (int e = tid; e < m * DK; e += BW_THREADS) {
+                const int sl = e / DK, jc = e % DK;
+                const size_t o = tok(t0 + sl) * DK + jc;
+                atomicAdd(&p.dq[o], acc_dq[e]);
+                atomicAdd(&p.dk_out[o], acc_dk[e]);
+                acc_dq[e] = 0.f;
+                acc_dk[e] = 0.f;
+            }
+            for (int e = tid; e < m * Lw * DK; e += BW_THREADS) {
+                const int sl = e / (Lw * DK), l = (e / DK) % Lw, jc = e % DK;
+                atomicAdd(&p.dw[(tok(t0 + sl) * L + l) * DK + jc], acc_dw[e]);
+                acc_dw[e] = 0.f;
+            }
+            if (tid < m) {
+                atomicAdd(&p.dalpha[tok(t0 + tid)], acc_da[tid]);
+                atomicAdd(&p.dbeta[tok(t0 + tid)], acc_db[tid]);
+                acc_da[tid] = 0.f;
+                acc_db[tid] = 0.f;
             }
         }
+        __syncthreads();  // the block's buffer is free for the block two steps ahead
     }
+    cp_async_wait<0>();
     if (p.dS0) store_state(p.dS0 + (head * dv + r) * DK, g);
 }
 
 template <typename IO, int DK>
 cudaError_t launch_bwd_t(const BwdArgs &a, cudaStream_t s) {
-    const size_t bytes = BwdSmem<DK>::bytes(a.L);
+    const size_t bytes = BwdSmem<IO, DK>::bytes(a.u == nullptr ? 0 : a.L);
     auto kern = scan_bwd_kernel<IO, DK>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (err != cudaSuccess) return err;

@@ -537,6 +537,9 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
         }
     }
     ok = mma_done_committed(ok);
+    // the record is written by bulk stores from shared memory that is idle at that point (Mqk over
+    // the lo [P; Mqw] tiles, the Wk pair over the D U tiles, O_w over K / Q, F_w over W / U):
+    // whole contiguous pieces instead of 16-byte stores to 64 different rows per warp
     if (ok) {
         float gr[CW];
         tmem_ld_n<CW>(taddr(tb, 32 * q, LY::cG + cg), gr);
@@ -544,10 +547,15 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
 #pragma unroll
         for (int j = 0; j < CW; ++j) gr[j] *= dec[j];
         if (q < 2) vst<CW>(sA + t_g * AS + cg, gr);
-        else store_split_n<CW>(rec + RC::MQK, rec + RC::MQK + C * 128, t_g, cg, gr);
+        else store_split_n<CW>(sm + LY::PL, sm + LY::MQWL, t_g, cg, gr);
     }
+    fence_async_smem();
     fence_before_sync();
     __syncthreads();
+    if (ok && tid == 0) {  // Mqk hi then lo: the PL and MQWL tiles are adjacent, as in the record
+        bulk_s2g(rec + RC::MQK, sm + LY::PL, 2 * C * 128);
+        bulk_commit();
+    }
     // T pair tiles: T diag(beta gamma) for Wk, then T itself for X_u
     auto store_t_pair = [&](bool scaled) {
         for (int e = tid; e < C * (C / 8); e += NTH) {
@@ -592,11 +600,19 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
             float x[32];
             tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
             tmem_wait_ld();
-            if (own_t) store32_split(rec + RC::WK, rec + RC::WKL, t_row, cc, x, RC::WK_BLK);
+            if (own_t) store32_split(sm + LY::DU, sm + LY::DUL, t_row, cc, x, LY::BLK);
         }
     }
+    fence_async_smem();
     fence_before_sync();
     __syncthreads();
+    if (ok && tid == 0) {  // Wk hi then lo: DU and DUL are adjacent, as WK and WKL in the record
+        static_assert(LY::DUL == LY::DU + RC::WK_BLK * (DK / 64) && RC::WKL == RC::WK + RC::WK_BLK * (DK / 64) &&
+                          LY::BLK == RC::WK_BLK,
+                      "the staged Wk pair has the record's layout");
+        bulk_s2g(rec + RC::WK, sm + LY::DU, 2 * RC::WK_BLK * (DK / 64));
+        bulk_commit();
+    }
     if (ok) store_t_pair(false);  // the Wk MMA has completed: the T tiles are free
 
     // the write terms, one rank at a time.  G_l = [K; Q] W_l^T is issued together with the
@@ -609,6 +625,7 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     if (ok && tid == 0) {
         if (mbar_wait(&w_bar[0], 0, p.status, lim)) issue_g(0);
         else failed_sh = 1;
+        bulk_wait_read();  // the staged Mqk and Wk are read out: the rank loop writes those tiles
     }
     ok = mma_done(ok);
     for (int l = 0; l < L && ok; ++l) {
@@ -669,7 +686,7 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
         }
     }
     // [sum P U; O_w]: the sum P U rows (lane quarters 0-1) become a hi / lo pair over the D U
-    // tiles, the O_w rows (quarters 2-3) go straight to the record
+    // tiles, the O_w rows (quarters 2-3) are staged over K / Q ([C][DV] fp32, the record's layout)
     if (ok) {
         const int t = 32 * (q & 1) + lane;
 #pragma unroll
@@ -687,7 +704,7 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
                     st16(sm + LY::DUL, off, lv);
                 }
             } else {
-                float *dst = reinterpret_cast<float *>(rec + RC::OW) + (size_t)t * DV + cc;
+                float *dst = reinterpret_cast<float *>(sm + LY::KQ) + (size_t)t * DV + cc;
 #pragma unroll
                 for (int j4 = 0; j4 < 32; j4 += 4)
                     *reinterpret_cast<float4 *>(dst + j4) = make_float4(x[j4], x[j4 + 1], x[j4 + 2], x[j4 + 3]);
@@ -695,6 +712,12 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
         }
     }
     sync_for_mma();
+    static_assert(C * DV * 4 <= LY::KQ_BLK * (DK / 64), "O_w fits over K and Q");
+    static_assert(RC::FW_SLICE * (DV / BV) <= LY::DU - LY::W, "F_w fits over W and U");
+    if (ok && tid == 0) {
+        bulk_s2g(rec + RC::OW, sm + LY::KQ, C * DV * 4);
+        bulk_commit();
+    }
     // X_u = T (sum P U)  (M = 64, into the same columns)
     if (ok && tid == 0) {
         const uint64_t dPU = make_desc(sb + LY::DU, LY::BLK, 1024, 2);
@@ -716,16 +739,24 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
             tmem_ld16(taddr(tb, 32 * q, LY::cF + cc), xh);
             tmem_ld16(taddr(tb, 32 * q, LY::cF + DV + cc), xl);
             tmem_wait_ld();
-            if (own_d) {
+            if (own_d) {  // staged over W / U in the record's layout
 #pragma unroll
                 for (int j4 = 0; j4 < 16; j4 += 4) {
                     const int j = cc + j4;
-                    *reinterpret_cast<float4 *>(rec + RC::FW + (j / BV) * RC::FW_SLICE + u_off<BV>(d_row, j % BV)) =
+                    *reinterpret_cast<float4 *>(sm + LY::W + (j / BV) * RC::FW_SLICE + u_off<BV>(d_row, j % BV)) =
                         make_float4(xh[j4] + xl[j4], xh[j4 + 1] + xl[j4 + 1], xh[j4 + 2] + xl[j4 + 2],
                                     xh[j4 + 3] + xl[j4 + 3]);
                 }
             }
         }
+    }
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    if (ok && tid == 0) {
+        bulk_s2g(rec + RC::FW, sm + LY::W, RC::FW_SLICE * (DV / BV));
+        bulk_commit();
+        bulk_wait_read_n<1>();  // the O_w store has read K / Q, where -X_u is staged next
     }
     ok = mma_done_committed(ok);
     // -X_u -> the U slot (staged over K and Q in the record's slice layout, one bulk store)
@@ -770,49 +801,58 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
 // ------------------------------------------------------------------------------------------------
 // state: one CTA per (value slice, head, batch), chunks in order
 //
-// Two MMA stages per chunk (8 instructions at d = 128 for the first, 4 + 4 for the second):
+// Two MMA stages per chunk (8 instructions at d = 128 for the first, 4 + 8 for the second):
 //   stage 1:  D1 = [Wk; Q] [S_hi | S_lo]                    (M = 128, N = 2 BV: X_s and QS)
-//             D1 += [Wk_lo; Wk] [S_hi | S_lo], TMEM lanes 64..127 masked off (only X_s gains the
+//             D1 += [Wk_lo; *] [S_hi | S_lo], TMEM lanes 64..127 masked off (only X_s gains the
 //             Wk_lo term), once the state of this CTA has grown past kBigState
 //   stage 2:  D4 = K^T [DY_hi | DY_lo]                      (the state update, on the chain)
-//             D3 = [Mqk_lo; Mqk_hi] [Y_hi | Y_lo]           (the output's intra-chunk term)
-// X_s and the Mqk_lo product sit in TMEM lanes 0..63, QS and the Mqk_hi product in lanes 64..127,
-// so the Y epilogue runs on sub-partitions 0-1 and the output epilogue on 2-3, where it does not
-// slow the MMA warp (sub-partition 0) issuing the next chunk's stage 1.  D1 is double-buffered in
-// TMEM.  K, Q arrive by TMA tiled loads, the per-chunk record (Wk, Wk_lo, Mqk, the U slice, g) by
-// bulk copies, into two chunk buffers: chunk c + 2 loads into chunk c's buffer as soon as its last
-// readers (the stage 2 MMAs and the Y epilogue) are done.  On the rank-L route the epilogue warps
-// fetch their F_w and O_w elements of a chunk straight from the record into registers.
+//             D3 = [Mqk_lo; Mqk_hi] [Y_hi | Y_lo], then D3 += [*; Mqk_lo] [Y_hi | Y_lo] with lanes
+//             0..63 masked off                              (the output's intra-chunk term)
+// X_s sits in TMEM lanes 0..63, QS and the whole Mqk Y term in lanes 64..127, so the Y epilogue
+// runs on sub-partitions 0-1 and the output epilogue on 2-3, where it does not slow the MMA warp
+// (sub-partition 0) issuing the next chunk's stage 1.  D1 is double-buffered in TMEM.  K, Q arrive
+// by TMA tiled loads, the per-chunk record (Wk, Mqk, the U slice, g, and on the rank-L route the
+// F_w slice) by bulk copies, into two chunk buffers: chunk c + 2 loads into chunk c's buffer as soon
+// as its last readers (the stage 2 MMAs and the state epilogue's F_w read) are done.
 //
 // Precision of X_s = Wk S^T: Wk is a rounded intermediate result, so its single-bf16 error (2^-9
 // relative) reaches Y scaled by |S|.  For states of order one that stays far below the bf16
 // tolerance, but writes with large directions (|w| ~ 8) grow the state into the hundreds.  Each
-// CTA therefore watches the largest |S| element of its slice and, from the chunk after it first
-// exceeds kBigState, adds the Wk_lo S term (Wk_lo = bf16(Wk - Wk_hi)) to X_s: 8 more MMAs on the
-// chain at d = 128.
+// CTA therefore watches the largest |S| element of its slice and, once one exceeds kBigState, adds
+// the Wk_lo S term (Wk_lo = bf16(Wk - Wk_hi)): the MMA thread loads the next chunk's Wk_lo over
+// the Y / D Y tiles (free between a chunk's stage 2 MMAs and the next chunk's Y epilogue) and
+// issues 8 more MMAs on the chain at d = 128.
 
 template <int DK, bool RL = false>
 struct StateLayout {
     static constexpr int BV = kBV<DK>;
     static constexpr int N2 = 2 * BV;                     // hi | lo side by side
     static constexpr int CH = BV / 4;                     // columns of one epilogue warp
-    static constexpr uint32_t KWQ_BLK = 4 * C * 128;      // [K; Wk_lo; Wk; Q] rows of one 64-col block
+    static constexpr uint32_t KWQ_BLK = 3 * C * 128;      // [K; Wk; Q] rows of one 64-col block
     static constexpr uint32_t U_BYTES = C * BV * 4;
     // double-buffered chunk inputs
     static constexpr uint32_t B_KWQ = 0;
     static constexpr uint32_t B_MQ = B_KWQ + KWQ_BLK * (DK / 64);   // [Mqk_lo; Mqk_hi]
     static constexpr uint32_t B_U = B_MQ + 2 * C * 128;
     static constexpr uint32_t B_G = B_U + U_BYTES;                   // g (64 floats)
-    static constexpr uint32_t BUF = B_G + 1024;
-    // S^T [d][hi | lo], Y [t][hi | lo], D Y [t][hi | lo]: MN-major, 64-column blocks
-    static constexpr uint32_t S_BLK = DK * 128;
-    static constexpr uint32_t S = 2 * BUF;
+    static constexpr uint32_t FW_BYTES = RL ? DK * BV * 4 : 0;       // F_w slice (rank L)
+    static constexpr uint32_t B_FW = B_G + 1024;
+    static constexpr uint32_t BUF = B_FW + FW_BYTES;
+    // Y [t][hi | lo], D Y [t][hi | lo], S^T [d][hi | lo]: MN-major, 64-column blocks.  Y and D Y
+    // are free from the completion of a chunk's stage 2 MMAs to its Y epilogue: Wk_lo of the next
+    // chunk (one 64-row K-major tile per 64 columns) is loaded over them when it is needed.
     static constexpr uint32_t Y_BLK = C * 128;
-    static constexpr uint32_t Y = S + S_BLK * (N2 / 64);
+    static constexpr uint32_t Y = 2 * BUF;
     static constexpr uint32_t DY = Y + Y_BLK * (N2 / 64);
-    static constexpr int OXS = BV + 4;                      // fp32 row stride of the output exchange
-    static constexpr uint32_t OX = DY + Y_BLK * (N2 / 64);
-    static constexpr uint32_t BYTES = OX + C * OXS * 4 + 1024;
+    static constexpr uint32_t WKL = Y;
+    static constexpr uint32_t WKL_BLK = C * 128;
+    static constexpr uint32_t S_BLK = DK * 128;
+    static constexpr uint32_t S = DY + Y_BLK * (N2 / 64);
+    static constexpr uint32_t BYTES = S + S_BLK * (N2 / 64) + 1024;
+    // the lane-masked Wk_lo MMA reads 128 rows from each 64-column block of Wk_lo: the rows past
+    // the last block (masked) are still inside the allocation
+    static_assert(WKL + WKL_BLK * (DK / 64) + WKL_BLK <= BYTES - 1024, "masked rows stay in bounds");
+    static_assert(WKL_BLK * (DK / 64) <= 2 * Y_BLK * (N2 / 64), "Wk_lo fits over Y and D Y");
     // TMEM columns: D1 (two buffers), D3, D4
     static constexpr uint32_t cD1 = 0, cD3 = 2 * N2, cD4 = 3 * N2;
     static constexpr uint32_t TCOLS = 4 * N2 <= 256 ? 256 : 512;
@@ -828,12 +868,18 @@ constexpr int ST_THREADS = EPI_THREADS + 64;
 // Largest |S| element below which X_s = Wk S^T is taken with Wk as one bf16 (its rounding then
 // moves Y by at most a few per cent of the bf16 tolerance); above it the Wk_lo term is added.
 constexpr float kBigState = 4.0f;
-// TMEM lanes 64..127 (the Q S rows of D1) masked off in the Wk_lo MMAs.
-__device__ __forceinline__ void xs_lane_mask(uint32_t (&m)[4]) {
+// Output-lane masks of an M = 128 MMA: lanes 64..127 kept as they are, or lanes 0..63.
+__device__ __forceinline__ void lane_mask_upper(uint32_t (&m)[4]) {
     m[0] = 0u;
     m[1] = 0u;
     m[2] = 0xffffffffu;
     m[3] = 0xffffffffu;
+}
+__device__ __forceinline__ void lane_mask_lower(uint32_t (&m)[4]) {
+    m[0] = 0xffffffffu;
+    m[1] = 0xffffffffu;
+    m[2] = 0u;
+    m[3] = 0u;
 }
 
 struct StateBars {
@@ -841,8 +887,8 @@ struct StateBars {
     uint64_t empty[2];     // chunk buffer released: the MMAs reading it (commit) + every epilogue warp
     uint64_t s_ready;      // S^T tile written (every epilogue warp)
     uint64_t y_ready;      // Y / DY tiles written (lane quarters 0-1), earlier chunk's output done (2-3)
-    uint64_t ox_full;      // output partial sums of the Mqk_lo rows written (lane quarters 0-1)
     uint64_t d1_full, d4_full, d3_full;  // MMA -> epilogue: accumulators complete
+    uint64_t lo_full;      // Wk_lo of the next chunk landed over Y / D Y (tx)
     uint64_t drain;                      // the MMA thread's last operations
 };
 
@@ -888,7 +934,6 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
     __shared__ uint32_t tmem_base_sh;
     __shared__ int failed_sh;
     __shared__ int big_sh;  // set once some |S| element of this slice exceeds kBigState
-    __shared__ int lo_sh[2];  // chunk buffer b holds Wk_lo (the load warp loads it once big_sh is set)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int v0 = blockIdx.x * BV, h = blockIdx.y, b = blockIdx.z;
@@ -904,15 +949,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
         }
         mbar_init(&bars.s_ready, EPI_WARPS);
         mbar_init(&bars.y_ready, EPI_WARPS);
-        mbar_init(&bars.ox_full, EPI_WARPS / 2);
         mbar_init(&bars.d1_full, 1);
         mbar_init(&bars.d4_full, 1);
         mbar_init(&bars.d3_full, 1);
+        mbar_init(&bars.lo_full, 1);
         mbar_init(&bars.drain, 1);
         mbar_fence_init();
         failed_sh = 0;
         big_sh = (p.flags & kForceWkLo) ? 1 : 0;
-        lo_sh[0] = lo_sh[1] = 0;
     }
     fence_before_sync();
     __syncthreads();
@@ -926,8 +970,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
     if (warp == EPI_WARPS + 1) {
         // ---------------- loads ----------------
         if (lane == 0) {
-            constexpr uint32_t bytes = 3 * (DK / 64) * C * 128 + 2 * C * 128 + LY::U_BYTES + C * 4;
-            constexpr uint32_t lo_bytes = (DK / 64) * C * 128;
+            constexpr uint32_t bytes = 3 * (DK / 64) * C * 128 + 2 * C * 128 + LY::U_BYTES + C * 4 + LY::FW_BYTES;
             int issued = -1;
             for (int c = 0; c < nch && !failed() && !(p.flags & kStallTest); ++c) {
                 if (c >= 2 && !mbar_wait(&bars.empty[c & 1], ((c - 2) >> 1) & 1, status, lim)) { fail(); break; }
@@ -935,24 +978,21 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 uint8_t *buf = sm + (c & 1) * LY::BUF;
                 uint64_t *bar = &bars.full[c & 1];
                 const int c0 = c * C;
-                // Wk_lo only once the state has grown large (the MMA warp reads lo_sh after this
-                // buffer's full barrier, which orders it after this store)
-                const bool lo = *(volatile int *)&big_sh != 0;
-                lo_sh[c & 1] = lo ? 1 : 0;
-                mbar_expect_tx(bar, bytes + (lo ? lo_bytes : 0u));
+                mbar_expect_tx(bar, bytes);
                 for (int blk = 0; blk < DK / 64; ++blk) {
                     uint8_t *dst = buf + LY::B_KWQ + blk * LY::KWQ_BLK;
                     tma_load_4d(dst, &maps.k, blk * 64, h, c0, b, bar);
-                    if (lo) bulk_g2s(dst + C * 128, rec + RC::WKL + blk * RC::WK_BLK, RC::WK_BLK, bar);
-                    bulk_g2s(dst + 2 * C * 128, rec + RC::WK + blk * RC::WK_BLK, RC::WK_BLK, bar);
-                    tma_load_4d(dst + 3 * C * 128, &maps.q, blk * 64, h, c0, b, bar);
+                    bulk_g2s(dst + C * 128, rec + RC::WK + blk * RC::WK_BLK, RC::WK_BLK, bar);
+                    tma_load_4d(dst + 2 * C * 128, &maps.q, blk * 64, h, c0, b, bar);
                 }
+                // once the state is large the MMA thread loads this chunk's Wk_lo: start it to L2
+                if (*(volatile int *)&big_sh) bulk_prefetch_l2(rec + RC::WKL, RC::WK_BLK * (DK / 64));
                 bulk_g2s(buf + LY::B_MQ, rec + RC::MQK + C * 128, C * 128, bar);   // Mqk_lo
                 bulk_g2s(buf + LY::B_MQ + C * 128, rec + RC::MQK, C * 128, bar);   // Mqk_hi
                 bulk_g2s(buf + LY::B_U, rec + RC::U + blockIdx.x * RC::U_SLICE, LY::U_BYTES, bar);
                 bulk_g2s(buf + LY::B_G, rec + RC::G, C * 4, bar);
-                if constexpr (RL)  // the F_w slice the epilogue warps fetch a chunk ahead: into L2 now
-                    bulk_prefetch_l2(rec + RC::FW + blockIdx.x * RC::FW_SLICE, RC::FW_SLICE);
+                if constexpr (RL)
+                    bulk_g2s(buf + LY::B_FW, rec + RC::FW + blockIdx.x * RC::FW_SLICE, LY::FW_BYTES, bar);
                 issued = c;
             }
             // let the copies still in flight land before the CTA can exit
@@ -970,8 +1010,24 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             const uint64_t dDY2 = make_desc(sb + LY::DY, LY::Y_BLK, 1024, 2);
             const uint32_t idS = idesc_bf16(128, N2, 0, 1);
             const uint32_t id4 = idesc_bf16(DK, N2, 1, 1);
-            uint32_t xmask[4];
-            xs_lane_mask(xmask);
+            auto oLO = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::WKL_BLK); };
+            uint32_t xmask[4], omask[4];
+            lane_mask_upper(xmask);  // the Wk_lo term: X_s rows only (lanes 64..127 hold Q S)
+            lane_mask_lower(omask);  // the Mqk_lo output term: output rows only (lanes 64..127)
+            // Wk_lo of chunk c over Y / D Y (bulk copies; lo_full counts its bytes)
+            uint32_t lo_phase = 0;
+            auto load_lo = [&](int c) {
+                const uint8_t *rec = record<DK, RL>(p, ws, nch, c);
+                mbar_expect_tx(&bars.lo_full, LY::WKL_BLK * (DK / 64));
+                for (int blk = 0; blk < DK / 64; ++blk)
+                    bulk_g2s(sm + LY::WKL + blk * LY::WKL_BLK, rec + RC::WKL + blk * RC::WK_BLK,
+                             RC::WK_BLK, &bars.lo_full);
+            };
+            bool lo = false;  // this chunk's Wk_lo is loaded (or on its way)
+            if (nch > 0 && *(volatile int *)&big_sh) {
+                load_lo(0);
+                lo = true;
+            }
             bool ok = nch == 0 || mbar_wait(&bars.full[0], 0, status, lim);
             for (int c = 0; c < nch && ok; ++c) {
                 const uint32_t bb = sb + (c & 1) * LY::BUF;
@@ -979,11 +1035,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 // back, is done: the epilogue warps work through the chunks in order)
                 if (!mbar_wait(&bars.s_ready, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
-                const uint64_t dWQ = make_desc(bb + LY::B_KWQ + 2 * C * 128, 16, 1024, 2);
+                const uint64_t dWQ = make_desc(bb + LY::B_KWQ + C * 128, 16, 1024, 2);
                 mma_steps<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dWQ, dS2, oKWQ, oMN, false);
-                if (*(volatile int *)&lo_sh[c & 1]) {  // X_s += Wk_lo S (rows 64..127 hold Q S: masked)
-                    const uint64_t dLW = make_desc(bb + LY::B_KWQ + C * 128, 16, 1024, 2);
-                    mma_steps_lanes<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dLW, dS2, oKWQ, oMN, true, xmask);
+                if (lo) {  // X_s += Wk_lo S, into the same accumulator with the Q S rows masked
+                    if (!mbar_wait(&bars.lo_full, lo_phase & 1, status, lim)) { ok = false; break; }
+                    ++lo_phase;
+                    const uint64_t dLW = make_desc(sb + LY::WKL, 16, 1024, 2);
+                    mma_steps_lanes<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dLW, dS2, oLO, oMN, true, xmask);
+                    lo = false;
                 }
                 mma_commit(&bars.d1_full);
                 // Y_c written, and the output epilogue of chunk c - 1 is done with D3
@@ -992,8 +1051,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 const uint64_t dKt = make_desc(bb + LY::B_KWQ, LY::KWQ_BLK, 1024, 2);
                 mma_steps<C / 16>(tb + LY::cD4, id4, dKt, dDY2, oMN, oMN, false);
                 mma_commit(&bars.d4_full);
+                // Mqk Y for the output rows (lanes 64..127): [Mqk_lo; Mqk_hi] Y puts the Mqk_hi rows
+                // there, then [Q rows; Mqk_lo] Y adds the Mqk_lo rows with lanes 0..63 masked
                 const uint64_t dMQ = make_desc(bb + LY::B_MQ, 16, 1024, 2);
                 mma_steps<C / 16>(tb + LY::cD3, idS, dMQ, dY2, oK0, oMN, false);
+                const uint64_t dMQlo = make_desc(bb + LY::B_MQ - C * 128, 16, 1024, 2);
+                mma_steps_lanes<C / 16>(tb + LY::cD3, idS, dMQlo, dY2, oK0, oMN, true, omask);
                 mma_commit(&bars.d3_full);
                 mma_commit(&bars.empty[c & 1]);
                 // the next chunk's inputs, off the chain while the state epilogue runs
@@ -1001,10 +1064,18 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                     ok = false;
                     break;
                 }
+                // once the state is large: the next chunk's Wk_lo over Y / D Y, as soon as this
+                // chunk's stage 2 MMAs (their last readers) have completed
+                if (c + 1 < nch && *(volatile int *)&big_sh) {
+                    if (!mbar_wait(&bars.d3_full, c & 1, status, lim)) { ok = false; break; }
+                    load_lo(c + 1);
+                    lo = true;
+                }
             }
             if (!ok) fail();
             mma_commit(&bars.drain);
             mbar_wait(&bars.drain, 0, nullptr, lim);
+            if (lo) mbar_wait(&bars.lo_full, lo_phase & 1, nullptr, lim);  // a copy still in flight lands
         }
     } else {
         // ---------------- epilogue: warps 0-15 ----------------
@@ -1012,12 +1083,11 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
         const int q = warp & 3;            // TMEM lane quarter
         const int j0 = (warp >> 2) * CH;   // first column of this warp in each BV-wide group
         const int lrow = 32 * q + lane;    // TMEM lane of this thread
-        const bool lowq = q < 2;           // lanes 0..63: X_s -> Y, and the Mqk_lo output partial
+        const bool lowq = q < 2;           // lanes 0..63: X_s -> Y; lanes 64..127: the output rows
         // state rows: lane = row for M = 128 (d = 128); lanes 32q + r, r < 16, for M = 64
         const bool own_d = (DK == 128) ? true : (lane < 16);
         const int d_row = (DK == 128) ? lrow : (16 * q + lane);
         const bool wr = !(p.flags & kNoWrite), out = !(p.flags & kNoOutput);
-        float *ox = (float *)(sm + LY::OX);
         float Sreg[CH];
 #pragma unroll
         for (int j = 0; j < CH; ++j) Sreg[j] = 0.f;
@@ -1040,36 +1110,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             watch_state();
         }
         warp_arrive(&bars.s_ready, lane);
-        // rank L: this thread's F_w elements of a chunk, fetched from the record (which the load warp
-        // prefetches into L2 two chunks ahead): a chunk ahead into registers when a thread holds 8
-        // of them, after the chunk's own Y epilogue when it holds 16 (keeping the registers of the
-        // two phases apart)
-        constexpr bool kEarlyFw = CH <= 8;
-        auto fetch_fw = [&](int cc, float (&dst)[CH]) {
-#pragma unroll
-            for (int j = 0; j < CH; ++j) dst[j] = 0.f;
-            if (RL && wr && own_d) {
-                const uint8_t *src = record<DK, RL>(p, ws, nch, cc) + RC::FW + blockIdx.x * RC::FW_SLICE;
-#pragma unroll
-                for (int j4 = 0; j4 < CH; j4 += 4) {
-                    const float4 f4 = __ldg(reinterpret_cast<const float4 *>(src + u_off<BV>(d_row, j0 + j4)));
-                    dst[j4] = f4.x;
-                    dst[j4 + 1] = f4.y;
-                    dst[j4 + 2] = f4.z;
-                    dst[j4 + 3] = f4.w;
-                }
-            }
-        };
-        float fw_next[CH];
-        if (kEarlyFw && nch > 0) fetch_fw(0, fw_next);
         bool ok = true;
         for (int c = 0; c < nch && ok; ++c) {
             const int c0 = c * C, n = min(C, T - c0);
             const uint8_t *buf = sm + (c & 1) * LY::BUF;
-            float fw[CH];
-#pragma unroll
-            for (int j = 0; j < CH; ++j) fw[j] = kEarlyFw ? fw_next[j] : 0.f;
-            if (kEarlyFw && c + 1 < nch) fetch_fw(c + 1, fw_next);
             if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status, lim)) { ok = false; break; }
             const float *g = reinterpret_cast<const float *>(buf + LY::B_G);
             const float g_last = g[C - 1];
@@ -1118,17 +1162,26 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 store_half_pair<BV, CH>(sm + LY::DY, LY::Y_BLK, t, j0, y);
             }
             warp_arrive(&bars.y_ready, lane);
-            if (!kEarlyFw) fetch_fw(c, fw);
             // state update S^T <- e^{g_n} S^T + K^T D Y (+ F_w)
             {
                 const float gC = __expf(g_last);
-                if (own_d) {  // e^{g_n} S^T (+ F_w) first: it does not depend on D4
+                if (own_d) {  // the size check of S_c and e^{g_n} S^T (+ F_w): no D4 needed yet
+                    watch_state();
 #pragma unroll
-                    for (int j = 0; j < CH; ++j) Sreg[j] = fmaf(Sreg[j], gC, fw[j]);
+                    for (int j = 0; j < CH; ++j) Sreg[j] *= gC;
+                    if (RL && wr) {
+#pragma unroll
+                        for (int j4 = 0; j4 < CH; j4 += 4) {
+                            const float4 f4 = *reinterpret_cast<const float4 *>(buf + LY::B_FW + u_off<BV>(d_row, j0 + j4));
+                            Sreg[j4] += f4.x;
+                            Sreg[j4 + 1] += f4.y;
+                            Sreg[j4 + 2] += f4.z;
+                            Sreg[j4 + 3] += f4.w;
+                        }
+                    }
                 }
-                // the epilogue's reads of the chunk buffer are done (U in the Y epilogue; g is held
-                // in registers): release it, so that the chunk two ahead loads while this one's
-                // state and output epilogues run
+                // the last read of the chunk buffer (g is held in registers): release it, so that
+                // the chunk two ahead loads while this one's state and output epilogues run
                 warp_arrive(&bars.empty[c & 1], lane);
                 if (!mbar_wait(&bars.d4_full, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
@@ -1143,25 +1196,11 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 }
             }
             warp_arrive(&bars.s_ready, lane);
-            if (own_d) watch_state();  // after the hand-off, off the chain
-            // output O = diag(e^g) QS + Mqk Y: the Mqk_lo rows (lanes 0..63) pass their partial
-            // sums through shared memory to the threads of the output rows (lanes 64..127)
-            if (!mbar_wait(&bars.d3_full, c & 1, status, lim)) { ok = false; break; }
-            fence_after_sync();
-            if (lowq) {
-                const int t = lrow;
-                float a[CH], bb[CH];
-                tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD3 + j0), a);
-                tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD3 + BV + j0), bb);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j4 = 0; j4 < CH; j4 += 4)
-                    *reinterpret_cast<float4 *>(ox + t * LY::OXS + j0 + j4) =
-                        make_float4(a[j4] + bb[j4], a[j4 + 1] + bb[j4 + 1], a[j4 + 2] + bb[j4 + 2],
-                                    a[j4 + 3] + bb[j4 + 3]);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.ox_full);
-            } else {
+            // output O = diag(e^g) QS + Mqk Y (+ O_w), by the threads of the output rows (TMEM lanes
+            // 64..127, where both the Q S rows of D1 and the whole Mqk Y term of D3 sit)
+            if (!lowq) {
+                if (!mbar_wait(&bars.d3_full, c & 1, status, lim)) { ok = false; break; }
+                fence_after_sync();
                 const int t = lrow - 64;
                 float up[CH], qs[CH];
                 {
@@ -1177,20 +1216,16 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
 #pragma unroll
                     for (int j = 0; j < CH; ++j) qs[j] = a[j] + bb[j];
                 }
-                if (!mbar_wait(&bars.ox_full, c & 1, status, lim)) { ok = false; break; }
                 if (t < n && out) {
                     const float gt = __expf(g_row);
                     __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t) * H + h) * dv + v0 + j0;
 #pragma unroll
                     for (int c8 = 0; c8 < CH / 8; ++c8) {
-                        const float4 p0 = *reinterpret_cast<const float4 *>(ox + t * LY::OXS + j0 + c8 * 8);
-                        const float4 p1 = *reinterpret_cast<const float4 *>(ox + t * LY::OXS + j0 + c8 * 8 + 4);
-                        const float pp[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
                         float r[8];
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
                             const int jj = c8 * 8 + j;
-                            r[j] = fmaf(gt, qs[jj], up[jj] + pp[j] + ow[jj]);
+                            r[j] = fmaf(gt, qs[jj], up[jj] + ow[jj]);
                         }
                         uint4 pk;
                         pk.x = pack_bf16(r[0], r[1]);

@@ -73,12 +73,18 @@ def test_producer_full_size_sampled(name):
 def test_producer_feeds_the_scan(d, L, T):
     """The producer's write terms through the scan, element by element, with the producer's raw
     (unnormalised) directions: |W_k a| is about 8 with these random weights, so the state grows
-    well beyond the unit-norm workloads.  Three comparisons, each at the bf16 tolerance
-    2e-2 (1 + |r|):
+    well beyond the unit-norm workloads.  Two comparisons element by element at the bf16
+    tolerance 2e-2 (1 + |r|):
       1. the GPU producer's u, w against the oracle producer;
       2. the GPU scan on the GPU producer's u, w against the oracle scan on the same bytes;
-      3. end to end: GPU producer -> GPU scan against oracle producer -> bf16 rounding (nearest
-         even) -> oracle scan."""
+    and, end to end, GPU producer -> GPU scan against oracle producer -> bf16 rounding (nearest
+    even) -> oracle scan.  The end-to-end pair is not held to the element-wise bound: the bf16
+    rounding of u, w is part of the pipeline, the GPU producer's fp32 arithmetic rounds a few
+    values to the other bf16 neighbour, and the scan carries such a one-ulp change of a write value
+    into later outputs with the gain |w| |q| (about 64 here), which can exceed 2e-2 (1 + |r|) on an
+    output that cancels to near zero.  Stages 1 and 2 bound the pipeline element by element; the
+    end-to-end check bounds the fraction of elements outside the tolerance (at most 1 in 10^4) and
+    their size (within 10 times the tolerance)."""
     from delta_rule_sequence_b200.prism import prism_scan_fwd, prism_write_producer
 
     wl = WORKLOADS["recsys"].with_(B=1, H=2, T=T, dk=d, dv=d, L=L)
@@ -101,8 +107,10 @@ def test_producer_feeds_the_scan(d, L, T):
     u_bf = torch.from_numpy(u_ref).to(torch.bfloat16)
     w_bf = torch.from_numpy(w_ref).to(torch.bfloat16)
     o_ref, S_ref = oracle.scan_ref(x["q"], x["k"], None, x["alpha"], x["beta"], u_bf, w_bf, None)
-    compare("o (producer -> scan)", o.float().cpu().numpy(), o_ref, TOL["bf16"])
-    compare("S_final (producer -> scan)", S.cpu().numpy(), S_ref, TOL["bf16"])
+    for name, got, ref in (("o", o.float().cpu().numpy(), o_ref), ("S_final", S.cpu().numpy(), S_ref)):
+        excess = np.abs(got - ref) / (TOL["bf16"] * (1.0 + np.abs(ref)))
+        assert (excess > 1.0).mean() <= 1e-4, (name, int((excess > 1.0).sum()), excess.size)
+        assert excess.max() <= 10.0, (name, float(excess.max()))
 
 
 def test_producer_leaves_no_tokens_untouched_and_no_status():
