@@ -801,19 +801,25 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
 // ------------------------------------------------------------------------------------------------
 // state: one CTA per (value slice, head, batch), chunks in order
 //
-// Two MMA stages per chunk (8 instructions at d = 128 for the first, 4 + 8 for the second):
+// Per chunk the chain's MMA thread issues (8 instructions at d = 128 for stage 1, 4 for D4):
 //   stage 1:  D1 = [Wk; Q] [S_hi | S_lo]                    (M = 128, N = 2 BV: X_s and QS)
 //             D1 += [Wk_lo; *] [S_hi | S_lo], TMEM lanes 64..127 masked off (only X_s gains the
 //             Wk_lo term), once the state of this CTA has grown past kBigState
-//   stage 2:  D4 = K^T [DY_hi | DY_lo]                      (the state update, on the chain)
-//             D3 = [Mqk_lo; Mqk_hi] [Y_hi | Y_lo], then D3 += [*; Mqk_lo] [Y_hi | Y_lo] with lanes
-//             0..63 masked off                              (the output's intra-chunk term)
+//   D4:       D4 = K^T [DY_hi | DY_lo]                      (the state update)
+// and a second thread, in its own warp, the output's intra-chunk term (8 instructions):
+//   D3:       D3 = [Mqk_lo; Mqk_hi] [Y_hi | Y_lo], then D3 += [*; Mqk_lo] [Y_hi | Y_lo] with lanes
+//             0..63 masked off
+// The chain of a chunk is stage 1 -> the Y epilogue -> D4 -> the state epilogue.  One thread
+// issues a tcgen05.mma only every 60-80 cycles, so D3 on the chain's thread put its issue time on
+// the chain; from its own thread it runs on the tensor pipe while the state epilogue does.  The tile
+// Y is double-buffered (D3 of chunk c may still read it while chunk c + 1's Y epilogue runs).
 // X_s sits in TMEM lanes 0..63, QS and the whole Mqk Y term in lanes 64..127, so the Y epilogue
-// runs on sub-partitions 0-1 and the output epilogue on 2-3, where it does not slow the MMA warp
-// (sub-partition 0) issuing the next chunk's stage 1.  D1 is double-buffered in TMEM.  K, Q arrive
-// by TMA tiled loads, the per-chunk record (Wk, Mqk, the U slice, g, and on the rank-L route the
-// F_w slice) by bulk copies, into two chunk buffers: chunk c + 2 loads into chunk c's buffer as soon
-// as its last readers (the stage 2 MMAs and the state epilogue's F_w read) are done.
+// runs on sub-partitions 0-1 and the output epilogue on 2-3.  D1 is double-buffered in TMEM.  K, Q
+// arrive by TMA tiled loads, the per-chunk record (Wk, Mqk, the U slice, g, and on the rank-L route
+// the F_w slice) by bulk copies, into two chunk buffers: chunk c + 2 loads into chunk c's buffer as
+// soon as its readers are done (D4 and the state epilogue's F_w read for most of it, D3 for U and
+// Mqk).  Every wait on a barrier that completes once per chunk is made when that barrier can be at
+// most one phase ahead of the waiter (parity waits cannot tell two phases apart).
 //
 // Precision of X_s = Wk S^T: Wk is a rounded intermediate result, so its single-bf16 error (2^-9
 // relative) reaches Y scaled by |S|.  For states of order one that stays far below the bf16
@@ -830,40 +836,49 @@ struct StateLayout {
     static constexpr int CH = BV / 4;                     // columns of one epilogue warp
     static constexpr uint32_t KWQ_BLK = 3 * C * 128;      // [K; Wk; Q] rows of one 64-col block
     static constexpr uint32_t U_BYTES = C * BV * 4;
-    // double-buffered chunk inputs
+    // double-buffered chunk inputs.  U and Mqk are loaded once the buffer's D3 has completed, so
+    // the 64 masked rows that D3's second MMA reads in front of Mqk_lo (the end of U) are not
+    // being written while it runs.
     static constexpr uint32_t B_KWQ = 0;
-    static constexpr uint32_t B_MQ = B_KWQ + KWQ_BLK * (DK / 64);   // [Mqk_lo; Mqk_hi]
-    static constexpr uint32_t B_U = B_MQ + 2 * C * 128;
-    static constexpr uint32_t B_G = B_U + U_BYTES;                   // g (64 floats)
+    static constexpr uint32_t B_U = B_KWQ + KWQ_BLK * (DK / 64);
+    static constexpr uint32_t B_MQ = B_U + U_BYTES;                   // [Mqk_lo; Mqk_hi]
+    static constexpr uint32_t B_G = B_MQ + 2 * C * 128;              // g (64 floats)
+    static_assert(U_BYTES >= C * 128 && B_MQ % 1024 == 0, "D3's masked rows fall in U");
     static constexpr uint32_t FW_BYTES = RL ? DK * BV * 4 : 0;       // F_w slice (rank L)
     static constexpr uint32_t B_FW = B_G + 1024;
     static constexpr uint32_t BUF = B_FW + FW_BYTES;
-    // Y [t][hi | lo], D Y [t][hi | lo], S^T [d][hi | lo]: MN-major, 64-column blocks.  Y and D Y
-    // are free from the completion of a chunk's stage 2 MMAs to its Y epilogue: Wk_lo of the next
-    // chunk (one 64-row K-major tile per 64 columns) is loaded over them when it is needed.
+    // Y [t][hi | lo] (two buffers, by chunk parity), D Y [t][hi | lo], S^T [d][hi | lo]: MN-major,
+    // 64-column blocks, in the order Y0, D Y, Y1, S.  Wk_lo of chunk c (one 64-row K-major tile per
+    // 64 columns) is loaded over D Y and chunk c's Y buffer, which are free from the completion of
+    // D4 of chunk c - 1 (the last reader of D Y) and of D3 of chunk c - 2 (the last reader of that
+    // Y buffer) to the Y epilogue of chunk c: they are adjacent for either parity.
     static constexpr uint32_t Y_BLK = C * 128;
-    static constexpr uint32_t Y = 2 * BUF;
-    static constexpr uint32_t DY = Y + Y_BLK * (N2 / 64);
-    static constexpr uint32_t WKL = Y;
+    static constexpr uint32_t YT = Y_BLK * (N2 / 64);   // one Y or D Y tile
+    static constexpr uint32_t Y0 = 2 * BUF;
+    static constexpr uint32_t DY = Y0 + YT;
+    static constexpr uint32_t Y1 = DY + YT;
     static constexpr uint32_t WKL_BLK = C * 128;
     static constexpr uint32_t S_BLK = DK * 128;
-    static constexpr uint32_t S = DY + Y_BLK * (N2 / 64);
+    static constexpr uint32_t S = Y1 + YT;
     static constexpr uint32_t BYTES = S + S_BLK * (N2 / 64) + 1024;
+    static constexpr uint32_t y_at(int c) { return (c & 1) ? Y1 : Y0; }
+    static constexpr uint32_t wkl_at(int c) { return (c & 1) ? DY : Y0; }
     // the lane-masked Wk_lo MMA reads 128 rows from each 64-column block of Wk_lo: the rows past
-    // the last block (masked) are still inside the allocation
-    static_assert(WKL + WKL_BLK * (DK / 64) + WKL_BLK <= BYTES - 1024, "masked rows stay in bounds");
-    static_assert(WKL_BLK * (DK / 64) <= 2 * Y_BLK * (N2 / 64), "Wk_lo fits over Y and D Y");
+    // the last block (masked, their products dropped) are still inside the allocation
+    static_assert(DY + WKL_BLK * (DK / 64) + WKL_BLK <= BYTES - 1024, "masked rows stay in bounds");
+    static_assert(WKL_BLK * (DK / 64) <= 2 * YT, "Wk_lo fits over D Y and one Y buffer");
     // TMEM columns: D1 (two buffers), D3, D4
     static constexpr uint32_t cD1 = 0, cD3 = 2 * N2, cD4 = 3 * N2;
     static constexpr uint32_t TCOLS = 4 * N2 <= 256 ? 256 : 512;
 };
 
 // Warp roles of the state kernel: warps 0-15 epilogue (warp w reads TMEM lane quarter w % 4 and
-// the column quarter w / 4 of every BV-wide group), warp 16 issues the MMAs, warp 17 the loads.
-// Every hand-off is an mbarrier (no CTA-wide barrier inside the chunk loop); every wait is bounded.
+// the column quarter w / 4 of every BV-wide group), warp 16 issues the chain's MMAs, warp 17 the
+// loads, warp 18 the D3 MMAs.  Every hand-off is an mbarrier (no CTA-wide barrier inside the chunk
+// loop); every wait is bounded.
 constexpr int EPI_WARPS = 16;
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
-constexpr int ST_THREADS = EPI_THREADS + 64;
+constexpr int ST_THREADS = EPI_THREADS + 96;
 
 // Largest |S| element below which X_s = Wk S^T is taken with Wk as one bf16 (its rounding then
 // moves Y by at most a few per cent of the bf16 tolerance); above it the Wk_lo term is added.
@@ -883,13 +898,17 @@ __device__ __forceinline__ void lane_mask_lower(uint32_t (&m)[4]) {
 }
 
 struct StateBars {
-    uint64_t full[2];      // chunk inputs landed (tx)
-    uint64_t empty[2];     // chunk buffer released: the MMAs reading it (commit) + every epilogue warp
+    uint64_t full[2];      // chunk inputs but U, Mqk landed (tx)
+    uint64_t full_mq[2];   // the chunk's U slice and Mqk landed (tx)
+    uint64_t empty[2];     // chunk buffer but U, Mqk released: D4 (commit) + every epilogue warp
+    uint64_t mq_empty[2];  // the buffer's U, Mqk and Y tile released: that chunk's D3 (commit)
     uint64_t s_ready;      // S^T tile written (every epilogue warp)
-    uint64_t y_ready;      // Y / DY tiles written (lane quarters 0-1), earlier chunk's output done (2-3)
+    uint64_t y_ready;      // D Y tile written (the warps of lane quarters 0-1)
+    uint64_t yq_ready[2];  // Y buffer written (the same warps), by chunk parity
+    uint64_t out_free;     // D3 read by the output epilogue (the warps of lane quarters 2-3)
     uint64_t d1_full, d4_full, d3_full;  // MMA -> epilogue: accumulators complete
     uint64_t lo_full;      // Wk_lo of the next chunk landed over Y / D Y (tx)
-    uint64_t drain;                      // the MMA thread's last operations
+    uint64_t drain, drain3;              // the MMA threads' last operations
 };
 
 
@@ -945,15 +964,21 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars.full[i], 1);
+            mbar_init(&bars.full_mq[i], 1);
             mbar_init(&bars.empty[i], 1 + EPI_WARPS);
+            mbar_init(&bars.mq_empty[i], 1);
         }
         mbar_init(&bars.s_ready, EPI_WARPS);
-        mbar_init(&bars.y_ready, EPI_WARPS);
+        mbar_init(&bars.y_ready, EPI_WARPS / 2);
+        mbar_init(&bars.yq_ready[0], EPI_WARPS / 2);
+        mbar_init(&bars.yq_ready[1], EPI_WARPS / 2);
+        mbar_init(&bars.out_free, EPI_WARPS / 2);
         mbar_init(&bars.d1_full, 1);
         mbar_init(&bars.d4_full, 1);
         mbar_init(&bars.d3_full, 1);
         mbar_init(&bars.lo_full, 1);
         mbar_init(&bars.drain, 1);
+        mbar_init(&bars.drain3, 1);
         mbar_fence_init();
         failed_sh = 0;
         big_sh = (p.flags & kForceWkLo) ? 1 : 0;
@@ -970,9 +995,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
     if (warp == EPI_WARPS + 1) {
         // ---------------- loads ----------------
         if (lane == 0) {
-            constexpr uint32_t bytes = 3 * (DK / 64) * C * 128 + 2 * C * 128 + LY::U_BYTES + C * 4 + LY::FW_BYTES;
-            int issued = -1;
+            constexpr uint32_t bytes = 3 * (DK / 64) * C * 128 + C * 4 + LY::FW_BYTES;
+            constexpr uint32_t bytes_mq = LY::U_BYTES + 2 * C * 128;
+            int issued = -1, issued_mq = -1;
             for (int c = 0; c < nch && !failed() && !(p.flags & kStallTest); ++c) {
+                // the buffer's main part frees after D4 of chunk c - 2, its U and Mqk after that
+                // chunk's D3 (the Y epilogue read U before the epilogue warps released the buffer)
                 if (c >= 2 && !mbar_wait(&bars.empty[c & 1], ((c - 2) >> 1) & 1, status, lim)) { fail(); break; }
                 const uint8_t *rec = record<DK, RL>(p, ws, nch, c);
                 uint8_t *buf = sm + (c & 1) * LY::BUF;
@@ -987,40 +1015,76 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 }
                 // once the state is large the MMA thread loads this chunk's Wk_lo: start it to L2
                 if (*(volatile int *)&big_sh) bulk_prefetch_l2(rec + RC::WKL, RC::WK_BLK * (DK / 64));
-                bulk_g2s(buf + LY::B_MQ, rec + RC::MQK + C * 128, C * 128, bar);   // Mqk_lo
-                bulk_g2s(buf + LY::B_MQ + C * 128, rec + RC::MQK, C * 128, bar);   // Mqk_hi
-                bulk_g2s(buf + LY::B_U, rec + RC::U + blockIdx.x * RC::U_SLICE, LY::U_BYTES, bar);
                 bulk_g2s(buf + LY::B_G, rec + RC::G, C * 4, bar);
                 if constexpr (RL)
                     bulk_g2s(buf + LY::B_FW, rec + RC::FW + blockIdx.x * RC::FW_SLICE, LY::FW_BYTES, bar);
                 issued = c;
+                if (c >= 2 && !mbar_wait(&bars.mq_empty[c & 1], ((c - 2) >> 1) & 1, status, lim)) { fail(); break; }
+                uint64_t *bar_mq = &bars.full_mq[c & 1];
+                mbar_expect_tx(bar_mq, bytes_mq);
+                bulk_g2s(buf + LY::B_U, rec + RC::U + blockIdx.x * RC::U_SLICE, LY::U_BYTES, bar_mq);
+                bulk_g2s(buf + LY::B_MQ, rec + RC::MQK + C * 128, C * 128, bar_mq);   // Mqk_lo
+                bulk_g2s(buf + LY::B_MQ + C * 128, rec + RC::MQK, C * 128, bar_mq);   // Mqk_hi
+                issued_mq = c;
             }
             // let the copies still in flight land before the CTA can exit
             for (int c = issued > 0 ? issued - 1 : 0; c <= issued; ++c)
                 mbar_wait(&bars.full[c & 1], (c >> 1) & 1, nullptr, lim);
+            for (int c = issued_mq > 0 ? issued_mq - 1 : 0; c <= issued_mq; ++c)
+                mbar_wait(&bars.full_mq[c & 1], (c >> 1) & 1, nullptr, lim);
         }
-    } else if (warp == EPI_WARPS) {
-        // ---------------- MMA issue ----------------
+    } else if (warp == EPI_WARPS + 2) {
+        // ---------------- D3 MMA issue ----------------
         if (lane == 0) {
-            auto oKWQ = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::KWQ_BLK); };
             auto oK0 = [](int ks) { return (uint64_t)koff_k_sw128(ks, 0); };
             auto oMN = [](int ks) { return (uint64_t)koff_mn_sw128(ks); };
+            const uint32_t idS = idesc_bf16(128, N2, 0, 1);
+            uint32_t omask[4];
+            lane_mask_lower(omask);  // the Mqk_lo output term: output rows only (lanes 64..127)
+            bool ok = true;
+            for (int c = 0; c < nch && ok; ++c) {
+                // D3 of chunk c: Mqk Y for the output rows (lanes 64..127).  [Mqk_lo; Mqk_hi] Y puts
+                // the Mqk_hi rows there, then [Q rows; Mqk_lo] Y adds the Mqk_lo rows with lanes
+                // 0..63 masked.  It waits for Y_c, the chunk's U / Mqk, and the output epilogue's
+                // read of D3 of chunk c - 1.
+                if (!mbar_wait(&bars.yq_ready[c & 1], (c >> 1) & 1, status, lim) ||
+                    !mbar_wait(&bars.full_mq[c & 1], (c >> 1) & 1, status, lim) ||
+                    (c > 0 && !mbar_wait(&bars.out_free, (c - 1) & 1, status, lim))) {
+                    ok = false;
+                    break;
+                }
+                fence_after_sync();
+                const uint32_t bb = sb + (c & 1) * LY::BUF;
+                const uint64_t dY2 = make_desc(sb + LY::y_at(c), LY::Y_BLK, 1024, 2);
+                mma_steps<C / 16>(tb + LY::cD3, idS, make_desc(bb + LY::B_MQ, 16, 1024, 2), dY2, oK0, oMN, false);
+                mma_steps_lanes<C / 16>(tb + LY::cD3, idS, make_desc(bb + LY::B_MQ - C * 128, 16, 1024, 2), dY2,
+                                        oK0, oMN, true, omask);
+                mma_commit(&bars.d3_full);
+                mma_commit(&bars.mq_empty[c & 1]);
+            }
+            if (!ok) fail();
+            mma_commit(&bars.drain3);
+            mbar_wait(&bars.drain3, 0, nullptr, lim);
+        }
+    } else if (warp == EPI_WARPS) {
+        // ---------------- chain MMA issue ----------------
+        if (lane == 0) {
+            auto oKWQ = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::KWQ_BLK); };
+            auto oMN = [](int ks) { return (uint64_t)koff_mn_sw128(ks); };
             const uint64_t dS2 = make_desc(sb + LY::S, LY::S_BLK, 1024, 2);
-            const uint64_t dY2 = make_desc(sb + LY::Y, LY::Y_BLK, 1024, 2);
             const uint64_t dDY2 = make_desc(sb + LY::DY, LY::Y_BLK, 1024, 2);
             const uint32_t idS = idesc_bf16(128, N2, 0, 1);
             const uint32_t id4 = idesc_bf16(DK, N2, 1, 1);
             auto oLO = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::WKL_BLK); };
-            uint32_t xmask[4], omask[4];
+            uint32_t xmask[4];
             lane_mask_upper(xmask);  // the Wk_lo term: X_s rows only (lanes 64..127 hold Q S)
-            lane_mask_lower(omask);  // the Mqk_lo output term: output rows only (lanes 64..127)
-            // Wk_lo of chunk c over Y / D Y (bulk copies; lo_full counts its bytes)
+            // Wk_lo of chunk c over D Y and Y buffer c % 2 (bulk copies; lo_full counts its bytes)
             uint32_t lo_phase = 0;
             auto load_lo = [&](int c) {
                 const uint8_t *rec = record<DK, RL>(p, ws, nch, c);
                 mbar_expect_tx(&bars.lo_full, LY::WKL_BLK * (DK / 64));
                 for (int blk = 0; blk < DK / 64; ++blk)
-                    bulk_g2s(sm + LY::WKL + blk * LY::WKL_BLK, rec + RC::WKL + blk * RC::WK_BLK,
+                    bulk_g2s(sm + LY::wkl_at(c) + blk * LY::WKL_BLK, rec + RC::WKL + blk * RC::WK_BLK,
                              RC::WK_BLK, &bars.lo_full);
             };
             bool lo = false;  // this chunk's Wk_lo is loaded (or on its way)
@@ -1040,36 +1104,33 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 if (lo) {  // X_s += Wk_lo S, into the same accumulator with the Q S rows masked
                     if (!mbar_wait(&bars.lo_full, lo_phase & 1, status, lim)) { ok = false; break; }
                     ++lo_phase;
-                    const uint64_t dLW = make_desc(sb + LY::WKL, 16, 1024, 2);
+                    const uint64_t dLW = make_desc(sb + LY::wkl_at(c), 16, 1024, 2);
                     mma_steps_lanes<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dLW, dS2, oLO, oMN, true, xmask);
                     lo = false;
                 }
                 mma_commit(&bars.d1_full);
-                // Y_c written, and the output epilogue of chunk c - 1 is done with D3
+                // D Y_c written
                 if (!mbar_wait(&bars.y_ready, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 const uint64_t dKt = make_desc(bb + LY::B_KWQ, LY::KWQ_BLK, 1024, 2);
                 mma_steps<C / 16>(tb + LY::cD4, id4, dKt, dDY2, oMN, oMN, false);
                 mma_commit(&bars.d4_full);
-                // Mqk Y for the output rows (lanes 64..127): [Mqk_lo; Mqk_hi] Y puts the Mqk_hi rows
-                // there, then [Q rows; Mqk_lo] Y adds the Mqk_lo rows with lanes 0..63 masked
-                const uint64_t dMQ = make_desc(bb + LY::B_MQ, 16, 1024, 2);
-                mma_steps<C / 16>(tb + LY::cD3, idS, dMQ, dY2, oK0, oMN, false);
-                const uint64_t dMQlo = make_desc(bb + LY::B_MQ - C * 128, 16, 1024, 2);
-                mma_steps_lanes<C / 16>(tb + LY::cD3, idS, dMQlo, dY2, oK0, oMN, true, omask);
-                mma_commit(&bars.d3_full);
                 mma_commit(&bars.empty[c & 1]);
-                // the next chunk's inputs, off the chain while the state epilogue runs
-                if (c + 1 < nch && !mbar_wait(&bars.full[(c + 1) & 1], ((c + 1) >> 1) & 1, status, lim)) {
-                    ok = false;
-                    break;
-                }
-                // once the state is large: the next chunk's Wk_lo over Y / D Y, as soon as this
-                // chunk's stage 2 MMAs (their last readers) have completed
-                if (c + 1 < nch && *(volatile int *)&big_sh) {
-                    if (!mbar_wait(&bars.d3_full, c & 1, status, lim)) { ok = false; break; }
-                    load_lo(c + 1);
-                    lo = true;
+                if (c + 1 < nch) {
+                    // once the state is large: the next chunk's Wk_lo over D Y and Y buffer
+                    // (c + 1) % 2, as soon as D4 of chunk c and D3 of chunk c - 1 have completed
+                    // (the latter cannot be a phase further on: D3 of chunk c + 1 needs this Wk_lo)
+                    if (*(volatile int *)&big_sh) {
+                        if (!mbar_wait(&bars.d4_full, c & 1, status, lim) ||
+                            (c >= 1 && !mbar_wait(&bars.mq_empty[(c + 1) & 1], ((c - 1) >> 1) & 1, status, lim))) {
+                            ok = false;
+                            break;
+                        }
+                        load_lo(c + 1);
+                        lo = true;
+                    }
+                    // the next chunk's inputs, off the chain while the state epilogue runs
+                    if (!mbar_wait(&bars.full[(c + 1) & 1], ((c + 1) >> 1) & 1, status, lim)) { ok = false; break; }
                 }
             }
             if (!ok) fail();
@@ -1119,25 +1180,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             const float g_last = g[C - 1];
             const float g_row = g[lowq ? lrow : lrow - 64];  // g of this thread's Y / output row
             const uint32_t d1 = LY::cD1 + (c & 1) * N2;
-            float ow[CH];  // rank L: O_w of this thread's output row, fetched early
-#pragma unroll
-            for (int j = 0; j < CH; ++j) ow[j] = 0.f;
-            if (RL && wr && out && !lowq && lrow - 64 < n) {
-                const float *src = reinterpret_cast<const float *>(record<DK, RL>(p, ws, nch, c) + RC::OW) +
-                                   (size_t)(lrow - 64) * dv + v0 + j0;
-#pragma unroll
-                for (int j4 = 0; j4 < CH; j4 += 4) {
-                    const float4 f4 = __ldg(reinterpret_cast<const float4 *>(src + j4));
-                    ow[j4] = f4.x;
-                    ow[j4 + 1] = f4.y;
-                    ow[j4 + 2] = f4.z;
-                    ow[j4 + 3] = f4.w;
-                }
-            }
-            // Y = U - X_s (lanes 0..63 of D1), and D Y
+            // Y = U - X_s (lanes 0..63 of D1), and D Y: D Y first (D4 waits for it), Y after the
+            // hand-off (D3 reads it after the next state hand-off)
             if (lowq) {
                 const int t = lrow;
                 const float dd = t < n ? __expf(g_last - g_row) : 0.f;
+                if (!mbar_wait(&bars.full_mq[c & 1], (c >> 1) & 1, status, lim)) { ok = false; break; }
                 float y[CH];  // U first: it does not depend on D1
 #pragma unroll
                 for (int j4 = 0; j4 < CH; j4 += 4) {
@@ -1154,14 +1202,20 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 tmem_ld_n<CH>(taddr(tb, 32 * q, d1 + j0), xh);
                 tmem_ld_n<CH>(taddr(tb, 32 * q, d1 + BV + j0), xl);
                 tmem_wait_ld();
+                float dy[CH];
 #pragma unroll
-                for (int j = 0; j < CH; ++j) y[j] -= xh[j] + xl[j];
-                store_half_pair<BV, CH>(sm + LY::Y, LY::Y_BLK, t, j0, y);
-#pragma unroll
-                for (int j = 0; j < CH; ++j) y[j] *= dd;
-                store_half_pair<BV, CH>(sm + LY::DY, LY::Y_BLK, t, j0, y);
+                for (int j = 0; j < CH; ++j) {
+                    y[j] -= xh[j] + xl[j];
+                    dy[j] = y[j] * dd;
+                }
+                store_half_pair<BV, CH>(sm + LY::DY, LY::Y_BLK, t, j0, dy);
+                warp_arrive(&bars.y_ready, lane);
+                // Y buffer c % 2 was last read by D3 of chunk c - 2, which has completed: the output
+                // warps saw it complete before they wrote S_c, and this chunk's stage 1, whose
+                // completion these warps saw, was issued after S_c
+                store_half_pair<BV, CH>(sm + LY::y_at(c), LY::Y_BLK, t, j0, y);
+                warp_arrive(&bars.yq_ready[c & 1], lane);
             }
-            warp_arrive(&bars.y_ready, lane);
             // state update S^T <- e^{g_n} S^T + K^T D Y (+ F_w)
             {
                 const float gC = __expf(g_last);
@@ -1199,6 +1253,23 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             // output O = diag(e^g) QS + Mqk Y (+ O_w), by the threads of the output rows (TMEM lanes
             // 64..127, where both the Q S rows of D1 and the whole Mqk Y term of D3 sit)
             if (!lowq) {
+                // rank L: O_w of this thread's row, loaded here because an mbarrier arrive waits
+                // for the thread's loads in flight: the next arrive (out_free) is off the chain
+                float ow[CH];
+#pragma unroll
+                for (int j = 0; j < CH; ++j) ow[j] = 0.f;
+                if (RL && wr && out && lrow - 64 < n) {
+                    const float *src = reinterpret_cast<const float *>(record<DK, RL>(p, ws, nch, c) + RC::OW) +
+                                       (size_t)(lrow - 64) * dv + v0 + j0;
+#pragma unroll
+                    for (int j4 = 0; j4 < CH; j4 += 4) {
+                        const float4 f4 = __ldg(reinterpret_cast<const float4 *>(src + j4));
+                        ow[j4] = f4.x;
+                        ow[j4 + 1] = f4.y;
+                        ow[j4 + 2] = f4.z;
+                        ow[j4 + 3] = f4.w;
+                    }
+                }
                 if (!mbar_wait(&bars.d3_full, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 const int t = lrow - 64;
@@ -1208,6 +1279,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                     tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD3 + j0), a);
                     tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD3 + BV + j0), bb);
                     tmem_wait_ld();
+                    warp_arrive(&bars.out_free, lane);  // D3 may be overwritten by the next chunk's
 #pragma unroll
                     for (int j = 0; j < CH; ++j) up[j] = a[j] + bb[j];
                     tmem_ld_n<CH>(taddr(tb, 32 * q, d1 + j0), a);
