@@ -90,7 +90,8 @@ struct GdnRec {
     static constexpr uint32_t U_SLICE = C * BV * 4;               // U, fp32, one value slice
     static constexpr uint32_t U = MQK + 2 * C * 128;
     static constexpr uint32_t G = U + U_SLICE * (DV / BV);        // g_t, 64 floats
-    static constexpr uint32_t OW = G + 1024;                      // O_w, fp32 [C][DV] (rank L)
+    static constexpr uint32_t OW_SLICE = C * BV * 4;              // O_w, fp32, one value slice
+    static constexpr uint32_t OW = G + 1024;                      // O_w slices [t][BV], XOR-swizzled (rank L)
     static constexpr uint32_t FW_SLICE = DK * BV * 4;             // F_w, fp32, one value slice
     static constexpr uint32_t FW = OW + (RL ? C * DV * 4 : 0);    // F_w slices [d][BV], XOR-swizzled
     static constexpr uint32_t BYTES = FW + (RL ? FW_SLICE * (DV / BV) : 0);
@@ -686,7 +687,7 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
         }
     }
     // [sum P U; O_w]: the sum P U rows (lane quarters 0-1) become a hi / lo pair over the D U
-    // tiles, the O_w rows (quarters 2-3) are staged over K / Q ([C][DV] fp32, the record's layout)
+    // tiles, the O_w rows (quarters 2-3) are staged over K / Q in the record's layout
     if (ok) {
         const int t = 32 * (q & 1) + lane;
 #pragma unroll
@@ -703,11 +704,14 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
                     st16(sm + LY::DU, off, hv);
                     st16(sm + LY::DUL, off, lv);
                 }
-            } else {
-                float *dst = reinterpret_cast<float *>(sm + LY::KQ) + (size_t)t * DV + cc;
+            } else {  // in the record's value-slice layout
+                uint8_t *stage = sm + LY::KQ;
 #pragma unroll
-                for (int j4 = 0; j4 < 32; j4 += 4)
-                    *reinterpret_cast<float4 *>(dst + j4) = make_float4(x[j4], x[j4 + 1], x[j4 + 2], x[j4 + 3]);
+                for (int j4 = 0; j4 < 32; j4 += 4) {
+                    const int j = cc + j4;
+                    *reinterpret_cast<float4 *>(stage + (j / BV) * RC::OW_SLICE + u_off<BV>(t, j % BV)) =
+                        make_float4(x[j4], x[j4 + 1], x[j4 + 2], x[j4 + 3]);
+                }
             }
         }
     }
@@ -842,11 +846,11 @@ struct StateLayout {
     static constexpr uint32_t B_KWQ = 0;
     static constexpr uint32_t B_U = B_KWQ + KWQ_BLK * (DK / 64);
     static constexpr uint32_t B_MQ = B_U + U_BYTES;                   // [Mqk_lo; Mqk_hi]
-    static constexpr uint32_t B_G = B_MQ + 2 * C * 128;              // g (64 floats)
     static_assert(U_BYTES >= C * 128 && B_MQ % 1024 == 0, "D3's masked rows fall in U");
     static constexpr uint32_t FW_BYTES = RL ? DK * BV * 4 : 0;       // F_w slice (rank L)
-    static constexpr uint32_t B_FW = B_G + 1024;
+    static constexpr uint32_t B_FW = B_MQ + 2 * C * 128;
     static constexpr uint32_t BUF = B_FW + FW_BYTES;
+    static_assert(BUF % 1024 == 0, "the second chunk buffer's tiles stay 1024-byte aligned");
     // Y [t][hi | lo] (two buffers, by chunk parity), D Y [t][hi | lo], S^T [d][hi | lo]: MN-major,
     // 64-column blocks, in the order Y0, D Y, Y1, S.  Wk_lo of chunk c (one 64-row K-major tile per
     // 64 columns) is loaded over D Y and chunk c's Y buffer, which are free from the completion of
@@ -860,7 +864,12 @@ struct StateLayout {
     static constexpr uint32_t WKL_BLK = C * 128;
     static constexpr uint32_t S_BLK = DK * 128;
     static constexpr uint32_t S = Y1 + YT;
-    static constexpr uint32_t BYTES = S + S_BLK * (N2 / 64) + 1024;
+    // rank L: one O_w slice buffer (the output epilogue's term, loaded a chunk ahead); g of the
+    // two chunks in flight
+    static constexpr uint32_t OWB = S + S_BLK * (N2 / 64);
+    static constexpr uint32_t OW_BYTES = RL ? U_BYTES : 0;
+    static constexpr uint32_t GB = OWB + OW_BYTES;
+    static constexpr uint32_t BYTES = GB + 2 * C * 4 + 1024;
     static constexpr uint32_t y_at(int c) { return (c & 1) ? Y1 : Y0; }
     static constexpr uint32_t wkl_at(int c) { return (c & 1) ? DY : Y0; }
     // the lane-masked Wk_lo MMA reads 128 rows from each 64-column block of Wk_lo: the rows past
@@ -908,6 +917,8 @@ struct StateBars {
     uint64_t out_free;     // D3 read by the output epilogue (the warps of lane quarters 2-3)
     uint64_t d1_full, d4_full, d3_full;  // MMA -> epilogue: accumulators complete
     uint64_t lo_full;      // Wk_lo of the next chunk landed over Y / D Y (tx)
+    uint64_t ow_full;      // rank L: the chunk's O_w slice landed (tx)
+    uint64_t ow_read;      // rank L: the O_w slice read (the warps of lane quarters 2-3)
     uint64_t drain, drain3;              // the MMA threads' last operations
 };
 
@@ -977,6 +988,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
         mbar_init(&bars.d4_full, 1);
         mbar_init(&bars.d3_full, 1);
         mbar_init(&bars.lo_full, 1);
+        mbar_init(&bars.ow_full, 1);
+        mbar_init(&bars.ow_read, EPI_WARPS / 2);
         mbar_init(&bars.drain, 1);
         mbar_init(&bars.drain3, 1);
         mbar_fence_init();
@@ -1015,7 +1028,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 }
                 // once the state is large the MMA thread loads this chunk's Wk_lo: start it to L2
                 if (*(volatile int *)&big_sh) bulk_prefetch_l2(rec + RC::WKL, RC::WK_BLK * (DK / 64));
-                bulk_g2s(buf + LY::B_G, rec + RC::G, C * 4, bar);
+                bulk_g2s(sm + LY::GB + (c & 1) * C * 4, rec + RC::G, C * 4, bar);
                 if constexpr (RL)
                     bulk_g2s(buf + LY::B_FW, rec + RC::FW + blockIdx.x * RC::FW_SLICE, LY::FW_BYTES, bar);
                 issued = c;
@@ -1166,6 +1179,21 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             for (int j = 0; j < CH; ++j) m = fmaxf(m, fabsf(Sreg[j]));
             if (m > kBigState) big_sh = 1;
         };
+        // rank L: the output's O_w term arrives in one shared-memory slice buffer by a bulk copy
+        // that the first output-row thread issues once every output warp has read the previous
+        // chunk's slice (ow_read), a chunk ahead of its use
+        const bool ow_on = RL && wr && out;
+        const bool ow_issuer = tid == 64;  // warp 2, lane 0 (lane quarter 2)
+        int ow_issued = 0, ow_seen = 0;
+        auto load_ow = [&](int c) {
+            if constexpr (RL) {
+                mbar_expect_tx(&bars.ow_full, LY::OW_BYTES);
+                bulk_g2s(sm + LY::OWB, record<DK, RL>(p, ws, nch, c) + RC::OW + blockIdx.x * RC::OW_SLICE,
+                         LY::OW_BYTES, &bars.ow_full);
+                ++ow_issued;
+            }
+        };
+        if (ow_on && ow_issuer && nch > 0) load_ow(0);
         if (own_d) {
             store_half_pair<BV, CH>(sm + LY::S, LY::S_BLK, d_row, j0, Sreg);
             watch_state();
@@ -1176,7 +1204,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             const int c0 = c * C, n = min(C, T - c0);
             const uint8_t *buf = sm + (c & 1) * LY::BUF;
             if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status, lim)) { ok = false; break; }
-            const float *g = reinterpret_cast<const float *>(buf + LY::B_G);
+            const float *g = reinterpret_cast<const float *>(sm + LY::GB + (c & 1) * C * 4);
             const float g_last = g[C - 1];
             const float g_row = g[lowq ? lrow : lrow - 64];  // g of this thread's Y / output row
             const uint32_t d1 = LY::cD1 + (c & 1) * N2;
@@ -1253,23 +1281,6 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             // output O = diag(e^g) QS + Mqk Y (+ O_w), by the threads of the output rows (TMEM lanes
             // 64..127, where both the Q S rows of D1 and the whole Mqk Y term of D3 sit)
             if (!lowq) {
-                // rank L: O_w of this thread's row, loaded here because an mbarrier arrive waits
-                // for the thread's loads in flight: the next arrive (out_free) is off the chain
-                float ow[CH];
-#pragma unroll
-                for (int j = 0; j < CH; ++j) ow[j] = 0.f;
-                if (RL && wr && out && lrow - 64 < n) {
-                    const float *src = reinterpret_cast<const float *>(record<DK, RL>(p, ws, nch, c) + RC::OW) +
-                                       (size_t)(lrow - 64) * dv + v0 + j0;
-#pragma unroll
-                    for (int j4 = 0; j4 < CH; j4 += 4) {
-                        const float4 f4 = __ldg(reinterpret_cast<const float4 *>(src + j4));
-                        ow[j4] = f4.x;
-                        ow[j4 + 1] = f4.y;
-                        ow[j4 + 2] = f4.z;
-                        ow[j4 + 3] = f4.w;
-                    }
-                }
                 if (!mbar_wait(&bars.d3_full, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 const int t = lrow - 64;
@@ -1287,6 +1298,24 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < CH; ++j) qs[j] = a[j] + bb[j];
+                }
+                float ow[CH];  // rank L: O_w of this thread's row
+#pragma unroll
+                for (int j = 0; j < CH; ++j) ow[j] = 0.f;
+                if (ow_on) {
+                    if (!mbar_wait(&bars.ow_full, c & 1, status, lim)) { ok = false; break; }
+                    ++ow_seen;
+                    if (t < n) {
+#pragma unroll
+                        for (int j4 = 0; j4 < CH; j4 += 4) {
+                            const float4 f4 = *reinterpret_cast<const float4 *>(sm + LY::OWB + u_off<BV>(t, j0 + j4));
+                            ow[j4] = f4.x;
+                            ow[j4 + 1] = f4.y;
+                            ow[j4 + 2] = f4.z;
+                            ow[j4 + 3] = f4.w;
+                        }
+                    }
+                    warp_arrive(&bars.ow_read, lane);
                 }
                 if (t < n && out) {
                     const float gt = __expf(g_row);
@@ -1307,9 +1336,16 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                         *reinterpret_cast<uint4 *>(dst + c8 * 8) = pk;
                     }
                 }
+                // the next chunk's O_w slice, once every output warp has read this one
+                if (ow_on && ow_issuer && c + 1 < nch) {
+                    if (!mbar_wait(&bars.ow_read, c & 1, status, lim)) { ok = false; break; }
+                    load_ow(c + 1);
+                }
             }
         }
         if (!ok) fail();
+        // a copy still in flight (the loop stopped early) lands before the CTA exits
+        if (ow_issuer && ow_issued > ow_seen) mbar_wait(&bars.ow_full, (ow_issued - 1) & 1, nullptr, lim);
         if (p.S_final && own_d && !failed()) {
 #pragma unroll
             for (int j = 0; j < CH; ++j) p.S_final[(head * dv + v0 + j0 + j) * DK + d_row] = Sreg[j];
