@@ -157,6 +157,14 @@ __global__ void __launch_bounds__(PREP_THREADS, 4) gdn_prep_kernel(ScanArgs p, c
     const bool stall = (p.flags & kStallPrep) != 0;
     const uint32_t lim = stall ? kStallTestPolls : kWaitPolls;
 
+    // The gates first: loads issued after the tile loads wait behind their data in the SM's
+    // memory pipeline (measured ~4000 cycles on the rank-L prep), and the first epilogue needs both.
+    float g_alpha = 1.f, g_beta = 0.f;
+    if (tid < C && tid < n) {
+        const size_t bth = ((size_t)b * T + c0 + tid) * H + h;
+        g_alpha = p.alpha[bth];
+        g_beta = p.beta[bth];
+    }
     // K and Q boxes by TMA (rows past the end of the sequence arrive as zeros: identity tokens)
     if (tid == 0) {
         mbar_init(&mma_bar, 1);
@@ -173,9 +181,8 @@ __global__ void __launch_bounds__(PREP_THREADS, 4) gdn_prep_kernel(ScanArgs p, c
     }
     if (warp == 0) tmem_alloc(&tmem_base_sh, 128);
     if (tid < C) {
-        const size_t bth = ((size_t)b * T + c0 + tid) * H + h;
-        sG[tid] = tid < n ? logf(p.alpha[bth]) : 0.f;
-        sBeta[tid] = tid < n ? p.beta[bth] : 0.f;
+        sG[tid] = tid < n ? logf(g_alpha) : 0.f;
+        sBeta[tid] = g_beta;
     }
     __syncthreads();
     if (warp == 0) {
@@ -449,6 +456,14 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     };
     int w_issued = 0, u_issued = 0;  // ranks whose W / U loads were issued (thread 0)
 
+    // The gates first: loads issued after the tile loads wait behind their data in the SM's
+    // memory pipeline (measured ~4000 cycles), and the first epilogue needs both.
+    float g_alpha = 1.f, g_beta = 0.f;
+    if (tid < C && tid < n) {
+        const size_t bth = ((size_t)b * T + c0 + tid) * H + h;
+        g_alpha = p.alpha[bth];
+        g_beta = p.beta[bth];
+    }
     if (tid == 0) {
         mbar_init(&mma_bar, 1);
         mbar_init(&ld_bar, 1);
@@ -471,9 +486,8 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     }
     if (warp == 0) tmem_alloc(&tmem_base_sh, LY::TCOLS);
     if (tid < C) {
-        const size_t bth = ((size_t)b * T + c0 + tid) * H + h;
-        sG[tid] = tid < n ? logf(p.alpha[bth]) : 0.f;
-        sBeta[tid] = tid < n ? p.beta[bth] : 0.f;
+        sG[tid] = tid < n ? logf(g_alpha) : 0.f;
+        sBeta[tid] = g_beta;
     }
     __syncthreads();
     if (warp == 0) {
