@@ -42,10 +42,11 @@ namespace {
 
 constexpr int NT = 128;  // prep threads
 
-// N consecutive TMEM columns of this thread's lane (N = 8, 16 or 32; warp-collective).
+// N consecutive TMEM columns of this thread's lane (N = 4, 8, 16 or 32; warp-collective).
 template <int N>
 __device__ __forceinline__ void tmem_ld_n(uint32_t a, float (&v)[N]) {
-    if constexpr (N == 8) tmem_ld8(a, v);
+    if constexpr (N == 4) tmem_ld4(a, v);
+    else if constexpr (N == 8) tmem_ld8(a, v);
     else if constexpr (N == 16) tmem_ld16(a, v);
     else tmem_ld32(a, v);
 }
@@ -80,9 +81,9 @@ struct GdnMaps {
 
 // One workspace record per (b, h, chunk).  The rank-L record (RL) adds the write's own terms:
 // O_w = sum_l Mqw_l U_l and F_w = sum_l W_l^T D U_l; its U slot holds -X_u = -T sum_l P_l U_l.
-template <int DK, bool RL = false>
+template <int DK, bool RL = false, int BV_ = kBV<DK>>
 struct GdnRec {
-    static constexpr int DV = DK, BV = kBV<DK>;
+    static constexpr int DV = DK, BV = BV_;
     static constexpr uint32_t WK_BLK = C * 128;                  // 64 rows x 128 B per 64 columns
     static constexpr uint32_t WK = 0;                             // Wk hi, bf16, K-major SW128
     static constexpr uint32_t WKL = WK + WK_BLK * (DK / 64);      // Wk lo (= bf16(Wk - hi)), same layout
@@ -98,11 +99,13 @@ struct GdnRec {
 };
 constexpr size_t kRecOffset = 1024;  // records start after the status block
 
-// Byte offset of U[t][j] in one value slice of BV fp32 columns: 16-byte chunks XORed with t % 8,
-// so that eight consecutive rows read at one column hit eight different bank groups.
+// Byte offset of U[t][j] in one value slice of BV fp32 columns: 16-byte chunks XORed with t % 8
+// (t % 4 for BV = 16, whose rows hold four chunks), so that consecutive rows read at one column
+// hit different bank groups.
 template <int BV>
 __device__ __forceinline__ uint32_t u_off(int t, int j) {
-    return (uint32_t)t * BV * 4 + ((((uint32_t)j >> 2) ^ ((uint32_t)t & 7)) << 4) + ((uint32_t)j & 3) * 4;
+    constexpr uint32_t mask = BV >= 32 ? 7u : (uint32_t)BV / 4 - 1;
+    return (uint32_t)t * BV * 4 + ((((uint32_t)j >> 2) ^ ((uint32_t)t & mask)) << 4) + ((uint32_t)j & 3) * 4;
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -128,11 +131,11 @@ struct PrepLayout {
 // w and w + 4 split the columns of every epilogue; the solve runs on warps 0-3.
 constexpr int PREP_THREADS = 256;
 
-template <int DK>
+template <int DK, int BV_>
 __global__ void __launch_bounds__(PREP_THREADS, 4) gdn_prep_kernel(ScanArgs p, const __grid_constant__ GdnMaps maps,
                                                                   uint8_t *ws, int nch) {
     using LY = PrepLayout<DK>;
-    using RC = GdnRec<DK>;
+    using RC = GdnRec<DK, false, BV_>;
     constexpr int DV = RC::DV, BV = RC::BV;
     constexpr int NTH = PREP_THREADS, NH = NTH / 128;
     extern __shared__ uint8_t smem_raw[];
@@ -407,7 +410,7 @@ struct LPrepLayout {
 template <int DK>
 constexpr int kLPrepThreads = DK == 128 ? 512 : 256;
 
-template <int DK>
+template <int DK, int BV_>
 __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_prep_kernel(ScanArgs p, const __grid_constant__ LMaps maps,
                                                                       uint8_t *ws, int nch) {
     using LY = LPrepLayout<DK>;
@@ -415,7 +418,7 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     constexpr int NH = NTH / 128;  // column splits of an epilogue
     constexpr int CW = C / NH;     // columns of G a thread owns
     static_assert(CW == 32 || CW == 16, "the G epilogues move 16 or 32 columns a thread");
-    using RC = GdnRec<DK, true>;
+    using RC = GdnRec<DK, true, BV_>;
     constexpr int DV = RC::DV, BV = RC::BV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -847,49 +850,62 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
 // the Y / D Y tiles (free between a chunk's stage 2 MMAs and the next chunk's Y epilogue) and
 // issues 8 more MMAs on the chain at d = 128.
 
-template <int DK, bool RL = false>
+template <int DK, bool RL = false, int BV_ = kBV<DK>>
 struct StateLayout {
-    static constexpr int BV = kBV<DK>;
+    static constexpr int BV = BV_;
     static constexpr int N2 = 2 * BV;                     // hi | lo side by side
     static constexpr int CH = BV / 4;                     // columns of one epilogue warp
+    // the value tiles (S^T, Y, D Y: [k][hi | lo], MN-major B operands): 64-column blocks with the
+    // 128-byte swizzle, or at BV = 16 one 32-column block with the 64-byte swizzle
+    static constexpr bool SW64 = N2 == 32;
+    static constexpr uint32_t ROWB = SW64 ? 64 : 128;     // bytes of one row of one block
+    static constexpr int NBLK = SW64 ? 1 : N2 / 64;
+    static constexpr uint32_t VT_SBO = 8 * ROWB;          // stride of 8-row groups
+    static constexpr uint32_t VT_LAYOUT = SW64 ? 4 : 2;
     static constexpr uint32_t KWQ_BLK = 3 * C * 128;      // [K; Wk; Q] rows of one 64-col block
     static constexpr uint32_t U_BYTES = C * BV * 4;
     // double-buffered chunk inputs.  U and Mqk are loaded once the buffer's D3 has completed, so
-    // the 64 masked rows that D3's second MMA reads in front of Mqk_lo (the end of U) are not
-    // being written while it runs.
+    // the 64 masked rows that D3's second MMA reads in front of Mqk_lo (the end of the U slot,
+    // padded to 64 rows of 128 bytes) are not being written while it runs.
+    static constexpr uint32_t U_SLOT = U_BYTES >= C * 128 ? U_BYTES : C * 128;
     static constexpr uint32_t B_KWQ = 0;
     static constexpr uint32_t B_U = B_KWQ + KWQ_BLK * (DK / 64);
-    static constexpr uint32_t B_MQ = B_U + U_BYTES;                   // [Mqk_lo; Mqk_hi]
-    static_assert(U_BYTES >= C * 128 && B_MQ % 1024 == 0, "D3's masked rows fall in U");
+    static constexpr uint32_t B_MQ = B_U + U_SLOT;                   // [Mqk_lo; Mqk_hi]
+    static_assert(B_MQ % 1024 == 0, "the Mqk tile stays 1024-byte aligned");
     static constexpr uint32_t FW_BYTES = RL ? DK * BV * 4 : 0;       // F_w slice (rank L)
     static constexpr uint32_t B_FW = B_MQ + 2 * C * 128;
     static constexpr uint32_t BUF = B_FW + FW_BYTES;
     static_assert(BUF % 1024 == 0, "the second chunk buffer's tiles stay 1024-byte aligned");
-    // Y [t][hi | lo] (two buffers, by chunk parity), D Y [t][hi | lo], S^T [d][hi | lo]: MN-major,
-    // 64-column blocks, in the order Y0, D Y, Y1, S.  Wk_lo of chunk c (one 64-row K-major tile per
-    // 64 columns) is loaded over D Y and chunk c's Y buffer, which are free from the completion of
-    // D4 of chunk c - 1 (the last reader of D Y) and of D3 of chunk c - 2 (the last reader of that
-    // Y buffer) to the Y epilogue of chunk c: they are adjacent for either parity.
-    static constexpr uint32_t Y_BLK = C * 128;
-    static constexpr uint32_t YT = Y_BLK * (N2 / 64);   // one Y or D Y tile
+    // Y [t][hi | lo] (two buffers, by chunk parity), D Y [t][hi | lo], S^T [d][hi | lo], in the
+    // order Y0, D Y, Y1, S.  Wk_lo of chunk c (one 64-row K-major tile per 64 columns) is loaded
+    // over D Y and chunk c's Y buffer, which are free from the completion of D4 of chunk c - 1 (the
+    // last reader of D Y) and of D3 of chunk c - 2 (the last reader of that Y buffer) to the Y
+    // epilogue of chunk c: they are adjacent for either parity.  At BV = 16 those tiles are too
+    // small and Wk_lo has a region of its own.
+    static constexpr uint32_t Y_BLK = C * ROWB;
+    static constexpr uint32_t YT = Y_BLK * NBLK;        // one Y or D Y tile
     static constexpr uint32_t Y0 = 2 * BUF;
     static constexpr uint32_t DY = Y0 + YT;
     static constexpr uint32_t Y1 = DY + YT;
     static constexpr uint32_t WKL_BLK = C * 128;
-    static constexpr uint32_t S_BLK = DK * 128;
+    static constexpr uint32_t S_BLK = DK * ROWB;
     static constexpr uint32_t S = Y1 + YT;
     // rank L: one O_w slice buffer (the output epilogue's term, loaded a chunk ahead); g of the
     // two chunks in flight
-    static constexpr uint32_t OWB = S + S_BLK * (N2 / 64);
+    static constexpr uint32_t OWB = S + S_BLK * NBLK;
     static constexpr uint32_t OW_BYTES = RL ? U_BYTES : 0;
     static constexpr uint32_t GB = OWB + OW_BYTES;
-    static constexpr uint32_t BYTES = GB + 2 * C * 4 + 1024;
+    static constexpr bool WKL_OVER_Y = WKL_BLK * (DK / 64) <= 2 * YT;
+    // Wk_lo's own region (with one tile of room for the masked rows past its last block)
+    static constexpr uint32_t WKD = (GB + 2 * C * 4 + 1023) / 1024 * 1024;
+    static constexpr uint32_t BYTES = (WKL_OVER_Y ? GB + 2 * C * 4 : WKD + WKL_BLK * (DK / 64 + 1)) + 1024;
     static constexpr uint32_t y_at(int c) { return (c & 1) ? Y1 : Y0; }
-    static constexpr uint32_t wkl_at(int c) { return (c & 1) ? DY : Y0; }
+    static constexpr uint32_t wkl_at(int c) { return WKL_OVER_Y ? ((c & 1) ? DY : Y0) : WKD; }
     // the lane-masked Wk_lo MMA reads 128 rows from each 64-column block of Wk_lo: the rows past
     // the last block (masked, their products dropped) are still inside the allocation
-    static_assert(DY + WKL_BLK * (DK / 64) + WKL_BLK <= BYTES - 1024, "masked rows stay in bounds");
-    static_assert(WKL_BLK * (DK / 64) <= 2 * YT, "Wk_lo fits over D Y and one Y buffer");
+    static_assert(wkl_at(1) + WKL_BLK * (DK / 64) + WKL_BLK <= BYTES - 1024 &&
+                      wkl_at(0) + WKL_BLK * (DK / 64) + WKL_BLK <= BYTES - 1024,
+                  "masked rows stay in bounds");
     // TMEM columns: D1 (two buffers), D3, D4
     static constexpr uint32_t cD1 = 0, cD3 = 2 * N2, cD4 = 3 * N2;
     static constexpr uint32_t TCOLS = 4 * N2 <= 256 ? 256 : 512;
@@ -937,22 +953,32 @@ struct StateBars {
 };
 
 
-// CH fp32 values at (row, j0 .. j0+CH) as a hi / lo pair into an MN-major tile of 64-column
-// 128B-swizzled blocks: hi at columns j0.., lo at BV + j0...
+// CH fp32 values at (row, j0 .. j0+CH) as a hi / lo pair into an MN-major value tile: hi at
+// columns j0.., lo at BV + j0...; 64-column 128B-swizzled blocks, or at BV = 16 (CH = 4) one
+// 32-column 64B-swizzled block.
 template <int BV, int CH>
 __device__ __forceinline__ void store_half_pair(uint8_t *tile, uint32_t blk_bytes, int row, int j0,
                                                 const float *x) {
+    if constexpr (CH == 4) {
+        static_assert(BV == 16, "four columns a thread: the 32-column tile");
+        uint2 hv, lv;
+        split4(x, hv, lv);
+        *reinterpret_cast<uint2 *>(tile + sw64_off(row, j0)) = hv;
+        *reinterpret_cast<uint2 *>(tile + sw64_off(row, BV + j0)) = lv;
+    } else {
 #pragma unroll
-    for (int c8 = 0; c8 < CH / 8; ++c8) {
-        uint4 hv, lv;
-        split8(x + c8 * 8, hv, lv);
-        st16(tile, sw128_off(row, j0 + c8 * 8, blk_bytes), hv);
-        st16(tile, sw128_off(row, BV + j0 + c8 * 8, blk_bytes), lv);
+        for (int c8 = 0; c8 < CH / 8; ++c8) {
+            uint4 hv, lv;
+            split8(x + c8 * 8, hv, lv);
+            st16(tile, sw128_off(row, j0 + c8 * 8, blk_bytes), hv);
+            st16(tile, sw128_off(row, BV + j0 + c8 * 8, blk_bytes), lv);
+        }
     }
 }
 
 template <int DK, bool RL>
 __device__ __forceinline__ const uint8_t *record(const ScanArgs &p, const uint8_t *ws, int nch, int c) {
+    static_assert(GdnRec<DK, RL, 16>::BYTES == GdnRec<DK, RL>::BYTES, "the record's size does not depend on the slice width");
     return ws + kRecOffset + (((size_t)blockIdx.z * p.H + blockIdx.y) * nch + c) * GdnRec<DK, RL>::BYTES;
 }
 
@@ -965,12 +991,12 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
     if (lane == 0) mbar_arrive(bar);
 }
 
-template <int DK, bool RL>
+template <int DK, bool RL, int BV_>
 __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                                                                  const __grid_constant__ GdnMaps maps,
                                                                  const uint8_t *ws, int nch) {
-    using LY = StateLayout<DK, RL>;
-    using RC = GdnRec<DK, RL>;
+    using LY = StateLayout<DK, RL, BV_>;
+    using RC = GdnRec<DK, RL, BV_>;
     constexpr int BV = LY::BV, N2 = LY::N2, CH = LY::CH;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -1064,7 +1090,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
         // ---------------- D3 MMA issue ----------------
         if (lane == 0) {
             auto oK0 = [](int ks) { return (uint64_t)koff_k_sw128(ks, 0); };
-            auto oMN = [](int ks) { return (uint64_t)koff_mn_sw128(ks); };
+            auto oVT = [](int ks) { return (uint64_t)(LY::SW64 ? koff_mn_sw64(ks) : koff_mn_sw128(ks)); };
             const uint32_t idS = idesc_bf16(128, N2, 0, 1);
             uint32_t omask[4];
             lane_mask_lower(omask);  // the Mqk_lo output term: output rows only (lanes 64..127)
@@ -1082,10 +1108,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 }
                 fence_after_sync();
                 const uint32_t bb = sb + (c & 1) * LY::BUF;
-                const uint64_t dY2 = make_desc(sb + LY::y_at(c), LY::Y_BLK, 1024, 2);
-                mma_steps<C / 16>(tb + LY::cD3, idS, make_desc(bb + LY::B_MQ, 16, 1024, 2), dY2, oK0, oMN, false);
+                const uint64_t dY2 = make_desc(sb + LY::y_at(c), LY::SW64 ? 0 : LY::Y_BLK, LY::VT_SBO, LY::VT_LAYOUT);
+                mma_steps<C / 16>(tb + LY::cD3, idS, make_desc(bb + LY::B_MQ, 16, 1024, 2), dY2, oK0, oVT, false);
                 mma_steps_lanes<C / 16>(tb + LY::cD3, idS, make_desc(bb + LY::B_MQ - C * 128, 16, 1024, 2), dY2,
-                                        oK0, oMN, true, omask);
+                                        oK0, oVT, true, omask);
                 mma_commit(&bars.d3_full);
                 mma_commit(&bars.mq_empty[c & 1]);
             }
@@ -1097,9 +1123,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
         // ---------------- chain MMA issue ----------------
         if (lane == 0) {
             auto oKWQ = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::KWQ_BLK); };
-            auto oMN = [](int ks) { return (uint64_t)koff_mn_sw128(ks); };
-            const uint64_t dS2 = make_desc(sb + LY::S, LY::S_BLK, 1024, 2);
-            const uint64_t dDY2 = make_desc(sb + LY::DY, LY::Y_BLK, 1024, 2);
+            auto oMN = [](int ks) { return (uint64_t)koff_mn_sw128(ks); };  // K^T (the K tile)
+            auto oVT = [](int ks) { return (uint64_t)(LY::SW64 ? koff_mn_sw64(ks) : koff_mn_sw128(ks)); };
+            const uint64_t dS2 = make_desc(sb + LY::S, LY::SW64 ? 0 : LY::S_BLK, LY::VT_SBO, LY::VT_LAYOUT);
+            const uint64_t dDY2 = make_desc(sb + LY::DY, LY::SW64 ? 0 : LY::Y_BLK, LY::VT_SBO, LY::VT_LAYOUT);
             const uint32_t idS = idesc_bf16(128, N2, 0, 1);
             const uint32_t id4 = idesc_bf16(DK, N2, 1, 1);
             auto oLO = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::WKL_BLK); };
@@ -1126,13 +1153,26 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 // back, is done: the epilogue warps work through the chunks in order)
                 if (!mbar_wait(&bars.s_ready, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
+                // S_c turned out large after the prefetch decision for this chunk was taken: its
+                // Wk_lo is loaded now (once per CTA; every later chunk's is prefetched).  The region
+                // is free: D4 of chunk c - 1 has completed (S_c was written after it), and D3 of
+                // chunk c - 2, the last reader of Y buffer c % 2, is waited for.
+                if (!lo && *(volatile int *)&big_sh) {
+                    if (LY::WKL_OVER_Y && c >= 2 &&
+                        !mbar_wait(&bars.mq_empty[c & 1], ((c - 2) >> 1) & 1, status, lim)) {
+                        ok = false;
+                        break;
+                    }
+                    load_lo(c);
+                    lo = true;
+                }
                 const uint64_t dWQ = make_desc(bb + LY::B_KWQ + C * 128, 16, 1024, 2);
-                mma_steps<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dWQ, dS2, oKWQ, oMN, false);
+                mma_steps<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dWQ, dS2, oKWQ, oVT, false);
                 if (lo) {  // X_s += Wk_lo S, into the same accumulator with the Q S rows masked
                     if (!mbar_wait(&bars.lo_full, lo_phase & 1, status, lim)) { ok = false; break; }
                     ++lo_phase;
                     const uint64_t dLW = make_desc(sb + LY::wkl_at(c), 16, 1024, 2);
-                    mma_steps_lanes<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dLW, dS2, oLO, oMN, true, xmask);
+                    mma_steps_lanes<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dLW, dS2, oLO, oVT, true, xmask);
                     lo = false;
                 }
                 mma_commit(&bars.d1_full);
@@ -1140,7 +1180,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 if (!mbar_wait(&bars.y_ready, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 const uint64_t dKt = make_desc(bb + LY::B_KWQ, LY::KWQ_BLK, 1024, 2);
-                mma_steps<C / 16>(tb + LY::cD4, id4, dKt, dDY2, oMN, oMN, false);
+                mma_steps<C / 16>(tb + LY::cD4, id4, dKt, dDY2, oMN, oVT, false);
                 mma_commit(&bars.d4_full);
                 mma_commit(&bars.empty[c & 1]);
                 if (c + 1 < nch) {
@@ -1261,8 +1301,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
             // state update S^T <- e^{g_n} S^T + K^T D Y (+ F_w)
             {
                 const float gC = __expf(g_last);
-                if (own_d) {  // the size check of S_c and e^{g_n} S^T (+ F_w): no D4 needed yet
-                    watch_state();
+                if (own_d) {  // e^{g_n} S^T (+ F_w): no D4 needed yet
 #pragma unroll
                     for (int j = 0; j < CH; ++j) Sreg[j] *= gC;
                     if (RL && wr) {
@@ -1286,9 +1325,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD4 + BV + j0), xl);
                 tmem_wait_ld();
                 if (own_d) {
+                    float m = 0.f;  // the size check of S_{c+1}, before the MMA thread reads the flag
 #pragma unroll
-                    for (int j = 0; j < CH; ++j) Sreg[j] += xh[j] + xl[j];
+                    for (int j = 0; j < CH; ++j) {
+                        Sreg[j] += xh[j] + xl[j];
+                        m = fmaxf(m, fabsf(Sreg[j]));
+                    }
                     store_half_pair<BV, CH>(sm + LY::S, LY::S_BLK, d_row, j0, Sreg);
+                    if (m > kBigState) big_sh = 1;
                 }
             }
             warp_arrive(&bars.s_ready, lane);
@@ -1334,6 +1378,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 if (t < n && out) {
                     const float gt = __expf(g_row);
                     __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t) * H + h) * dv + v0 + j0;
+                    if constexpr (CH == 4) {  // one 8-byte store
+                        float r[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) r[j] = fmaf(gt, qs[j], up[j] + ow[j]);
+                        *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]));
+                    }
 #pragma unroll
                     for (int c8 = 0; c8 < CH / 8; ++c8) {
                         float r[8];
@@ -1405,13 +1455,37 @@ bool gdn_maps(const ScanArgs &a, GdnMaps *maps) {
            act_map(&maps->v, a.v, a.B, a.T, a.H, a.dv, 64);
 }
 
+// Host: the SM count of the current device (cached per device).
+int device_sms() {
+    static int sms[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        sms[dev] = n;
+    }
+    return sms[dev];
+}
+
+// Value-slice width of the state kernel, and of the record's slice-major parts, which the prep
+// writes to match (both take it from the same shape): 16 at d = 128 when 16-wide slices still
+// give every in-order chain an SM of its own (few sequences: each chain then moves half the value
+// columns per chunk through its SM's shared memory, on twice as many SMs), else kBV.
 template <int DK>
-cudaError_t launch_gdn_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
+int slice_width(const ScanArgs &a) {
+    if (DK != 128) return kBV<DK>;
+    const long long chains = (long long)a.B * a.H * (a.dv / 16);
+    return chains <= device_sms() ? 16 : kBV<DK>;
+}
+
+template <int DK, int BV>
+cudaError_t launch_gdn_prep_bv(const ScanArgs &a, void *ws, cudaStream_t s) {
     const int nch = (a.T + C - 1) / C;
     GdnMaps maps;
     if (!gdn_maps<DK>(a, &maps)) return cudaErrorInvalidValue;
     using LY = PrepLayout<DK>;
-    auto kern = gdn_prep_kernel<DK>;
+    auto kern = gdn_prep_kernel<DK, BV>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
     if (err != cudaSuccess) return err;
     dim3 grid(nch, a.H, a.B);
@@ -1420,16 +1494,23 @@ cudaError_t launch_gdn_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+template <int DK>
+cudaError_t launch_gdn_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
+    if constexpr (DK == 128)
+        if (slice_width<DK>(a) == 16) return launch_gdn_prep_bv<DK, 16>(a, ws, s);
+    return launch_gdn_prep_bv<DK, kBV<DK>>(a, ws, s);
+}
+
 // The state kernel reads only K and Q through tensor maps (v may be absent on the rank-L route).
-template <int DK, bool RL>
-cudaError_t launch_gdn_state_t(const ScanArgs &a, const void *ws, cudaStream_t s) {
+template <int DK, bool RL, int BV>
+cudaError_t launch_gdn_state_bv(const ScanArgs &a, const void *ws, cudaStream_t s) {
     const int nch = (a.T + C - 1) / C;
     GdnMaps maps = {};
     if (!act_map(&maps.k, a.k, a.B, a.T, a.H, DK, 64) || !act_map(&maps.q, a.q, a.B, a.T, a.H, DK, 64))
         return cudaErrorInvalidValue;
-    using LY = StateLayout<DK, RL>;
-    static_assert(LY::BYTES <= 227 * 1024, "shared memory budget");
-    auto kern = gdn_state_kernel<DK, RL>;
+    using LY = StateLayout<DK, RL, BV>;
+    static_assert(LY::BYTES + 256 <= 227 * 1024, "shared memory budget (with the static part)");
+    auto kern = gdn_state_kernel<DK, RL, BV>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
     if (err != cudaSuccess) return err;
     dim3 grid(a.dv / LY::BV, a.H, a.B);
@@ -1438,8 +1519,15 @@ cudaError_t launch_gdn_state_t(const ScanArgs &a, const void *ws, cudaStream_t s
     return cudaGetLastError();
 }
 
-template <int DK>
-cudaError_t launch_lrank_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
+template <int DK, bool RL>
+cudaError_t launch_gdn_state_t(const ScanArgs &a, const void *ws, cudaStream_t s) {
+    if constexpr (DK == 128)
+        if (slice_width<DK>(a) == 16) return launch_gdn_state_bv<DK, RL, 16>(a, ws, s);
+    return launch_gdn_state_bv<DK, RL, kBV<DK>>(a, ws, s);
+}
+
+template <int DK, int BV>
+cudaError_t launch_lrank_prep_bv(const ScanArgs &a, void *ws, cudaStream_t s) {
     const int nch = (a.T + C - 1) / C;
     LMaps maps;
     if (!act_map(&maps.k, a.k, a.B, a.T, a.H, DK, 64) || !act_map(&maps.q, a.q, a.B, a.T, a.H, DK, 64) ||
@@ -1448,13 +1536,20 @@ cudaError_t launch_lrank_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
         return cudaErrorInvalidValue;
     using LY = LPrepLayout<DK>;
     static_assert(LY::BYTES <= 227 * 1024, "shared memory budget");
-    auto kern = lrank_prep_kernel<DK>;
+    auto kern = lrank_prep_kernel<DK, BV>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
     if (err != cudaSuccess) return err;
     dim3 grid(nch, a.H, a.B);
     launch_probe_mark(s);
     kern<<<grid, kLPrepThreads<DK>, LY::BYTES, s>>>(a, maps, (uint8_t *)ws, nch);
     return cudaGetLastError();
+}
+
+template <int DK>
+cudaError_t launch_lrank_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
+    if constexpr (DK == 128)
+        if (slice_width<DK>(a) == 16) return launch_lrank_prep_bv<DK, 16>(a, ws, s);
+    return launch_lrank_prep_bv<DK, kBV<DK>>(a, ws, s);
 }
 
 }  // namespace

@@ -18,7 +18,10 @@ of the affine elements gives the same result):
 
 Every case runs on the Gated-DeltaNet route (u, w absent) and on the rank-L route, at bf16 on the
 tensor-core kernels (d = 64 and 128) and at fp32 on the CUDA-core kernel, over T = 200 tokens
-(three 64-token chunks and a ragged tail)."""
+(three 64-token chunks and a ragged tail).  At d = 128 the state kernel splits the value columns
+into slices of 16 when there are few sequences and of 32 otherwise (the slice width follows from
+B H and the SM count); the d = 128 bf16 cases run once with two heads (16-wide slices) and once
+with enough heads for 32-wide ones."""
 import numpy as np
 import pytest
 import torch
@@ -47,9 +50,14 @@ ROUTES = [("gdn", 128, 1, "bf16"), ("gdn", 64, 1, "bf16"), ("gdn", 32, 1, "f32")
 T = 200
 
 
-def _base(route, d, L, io, seed):
+def _heads_for_wide_slices():
+    """Enough heads that 16-wide value slices at d = 128 would outnumber the SMs."""
+    return torch.cuda.get_device_properties(0).multi_processor_count // 8 + 1
+
+
+def _base(route, d, L, io, seed, H=2):
     wl = WORKLOADS["gdn" if route == "gdn" else "recsys"].with_(
-        B=1, H=2, T=T, dk=d, dv=d, L=L, io=io, s0_std=0.0)
+        B=1, H=H, T=T, dk=d, dv=d, L=L, io=io, s0_std=0.0)
     return wl, make_inputs(wl, seed=seed)
 
 
@@ -123,6 +131,16 @@ def test_edge_regime_matches_oracle(case, route, d, L, io):
     wl, x = _base(route, d, L, io, seed)
     x = _edge(x, wl, case, seed)
     check_scan_full(x, wl.chunk, io)
+
+
+@pytest.mark.parametrize("case", CASES)
+@pytest.mark.parametrize("route,L", [("gdn", 1), ("rank", 2)])
+def test_edge_regime_32_wide_slices(case, route, L):
+    """The same regimes at d = 128 with enough heads for the 32-wide value slices."""
+    seed = CASES.index(case) * 7 + 128 + L + 1
+    wl, x = _base(route, 128, L, "bf16", seed, H=_heads_for_wide_slices())
+    x = _edge(x, wl, case, seed)
+    check_scan_full(x, wl.chunk, "bf16")
 
 
 def test_overwrite_returns_the_values():
