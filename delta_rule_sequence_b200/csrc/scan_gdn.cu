@@ -1153,6 +1153,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 // back, is done: the epilogue warps work through the chunks in order)
                 if (!mbar_wait(&bars.s_ready, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
+                const uint64_t dWQ = make_desc(bb + LY::B_KWQ + C * 128, 16, 1024, 2);
+                mma_steps<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dWQ, dS2, oKWQ, oVT, false);
                 // S_c turned out large after the prefetch decision for this chunk was taken: its
                 // Wk_lo is loaded now (once per CTA; every later chunk's is prefetched).  The region
                 // is free: D4 of chunk c - 1 has completed (S_c was written after it), and D3 of
@@ -1166,8 +1168,6 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                     load_lo(c);
                     lo = true;
                 }
-                const uint64_t dWQ = make_desc(bb + LY::B_KWQ + C * 128, 16, 1024, 2);
-                mma_steps<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dWQ, dS2, oKWQ, oVT, false);
                 if (lo) {  // X_s += Wk_lo S, into the same accumulator with the Q S rows masked
                     if (!mbar_wait(&bars.lo_full, lo_phase & 1, status, lim)) { ok = false; break; }
                     ++lo_phase;
@@ -1325,14 +1325,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 tmem_ld_n<CH>(taddr(tb, 32 * q, LY::cD4 + BV + j0), xl);
                 tmem_wait_ld();
                 if (own_d) {
-                    float m = 0.f;  // the size check of S_{c+1}, before the MMA thread reads the flag
+                    float m[2] = {0.f, 0.f};  // the size check of S_{c+1} (two independent chains)
 #pragma unroll
                     for (int j = 0; j < CH; ++j) {
                         Sreg[j] += xh[j] + xl[j];
-                        m = fmaxf(m, fabsf(Sreg[j]));
+                        m[j & 1] = fmaxf(m[j & 1], fabsf(Sreg[j]));
                     }
                     store_half_pair<BV, CH>(sm + LY::S, LY::S_BLK, d_row, j0, Sreg);
-                    if (m > kBigState) big_sh = 1;
+                    if (fmaxf(m[0], m[1]) > kBigState) big_sh = 1;
                 }
             }
             warp_arrive(&bars.s_ready, lane);
