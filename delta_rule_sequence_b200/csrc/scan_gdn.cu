@@ -385,18 +385,23 @@ struct LPrepLayout {
     static constexpr uint32_t DUL = DU + BLK * (DK / 64);
     static constexpr uint32_t T1 = DUL + BLK * (DK / 64);    // T diag(beta gamma), then T: hi, lo
     static constexpr uint32_t T1L = T1 + BLK;
-    // [P_l; Mqw_l] as two M = 128 operands: the lo rows after the T tiles, the hi rows over the
-    // solve buffer (free once both T tiles are built)
+    // At d = 128 the solve (warps 0-7) and the rank loop (warps 8-15) run at the same time; at
+    // d = 64 (8 warps, two CTAs per SM) one after the other.
+    static constexpr bool SPLIT = DK == 128;
+    // [P_l; Mqw_l] as two M = 128 operands: the lo rows after the T tiles, the hi rows after them
+    // (SPLIT) or over the solve buffer (free once both T tiles are built)
     static constexpr uint32_t PL = T1L + BLK;
     static constexpr uint32_t MQWL = PL + BLK;
-    static constexpr uint32_t AF = MQWL + BLK;               // fp32 A, solved in place into T
-    static constexpr uint32_t P = AF;
+    static constexpr uint32_t AF = MQWL + BLK + (SPLIT ? 2 * BLK : 0);  // fp32 A, solved in place into T
+    static constexpr uint32_t P = SPLIT ? MQWL + BLK : AF;
     static constexpr uint32_t MQW = P + BLK;
     static constexpr uint32_t TMP = AF + C * AS * 4;
     static constexpr uint32_t GATES = TMP + kSolveTmpFloats * 4;   // g, beta, gamma, D
     static constexpr uint32_t BYTES = GATES + 4 * C * 4 + 1024;
     static_assert(KQ_BLK * (DK / 64) >= (uint32_t)C * DK * 4, "-X_u staging fits over K and Q");
-    static_assert(MQW + BLK <= TMP, "the hi P / Mqw rows fit over the solve matrix");
+    static_assert(SPLIT || MQW + BLK <= TMP, "the hi P / Mqw rows fit over the solve matrix");
+    static_assert(!SPLIT || (MQW + BLK == AF && MQWL + BLK == P && (uint32_t)C * DK * 4 <= 4 * BLK),
+                  "O_w is staged over the four [P; Mqw] tiles");
     static_assert(DK == 128 || 2 * (BYTES + 1024 + 64) <= 228 * 1024, "two CTAs share an SM at d = 64");
     // TMEM: G (64 columns, M = 128); Wk, then [sum P U; O_w] (M = 128), then X_u (DK columns);
     // F_w as its D U_hi and D U_lo halves (2 DK columns)
@@ -570,13 +575,16 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     fence_async_smem();
     fence_before_sync();
     __syncthreads();
-    if (ok && tid == 0) {  // Mqk hi then lo: the PL and MQWL tiles are adjacent, as in the record
+    // Mqk hi then lo (the PL and MQWL tiles are adjacent, as in the record), stored by the thread
+    // that later waits for the store before the P / Mqw epilogue writes those tiles
+    constexpr int kRankIssuer = LY::SPLIT ? 256 : 0;
+    if (ok && tid == kRankIssuer) {
         bulk_s2g(rec + RC::MQK, sm + LY::PL, 2 * C * 128);
         bulk_commit();
     }
     // T pair tiles: T diag(beta gamma) for Wk, then T itself for X_u
-    auto store_t_pair = [&](bool scaled) {
-        for (int e = tid; e < C * (C / 8); e += NTH) {
+    auto store_t_pair = [&](bool scaled, int first, int step) {
+        for (int e = first; e < C * (C / 8); e += step) {
             const int t = e / (C / 8), c8 = e % (C / 8);
             float a[8];
             vld<8>(sA + t * AS + c8 * 8, a);
@@ -592,175 +600,373 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
             st16(sm + LY::T1L, off, lv);
         }
     };
-    if (ok) {
-        if constexpr (NTH == 512) {  // the solve on warps 0-7
-            if (tid < 256) solve_unit_lower<256>(sA, sA, sTmp, tid, [] { named_sync(3, 256); });
-            __syncthreads();
-        } else {
+    if constexpr (!LY::SPLIT) {
+        if (ok) {
             solve_unit_lower<NTH>(sA, sA, sTmp, tid);  // ends with a CTA barrier
-        }
-        store_t_pair(true);
-    }
-    sync_for_mma();
-    // Wk = T diag(beta gamma) K  (M = 64; row r of an M = 64 accumulator sits in lane 32 (r / 16) + r % 16)
-    const uint64_t dKmn = make_desc(sb + LY::KQ, LY::KQ_BLK, 1024, 2);
-    if (ok && tid == 0) {
-        const uint32_t id = idesc_bf16(64, DK, 0, 1);
-        mma_steps<C / 16>(tb + LY::cA, id, make_desc(sb + LY::T1, 16, 1024, 2), dKmn, ok0, omn, false);
-        mma_steps<C / 16>(tb + LY::cA, id, make_desc(sb + LY::T1L, 16, 1024, 2), dKmn, ok0, omn, true);
-    }
-    ok = mma_done(ok);
-    const bool own_t = lane < 16;
-    const int t_row = 16 * q + lane;
-    if (ok) {
-#pragma unroll
-        for (int cc = hs * (DK / NH); cc < (hs + 1) * (DK / NH); cc += 32) {
-            float x[32];
-            tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
-            tmem_wait_ld();
-            if (own_t) store32_split(sm + LY::DU, sm + LY::DUL, t_row, cc, x, LY::BLK);
-        }
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    if (ok && tid == 0) {  // Wk hi then lo: DU and DUL are adjacent, as WK and WKL in the record
-        static_assert(LY::DUL == LY::DU + RC::WK_BLK * (DK / 64) && RC::WKL == RC::WK + RC::WK_BLK * (DK / 64) &&
-                          LY::BLK == RC::WK_BLK,
-                      "the staged Wk pair has the record's layout");
-        bulk_s2g(rec + RC::WK, sm + LY::DU, 2 * RC::WK_BLK * (DK / 64));
-        bulk_commit();
-    }
-    if (ok) store_t_pair(false);  // the Wk MMA has completed: the T tiles are free
-
-    // the write terms, one rank at a time.  G_l = [K; Q] W_l^T is issued together with the
-    // previous rank's MMAs (W is double-buffered), so each rank waits for one MMA batch.
-    const uint32_t idV = idesc_bf16(64, DV, 0, 1);
-    auto issue_g = [&](int l) {  // thread 0, once W_l has landed
-        const uint64_t dW = make_desc(sb + LY::W + (l & 1) * LY::TILE, 16, 1024, 2);
-        mma_steps<DK / 16>(tb + LY::cG, idesc_bf16(128, C, 0, 0), dKQ, dW, okq, okb, false);
-    };
-    if (ok && tid == 0) {
-        if (mbar_wait(&w_bar[0], 0, p.status, lim)) issue_g(0);
-        else failed_sh = 1;
-        bulk_wait_read();  // the staged Mqk and Wk are read out: the rank loop writes those tiles
-    }
-    ok = mma_done(ok);
-    for (int l = 0; l < L && ok; ++l) {
-        const uint32_t wb = LY::W + (l & 1) * LY::TILE, ub = LY::U + (l % NBU) * LY::TILE;
-        const uint64_t dWmn = make_desc(sb + wb, LY::BLK, 1024, 2);
-        const uint64_t dU = make_desc(sb + ub, LY::BLK, 1024, 2);
-        if (tid == 0 && l + 2 < L) {  // the rank after the ones in flight: start it toward L2
-            for (int blk = 0; blk < DK / 64; ++blk) {
-                tma_prefetch_4d(&maps.w, blk * 64, h * L + l + 2, c0, b);
-                tma_prefetch_4d(&maps.u, blk * 64, h * L + l + 2, c0, b);
-            }
-        }
-        {   // P_l (rows of K W^T, quarters 0-1) and Mqw_l (rows of Q W^T, quarters 2-3) as pairs
-            float gr[CW];
-            tmem_ld_n<CW>(taddr(tb, 32 * q, LY::cG + cg), gr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < CW; ++j) gr[j] *= dec[j];
-            store_split_n<CW>(sm + (q < 2 ? LY::P : LY::MQW), sm + (q < 2 ? LY::PL : LY::MQWL), t_g, cg, gr);
-        }
-        if (!mbar_wait(&u_bar[l % NBU], (l / NBU) & 1, p.status, lim)) failed_sh = 1;
-        for (int e = tid; e < C * (DV / 8); e += NTH) {  // D U_l as a hi / lo pair
-            const int t = e / (DV / 8), c8 = e % (DV / 8);
-            const uint32_t off = sw128_off(t, c8 * 8, LY::BLK);
-            const uint4 uv = *reinterpret_cast<const uint4 *>(sm + ub + off);
-            const __nv_bfloat16 *hv = reinterpret_cast<const __nv_bfloat16 *>(&uv);
-            float du[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) du[j] = sD[t] * __bfloat162float(hv[j]);
-            uint4 dh, dl;
-            split8(du, dh, dl);
-            st16(sm + LY::DU, off, dh);
-            st16(sm + LY::DUL, off, dl);
+            store_t_pair(true, tid, NTH);
         }
         sync_for_mma();
-        ok = failed_sh == 0;
+        // Wk = T diag(beta gamma) K  (M = 64; row r of an M = 64 accumulator sits in lane 32 (r / 16) + r % 16)
+        const uint64_t dKmn = make_desc(sb + LY::KQ, LY::KQ_BLK, 1024, 2);
         if (ok && tid == 0) {
-            const bool acc = l > 0;
-            // [sum P U; O_w] += [P_l; Mqw_l] U_l  (M = 128, accumulated over l in the Wk columns)
-            const uint32_t idPU = idesc_bf16(128, DV, 0, 1);
-            mma_steps<C / 16>(tb + LY::cA, idPU, make_desc(sb + LY::P, 16, 1024, 2), dU, ok0, omn, acc);
-            mma_steps<C / 16>(tb + LY::cA, idPU, make_desc(sb + LY::PL, 16, 1024, 2), dU, ok0, omn, true);
-            // F_w += W_l^T [D U_l hi | D U_l lo]  (M = DK: W_l read as an MN-major A operand;
-            // N = 2 DV: the D U tiles sit side by side as one operand)
-            const uint32_t idF = idesc_bf16(DK, 2 * DV, 1, 1);
-            mma_steps<C / 16>(tb + LY::cF, idF, dWmn, make_desc(sb + LY::DU, LY::BLK, 1024, 2), omn, omn, acc);
-            // the next rank's G (its epilogue read of the G columns above is complete)
-            if (l + 1 < L) {
-                if (mbar_wait(&w_bar[(l + 1) & 1], ((l + 1) >> 1) & 1, p.status, lim)) issue_g(l + 1);
-                else failed_sh = 1;
-            }
+            const uint32_t id = idesc_bf16(64, DK, 0, 1);
+            mma_steps<C / 16>(tb + LY::cA, id, make_desc(sb + LY::T1, 16, 1024, 2), dKmn, ok0, omn, false);
+            mma_steps<C / 16>(tb + LY::cA, id, make_desc(sb + LY::T1L, 16, 1024, 2), dKmn, ok0, omn, true);
         }
         ok = mma_done(ok);
-        // rank l's W and U buffers are free: W_{l+2} and U_{l+NBU} load into them
-        if (ok && tid == 0) {
-            if (w_issued < L) load_w(w_issued++);
-            if (u_issued < L) load_u(u_issued++);
+        const bool own_t = lane < 16;
+        const int t_row = 16 * q + lane;
+        if (ok) {
+    #pragma unroll
+            for (int cc = hs * (DK / NH); cc < (hs + 1) * (DK / NH); cc += 32) {
+                float x[32];
+                tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
+                tmem_wait_ld();
+                if (own_t) store32_split(sm + LY::DU, sm + LY::DUL, t_row, cc, x, LY::BLK);
+            }
         }
-    }
-    // [sum P U; O_w]: the sum P U rows (lane quarters 0-1) become a hi / lo pair over the D U
-    // tiles, the O_w rows (quarters 2-3) are staged over K / Q in the record's layout
-    if (ok) {
-        const int t = 32 * (q & 1) + lane;
-#pragma unroll
-        for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
-            float x[32];
-            tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
-            tmem_wait_ld();
-            if (q < 2) {
-#pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
-                    uint4 hv, lv;
-                    split8(x + 8 * c8, hv, lv);
-                    const uint32_t off = sw128_off(t, cc + 8 * c8, LY::BLK);
-                    st16(sm + LY::DU, off, hv);
-                    st16(sm + LY::DUL, off, lv);
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        if (ok && tid == 0) {  // Wk hi then lo: DU and DUL are adjacent, as WK and WKL in the record
+            static_assert(LY::DUL == LY::DU + RC::WK_BLK * (DK / 64) && RC::WKL == RC::WK + RC::WK_BLK * (DK / 64) &&
+                              LY::BLK == RC::WK_BLK,
+                          "the staged Wk pair has the record's layout");
+            bulk_s2g(rec + RC::WK, sm + LY::DU, 2 * RC::WK_BLK * (DK / 64));
+            bulk_commit();
+        }
+        if (ok) store_t_pair(false, tid, NTH);  // the Wk MMA has completed: the T tiles are free
+
+        // the write terms, one rank at a time.  G_l = [K; Q] W_l^T is issued together with the
+        // previous rank's MMAs (W is double-buffered), so each rank waits for one MMA batch.
+        const uint32_t idV = idesc_bf16(64, DV, 0, 1);
+        auto issue_g = [&](int l) {  // thread 0, once W_l has landed
+            const uint64_t dW = make_desc(sb + LY::W + (l & 1) * LY::TILE, 16, 1024, 2);
+            mma_steps<DK / 16>(tb + LY::cG, idesc_bf16(128, C, 0, 0), dKQ, dW, okq, okb, false);
+        };
+        if (ok && tid == 0) {
+            if (mbar_wait(&w_bar[0], 0, p.status, lim)) issue_g(0);
+            else failed_sh = 1;
+            bulk_wait_read();  // the staged Mqk and Wk are read out: the rank loop writes those tiles
+        }
+        ok = mma_done(ok);
+        for (int l = 0; l < L && ok; ++l) {
+            const uint32_t wb = LY::W + (l & 1) * LY::TILE, ub = LY::U + (l % NBU) * LY::TILE;
+            const uint64_t dWmn = make_desc(sb + wb, LY::BLK, 1024, 2);
+            const uint64_t dU = make_desc(sb + ub, LY::BLK, 1024, 2);
+            if (tid == 0 && l + 2 < L) {  // the rank after the ones in flight: start it toward L2
+                for (int blk = 0; blk < DK / 64; ++blk) {
+                    tma_prefetch_4d(&maps.w, blk * 64, h * L + l + 2, c0, b);
+                    tma_prefetch_4d(&maps.u, blk * 64, h * L + l + 2, c0, b);
                 }
-            } else {  // in the record's value-slice layout
-                uint8_t *stage = sm + LY::KQ;
-#pragma unroll
-                for (int j4 = 0; j4 < 32; j4 += 4) {
-                    const int j = cc + j4;
-                    *reinterpret_cast<float4 *>(stage + (j / BV) * RC::OW_SLICE + u_off<BV>(t, j % BV)) =
-                        make_float4(x[j4], x[j4 + 1], x[j4 + 2], x[j4 + 3]);
+            }
+            {   // P_l (rows of K W^T, quarters 0-1) and Mqw_l (rows of Q W^T, quarters 2-3) as pairs
+                float gr[CW];
+                tmem_ld_n<CW>(taddr(tb, 32 * q, LY::cG + cg), gr);
+                tmem_wait_ld();
+    #pragma unroll
+                for (int j = 0; j < CW; ++j) gr[j] *= dec[j];
+                store_split_n<CW>(sm + (q < 2 ? LY::P : LY::MQW), sm + (q < 2 ? LY::PL : LY::MQWL), t_g, cg, gr);
+            }
+            if (!mbar_wait(&u_bar[l % NBU], (l / NBU) & 1, p.status, lim)) failed_sh = 1;
+            for (int e = tid; e < C * (DV / 8); e += NTH) {  // D U_l as a hi / lo pair
+                const int t = e / (DV / 8), c8 = e % (DV / 8);
+                const uint32_t off = sw128_off(t, c8 * 8, LY::BLK);
+                const uint4 uv = *reinterpret_cast<const uint4 *>(sm + ub + off);
+                const __nv_bfloat16 *hv = reinterpret_cast<const __nv_bfloat16 *>(&uv);
+                float du[8];
+    #pragma unroll
+                for (int j = 0; j < 8; ++j) du[j] = sD[t] * __bfloat162float(hv[j]);
+                uint4 dh, dl;
+                split8(du, dh, dl);
+                st16(sm + LY::DU, off, dh);
+                st16(sm + LY::DUL, off, dl);
+            }
+            sync_for_mma();
+            ok = failed_sh == 0;
+            if (ok && tid == 0) {
+                const bool acc = l > 0;
+                // [sum P U; O_w] += [P_l; Mqw_l] U_l  (M = 128, accumulated over l in the Wk columns)
+                const uint32_t idPU = idesc_bf16(128, DV, 0, 1);
+                mma_steps<C / 16>(tb + LY::cA, idPU, make_desc(sb + LY::P, 16, 1024, 2), dU, ok0, omn, acc);
+                mma_steps<C / 16>(tb + LY::cA, idPU, make_desc(sb + LY::PL, 16, 1024, 2), dU, ok0, omn, true);
+                // F_w += W_l^T [D U_l hi | D U_l lo]  (M = DK: W_l read as an MN-major A operand;
+                // N = 2 DV: the D U tiles sit side by side as one operand)
+                const uint32_t idF = idesc_bf16(DK, 2 * DV, 1, 1);
+                mma_steps<C / 16>(tb + LY::cF, idF, dWmn, make_desc(sb + LY::DU, LY::BLK, 1024, 2), omn, omn, acc);
+                // the next rank's G (its epilogue read of the G columns above is complete)
+                if (l + 1 < L) {
+                    if (mbar_wait(&w_bar[(l + 1) & 1], ((l + 1) >> 1) & 1, p.status, lim)) issue_g(l + 1);
+                    else failed_sh = 1;
+                }
+            }
+            ok = mma_done(ok);
+            // rank l's W and U buffers are free: W_{l+2} and U_{l+NBU} load into them
+            if (ok && tid == 0) {
+                if (w_issued < L) load_w(w_issued++);
+                if (u_issued < L) load_u(u_issued++);
+            }
+        }
+        // [sum P U; O_w]: the sum P U rows (lane quarters 0-1) become a hi / lo pair over the D U
+        // tiles, the O_w rows (quarters 2-3) are staged over K / Q in the record's layout
+        if (ok) {
+            const int t = 32 * (q & 1) + lane;
+    #pragma unroll
+            for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
+                float x[32];
+                tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
+                tmem_wait_ld();
+                if (q < 2) {
+    #pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        uint4 hv, lv;
+                        split8(x + 8 * c8, hv, lv);
+                        const uint32_t off = sw128_off(t, cc + 8 * c8, LY::BLK);
+                        st16(sm + LY::DU, off, hv);
+                        st16(sm + LY::DUL, off, lv);
+                    }
+                } else {  // in the record's value-slice layout
+                    uint8_t *stage = sm + LY::KQ;
+    #pragma unroll
+                    for (int j4 = 0; j4 < 32; j4 += 4) {
+                        const int j = cc + j4;
+                        *reinterpret_cast<float4 *>(stage + (j / BV) * RC::OW_SLICE + u_off<BV>(t, j % BV)) =
+                            make_float4(x[j4], x[j4 + 1], x[j4 + 2], x[j4 + 3]);
+                    }
                 }
             }
         }
-    }
-    sync_for_mma();
-    static_assert(C * DV * 4 <= LY::KQ_BLK * (DK / 64), "O_w fits over K and Q");
-    static_assert(RC::FW_SLICE * (DV / BV) <= LY::DU - LY::W, "F_w fits over W and U");
-    if (ok && tid == 0) {
-        bulk_s2g(rec + RC::OW, sm + LY::KQ, C * DV * 4);
-        bulk_commit();
-    }
-    // X_u = T (sum P U)  (M = 64, into the same columns)
-    if (ok && tid == 0) {
-        const uint64_t dPU = make_desc(sb + LY::DU, LY::BLK, 1024, 2);
-        const uint64_t dPUL = make_desc(sb + LY::DUL, LY::BLK, 1024, 2);
-        const uint64_t dT = make_desc(sb + LY::T1, 16, 1024, 2), dTL = make_desc(sb + LY::T1L, 16, 1024, 2);
-        mma_steps<C / 16>(tb + LY::cA, idV, dT, dPU, ok0, omn, false);
-        mma_steps<C / 16>(tb + LY::cA, idV, dT, dPUL, ok0, omn, true);
-        mma_steps<C / 16>(tb + LY::cA, idV, dTL, dPU, ok0, omn, true);
-        mma_commit(&mma_bar);
-    }
-    // F_w (its MMAs are complete) while X_u runs: the D U_hi and D U_lo halves summed; rows d:
-    // lane = d for M = 128 (DK = 128), lanes 32q + r, r < 16, for M = 64
-    if (ok) {
-        const bool own_d = (DK == 128) ? true : (lane < 16);
-        const int d_row = (DK == 128) ? 32 * q + lane : (16 * q + lane);
+        sync_for_mma();
+        static_assert(C * DV * 4 <= LY::KQ_BLK * (DK / 64), "O_w fits over K and Q");
+        static_assert(RC::FW_SLICE * (DV / BV) <= LY::DU - LY::W, "F_w fits over W and U");
+        if (ok && tid == 0) {
+            bulk_s2g(rec + RC::OW, sm + LY::KQ, C * DV * 4);
+            bulk_commit();
+        }
+        // X_u = T (sum P U)  (M = 64, into the same columns)
+        if (ok && tid == 0) {
+            const uint64_t dPU = make_desc(sb + LY::DU, LY::BLK, 1024, 2);
+            const uint64_t dPUL = make_desc(sb + LY::DUL, LY::BLK, 1024, 2);
+            const uint64_t dT = make_desc(sb + LY::T1, 16, 1024, 2), dTL = make_desc(sb + LY::T1L, 16, 1024, 2);
+            mma_steps<C / 16>(tb + LY::cA, idV, dT, dPU, ok0, omn, false);
+            mma_steps<C / 16>(tb + LY::cA, idV, dT, dPUL, ok0, omn, true);
+            mma_steps<C / 16>(tb + LY::cA, idV, dTL, dPU, ok0, omn, true);
+            mma_commit(&mma_bar);
+        }
+        // F_w (its MMAs are complete) while X_u runs: the D U_hi and D U_lo halves summed; rows d:
+        // lane = d for M = 128 (DK = 128), lanes 32q + r, r < 16, for M = 64
+        if (ok) {
+            const bool own_d = (DK == 128) ? true : (lane < 16);
+            const int d_row = (DK == 128) ? 32 * q + lane : (16 * q + lane);
+    #pragma unroll
+            for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 16) {
+                float xh[16], xl[16];
+                tmem_ld16(taddr(tb, 32 * q, LY::cF + cc), xh);
+                tmem_ld16(taddr(tb, 32 * q, LY::cF + DV + cc), xl);
+                tmem_wait_ld();
+                if (own_d) {  // staged over W / U in the record's layout
+    #pragma unroll
+                    for (int j4 = 0; j4 < 16; j4 += 4) {
+                        const int j = cc + j4;
+                        *reinterpret_cast<float4 *>(sm + LY::W + (j / BV) * RC::FW_SLICE + u_off<BV>(d_row, j % BV)) =
+                            make_float4(xh[j4] + xl[j4], xh[j4 + 1] + xl[j4 + 1], xh[j4 + 2] + xl[j4 + 2],
+                                        xh[j4 + 3] + xl[j4 + 3]);
+                    }
+                }
+            }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        if (ok && tid == 0) {
+            bulk_s2g(rec + RC::FW, sm + LY::W, RC::FW_SLICE * (DV / BV));
+            bulk_commit();
+            bulk_wait_read_n<1>();  // the O_w store has read K / Q, where -X_u is staged next
+        }
+        ok = mma_done_committed(ok);
+        // -X_u -> the U slot (staged over K and Q in the record's slice layout, one bulk store)
+        if (ok) {
+            uint8_t *stage = sm + LY::KQ;
+    #pragma unroll
+            for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
+                float x[32];
+                tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
+                tmem_wait_ld();
+                if (own_t) {
+    #pragma unroll
+                    for (int j4 = 0; j4 < 32; j4 += 4) {
+                        const int j = cc + j4;
+                        *reinterpret_cast<float4 *>(stage + (j / BV) * RC::U_SLICE + u_off<BV>(t_row, j % BV)) =
+                            make_float4(-x[j4], -x[j4 + 1], -x[j4 + 2], -x[j4 + 3]);
+                    }
+                }
+            }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        if (ok && tid == 0) {
+            bulk_s2g(rec + RC::U, sm + LY::KQ, (uint32_t)(C * DV * 4));
+            bulk_commit();
+            bulk_wait_read();  // the staging buffer is read out before the CTA frees it; the kernel's
+                               // end makes the writes visible to the next launch
+        }
+    } else {
+        // ---- d = 128: the solve (warps 0-7) and the rank loop (warps 8-15) at the same time; the
+        // rank loop needs none of T (only Wk and X_u do, and they follow the join) ----
+        constexpr int GS = 256, GR = NTH - GS;  // the two groups' threads
+        const bool r_issuer = tid == kRankIssuer;
+        const uint32_t idV = idesc_bf16(64, DV, 0, 1);
+        const uint64_t dKmn = make_desc(sb + LY::KQ, LY::KQ_BLK, 1024, 2);
+        const bool own_t = lane < 16;
+        const int t_row = 16 * q + lane;
+        int w_next = stall ? 0 : (L < 2 ? L : 2), u_next = stall ? 0 : (L < NBU ? L : NBU);  // (issuer)
+        if (tid < GS) {
+            if (ok) {
+                solve_unit_lower<GS>(sA, sA, sTmp, tid, [] { named_sync(3, GS); });
+                store_t_pair(true, tid, GS);  // T diag(beta gamma) for Wk
+            }
+        } else {
+            // The write terms, one rank at a time, on this group's 8 warps (TMEM lane quarter
+            // warp % 4, two column halves).  G_l = [K; Q] W_l^T is issued together with the
+            // previous rank's MMAs (W is double-buffered), so each rank waits for one MMA batch.
+            constexpr int CWR = C / 2;
+            const int cgr = ((warp - GS / 32) >> 2) * CWR;
+            const int rt = tid - GS;
+            float decr[CWR];  // the G epilogue factors of this thread's row and columns
+            {
+                const float gt = sG[t_g], sc = q < 2 ? sBeta[t_g] : 1.f;
 #pragma unroll
-        for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 16) {
-            float xh[16], xl[16];
-            tmem_ld16(taddr(tb, 32 * q, LY::cF + cc), xh);
-            tmem_ld16(taddr(tb, 32 * q, LY::cF + DV + cc), xl);
-            tmem_wait_ld();
-            if (own_d) {  // staged over W / U in the record's layout
+                for (int j = 0; j < CWR; ++j) {
+                    const int i = cgr + j;
+                    decr[j] = (q < 2 ? i < t_g : i <= t_g) ? sc * __expf(gt - sG[i]) : 0.f;
+                }
+            }
+            uint32_t rph = mph;  // mma_bar phases this group has waited for
+            auto r_done = [&](bool issued) -> bool {  // the issuer commits; the group waits
+                if (r_issuer && issued) mma_commit(&mma_bar);
+                __syncwarp();
+                if (issued && !mbar_wait(&mma_bar, rph & 1, p.status, lim)) failed_sh = 1;
+                if (issued) rph++;
+                fence_after_sync();
+                named_sync(4, GR);
+                return failed_sh == 0;
+            };
+            auto issue_g = [&](int l) {  // the issuer, once W_l has landed
+                const uint64_t dW = make_desc(sb + LY::W + (l & 1) * LY::TILE, 16, 1024, 2);
+                mma_steps<DK / 16>(tb + LY::cG, idesc_bf16(128, C, 0, 0), dKQ, dW, okq, okb, false);
+            };
+            bool rok = ok;
+            if (rok && r_issuer) {
+                if (mbar_wait(&w_bar[0], 0, p.status, lim)) issue_g(0);
+                else failed_sh = 1;
+                bulk_wait_read();  // the staged Mqk is read out: the P / Mqw epilogue writes its tiles
+            }
+            rok = r_done(rok);
+            for (int l = 0; l < L && rok; ++l) {
+                const uint32_t wb = LY::W + (l & 1) * LY::TILE, ub = LY::U + (l % NBU) * LY::TILE;
+                const uint64_t dWmn = make_desc(sb + wb, LY::BLK, 1024, 2);
+                const uint64_t dU = make_desc(sb + ub, LY::BLK, 1024, 2);
+                if (r_issuer && l + 2 < L) {  // the rank after the ones in flight: start it toward L2
+                    for (int blk = 0; blk < DK / 64; ++blk) {
+                        tma_prefetch_4d(&maps.w, blk * 64, h * L + l + 2, c0, b);
+                        tma_prefetch_4d(&maps.u, blk * 64, h * L + l + 2, c0, b);
+                    }
+                }
+                {   // P_l (rows of K W^T, quarters 0-1) and Mqw_l (rows of Q W^T, quarters 2-3) as pairs
+                    float gr[CWR];
+                    tmem_ld_n<CWR>(taddr(tb, 32 * q, LY::cG + cgr), gr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < CWR; ++j) gr[j] *= decr[j];
+                    store_split_n<CWR>(sm + (q < 2 ? LY::P : LY::MQW), sm + (q < 2 ? LY::PL : LY::MQWL), t_g, cgr, gr);
+                }
+                if (!mbar_wait(&u_bar[l % NBU], (l / NBU) & 1, p.status, lim)) failed_sh = 1;
+                for (int e = rt; e < C * (DV / 8); e += GR) {  // D U_l as a hi / lo pair
+                    const int t = e / (DV / 8), c8 = e % (DV / 8);
+                    const uint32_t off = sw128_off(t, c8 * 8, LY::BLK);
+                    const uint4 uv = *reinterpret_cast<const uint4 *>(sm + ub + off);
+                    const __nv_bfloat16 *hv = reinterpret_cast<const __nv_bfloat16 *>(&uv);
+                    float du[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) du[j] = sD[t] * __bfloat162float(hv[j]);
+                    uint4 dh, dl;
+                    split8(du, dh, dl);
+                    st16(sm + LY::DU, off, dh);
+                    st16(sm + LY::DUL, off, dl);
+                }
+                fence_async_smem();
+                fence_before_sync();
+                named_sync(4, GR);
+                fence_after_sync();
+                rok = failed_sh == 0;
+                if (rok && r_issuer) {
+                    const bool acc = l > 0;
+                    // [sum P U; O_w] += [P_l; Mqw_l] U_l  (M = 128, accumulated over l)
+                    const uint32_t idPU = idesc_bf16(128, DV, 0, 1);
+                    mma_steps<C / 16>(tb + LY::cA, idPU, make_desc(sb + LY::P, 16, 1024, 2), dU, ok0, omn, acc);
+                    mma_steps<C / 16>(tb + LY::cA, idPU, make_desc(sb + LY::PL, 16, 1024, 2), dU, ok0, omn, true);
+                    // F_w += W_l^T [D U_l hi | D U_l lo]  (M = DK: W_l read as an MN-major A operand;
+                    // N = 2 DV: the D U tiles sit side by side as one operand)
+                    const uint32_t idF = idesc_bf16(DK, 2 * DV, 1, 1);
+                    mma_steps<C / 16>(tb + LY::cF, idF, dWmn, make_desc(sb + LY::DU, LY::BLK, 1024, 2), omn, omn, acc);
+                    // the next rank's G (its epilogue read of the G columns above is complete)
+                    if (l + 1 < L) {
+                        if (mbar_wait(&w_bar[(l + 1) & 1], ((l + 1) >> 1) & 1, p.status, lim)) issue_g(l + 1);
+                        else failed_sh = 1;
+                    }
+                }
+                rok = r_done(rok);
+                // rank l's W and U buffers are free: W_{l+2} and U_{l+NBU} load into them
+                if (rok && r_issuer) {
+                    if (w_next < L) load_w(w_next++);
+                    if (u_next < L) load_u(u_next++);
+                }
+            }
+        }
+        // the join: T diag(beta gamma) built, every rank's MMAs complete
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        ok = failed_sh == 0;
+        mph = 2 + L;  // G, G_0 and one batch per rank have completed on mma_bar
+        // [sum P U; O_w] and F_w read out: the sum P U rows (lane quarters 0-1) become a hi / lo
+        // pair over the D U tiles (X_u's operand); O_w (quarters 2-3) is staged over the four
+        // [P; Mqw] tiles and F_w (its D U_hi and D U_lo halves summed; row d = lane) over W / U,
+        // both in the record's value-slice layout
+        if (ok) {
+            const int t = 32 * (q & 1) + lane;
+#pragma unroll
+            for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
+                float x[32];
+                tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
+                tmem_wait_ld();
+                if (q < 2) {
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        uint4 hv, lv;
+                        split8(x + 8 * c8, hv, lv);
+                        const uint32_t off = sw128_off(t, cc + 8 * c8, LY::BLK);
+                        st16(sm + LY::DU, off, hv);
+                        st16(sm + LY::DUL, off, lv);
+                    }
+                } else {
+#pragma unroll
+                    for (int j4 = 0; j4 < 32; j4 += 4) {
+                        const int j = cc + j4;
+                        *reinterpret_cast<float4 *>(sm + LY::PL + (j / BV) * RC::OW_SLICE + u_off<BV>(t, j % BV)) =
+                            make_float4(x[j4], x[j4 + 1], x[j4 + 2], x[j4 + 3]);
+                    }
+                }
+            }
+            const int d_row = 32 * q + lane;
+#pragma unroll
+            for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 16) {
+                float xh[16], xl[16];
+                tmem_ld16(taddr(tb, 32 * q, LY::cF + cc), xh);
+                tmem_ld16(taddr(tb, 32 * q, LY::cF + DV + cc), xl);
+                tmem_wait_ld();
 #pragma unroll
                 for (int j4 = 0; j4 < 16; j4 += 4) {
                     const int j = cc + j4;
@@ -770,42 +976,88 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
                 }
             }
         }
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    if (ok && tid == 0) {
-        bulk_s2g(rec + RC::FW, sm + LY::W, RC::FW_SLICE * (DV / BV));
-        bulk_commit();
-        bulk_wait_read_n<1>();  // the O_w store has read K / Q, where -X_u is staged next
-    }
-    ok = mma_done_committed(ok);
-    // -X_u -> the U slot (staged over K and Q in the record's slice layout, one bulk store)
-    if (ok) {
-        uint8_t *stage = sm + LY::KQ;
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        static_assert(RC::FW_SLICE * (DV / BV) <= LY::DU - LY::W, "F_w fits over W and U");
+        if (ok && tid == 0) {
+            bulk_s2g(rec + RC::OW, sm + LY::PL, C * DV * 4);
+            bulk_s2g(rec + RC::FW, sm + LY::W, RC::FW_SLICE * (DV / BV));
+            bulk_commit();
+            // Wk = T diag(beta gamma) K  (M = 64, into the columns just read out)
+            const uint32_t id = idesc_bf16(64, DK, 0, 1);
+            mma_steps<C / 16>(tb + LY::cA, id, make_desc(sb + LY::T1, 16, 1024, 2), dKmn, ok0, omn, false);
+            mma_steps<C / 16>(tb + LY::cA, id, make_desc(sb + LY::T1L, 16, 1024, 2), dKmn, ok0, omn, true);
+        }
+        ok = mma_done(ok);
+        // Wk as a hi / lo pair staged over K / Q (the Wk MMA was their last reader; hi and lo are
+        // adjacent there as WK and WKL in the record), then T itself over the T tiles for X_u
+        static_assert(2 * RC::WK_BLK * (DK / 64) <= LY::KQ_BLK * (DK / 64) && LY::BLK == RC::WK_BLK &&
+                          RC::WKL == RC::WK + RC::WK_BLK * (DK / 64),
+                      "the staged Wk pair has the record's layout");
+        if (ok) {
 #pragma unroll
-        for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
-            float x[32];
-            tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
-            tmem_wait_ld();
-            if (own_t) {
+            for (int cc = hs * (DK / NH); cc < (hs + 1) * (DK / NH); cc += 32) {
+                float x[32];
+                tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
+                tmem_wait_ld();
+                if (own_t) store32_split(sm + LY::KQ, sm + LY::KQ + RC::WK_BLK * (DK / 64), t_row, cc, x, LY::BLK);
+            }
+            store_t_pair(false, tid, NTH);
+        }
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (ok && tid == 0) {
+            bulk_s2g(rec + RC::WK, sm + LY::KQ, 2 * RC::WK_BLK * (DK / 64));
+            bulk_commit();
+            // X_u = T (sum P U)  (M = 64, into the same columns, read out above)
+            const uint64_t dPU = make_desc(sb + LY::DU, LY::BLK, 1024, 2);
+            const uint64_t dPUL = make_desc(sb + LY::DUL, LY::BLK, 1024, 2);
+            const uint64_t dT = make_desc(sb + LY::T1, 16, 1024, 2), dTL = make_desc(sb + LY::T1L, 16, 1024, 2);
+            mma_steps<C / 16>(tb + LY::cA, idV, dT, dPU, ok0, omn, false);
+            mma_steps<C / 16>(tb + LY::cA, idV, dT, dPUL, ok0, omn, true);
+            mma_steps<C / 16>(tb + LY::cA, idV, dTL, dPU, ok0, omn, true);
+        }
+        ok = mma_done(ok);
+        // -X_u -> the U slot, staged over the D U tiles (the X_u MMA was their last reader)
+        static_assert((uint32_t)C * DV * 4 <= 2 * LY::BLK * (DK / 64), "-X_u fits over the D U tiles");
+        if (ok) {
 #pragma unroll
-                for (int j4 = 0; j4 < 32; j4 += 4) {
-                    const int j = cc + j4;
-                    *reinterpret_cast<float4 *>(stage + (j / BV) * RC::U_SLICE + u_off<BV>(t_row, j % BV)) =
-                        make_float4(-x[j4], -x[j4 + 1], -x[j4 + 2], -x[j4 + 3]);
+            for (int cc = hs * (DV / NH); cc < (hs + 1) * (DV / NH); cc += 32) {
+                float x[32];
+                tmem_ld32(taddr(tb, 32 * q, LY::cA + cc), x);
+                tmem_wait_ld();
+                if (own_t) {
+#pragma unroll
+                    for (int j4 = 0; j4 < 32; j4 += 4) {
+                        const int j = cc + j4;
+                        *reinterpret_cast<float4 *>(sm + LY::DU + (j / BV) * RC::U_SLICE + u_off<BV>(t_row, j % BV)) =
+                            make_float4(-x[j4], -x[j4 + 1], -x[j4 + 2], -x[j4 + 3]);
+                    }
                 }
             }
         }
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    if (ok && tid == 0) {
-        bulk_s2g(rec + RC::U, sm + LY::KQ, (uint32_t)(C * DV * 4));
-        bulk_commit();
-        bulk_wait_read();  // the staging buffer is read out before the CTA frees it; the kernel's
-                           // end makes the writes visible to the next launch
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        if (ok && tid == 0) {
+            bulk_s2g(rec + RC::U, sm + LY::DU, (uint32_t)(C * DV * 4));
+            bulk_commit();
+        }
+        // every bulk store has read its staging before the CTA frees the shared memory; the
+        // kernel's end makes the writes visible to the next launch
+        if (tid == 0 || r_issuer) bulk_wait_read();
+        // after a failure, the rank loop's tile loads still in flight land before the CTA exits
+        if (!ok && r_issuer && !stall) {
+            for (int l = w_next > 2 ? w_next - 2 : 0; l < w_next; ++l)
+                mbar_wait(&w_bar[l & 1], (l >> 1) & 1, nullptr, kStallTestPolls);
+            for (int l = u_next > NBU ? u_next - NBU : 0; l < u_next; ++l)
+                mbar_wait(&u_bar[l % NBU], (l / NBU) & 1, nullptr, kStallTestPolls);
+        }
+        w_issued = u_issued = 0;  // (the drain below covers K / Q only)
     }
     // after a failure, let the tile loads still in flight land before the CTA exits
     if (!ok && tid == 0 && !stall) {
