@@ -395,6 +395,10 @@ struct LPrepLayout {
     static constexpr uint32_t AF = MQWL + BLK + (SPLIT ? 2 * BLK : 0);  // fp32 A, solved in place into T
     static constexpr uint32_t P = SPLIT ? MQWL + BLK : AF;
     static constexpr uint32_t MQW = P + BLK;
+    // Mqk (hi, lo) staged for its bulk store: over the T tiles (SPLIT: the rank loop writes the
+    // [P; Mqw] tiles while the solve runs) or over the lo [P; Mqw] tiles
+    static constexpr uint32_t MQK_HI = SPLIT ? T1 : PL;
+    static_assert(T1L == T1 + BLK && MQWL == PL + BLK && BLK == C * 128, "Mqk hi / lo staged adjacent");
     static constexpr uint32_t TMP = AF + C * AS * 4;
     static constexpr uint32_t GATES = TMP + kSolveTmpFloats * 4;   // g, beta, gamma, D
     static constexpr uint32_t BYTES = GATES + 4 * C * 4 + 1024;
@@ -570,16 +574,18 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
 #pragma unroll
         for (int j = 0; j < CW; ++j) gr[j] *= dec[j];
         if (q < 2) vst<CW>(sA + t_g * AS + cg, gr);
-        else store_split_n<CW>(sm + LY::PL, sm + LY::MQWL, t_g, cg, gr);
+        else store_split_n<CW>(sm + LY::MQK_HI, sm + LY::MQK_HI + C * 128, t_g, cg, gr);
     }
     fence_async_smem();
     fence_before_sync();
     __syncthreads();
-    // Mqk hi then lo (the PL and MQWL tiles are adjacent, as in the record), stored by the thread
-    // that later waits for the store before the P / Mqw epilogue writes those tiles
+    // Mqk hi then lo (two adjacent tiles, as in the record), stored by thread 0, which waits for
+    // the store to have read them before those tiles are written again (by the T pair at d = 128,
+    // by the first P / Mqw epilogue at d = 64)
     constexpr int kRankIssuer = LY::SPLIT ? 256 : 0;
-    if (ok && tid == kRankIssuer) {
-        bulk_s2g(rec + RC::MQK, sm + LY::PL, 2 * C * 128);
+    constexpr int kSolveThreads = 256;  // (SPLIT) the solve's warps: 0-7
+    if (ok && tid == 0) {
+        bulk_s2g(rec + RC::MQK, sm + LY::MQK_HI, 2 * C * 128);
         bulk_commit();
     }
     // T pair tiles: T diag(beta gamma) for Wk, then T itself for X_u
@@ -814,7 +820,7 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     } else {
         // ---- d = 128: the solve (warps 0-7) and the rank loop (warps 8-15) at the same time; the
         // rank loop needs none of T (only Wk and X_u do, and they follow the join) ----
-        constexpr int GS = 256, GR = NTH - GS;  // the two groups' threads
+        constexpr int GS = kSolveThreads, RB = 256, GR = NTH - RB;  // the solve's and the rank loop's threads
         const bool r_issuer = tid == kRankIssuer;
         const uint32_t idV = idesc_bf16(64, DV, 0, 1);
         const uint64_t dKmn = make_desc(sb + LY::KQ, LY::KQ_BLK, 1024, 2);
@@ -824,15 +830,17 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
         if (tid < GS) {
             if (ok) {
                 solve_unit_lower<GS>(sA, sA, sTmp, tid, [] { named_sync(3, GS); });
+                if (tid == 0) bulk_wait_read();  // the Mqk staged over the T tiles is read out
+                named_sync(3, GS);
                 store_t_pair(true, tid, GS);  // T diag(beta gamma) for Wk
             }
-        } else {
+        } else if (tid >= RB) {
             // The write terms, one rank at a time, on this group's 8 warps (TMEM lane quarter
             // warp % 4, two column halves).  G_l = [K; Q] W_l^T is issued together with the
             // previous rank's MMAs (W is double-buffered), so each rank waits for one MMA batch.
             constexpr int CWR = C / 2;
-            const int cgr = ((warp - GS / 32) >> 2) * CWR;
-            const int rt = tid - GS;
+            const int cgr = ((warp - RB / 32) >> 2) * CWR;
+            const int rt = tid - RB;
             float decr[CWR];  // the G epilogue factors of this thread's row and columns
             {
                 const float gt = sG[t_g], sc = q < 2 ? sBeta[t_g] : 1.f;
@@ -860,7 +868,6 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
             if (rok && r_issuer) {
                 if (mbar_wait(&w_bar[0], 0, p.status, lim)) issue_g(0);
                 else failed_sh = 1;
-                bulk_wait_read();  // the staged Mqk is read out: the P / Mqw epilogue writes its tiles
             }
             rok = r_done(rok);
             for (int l = 0; l < L && rok; ++l) {
