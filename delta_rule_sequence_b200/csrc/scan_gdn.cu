@@ -401,7 +401,11 @@ struct LPrepLayout {
     static_assert(T1L == T1 + BLK && MQWL == PL + BLK && BLK == C * 128, "Mqk hi / lo staged adjacent");
     static constexpr uint32_t TMP = AF + C * AS * 4;
     static constexpr uint32_t GATES = TMP + kSolveTmpFloats * 4;   // g, beta, gamma, D
-    static constexpr uint32_t BYTES = GATES + 4 * C * 4 + 1024;
+    // (SPLIT) the chunk's decay matrix e^{g_t - g_i} (i <= t, else 0), fp32 [C][AS] (rows padded
+    // like A's, so that a warp reading 32 rows at one column spreads over the banks): every G
+    // epilogue scales by it instead of recomputing its exponentials per thread
+    static constexpr uint32_t DECAY = GATES + 4 * C * 4;
+    static constexpr uint32_t BYTES = DECAY + (SPLIT ? C * AS * 4 : 0) + 1024;
     static_assert(KQ_BLK * (DK / 64) >= (uint32_t)C * DK * 4, "-X_u staging fits over K and Q");
     static_assert(SPLIT || MQW + BLK <= TMP, "the hi P / Mqw rows fit over the solve matrix");
     static_assert(!SPLIT || (MQW + BLK == AF && MQWL + BLK == P && (uint32_t)C * DK * 4 <= 4 * BLK),
@@ -554,15 +558,36 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
     // beta_t e^{g_t - g_i} for i < t on the K rows (lane quarters 0-1: A and P_l), e^{g_t - g_i}
     // for i <= t on the Q rows (quarters 2-3: Mqk and Mqw_l).
     const int t_g = (q & 1) * 32 + lane, cg = hs * CW;
-    float dec[CW];
-    {
-        const float gt = sG[t_g], sc = q < 2 ? sBeta[t_g] : 1.f;
+    float *sE = (float *)(sm + LY::DECAY);
+    // the factors of a G epilogue row t_g, columns c0 .. c0 + N: from the decay matrix (SPLIT) or
+    // computed here
+    auto g_factors = [&](int c0, auto &f) {
+        constexpr int N = sizeof(f) / sizeof(float);
+        const float sc = q < 2 ? sBeta[t_g] : 1.f;
+        if constexpr (LY::SPLIT) {
+            vld<N>(sE + t_g * AS + c0, f);
 #pragma unroll
-        for (int j = 0; j < CW; ++j) {
-            const int i = cg + j;
-            dec[j] = (q < 2 ? i < t_g : i <= t_g) ? sc * __expf(gt - sG[i]) : 0.f;
+            for (int j = 0; j < N; ++j) f[j] = (q < 2 && c0 + j == t_g) ? 0.f : sc * f[j];
+        } else {
+            const float gt = sG[t_g];
+#pragma unroll
+            for (int j = 0; j < N; ++j) {
+                const int i = c0 + j;
+                f[j] = (q < 2 ? i < t_g : i <= t_g) ? sc * __expf(gt - sG[i]) : 0.f;
+            }
+        }
+    };
+    if constexpr (LY::SPLIT) {  // the decay matrix while the MMA runs: 8 exponentials a thread
+        for (int e = tid; e < C * C; e += NTH) {
+            const int t = e / C, i = e % C;
+            sE[t * AS + i] = i <= t ? __expf(sG[t] - sG[i]) : 0.f;
         }
     }
+    float dec[CW];
+    if constexpr (LY::SPLIT) {
+        __syncthreads();  // the decay matrix is complete
+    }
+    g_factors(cg, dec);
     ok = mma_done_committed(ok);
     // the record is written by bulk stores from shared memory that is idle at that point (Mqk over
     // the lo [P; Mqw] tiles, the Wk pair over the D U tiles, O_w over K / Q, F_w over W / U):
@@ -842,14 +867,7 @@ __global__ void __launch_bounds__(kLPrepThreads<DK>, DK == 64 ? 2 : 1) lrank_pre
             const int cgr = ((warp - RB / 32) >> 2) * CWR;
             const int rt = tid - RB;
             float decr[CWR];  // the G epilogue factors of this thread's row and columns
-            {
-                const float gt = sG[t_g], sc = q < 2 ? sBeta[t_g] : 1.f;
-#pragma unroll
-                for (int j = 0; j < CWR; ++j) {
-                    const int i = cgr + j;
-                    decr[j] = (q < 2 ? i < t_g : i <= t_g) ? sc * __expf(gt - sG[i]) : 0.f;
-                }
-            }
+            g_factors(cgr, decr);
             uint32_t rph = mph;  // mma_bar phases this group has waited for
             auto r_done = [&](bool issued) -> bool {  // the issuer commits; the group waits
                 if (r_issuer && issued) mma_commit(&mma_bar);
