@@ -1428,7 +1428,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 const uint32_t bb = sb + (c & 1) * LY::BUF;
                 // S_c written (which also means every epilogue read of this D1 buffer, two chunks
                 // back, is done: the epilogue warps work through the chunks in order)
-                if (!mbar_wait(&bars.s_ready, c & 1, status, lim)) { ok = false; break; }
+                if (!mbar_wait_spin(&bars.s_ready, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 const uint64_t dWQ = make_desc(bb + LY::B_KWQ + C * 128, 16, 1024, 2);
                 mma_steps<DK / 16>(tb + LY::cD1 + (c & 1) * N2, idS, dWQ, dS2, oKWQ, oVT, false);
@@ -1454,7 +1454,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 }
                 mma_commit(&bars.d1_full);
                 // D Y_c written
-                if (!mbar_wait(&bars.y_ready, c & 1, status, lim)) { ok = false; break; }
+                if (!mbar_wait_spin(&bars.y_ready, c & 1, status, lim)) { ok = false; break; }
                 fence_after_sync();
                 const uint64_t dKt = make_desc(bb + LY::B_KWQ, LY::KWQ_BLK, 1024, 2);
                 mma_steps<C / 16>(tb + LY::cD4, id4, dKt, dDY2, oMN, oVT, false);

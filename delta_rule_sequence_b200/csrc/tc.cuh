@@ -290,6 +290,25 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint64_t *bar, uint32_t parity
     return ok;
 }
 
+__device__ __forceinline__ uint32_t mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok;
+}
+// The same wait by non-suspending polls (64 per unit of the limit), for a thread every one of
+// whose waits is on the critical path (a suspended try_wait can wake later than the completion).
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, uint32_t *status, uint32_t limit) {
+    for (uint32_t i = 0; i < 64u * limit; ++i)
+        if (mbar_test_wait(bar, parity)) return true;
+    record_status(status, PRISM_ERR_TIMEOUT);
+    return false;
+}
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
