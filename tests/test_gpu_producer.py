@@ -38,7 +38,10 @@ def _run(p):
 
 
 @pytest.mark.parametrize("d,L,B,H,T", [(64, 3, 1, 2, 200), (128, 2, 2, 1, 130), (64, 1, 1, 1, 64),
-                                       (128, 5, 1, 2, 1), (64, 4, 2, 2, 257), (128, 1, 1, 1, 128)])
+                                       (128, 5, 1, 2, 1), (64, 4, 2, 2, 257), (128, 1, 1, 1, 128),
+                                       # more 128-token tiles than SMs, so a CTA walks several tiles
+                                       # and crosses heads: weights resident (L <= 4) and streamed
+                                       (64, 3, 3, 5, 2000), (64, 6, 2, 3, 4173)])
 def test_producer_matches_oracle(d, L, B, H, T):
     wl = WORKLOADS["recsys"].with_(B=B, H=H, T=T, dk=d, dv=d, L=L)
     p = make_producer_inputs(wl, seed=d + L + T)
@@ -113,13 +116,14 @@ def test_producer_feeds_the_scan(d, L, T):
         assert excess.max() <= 10.0, (name, float(excess.max()))
 
 
-def test_producer_leaves_no_tokens_untouched_and_no_status():
+@pytest.mark.parametrize("d,L", [(128, 2), (64, 5)])
+def test_producer_leaves_no_tokens_untouched_and_no_status(d, L):
     """T not a multiple of the tile: every output element is written (the buffers start as NaN)."""
     from delta_rule_sequence_b200.prism import prism_write_producer
 
-    wl = WORKLOADS["long"].with_(H=3, T=333, L=2)
+    wl = WORKLOADS["long"].with_(H=3, T=333, L=L, dk=d, dv=d)
     p = to_device(make_producer_inputs(wl, seed=9))
-    u = torch.full((1, 333, 3, 2, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    u = torch.full((1, 333, 3, L, d), float("nan"), dtype=torch.bfloat16, device="cuda")
     w = torch.full_like(u, float("nan"))
     prism_write_producer(p["x"], p["v"], p["conv"], p["Wk"], p["Wp"], p["beta"], u=u, w=w)
     torch.cuda.synchronize()
