@@ -12,22 +12,20 @@
 // The anchor depends only on the input window, so every token's chain runs at once; the 2L
 // projections of a token are one GEMM row against the stacked weights [W_k^(l); W_p^(l)].
 //
-// Both kernels work on tiles of 128 tokens of one (batch, head): epilogue warps build the anchor
-// tile (the A operand, as a bf16 hi / lo pair: a single bf16 anchor lets the residual chain
-// amplify its rounding past the bf16 output tolerance by the fourth rank) and hold the residual in
-// registers (one token row a thread); one thread issues, for each l, one M = 128, N = 2d MMA of the
-// anchor against the stacked weights into a TMEM accumulator, so the MMA of rank l + 1 runs while
-// the epilogue of rank l reads k^(l) and p^(l), applies the GELU step and writes u and w.
-//
-// d = 64 (write_producer_ring_kernel): persistent, one CTA per SM walking a contiguous range of
-// tiles (head-major, so a CTA's tiles share their weights).  A load warp brings each tile's x rows
-// (with the 3-token causal halo; rows before the sequence start read as zeros) and v rows by TMA
+// One kernel (write_producer_ring_kernel), persistent: one CTA per SM walks a contiguous range of
+// 128-token tiles of one (batch, head) at a time (head-major order, so a CTA's tiles share their
+// weights).  Its epilogue warps build the anchor tile (the A operand, as a bf16 hi / lo pair: a
+// single bf16 anchor lets the residual chain amplify its rounding past the bf16 output tolerance by
+// the fourth rank) and hold the residual in registers (one token row, 16 columns a thread); one
+// thread issues, for each l, one M = 128, N = 128 MMA pair of the anchor against the stacked
+// weights into one of four TMEM accumulators, so the MMA of rank l + 1 runs while the epilogue of
+// rank l reads k^(l) and p^(l), applies the GELU step and writes u and w.  A load warp brings each
+// tile's x rows (with the 3-token causal halo; rows before the sequence start read as zeros) by TMA
 // into swizzled shared memory while the previous tile is in its epilogue, and keeps the weights of
-// up to four ranks resident (more ranks stream through four slots); four TMEM accumulators form a
-// ring; each epilogue warp stages its 32 x 16 block of u and w in shared memory and writes it with
-// one TMA store a rank, so no thread issues a global store.
-// d = 128 (write_producer_kernel): one CTA per tile, the weights double-buffered per l, u and w
-// written by the epilogue threads.
+// up to NW ranks resident (more ranks stream through NW slots).  Each epilogue warp stages its
+// 32 x 16 blocks of w and u in shared memory and writes each with one TMA store, so no thread
+// issues a global store.  At d = 128 the two CTAs of a pair take one 64-column half of k, p, u, w
+// each (the residual chain is column-wise); both build the whole anchor (the MMA's K).
 // Every wait is a bounded mbarrier poll that records PRISM_ERR_TIMEOUT in the library's producer
 // status word.
 
@@ -45,9 +43,7 @@ namespace {
 
 __device__ uint32_t g_producer_status;
 
-constexpr int PT = 128;                    // tokens per CTA (TMEM lanes, M of the MMA)
-constexpr int P_EPI = 8;                   // epilogue warps
-constexpr int P_THREADS = 32 * (P_EPI + 1);
+constexpr int PT = 128;                    // tokens per tile (TMEM lanes, M of the MMA)
 
 // GELU(z) = z Phi(z) with erf from Abramowitz & Stegun, Handbook of Mathematical Functions,
 // formula 7.1.26 (absolute error at most 1.5e-7 for x >= 0):
@@ -128,19 +124,6 @@ __device__ __forceinline__ void gelu_step(const float *p, float *r, float bl, fl
     }
 }
 
-template <int D>
-struct ProdLayout {
-    static constexpr uint32_t A_BLK = PT * 128;            // 128 token rows x 64 bf16 columns
-    static constexpr uint32_t A = 0;                       // anchor hi tile, K-major SW128
-    static constexpr uint32_t A_LO = A + A_BLK * (D / 64); // anchor lo tile
-    static constexpr uint32_t W_BLK = 2 * D * 128;         // [W_k; W_p] rows of one 64-col block
-    static constexpr uint32_t WBUF = W_BLK * (D / 64);
-    static constexpr uint32_t W = A_LO + A_BLK * (D / 64); // two weight buffers
-    static constexpr uint32_t BYTES = W + 2 * WBUF + 1024;
-    static constexpr uint32_t TCOLS = 4 * D <= 256 ? 256 : 512;   // two [k | p] accumulators
-    static_assert(BYTES <= 227 * 1024, "shared memory budget");
-};
-
 __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
 #pragma unroll
@@ -156,223 +139,90 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
                       pack_bf16(f[6], f[7]));
 }
 
-template <int D>
-__global__ void __launch_bounds__(P_THREADS, D == 64 ? 2 : 1) write_producer_kernel(ProducerArgs p,
-                                                                     const __grid_constant__ CUtensorMap mk,
-                                                                     const __grid_constant__ CUtensorMap mp) {
-    using LY = ProdLayout<D>;
-    constexpr int HALF = D / 2;  // columns of an epilogue thread
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t wbar[2], full[2], tfree[2], a_ready, drain;
-    __shared__ uint32_t tmem_base_sh;
-    __shared__ int failed_sh;
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int t0 = blockIdx.x * PT, h = blockIdx.y, b = blockIdx.z;
-    const int T = p.T, H = p.H, L = p.L;
-    const uint32_t sb = smem_u32(sm);
-    uint32_t *status = &g_producer_status;
-    const uint32_t lim = p.stall ? kStallTestPolls : kWaitPolls;
-
-    if (warp == P_EPI) tmem_alloc(&tmem_base_sh, LY::TCOLS);
-    if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&wbar[i], 1);
-            mbar_init(&full[i], 1);
-            mbar_init(&tfree[i], P_EPI);
-        }
-        mbar_init(&a_ready, P_EPI);
-        mbar_init(&drain, 1);
-        mbar_fence_init();
-        failed_sh = 0;
-    }
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tb = tmem_base_sh;
-
-    if (warp == P_EPI) {
-        // ---------------- weights by TMA, one MMA per rank ----------------
-        if (lane == 0) {
-            auto load_w = [&](int l) {  // [W_k^(l); W_p^(l)] into buffer l % 2
-                const int bi = l & 1;
-                uint8_t *dst = sm + LY::W + bi * LY::WBUF;
-                mbar_expect_tx(&wbar[bi], LY::WBUF);
-                for (int blk = 0; blk < D / 64; ++blk) {
-                    tma_load_4d(dst + blk * LY::W_BLK, &mk, blk * 64, 0, l, h, &wbar[bi]);
-                    tma_load_4d(dst + blk * LY::W_BLK + D * 128, &mp, blk * 64, 0, l, h, &wbar[bi]);
-                }
-            };
-            int issued = 0;
-            if (!p.stall)
-                for (; issued < L && issued < 2; ++issued) load_w(issued);
-            bool ok = mbar_wait(&a_ready, 0, status, lim);
-            const uint32_t id = idesc_bf16(128, 2 * D, 0, 0);
-            auto oa = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::A_BLK); };
-            auto ow = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::W_BLK); };
-            const uint64_t dA = make_desc(sb + LY::A, 16, 1024, 2);
-            const uint64_t dAl = make_desc(sb + LY::A_LO, 16, 1024, 2);
-            for (int l = 0; l < L && ok; ++l) {
-                const int bi = l & 1;
-                if (!mbar_wait(&wbar[bi], (l >> 1) & 1, status, lim)) { ok = false; break; }
-                // the epilogue of rank l - 2 has read this accumulator
-                if (l >= 2 && !mbar_wait(&tfree[bi], ((l - 2) >> 1) & 1, status, lim)) { ok = false; break; }
-                fence_after_sync();
-                const uint64_t dW = make_desc(sb + LY::W + bi * LY::WBUF, 16, 1024, 2);
-                // the anchor as a bf16 hi / lo pair: (a_hi + a_lo) W^T, the weights exact bf16
-                mma_steps<D / 16>(tb + bi * 2 * D, id, dA, dW, oa, ow, false);
-                mma_steps<D / 16>(tb + bi * 2 * D, id, dAl, dW, oa, ow, true);
-                mma_commit(&full[bi]);
-                if (issued < L) {  // W of rank l + 2 into this buffer once the MMA has read it
-                    if (!mbar_wait(&full[bi], (l >> 1) & 1, status, lim)) { ok = false; break; }
-                    load_w(issued++);
-                }
-            }
-            if (!ok) failed_sh = 1;
-            mma_commit(&drain);
-            mbar_wait(&drain, 0, nullptr, lim);
-            // after a failure, weight loads still in flight land before the CTA exits
-            if (!ok)
-                for (int l = issued > 2 ? issued - 2 : 0; l < issued; ++l)
-                    mbar_wait(&wbar[l & 1], (l >> 1) & 1, nullptr, kStallTestPolls);
-        }
-    } else {
-        // ---------------- anchor, then the residual chain, rank by rank ----------------
-        const int q = warp & 3, hs = warp >> 2;  // TMEM lane quarter, column half
-        const int row = 32 * q + lane, t = t0 + row;
-        const bool live = t < T;
-        const int c_base = hs * HALF;
-        const size_t tok = ((size_t)b * T + t) * H + h;
-        const __nv_bfloat16 *x = (const __nv_bfloat16 *)p.x;
-        const __nv_bfloat16 *v = (const __nv_bfloat16 *)p.v;
-        float r[HALF];
-#pragma unroll
-        for (int c8 = 0; c8 < HALF; c8 += 8) {
-            const int col = c_base + c8;
-            float a8[8], xf[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) a8[i] = 0.f;
-            if (live) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (t - j >= 0) {
-                        const uint4 xv = *reinterpret_cast<const uint4 *>(x + (((size_t)b * T + t - j) * H + h) * D + col);
-                        unpack8(xv, xf);
-                        const float *cj = p.conv + ((size_t)h * 4 + j) * D + col;
-                        const float4 c0 = *reinterpret_cast<const float4 *>(cj);
-                        const float4 c1 = *reinterpret_cast<const float4 *>(cj + 4);
-                        const float cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) a8[i] = fmaf(cw[i], xf[i], a8[i]);
-                    }
-                }
-                unpack8(*reinterpret_cast<const uint4 *>(v + tok * D + col), r + c8);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) r[c8 + i] = 0.f;
-            }
-            uint4 hi, lo;
-            split8(a8, hi, lo);
-            const uint32_t off = sw128_off(row, col, LY::A_BLK);
-            st16(sm + LY::A, off, hi);
-            st16(sm + LY::A_LO, off, lo);
-        }
-        fence_async_smem();
-        fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_ready);
-
-        __nv_bfloat16 *uo = (__nv_bfloat16 *)p.u, *wo = (__nv_bfloat16 *)p.w;
-        bool ok = true;
-        for (int l = 0; l < L && ok; ++l) {
-            const int bi = l & 1;
-            if (!mbar_wait(&full[bi], (l >> 1) & 1, status, lim)) { ok = false; break; }
-            fence_after_sync();
-            const float bl = live ? p.beta[tok * L + l] : 0.f;
-            const size_t orow = (tok * L + l) * D;
-            // 16 columns at a time (directions, then gains), few registers beyond the residual
-#pragma unroll
-            for (int ci = 0; ci < HALF / 16; ++ci) {
-                const int col = c_base + 16 * ci;
-                float kk[16];
-                tmem_ld16(taddr(tb, 32 * q, bi * 2 * D + col), kk);
-                tmem_wait_ld();
-                if (live) {
-                    *reinterpret_cast<uint4 *>(wo + orow + col) = pack8(kk);
-                    *reinterpret_cast<uint4 *>(wo + orow + col + 8) = pack8(kk + 8);
-                }
-                float pp[16];
-                tmem_ld16(taddr(tb, 32 * q, bi * 2 * D + D + col), pp);
-                tmem_wait_ld();
-                gelu_step<16>(pp, r + 16 * ci, bl, pp);
-                if (live) {
-                    *reinterpret_cast<uint4 *>(uo + orow + col) = pack8(pp);
-                    *reinterpret_cast<uint4 *>(uo + orow + col + 8) = pack8(pp + 8);
-                }
-            }
-            fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tfree[bi]);
-        }
-        if (!ok) failed_sh = 1;
-    }
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    if (warp == P_EPI) tmem_dealloc(tb, LY::TCOLS);
-}
-
 // ------------------------------------------------------------------------------------------------
-// d = 64: the persistent producer
+// The persistent producer.  Each CTA writes 64 output columns of every token of its tiles: all of
+// them at d = 64; at d = 128 the two CTAs of a pair split the columns (the residual chain is
+// column-wise, so the halves are independent; both build the whole anchor, which is the MMA's K).
 
-constexpr int RCW = 16;    // columns of one epilogue thread
-constexpr int RNW = 4;     // weight slots, one rank's [W_k; W_p] each
-constexpr int RNACC = 4;   // TMEM accumulators, one rank's [k | p] each
+constexpr int RCW = 16;    // output columns of one epilogue thread
+constexpr int RNACC = 4;   // TMEM accumulators, one rank's [k | p] (128 columns) each
 
 template <int D>
 struct RingLayout {
-    static constexpr int NCS = D / RCW;                     // column slices
-    static constexpr int EPI = 4 * NCS;                     // epilogue warps (TMEM lane quarter x slice)
+    static constexpr int HALVES = D / 64;                   // CTAs per tile
+    static constexpr int NH = 64;                           // output columns of a CTA
+    static constexpr int EPI = 4 * (NH / RCW);              // epilogue warps (TMEM lane quarter x slice)
+    static constexpr int ACW = D / 4;                       // anchor columns of an epilogue thread
     static constexpr int LOADW = EPI, MMAW = EPI + 1;       // the load warp, the MMA warp
     static constexpr int THREADS = 32 * (EPI + 2);
-    static constexpr uint32_t A_BLK = PT * 128;
-    static constexpr uint32_t A = 0, A_LO = A_BLK;          // anchor hi / lo, K-major SW128
+    static constexpr int NW = D == 64 ? 4 : 2;              // weight slots (one rank's half of [W_k; W_p])
+    static constexpr int NBOX = D == 64 ? 4 : 3;            // output staging boxes of a warp (a ring)
+    static constexpr uint32_t A_BLK = PT * 128;             // 128 rows x 64 bf16 columns
+    static constexpr uint32_t A = 0, A_LO = A_BLK * HALVES; // anchor hi / lo, K-major SW128
     static constexpr int XROWS = PT + 3;                    // x rows t0 - 3 .. t0 + PT - 1
-    static constexpr uint32_t X = 2 * A_BLK;                // SW128 rows of 128 bytes
-    static constexpr uint32_t X_BYTES = XROWS * 128;
-    static constexpr uint32_t V = (X + X_BYTES + 1023) / 1024 * 1024;
-    static constexpr uint32_t V_BYTES = PT * 128;
-    static constexpr uint32_t WSLOT = 2 * D * 128;          // [W_k; W_p] of one rank, K-major SW128
+    static constexpr uint32_t XBOX_TX = XROWS * 128;        // one 64-column box of x rows (SW128)
+    static constexpr uint32_t XBOX = (XBOX_TX + 1023) / 1024 * 1024;
+    static constexpr uint32_t X = 2 * A_BLK * HALVES;
+    static constexpr uint32_t V = X + HALVES * XBOX;        // v rows (d = 64 only; SW128)
+    static constexpr uint32_t V_BYTES = D == 64 ? PT * 128 : 0;
+    static constexpr uint32_t WBLK = 2 * NH * 128;          // [W_k; W_p] rows of one 64-column K block
+    static constexpr uint32_t WSLOT = WBLK * HALVES;
     static constexpr uint32_t W = V + V_BYTES;
     static constexpr uint32_t BOX = 32 * RCW * 2;           // one warp's 32 rows x 16 columns (SW32)
-    static constexpr uint32_t OUT = W + RNW * WSLOT;        // [warp][buffer][w, u]
-    static constexpr uint32_t BYTES = OUT + EPI * 4 * BOX + 1024;
-    static_assert(D == 64, "one 64-column block per row");
+    static constexpr uint32_t OUT = W + NW * WSLOT;         // [warp][box]
+    static constexpr uint32_t BYTES = OUT + EPI * NBOX * BOX + 1024;
+    static constexpr uint32_t XV_TX = HALVES * XBOX_TX + V_BYTES;
+    static_assert(D == 64 || D == 128, "widths");
     static_assert(BYTES <= 227 * 1024, "shared memory budget");
-    static_assert(RNACC * 2 * D <= 512, "TMEM columns");
+    static_assert(RNACC * 2 * NH <= 512, "TMEM columns");
 };
 
 struct RingMaps {
     CUtensorMap x, v, wk, wp, u, w;
 };
 
+// Walks tiles n0, n0 + 1, ... of the head-major order n = (h B + b) nt + j with 32-bit steps.
+struct TileWalk {
+    int j, bh, left;  // tile within its sequence, sequence index h B + b, tiles still to visit
+    int nt, B;
+    __device__ TileWalk(long long n0, long long n1, int nt_, int B_) : nt(nt_), B(B_) {
+        j = (int)(n0 % nt_);
+        bh = (int)(n0 / nt_);
+        left = (int)(n1 - n0);
+    }
+    __device__ bool more() const { return left > 0; }
+    __device__ void next() {
+        --left;
+        if (++j == nt) {
+            j = 0;
+            ++bh;
+        }
+    }
+    __device__ int b() const { return bh % B; }
+    __device__ int h() const { return bh / B; }
+    // the next tile (if any) belongs to another head
+    __device__ bool last_of_head() const { return left == 1 || (j + 1 == nt && (bh + 1) / B != bh / B); }
+};
+
 template <int D>
 __global__ void __launch_bounds__(RingLayout<D>::THREADS, 1)
     write_producer_ring_kernel(ProducerArgs p, const __grid_constant__ RingMaps maps, long long ntiles) {
     using LY = RingLayout<D>;
+    constexpr int NW = LY::NW, NH = LY::NH;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     __shared__ uint64_t xv_full, xv_free, a_ready, drain;
-    __shared__ uint64_t w_full[RNW], w_free[RNW], acc_full[RNACC], acc_free[RNACC];
+    __shared__ uint64_t w_full[NW], w_free[NW], acc_full[RNACC], acc_free[RNACC];
     __shared__ uint32_t tmem_base_sh;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = p.T, H = p.H, B = p.B, L = p.L;
-    const long long nt = (T + PT - 1) / PT;  // tiles per sequence
+    const int half = blockIdx.x % LY::HALVES;  // which 64 output columns
+    const long long G = gridDim.x / LY::HALVES, pid = blockIdx.x / LY::HALVES;
+    const int nt = (T + PT - 1) / PT;  // tiles per sequence
     // this CTA's contiguous range of tiles; tile n = (h * B + b) * nt + j
-    const long long n0 = ntiles * blockIdx.x / gridDim.x, n1 = ntiles * (blockIdx.x + 1) / gridDim.x;
-    const bool resident = L <= RNW;  // the weights of all ranks stay in their slots per head
+    const long long n0 = ntiles * pid / G, n1 = ntiles * (pid + 1) / G;
+    const bool resident = L <= NW;  // the weights of all ranks stay in their slots per head
     const uint32_t sb = smem_u32(sm);
     uint32_t *status = &g_producer_status;
     const uint32_t lim = p.stall ? kStallTestPolls : kWaitPolls;
@@ -383,7 +233,7 @@ __global__ void __launch_bounds__(RingLayout<D>::THREADS, 1)
         mbar_init(&xv_free, LY::EPI);
         mbar_init(&a_ready, LY::EPI);
         mbar_init(&drain, 1);
-        for (int i = 0; i < RNW; ++i) {
+        for (int i = 0; i < NW; ++i) {
             mbar_init(&w_full[i], 1);
             mbar_init(&w_free[i], 1);
         }
@@ -399,25 +249,30 @@ __global__ void __launch_bounds__(RingLayout<D>::THREADS, 1)
     const uint32_t tb = tmem_base_sh;
 
     if (warp == LY::LOADW) {
-        // ---------------- x and v rows of each tile; the weights ----------------
+        // ---------------- x (and v) rows of each tile; the weights ----------------
         if (lane == 0 && !p.stall) {
-            int epoch = -1, prev_h = -1;
-            long long k = 0;
-            uint32_t wfills[RNW] = {0, 0, 0, 0};  // loads issued into each weight slot
+            int epoch = -1, prev_h = -1, k = 0;
+            uint32_t wfills[NW] = {};  // loads issued into each weight slot
             bool ok = true;
             auto load_w = [&](int slot, int h, int l) {
                 uint8_t *dst = sm + LY::W + slot * LY::WSLOT;
                 mbar_expect_tx(&w_full[slot], LY::WSLOT);
-                tma_load_4d(dst, &maps.wk, 0, 0, l, h, &w_full[slot]);
-                tma_load_4d(dst + D * 128, &maps.wp, 0, 0, l, h, &w_full[slot]);
-                ++wfills[slot];
+#pragma unroll
+                for (int kb = 0; kb < LY::HALVES; ++kb) {
+                    tma_load_4d(dst + kb * LY::WBLK, &maps.wk, kb * 64, half * NH, l, h, &w_full[slot]);
+                    tma_load_4d(dst + kb * LY::WBLK + NH * 128, &maps.wp, kb * 64, half * NH, l, h, &w_full[slot]);
+                }
+#pragma unroll
+                for (int i = 0; i < NW; ++i) wfills[i] += i == slot;
             };
-            for (long long n = n0; n < n1 && ok; ++n, ++k) {
-                const int j = (int)(n % nt), bh = (int)(n / nt), b = bh % B, h = bh / B;
+            for (TileWalk tw(n0, n1, nt, B); tw.more() && ok; tw.next(), ++k) {
+                const int j = tw.j, b = tw.b(), h = tw.h();
                 if (k >= 1 && !mbar_wait(&xv_free, (uint32_t)((k - 1) & 1), status, lim)) { ok = false; break; }
-                mbar_expect_tx(&xv_full, LY::X_BYTES + LY::V_BYTES);
-                tma_load_4d(sm + LY::X, &maps.x, 0, h, j * PT - 3, b, &xv_full);
-                tma_load_4d(sm + LY::V, &maps.v, 0, h, j * PT, b, &xv_full);
+                mbar_expect_tx(&xv_full, LY::XV_TX);
+#pragma unroll
+                for (int xb = 0; xb < LY::HALVES; ++xb)
+                    tma_load_4d(sm + LY::X + xb * LY::XBOX, &maps.x, xb * 64, h, j * PT - 3, b, &xv_full);
+                if constexpr (D == 64) tma_load_4d(sm + LY::V, &maps.v, 0, h, j * PT, b, &xv_full);
                 if (resident) {
                     if (h == prev_h) continue;
                     prev_h = h;
@@ -428,9 +283,9 @@ __global__ void __launch_bounds__(RingLayout<D>::THREADS, 1)
                     }
                 } else {
                     for (int l = 0; l < L && ok; ++l) {
-                        const long long use = k * L + l;
-                        const int slot = (int)(use % RNW);
-                        const long long f = use / RNW;
+                        const uint32_t use = (uint32_t)k * L + l;
+                        const int slot = (int)(use % NW);
+                        const uint32_t f = use / NW;
                         if (f >= 1 && !mbar_wait(&w_free[slot], (uint32_t)((f - 1) & 1), status, lim)) ok = false;
                         else load_w(slot, h, l);
                     }
@@ -439,33 +294,34 @@ __global__ void __launch_bounds__(RingLayout<D>::THREADS, 1)
             // loads still in flight land before the CTA exits (in a normal run every one has
             // been waited for by its consumer already)
             if (k > 0) mbar_wait(&xv_full, (uint32_t)((k - 1) & 1), nullptr, lim);
-            for (int i = 0; i < RNW; ++i)
+#pragma unroll
+            for (int i = 0; i < NW; ++i)
                 if (wfills[i]) mbar_wait(&w_full[i], (wfills[i] - 1) & 1, nullptr, lim);
         }
     } else if (warp == LY::MMAW) {
-        // ---------------- one M = 128, N = 2d MMA pair (anchor hi, lo) per rank ----------------
+        // ---------------- one M = 128, N = 128 MMA pair (anchor hi, lo) per rank ----------------
         if (lane == 0) {
-            const uint32_t id = idesc_bf16(128, 2 * D, 0, 0);
+            const uint32_t id = idesc_bf16(128, 2 * NH, 0, 0);
             auto oa = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::A_BLK); };
-            auto ow = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::WSLOT); };
+            auto ow = [](int ks) { return (uint64_t)koff_k_sw128(ks, LY::WBLK); };
             const uint64_t dA = make_desc(sb + LY::A, 16, 1024, 2);
             const uint64_t dAl = make_desc(sb + LY::A_LO, 16, 1024, 2);
             int epoch = -1, prev_h = -1;
-            long long k = 0, g = 0;
+            uint32_t k = 0, g = 0;
             bool ok = true;
-            for (long long n = n0; n < n1 && ok; ++n, ++k) {
-                const int h = (int)(n / nt) / B;
+            for (TileWalk tw(n0, n1, nt, B); tw.more() && ok; tw.next(), ++k) {
+                const int h = tw.h();
                 if (h != prev_h) {
                     prev_h = h;
                     ++epoch;
                 }
                 // the last of this CTA's tiles on this head releases the resident weights
-                const bool last_of_head = n + 1 == n1 || (int)((n + 1) / nt) / B != h;
+                const bool last_of_head = tw.last_of_head();
                 if (!mbar_wait(&a_ready, (uint32_t)(k & 1), status, lim)) { ok = false; break; }
                 for (int l = 0; l < L; ++l, ++g) {
-                    const long long use = k * L + l;
-                    const int ws = resident ? l : (int)(use % RNW);
-                    const uint32_t wpar = resident ? (uint32_t)(epoch & 1) : (uint32_t)((use / RNW) & 1);
+                    const uint32_t use = k * L + l;
+                    const int ws = resident ? l : (int)(use % NW);
+                    const uint32_t wpar = resident ? (uint32_t)(epoch & 1) : (uint32_t)((use / NW) & 1);
                     const int slot = (int)(g % RNACC);
                     if (!mbar_wait(&w_full[ws], wpar, status, lim) ||
                         (g >= RNACC && !mbar_wait(&acc_free[slot], (uint32_t)((g / RNACC - 1) & 1), status, lim))) {
@@ -474,7 +330,7 @@ __global__ void __launch_bounds__(RingLayout<D>::THREADS, 1)
                     }
                     fence_after_sync();
                     const uint64_t dW = make_desc(sb + LY::W + ws * LY::WSLOT, 16, 1024, 2);
-                    const uint32_t acc = tb + slot * 2 * D;
+                    const uint32_t acc = tb + slot * 2 * NH;
                     mma_steps<D / 16>(acc, id, dA, dW, oa, ow, false);
                     mma_steps<D / 16>(acc, id, dAl, dW, oa, ow, true);
                     mma_commit(&acc_full[slot]);
@@ -487,45 +343,95 @@ __global__ void __launch_bounds__(RingLayout<D>::THREADS, 1)
     } else {
         // ---------------- anchor, residual chain, staged TMA stores ----------------
         const int q = warp & 3, cs = warp >> 2;  // TMEM lane quarter, column slice
-        const int row = 32 * q + lane, col0 = cs * RCW;
-        uint8_t *ob = sm + LY::OUT + warp * 4 * LY::BOX;  // [buffer][w, u]
-        long long k = 0, g = 0;
+        const int row = 32 * q + lane, col0 = cs * RCW, ocol = half * NH + col0;
+        uint8_t *ob = sm + LY::OUT + warp * LY::NBOX * LY::BOX;
+        const __nv_bfloat16 *vg = (const __nv_bfloat16 *)p.v;
+        const int sw = (lane >> 2) & 1;  // SW32 staging: the 16-byte chunk index XOR row bit 2
+        uint4 vnext[2] = {};             // d = 128: the next tile's v columns, loaded a rank ahead
+        auto load_v = [&](int j, int b, int h) {
+            const int t = j * PT + row;
+            if (t < T) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(vg + (((size_t)b * T + t) * H + h) * D + ocol);
+                vnext[0] = src[0];
+                vnext[1] = src[1];
+            } else {
+                vnext[0] = vnext[1] = make_uint4(0, 0, 0, 0);
+            }
+        };
+        if constexpr (D != 64)
+            if (n0 < n1) {
+                const TileWalk tw(n0, n1, nt, B);
+                load_v(tw.j, tw.b(), tw.h());
+            }
+        uint32_t k = 0, g = 0, m = 0;  // tiles, ranks, staging boxes of this thread so far
         bool ok = true;
-        for (long long n = n0; n < n1 && ok; ++n, ++k) {
-            const int j = (int)(n % nt), bh = (int)(n / nt), b = bh % B, h = bh / B;
+        auto box = [&]() {  // the next staging box, once its previous store has read it
+            if (lane == 0 && m >= LY::NBOX) bulk_wait_read_n<LY::NBOX - 1>();
+            __syncwarp();
+            return ob + (uint32_t)(m % LY::NBOX) * LY::BOX;
+        };
+        auto put = [&](uint8_t *bx, const float *v16, const CUtensorMap *map, int l, int h, int t0, int b) {
+            st16(bx, lane * 32 + ((0 ^ sw) << 4), pack8(v16));
+            st16(bx, lane * 32 + ((1 ^ sw) << 4), pack8(v16 + 8));
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_5d(map, bx, ocol, l, h, t0 + 32 * q, b);
+                bulk_commit();
+            }
+            ++m;
+        };
+        for (TileWalk tw(n0, n1, nt, B); tw.more() && ok; tw.next(), ++k) {
+            const int j = tw.j, b = tw.b(), h = tw.h();
             const int t0 = j * PT, t = t0 + row;
             const bool live = t < T;
             const size_t tok = ((size_t)b * T + t) * H + h;
-            // ShortConv taps of this head (broadcast loads, L1 hits after the first tile)
-            float a[RCW], r[RCW];
-#pragma unroll
-            for (int i = 0; i < RCW; ++i) a[i] = 0.f;
+            float r[RCW];
             if (!mbar_wait(&xv_full, (uint32_t)(k & 1), status, lim)) { ok = false; break; }
+            // the anchor's columns [cs ACW, (cs + 1) ACW) of this token row, 16 at a time
 #pragma unroll
-            for (int tap = 0; tap < 4; ++tap) {
-                const float *cj = p.conv + ((size_t)h * 4 + tap) * D + col0;
-                const int xr = row + 3 - tap;  // x stage row of token t - tap
+            for (int a16 = 0; a16 < LY::ACW / 16; ++a16) {
+                const int acol = cs * LY::ACW + 16 * a16, xb = acol >> 6;
+                float a[16];
 #pragma unroll
-                for (int c8 = 0; c8 < RCW / 8; ++c8) {
-                    const int chunk = (col0 >> 3) + c8;
-                    float xf[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(sm + LY::X + xr * 128 + ((chunk ^ (xr & 7)) << 4)), xf);
-                    const float4 c0 = *reinterpret_cast<const float4 *>(cj + 8 * c8);
-                    const float4 c1 = *reinterpret_cast<const float4 *>(cj + 8 * c8 + 4);
-                    const float cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                for (int i = 0; i < 16; ++i) a[i] = 0.f;
+#pragma unroll 1  // (unrolled, the taps' loads are all hoisted and spill)
+                for (int tap = 0; tap < 4; ++tap) {
+                    // ShortConv taps of this head (broadcast loads, L1 hits after the first tile)
+                    const float *cj = p.conv + ((size_t)h * 4 + tap) * D + acol;
+                    const int xr = row + 3 - tap;  // x stage row of token t - tap
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) a[8 * c8 + i] = fmaf(cw[i], xf[i], a[8 * c8 + i]);
+                    for (int c8 = 0; c8 < 2; ++c8) {
+                        const int chunk = ((acol & 63) >> 3) + c8;
+                        float xf[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(sm + LY::X + xb * LY::XBOX + xr * 128 +
+                                                                 ((chunk ^ (xr & 7)) << 4)), xf);
+                        const float4 c0 = *reinterpret_cast<const float4 *>(cj + 8 * c8);
+                        const float4 c1 = *reinterpret_cast<const float4 *>(cj + 8 * c8 + 4);
+                        const float cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) a[8 * c8 + i] = fmaf(cw[i], xf[i], a[8 * c8 + i]);
+                    }
+                }
+#pragma unroll
+                for (int c8 = 0; c8 < 2; ++c8) {
+                    uint4 hi, lo;
+                    split8(a + 8 * c8, hi, lo);
+                    const uint32_t off = sw128_off(row, acol + 8 * c8, LY::A_BLK);
+                    st16(sm + LY::A, off, hi);
+                    st16(sm + LY::A_LO, off, lo);
                 }
             }
+            if constexpr (D == 64) {
 #pragma unroll
-            for (int c8 = 0; c8 < RCW / 8; ++c8) {
-                const int chunk = (col0 >> 3) + c8;
-                unpack8(*reinterpret_cast<const uint4 *>(sm + LY::V + row * 128 + ((chunk ^ (row & 7)) << 4)), r + 8 * c8);
-                uint4 hi, lo;
-                split8(a + 8 * c8, hi, lo);
-                const uint32_t off = sw128_off(row, col0 + 8 * c8, LY::A_BLK);
-                st16(sm + LY::A, off, hi);
-                st16(sm + LY::A_LO, off, lo);
+                for (int c8 = 0; c8 < 2; ++c8) {
+                    const int chunk = (col0 >> 3) + c8;
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + LY::V + row * 128 + ((chunk ^ (row & 7)) << 4)),
+                            r + 8 * c8);
+                }
+            } else {
+                unpack8(vnext[0], r);
+                unpack8(vnext[1], r + 8);
             }
             fence_async_smem();
             fence_before_sync();
@@ -540,32 +446,24 @@ __global__ void __launch_bounds__(RingLayout<D>::THREADS, 1)
                 if (!mbar_wait(&acc_full[slot], (uint32_t)((g / RNACC) & 1), status, lim)) { ok = false; break; }
                 fence_after_sync();
                 float kk[RCW], pp[RCW];
-                tmem_ld16(taddr(tb, 32 * q, slot * 2 * D + col0), kk);
-                tmem_ld16(taddr(tb, 32 * q, slot * 2 * D + D + col0), pp);
+                tmem_ld16(taddr(tb, 32 * q, slot * 2 * NH + col0), kk);
+                tmem_ld16(taddr(tb, 32 * q, slot * 2 * NH + NH + col0), pp);
                 tmem_wait_ld();
                 fence_before_sync();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&acc_free[slot]);
-                    if (g >= 2) bulk_wait_read_n<1>();  // the stores of rank g - 2 have read this buffer
-                }
+                if (lane == 0) mbar_arrive(&acc_free[slot]);
+                // global loads after the arrive (an arrive waits for this thread's loads in flight)
                 const float bcur = bl;
                 if (l + 1 < L && live) bl = p.beta[tok * L + l + 1];
-                __syncwarp();
-                uint8_t *bw = ob + (uint32_t)(g & 1) * 2 * LY::BOX, *bu = bw + LY::BOX;
-                const int sw = (lane >> 2) & 1;  // SW32: the 16-byte chunk index XOR row bit 2
-                st16(bw, lane * 32 + ((0 ^ sw) << 4), pack8(kk));
-                st16(bw, lane * 32 + ((1 ^ sw) << 4), pack8(kk + 8));
+                if constexpr (D != 64)
+                    if (l + 1 == L && tw.left > 1) {
+                        TileWalk nx = tw;
+                        nx.next();
+                        load_v(nx.j, nx.b(), nx.h());
+                    }
+                put(box(), kk, &maps.w, l, h, t0, b);
                 gelu_step<RCW>(pp, r, bcur, pp);
-                st16(bu, lane * 32 + ((0 ^ sw) << 4), pack8(pp));
-                st16(bu, lane * 32 + ((1 ^ sw) << 4), pack8(pp + 8));
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_5d(&maps.w, bw, col0, l, h, t0 + 32 * q, b);
-                    tma_store_5d(&maps.u, bu, col0, l, h, t0 + 32 * q, b);
-                    bulk_commit();
-                }
+                put(box(), pp, &maps.u, l, h, t0, b);
             }
         }
         if (lane == 0) bulk_wait_all();
@@ -592,12 +490,12 @@ PFN_cuTensorMapEncodeTiled_v12000 map_encoder() {
 
 // 4-D map over bf16 weights [H, L, d, d] (row = output index): dims {d_in, d_out, L, H}, box
 // {64, d, 1, 1} (one 64-column block of one (h, l) matrix).
-bool weight_map(CUtensorMap *m, const void *base, int H, int L, int d) {
+bool weight_map(CUtensorMap *m, const void *base, int H, int L, int d, int rows) {
     auto enc = map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)H};
     const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)d * d * 2, (cuuint64_t)L * d * d * 2};
-    const cuuint32_t box[4] = {64, (cuuint32_t)d, 1, 1};
+    const cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -640,36 +538,21 @@ int device_sms() {
     return n;
 }
 
+template <int D>
 cudaError_t launch_producer_ring(const ProducerArgs &a, cudaStream_t s) {
-    constexpr int D = 64;
     using LY = RingLayout<D>;
     RingMaps maps;
     if (!act_map(&maps.x, a.x, a.B, a.T, a.H, D, LY::XROWS) || !act_map(&maps.v, a.v, a.B, a.T, a.H, D, PT) ||
-        !weight_map(&maps.wk, a.Wk, a.H, a.L, D) || !weight_map(&maps.wp, a.Wp, a.H, a.L, D) ||
+        !weight_map(&maps.wk, a.Wk, a.H, a.L, D, LY::NH) || !weight_map(&maps.wp, a.Wp, a.H, a.L, D, LY::NH) ||
         !out_map(&maps.u, a.u, a.B, a.T, a.H, a.L, D) || !out_map(&maps.w, a.w, a.B, a.T, a.H, a.L, D))
         return cudaErrorInvalidValue;
     auto kern = write_producer_ring_kernel<D>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
     if (err != cudaSuccess) return err;
     const long long ntiles = (long long)a.H * a.B * ((a.T + PT - 1) / PT);
-    const int grid = (int)std::min<long long>(ntiles, device_sms());
+    const int pairs = (int)std::min<long long>(ntiles, std::max(1, device_sms() / LY::HALVES));
     launch_probe_mark(s);
-    kern<<<grid, LY::THREADS, LY::BYTES, s>>>(a, maps, ntiles);
-    return cudaGetLastError();
-}
-
-template <int D>
-cudaError_t launch_producer_t(const ProducerArgs &a, cudaStream_t s) {
-    CUtensorMap mk, mp;
-    if (!weight_map(&mk, a.Wk, a.H, a.L, D) || !weight_map(&mp, a.Wp, a.H, a.L, D))
-        return cudaErrorInvalidValue;
-    using LY = ProdLayout<D>;
-    auto kern = write_producer_kernel<D>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
-    if (err != cudaSuccess) return err;
-    dim3 grid((a.T + PT - 1) / PT, a.H, a.B);
-    launch_probe_mark(s);
-    kern<<<grid, P_THREADS, LY::BYTES, s>>>(a, mk, mp);
+    kern<<<pairs * LY::HALVES, LY::THREADS, LY::BYTES, s>>>(a, maps, ntiles);
     return cudaGetLastError();
 }
 
@@ -677,7 +560,7 @@ cudaError_t launch_producer_t(const ProducerArgs &a, cudaStream_t s) {
 
 cudaError_t launch_write_producer(const ProducerArgs &a, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
-    return a.d == 128 ? launch_producer_t<128>(a, s) : launch_producer_ring(a, s);
+    return a.d == 128 ? launch_producer_ring<128>(a, s) : launch_producer_ring<64>(a, s);
 }
 
 // Read and clear the producer's status word (PRISM_OK or PRISM_ERR_TIMEOUT).
