@@ -88,6 +88,16 @@ __device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigne
     return d;
 }
 
+// 5-D tiled TMA store of one box from shared memory (rows outside the tensor are not written),
+// in this thread's current bulk group.
+__device__ __forceinline__ void tma_store_5d(const void *tmap, const void *src, int x, int y, int z, int w,
+                                             int v) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4, %5}], [%6];"
+        ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(v), "r"(smem_u32(src))
+        : "memory");
+}
+
 // One residual step on N columns (N even): z = p r, delta = GELU(z), r -= delta, u = bl delta
 // (u may alias p).
 template <int N>

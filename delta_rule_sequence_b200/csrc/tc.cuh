@@ -116,16 +116,6 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int x, 
         : "memory");
 }
 
-// 5-D tiled TMA store of one box from shared memory (rows outside the tensor are not written),
-// in this thread's current bulk group.
-__device__ __forceinline__ void tma_store_5d(const void *tmap, const void *src, int x, int y, int z, int w,
-                                             int v) {
-    asm volatile(
-        "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4, %5}], [%6];"
-        ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(v), "r"(smem_u32(src))
-        : "memory");
-}
-
 // Prefetch of one 4-D tiled box into L2 (no shared memory, no completion signal).
 __device__ __forceinline__ void tma_prefetch_4d(const void *tmap, int x, int y, int z, int w) {
     asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];"
