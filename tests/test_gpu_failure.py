@@ -81,10 +81,11 @@ def test_scan_kernels_give_up_and_report_a_timeout(name, flags):
     check_scan_full(make_inputs(wl, seed=4), wl.chunk, wl.io)
 
 
-def test_producer_gives_up_and_reports_a_timeout():
+@pytest.mark.parametrize("d", [64, 128])
+def test_producer_gives_up_and_reports_a_timeout(d):
     from delta_rule_sequence_b200 import prism
 
-    wl = WORKLOADS["recsys"].with_(B=1, H=2, T=200, L=3)
+    wl = WORKLOADS["recsys"].with_(B=1, H=2, T=200, L=3, dk=d, dv=d)
     p = to_device(make_producer_inputs(wl, seed=5))
     call = lambda: prism.prism_write_producer(p["x"], p["v"], p["conv"], p["Wk"], p["Wp"], p["beta"])
     _with_flags(STALL_PRODUCER, call)
