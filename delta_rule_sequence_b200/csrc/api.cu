@@ -380,7 +380,7 @@ prism_status prism_write_producer(const prism_shape *shape, const void *x, const
     if (s.io != PRISM_BF16 && s.io != PRISM_F32) return PRISM_ERR_INVALID_ARG;
     if (s.io != PRISM_BF16 || s.dk != s.dv || (s.dk != 64 && s.dk != 128) || s.L > 64)
         return PRISM_ERR_UNSUPPORTED;
-    if (s.B > 65535 || s.H > 65535) return PRISM_ERR_UNSUPPORTED;
+    if (s.B > 65535 || s.H > 65535 || (long long)s.B * s.H > 0x7fffffffLL) return PRISM_ERR_UNSUPPORTED;
     if ((long long)s.B * s.H * s.T == 0) return PRISM_OK;
     for (const void *ptr : {x, v, (const void *)conv, Wk, Wp, (const void *)u, (const void *)w})
         if (!ptr || !aligned16(ptr)) return PRISM_ERR_INVALID_ARG;
