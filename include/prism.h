@@ -223,9 +223,11 @@ prism_status prism_scan_fwd_noalloc(const prism_shape *shape, const void *q, con
  *   Wk, Wp   [H,L,d,d]   bf16          beta  [B,T,H,L] fp32 (4-byte aligned)
  *   u, w     [B,T,H,L,d] bf16 outputs  (must not overlap each other or any input)
  * Uses shape->B, H, T, dk, dv, L, io; requires io == PRISM_BF16 and dk == dv in {64, 128}
- * (PRISM_ERR_UNSUPPORTED otherwise), 1 <= L <= 64, B <= 65535, H <= 65535 and B * H < 2^31.  The two projections run on the tensor cores
- * from the anchor as a bf16 hi / lo pair with fp32 accumulation; the residual chain and GELU in
- * fp32; u, w are rounded to bf16 (nearest even).  A bounded wait that gives up records PRISM_ERR_TIMEOUT in the library's
+ * (PRISM_ERR_UNSUPPORTED otherwise), 1 <= L <= 64, B <= 65535, H <= 65535 and B * H < 2^31.
+ * The two projections run on the tensor cores from the anchor as a bf16 hi / lo pair with fp32
+ * accumulation; the residual chain and GELU in fp32, GELU's erf by Abramowitz & Stegun, Handbook
+ * of Mathematical Functions, 7.1.26 (absolute error at most 1.5e-7); u, w are rounded to bf16
+ * (nearest even).  A bounded wait that gives up records PRISM_ERR_TIMEOUT in the library's
  * producer status word (prism_query_device_status).
  */
 prism_status prism_write_producer(const prism_shape *shape, const void *x, const void *v,
