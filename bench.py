@@ -69,7 +69,7 @@ KERNEL_SOURCES = {
     "lrank_prep_kernel": _GDN_SOURCES,
     "gdn_state_kernel": _GDN_SOURCES,
     "decode_kernel": ["csrc/decode.cu", "csrc/common.cuh"],
-    "write_producer_kernel": ["csrc/producer.cu", "csrc/producer.cuh", "csrc/chunk_common.cuh",
+    "write_producer_ring_kernel": ["csrc/producer.cu", "csrc/producer.cuh", "csrc/chunk_common.cuh",
                               "csrc/tc.cuh", "csrc/common.cuh"],
 }
 
@@ -529,9 +529,9 @@ def time_producer(wl, dev, stream, peaks, rank, max_over_ranks, barrier, world, 
     return {"workload": f"write producer on {wl.name}: B={wl.B} H={wl.H} T={wl.T} d={wl.dk} L={wl.L} "
                         f"bf16 I/O, random weights",
             "ms_per_call": ms, "tokens_per_s": world * wl.B * wl.T / (ms / 1e3), "launches": 1,
-            "ms_per_launch": {"write_producer_kernel": kern_ms},
-            "dram_bytes_per_launch": {"write_producer_kernel":
-                                      committed_traffic("producer_" + wl.name, "write_producer_kernel")},
+            "ms_per_launch": {"write_producer_ring_kernel": kern_ms},
+            "dram_bytes_per_launch": {"write_producer_ring_kernel":
+                                      committed_traffic("producer_" + wl.name, "write_producer_ring_kernel")},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                          "algorithmic_bytes": alg, "algorithmic_flops": fl,
