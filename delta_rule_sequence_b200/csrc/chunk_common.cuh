@@ -63,21 +63,6 @@ __device__ __forceinline__ uint64_t desc_vt(uint32_t base, int ks) {
     else return desc_mn_sw128(base, ks, C * 128);  // a single MN block; LBO unused
 }
 
-// hi / lo bf16 pair of 4 floats
-__device__ __forceinline__ void split4(const float *x, uint2 &hi, uint2 &lo) {
-    uint32_t h[2], l[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-        float2 hf = __bfloat1622float2(hh);
-        __nv_bfloat162 ll = __floats2bfloat162_rn(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
-        h[i] = *reinterpret_cast<uint32_t *>(&hh);
-        l[i] = *reinterpret_cast<uint32_t *>(&ll);
-    }
-    hi = make_uint2(h[0], h[1]);
-    lo = make_uint2(l[0], l[1]);
-}
-
 // hi / lo bf16 pair of 8 floats
 __device__ __forceinline__ void split8(const float *x, uint4 &hi, uint4 &lo) {
     uint32_t h[4], l[4];

@@ -1131,7 +1131,11 @@ template <int DK, bool RL = false, int BV_ = kBV<DK>>
 struct StateLayout {
     static constexpr int BV = BV_;
     static constexpr int N2 = 2 * BV;                     // hi | lo side by side
-    static constexpr int CH = BV / 4;                     // columns of one epilogue warp
+    // epilogue warps: four per TMEM lane quarter (eight at BV = 16, whose hand-offs then wait for
+    // half as many warps; eight columns a thread in both cases but at d = 64)
+    static constexpr int EPI = BV == 16 ? 8 : 16;
+    static constexpr int CH = BV / (EPI / 4);             // columns of one epilogue warp
+    static constexpr int THREADS = 32 * EPI + 96;         // + the chain MMA, load and D3 warps
     // the value tiles (S^T, Y, D Y: [k][hi | lo], MN-major B operands): 64-column blocks with the
     // 128-byte swizzle, or at BV = 16 one 32-column block with the 64-byte swizzle
     static constexpr bool SW64 = N2 == 32;
@@ -1188,13 +1192,10 @@ struct StateLayout {
     static constexpr uint32_t TCOLS = 4 * N2 <= 256 ? 256 : 512;
 };
 
-// Warp roles of the state kernel: warps 0-15 epilogue (warp w reads TMEM lane quarter w % 4 and
-// the column quarter w / 4 of every BV-wide group), warp 16 issues the chain's MMAs, warp 17 the
-// loads, warp 18 the D3 MMAs.  Every hand-off is an mbarrier (no CTA-wide barrier inside the chunk
-// loop); every wait is bounded.
-constexpr int EPI_WARPS = 16;
-constexpr int EPI_THREADS = 32 * EPI_WARPS;
-constexpr int ST_THREADS = EPI_THREADS + 96;
+// Warp roles of the state kernel: warps 0 .. EPI-1 epilogue (warp w reads TMEM lane quarter w % 4
+// and the column group w / 4 of every BV-wide group), warp EPI issues the chain's MMAs, warp
+// EPI + 1 the loads, warp EPI + 2 the D3 MMAs.  Every hand-off is an mbarrier (no CTA-wide barrier
+// inside the chunk loop); every wait is bounded.
 
 // Largest |S| element below which X_s = Wk S^T is taken with Wk as one bf16 (its rounding then
 // moves Y by at most a few per cent of the bf16 tolerance); above it the Wk_lo term is added.
@@ -1231,17 +1232,17 @@ struct StateBars {
 
 
 // CH fp32 values at (row, j0 .. j0+CH) as a hi / lo pair into an MN-major value tile: hi at
-// columns j0.., lo at BV + j0...; 64-column 128B-swizzled blocks, or at BV = 16 (CH = 4) one
-// 32-column 64B-swizzled block.
+// columns j0.., lo at BV + j0...; 64-column 128B-swizzled blocks, or at BV = 16 one 32-column
+// 64B-swizzled block (eight columns a thread).
 template <int BV, int CH>
 __device__ __forceinline__ void store_half_pair(uint8_t *tile, uint32_t blk_bytes, int row, int j0,
                                                 const float *x) {
-    if constexpr (CH == 4) {
-        static_assert(BV == 16, "four columns a thread: the 32-column tile");
-        uint2 hv, lv;
-        split4(x, hv, lv);
-        *reinterpret_cast<uint2 *>(tile + sw64_off(row, j0)) = hv;
-        *reinterpret_cast<uint2 *>(tile + sw64_off(row, BV + j0)) = lv;
+    if constexpr (BV == 16) {
+        static_assert(CH == 8, "eight columns a thread of the 32-column tile");
+        uint4 hv, lv;
+        split8(x, hv, lv);
+        st16(tile, sw64_off(row, j0), hv);
+        st16(tile, sw64_off(row, BV + j0), lv);
     } else {
 #pragma unroll
         for (int c8 = 0; c8 < CH / 8; ++c8) {
@@ -1269,12 +1270,12 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
 }
 
 template <int DK, bool RL, int BV_>
-__global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
+__global__ void __launch_bounds__(StateLayout<DK, RL, BV_>::THREADS, 1) gdn_state_kernel(ScanArgs p,
                                                                  const __grid_constant__ GdnMaps maps,
                                                                  const uint8_t *ws, int nch) {
     using LY = StateLayout<DK, RL, BV_>;
     using RC = GdnRec<DK, RL, BV_>;
-    constexpr int BV = LY::BV, N2 = LY::N2, CH = LY::CH;
+    constexpr int BV = LY::BV, N2 = LY::N2, CH = LY::CH, EPI_WARPS = LY::EPI;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     __shared__ StateBars bars;
@@ -1655,12 +1656,6 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_state_kernel(ScanArgs p,
                 if (t < n && out) {
                     const float gt = __expf(g_row);
                     __nv_bfloat16 *dst = o + (((size_t)b * T + c0 + t) * H + h) * dv + v0 + j0;
-                    if constexpr (CH == 4) {  // one 8-byte store
-                        float r[4];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) r[j] = fmaf(gt, qs[j], up[j] + ow[j]);
-                        *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]));
-                    }
 #pragma unroll
                     for (int c8 = 0; c8 < CH / 8; ++c8) {
                         float r[8];
@@ -1792,7 +1787,7 @@ cudaError_t launch_gdn_state_bv(const ScanArgs &a, const void *ws, cudaStream_t 
     if (err != cudaSuccess) return err;
     dim3 grid(a.dv / LY::BV, a.H, a.B);
     launch_probe_mark(s);
-    kern<<<grid, ST_THREADS, LY::BYTES, s>>>(a, maps, (const uint8_t *)ws, nch);
+    kern<<<grid, LY::THREADS, LY::BYTES, s>>>(a, maps, (const uint8_t *)ws, nch);
     return cudaGetLastError();
 }
 
