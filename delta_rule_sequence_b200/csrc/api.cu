@@ -25,7 +25,7 @@ cudaError_t launch_segment_element(const ScanArgs &a, int route, bool io_f32, vo
 cudaError_t launch_state_fold(int BH, int dk, int dv, const float *S_in, const float *E, const float *f,
                               float *S_out, cudaStream_t s);
 cudaError_t noalloc_status(uint32_t *out);
-size_t bwd_workspace_bytes(int B, int H, int T, int dk, int dv);
+size_t bwd_workspace_bytes(int B, int H, int T, int dk, int dv, bool io_f32);
 cudaError_t launch_scan_bwd(const ScanArgs &f, const void *dO, const float *dS_final, float *dq,
                             float *dk, float *dv, float *dalpha, float *dbeta, float *du, float *dw,
                             float *dS0, void *ws, bool io_f32, cudaStream_t s);
@@ -308,7 +308,7 @@ prism_status prism_scan_bwd_workspace_size(const prism_shape *shape, size_t *byt
     if (!shape || !bytes) return PRISM_ERR_INVALID_ARG;
     const prism_shape &s = *shape;
     if (s.B < 0 || s.H < 0 || s.T < 0 || !width_ok(s.dk) || !width_ok(s.dv)) return PRISM_ERR_INVALID_ARG;
-    *bytes = prism::bwd_workspace_bytes(s.B, s.H, s.T, s.dk, s.dv);
+    *bytes = prism::bwd_workspace_bytes(s.B, s.H, s.T, s.dk, s.dv, s.io == PRISM_F32);
     return PRISM_OK;
 }
 

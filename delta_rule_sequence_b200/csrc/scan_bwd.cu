@@ -23,9 +23,20 @@
 // checkpoint into a per-CTA workspace buffer (and S_{t-1} k_t into shared memory) and walks the
 // chunk's tokens backwards.  All arithmetic is fp32 from the exact input values.
 
+#include <algorithm>
+
 #include "tc.cuh"
 
 namespace prism {
+
+// the forward's two-kernel routes (scan_gdn.cu)
+cudaError_t launch_gdn_prep(const ScanArgs &a, void *ws, cudaStream_t s);
+cudaError_t launch_gdn_state(const ScanArgs &a, const void *ws, cudaStream_t s);
+cudaError_t launch_lrank_prep(const ScanArgs &a, void *ws, cudaStream_t s);
+cudaError_t launch_lrank_state(const ScanArgs &a, const void *ws, cudaStream_t s);
+size_t gdn_workspace_bytes(int B, int H, int T, int dk);
+size_t lrank_workspace_bytes(int B, int H, int T, int dk);
+
 namespace {
 
 constexpr int BW_NW = 16;              // value rows (warps) per CTA
@@ -41,6 +52,12 @@ struct BwdArgs {
     float *dq, *dk_out, *dv_out, *dalpha, *dbeta, *du, *dw, *dS0;
     float *ckpt;     // [B, H, nch, dv, dk] state at each chunk start
     float *scratch;  // per CTA: [BW_C + 1][BW_NW][dk] states of the current chunk
+    // chunk-parallel mode (ns > 0): the chunk-entry states are given in ckpt, and gexit holds the
+    // gradient scan's state at each of its NR chunk starts (the gradient of the state at the end
+    // of chunk c, plus that chunk's last output term, sits at NR - 1 - c); blockIdx.z = b ns + split,
+    // each split walking its own contiguous range of chunks
+    const float *gexit;
+    int NR, ns;
 };
 
 // One staged block of BW_TB tokens (io type unless noted): k, q [TB][DK]; w [TB][L][DK];
@@ -94,7 +111,8 @@ __global__ void __launch_bounds__(BW_THREADS) scan_bwd_kernel(BwdArgs p) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r0 = blockIdx.x * BW_NW, r = r0 + warp;  // this warp's value row
-    const int h = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.y, b = p.ns ? (int)blockIdx.z / p.ns : (int)blockIdx.z;
+    const int split = p.ns ? (int)blockIdx.z % p.ns : 0;
     const int H = p.H, T = p.T, dv = p.dv, nch = p.nch;
     const size_t head = (size_t)b * H + h;
     const IO *q = (const IO *)p.q, *k = (const IO *)p.k, *v = (const IO *)p.v;
@@ -208,9 +226,14 @@ __global__ void __launch_bounds__(BW_THREADS) scan_bwd_kernel(BwdArgs p) {
     // the last: its blocks forwards (recomputing the states), then backwards
     enum { kFwd, kRecomp, kRev };
     const int last_sb = (nch - 1) * BW_SPC, m_last = nsb - last_sb;  // blocks of the last interval
+    // chunk-parallel mode: no forward sweep, and this CTA's chunks [c_lo, c_hi) only
+    const int c_lo = p.ns ? (int)((long long)nch * split / p.ns) : 0;
+    const int c_hi = p.ns ? (int)((long long)nch * (split + 1) / p.ns) : nch;
+    const int fwd = p.ns ? 0 : nsb;  // forward-sweep steps
     auto schedule = [&](int j, int &sb, int &mode) {
-        if (j < nsb) { sb = j; mode = kFwd; return; }
-        int j2 = j - nsb, c, kk, m;
+        if (j < fwd) { sb = j; mode = kFwd; return; }
+        int j2 = j - fwd, c, kk, m;
+        if (c_hi < nch) j2 += 2 * m_last + 2 * BW_SPC * (nch - 1 - c_hi);  // skip the later chunks
         if (j2 < 2 * m_last) {
             c = nch - 1; kk = j2; m = m_last;
         } else {
@@ -220,7 +243,10 @@ __global__ void __launch_bounds__(BW_THREADS) scan_bwd_kernel(BwdArgs p) {
         mode = kk < m ? kRecomp : kRev;
         sb = c * BW_SPC + (kk < m ? kk : 2 * m - 1 - kk);
     };
-    const int steps = 3 * nsb;
+    const int steps = p.ns ? (c_hi <= c_lo ? 0
+                                          : (c_hi == nch ? 2 * m_last + 2 * BW_SPC * (nch - 1 - c_lo)
+                                                         : 2 * BW_SPC * (c_hi - c_lo)))
+                           : 3 * nsb;
 
     float s[E], g[E];
     if (p.S0) load_state(p.S0 + (head * dv + r) * DK, s);
@@ -263,6 +289,17 @@ __global__ void __launch_bounds__(BW_THREADS) scan_bwd_kernel(BwdArgs p) {
             if (ci0 == 0) {
                 load_state(ckpt_row(c), s);
                 store_state(scr, s);
+                if (p.ns) {
+                    // the gradient at the chunk's end from everything after it: the gradient scan's
+                    // state there less the chunk's last output term, which the reverse pass adds
+                    load_state(p.gexit + ((head * p.NR + (p.NR - 1 - c)) * dv + r) * DK, g);
+                    const int tl = (c + 1) * BW_C - 1;
+                    if (tl < T) {
+                        const float dd = ld_io<IO>(dO, tok(tl) * dv + r);
+#pragma unroll
+                        for (int e = 0; e < E; ++e) g[e] -= dd * ld_io<IO>(q, tok(tl) * DK + lane + 32 * e);
+                    }
+                }
             }
             for (int i = 0; i < m; ++i) {
                 const float pki = step(s, buf, i);
@@ -353,7 +390,45 @@ __global__ void __launch_bounds__(BW_THREADS) scan_bwd_kernel(BwdArgs p) {
         __syncthreads();  // the block's buffer is free for the block two steps ahead
     }
     cp_async_wait<0>();
-    if (p.dS0) store_state(p.dS0 + (head * dv + r) * DK, g);
+    if (p.dS0 && !p.ns) store_state(p.dS0 + (head * dv + r) * DK, g);
+}
+
+// The gradient scan's inputs (chunk-parallel backward).  With G_t the gradient of the state after
+// token t (0-indexed tokens; G_{T-1} = dS_final + dO_{T-1} q_{T-1}^T, G_{t-1} = G_t A_t +
+// dO_{t-1} q_{t-1}^T, A_t = alpha_t (I - beta_t k_t k_t^T), dS0 = G_{-1} = G_0 A_0), the gradient
+// runs as the scan's own recurrence over the tokens in reverse: position P + i carries token
+// T - 1 - i's transition and the rank-1 write u = dO, w = q of the token before it (none for
+// i = T - 1).  P = 64 - T % 64 positions in front (identity transitions; the last of them writes
+// dO_{T-1} q_{T-1}^T onto the entry state dS_final) align the scan's 64-token chunks with the
+// forward's chunk ends.  One thread a 16-byte piece of a row; bf16 rows are copied bit for bit.
+template <typename IO>
+__global__ void __launch_bounds__(128) bwd_reverse_kernel(int B, int T, int H, int dk, int dv, int P,
+                                                          const IO *q, const IO *k, const float *alpha,
+                                                          const float *beta, const IO *dO, IO *kr,
+                                                          IO *ur, IO *wr, float *ar, float *br) {
+    const int Tp = T + P;
+    const long long idx = blockIdx.x;  // (b, position, h)
+    const int h = (int)(idx % H), pos = (int)((idx / H) % Tp), b = (int)(idx / ((long long)H * Tp));
+    int tk = -1, tw = -1;  // source tokens of the transition and of the write
+    if (pos == P - 1) tw = T - 1;
+    else if (pos >= P) {
+        tk = T - 1 - (pos - P);
+        tw = tk - 1;
+    }
+    auto src = [&](int t) { return ((size_t)b * T + t) * H + h; };
+    const size_t dst = idx;  // ((b Tp + pos) H + h)
+    constexpr int PER = 16 / (int)sizeof(IO);
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    for (int c = threadIdx.x; c < dk / PER; c += blockDim.x) {
+        reinterpret_cast<uint4 *>(kr + dst * dk)[c] = tk >= 0 ? reinterpret_cast<const uint4 *>(k + src(tk) * dk)[c] : zero;
+        reinterpret_cast<uint4 *>(wr + dst * dk)[c] = tw >= 0 ? reinterpret_cast<const uint4 *>(q + src(tw) * dk)[c] : zero;
+    }
+    for (int c = threadIdx.x; c < dv / PER; c += blockDim.x)
+        reinterpret_cast<uint4 *>(ur + dst * dv)[c] = tw >= 0 ? reinterpret_cast<const uint4 *>(dO + src(tw) * dv)[c] : zero;
+    if (threadIdx.x == 0) {
+        ar[dst] = tk >= 0 ? alpha[src(tk)] : 1.f;
+        br[dst] = tk >= 0 ? beta[src(tk)] : 0.f;
+    }
 }
 
 template <typename IO, int DK>
@@ -362,7 +437,7 @@ cudaError_t launch_bwd_t(const BwdArgs &a, cudaStream_t s) {
     auto kern = scan_bwd_kernel<IO, DK>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (err != cudaSuccess) return err;
-    dim3 grid(a.dv / BW_NW, a.H, a.B);
+    dim3 grid(a.dv / BW_NW, a.H, a.B * (a.ns ? a.ns : 1));
     launch_probe_mark(s);
     kern<<<grid, BW_THREADS, bytes, s>>>(a);
     return cudaGetLastError();
@@ -370,12 +445,81 @@ cudaError_t launch_bwd_t(const BwdArgs &a, cudaStream_t s) {
 
 }  // namespace
 
-// Workspace of the backward after the status block: the chunk-start states of every row, and one
-// chunk of states per CTA.
-size_t bwd_workspace_bytes(int B, int H, int T, int dk, int dv) {
-    const size_t nch = (size_t)((T + BW_C - 1) / BW_C);
-    const size_t ctas = (size_t)B * H * (dv / BW_NW);
-    return kStatusBytes + sizeof(float) * ((size_t)B * H * nch * dv * dk + ctas * (BW_C + 1) * BW_NW * dk);
+// The chunk-parallel backward (bf16 I/O on the tensor-core shapes): the forward scan writes every
+// chunk's entry state, the gradient scan (the forward's own kernels on the reversed tokens, above)
+// writes the gradient at every chunk end, and then every chunk's token-level reverse pass runs on
+// its own, split into ns ranges of chunks per sequence so that the grid fills the GPU several times.
+namespace {
+
+bool chunked_bwd(int dk, int dv, bool io_f32) { return !io_f32 && dk == dv && (dk == 64 || dk == 128); }
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+        return 148;
+    return n;
+}
+
+int bwd_splits(int B, int H, int dv, int nch) {
+    const long long base = (long long)B * H * (dv / BW_NW);  // CTAs of one split
+    const long long want = (8LL * sm_count() + base - 1) / base;
+    return (int)std::max(1LL, std::min<long long>({want, (long long)nch, 65535LL / std::max(B, 1)}));
+}
+
+struct BwdLayout {  // byte offsets into the workspace
+    size_t ckpt, gexit, scratch, kr, ur, wr, ar, br, rec, total;
+    int nch, P, Tp, NR, ns;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+BwdLayout bwd_layout(int B, int H, int T, int dk, int dv, bool io_f32) {
+    BwdLayout l{};
+    l.nch = (T + BW_C - 1) / BW_C;
+    const size_t heads = (size_t)B * H, st = (size_t)dv * dk * sizeof(float);
+    const bool chunked = chunked_bwd(dk, dv, io_f32) && T > 0;
+    l.ns = chunked ? bwd_splits(B, H, dv, l.nch) : 0;
+    l.P = BW_C - T % BW_C;  // 1 .. 64 identity positions in front of the reversed tokens
+    l.Tp = T + l.P;
+    l.NR = l.Tp / BW_C;
+    size_t o = kStatusBytes;
+    l.ckpt = o;
+    o = align256(o + heads * l.nch * st);
+    const size_t ctas = heads * (dv / BW_NW) * (size_t)(l.ns ? l.ns : 1);
+    l.scratch = o;
+    o = align256(o + ctas * (BW_C + 1) * BW_NW * dk * sizeof(float));
+    if (chunked) {
+        const size_t ntok = heads * l.Tp, io = 2;
+        l.gexit = o;
+        o = align256(o + heads * l.NR * st);
+        l.kr = o;
+        o = align256(o + ntok * dk * io);
+        l.ur = o;
+        o = align256(o + ntok * dv * io);
+        l.wr = o;
+        o = align256(o + ntok * dk * io);
+        l.ar = o;
+        o = align256(o + ntok * sizeof(float));
+        l.br = o;
+        o = align256(o + ntok * sizeof(float));
+        // the forward's records (either write form), then the gradient scan's, in one region
+        l.rec = o;
+        const size_t rec = std::max({gdn_workspace_bytes(B, H, T, dk), lrank_workspace_bytes(B, H, T, dk),
+                                     lrank_workspace_bytes(B, H, l.Tp, dk)});
+        o = align256(o + rec);
+    }
+    l.total = o;
+    return l;
+}
+
+}  // namespace
+
+// Workspace of the backward after the status block: the chunk-start states of every row, one
+// chunk of states per CTA, and for the chunk-parallel form the gradient scan's chunk states, its
+// inputs and the scans' records.
+size_t bwd_workspace_bytes(int B, int H, int T, int dk, int dv, bool io_f32) {
+    return bwd_layout(B, H, T, dk, dv, io_f32).total;
 }
 
 // The gradients (fp32).  dq, dk, dw, dalpha, dbeta are sums over value rows (atomic adds): they are
@@ -406,8 +550,59 @@ cudaError_t launch_scan_bwd(const ScanArgs &f, const void *dO, const float *dS_f
     a.alpha = f.alpha; a.beta = f.beta; a.S0 = f.S0; a.dS_final = dS_final;
     a.dq = dq; a.dk_out = dk; a.dv_out = dv; a.dalpha = dalpha; a.dbeta = dbeta;
     a.du = du; a.dw = dw; a.dS0 = dS0;
-    a.ckpt = (float *)((uint8_t *)ws + kStatusBytes);
-    a.scratch = a.ckpt + (size_t)f.B * f.H * a.nch * f.dv * f.dk;
+    const BwdLayout lay = bwd_layout(f.B, f.H, f.T, f.dk, f.dv, io_f32);
+    uint8_t *wb = (uint8_t *)ws;
+    a.ckpt = (float *)(wb + lay.ckpt);
+    a.scratch = (float *)(wb + lay.scratch);
+    a.gexit = nullptr;
+    a.NR = 0;
+    a.ns = 0;
+    if (lay.ns) {
+        // 1. the forward over the same tokens, keeping every chunk's entry state (no outputs)
+        ScanArgs fa = f;
+        fa.o = nullptr;
+        fa.S_final = nullptr;
+        fa.flags = kNoOutput;
+        fa.ckpt = a.ckpt;
+        void *rec = wb + lay.rec;
+        const bool gdn = f.u == nullptr;
+        if ((err = gdn ? launch_gdn_prep(fa, rec, s) : launch_lrank_prep(fa, rec, s)) != cudaSuccess) return err;
+        if ((err = gdn ? launch_gdn_state(fa, rec, s) : launch_lrank_state(fa, rec, s)) != cudaSuccess) return err;
+        // 2. the gradient scan's inputs, then the scan itself (rank-1 write), which leaves the
+        //    gradient at every chunk end in gexit and dS0 in its exit state
+        const __nv_bfloat16 *qb = (const __nv_bfloat16 *)f.q, *kb = (const __nv_bfloat16 *)f.k;
+        __nv_bfloat16 *kr = (__nv_bfloat16 *)(wb + lay.kr), *ur = (__nv_bfloat16 *)(wb + lay.ur),
+                      *wr = (__nv_bfloat16 *)(wb + lay.wr);
+        float *ar = (float *)(wb + lay.ar), *br = (float *)(wb + lay.br);
+        launch_probe_mark(s);
+        bwd_reverse_kernel<__nv_bfloat16><<<(unsigned)((size_t)f.B * lay.Tp * f.H), 128, 0, s>>>(
+            f.B, f.T, f.H, f.dk, f.dv, lay.P, qb, kb, f.alpha, f.beta, (const __nv_bfloat16 *)dO, kr, ur, wr,
+            ar, br);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        ScanArgs ra = f;
+        ra.T = lay.Tp;
+        ra.L = 1;
+        ra.q = kr;
+        ra.k = kr;
+        ra.v = kr;  // (not read by the rank-L write; dv == dk)
+        ra.alpha = ar;
+        ra.beta = br;
+        ra.u = ur;
+        ra.w = wr;
+        ra.S0 = dS_final;
+        ra.o = nullptr;
+        ra.S_final = dS0;
+        ra.flags = kNoOutput;
+        float *gexit = (float *)(wb + lay.gexit);
+        ra.ckpt = gexit;
+        if ((err = launch_lrank_prep(ra, rec, s)) != cudaSuccess) return err;
+        if ((err = launch_lrank_state(ra, rec, s)) != cudaSuccess) return err;
+        // 3. every chunk's own gradients from (its entry state, the gradient at its end)
+        a.gexit = gexit;
+        a.NR = lay.NR;
+        a.ns = lay.ns;
+        a.dS0 = nullptr;  // written by the gradient scan
+    }
     if (io_f32) {
         switch (f.dk) {
             case 32: return launch_bwd_t<float, 32>(a, s);

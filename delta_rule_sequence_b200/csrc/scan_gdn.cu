@@ -1535,6 +1535,11 @@ __global__ void __launch_bounds__(StateLayout<DK, RL, BV_>::THREADS, 1) gdn_stat
         for (int c = 0; c < nch && ok; ++c) {
             const int c0 = c * C, n = min(C, T - c0);
             const uint8_t *buf = sm + (c & 1) * LY::BUF;
+            if (p.ckpt && own_d) {  // the chunk's entry state, for the backward
+                float *ck = p.ckpt + ((head * nch + c) * dv + v0 + j0) * DK + d_row;
+#pragma unroll
+                for (int j = 0; j < CH; ++j) ck[(size_t)j * DK] = Sreg[j];
+            }
             if (!mbar_wait(&bars.full[c & 1], (c >> 1) & 1, status, lim)) { ok = false; break; }
             const float *g = reinterpret_cast<const float *>(sm + LY::GB + (c & 1) * C * 4);
             const float g_last = g[C - 1];
