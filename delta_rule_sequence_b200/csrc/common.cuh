@@ -20,9 +20,6 @@ struct ScanArgs {
     float *S_final;
     uint32_t *status;  // device status word (PRISM_OK / PRISM_ERR_TIMEOUT), may be null
     int flags;         // kNoWrite | kS0Identity | kNoOutput (segment passes of the segmented scan)
-    // tensor-core state kernel only, may be null: the entry state of every 64-token chunk,
-    // [B, H, ceil(T / 64), dv, dk] fp32 (the backward's checkpoints)
-    float *ckpt = nullptr;
 };
 
 // Flags of a scan pass.  kNoWrite: the write term is zero (u = 0 / v = 0);  kS0Identity: the entry

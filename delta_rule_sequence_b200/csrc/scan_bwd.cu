@@ -31,9 +31,9 @@ namespace prism {
 
 // the forward's two-kernel routes (scan_gdn.cu)
 cudaError_t launch_gdn_prep(const ScanArgs &a, void *ws, cudaStream_t s);
-cudaError_t launch_gdn_state(const ScanArgs &a, const void *ws, cudaStream_t s);
+cudaError_t launch_gdn_state(const ScanArgs &a, const void *ws, cudaStream_t s, float *ckpt);
 cudaError_t launch_lrank_prep(const ScanArgs &a, void *ws, cudaStream_t s);
-cudaError_t launch_lrank_state(const ScanArgs &a, const void *ws, cudaStream_t s);
+cudaError_t launch_lrank_state(const ScanArgs &a, const void *ws, cudaStream_t s, float *ckpt);
 size_t gdn_workspace_bytes(int B, int H, int T, int dk);
 size_t lrank_workspace_bytes(int B, int H, int T, int dk);
 
@@ -563,11 +563,11 @@ cudaError_t launch_scan_bwd(const ScanArgs &f, const void *dO, const float *dS_f
         fa.o = nullptr;
         fa.S_final = nullptr;
         fa.flags = kNoOutput;
-        fa.ckpt = a.ckpt;
         void *rec = wb + lay.rec;
         const bool gdn = f.u == nullptr;
         if ((err = gdn ? launch_gdn_prep(fa, rec, s) : launch_lrank_prep(fa, rec, s)) != cudaSuccess) return err;
-        if ((err = gdn ? launch_gdn_state(fa, rec, s) : launch_lrank_state(fa, rec, s)) != cudaSuccess) return err;
+        if ((err = gdn ? launch_gdn_state(fa, rec, s, a.ckpt) : launch_lrank_state(fa, rec, s, a.ckpt)) != cudaSuccess)
+            return err;
         // 2. the gradient scan's inputs, then the scan itself (rank-1 write), which leaves the
         //    gradient at every chunk end in gexit and dS0 in its exit state
         const __nv_bfloat16 *qb = (const __nv_bfloat16 *)f.q, *kb = (const __nv_bfloat16 *)f.k;
@@ -594,9 +594,8 @@ cudaError_t launch_scan_bwd(const ScanArgs &f, const void *dO, const float *dS_f
         ra.S_final = dS0;
         ra.flags = kNoOutput;
         float *gexit = (float *)(wb + lay.gexit);
-        ra.ckpt = gexit;
         if ((err = launch_lrank_prep(ra, rec, s)) != cudaSuccess) return err;
-        if ((err = launch_lrank_state(ra, rec, s)) != cudaSuccess) return err;
+        if ((err = launch_lrank_state(ra, rec, s, gexit)) != cudaSuccess) return err;
         // 3. every chunk's own gradients from (its entry state, the gradient at its end)
         a.gexit = gexit;
         a.NR = lay.NR;

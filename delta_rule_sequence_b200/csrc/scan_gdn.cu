@@ -1269,10 +1269,12 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
     if (lane == 0) mbar_arrive(bar);
 }
 
-template <int DK, bool RL, int BV_>
+// CK: also write the entry state of every chunk to ckpt, [B, H, nch, dv, dk] fp32 (the backward's
+// checkpoints; a separate instantiation, so the forward's chunk loop carries no test for it).
+template <int DK, bool RL, int BV_, bool CK>
 __global__ void __launch_bounds__(StateLayout<DK, RL, BV_>::THREADS, 1) gdn_state_kernel(ScanArgs p,
                                                                  const __grid_constant__ GdnMaps maps,
-                                                                 const uint8_t *ws, int nch) {
+                                                                 const uint8_t *ws, int nch, float *ckpt) {
     using LY = StateLayout<DK, RL, BV_>;
     using RC = GdnRec<DK, RL, BV_>;
     constexpr int BV = LY::BV, N2 = LY::N2, CH = LY::CH, EPI_WARPS = LY::EPI;
@@ -1535,8 +1537,8 @@ __global__ void __launch_bounds__(StateLayout<DK, RL, BV_>::THREADS, 1) gdn_stat
         for (int c = 0; c < nch && ok; ++c) {
             const int c0 = c * C, n = min(C, T - c0);
             const uint8_t *buf = sm + (c & 1) * LY::BUF;
-            if (p.ckpt && own_d) {  // the chunk's entry state, for the backward
-                float *ck = p.ckpt + ((head * nch + c) * dv + v0 + j0) * DK + d_row;
+            if (CK && own_d) {  // the chunk's entry state, for the backward
+                float *ck = ckpt + ((head * nch + c) * dv + v0 + j0) * DK + d_row;
 #pragma unroll
                 for (int j = 0; j < CH; ++j) ck[(size_t)j * DK] = Sreg[j];
             }
@@ -1780,27 +1782,27 @@ cudaError_t launch_gdn_prep_t(const ScanArgs &a, void *ws, cudaStream_t s) {
 
 // The state kernel reads only K and Q through tensor maps (v may be absent on the rank-L route).
 template <int DK, bool RL, int BV>
-cudaError_t launch_gdn_state_bv(const ScanArgs &a, const void *ws, cudaStream_t s) {
+cudaError_t launch_gdn_state_bv(const ScanArgs &a, const void *ws, cudaStream_t s, float *ckpt) {
     const int nch = (a.T + C - 1) / C;
     GdnMaps maps = {};
     if (!act_map(&maps.k, a.k, a.B, a.T, a.H, DK, 64) || !act_map(&maps.q, a.q, a.B, a.T, a.H, DK, 64))
         return cudaErrorInvalidValue;
     using LY = StateLayout<DK, RL, BV>;
     static_assert(LY::BYTES + 256 <= 227 * 1024, "shared memory budget (with the static part)");
-    auto kern = gdn_state_kernel<DK, RL, BV>;
+    auto kern = ckpt ? gdn_state_kernel<DK, RL, BV, true> : gdn_state_kernel<DK, RL, BV, false>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::BYTES);
     if (err != cudaSuccess) return err;
     dim3 grid(a.dv / LY::BV, a.H, a.B);
     launch_probe_mark(s);
-    kern<<<grid, LY::THREADS, LY::BYTES, s>>>(a, maps, (const uint8_t *)ws, nch);
+    kern<<<grid, LY::THREADS, LY::BYTES, s>>>(a, maps, (const uint8_t *)ws, nch, ckpt);
     return cudaGetLastError();
 }
 
 template <int DK, bool RL>
-cudaError_t launch_gdn_state_t(const ScanArgs &a, const void *ws, cudaStream_t s) {
+cudaError_t launch_gdn_state_t(const ScanArgs &a, const void *ws, cudaStream_t s, float *ckpt) {
     if constexpr (DK == 128)
-        if (slice_width<DK>(a) == 16) return launch_gdn_state_bv<DK, RL, 16>(a, ws, s);
-    return launch_gdn_state_bv<DK, RL, kBV<DK>>(a, ws, s);
+        if (slice_width<DK>(a) == 16) return launch_gdn_state_bv<DK, RL, 16>(a, ws, s, ckpt);
+    return launch_gdn_state_bv<DK, RL, kBV<DK>>(a, ws, s, ckpt);
 }
 
 template <int DK, int BV>
@@ -1851,9 +1853,11 @@ cudaError_t launch_gdn_prep(const ScanArgs &a, void *ws, cudaStream_t s) {
     return a.dk == 128 ? launch_gdn_prep_t<128>(a, ws, s) : launch_gdn_prep_t<64>(a, ws, s);
 }
 
-cudaError_t launch_gdn_state(const ScanArgs &a, const void *ws, cudaStream_t s) {
-    return a.dk == 128 ? launch_gdn_state_t<128, false>(a, ws, s) : launch_gdn_state_t<64, false>(a, ws, s);
+// ckpt (optional): every chunk's entry state, [B, H, ceil(T / 64), dv, dk] fp32
+cudaError_t launch_gdn_state(const ScanArgs &a, const void *ws, cudaStream_t s, float *ckpt) {
+    return a.dk == 128 ? launch_gdn_state_t<128, false>(a, ws, s, ckpt) : launch_gdn_state_t<64, false>(a, ws, s, ckpt);
 }
+cudaError_t launch_gdn_state(const ScanArgs &a, const void *ws, cudaStream_t s) { return launch_gdn_state(a, ws, s, nullptr); }
 
 cudaError_t launch_scan_gdn(const ScanArgs &a, void *ws, cudaStream_t s) {
     cudaError_t err = launch_gdn_prep(a, ws, s);
@@ -1868,9 +1872,10 @@ cudaError_t launch_lrank_prep(const ScanArgs &a, void *ws, cudaStream_t s) {
     return a.dk == 128 ? launch_lrank_prep_t<128>(a, ws, s) : launch_lrank_prep_t<64>(a, ws, s);
 }
 
-cudaError_t launch_lrank_state(const ScanArgs &a, const void *ws, cudaStream_t s) {
-    return a.dk == 128 ? launch_gdn_state_t<128, true>(a, ws, s) : launch_gdn_state_t<64, true>(a, ws, s);
+cudaError_t launch_lrank_state(const ScanArgs &a, const void *ws, cudaStream_t s, float *ckpt) {
+    return a.dk == 128 ? launch_gdn_state_t<128, true>(a, ws, s, ckpt) : launch_gdn_state_t<64, true>(a, ws, s, ckpt);
 }
+cudaError_t launch_lrank_state(const ScanArgs &a, const void *ws, cudaStream_t s) { return launch_lrank_state(a, ws, s, nullptr); }
 
 cudaError_t launch_scan_lrank(const ScanArgs &a, void *ws, cudaStream_t s) {
     cudaError_t err = launch_lrank_prep(a, ws, s);
