@@ -17,11 +17,15 @@
 // ...), its dot products are warp reductions, and only dq, dk, dw, dalpha and dbeta sum over rows
 // (per token in shared memory across the CTA's warps, then one atomic add per element and CTA).
 //
-// The backward needs S_{t-1} and S_t at every token, in reverse order.  Each CTA first runs the
-// forward recurrence for its rows and writes the state at every 64-token chunk start to the
-// workspace; then, chunk by chunk from the last, it recomputes the chunk's states from that
-// checkpoint into a per-CTA workspace buffer (and S_{t-1} k_t into shared memory) and walks the
-// chunk's tokens backwards.  All arithmetic is fp32 from the exact input values.
+// The backward needs S_{t-1} and S_t at every token, in reverse order.  Sequential form: each CTA
+// first runs the forward recurrence for its rows and writes the state at every 64-token chunk
+// start to the workspace; then, chunk by chunk from the last, it recomputes the chunk's states
+// from that checkpoint into a per-CTA workspace buffer (and S_{t-1} k_t into shared memory) and
+// walks the chunk's tokens backwards, carrying G from chunk to chunk.  All arithmetic is fp32 from
+// the exact input values.  Chunk-parallel form (bf16 I/O, dk == dv in {64, 128}): the forward's
+// tensor-core scan writes the chunk-entry states, the same scan over the reversed tokens (see
+// bwd_reverse_kernel) writes the gradient at every chunk end, and the CTAs, each on its own range
+// of chunks, run only the recompute and reverse passes, reloading G at every chunk end.
 
 #include <algorithm>
 

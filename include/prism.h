@@ -107,8 +107,10 @@ prism_status prism_scan_fwd(const prism_shape *shape, const void *q, const void 
 
 /*
  * prism_scan_bwd_workspace_size -- bytes of device workspace prism_scan_bwd needs for `shape`:
- * the status block, the state of every (b, h) at each 64-token chunk start, and one chunk of
- * states per CTA.  Writes *bytes.
+ * the status block, the state of every (b, h) at each 64-token chunk start, one chunk of states
+ * per CTA, and for the chunk-parallel form (bf16 I/O, dk == dv in {64, 128}) the gradient at
+ * every chunk end, the reversed token layout and the scans' per-chunk records.  Depends on the
+ * current device's SM count.  Writes *bytes.
  */
 prism_status prism_scan_bwd_workspace_size(const prism_shape *shape, size_t *bytes);
 
@@ -133,9 +135,13 @@ prism_status prism_scan_bwd_workspace_size(const prism_shape *shape, size_t *byt
  *   du, dw    [B,T,H,L,dv], [B,T,H,L,dk] fp32   outputs, rank-L write only (ignored otherwise)
  *   dS0       [B,H,dv,dk] fp32    output, or NULL to skip
  *   workspace, ws_bytes           at least prism_scan_bwd_workspace_size bytes, 256-byte aligned
- * Every pointer 16-byte aligned; no gradient may overlap another or an input.  All arithmetic is
- * fp32 on CUDA cores from the exact input values: each CTA re-runs the forward recurrence for its
- * value rows (checkpointing every 64 tokens), then walks the tokens backwards chunk by chunk.
+ * Every pointer 16-byte aligned; no gradient may overlap another or an input.  With bf16 I/O and
+ * dk == dv in {64, 128} the work is chunk-parallel: the forward scan's tensor-core kernels write
+ * every 64-token chunk's entry state and, run over the reversed tokens with the rank-1 write
+ * dO q^T, the gradient at every chunk end (and dS0); every chunk's token-level reverse pass then
+ * runs on its own, in fp32 on CUDA cores.  Otherwise each CTA re-runs the forward recurrence for
+ * its value rows (checkpointing every 64 tokens) and walks the tokens backwards chunk by chunk,
+ * all in fp32 on CUDA cores from the exact input values.
  * dq, dk, dw, dalpha and dbeta are sums over value rows accumulated with atomic adds (cleared on
  * the stream first), so their last bits depend on the order of those adds.  Tested against
  * |x - r| <= tol (1 + |r|) with tol = 2e-2 (bf16 I/O) and 1e-4 (fp32 I/O).
