@@ -62,6 +62,9 @@ def _names(gdn, dS0=True):
     ("recsys", dict(B=1, H=2, T=100, L=2, io="f32")),
     ("recsys", dict(B=1, H=1, T=90, dk=32, dv=64, L=2, io="f32")),
     ("gdn", dict(B=1, H=2, T=129, dk=128, dv=64, io="f32")),
+    # chunk-parallel form at its edges: one token, and one token past a chunk
+    ("gdn", dict(B=1, H=2, T=1)),
+    ("recsys", dict(B=1, H=1, T=65, L=2)),
 ])
 def test_backward_matches_oracle(name, over):
     wl = WORKLOADS[name].with_(**over)
